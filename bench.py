@@ -1,0 +1,447 @@
+"""Throughput of the Engram layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the layer's hot path over one batch of the 27B-shaped
+workload (8 sequences x 4,096 tokens, d 2,560, 16 hash heads x 80 dims over a
+5.7B-parameter bf16 table): compress + n-gram + hash, row gather, then the two
+fused tensor-core passes (gate partials; gate + value + causal conv +
+residual).  Inputs are seeded and synthetic and stay resident in HBM; the
+table (11.4 GB) and the hidden state (168 MB) exceed the 126 MB L2, so no
+flush is needed between steps.
+
+With N > 1 (torchrun), every rank runs an independent replica on its own
+batch (weak scaling, no collective on the data path); timing is the max over
+ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("Engram layer tokens/s (fwd, fwd+bwd) and achieved HBM GB/s / tensor-pipe % of "
+          "B200 peak")
+WORKLOAD = "layer27b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- distribution
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def dist_init(backend: str):
+    import torch.distributed as dist
+    ws, rank, _ = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return ws, rank
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(x: float) -> float:
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each replica draws its own token batch."""
+    return base + 7919 * rank
+
+
+# ---------------------------------------------------------------- peaks, clocks
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                     power=float(parts[3]), hw=parts[5], hwt=parts[6],
+                                     swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        smax = max(r["smax"] for r in rows)
+        loaded = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = set()
+        for r in rows:
+            if r["hw"] == "Active":
+                reasons.add("hw_slowdown")
+            if r["hwt"] == "Active":
+                reasons.add("hw_thermal_slowdown")
+            if r["swt"] == "Active":
+                reasons.add("sw_thermal_slowdown")
+            if r["pcap"] == "Active":
+                reasons.add("sw_power_cap")
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, ids, keys, mult, table_rows_fn, dense_host, n_seq: int, n_tok: int):
+    """The oracle end to end (projection, hash, gather, fusion) on the first
+    `n_tok` tokens of each of the first `n_seq` sequences of the batch.
+    Returns (tokens, seconds, threads)."""
+    from oracle import engram_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        threads = 1
+    t0 = time.perf_counter()
+    proj, V_c = O.build_vocab_proj(keys)
+    sub = np.ascontiguousarray(ids[:n_seq, :n_tok])
+    idx = O.hash_indices(proj, sub, mult, np.array(w.rows), w.K, V_c).reshape(-1, w.J)
+    e = table_rows_fn(idx)
+    h = dense_host["h"][: n_seq * n_tok]
+    O.layer_forward(e, h, dense_host["Wk"], dense_host["Wv"], dense_host["conv_w"], n_tok)
+    return n_seq * n_tok, time.perf_counter() - t0, threads
+
+
+# ---------------------------------------------------------------- our path
+
+def run_ours(args):
+    import torch
+
+    from hashed_gram_conditional_engram_b200 import build as _b
+    _b.build()
+    from hashed_gram_conditional_engram_b200 import engram as eg
+    from hashed_gram_conditional_engram_b200 import synth
+
+    ws_, rank = dist_init("nccl")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.workload(WORKLOAD)
+
+    # ---- inputs (seeded, synthetic, resident in HBM)
+    w_rank = synth.Workload(**{**w.__dict__, "seed": rank_seed(w.seed, rank)})
+    ids_np = synth.host_ids_keys(w_rank)[0]
+    keys_np = synth.host_ids_keys(w)[1]
+    mult = synth.hash_multipliers(synth.layer_seed(w, 0), w.J)
+    table = synth.device_table(w, device=dev)
+    dense = synth.device_dense(w, device=dev)
+    keys = torch.from_numpy(keys_np).to(dev)
+    proj = torch.empty(w.V, dtype=torch.int32, device=dev)
+    vb = eg.engram_workspace_size(None, eg.WS_VOCAB, w.V)
+    vws = torch.empty(vb, dtype=torch.uint8, device=dev)
+    V_c = eg.engram_build_vocab_proj(keys, w.V, proj, vws, vb)
+    del vws
+    cfg = eg.make_cfg(w.K, w.D_h, w.d, 1, w.V, V_c, eg.BF16, w.rows, mult)
+    N = w.N
+    ids = torch.from_numpy(ids_np).to(dev)
+    idx = torch.empty((w.B, w.T, w.J), dtype=torch.int32, device=dev)
+    e = torch.empty((N, w.E), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((w.B, w.T, 1, w.d), dtype=torch.bfloat16, device=dev)
+    saved = torch.empty(eg.engram_saved_size(cfg, N), dtype=torch.uint8, device=dev)
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+    fws = torch.empty(fb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        eg.engram_hash_indices(cfg, proj, ids, w.B, w.T, None, idx, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        eg.engram_gather(cfg, idx, table, N, e, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        eg.engram_forward(cfg, idx, None, e, dense["h"], dense["Wk"], dense["Wv"],
+                          dense["conv_w"], None, out, saved, w.B, w.T, fws, fb, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if eg.engram_get_status(stream) != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    clocks = clk.summary()
+    elapsed_ms = start.elapsed_time(end)
+    t_hash = sum(ev[0].elapsed_time(ev[1]) for ev in evs) / args.steps
+    t_gather = sum(ev[1].elapsed_time(ev[2]) for ev in evs) / args.steps
+    t_fuse = sum(ev[2].elapsed_time(ev[3]) for ev in evs) / args.steps
+    if eg.engram_get_status(stream) != 0:
+        raise RuntimeError("device status word set during timing")
+    elapsed_ms = max_over_ranks(elapsed_ms)
+    ms_per_step = elapsed_ms / args.steps
+    value = N * ws_ * args.steps / (elapsed_ms / 1e3)
+
+    # ---- end to end through the public API with host buffers
+    ids_h = torch.from_numpy(ids_np).pin_memory()
+    h_h = dense["h"].cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    ids_d = torch.empty_like(ids)
+    h_d = torch.empty_like(dense["h"])
+
+    def e2e_step():
+        ids_d.copy_(ids_h, non_blocking=True)
+        h_d.copy_(h_h, non_blocking=True)
+        eg.engram_hash_indices(cfg, proj, ids_d, w.B, w.T, None, idx, stream)
+        eg.engram_forward(cfg, idx, table, e, h_d, dense["Wk"], dense["Wv"], dense["conv_w"],
+                          None, out, saved, w.B, w.T, fws, fb, stream)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_steps = max(3, min(args.steps, 20))
+    barrier()
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2))
+    e2e_value = N * ws_ * e2e_steps / (e2e_ms / 1e3)
+    h2d = ids_h.numel() * 4 + h_h.numel() * 2
+    d2h = out_h.numel() * 2
+
+    # ---- roofline of the dominant kernel (the two fused tensor-core passes)
+    peaks, peak_src = load_peaks()
+    flops = 2 * 2.0 * N * w.E * w.d            # k and v projections, algorithmic
+    achieved = flops / (t_fuse / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic_layer27b.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            traffic = json.load(f).get("fused_tc_traffic_bytes_per_step")
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if ws_ == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline_ours(w, ids_np, keys_np, mult, table, dense)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Zipf(1.1) ids, N(0,0.02) bf16 table and weights, N(0,1) h)",
+            "config": {
+                "workload": "layer27b: 27B-shaped Engram layer forward, 8 x 4,096 tokens, "
+                            "d_model 2,560, orders {2,3} x 8 heads x 80 dims, 16 primes "
+                            "<= 4,450,001 (5.7B bf16 params), vocab 129,280 -> 99,546",
+                "global_batch": N * ws_, "seq_len": w.T, "parallelism": f"dp{ws_} (replicas)",
+                "l2": "inputs larger than L2 (table 11.4 GB, h 168 MB per step); no flush",
+            },
+            "breakdown_ms": {"hash": t_hash, "gather": t_gather, "fused_tc_passes": t_fuse},
+            "gather_gbs": (N * w.J * 4 + N * w.J * w.D_h * 2 + N * w.E * 2) / (t_gather / 1e3) / 1e9,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "tc_fused_kernel (pass K + pass V)",
+                         "peak_source": f"{peak_src} bf16_tflops (burst)"},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+    barrier()
+    return line
+
+
+def cpu_baseline_ours(w, ids_np, keys_np, mult, table, dense):
+    """The oracle on a bounded sample of the same workload (one sequence)."""
+    import torch
+    from oracle import engram_oracle as O
+    base = np.concatenate([[0], np.cumsum(w.rows)[:-1]])
+    n_seq = 2
+    dense_host = {
+        "h": dense["h"][:n_seq].reshape(-1, 1, w.d).double().cpu().numpy(),
+        "Wk": dense["Wk"].double().cpu().numpy(),
+        "Wv": dense["Wv"].double().cpu().numpy(),
+        "conv_w": dense["conv_w"].double().cpu().numpy(),
+    }
+
+    def rows_fn(idx):
+        r = torch.from_numpy((base[None, :] + idx).reshape(-1)).to(table.device)
+        rows = table.view(-1, w.D_h).index_select(0, r).double().cpu().numpy()
+        return rows.reshape(idx.shape[0], w.E)
+
+    tok, sec, thr = oracle_sample(w, ids_np, keys_np, mult, rows_fn, dense_host, n_seq, w.T)
+    return {"value": tok / sec, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "sample": f"first {n_seq} sequences of the batch ({tok} tokens), oracle end to "
+                      f"end in fp64 ({sec:.1f} s)"}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: each step is the first
+    1,024 tokens of one sequence of this workload, end to end.  Needs no GPU:
+    the table rows the sample touches are drawn on the host, row by row, with
+    the workload's N(0, 0.02) statistics."""
+    from hashed_gram_conditional_engram_b200 import synth
+    ws_, rank = dist_init("gloo")
+    if rank != 0:
+        barrier()
+        return None
+    w = synth.workload(WORKLOAD)
+    ids_np, keys_np = synth.host_ids_keys(w)
+    mult = synth.hash_multipliers(synth.layer_seed(w, 0), w.J)
+    rng = np.random.default_rng(w.seed + 3)
+    n_tok = 1024
+    dense_host = {
+        "h": rng.standard_normal((n_tok, 1, w.d)),
+        "Wk": rng.standard_normal((1, w.d, w.E)) * 0.02,
+        "Wv": rng.standard_normal((w.d, w.E)) * 0.02,
+        "conv_w": rng.standard_normal((w.d, 4)) * 0.5,
+    }
+    cache = {}
+
+    def rows_fn(idx):
+        # rows drawn on demand per (head, slot): the same row always gets the
+        # same values, as a stored table would give
+        out = np.empty((idx.shape[0], w.E))
+        for j in range(w.J):
+            for n, s in enumerate(idx[:, j].tolist()):
+                key = (j, s)
+                if key not in cache:
+                    cache[key] = np.random.default_rng(hash(key) & 0xffffffff).standard_normal(w.D_h) * 0.02
+                out[n, j * w.D_h:(j + 1) * w.D_h] = cache[key]
+        return out
+
+    times, thr = [], 1
+    for i in range(args.warmup + args.steps):
+        tok, sec, thr = oracle_sample(w, ids_np, keys_np, mult, rows_fn, dense_host, 1, n_tok)
+        if i >= args.warmup:
+            times.append(sec)
+    sec = sum(times) / len(times)
+    value = n_tok / sec
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": "layer27b: 27B-shaped Engram layer forward, 8 x 4,096 tokens, "
+                               "d_model 2,560, orders {2,3} x 8 heads x 80 dims; oracle sample: "
+                               "1,024 tokens per step", "global_batch": n_tok, "seq_len": w.T,
+                   "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                         "sample": "first 1,024 tokens of one sequence per step, end to end "
+                                   "in fp64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    barrier()
+    return line
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

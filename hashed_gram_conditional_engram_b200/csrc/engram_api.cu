@@ -1,0 +1,282 @@
+// C ABI of libengram_b200.so: argument checks, workspace carving, launches.
+// Declarations and their contracts: include/engram.h.
+#include <cstring>
+#include <mutex>
+
+#include "internal.cuh"
+
+namespace engram {
+
+namespace {
+
+__device__ unsigned int g_status;  // one status word per device
+
+constexpr int kMaxDevices = 64;
+unsigned int* g_status_addr[kMaxDevices] = {nullptr};
+std::mutex g_status_mu;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cfg(const engram_cfg_t* c) {
+  if (c == nullptr) return ENGRAM_ERR_INVALID_ARG;
+  if (c->K < 1 || 2 * c->K > ENGRAM_MAX_HEADS || (2 * c->K) % 4 != 0) return ENGRAM_ERR_INVALID_ARG;
+  if (c->D_h < 1 || c->d_model < 1 || c->n_branch < 1) return ENGRAM_ERR_INVALID_ARG;
+  if (c->V_raw < 1 || c->V_c < 1 || c->V_c > c->V_raw) return ENGRAM_ERR_INVALID_ARG;
+  if (c->dtype != ENGRAM_F32 && c->dtype != ENGRAM_BF16) return ENGRAM_ERR_INVALID_ARG;
+  const int es = c->dtype == ENGRAM_F32 ? 4 : 2;
+  if ((c->D_h * es) % 16 != 0) return ENGRAM_ERR_MISALIGNED;
+  for (int j = 0; j < 2 * c->K; ++j) {
+    const int64_t P = c->rows[j];
+    // slots must fit int32 and a prime row count is odd and > 2
+    if (P < 3 || P > 0x7fffffffLL || (P & 1) == 0) return ENGRAM_ERR_INVALID_ARG;
+  }
+  return ENGRAM_OK;
+}
+
+inline int elem_bytes(const engram_cfg_t* c) { return c->dtype == ENGRAM_F32 ? 4 : 2; }
+
+}  // namespace
+
+unsigned int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (g_status_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    g_status_addr[dev] = static_cast<unsigned int*>(p);
+  }
+  return g_status_addr[dev];
+}
+
+HeadParams make_head_params(const engram_cfg_t* cfg) {
+  HeadParams hp;
+  std::memset(&hp, 0, sizeof(hp));
+  hp.K = cfg->K;
+  hp.J = 2 * cfg->K;
+  hp.D_h = cfg->D_h;
+  hp.E = hp.J * cfg->D_h;
+  hp.V_raw = cfg->V_raw;
+  hp.V_c = cfg->V_c;
+  int64_t base = 0;
+  for (int j = 0; j < hp.J; ++j) {
+    for (int i = 0; i < 3; ++i) hp.mult[j][i] = cfg->mult[j][i];
+    hp.P[j] = (uint64_t)cfg->rows[j];
+    hp.mu[j] = ~0ull / hp.P[j];
+    hp.row_base[j] = base;
+    base += cfg->rows[j];
+  }
+  return hp;
+}
+
+}  // namespace engram
+
+using namespace engram;
+
+extern "C" {
+
+size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n) {
+  if (n < 0) return 0;
+  if (call == ENGRAM_WS_VOCAB) return vocab_ws_bytes(n);
+  if (check_cfg(cfg) != ENGRAM_OK) return 0;
+  const int M = cfg->n_branch, d = cfg->d_model, E = 2 * cfg->K * cfg->D_h;
+  switch (call) {
+    case ENGRAM_WS_FORWARD:
+      if (cfg->dtype == ENGRAM_F32) return f32_saved_bytes(n, M, d);
+      return tc_forward_ws_bytes(n, d, E);
+    case ENGRAM_WS_BACKWARD:
+      return backward_f32_ws_bytes(n, M, d, E) + table_grad_ws_bytes(n * 2 * cfg->K);
+    case ENGRAM_WS_TABLE_GRAD:
+      return table_grad_ws_bytes(n * 2 * cfg->K);
+    default:
+      return 0;
+  }
+}
+
+size_t engram_saved_size(const engram_cfg_t* cfg, int64_t n_tok) {
+  if (check_cfg(cfg) != ENGRAM_OK || n_tok < 0) return 0;
+  if (cfg->dtype == ENGRAM_F32) return f32_saved_bytes(n_tok, cfg->n_branch, cfg->d_model);
+  return (size_t)n_tok * cfg->n_branch * sizeof(float);  // alpha
+}
+
+int engram_build_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_c_out,
+                            void* ws, size_t ws_bytes, void* stream) {
+  if (V < 1 || keys == nullptr || proj == nullptr || V_c_out == nullptr || ws == nullptr)
+    return ENGRAM_ERR_INVALID_ARG;
+  if (!aligned16(keys) || !aligned16(proj) || !aligned16(ws)) return ENGRAM_ERR_MISALIGNED;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  return launch_vocab_proj(keys, V, proj, V_c_out, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+int engram_hash_indices(const engram_cfg_t* cfg, const int32_t* proj, const int32_t* ids,
+                        int32_t B, int32_t T, int32_t* ngram_state, int32_t* idx, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (B < 0 || T < 0 || proj == nullptr || idx == nullptr || (B * (int64_t)T > 0 && ids == nullptr))
+    return ENGRAM_ERR_INVALID_ARG;
+  if (ngram_state != nullptr && T != 1) return ENGRAM_ERR_INVALID_ARG;
+  if (!aligned16(proj) || !aligned16(ids) || !aligned16(idx) ||
+      (ngram_state && !aligned16(ngram_state)))
+    return ENGRAM_ERR_MISALIGNED;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  return launch_hash(make_head_params(cfg), proj, ids, B, T, ngram_state, idx,
+                     (cudaStream_t)stream);
+}
+
+int engram_gather(const engram_cfg_t* cfg, const int32_t* idx, const void* table, int64_t n_tok,
+                  void* e, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (n_tok < 0 || (n_tok > 0 && (idx == nullptr || table == nullptr || e == nullptr)))
+    return ENGRAM_ERR_INVALID_ARG;
+  if (!aligned16(idx) || !aligned16(table) || !aligned16(e)) return ENGRAM_ERR_MISALIGNED;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  return launch_gather(make_head_params(cfg), idx, table, n_tok, elem_bytes(cfg), e,
+                       (cudaStream_t)stream);
+}
+
+int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* table, void* e,
+                   const void* h, const void* Wk, const void* Wv, const float* conv_w,
+                   float* conv_state, void* out, float* saved, int32_t B, int32_t T, void* ws,
+                   size_t ws_bytes, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (B < 0 || T < 0) return ENGRAM_ERR_INVALID_ARG;
+  const int64_t N = (int64_t)B * T;
+  if (conv_state != nullptr && T != 1) return ENGRAM_ERR_INVALID_ARG;
+  if (N == 0) return ENGRAM_OK;
+  if (e == nullptr || h == nullptr || Wk == nullptr || Wv == nullptr || conv_w == nullptr ||
+      out == nullptr || (table != nullptr && idx == nullptr))
+    return ENGRAM_ERR_INVALID_ARG;
+  if (!aligned16(idx) || !aligned16(table) || !aligned16(e) || !aligned16(h) || !aligned16(Wk) ||
+      !aligned16(Wv) || !aligned16(conv_w) || !aligned16(conv_state) || !aligned16(out) ||
+      !aligned16(saved) || !aligned16(ws))
+    return ENGRAM_ERR_MISALIGNED;
+  if (ws_bytes < engram_workspace_size(cfg, ENGRAM_WS_FORWARD, N)) return ENGRAM_ERR_WORKSPACE;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  const HeadParams hp = make_head_params(cfg);
+  const int M = cfg->n_branch, d = cfg->d_model, E = hp.E;
+  if (cfg->dtype == ENGRAM_BF16 && !tc_supported(d, E, M)) return ENGRAM_ERR_UNSUPPORTED;
+  if (table != nullptr) {
+    rc = launch_gather(hp, idx, table, N, elem_bytes(cfg), e, s);
+    if (rc) return rc;
+  }
+  if (cfg->dtype == ENGRAM_F32) {
+    void* sv_base = saved != nullptr ? static_cast<void*>(saved) : ws;
+    F32Saved sv = f32_saved_layout(sv_base, N, M, d);
+    return launch_forward_f32(static_cast<const float*>(e), static_cast<const float*>(h),
+                              static_cast<const float*>(Wk), static_cast<const float*>(Wv), conv_w,
+                              conv_state, static_cast<float*>(out), sv, N, T, M, d, E, s);
+  }
+  return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
+                           static_cast<const __nv_bfloat16*>(Wk),
+                           static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
+                           static_cast<__nv_bfloat16*>(out), saved, N, T, d, E, ws, ws_bytes, s);
+}
+
+int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,
+                    const void* Wk, const void* Wv, const float* conv_w, const float* saved,
+                    const float* dout, float* dh, float* dWk, float* dWv, float* dconv_w, float* de,
+                    int64_t* dtab_keys, float* dtab_rows, int32_t* n_unique, int32_t B, int32_t T,
+                    void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (cfg->dtype != ENGRAM_F32) return ENGRAM_ERR_UNSUPPORTED;
+  if (B < 0 || T < 0) return ENGRAM_ERR_INVALID_ARG;
+  const int64_t N = (int64_t)B * T;
+  if (idx == nullptr || e == nullptr || h == nullptr || Wk == nullptr || Wv == nullptr ||
+      conv_w == nullptr || saved == nullptr || dout == nullptr || dh == nullptr || dWk == nullptr ||
+      dWv == nullptr || dconv_w == nullptr || dtab_keys == nullptr || dtab_rows == nullptr ||
+      n_unique == nullptr || ws == nullptr)
+    return ENGRAM_ERR_INVALID_ARG;
+  if (!aligned16(idx) || !aligned16(e) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) ||
+      !aligned16(conv_w) || !aligned16(saved) || !aligned16(dout) || !aligned16(dh) ||
+      !aligned16(dWk) || !aligned16(dWv) || !aligned16(dconv_w) || !aligned16(de) ||
+      !aligned16(dtab_keys) || !aligned16(dtab_rows) || !aligned16(ws))
+    return ENGRAM_ERR_MISALIGNED;
+  if (ws_bytes < engram_workspace_size(cfg, ENGRAM_WS_BACKWARD, N)) return ENGRAM_ERR_WORKSPACE;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  const HeadParams hp = make_head_params(cfg);
+  const int M = cfg->n_branch, d = cfg->d_model, E = hp.E;
+  const size_t bw = backward_f32_ws_bytes(N, M, d, E);
+  // de lives at the end of the dense-backward workspace unless the caller wants it
+  float* de_buf = de;
+  if (de_buf == nullptr) {
+    const size_t de_bytes = ((size_t)N * E * 4 + 255) & ~(size_t)255;
+    de_buf = reinterpret_cast<float*>(static_cast<char*>(ws) + bw - de_bytes);
+  }
+  F32Saved sv = f32_saved_layout(const_cast<float*>(saved), N, M, d);
+  rc = launch_backward_f32(static_cast<const float*>(e), static_cast<const float*>(h),
+                           static_cast<const float*>(Wk), static_cast<const float*>(Wv), conv_w,
+                           sv, dout, dh, dWk, dWv, dconv_w, de_buf, N, T, M, d, E, ws, s);
+  if (rc) return rc;
+  return launch_table_grad(hp, idx, de_buf, N, dtab_keys, dtab_rows, n_unique,
+                           static_cast<char*>(ws) + bw, ws_bytes - bw, s);
+}
+
+int engram_table_grad(const engram_cfg_t* cfg, const int32_t* idx, const float* de, int64_t n_tok,
+                      int64_t* dtab_keys, float* dtab_rows, int32_t* n_unique, void* ws,
+                      size_t ws_bytes, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (n_tok < 0 || n_unique == nullptr) return ENGRAM_ERR_INVALID_ARG;
+  if (n_tok > 0 && (idx == nullptr || de == nullptr || dtab_keys == nullptr ||
+                    dtab_rows == nullptr || ws == nullptr))
+    return ENGRAM_ERR_INVALID_ARG;
+  if ((int64_t)n_tok * 2 * cfg->K >= 0x7fffffffLL) return ENGRAM_ERR_UNSUPPORTED;
+  if (!aligned16(idx) || !aligned16(de) || !aligned16(dtab_keys) || !aligned16(dtab_rows) ||
+      !aligned16(ws))
+    return ENGRAM_ERR_MISALIGNED;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  return launch_table_grad(make_head_params(cfg), idx, de, n_tok, dtab_keys, dtab_rows, n_unique,
+                           ws, ws_bytes, (cudaStream_t)stream);
+}
+
+int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const void* host_table,
+                             int64_t n_tok, void* e, void* side_stream, void* done_event) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (n_tok < 0 || (n_tok > 0 && (idx == nullptr || host_table == nullptr || e == nullptr)))
+    return ENGRAM_ERR_INVALID_ARG;
+  if (!aligned16(idx) || !aligned16(host_table) || !aligned16(e)) return ENGRAM_ERR_MISALIGNED;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)side_stream;
+  if (n_tok > 0) {
+    // the device-side address of the pinned host range (equal to the host
+    // address under unified addressing; fails if the memory is not mapped)
+    void* dev_ptr = nullptr;
+    if (cudaHostGetDevicePointer(&dev_ptr, const_cast<void*>(host_table), 0) != cudaSuccess) {
+      cudaGetLastError();
+      return ENGRAM_ERR_INVALID_ARG;
+    }
+    rc = launch_gather(make_head_params(cfg), idx, dev_ptr, n_tok, elem_bytes(cfg), e, s);
+    if (rc) return rc;
+  }
+  if (done_event != nullptr) return ck(cudaEventRecord((cudaEvent_t)done_event, s));
+  return ENGRAM_OK;
+}
+
+int engram_get_status(void* stream) {
+  unsigned int* p = status_ptr();
+  if (p == nullptr) return ENGRAM_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned int v = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ENGRAM_ERR_CUDA;
+  if (cudaMemcpyAsync(&v, p, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ENGRAM_ERR_CUDA;
+  if (cudaMemsetAsync(p, 0, sizeof(v), s) != cudaSuccess) return ENGRAM_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ENGRAM_ERR_CUDA;
+  return (int)(v & 0x7fffffffu);
+}
+
+int engram_device_sm_count(void) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ENGRAM_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return ENGRAM_ERR_CUDA;
+  return sms;
+}
+
+}  // extern "C"

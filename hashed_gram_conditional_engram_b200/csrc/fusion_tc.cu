@@ -1,0 +1,681 @@
+// bf16 fusion stage on the sm_100a tensor cores.
+//
+// The two projections k = W_k e and v = W_v e are the layer's only dense
+// contractions (discuss.deepseek.club 二.1 (2): h is the query, e the key and
+// value, combined by matrix products).  Each runs as one persistent tcgen05
+// GEMM pass with the rest of the layer fused into its epilogue:
+//
+//   pass K:  C = e * W_k^T tile by tile; the epilogue reduces each row of the
+//            tile to (sum k^2, sum h*k, sum h^2) partials -- k never reaches HBM.
+//   pass V:  C = e * W_v^T; the epilogue finishes the gate from the partials,
+//            alpha = sigmoid(<h, k> r_h r_k / sqrt(d)), scales v, runs the
+//            width-4 depthwise causal conv along the rows of the tile, applies
+//            SiLU and adds h + vt + SiLU(y) (sechub.in answer: short depthwise
+//            causal conv; discuss.deepseek.club 二.1 (2): 1-D conv, residual).
+//
+// The causal conv needs vt of the three tokens before each row.  Pass V walks
+// the tokens in overlapping tiles of 128 rows that advance by 125: the first
+// three rows of a tile are a recomputed halo and produce no output.  In decode
+// (one token per sequence) the three earlier vt come from the conv state.
+//
+// Pipeline per CTA (one CTA per SM, 320 threads):
+//   warp 0      one lane issues TMA loads of A (e) and B (W) tiles into a ring
+//               of shared-memory stages (128-byte swizzle, K-major);
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
+//               K=16 per instruction) into one of two TMEM accumulators;
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4).. (its rows), half
+//               of the tile's columns each, 32 columns per tcgen05.ld.
+// mbarriers link the roles; every wait is bounded in time and, when it runs
+// out, sets ENGRAM_STATUS_TIMEOUT and winds the CTA down without hanging.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "internal.cuh"
+
+namespace engram {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle row
+constexpr int UMMA_K = 16;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + NUM_EPI_WARPS * 32;
+constexpr int HALO = 3;  // conv width 4 - 1
+constexpr float RMS_EPS = 1e-6f;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
+constexpr unsigned FULL = 0xffffffffu;
+
+enum { MODE_GATE_PARTIAL = 0, MODE_VALUE_CONV = 1 };
+
+struct TcArgs {
+  int num_m_tiles, num_n_tiles, num_k_tiles;
+  int m_stride, m_offset;
+  int64_t N;
+  int T;
+  int d;
+  int n_part;
+  const __nv_bfloat16* h;
+  __nv_bfloat16* out;
+  float4* part;
+  const float4* conv_w;
+  float* conv_state;
+  float* alpha_out;
+  unsigned int* status;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait until the phase of `bar` with the given parity has completed.  Gives
+// up (returns false) when the CTA is aborting or after WAIT_LIMIT_NS, which
+// starts the abort and flags the status word.
+__device__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                             unsigned int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spin & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > WAIT_LIMIT_NS) {
+        *abort_flag = 1;
+        atomicOr(status, ENGRAM_STATUS_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Same, ignoring the abort flag: used to let in-flight copies and MMAs land
+// before the CTA releases its shared memory and TMEM.
+__device__ bool wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand tile written by TMA
+// with 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);  // start address
+  d |= (uint64_t)1 << 16;                   // leading byte offset (unused when swizzled)
+  d |= (uint64_t)(1024 >> 4) << 32;         // stride byte offset: 8 rows x 128 B
+  d |= (uint64_t)1 << 46;                   // descriptor version of sm_100
+  d |= (uint64_t)2 << 61;                   // 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
+  uint32_t u[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+        "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
+        "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]),
+        "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]), "=r"(u[25]),
+        "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// 32 bf16 (64 bytes) -> fp32
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, float (&x)[32]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint4 w = __ldg(q + v);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[v * 8 + 2 * i] = __uint_as_float(ws[i] << 16);
+      x[v * 8 + 2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int BN, int STAGES>
+struct TcShape {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int HALF_COLS = BN / 2;
+  static constexpr int NCHUNK = HALF_COLS / 32;
+  static constexpr int XBUF_FLOATS = 2 * 2 * NCHUNK * 4 * 3 * 32;  // [parity][half][chunk][quad][3][32]
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 +
+                                 (size_t)XBUF_FLOATS * 4;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "N tile");
+  static_assert(2 * STAGES + 5 <= 30, "barrier area");
+};
+
+template <int BN, int STAGES, int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ TcArgs args) {
+  using S = TcShape<BN, STAGES>;
+  constexpr uint32_t STAGE_TX = S::A_BYTES + S::B_BYTES;
+  // instruction descriptor: fp32 accumulate, bf16 A and B, both K-major,
+  // N >> 3 at bit 17, M >> 4 at bit 24
+  constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                             ((uint32_t)(BM >> 4) << 24);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * S::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * S::B_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 30);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 31);
+  float* xbuf = reinterpret_cast<float*>(bars + 32);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_tiles = args.num_m_tiles * args.num_n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], NUM_EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int mt = tile / args.num_n_tiles, nt = tile - mt * args.num_n_tiles;
+        const int row0 = mt * args.m_stride + args.m_offset;
+        const int col0 = nt * BN;
+        bool ok = true;
+        for (int kt = 0; kt < args.num_k_tiles; ++kt) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[stage], STAGE_TX);
+          tma_load_2d(sA + stage * S::A_BYTES, &tmA, &full[stage], kt * BK, row0);
+          tma_load_2d(sB + stage * S::B_BYTES, &tmB, &full[stage], kt * BK, col0);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      // every issued copy must land before the CTA exits
+      for (int s = 0; s < STAGES; ++s) {
+        const uint32_t n_s = issued > (uint32_t)s ? (issued - 1 - s) / STAGES + 1 : 0;
+        if (n_s > 0) wait_drain(&full[s], (n_s - 1) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kt = 0; kt < args.num_k_tiles; ++kt) {
+          if (!wait_bounded(&full[stage], phase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * S::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * S::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            umma_bf16(d_tmem, sw128_desc(a0 + k * UMMA_K * 2), sw128_desc(b0 + k * UMMA_K * 2),
+                      IDESC, (kt | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // all issued MMAs complete before TMEM is released
+      umma_commit(drain);
+      wait_drain(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int quad = warp & 3;  // TMEM lanes this warp may read
+    const int half = ew >> 2;   // column half of the tile
+    const int rloc = quad * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int iter = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
+      const int mt = tile / args.num_n_tiles, nt = tile - mt * args.num_n_tiles;
+      int got = 0;
+      if (lane == 0) got = wait_bounded(&tfull[acc], acc_phase, abort_flag, args.status) ? 1 : 0;
+      got = __shfl_sync(FULL, got, 0);
+      tc_fence_after();
+      const int64_t n = (int64_t)mt * args.m_stride + args.m_offset + rloc;
+      const bool valid = n >= 0 && n < args.N;
+      const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN) +
+                             (uint32_t)(half * S::HALF_COLS);
+      const int col_base = nt * BN + half * S::HALF_COLS;
+
+      if (MODE == MODE_GATE_PARTIAL) {
+        float kk = 0.f, hk = 0.f, hh = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < S::NCHUNK; ++c) {
+          float v[32];
+          __syncwarp();
+          if (got) {
+            tmem_ld32(t_row + c * 32, v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+          if (valid) {
+            float hv[32];
+            load_bf16x32(args.h + n * args.d + col_base + c * 32, hv);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              kk = fmaf(v[i], v[i], kk);
+              hk = fmaf(hv[i], v[i], hk);
+              hh = fmaf(hv[i], hv[i], hh);
+            }
+          }
+        }
+        if (valid) args.part[n * args.n_part + nt * 2 + half] = make_float4(kk, hk, hh, 0.f);
+      } else {
+        // gate of this row from the partials of every column tile
+        float alpha = 0.f;
+        if (valid) {
+          const float4* pr = args.part + n * args.n_part;
+          float kk = 0.f, hk = 0.f, hh = 0.f;
+          for (int i = 0; i < args.n_part; ++i) {
+            const float4 q = pr[i];
+            kk += q.x;
+            hk += q.y;
+            hh += q.z;
+          }
+          const float invd = 1.0f / (float)args.d;
+          const float rh = rsqrtf(hh * invd + RMS_EPS), rk = rsqrtf(kk * invd + RMS_EPS);
+          const float z = hk * rh * rk * rsqrtf((float)args.d);
+          alpha = 1.0f / (1.0f + expf(-z));
+        }
+        const bool decode = args.conv_state != nullptr;
+        const bool is_out = valid && rloc >= -args.m_offset;
+        if (is_out && args.alpha_out != nullptr && nt == 0 && half == 0) args.alpha_out[n] = alpha;
+        const int pos = valid ? (int)(n % args.T) : 0;
+#pragma unroll 1
+        for (int c = 0; c < S::NCHUNK; ++c) {
+          float v[32];
+          __syncwarp();
+          if (got) {
+            tmem_ld32(t_row + c * 32, v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= alpha;  // vt
+          const int col = col_base + c * 32;
+          const float* xp = nullptr;
+          if (!decode) {
+            // lanes 29..31 publish vt for lanes 0..2 of the next quadrant
+            float* xw =
+                xbuf + (((((iter & 1) * 2 + half) * S::NCHUNK + c) * 4 + quad) * 3) * 32;
+            if (lane >= 29) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) xw[(lane - 29) * 32 + i] = v[i];
+            }
+            named_bar_sync(1 + half, 128);
+            xp = xbuf +
+                 (((((iter & 1) * 2 + half) * S::NCHUNK + c) * 4 + ((quad + 3) & 3)) * 3) * 32;
+          }
+          float hv[32];
+          if (is_out) {
+            load_bf16x32(args.h + n * args.d + col, hv);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) hv[i] = 0.f;
+          }
+          float* st = (decode && is_out) ? args.conv_state + n * 3 * args.d + col : nullptr;
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float o[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int k = i + u;
+              float a1 = 0.f, a2 = 0.f, a3 = 0.f;  // vt of rows t-1, t-2, t-3
+              if (decode) {
+                if (st != nullptr) {
+                  a3 = st[k];
+                  a2 = st[args.d + k];
+                  a1 = st[2 * args.d + k];
+                  st[k] = a2;
+                  st[args.d + k] = a1;
+                  st[2 * args.d + k] = v[k];
+                }
+              } else {
+                float b1 = __shfl_up_sync(FULL, v[k], 1);
+                float b2 = __shfl_up_sync(FULL, v[k], 2);
+                float b3 = __shfl_up_sync(FULL, v[k], 3);
+                if (lane == 0) {
+                  b1 = xp[2 * 32 + k];
+                  b2 = xp[1 * 32 + k];
+                  b3 = xp[0 * 32 + k];
+                } else if (lane == 1) {
+                  b2 = xp[2 * 32 + k];
+                  b3 = xp[1 * 32 + k];
+                } else if (lane == 2) {
+                  b3 = xp[2 * 32 + k];
+                }
+                a1 = pos >= 1 ? b1 : 0.f;
+                a2 = pos >= 2 ? b2 : 0.f;
+                a3 = pos >= 3 ? b3 : 0.f;
+              }
+              const float4 w = __ldg(args.conv_w + col + k);
+              float y = w.w * v[k];
+              y = fmaf(w.z, a1, y);
+              y = fmaf(w.y, a2, y);
+              y = fmaf(w.x, a3, y);
+              const float sy = y / (1.0f + expf(-y));
+              o[u] = hv[k] + v[k] + sy;
+            }
+            packed[i / 2] = pack_bf16x2(o[0], o[1]);
+          }
+          if (is_out) {
+            uint4* dst = reinterpret_cast<uint4*>(args.out + n * args.d + col);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                                  packed[4 * q + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols contiguous), boxes of 64 columns x box_rows.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int MODE>
+int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, cudaStream_t s) {
+  using S = TcShape<BN, STAGES>;
+  auto kern = tc_fused_kernel<BN, STAGES, MODE>;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return ENGRAM_ERR_CUDA;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM) !=
+        cudaSuccess)
+      return ENGRAM_ERR_CUDA;
+    configured[dev] = true;
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = a.num_m_tiles * a.num_n_tiles;
+  const int grid = tiles < sms ? tiles : sms;
+  if (grid <= 0) return ENGRAM_OK;
+  kern<<<grid, NUM_THREADS, S::SMEM, s>>>(ta, tb, a);
+  return ck(cudaGetLastError());
+}
+
+template <int BN, int STAGES>
+int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
+              const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
+              float* alpha_saved, int64_t N, int T, int d, int E, float4* part,
+              cudaStream_t s) {
+  CUtensorMap ta, tbk, tbv;
+  if (!make_tmap(&ta, e, (uint64_t)E, (uint64_t)N, BM)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&tbk, Wk, (uint64_t)E, (uint64_t)d, BN)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&tbv, Wv, (uint64_t)E, (uint64_t)d, BN)) return ENGRAM_ERR_CUDA;
+  TcArgs a;
+  a.num_n_tiles = d / BN;
+  a.num_k_tiles = E / BK;
+  a.N = N;
+  a.T = T;
+  a.d = d;
+  a.n_part = 2 * a.num_n_tiles;
+  a.h = h;
+  a.out = out;
+  a.part = part;
+  a.conv_w = reinterpret_cast<const float4*>(conv_w);
+  a.conv_state = conv_state;
+  a.alpha_out = alpha_saved;
+  a.status = status_ptr();
+  // pass K: gate partials
+  a.m_stride = BM;
+  a.m_offset = 0;
+  a.num_m_tiles = (int)((N + BM - 1) / BM);
+  int rc = launch_pass<BN, STAGES, MODE_GATE_PARTIAL>(ta, tbk, a, s);
+  if (rc) return rc;
+  // pass V: gate, conv, residual (overlapping tiles with a 3-row halo, or
+  // plain tiles plus the conv state in decode)
+  if (conv_state != nullptr) {
+    a.m_stride = BM;
+    a.m_offset = 0;
+  } else {
+    a.m_stride = BM - HALO;
+    a.m_offset = -HALO;
+  }
+  a.num_m_tiles = (int)((N + a.m_stride - 1) / a.m_stride);
+  return launch_pass<BN, STAGES, MODE_VALUE_CONV>(ta, tbv, a, s);
+}
+
+inline bool use_wide(int64_t N, int d) { return d % 256 == 0 && N > 4096; }
+
+}  // namespace
+
+int tc_supported(int d, int E, int M) {
+  return M == 1 && E % BK == 0 && E >= BK && d % 64 == 0 && d >= 64;
+}
+
+size_t tc_forward_ws_bytes(int64_t N, int d, int E) {
+  (void)E;
+  const int BN = use_wide(N, d) ? 256 : 64;
+  return (size_t)N * 2 * (d / BN) * sizeof(float4);
+}
+
+int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
+                      const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
+                      __nv_bfloat16* out, float* alpha_saved, int64_t N, int T, int d, int E,
+                      void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (ws_bytes < tc_forward_ws_bytes(N, d, E) || ws == nullptr) return ENGRAM_ERR_WORKSPACE;
+  if (N > 0x7fffffffLL - 256) return ENGRAM_ERR_UNSUPPORTED;
+  float4* part = static_cast<float4*>(ws);
+  if (use_wide(N, d))
+    return run_layer<256, 4>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
+                             s);
+  return run_layer<64, 8>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part, s);
+}
+
+}  // namespace engram

@@ -1,0 +1,75 @@
+// Internal declarations shared by the translation units of libengram_b200.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/engram.h"
+
+namespace engram {
+
+// Per-head constants handed to kernels by value.
+struct HeadParams {
+  int J, K, D_h, E;
+  int32_t V_raw, V_c;
+  uint64_t mult[ENGRAM_MAX_HEADS][3];
+  uint64_t P[ENGRAM_MAX_HEADS];
+  uint64_t mu[ENGRAM_MAX_HEADS];        // floor((2^64 - 1) / P_j), Barrett reciprocal
+  int64_t row_base[ENGRAM_MAX_HEADS];   // first packed-table row of head j
+};
+
+HeadParams make_head_params(const engram_cfg_t* cfg);
+
+// The device status word of the current device (a __device__ variable).
+unsigned int* status_ptr();
+
+inline int ck(cudaError_t e) { return e == cudaSuccess ? ENGRAM_OK : ENGRAM_ERR_CUDA; }
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float bfbits2f(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+// ---------------------------------------------------------------- launches
+int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, int B, int T,
+                int32_t* ngram_state, int32_t* idx, cudaStream_t s);
+int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,
+                  int elem_bytes, void* e, cudaStream_t s);
+
+// fp32 CUDA-core path (small layers)
+struct F32Saved {
+  float* alpha;   // [N, M]
+  float* k;       // [N, M, d]
+  float* v;       // [N, d]
+  float* y;       // [N, M, d]
+};
+F32Saved f32_saved_layout(void* base, int64_t N, int M, int d);
+size_t f32_saved_bytes(int64_t N, int M, int d);
+int launch_forward_f32(const float* e, const float* h, const float* Wk, const float* Wv,
+                       const float* conv_w, float* conv_state, float* out, F32Saved sv, int64_t N,
+                       int T, int M, int d, int E, cudaStream_t s);
+size_t backward_f32_ws_bytes(int64_t N, int M, int d, int E);
+int launch_backward_f32(const float* e, const float* h, const float* Wk, const float* Wv,
+                        const float* conv_w, F32Saved sv, const float* dout, float* dh, float* dWk,
+                        float* dWv, float* dconv_w, float* de, int64_t N, int T, int M, int d,
+                        int E, void* ws, cudaStream_t s);
+
+// sort / scan / segmented reduce
+size_t table_grad_ws_bytes(int64_t n_items);
+int launch_table_grad(const HeadParams& hp, const int32_t* idx, const float* de, int64_t n_tok,
+                      int64_t* keys, float* rows, int32_t* n_unique, void* ws, size_t ws_bytes,
+                      cudaStream_t s);
+size_t vocab_ws_bytes(int64_t V);
+int launch_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_c_out, void* ws,
+                      size_t ws_bytes, cudaStream_t s);
+
+// bf16 tensor-core path (sm_100a tcgen05)
+size_t tc_forward_ws_bytes(int64_t N, int d, int E);
+int tc_supported(int d, int E, int M);
+int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
+                      const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
+                      __nv_bfloat16* out, float* alpha_saved, int64_t N, int T, int d, int E,
+                      void* ws, size_t ws_bytes, cudaStream_t s);
+
+}  // namespace engram

@@ -1,0 +1,167 @@
+// Retrieval kernels: fused compress + suffix n-gram + multi-head hash, and the
+// row gather that builds e_t.
+//
+// Method: discuss.deepseek.club 二.1 (1) (vocabulary projection, multi-head
+// hashing into per-head tables, concatenation of the retrieved rows);
+// gitcode.csdn.net blog "Engram 到底怎么工作的", 第一步 / 第二步 (the last two and
+// last three tokens address several slots of a large table).
+#include "internal.cuh"
+
+namespace engram {
+
+namespace {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// x mod P for P < 2^63 odd, by Barrett reduction (P. Barrett, CRYPTO '86):
+// with mu = floor((2^64-1)/P) = floor(2^64/P) (P does not divide 2^64),
+// q = floor(x*mu / 2^64) is floor(x/P) or one less, so one conditional
+// subtraction finishes the remainder.
+__device__ __forceinline__ uint64_t mod_prime(uint64_t x, uint64_t P, uint64_t mu) {
+  uint64_t q = __umul64hi(x, mu);
+  uint64_t r = x - q * P;
+  return r >= P ? r - P : r;
+}
+
+// Compressed id of flat token m, PAD for m < 0; -1 for a raw id out of range.
+__device__ __forceinline__ int32_t token_cid(const int32_t* __restrict__ proj,
+                                             const int32_t* __restrict__ ids, int64_t m,
+                                             int32_t V_raw, int32_t pad) {
+  if (m < 0) return pad;
+  int32_t x = __ldg(ids + m);
+  if (x < 0 || x >= V_raw) return -1;
+  return __ldg(proj + x);
+}
+
+// One thread per token in flat order.  c_{t-1} and c_{t-2} travel from the
+// neighbouring lanes by warp shuffles; lanes 0 and 1 fetch the two tokens
+// before the warp themselves.
+__global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HeadParams hp,
+                                                   const int32_t* __restrict__ proj,
+                                                   const int32_t* __restrict__ ids, int64_t N,
+                                                   int T, int32_t* __restrict__ ngram_state,
+                                                   int32_t* __restrict__ idx,
+                                                   unsigned int* status) {
+  const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int32_t pad = hp.V_c;
+  const bool live = n < N;
+
+  int32_t c0 = live ? token_cid(proj, ids, n, hp.V_raw, pad) : pad;
+  int32_t c1 = __shfl_up_sync(FULL, c0, 1);
+  int32_t c2 = __shfl_up_sync(FULL, c0, 2);
+  if (!live) return;
+  if (lane == 0) c1 = token_cid(proj, ids, n - 1, hp.V_raw, pad);
+  if (lane <= 1) c2 = token_cid(proj, ids, n - 2, hp.V_raw, pad);
+
+  if (ngram_state != nullptr) {
+    // decode: one token per sequence, history from the rolling state
+    c1 = ngram_state[2 * n + 0];
+    c2 = ngram_state[2 * n + 1];
+    ngram_state[2 * n + 0] = c0;
+    ngram_state[2 * n + 1] = c1;
+  } else {
+    const int t = (int)(n % T);
+    if (t < 1) c1 = pad;
+    if (t < 2) c2 = pad;
+  }
+  if (c0 < 0) atomicOr(status, ENGRAM_STATUS_BAD_ID);
+  const bool bad2 = (c0 < 0) | (c1 < 0);
+  const bool bad3 = bad2 | (c2 < 0);
+
+  const uint64_t g0 = (uint64_t)(uint32_t)c0, g1 = (uint64_t)(uint32_t)c1,
+                 g2 = (uint64_t)(uint32_t)c2;
+  int32_t* dst = idx + n * hp.J;
+  // J is a multiple of 4 (host check): 16-byte stores of four slots
+  for (int j0 = 0; j0 < hp.J; j0 += 4) {
+    int32_t s[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u;
+      uint64_t x = g0 * hp.mult[j][0];
+      x ^= g1 * hp.mult[j][1];
+      const bool tri = j >= hp.K;
+      if (tri) x ^= g2 * hp.mult[j][2];
+      const bool bad = tri ? bad3 : bad2;
+      s[u] = bad ? -1 : (int32_t)mod_prime(x, hp.P[j], hp.mu[j]);
+    }
+    *reinterpret_cast<int4*>(dst + j0) = make_int4(s[0], s[1], s[2], s[3]);
+  }
+}
+
+// Row gather with 16-byte vectors.  The e row of a token is J*CR chunks of 16
+// bytes (CR per head row); consecutive threads take consecutive chunks, so the
+// stores are fully coalesced and each head row is read as CR adjacent
+// vectors.  Every thread keeps UNROLL loads in flight before storing.
+template <int UNROLL>
+__global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ HeadParams hp,
+                                                     const int32_t* __restrict__ idx,
+                                                     const uint4* __restrict__ table,
+                                                     int64_t n_tok, int CR,
+                                                     uint4* __restrict__ e,
+                                                     unsigned int* status) {
+  const int per_tok = hp.J * CR;
+  const int64_t total = n_tok * per_tok;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < total;
+       base += stride * UNROLL) {
+    uint4 v[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t g = base + u * stride;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (g < total) {
+        const int64_t n = g / per_tok;
+        const int r = (int)(g - n * per_tok);
+        const int j = r / CR;
+        const int c = r - j * CR;
+        const int32_t s = __ldg(idx + n * hp.J + j);
+        if (s >= 0 && (uint64_t)s < hp.P[j]) {
+          v[u] = __ldg(table + (hp.row_base[j] + s) * CR + c);
+        } else if (s != -1) {
+          atomicOr(status, ENGRAM_STATUS_BAD_INDEX);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t g = base + u * stride;
+      if (g < total) e[g] = v[u];
+    }
+  }
+}
+
+}  // namespace
+
+int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, int B, int T,
+                int32_t* ngram_state, int32_t* idx, cudaStream_t s) {
+  const int64_t N = (int64_t)B * T;
+  if (N == 0) return ENGRAM_OK;
+  const int threads = 256;
+  const int64_t blocks = (N + threads - 1) / threads;
+  hash_kernel<<<(unsigned)blocks, threads, 0, s>>>(hp, proj, ids, N, T, ngram_state, idx,
+                                                   status_ptr());
+  return ck(cudaGetLastError());
+}
+
+int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,
+                  int elem_bytes, void* e, cudaStream_t s) {
+  if (n_tok == 0) return ENGRAM_OK;
+  const int CR = hp.D_h * elem_bytes / 16;
+  const int64_t total = n_tok * hp.J * CR;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  constexpr int UNROLL = 8;
+  const int threads = 256;
+  int64_t blocks = (total + (int64_t)threads * UNROLL - 1) / ((int64_t)threads * UNROLL);
+  const int64_t cap = (int64_t)sms * 8;  // 8 resident blocks of 256 threads per SM
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  gather_kernel<UNROLL><<<(unsigned)blocks, threads, 0, s>>>(
+      hp, idx, static_cast<const uint4*>(table), n_tok, CR, static_cast<uint4*>(e),
+      status_ptr());
+  return ck(cudaGetLastError());
+}
+
+}  // namespace engram

@@ -1,0 +1,240 @@
+/*
+ * engram.h -- C ABI of libengram_b200.so, the Engram conditional-memory layer
+ * on B200 (sm_100a).
+ *
+ * The layer ("Conditional Memory via Scalable Lookup: A New Axis of Sparsity
+ * for Large Language Models", as summarised by the pages cited below) does,
+ * for every token position t of every sequence:
+ *   1. compress the raw id through a vocabulary projection,
+ *   2. form the suffix 2-gram and 3-gram of compressed ids,
+ *   3. hash each n-gram through K independent heads into per-head tables,
+ *   4. gather and concatenate the J = 2K head rows into e_t,
+ *   5. gate a value projection by alpha_t = sigmoid(<RMSNorm(h_t), RMSNorm(W_k e_t)>/sqrt(d)),
+ *   6. pass alpha_t * W_v e_t through a width-4 depthwise causal conv with SiLU
+ *      and add both onto the residual stream:
+ *        out_t = h_t + vt_t + SiLU(sum_i w[:, i] * vt_{t-3+i}),  vt = alpha * W_v e.
+ *
+ * Page citations used below:
+ *   [p1] reportify.cn tag page 条件记忆, digests 技术方案 / 技术创新与架构 / 关键技术
+ *   [p2] sechub.in answer: 2-/3-gram suffixes, gate, short depthwise causal conv,
+ *        indices known before the forward pass, host-memory prefetch
+ *   [p4] gitcode.csdn.net blog, "Engram 到底怎么工作的": 第一步 .. 第四步,
+ *        end-to-end training with consistent slot gradients, offload to DRAM
+ *   [p5] discuss.deepseek.club, 二.1 (1) hash retrieval, 二.1 (2) gate and conv,
+ *        二.2 multi-branch integration and host prefetch
+ *
+ * Conventions for every call:
+ *   - All device pointers are raw CUDA device addresses, 16-byte aligned.
+ *     Host pointers are named so.  The caller owns every buffer; the library
+ *     allocates no device memory and keeps no state besides one device status
+ *     word per device.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous and never synchronise, except
+ *     engram_build_vocab_proj (returns V_c on the host) and engram_get_status.
+ *   - Return value: ENGRAM_OK (0) or a negative ENGRAM_ERR_* code.  Host-side
+ *     argument errors launch nothing.  Data errors found on the device (a raw
+ *     id outside [0, V_raw), a row index outside its table) never trap: the
+ *     kernel writes idx = -1 / a zero row and sets a bit of the status word,
+ *     read and cleared by engram_get_status.
+ *   - Layouts are row-major, the last index fastest.  Token order is flat:
+ *     token n = b*T + t.
+ */
+#ifndef ENGRAM_B200_H
+#define ENGRAM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ENGRAM_MAX_HEADS 32 /* J = 2K <= 32 */
+#define ENGRAM_CONV_K 4     /* causal conv width */
+
+enum { ENGRAM_F32 = 0, ENGRAM_BF16 = 1 };
+
+enum {
+  ENGRAM_OK = 0,
+  ENGRAM_ERR_INVALID_ARG = -1, /* null pointer, bad size or bad config */
+  ENGRAM_ERR_MISALIGNED = -2,  /* a pointer is not 16-byte aligned */
+  ENGRAM_ERR_WORKSPACE = -3,   /* ws_bytes below engram_workspace_size */
+  ENGRAM_ERR_UNSUPPORTED = -4, /* shape/dtype combination not built */
+  ENGRAM_ERR_CUDA = -5,        /* a CUDA runtime call failed */
+  ENGRAM_ERR_TIMEOUT = -6      /* status word reports a pipeline wait that ran out */
+};
+
+/* bits of the device status word */
+#define ENGRAM_STATUS_BAD_ID 1u    /* raw token id outside [0, V_raw) */
+#define ENGRAM_STATUS_BAD_INDEX 2u /* gathered row index outside [0, P_j) */
+#define ENGRAM_STATUS_TIMEOUT 4u   /* a bounded wait inside a kernel gave up */
+
+/*
+ * Layer configuration (host memory, read during the call only).
+ *   K        hash heads per n-gram order; J = 2K heads: heads 0..K-1 hash the
+ *            2-gram, heads K..2K-1 the 3-gram ([p5 二.1 (1)] 多头哈希).
+ *   D_h      dims of one table row; E = J * D_h is the width of e_t.
+ *   d_model  width d of h and out.
+ *   n_branch M hidden-state branches; each has its own W_k and gate, the
+ *            table, W_v and conv weights are shared ([p5 二.2] 多分支架构集成).
+ *   V_raw    raw vocabulary size; V_c compressed size; PAD id = V_c.
+ *   dtype    ENGRAM_F32 or ENGRAM_BF16: storage of table, e, h, W_k, W_v, out.
+ *   rows[j]  P_j, row count (a prime) of head j's table.  Head j's rows sit
+ *            in one packed table after those of heads 0..j-1.
+ *   mult[j]  odd 64-bit multipliers of head j for n-gram positions 0, 1, 2
+ *            (position i holds c_{t-i}).  Slot of head j:
+ *              (XOR_i c_{t-i} * mult[j][i]  mod 2^64)  mod P_j.
+ */
+typedef struct engram_cfg {
+  int32_t K;
+  int32_t D_h;
+  int32_t d_model;
+  int32_t n_branch;
+  int32_t V_raw;
+  int32_t V_c;
+  int32_t dtype;
+  int32_t reserved;
+  int64_t rows[ENGRAM_MAX_HEADS];
+  uint64_t mult[ENGRAM_MAX_HEADS][3];
+} engram_cfg_t;
+
+/* which call engram_workspace_size sizes */
+enum {
+  ENGRAM_WS_VOCAB = 0,     /* engram_build_vocab_proj, n = V */
+  ENGRAM_WS_FORWARD = 1,   /* engram_forward, n = tokens */
+  ENGRAM_WS_BACKWARD = 2,  /* engram_backward, n = tokens */
+  ENGRAM_WS_TABLE_GRAD = 3 /* engram_table_grad, n = tokens */
+};
+
+/* Bytes of device workspace the call needs for n items (0 = none).  Returns
+ * 0 as well for an invalid configuration (the call itself then reports it). */
+size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n);
+
+/* Bytes of the `saved` buffer engram_forward fills for engram_backward. */
+size_t engram_saved_size(const engram_cfg_t* cfg, int64_t n_tok);
+
+/*
+ * Vocabulary projection ([p5 二.1 (1)] 词汇投影; [p1] 分词器压缩: ids of one
+ * meaning but different surface form share one compressed id, ~23% fewer ids).
+ *   keys  device int64 [V]: canonical key of each raw id (ids with equal keys
+ *         merge).
+ *   proj  device int32 [V], out: compressed id of each raw id.  Compressed ids
+ *         number the distinct keys in order of first occurrence by raw id.
+ *   V_c_out host int32, out: number of distinct keys.
+ *   ws    device workspace of engram_workspace_size(NULL-ok, ENGRAM_WS_VOCAB, V).
+ * One-time set-up: synchronises `stream` to return V_c.
+ */
+int engram_build_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_c_out,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Steps 1-3: compress, suffix n-grams, multi-head hash ([p4 第一步, 第二步];
+ * [p2] 2-gram / 3-gram suffixes; [p5 二.1 (1)]).
+ *   proj  device int32 [V_raw].      ids  device int32 [B, T] raw ids.
+ *   idx   device int32 [B, T, J], out: slot of each head (-1 for a token whose
+ *         n-gram holds an invalid raw id; the status word then has BAD_ID).
+ *   ngram_state  NULL for whole sequences (positions before t = 0 are PAD).
+ *         Non-NULL selects decode: T must be 1; device int32 [B, 2] holds
+ *         (c_{t-1}, c_{t-2}) of each sequence, PAD at the start, and is
+ *         updated in place.
+ * The indices depend on the ids alone, so they can be computed ahead of the
+ * layer ([p2]: known before the forward pass; [p4] prefetch).
+ */
+int engram_hash_indices(const engram_cfg_t* cfg, const int32_t* proj, const int32_t* ids,
+                        int32_t B, int32_t T, int32_t* ngram_state, int32_t* idx, void* stream);
+
+/*
+ * Step 4: e[n, j*D_h:(j+1)*D_h] = table[rowbase_j + idx[n, j]] ([p5 二.1 (1)]
+ * 拼接检索结果).  table: device, packed heads, dtype cfg->dtype.
+ * e: device [n_tok, E], out.  An exact copy.
+ */
+int engram_gather(const engram_cfg_t* cfg, const int32_t* idx, const void* table, int64_t n_tok,
+                  void* e, void* stream);
+
+/*
+ * Steps 4-6: the whole layer for B sequences of T tokens.
+ *   idx     device int32 [B, T, J] from engram_hash_indices.
+ *   table   device packed table, or NULL when `e` already holds the gathered
+ *           rows (host-resident tables: see engram_forward_hosttable).
+ *   e       device [B*T, E] (cfg->dtype): written by the gather when table is
+ *           non-NULL, read by the projections.
+ *   h       device [B, T, M, d] hidden state (cfg->dtype).
+ *   Wk      device [M, d, E] key projections, Wv device [d, E] value
+ *           projection (cfg->dtype; k = W_k e, v = W_v e: the contraction runs
+ *           along the contiguous axis).
+ *   conv_w  device fp32 [d, 4]: y_t = sum_i conv_w[:, i] * vt_{t-3+i}.
+ *   conv_state NULL for whole sequences.  Non-NULL selects decode (T == 1):
+ *           device fp32 [B, M, 3, d], vt of the three previous steps, oldest
+ *           first, zeros at the start; updated in place.
+ *   out     device [B, T, M, d] (cfg->dtype).
+ *   saved   device, engram_saved_size bytes, or NULL: what engram_backward needs.
+ *   ws      device workspace of engram_workspace_size(cfg, ENGRAM_WS_FORWARD, B*T).
+ * bf16: tables, e, h, W, out in bf16; products, gate, conv in fp32; the output
+ * is rounded once.  f32: everything fp32.
+ * ([p5 二.1 (2)] gate with h as query and e as key/value, 1-D conv, residual;
+ * [p4 第三步, 第四步]; [p2] short depthwise causal conv.)
+ */
+int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* table, void* e,
+                   const void* h, const void* Wk, const void* Wv, const float* conv_w,
+                   float* conv_state, void* out, float* saved, int32_t B, int32_t T, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/*
+ * Backward of engram_forward for L = sum(dout * out) ([p4]: end-to-end
+ * training; lookups are deterministic, so a slot gets consistent gradients).
+ * Inputs as in engram_forward (e as the forward left it, saved from it) and
+ *   dout     device fp32 [B, T, M, d].
+ * Outputs (device fp32, overwritten):
+ *   dh [B, T, M, d], dWk [M, d, E], dWv [d, E], dconv_w [d, 4],
+ *   de       [B*T, E] or NULL,
+ *   dtab_keys int64 [<= B*T*J]: packed-table row ids, ascending, unique,
+ *   dtab_rows [<= B*T*J, D_h]: gradient of those rows,
+ *   n_unique device int32 [1]: number of rows written.
+ * Each table row's gradient is summed in fp32 over its tokens in ascending
+ * token order (see engram_table_grad), so it is reproducible bit for bit.
+ * Built for ENGRAM_F32 configurations.
+ */
+int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,
+                    const void* Wk, const void* Wv, const float* conv_w, const float* saved,
+                    const float* dout, float* dh, float* dWk, float* dWv, float* dconv_w, float* de,
+                    int64_t* dtab_keys, float* dtab_rows, int32_t* n_unique, int32_t B, int32_t T,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Sparse table gradient alone: a stable sort of the (row id, token) pairs by
+ * row id, then one fp32 sum per row and dimension over its tokens in
+ * ascending order, each starting from +0.
+ *   idx device int32 [n_tok, J]; de device fp32 [n_tok, E].
+ *   Outputs as in engram_backward.
+ */
+int engram_table_grad(const engram_cfg_t* cfg, const int32_t* idx, const float* de, int64_t n_tok,
+                      int64_t* dtab_keys, float* dtab_rows, int32_t* n_unique, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/*
+ * Gather from a table in pinned, mapped host memory over PCIe ([p5 二.2]
+ * the host fetches memory rows while the GPU runs earlier layers; [p4]
+ * a 100B-parameter table kept in DRAM; [p2] prefetch over PCIe).
+ *   host_table  pinned host memory (cudaHostAlloc / cudaHostRegister with
+ *               mapping), packed as the device table.
+ *   e           device [n_tok, E], out.
+ *   side_stream the stream to run on; done_event (cudaEvent_t as void*, may
+ *               be NULL) is recorded after the gather so the compute stream can
+ *               wait on it before engram_forward(table = NULL, e).
+ */
+int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const void* host_table,
+                             int64_t n_tok, void* e, void* side_stream, void* done_event);
+
+/* Synchronises `stream`, then returns the device status word of the current
+ * device (bits ENGRAM_STATUS_*) and clears it; a negative value is an
+ * ENGRAM_ERR_* code. */
+int engram_get_status(void* stream);
+
+/* Multiprocessor count of the current device, or a negative ENGRAM_ERR_*. */
+int engram_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENGRAM_B200_H */

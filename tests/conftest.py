@@ -8,3 +8,5 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
+    from hashed_gram_conditional_engram_b200 import build
+    build.build()

@@ -1,0 +1,69 @@
+"""The C ABI library loads, exports every entry point include/engram.h
+declares, and its host-side checks answer without touching a GPU."""
+import os
+import re
+
+import numpy as np
+
+from hashed_gram_conditional_engram_b200 import engram as eg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "engram.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(engram_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = eg.lib()
+    names = declared_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(eg.EXPORTED)
+
+
+def _cfg(**kw):
+    a = dict(K=2, D_h=16, d_model=64, n_branch=1, V_raw=1000, V_c=770, dtype=eg.F32,
+             rows=[1009] * 4, mult=np.ones((4, 3), np.uint64))
+    a.update(kw)
+    return eg.make_cfg(**a)
+
+
+def test_workspace_sizes_host_only():
+    c = _cfg()
+    assert eg.engram_workspace_size(c, eg.WS_FORWARD, 64) > 0
+    assert eg.engram_workspace_size(c, eg.WS_BACKWARD, 64) > eg.engram_workspace_size(
+        c, eg.WS_TABLE_GRAD, 64)
+    assert eg.engram_workspace_size(None, eg.WS_VOCAB, 129280) > 129280 * 8
+    assert eg.engram_saved_size(c, 64) >= 64 * (1 + 3 * 64) * 4
+    b = _cfg(K=8, D_h=80, d_model=2560, dtype=eg.BF16, rows=[4449997] * 16,
+             mult=np.ones((16, 3), np.uint64))
+    # bf16: gate partials, 2 per 256-column tile per token
+    assert eg.engram_workspace_size(b, eg.WS_FORWARD, 32768) == 32768 * 20 * 16
+    assert eg.engram_saved_size(b, 32768) == 32768 * 4
+
+
+def test_invalid_configurations_rejected_before_any_launch():
+    bad = [
+        _cfg(K=0),
+        _cfg(D_h=6),                     # 24-byte rows: not a multiple of 16 bytes
+        _cfg(rows=[1009, 1009, 1008, 1009]),  # even row count
+        _cfg(rows=[1009, 1009, 1, 1009]),
+        _cfg(V_c=1001), _cfg(dtype=7), _cfg(K=3, rows=[1009] * 6,
+                                            mult=np.ones((6, 3), np.uint64)),  # J % 4 != 0
+    ]
+    big = _cfg()
+    big.K = 17                             # J = 34 > 32 heads
+    bad.append(big)
+    for c in bad:
+        assert eg.engram_workspace_size(c, eg.WS_FORWARD, 64) == 0
+        rc = eg.lib().engram_hash_indices(c, None, None, 1, 1, None, None, None)
+        assert rc in (-1, -2), rc
+
+
+def test_error_names():
+    e = eg.EngramError("engram_forward", -4)
+    assert "UNSUPPORTED" in str(e)
