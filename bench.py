@@ -326,11 +326,11 @@ def run_ours(args):
             "gather_gbs": (N * w.J * 4 + N * w.J * w.D_h * 2 + N * w.E * 2) / (t_gather / 1e3) / 1e9,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "tc_fused_kernel (pass K + pass V)",
+                         "kernel": "engram_forward(table=NULL): tc_fused_kernel pass K, gate kernel, tc_fused_kernel pass V",
                          "peak_source": f"{peak_src} bf16_tflops (burst)"},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": 5 * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }

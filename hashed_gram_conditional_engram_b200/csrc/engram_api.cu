@@ -82,7 +82,7 @@ size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n) {
   const int M = cfg->n_branch, d = cfg->d_model, E = 2 * cfg->K * cfg->D_h;
   switch (call) {
     case ENGRAM_WS_FORWARD:
-      if (cfg->dtype == ENGRAM_F32) return f32_saved_bytes(n, M, d);
+      if (cfg->dtype == ENGRAM_F32) return f32_forward_ws_bytes(n, M, d);
       return tc_forward_ws_bytes(n, d, E);
     case ENGRAM_WS_BACKWARD:
       return backward_f32_ws_bytes(n, M, d, E) + table_grad_ws_bytes(n * 2 * cfg->K);
@@ -162,13 +162,10 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
     rc = launch_gather(hp, idx, table, N, elem_bytes(cfg), e, s);
     if (rc) return rc;
   }
-  if (cfg->dtype == ENGRAM_F32) {
-    void* sv_base = saved != nullptr ? static_cast<void*>(saved) : ws;
-    F32Saved sv = f32_saved_layout(sv_base, N, M, d);
+  if (cfg->dtype == ENGRAM_F32)
     return launch_forward_f32(static_cast<const float*>(e), static_cast<const float*>(h),
                               static_cast<const float*>(Wk), static_cast<const float*>(Wv), conv_w,
-                              conv_state, static_cast<float*>(out), sv, N, T, M, d, E, s);
-  }
+                              conv_state, static_cast<float*>(out), saved, N, T, M, d, E, ws, s);
   return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
                            static_cast<const __nv_bfloat16*>(Wk),
                            static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
@@ -186,7 +183,7 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
   if (B < 0 || T < 0) return ENGRAM_ERR_INVALID_ARG;
   const int64_t N = (int64_t)B * T;
   if (idx == nullptr || e == nullptr || h == nullptr || Wk == nullptr || Wv == nullptr ||
-      conv_w == nullptr || saved == nullptr || dout == nullptr || dh == nullptr || dWk == nullptr ||
+      conv_w == nullptr || dout == nullptr || dh == nullptr || dWk == nullptr ||
       dWv == nullptr || dconv_w == nullptr || dtab_keys == nullptr || dtab_rows == nullptr ||
       n_unique == nullptr || ws == nullptr)
     return ENGRAM_ERR_INVALID_ARG;
@@ -201,13 +198,9 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
   const HeadParams hp = make_head_params(cfg);
   const int M = cfg->n_branch, d = cfg->d_model, E = hp.E;
   const size_t bw = backward_f32_ws_bytes(N, M, d, E);
-  // de lives at the end of the dense-backward workspace unless the caller wants it
-  float* de_buf = de;
-  if (de_buf == nullptr) {
-    const size_t de_bytes = ((size_t)N * E * 4 + 255) & ~(size_t)255;
-    de_buf = reinterpret_cast<float*>(static_cast<char*>(ws) + bw - de_bytes);
-  }
-  F32Saved sv = f32_saved_layout(const_cast<float*>(saved), N, M, d);
+  // de lives in the dense-backward workspace unless the caller wants it
+  float* de_buf = de != nullptr ? de : backward_f32_de_slot(ws, N, M, d, E);
+  F32Saved sv = f32_saved_layout(saved != nullptr ? const_cast<float*>(saved) : ws, N, M, d);
   rc = launch_backward_f32(static_cast<const float*>(e), static_cast<const float*>(h),
                            static_cast<const float*>(Wk), static_cast<const float*>(Wv), conv_w,
                            sv, dout, dh, dWk, dWv, dconv_w, de_buf, N, T, M, d, E, ws, s);

@@ -61,7 +61,8 @@ struct TcArgs {
   float4* part;
   const float4* conv_w;
   float* conv_state;
-  float* alpha_out;
+  float* alpha_out;     // pass V: optional copy of alpha for the caller
+  const float* alpha;   // pass V: gate of every token, from the gate kernel
   unsigned int* status;
 };
 
@@ -215,6 +216,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
   for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -248,11 +257,16 @@ struct TcShape {
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int HALF_COLS = BN / 2;
   static constexpr int NCHUNK = HALF_COLS / 32;
-  static constexpr int XBUF_FLOATS = 2 * 2 * NCHUNK * 4 * 3 * 32;  // [parity][half][chunk][quad][3][32]
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 +
-                                 (size_t)XBUF_FLOATS * 4;
+  // pass V stages the scaled values of 16 columns of all 128 rows per half:
+  // rows of 20 floats (16 + 4 pad) keep 16-byte vectors conflict-free
+  static constexpr int SB_STRIDE = 20;
+  static constexpr int TAP_BYTES = 2 * HALF_COLS * 16;
+  static constexpr int SB_BYTES = 2 * BM * SB_STRIDE * 4;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 + TAP_BYTES +
+                                 SB_BYTES;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "N tile");
   static_assert(2 * STAGES + 5 <= 30, "barrier area");
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
 template <int BN, int STAGES, int MODE>
@@ -279,7 +293,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 30);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 31);
-  float* xbuf = reinterpret_cast<float*>(bars + 32);
+  float4* tapbuf = reinterpret_cast<float4*>(bars + 32);
+  float* stagebuf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(tapbuf) + S::TAP_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_tiles = args.num_m_tiles * args.num_n_tiles;
@@ -390,8 +405,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int rloc = quad * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    int iter = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mt = tile / args.num_n_tiles, nt = tile - mt * args.num_n_tiles;
       int got = 0;
       if (lane == 0) got = wait_bounded(&tfull[acc], acc_phase, abort_flag, args.status) ? 1 : 0;
@@ -403,10 +417,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                              (uint32_t)(half * S::HALF_COLS);
       const int col_base = nt * BN + half * S::HALF_COLS;
 
+      // the next tile of this CTA: pull its rows of h (and, in pass V, of the
+      // gate partials) into L2 while this tile's epilogue runs
+      {
+        const int nxt = tile + (int)gridDim.x;
+        if (nxt < num_tiles) {
+          const int mt2 = nxt / args.num_n_tiles, nt2 = nxt - mt2 * args.num_n_tiles;
+          const int64_t n2 = (int64_t)mt2 * args.m_stride + args.m_offset + rloc;
+          if (n2 >= 0 && n2 < args.N) {
+            const __nv_bfloat16* hp2 = args.h + n2 * args.d + nt2 * BN + half * S::HALF_COLS;
+            for (int b = 0; b < S::HALF_COLS * 2; b += 128) prefetch_l2(hp2 + b / 2);
+            if (MODE == MODE_VALUE_CONV && (rloc & 31) == 0) prefetch_l2(args.alpha + n2);
+          }
+        }
+      }
       if (MODE == MODE_GATE_PARTIAL) {
         float kk = 0.f, hk = 0.f, hh = 0.f;
 #pragma unroll 1
         for (int c = 0; c < S::NCHUNK; ++c) {
+          if (valid && c + 1 < S::NCHUNK)
+            prefetch_l1(args.h + n * args.d + col_base + (c + 1) * 32);
           float v[32];
           __syncwarp();
           if (got) {
@@ -428,28 +458,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (valid) args.part[n * args.n_part + nt * 2 + half] = make_float4(kk, hk, hh, 0.f);
       } else {
-        // gate of this row from the partials of every column tile
-        float alpha = 0.f;
-        if (valid) {
-          const float4* pr = args.part + n * args.n_part;
-          float kk = 0.f, hk = 0.f, hh = 0.f;
-          for (int i = 0; i < args.n_part; ++i) {
-            const float4 q = pr[i];
-            kk += q.x;
-            hk += q.y;
-            hh += q.z;
-          }
-          const float invd = 1.0f / (float)args.d;
-          const float rh = rsqrtf(hh * invd + RMS_EPS), rk = rsqrtf(kk * invd + RMS_EPS);
-          const float z = hk * rh * rk * rsqrtf((float)args.d);
-          alpha = 1.0f / (1.0f + expf(-z));
-        }
+        const float alpha = valid ? __ldg(args.alpha + n) : 0.f;
         const bool decode = args.conv_state != nullptr;
         const bool is_out = valid && rloc >= -args.m_offset;
-        if (is_out && args.alpha_out != nullptr && nt == 0 && half == 0) args.alpha_out[n] = alpha;
         const int pos = valid ? (int)(n % args.T) : 0;
+        // causal masks: vt of rows t-1, t-2, t-3 count only inside the sequence
+        const float m1 = pos >= 1 ? 1.f : 0.f, m2 = pos >= 2 ? 1.f : 0.f,
+                    m3 = pos >= 3 ? 1.f : 0.f;
+        float4* taps = tapbuf + half * S::HALF_COLS;
+        float* sb = stagebuf + half * (BM * S::SB_STRIDE);
+        // conv taps of this half's columns, shared by its four warps
+        for (int c = rloc; c < S::HALF_COLS; c += 128) taps[c] = __ldg(args.conv_w + col_base + c);
+        // h of this row, loaded one 16-column sub-chunk ahead of its use
+        const uint4* hrow = reinterpret_cast<const uint4*>(args.h + n * args.d + col_base);
+        uint4 hcur[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) hcur[q] = is_out ? __ldg(hrow + q) : make_uint4(0, 0, 0, 0);
+        named_bar_sync(1 + half, 128);
 #pragma unroll 1
         for (int c = 0; c < S::NCHUNK; ++c) {
+          if (is_out && c + 1 < S::NCHUNK) prefetch_l1(hrow + 4 * (c + 1));
           float v[32];
           __syncwarp();
           if (got) {
@@ -461,80 +489,95 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] *= alpha;  // vt
           const int col = col_base + c * 32;
-          const float* xp = nullptr;
-          if (!decode) {
-            // lanes 29..31 publish vt for lanes 0..2 of the next quadrant
-            float* xw =
-                xbuf + (((((iter & 1) * 2 + half) * S::NCHUNK + c) * 4 + quad) * 3) * 32;
-            if (lane >= 29) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) xw[(lane - 29) * 32 + i] = v[i];
+          for (int sub = 0; sub < 2; ++sub) {
+            const int c0 = sub * 16;
+            const int sc = 2 * c + sub;
+            uint4 hnx[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+              hnx[q] = (is_out && sc + 1 < 2 * S::NCHUNK) ? __ldg(hrow + 2 * (sc + 1) + q)
+                                                          : make_uint4(0, 0, 0, 0);
+            float hv[16];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const uint4 wv = hcur[q];
+              const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                hv[q * 8 + 2 * i] = __uint_as_float(ws[i] << 16);
+                hv[q * 8 + 2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+              }
             }
-            named_bar_sync(1 + half, 128);
-            xp = xbuf +
-                 (((((iter & 1) * 2 + half) * S::NCHUNK + c) * 4 + ((quad + 3) & 3)) * 3) * 32;
-          }
-          float hv[32];
-          if (is_out) {
-            load_bf16x32(args.h + n * args.d + col, hv);
-          } else {
+            float* st = (decode && is_out) ? args.conv_state + n * 3 * args.d + col + c0 : nullptr;
+            const float4* r1 = nullptr;
+            const float4* r2 = nullptr;
+            const float4* r3 = nullptr;
+            if (!decode) {
+              // publish this row's 16 values, then read the three rows above
+              float4* mine = reinterpret_cast<float4*>(sb + rloc * S::SB_STRIDE);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) hv[i] = 0.f;
-          }
-          float* st = (decode && is_out) ? args.conv_state + n * 3 * args.d + col : nullptr;
-          uint32_t packed[16];
+              for (int q = 0; q < 4; ++q)
+                mine[q] = make_float4(v[c0 + 4 * q], v[c0 + 4 * q + 1], v[c0 + 4 * q + 2],
+                                      v[c0 + 4 * q + 3]);
+              named_bar_sync(1 + half, 128);
+              const int rr = rloc >= 3 ? rloc : 3;  // halo rows read a valid row, masked below
+              r1 = reinterpret_cast<const float4*>(sb + (rr - 1) * S::SB_STRIDE);
+              r2 = reinterpret_cast<const float4*>(sb + (rr - 2) * S::SB_STRIDE);
+              r3 = reinterpret_cast<const float4*>(sb + (rr - 3) * S::SB_STRIDE);
+            }
+            uint32_t packed[8];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float o[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int k = i + u;
-              float a1 = 0.f, a2 = 0.f, a3 = 0.f;  // vt of rows t-1, t-2, t-3
+            for (int q = 0; q < 4; ++q) {
+              float a1[4], a2[4], a3[4];  // vt of rows t-1, t-2, t-3, four columns
               if (decode) {
                 if (st != nullptr) {
-                  a3 = st[k];
-                  a2 = st[args.d + k];
-                  a1 = st[2 * args.d + k];
-                  st[k] = a2;
-                  st[args.d + k] = a1;
-                  st[2 * args.d + k] = v[k];
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    const int k = 4 * q + u;
+                    a3[u] = st[k];
+                    a2[u] = st[args.d + k];
+                    a1[u] = st[2 * args.d + k];
+                    st[k] = a2[u];
+                    st[args.d + k] = a1[u];
+                    st[2 * args.d + k] = v[c0 + k];
+                  }
+                } else {
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) a1[u] = a2[u] = a3[u] = 0.f;
                 }
               } else {
-                float b1 = __shfl_up_sync(FULL, v[k], 1);
-                float b2 = __shfl_up_sync(FULL, v[k], 2);
-                float b3 = __shfl_up_sync(FULL, v[k], 3);
-                if (lane == 0) {
-                  b1 = xp[2 * 32 + k];
-                  b2 = xp[1 * 32 + k];
-                  b3 = xp[0 * 32 + k];
-                } else if (lane == 1) {
-                  b2 = xp[2 * 32 + k];
-                  b3 = xp[1 * 32 + k];
-                } else if (lane == 2) {
-                  b3 = xp[2 * 32 + k];
-                }
-                a1 = pos >= 1 ? b1 : 0.f;
-                a2 = pos >= 2 ? b2 : 0.f;
-                a3 = pos >= 3 ? b3 : 0.f;
+                const float4 x1 = r1[q], x2 = r2[q], x3 = r3[q];
+                a1[0] = x1.x * m1; a1[1] = x1.y * m1; a1[2] = x1.z * m1; a1[3] = x1.w * m1;
+                a2[0] = x2.x * m2; a2[1] = x2.y * m2; a2[2] = x2.z * m2; a2[3] = x2.w * m2;
+                a3[0] = x3.x * m3; a3[1] = x3.y * m3; a3[2] = x3.z * m3; a3[3] = x3.w * m3;
               }
-              const float4 w = __ldg(args.conv_w + col + k);
-              float y = w.w * v[k];
-              y = fmaf(w.z, a1, y);
-              y = fmaf(w.y, a2, y);
-              y = fmaf(w.x, a3, y);
-              const float sy = y / (1.0f + expf(-y));
-              o[u] = hv[k] + v[k] + sy;
-            }
-            packed[i / 2] = pack_bf16x2(o[0], o[1]);
-          }
-          if (is_out) {
-            uint4* dst = reinterpret_cast<uint4*>(args.out + n * args.d + col);
+              float o[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
-                                  packed[4 * q + 3]);
+              for (int u = 0; u < 4; ++u) {
+                const int k = 4 * q + u;
+                const float4 w = taps[c * 32 + c0 + k];
+                float y = w.w * v[c0 + k];
+                y = fmaf(w.z, a1[u], y);
+                y = fmaf(w.y, a2[u], y);
+                y = fmaf(w.x, a3[u], y);
+                const float sy = __fdividef(y, 1.0f + __expf(-y));  // SiLU
+                o[u] = hv[k] + v[c0 + k] + sy;
+              }
+              packed[2 * q] = pack_bf16x2(o[0], o[1]);
+              packed[2 * q + 1] = pack_bf16x2(o[2], o[3]);
+            }
+            if (is_out) {
+              uint4* dst = reinterpret_cast<uint4*>(args.out + n * args.d + col + c0);
+              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            }
+            if (!decode) named_bar_sync(1 + half, 128);  // reads done before the next write
+#pragma unroll
+            for (int q = 0; q < 2; ++q) hcur[q] = hnx[q];
           }
         }
+        if (decode) named_bar_sync(1 + half, 128);  // taps read before the next tile loads them
       }
       tc_fence_before();
       __syncwarp();
@@ -550,6 +593,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
+}
+
+// alpha of every token from the gate partials of pass K (fixed order):
+// alpha = sigmoid(<h, k> r_h r_k / sqrt(d)), r_x = (mean(x^2) + eps)^(-1/2).
+__global__ void __launch_bounds__(256) gate_from_partials_kernel(const float4* __restrict__ part,
+                                                                 int n_part, int64_t N, int d,
+                                                                 float* __restrict__ alpha,
+                                                                 float* __restrict__ alpha_copy) {
+  const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  const float4* pr = part + n * n_part;
+  float kk = 0.f, hk = 0.f, hh = 0.f;
+  for (int i = 0; i < n_part; ++i) {
+    const float4 q = __ldg(pr + i);
+    kk += q.x;
+    hk += q.y;
+    hh += q.z;
+  }
+  const float invd = 1.0f / (float)d;
+  const float rh = rsqrtf(hh * invd + RMS_EPS), rk = rsqrtf(kk * invd + RMS_EPS);
+  const float a = 1.0f / (1.0f + expf(-(hk * rh * rk * rsqrtf((float)d))));
+  alpha[n] = a;
+  if (alpha_copy != nullptr) alpha_copy[n] = a;
 }
 
 // ------------------------------------------------------------------ host side
@@ -612,7 +678,7 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, c
 template <int BN, int STAGES>
 int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
-              float* alpha_saved, int64_t N, int T, int d, int E, float4* part,
+              float* alpha_saved, int64_t N, int T, int d, int E, float4* part, float* alpha,
               cudaStream_t s) {
   CUtensorMap ta, tbk, tbv;
   if (!make_tmap(&ta, e, (uint64_t)E, (uint64_t)N, BM)) return ENGRAM_ERR_CUDA;
@@ -631,6 +697,7 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.conv_w = reinterpret_cast<const float4*>(conv_w);
   a.conv_state = conv_state;
   a.alpha_out = alpha_saved;
+  a.alpha = nullptr;
   a.status = status_ptr();
   // pass K: gate partials
   a.m_stride = BM;
@@ -638,6 +705,9 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.num_m_tiles = (int)((N + BM - 1) / BM);
   int rc = launch_pass<BN, STAGES, MODE_GATE_PARTIAL>(ta, tbk, a, s);
   if (rc) return rc;
+  gate_from_partials_kernel<<<(unsigned)((N + 255) / 256), 256, 0, s>>>(part, a.n_part, N, d,
+                                                                        alpha, alpha_saved);
+  a.alpha = alpha;
   // pass V: gate, conv, residual (overlapping tiles with a 3-row halo, or
   // plain tiles plus the conv state in decode)
   if (conv_state != nullptr) {
@@ -662,7 +732,8 @@ int tc_supported(int d, int E, int M) {
 size_t tc_forward_ws_bytes(int64_t N, int d, int E) {
   (void)E;
   const int BN = use_wide(N, d) ? 256 : 64;
-  return (size_t)N * 2 * (d / BN) * sizeof(float4);
+  const size_t part = (size_t)N * 2 * (d / BN) * sizeof(float4);
+  return part + (((size_t)N * sizeof(float) + 255) & ~(size_t)255);
 }
 
 int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
@@ -671,11 +742,16 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
                       void* ws, size_t ws_bytes, cudaStream_t s) {
   if (ws_bytes < tc_forward_ws_bytes(N, d, E) || ws == nullptr) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL - 256) return ENGRAM_ERR_UNSUPPORTED;
+  const bool wide = use_wide(N, d);
+  const int BN = wide ? 256 : 64;
   float4* part = static_cast<float4*>(ws);
-  if (use_wide(N, d))
+  float* alpha = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                          (size_t)N * 2 * (d / BN) * sizeof(float4));
+  if (wide)
     return run_layer<256, 4>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
-                             s);
-  return run_layer<64, 8>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part, s);
+                             alpha, s);
+  return run_layer<64, 8>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
+                          alpha, s);
 }
 
 }  // namespace engram

@@ -1,0 +1,100 @@
+"""Runs one kernel family of the library on seeded synthetic inputs of a given
+shape, a few times, for profiling a kernel alone (e.g. under Nsight Compute)
+without the rest of the layer's inputs on the device.
+
+    python -m hashed_gram_conditional_engram_b200.kernel_cases fused \
+        [--tokens 32768] [--d 2560] [--heads 16] [--dh 80] [--seq 4096] [--reps 3]
+    python -m hashed_gram_conditional_engram_b200.kernel_cases gather [...]
+    python -m hashed_gram_conditional_engram_b200.kernel_cases hash [...]
+
+`fused` runs engram_forward with table = NULL on random gathered rows, i.e.
+the two tensor-core passes; `gather` gathers from a table of --rows rows per
+head; `hash` runs the compress + n-gram + hash kernel.  Defaults are the
+27B-shaped layer's dimensions.  Prints the device time per repetition.
+"""
+from __future__ import annotations
+
+import argparse
+
+import numpy as np
+import torch
+
+from . import engram as eg
+from . import synth
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("kernel", choices=["fused", "gather", "hash"])
+    ap.add_argument("--tokens", type=int, default=32768)
+    ap.add_argument("--seq", type=int, default=4096)
+    ap.add_argument("--d", type=int, default=2560)
+    ap.add_argument("--heads", type=int, default=16)
+    ap.add_argument("--dh", type=int, default=80)
+    ap.add_argument("--rows", type=int, default=4_450_001)
+    ap.add_argument("--reps", type=int, default=3)
+    a = ap.parse_args(argv)
+    from . import build
+    build.build()
+    dev = torch.device("cuda")
+    K = a.heads // 2
+    E = a.heads * a.dh
+    B = a.tokens // a.seq
+    T = a.seq
+    N = B * T
+    rows = synth.primes_at_most(a.rows, a.heads)
+    mult = synth.hash_multipliers(12345, a.heads)
+    cfg = eg.make_cfg(K, a.dh, a.d, 1, 129280, synth.compressed_vocab(129280), eg.BF16, rows, mult)
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    if a.kernel == "fused":
+        e = (torch.randn((N, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        h = torch.randn((N, a.d), generator=g, device=dev).to(torch.bfloat16)
+        Wk = (torch.randn((a.d, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        Wv = (torch.randn((a.d, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        cw = torch.randn((a.d, 4), generator=g, device=dev) * 0.5
+        out = torch.empty_like(h)
+        nb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        saved = torch.empty(N, dtype=torch.float32, device=dev)
+
+        def run():
+            eg.engram_forward(cfg, None, None, e, h, Wk, Wv, cw, None, out, saved, B, T, ws, nb)
+    elif a.kernel == "gather":
+        table = torch.empty(sum(rows) * a.dh, dtype=torch.bfloat16, device=dev)
+        table.normal_(0.0, 0.02, generator=g)
+        rng = np.random.default_rng(3)
+        idx = torch.from_numpy(np.stack([rng.integers(0, P, N) for P in rows], -1)
+                               .astype(np.int32)).to(dev)
+        e = torch.empty((N, E), dtype=torch.bfloat16, device=dev)
+
+        def run():
+            eg.engram_gather(cfg, idx, table, N, e)
+    else:
+        ids_np, keys_np = synth.host_ids_keys(synth.workload("layer27b"))
+        keys = torch.from_numpy(keys_np).to(dev)
+        proj = torch.empty(129280, dtype=torch.int32, device=dev)
+        vb = eg.engram_workspace_size(None, eg.WS_VOCAB, 129280)
+        vws = torch.empty(vb, dtype=torch.uint8, device=dev)
+        eg.engram_build_vocab_proj(keys, 129280, proj, vws, vb)
+        ids = torch.from_numpy(ids_np.reshape(-1)[:N].copy()).to(dev)
+        idx = torch.empty((N, a.heads), dtype=torch.int32, device=dev)
+
+        def run():
+            eg.engram_hash_indices(cfg, proj, ids, B, T, None, idx)
+
+    for r in range(a.reps):
+        ev0.record()
+        run()
+        ev1.record()
+        torch.cuda.synchronize()
+        print(f"{a.kernel} rep {r}: {ev0.elapsed_time(ev1) * 1e3:.1f} us")
+    st = eg.engram_get_status()
+    if st != 0:
+        raise SystemExit(f"device status word {st}")
+
+
+if __name__ == "__main__":
+    main()

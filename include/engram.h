@@ -170,7 +170,8 @@ int engram_gather(const engram_cfg_t* cfg, const int32_t* idx, const void* table
  *   saved   device, engram_saved_size bytes, or NULL: what engram_backward needs.
  *   ws      device workspace of engram_workspace_size(cfg, ENGRAM_WS_FORWARD, B*T).
  * bf16: tables, e, h, W, out in bf16; products, gate, conv in fp32; the output
- * is rounded once.  f32: everything fp32.
+ * is rounded once.  f32: tables, e, h, W, out in fp32; the arithmetic runs in
+ * fp64 and every stored value is rounded to fp32 once.
  * ([p5 二.1 (2)] gate with h as query and e as key/value, 1-D conv, residual;
  * [p4 第三步, 第四步]; [p2] short depthwise causal conv.)
  */
@@ -182,7 +183,10 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
 /*
  * Backward of engram_forward for L = sum(dout * out) ([p4]: end-to-end
  * training; lookups are deterministic, so a slot gets consistent gradients).
- * Inputs as in engram_forward (e as the forward left it, saved from it) and
+ * Inputs as in engram_forward (e as the forward left it; saved may be NULL:
+ * the fp32 backward recomputes the forward's intermediates in fp64 from e, h
+ * and the weights and keeps every product and sum in fp64, so each gradient
+ * carries one fp32 rounding) and
  *   dout     device fp32 [B, T, M, d].
  * Outputs (device fp32, overwritten):
  *   dh [B, T, M, d], dWk [M, d, E], dWv [d, E], dconv_w [d, 4],
