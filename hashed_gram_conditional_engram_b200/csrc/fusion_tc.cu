@@ -41,7 +41,8 @@ constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle row
 constexpr int UMMA_K = 16;
 constexpr int NUM_EPI_WARPS = 8;
-constexpr int NUM_THREADS = 64 + NUM_EPI_WARPS * 32;
+constexpr int HP_WARP = 2 + NUM_EPI_WARPS;  // pass V: warp that streams h tiles in by TMA
+constexpr int NUM_THREADS = 64 + NUM_EPI_WARPS * 32 + 32;
 constexpr int HALO = 3;  // conv width 4 - 1
 constexpr float RMS_EPS = 1e-6f;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
@@ -250,30 +251,34 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // ------------------------------------------------------------------ kernel
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int MODE>
 struct TcShape {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int HALF_COLS = BN / 2;
   static constexpr int NCHUNK = HALF_COLS / 32;
+  // pass V: ring of h chunks (128 rows x 32 columns for each half, 64-byte
+  // swizzle), filled by TMA ahead of the epilogue
+  static constexpr int HSLOTS = MODE == MODE_VALUE_CONV ? 3 : 0;
+  static constexpr int HSLOT_BYTES = 2 * BM * 32 * 2;
   // pass V stages the scaled values of 16 columns of all 128 rows per half:
   // rows of 20 floats (16 + 4 pad) keep 16-byte vectors conflict-free
   static constexpr int SB_STRIDE = 20;
   static constexpr int TAP_BYTES = 2 * HALF_COLS * 16;
   static constexpr int SB_BYTES = 2 * BM * SB_STRIDE * 4;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256 + TAP_BYTES +
-                                 SB_BYTES;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) +
+                                 (size_t)HSLOTS * HSLOT_BYTES + 256 + TAP_BYTES + SB_BYTES;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "N tile");
-  static_assert(2 * STAGES + 5 <= 30, "barrier area");
+  static_assert(2 * STAGES + 11 <= 30, "barrier area");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
 template <int BN, int STAGES, int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ TcArgs args) {
-  using S = TcShape<BN, STAGES>;
+                    const __grid_constant__ CUtensorMap tmH, const __grid_constant__ TcArgs args) {
+  using S = TcShape<BN, STAGES, MODE>;
   constexpr uint32_t STAGE_TX = S::A_BYTES + S::B_BYTES;
   // instruction descriptor: fp32 accumulate, bf16 A and B, both K-major,
   // N >> 3 at bit 17, M >> 4 at bit 24
@@ -285,12 +290,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * S::B_BYTES);
+  uint8_t* hring = sB + STAGES * S::B_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(hring + S::HSLOTS * S::HSLOT_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
+  uint64_t* hfull = drain + 1;
+  uint64_t* hempty = hfull + 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 30);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 31);
   float4* tapbuf = reinterpret_cast<float4*>(bars + 32);
@@ -309,11 +317,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&tempty[a], NUM_EPI_WARPS);
     }
     mbar_init(drain, 1);
+    for (int b = 0; b < S::HSLOTS; ++b) {
+      mbar_init(&hfull[b], 1);
+      mbar_init(&hempty[b], NUM_EPI_WARPS);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (MODE == MODE_VALUE_CONV) prefetch_tmap(&tmH);
   }
   if (warp == 1) {
     __syncwarp();
@@ -397,6 +410,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       umma_commit(drain);
       wait_drain(drain, 0);
     }
+  } else if (warp == HP_WARP) {
+    // ------------------------------------------------------------ h producer
+    if (MODE == MODE_VALUE_CONV && lane == 0) {
+      int slot = 0;
+      uint32_t ph = 0;
+      uint32_t issued = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int mt = tile / args.num_n_tiles, nt = tile - mt * args.num_n_tiles;
+        const int row0 = mt * args.m_stride + args.m_offset;
+        bool ok = true;
+        for (int c = 0; c < S::NCHUNK; ++c) {
+          if (!wait_bounded(&hempty[slot], ph ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&hfull[slot], S::HSLOT_BYTES);
+          uint8_t* dst = hring + slot * S::HSLOT_BYTES;
+          tma_load_2d(dst, &tmH, &hfull[slot], nt * BN + c * 32, row0);
+          tma_load_2d(dst + S::HSLOT_BYTES / 2, &tmH, &hfull[slot], nt * BN + S::HALF_COLS + c * 32,
+                      row0);
+          ++issued;
+          if (++slot == S::HSLOTS) {
+            slot = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      for (int b = 0; b < S::HSLOTS; ++b) {
+        const uint32_t n_b = issued > (uint32_t)b ? (issued - 1 - b) / S::HSLOTS + 1 : 0;
+        if (n_b > 0) wait_drain(&hfull[b], (n_b - 1) & 1u);
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
@@ -405,7 +451,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int rloc = quad * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    uint32_t hcnt = 0;  // h chunks consumed so far (pass V)
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mt = tile / args.num_n_tiles, nt = tile - mt * args.num_n_tiles;
       int got = 0;
       if (lane == 0) got = wait_bounded(&tfull[acc], acc_phase, abort_flag, args.status) ? 1 : 0;
@@ -425,8 +472,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int mt2 = nxt / args.num_n_tiles, nt2 = nxt - mt2 * args.num_n_tiles;
           const int64_t n2 = (int64_t)mt2 * args.m_stride + args.m_offset + rloc;
           if (n2 >= 0 && n2 < args.N) {
-            const __nv_bfloat16* hp2 = args.h + n2 * args.d + nt2 * BN + half * S::HALF_COLS;
-            for (int b = 0; b < S::HALF_COLS * 2; b += 128) prefetch_l2(hp2 + b / 2);
+            if (MODE == MODE_GATE_PARTIAL) {
+              const __nv_bfloat16* hp2 = args.h + n2 * args.d + nt2 * BN + half * S::HALF_COLS;
+              for (int b = 0; b < S::HALF_COLS * 2; b += 128) prefetch_l2(hp2 + b / 2);
+            }
             if (MODE == MODE_VALUE_CONV && (rloc & 31) == 0) prefetch_l2(args.alpha + n2);
           }
         }
@@ -435,8 +484,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float kk = 0.f, hk = 0.f, hh = 0.f;
 #pragma unroll 1
         for (int c = 0; c < S::NCHUNK; ++c) {
-          if (valid && c + 1 < S::NCHUNK)
-            prefetch_l1(args.h + n * args.d + col_base + (c + 1) * 32);
           float v[32];
           __syncwarp();
           if (got) {
@@ -469,15 +516,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float* sb = stagebuf + half * (BM * S::SB_STRIDE);
         // conv taps of this half's columns, shared by its four warps
         for (int c = rloc; c < S::HALF_COLS; c += 128) taps[c] = __ldg(args.conv_w + col_base + c);
-        // h of this row, loaded one 16-column sub-chunk ahead of its use
-        const uint4* hrow = reinterpret_cast<const uint4*>(args.h + n * args.d + col_base);
-        uint4 hcur[2];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) hcur[q] = is_out ? __ldg(hrow + q) : make_uint4(0, 0, 0, 0);
         named_bar_sync(1 + half, 128);
 #pragma unroll 1
-        for (int c = 0; c < S::NCHUNK; ++c) {
-          if (is_out && c + 1 < S::NCHUNK) prefetch_l1(hrow + 4 * (c + 1));
+        for (int c = 0; c < S::NCHUNK; ++c, ++hcnt) {
+          // this chunk of h: 128 rows x 32 columns of this half, 64-byte
+          // swizzled rows (16-byte piece q of row r sits at q ^ ((r >> 1) & 3))
+          const uint32_t hslot = hcnt % S::HSLOTS;
+          int hgot = 0;
+          if (lane == 0)
+            hgot = wait_bounded(&hfull[hslot], (hcnt / S::HSLOTS) & 1u, abort_flag, args.status)
+                       ? 1 : 0;
+          hgot = __shfl_sync(FULL, hgot, 0);
+          const uint8_t* hrow_s = hring + hslot * S::HSLOT_BYTES + half * (S::HSLOT_BYTES / 2) +
+                                  rloc * 64;
+          const int hsw = (rloc >> 1) & 3;
           float v[32];
           __syncwarp();
           if (got) {
@@ -492,16 +544,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub) {
             const int c0 = sub * 16;
-            const int sc = 2 * c + sub;
-            uint4 hnx[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q)
-              hnx[q] = (is_out && sc + 1 < 2 * S::NCHUNK) ? __ldg(hrow + 2 * (sc + 1) + q)
-                                                          : make_uint4(0, 0, 0, 0);
             float hv[16];
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-              const uint4 wv = hcur[q];
+              const uint4 wv = hgot ? *reinterpret_cast<const uint4*>(
+                                          hrow_s + (((2 * sub + q) ^ hsw) << 4))
+                                    : make_uint4(0, 0, 0, 0);
               const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
@@ -573,9 +621,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
             }
             if (!decode) named_bar_sync(1 + half, 128);  // reads done before the next write
-#pragma unroll
-            for (int q = 0; q < 2; ++q) hcur[q] = hnx[q];
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&hempty[hslot]);
         }
         if (decode) named_bar_sync(1 + half, 128);  // taps read before the next tile loads them
       }
@@ -639,22 +687,24 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [rows, cols] (cols contiguous), boxes of 64 columns x box_rows.
-bool make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+// 2-D bf16 tensor [rows, cols] (cols contiguous), boxes of box_cols x box_rows.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+               uint32_t box_rows, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int BN, int STAGES, int MODE>
-int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, cudaStream_t s) {
-  using S = TcShape<BN, STAGES>;
+int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& th,
+                const TcArgs& a, cudaStream_t s) {
+  using S = TcShape<BN, STAGES, MODE>;
   auto kern = tc_fused_kernel<BN, STAGES, MODE>;
   static bool configured[64] = {false};
   int dev = 0;
@@ -671,19 +721,22 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, c
   const int tiles = a.num_m_tiles * a.num_n_tiles;
   const int grid = tiles < sms ? tiles : sms;
   if (grid <= 0) return ENGRAM_OK;
-  kern<<<grid, NUM_THREADS, S::SMEM, s>>>(ta, tb, a);
+  kern<<<grid, NUM_THREADS, S::SMEM, s>>>(ta, tb, th, a);
   return ck(cudaGetLastError());
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES_K, int STAGES_V>
 int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
               float* alpha_saved, int64_t N, int T, int d, int E, float4* part, float* alpha,
               cudaStream_t s) {
-  CUtensorMap ta, tbk, tbv;
-  if (!make_tmap(&ta, e, (uint64_t)E, (uint64_t)N, BM)) return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&tbk, Wk, (uint64_t)E, (uint64_t)d, BN)) return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&tbv, Wv, (uint64_t)E, (uint64_t)d, BN)) return ENGRAM_ERR_CUDA;
+  CUtensorMap ta, tbk, tbv, th;
+  const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_tmap(&ta, e, (uint64_t)E, (uint64_t)N, BK, BM, sw128)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&tbk, Wk, (uint64_t)E, (uint64_t)d, BK, BN, sw128)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&tbv, Wv, (uint64_t)E, (uint64_t)d, BK, BN, sw128)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&th, h, (uint64_t)d, (uint64_t)N, 32, BM, CU_TENSOR_MAP_SWIZZLE_64B))
+    return ENGRAM_ERR_CUDA;
   TcArgs a;
   a.num_n_tiles = d / BN;
   a.num_k_tiles = E / BK;
@@ -703,7 +756,7 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.m_stride = BM;
   a.m_offset = 0;
   a.num_m_tiles = (int)((N + BM - 1) / BM);
-  int rc = launch_pass<BN, STAGES, MODE_GATE_PARTIAL>(ta, tbk, a, s);
+  int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL>(ta, tbk, th, a, s);
   if (rc) return rc;
   gate_from_partials_kernel<<<(unsigned)((N + 255) / 256), 256, 0, s>>>(part, a.n_part, N, d,
                                                                         alpha, alpha_saved);
@@ -718,7 +771,7 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
     a.m_offset = -HALO;
   }
   a.num_m_tiles = (int)((N + a.m_stride - 1) / a.m_stride);
-  return launch_pass<BN, STAGES, MODE_VALUE_CONV>(ta, tbv, a, s);
+  return launch_pass<BN, STAGES_V, MODE_VALUE_CONV>(ta, tbv, th, a, s);
 }
 
 inline bool use_wide(int64_t N, int d) { return d % 256 == 0 && N > 4096; }
@@ -748,9 +801,9 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
   float* alpha = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                           (size_t)N * 2 * (d / BN) * sizeof(float4));
   if (wide)
-    return run_layer<256, 4>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
+    return run_layer<256, 4, 3>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
                              alpha, s);
-  return run_layer<64, 8>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
+  return run_layer<64, 8, 6>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
                           alpha, s);
 }
 
