@@ -48,7 +48,9 @@ constexpr float RMS_EPS = 1e-6f;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 constexpr unsigned FULL = 0xffffffffu;
 
-enum { MODE_GATE_PARTIAL = 0, MODE_VALUE_CONV = 1 };
+// pass K; pass V over whole sequences (conv history from the rows above);
+// pass V in decode (one token per sequence, conv history from the state)
+enum { MODE_GATE_PARTIAL = 0, MODE_VALUE_CONV = 1, MODE_VALUE_DECODE = 2 };
 
 struct TcArgs {
   int num_m_tiles, num_n_tiles, num_k_tiles;
@@ -88,14 +90,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One bounded wait on a phase: the thread sleeps in hardware until the phase
+// completes or about 20 us pass (no busy spinning that would take issue slots
+// from the epilogue warps).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
       : "memory");
   return ok != 0;
 }
@@ -115,7 +120,7 @@ __device__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort
   const uint64_t t0 = global_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 63u) == 0) {
+    if ((spin & 3u) == 0) {
       if (*abort_flag) return false;
       if (global_ns() - t0 > WAIT_LIMIT_NS) {
         *abort_flag = 1;
@@ -143,6 +148,27 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// bf16 box from shared memory to global memory (rows outside the tensor are
+// not written); completion tracked by bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0,
+                                             int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// the shared-memory sources of this thread's bulk stores have been read
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -225,6 +251,30 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }
 
+// 16 consecutive fp32 columns of this thread's TMEM lane, without waiting:
+// the registers are valid only after tmem_wait16 on the same array.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&u)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+        "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
+        "=r"(u[14]), "=r"(u[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Waits for this thread's outstanding TMEM loads; naming the registers keeps
+// the compiler from moving their uses above the wait.
+__device__ __forceinline__ void tmem_wait16(uint32_t (&u)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(u[0]), "+r"(u[1]), "+r"(u[2]), "+r"(u[3]), "+r"(u[4]), "+r"(u[5]),
+                 "+r"(u[6]), "+r"(u[7]), "+r"(u[8]), "+r"(u[9]), "+r"(u[10]), "+r"(u[11]),
+                 "+r"(u[12]), "+r"(u[13]), "+r"(u[14]), "+r"(u[15])
+               :
+               : "memory");
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -253,41 +303,49 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 template <int BN, int STAGES, int MODE>
 struct TcShape {
+  static constexpr bool VPASS = MODE != MODE_GATE_PARTIAL;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int TMEM_COLS = 2 * BN;
+  // pass K (tokens on TMEM lanes, features on columns): each epilogue warp
+  // takes half of the tile's columns, 32 at a time
   static constexpr int HALF_COLS = BN / 2;
   static constexpr int NCHUNK = HALF_COLS / 32;
-  // pass V: ring of h chunks (128 rows x 32 columns for each half, 64-byte
-  // swizzle), filled by TMA ahead of the epilogue
-  static constexpr int HSLOTS = MODE == MODE_VALUE_CONV ? 3 : 0;
-  static constexpr int HSLOT_BYTES = 2 * BM * 32 * 2;
-  // pass V stages the scaled values of 16 columns of all 128 rows per half:
-  // rows of 20 floats (16 + 4 pad) keep 16-byte vectors conflict-free
-  static constexpr int SB_STRIDE = 20;
-  static constexpr int TAP_BYTES = 2 * HALF_COLS * 16;
-  static constexpr int SB_BYTES = 2 * BM * SB_STRIDE * 4;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) +
-                                 (size_t)HSLOTS * HSLOT_BYTES + 256 + TAP_BYTES + SB_BYTES;
+  // pass V (features on TMEM lanes, tokens on columns): each epilogue warp
+  // takes half of the tile's tokens, 32 at a time; h arrives by TMA in slots
+  // of two boxes (one per half) of 32 tokens x 128 features
+  static constexpr int HSLOTS = VPASS ? 4 : 0;
+  static constexpr int HBOX_BYTES = 32 * BM * 2;
+  static constexpr int HSLOT_BYTES = 2 * HBOX_BYTES;
+  static constexpr int ALPHA_BYTES = VPASS ? 2 * BN * 4 : 0;  // gates of a tile, two tiles
+  static constexpr size_t SMEM = (size_t)STAGES * (A_BYTES + B_BYTES) +
+                                 (size_t)HSLOTS * HSLOT_BYTES + 256 + ALPHA_BYTES;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "N tile");
-  static_assert(2 * STAGES + 11 <= 30, "barrier area");
+  static_assert(2 * STAGES + 13 <= 30, "barrier area");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
 template <int BN, int STAGES, int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmH, const __grid_constant__ TcArgs args) {
+                    const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmO,
+                    const __grid_constant__ CUtensorMap tmO29, const __grid_constant__ TcArgs args) {
   using S = TcShape<BN, STAGES, MODE>;
+  constexpr bool VPASS = S::VPASS;
   constexpr uint32_t STAGE_TX = S::A_BYTES + S::B_BYTES;
   // instruction descriptor: fp32 accumulate, bf16 A and B, both K-major,
   // N >> 3 at bit 17, M >> 4 at bit 24
   constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                              ((uint32_t)(BM >> 4) << 24);
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // The kernel declares no static shared memory, so the dynamic block starts
+  // at the base of the CTA's window.  Addressing everything from the
+  // __shared__ array keeps every access a shared-memory instruction.
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {  // 128-byte swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(args.status, ENGRAM_STATUS_TIMEOUT);
+    return;
+  }
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::A_BYTES;
   uint8_t* hring = sB + STAGES * S::B_BYTES;
@@ -298,14 +356,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* hfull = drain + 1;
-  uint64_t* hempty = hfull + 3;
+  uint64_t* hempty = hfull + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 30);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 31);
-  float4* tapbuf = reinterpret_cast<float4*>(bars + 32);
-  float* stagebuf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(tapbuf) + S::TAP_BYTES);
+  float* alpha_s = reinterpret_cast<float*>(bars + 32);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_tiles = args.num_m_tiles * args.num_n_tiles;
+
+  // Tile t covers token block t / num_n_tiles and feature block
+  // t % num_n_tiles.  Pass K multiplies e (tokens, A) by W_k (features, B);
+  // pass V multiplies W_v (features, A) by e (tokens, B).
+  auto operand_rows = [&](int tile, int& arow, int& brow) {
+    const int mi = tile / args.num_n_tiles, ni = tile - mi * args.num_n_tiles;
+    const int tok0 = mi * args.m_stride + args.m_offset;
+    if (VPASS) {
+      arow = ni * BM;
+      brow = tok0;
+    } else {
+      arow = tok0;
+      brow = ni * BN;
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -319,14 +391,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(drain, 1);
     for (int b = 0; b < S::HSLOTS; ++b) {
       mbar_init(&hfull[b], 1);
-      mbar_init(&hempty[b], NUM_EPI_WARPS);
+      mbar_init(&hempty[b], 2);  // one release per half, after its output box is stored
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    if (MODE == MODE_VALUE_CONV) prefetch_tmap(&tmH);
+    if (VPASS) {
+      prefetch_tmap(&tmH);
+      prefetch_tmap(&tmO);
+      prefetch_tmap(&tmO29);
+    }
   }
   if (warp == 1) {
     __syncwarp();
@@ -338,15 +414,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ operand producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        const int mt = tile / args.num_n_tiles, nt = tile - mt * args.num_n_tiles;
-        const int row0 = mt * args.m_stride + args.m_offset;
-        const int col0 = nt * BN;
+        int arow, brow;
+        operand_rows(tile, arow, brow);
         bool ok = true;
         for (int kt = 0; kt < args.num_k_tiles; ++kt) {
           if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
@@ -354,8 +429,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           mbar_expect_tx(&full[stage], STAGE_TX);
-          tma_load_2d(sA + stage * S::A_BYTES, &tmA, &full[stage], kt * BK, row0);
-          tma_load_2d(sB + stage * S::B_BYTES, &tmB, &full[stage], kt * BK, col0);
+          tma_load_2d(sA + stage * S::A_BYTES, &tmA, &full[stage], kt * BK, arow);
+          tma_load_2d(sB + stage * S::B_BYTES, &tmB, &full[stage], kt * BK, brow);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -411,25 +486,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       wait_drain(drain, 0);
     }
   } else if (warp == HP_WARP) {
-    // ------------------------------------------------------------ h producer
-    if (MODE == MODE_VALUE_CONV && lane == 0) {
+    // ------------------------------------------------------------ h producer (pass V)
+    if (VPASS && lane == 0) {
+      constexpr int NCH = (BN / 2) / 32;
       int slot = 0;
       uint32_t ph = 0;
       uint32_t issued = 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        const int mt = tile / args.num_n_tiles, nt = tile - mt * args.num_n_tiles;
-        const int row0 = mt * args.m_stride + args.m_offset;
+        const int mi = tile / args.num_n_tiles, ni = tile - mi * args.num_n_tiles;
+        const int tok0 = mi * args.m_stride + args.m_offset;
         bool ok = true;
-        for (int c = 0; c < S::NCHUNK; ++c) {
+        for (int c = 0; c < NCH; ++c) {
           if (!wait_bounded(&hempty[slot], ph ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
           }
           mbar_expect_tx(&hfull[slot], S::HSLOT_BYTES);
           uint8_t* dst = hring + slot * S::HSLOT_BYTES;
-          tma_load_2d(dst, &tmH, &hfull[slot], nt * BN + c * 32, row0);
-          tma_load_2d(dst + S::HSLOT_BYTES / 2, &tmH, &hfull[slot], nt * BN + S::HALF_COLS + c * 32,
-                      row0);
+          tma_load_2d(dst, &tmH, &hfull[slot], ni * BM, tok0 + c * 32);
+          tma_load_2d(dst + S::HBOX_BYTES, &tmH, &hfull[slot], ni * BM, tok0 + BN / 2 + c * 32);
           ++issued;
           if (++slot == S::HSLOTS) {
             slot = 0;
@@ -446,41 +521,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
-    const int quad = warp & 3;  // TMEM lanes this warp may read
-    const int half = ew >> 2;   // column half of the tile
-    const int rloc = quad * 32 + lane;
+    const int quad = warp & 3;  // TMEM lanes this warp may read: 32 * quad ..
+    const int half = ew >> 2;   // which half of the tile's columns
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t hcnt = 0;  // h chunks consumed so far (pass V)
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int mt = tile / args.num_n_tiles, nt = tile - mt * args.num_n_tiles;
+    uint32_t hslot = 0, hphase = 0;  // pass V: next h ring slot and its phase parity
+    int iter = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
+      const int mi = tile / args.num_n_tiles, ni = tile - mi * args.num_n_tiles;
+      const int64_t tok0 = (int64_t)mi * args.m_stride + args.m_offset;
       int got = 0;
       if (lane == 0) got = wait_bounded(&tfull[acc], acc_phase, abort_flag, args.status) ? 1 : 0;
       got = __shfl_sync(FULL, got, 0);
       tc_fence_after();
-      const int64_t n = (int64_t)mt * args.m_stride + args.m_offset + rloc;
-      const bool valid = n >= 0 && n < args.N;
-      const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN) +
-                             (uint32_t)(half * S::HALF_COLS);
-      const int col_base = nt * BN + half * S::HALF_COLS;
+      const uint32_t t_acc = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
 
-      // the next tile of this CTA: pull its rows of h (and, in pass V, of the
-      // gate partials) into L2 while this tile's epilogue runs
-      {
-        const int nxt = tile + (int)gridDim.x;
-        if (nxt < num_tiles) {
-          const int mt2 = nxt / args.num_n_tiles, nt2 = nxt - mt2 * args.num_n_tiles;
-          const int64_t n2 = (int64_t)mt2 * args.m_stride + args.m_offset + rloc;
-          if (n2 >= 0 && n2 < args.N) {
-            if (MODE == MODE_GATE_PARTIAL) {
-              const __nv_bfloat16* hp2 = args.h + n2 * args.d + nt2 * BN + half * S::HALF_COLS;
+      if constexpr (!VPASS) {
+        // pass K: this lane's token, half of the tile's features
+        const int64_t n = tok0 + quad * 32 + lane;
+        const bool valid = n >= 0 && n < args.N;
+        const int col_base = ni * BN + half * S::HALF_COLS;
+        const uint32_t t_row = t_acc + (uint32_t)(half * S::HALF_COLS);
+        {  // pull the next tile's rows of h into L2 while this one is reduced
+          const int nxt = tile + (int)gridDim.x;
+          if (nxt < num_tiles) {
+            const int mi2 = nxt / args.num_n_tiles, ni2 = nxt - mi2 * args.num_n_tiles;
+            const int64_t n2 = (int64_t)mi2 * args.m_stride + args.m_offset + quad * 32 + lane;
+            if (n2 >= 0 && n2 < args.N) {
+              const __nv_bfloat16* hp2 = args.h + n2 * args.d + ni2 * BN + half * S::HALF_COLS;
               for (int b = 0; b < S::HALF_COLS * 2; b += 128) prefetch_l2(hp2 + b / 2);
             }
-            if (MODE == MODE_VALUE_CONV && (rloc & 31) == 0) prefetch_l2(args.alpha + n2);
           }
         }
-      }
-      if (MODE == MODE_GATE_PARTIAL) {
         float kk = 0.f, hk = 0.f, hh = 0.f;
 #pragma unroll 1
         for (int c = 0; c < S::NCHUNK; ++c) {
@@ -503,129 +575,143 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        if (valid) args.part[n * args.n_part + nt * 2 + half] = make_float4(kk, hk, hh, 0.f);
+        if (valid) args.part[n * args.n_part + ni * 2 + half] = make_float4(kk, hk, hh, 0.f);
       } else {
-        const float alpha = valid ? __ldg(args.alpha + n) : 0.f;
-        const bool decode = args.conv_state != nullptr;
-        const bool is_out = valid && rloc >= -args.m_offset;
-        const int pos = valid ? (int)(n % args.T) : 0;
-        // causal masks: vt of rows t-1, t-2, t-3 count only inside the sequence
-        const float m1 = pos >= 1 ? 1.f : 0.f, m2 = pos >= 2 ? 1.f : 0.f,
-                    m3 = pos >= 3 ? 1.f : 0.f;
-        float4* taps = tapbuf + half * S::HALF_COLS;
-        float* sb = stagebuf + half * (BM * S::SB_STRIDE);
-        // conv taps of this half's columns, shared by its four warps
-        for (int c = rloc; c < S::HALF_COLS; c += 128) taps[c] = __ldg(args.conv_w + col_base + c);
-        named_bar_sync(1 + half, 128);
-#pragma unroll 1
-        for (int c = 0; c < S::NCHUNK; ++c, ++hcnt) {
-          // this chunk of h: 128 rows x 32 columns of this half, 64-byte
-          // swizzled rows (16-byte piece q of row r sits at q ^ ((r >> 1) & 3))
-          const uint32_t hslot = hcnt % S::HSLOTS;
-          int hgot = 0;
-          if (lane == 0)
-            hgot = wait_bounded(&hfull[hslot], (hcnt / S::HSLOTS) & 1u, abort_flag, args.status)
-                       ? 1 : 0;
-          hgot = __shfl_sync(FULL, hgot, 0);
-          const uint8_t* hrow_s = hring + hslot * S::HSLOT_BYTES + half * (S::HSLOT_BYTES / 2) +
-                                  rloc * 64;
-          const int hsw = (rloc >> 1) & 3;
-          float v[32];
+        // pass V: this lane's feature, half of the tile's tokens.  The causal
+        // conv walks the tokens in order with vt of the three previous tokens
+        // of the same sequence in registers.
+        constexpr bool DECODE = MODE == MODE_VALUE_DECODE;
+        constexpr int HALF_TOK = BN / 2;
+        constexpr int NCH = HALF_TOK / 32;
+        const int feat = ni * BM + quad * 32 + lane;
+        const int T = args.T;
+        // gates of the tile's tokens, staged once by all epilogue warps
+        float* al = alpha_s + (iter & 1) * BN;
+        for (int i = ew * 32 + lane; i < BN; i += NUM_EPI_WARPS * 32) {
+          const int64_t n = tok0 + i;
+          al[i] = (n >= 0 && n < args.N) ? __ldg(args.alpha + n) : 0.f;
+        }
+        named_bar_sync(1, NUM_EPI_WARPS * 32);
+        const float4 w = __ldg(args.conv_w + feat);  // taps: w.x for t-3 .. w.w for t
+        const int j0 = half * HALF_TOK;              // first tile column of this warp
+        const int first_out = -args.m_offset;        // halo columns produce no output
+        int pos = (int)((((tok0 + j0) % T) + T) % T);  // sequence position of column j0
+        float s1 = 0.f, s2 = 0.f, s3 = 0.f;           // vt of tokens t-1, t-2, t-3
+        if (!DECODE && j0 > 0) {
+          // the three columns before this half, recomputed from TMEM
+          uint32_t u4[16];
           __syncwarp();
           if (got) {
-            tmem_ld32(t_row + c * 32, v);
+            tmem_ld16(t_acc + (uint32_t)(j0 - 16), u4);
+            tmem_wait16(u4);
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            for (int i = 0; i < 16; ++i) u4[i] = 0u;
           }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;  // vt
-          const int col = col_base + c * 32;
+          for (int i = 13; i < 16; ++i) {
+            const int pq = (((pos - (16 - i)) % T) + T) % T;
+            const float vt = al[j0 - 16 + i] * __uint_as_float(u4[i]);
+            if (pq == 0) s1 = s2 = s3 = 0.f;
+            s3 = s2;
+            s2 = s1;
+            s1 = vt;
+          }
+        }
+#pragma unroll 1
+        for (int c = 0; c < NCH; ++c) {
+          int hgot = 0;
+          if (lane == 0) hgot = wait_bounded(&hfull[hslot], hphase, abort_flag, args.status) ? 1 : 0;
+          hgot = __shfl_sync(FULL, hgot, 0);
+          // h of token jj and feature f of this box: box[jj * BM + f]; the
+          // output of the same element replaces it in place
+          uint8_t* box = hring + hslot * S::HSLOT_BYTES + half * S::HBOX_BYTES;
+          uint16_t* hs = reinterpret_cast<uint16_t*>(box) + quad * 32 + lane;
+          uint32_t u[16], un[16];
+          __syncwarp();
+          if (got) {
+            tmem_ld16(t_acc + (uint32_t)(j0 + c * 32), u);
+            tmem_ld16(t_acc + (uint32_t)(j0 + c * 32 + 16), un);
+            tmem_wait16(u);
+          } else {
 #pragma unroll
-          for (int sub = 0; sub < 2; ++sub) {
-            const int c0 = sub * 16;
-            float hv[16];
+            for (int i = 0; i < 16; ++i) u[i] = un[i] = 0u;
+          }
+          const int jb = j0 + c * 32;
+          const int64_t nb = tok0 + jb;
+          const float4* al4 = reinterpret_cast<const float4*>(al + jb);
+          // no sequence starts inside the chunk: no per-token checks
+          const bool clean = !DECODE && pos + 32 <= T && pos != 0;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const uint4 wv = hgot ? *reinterpret_cast<const uint4*>(
-                                          hrow_s + (((2 * sub + q) ^ hsw) << 4))
-                                    : make_uint4(0, 0, 0, 0);
-              const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+          for (int g = 0; g < 2; ++g) {
+            if (g == 1) {
+              if (got) tmem_wait16(un);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                hv[q * 8 + 2 * i] = __uint_as_float(ws[i] << 16);
-                hv[q * 8 + 2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
-              }
+              for (int i = 0; i < 16; ++i) u[i] = un[i];
             }
-            float* st = (decode && is_out) ? args.conv_state + n * 3 * args.d + col + c0 : nullptr;
-            const float4* r1 = nullptr;
-            const float4* r2 = nullptr;
-            const float4* r3 = nullptr;
-            if (!decode) {
-              // publish this row's 16 values, then read the three rows above
-              float4* mine = reinterpret_cast<float4*>(sb + rloc * S::SB_STRIDE);
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                mine[q] = make_float4(v[c0 + 4 * q], v[c0 + 4 * q + 1], v[c0 + 4 * q + 2],
-                                      v[c0 + 4 * q + 3]);
-              named_bar_sync(1 + half, 128);
-              const int rr = rloc >= 3 ? rloc : 3;  // halo rows read a valid row, masked below
-              r1 = reinterpret_cast<const float4*>(sb + (rr - 1) * S::SB_STRIDE);
-              r2 = reinterpret_cast<const float4*>(sb + (rr - 2) * S::SB_STRIDE);
-              r3 = reinterpret_cast<const float4*>(sb + (rr - 3) * S::SB_STRIDE);
-            }
-            uint32_t packed[8];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              float a1[4], a2[4], a3[4];  // vt of rows t-1, t-2, t-3, four columns
-              if (decode) {
-                if (st != nullptr) {
+              const float4 a4 = al4[g * 4 + q];
+              const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                  for (int u = 0; u < 4; ++u) {
-                    const int k = 4 * q + u;
-                    a3[u] = st[k];
-                    a2[u] = st[args.d + k];
-                    a1[u] = st[2 * args.d + k];
-                    st[k] = a2[u];
-                    st[args.d + k] = a1[u];
-                    st[2 * args.d + k] = v[c0 + k];
+              for (int r = 0; r < 4; ++r) {
+                const int jj = g * 16 + q * 4 + r;
+                const float vt = av[r] * __uint_as_float(u[q * 4 + r]);
+                float y;
+                if (DECODE) {
+                  const int64_t n = nb + jj;
+                  float a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                  if (n < args.N) {
+                    float* st = args.conv_state + n * 3 * args.d + feat;
+                    a3 = st[0];
+                    a2 = st[args.d];
+                    a1 = st[2 * args.d];
+                    st[0] = a2;
+                    st[args.d] = a1;
+                    st[2 * args.d] = vt;
                   }
+                  y = fmaf(w.x, a3, fmaf(w.y, a2, fmaf(w.z, a1, w.w * vt)));
                 } else {
-#pragma unroll
-                  for (int u = 0; u < 4; ++u) a1[u] = a2[u] = a3[u] = 0.f;
+                  if (!clean) {
+                    if (pos == 0) s1 = s2 = s3 = 0.f;  // a sequence starts at this token
+                    pos = (pos + 1 == T) ? 0 : pos + 1;
+                  }
+                  y = fmaf(w.x, s3, fmaf(w.y, s2, fmaf(w.z, s1, w.w * vt)));
+                  s3 = s2;
+                  s2 = s1;
+                  s1 = vt;
                 }
-              } else {
-                const float4 x1 = r1[q], x2 = r2[q], x3 = r3[q];
-                a1[0] = x1.x * m1; a1[1] = x1.y * m1; a1[2] = x1.z * m1; a1[3] = x1.w * m1;
-                a2[0] = x2.x * m2; a2[1] = x2.y * m2; a2[2] = x2.z * m2; a2[3] = x2.w * m2;
-                a3[0] = x3.x * m3; a3[1] = x3.y * m3; a3[2] = x3.z * m3; a3[3] = x3.w * m3;
+                const float hv = __uint_as_float(((uint32_t)hs[jj * BM]) << 16);
+                const float o = hv + vt + __fdividef(y, 1.0f + __expf(-y));  // h + vt + SiLU(y)
+                hs[jj * BM] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
               }
-              float o[4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int k = 4 * q + u;
-                const float4 w = taps[c * 32 + c0 + k];
-                float y = w.w * v[c0 + k];
-                y = fmaf(w.z, a1[u], y);
-                y = fmaf(w.y, a2[u], y);
-                y = fmaf(w.x, a3[u], y);
-                const float sy = __fdividef(y, 1.0f + __expf(-y));  // SiLU
-                o[u] = hv[k] + v[c0 + k] + sy;
-              }
-              packed[2 * q] = pack_bf16x2(o[0], o[1]);
-              packed[2 * q + 1] = pack_bf16x2(o[2], o[3]);
             }
-            if (is_out) {
-              uint4* dst = reinterpret_cast<uint4*>(args.out + n * args.d + col + c0);
-              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-            }
-            if (!decode) named_bar_sync(1 + half, 128);  // reads done before the next write
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&hempty[hslot]);
+          if (clean) {
+            pos += 32;
+            if (pos == T) pos = 0;
+          }
+          // the half's four warps have written the box: one thread stores it
+          fence_async_shared();
+          named_bar_sync(2 + half, 128);
+          if (ew == half * 4 && lane == 0) {
+            if (hgot && got) {
+              if (jb < first_out) {
+                // the first tokens of the tile are the conv halo of the
+                // previous tile: store from the first output token on
+                tma_store_2d(&tmO29, box + first_out * BM * 2, ni * BM, (int)(nb + first_out));
+              } else {
+                tma_store_2d(&tmO, box, ni * BM, (int)nb);
+              }
+              tma_store_wait_read();
+            }
+            mbar_arrive(&hempty[hslot]);
+          }
+          if (++hslot == (uint32_t)S::HSLOTS) {
+            hslot = 0;
+            hphase ^= 1u;
+          }
         }
-        if (decode) named_bar_sync(1 + half, 128);  // taps read before the next tile loads them
       }
       tc_fence_before();
       __syncwarp();
@@ -633,6 +719,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    // output boxes of pass V fully written before the CTA exits
+    if (VPASS && ew == half * 4 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
   __syncthreads();
@@ -703,7 +791,7 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
 
 template <int BN, int STAGES, int MODE>
 int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& th,
-                const TcArgs& a, cudaStream_t s) {
+                const CUtensorMap& to, const CUtensorMap& to29, const TcArgs& a, cudaStream_t s) {
   using S = TcShape<BN, STAGES, MODE>;
   auto kern = tc_fused_kernel<BN, STAGES, MODE>;
   static bool configured[64] = {false};
@@ -721,7 +809,7 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   const int tiles = a.num_m_tiles * a.num_n_tiles;
   const int grid = tiles < sms ? tiles : sms;
   if (grid <= 0) return ENGRAM_OK;
-  kern<<<grid, NUM_THREADS, S::SMEM, s>>>(ta, tb, th, a);
+  kern<<<grid, NUM_THREADS, S::SMEM, s>>>(ta, tb, th, to, to29, a);
   return ck(cudaGetLastError());
 }
 
@@ -730,20 +818,28 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
               float* alpha_saved, int64_t N, int T, int d, int E, float4* part, float* alpha,
               cudaStream_t s) {
-  CUtensorMap ta, tbk, tbv, th;
   const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_tmap(&ta, e, (uint64_t)E, (uint64_t)N, BK, BM, sw128)) return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&tbk, Wk, (uint64_t)E, (uint64_t)d, BK, BN, sw128)) return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&tbv, Wv, (uint64_t)E, (uint64_t)d, BK, BN, sw128)) return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&th, h, (uint64_t)d, (uint64_t)N, 32, BM, CU_TENSOR_MAP_SWIZZLE_64B))
+  // pass K: A = e (128 tokens per tile), B = W_k (BN features per tile)
+  CUtensorMap ta_k, tb_k, ta_v, tb_v, th, to, to29;
+  if (!make_tmap(&ta_k, e, (uint64_t)E, (uint64_t)N, BK, BM, sw128)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&tb_k, Wk, (uint64_t)E, (uint64_t)d, BK, BN, sw128)) return ENGRAM_ERR_CUDA;
+  // pass V: A = W_v (128 features per tile), B = e (BN tokens per tile);
+  // h in boxes of 32 tokens x 128 features
+  if (!make_tmap(&ta_v, Wv, (uint64_t)E, (uint64_t)d, BK, BM, sw128)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&tb_v, e, (uint64_t)E, (uint64_t)N, BK, BN, sw128)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&th, h, (uint64_t)d, (uint64_t)N, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return ENGRAM_ERR_CUDA;
+  // out in the same boxes; a 29-token box skips the 3 halo tokens of a tile
+  if (!make_tmap(&to, out, (uint64_t)d, (uint64_t)N, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&to29, out, (uint64_t)d, (uint64_t)N, BM, 32 - HALO, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ENGRAM_ERR_CUDA;
   TcArgs a;
-  a.num_n_tiles = d / BN;
   a.num_k_tiles = E / BK;
   a.N = N;
   a.T = T;
   a.d = d;
-  a.n_part = 2 * a.num_n_tiles;
+  a.n_part = 2 * (d / BN);
   a.h = h;
   a.out = out;
   a.part = part;
@@ -752,26 +848,30 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.alpha_out = alpha_saved;
   a.alpha = nullptr;
   a.status = status_ptr();
-  // pass K: gate partials
+  // pass K: gate partials, tiles of 128 tokens x BN features
+  a.num_n_tiles = d / BN;
   a.m_stride = BM;
   a.m_offset = 0;
   a.num_m_tiles = (int)((N + BM - 1) / BM);
-  int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL>(ta, tbk, th, a, s);
+  int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL>(ta_k, tb_k, th, to, to29, a, s);
   if (rc) return rc;
   gate_from_partials_kernel<<<(unsigned)((N + 255) / 256), 256, 0, s>>>(part, a.n_part, N, d,
                                                                         alpha, alpha_saved);
   a.alpha = alpha;
-  // pass V: gate, conv, residual (overlapping tiles with a 3-row halo, or
-  // plain tiles plus the conv state in decode)
+  // pass V: tiles of 128 features x BN tokens.  Whole sequences: the token
+  // tiles overlap by 3 (the conv halo, recomputed); decode: plain tiles.
+  a.num_n_tiles = d / BM;
   if (conv_state != nullptr) {
-    a.m_stride = BM;
+    a.m_stride = BN;
     a.m_offset = 0;
   } else {
-    a.m_stride = BM - HALO;
+    a.m_stride = BN - HALO;
     a.m_offset = -HALO;
   }
   a.num_m_tiles = (int)((N + a.m_stride - 1) / a.m_stride);
-  return launch_pass<BN, STAGES_V, MODE_VALUE_CONV>(ta, tbv, th, a, s);
+  if (conv_state != nullptr)
+    return launch_pass<BN, STAGES_V, MODE_VALUE_DECODE>(ta_v, tb_v, th, to, to29, a, s);
+  return launch_pass<BN, STAGES_V, MODE_VALUE_CONV>(ta_v, tb_v, th, to, to29, a, s);
 }
 
 inline bool use_wide(int64_t N, int d) { return d % 256 == 0 && N > 4096; }
@@ -779,7 +879,7 @@ inline bool use_wide(int64_t N, int d) { return d % 256 == 0 && N > 4096; }
 }  // namespace
 
 int tc_supported(int d, int E, int M) {
-  return M == 1 && E % BK == 0 && E >= BK && d % 64 == 0 && d >= 64;
+  return M == 1 && E % BK == 0 && E >= BK && d % BM == 0 && d >= BM;
 }
 
 size_t tc_forward_ws_bytes(int64_t N, int d, int E) {

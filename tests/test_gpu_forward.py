@@ -106,7 +106,7 @@ def _bf16_unit_case(B, T, d, K, D_h, seed, rows=None, decode_steps=0):
 @pytest.mark.parametrize("B,T,d,K,D_h", [
     (3, 100, 256, 2, 32),      # narrow tiles (N=64), ragged last M tile
     (1, 1, 128, 2, 32),        # a single token
-    (4, 2, 192, 2, 16),        # every token within the conv's start-up
+    (4, 2, 128, 2, 16),        # every token within the conv's start-up
     (2, 2500, 512, 2, 32),     # wide tiles (N=256), 40 overlapping V tiles of 125
     (1, 4100, 256, 4, 16),     # wide tiles with several sequences per tile boundary
 ])
