@@ -302,8 +302,15 @@ def run_ours(args):
     traffic = None
     tp = os.path.join(ROOT, "profiles", "traffic_layer27b.json")
     if os.path.exists(tp):
+        # the counters apply only to the kernel source they were taken from
+        import hashlib
         with open(tp) as f:
-            traffic = json.load(f).get("fused_tc_traffic_bytes_per_step")
+            rec = json.load(f)
+        src = os.path.join(ROOT, "hashed_gram_conditional_engram_b200", "csrc", "fusion_tc.cu")
+        with open(src, "rb") as f:
+            sha = hashlib.sha1(f.read()).hexdigest()
+        if rec.get("source_sha1_fusion_tc") == sha:
+            traffic = rec.get("fused_tc_traffic_bytes_per_step")
 
     line = None
     if rank == 0:
