@@ -227,6 +227,22 @@ int engram_table_grad(const engram_cfg_t* cfg, const int32_t* idx, const float* 
                            ws, ws_bytes, (cudaStream_t)stream);
 }
 
+int engram_table_grad_noalloc(const engram_cfg_t* cfg, const int32_t* idx, const float* de,
+                              int64_t n_tok, int64_t* dtab_keys, float* dtab_rows,
+                              int32_t* n_unique, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (n_tok < 0 || n_unique == nullptr) return ENGRAM_ERR_INVALID_ARG;
+  if (n_tok > 0 && (idx == nullptr || de == nullptr || dtab_keys == nullptr || dtab_rows == nullptr))
+    return ENGRAM_ERR_INVALID_ARG;
+  if (!aligned16(idx) || !aligned16(de) || !aligned16(dtab_keys) || !aligned16(dtab_rows))
+    return ENGRAM_ERR_MISALIGNED;
+  if (n_tok * 2 * cfg->K > ENGRAM_NOALLOC_MAX_ITEMS) return ENGRAM_ERR_TOO_LARGE;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  return launch_table_grad_noalloc(make_head_params(cfg), idx, de, n_tok, dtab_keys, dtab_rows,
+                                   n_unique, (cudaStream_t)stream);
+}
+
 int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const void* host_table,
                              int64_t n_tok, void* e, void* side_stream, void* done_event) {
   int rc = check_cfg(cfg);

@@ -63,6 +63,9 @@ int launch_table_grad(const HeadParams& hp, const int32_t* idx, const float* de,
                       int64_t* keys, float* rows, int32_t* n_unique, void* ws, size_t ws_bytes,
                       cudaStream_t s);
 size_t vocab_ws_bytes(int64_t V);
+int launch_table_grad_noalloc(const HeadParams& hp, const int32_t* idx, const float* de,
+                              int64_t n_tok, int64_t* keys, float* rows, int32_t* n_unique,
+                              cudaStream_t s);
 int launch_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_c_out, void* ws,
                       size_t ws_bytes, cudaStream_t s);
 

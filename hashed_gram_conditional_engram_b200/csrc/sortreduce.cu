@@ -9,6 +9,8 @@
 //  * the vocabulary projection: a stable sort by key groups the raw ids of one
 //    key with the smallest id first; compressed ids number the groups in order
 //    of that first id (discuss.deepseek.club 二.1 (1) 词汇投影).
+#include <mutex>
+
 #include "internal.cuh"
 
 namespace engram {
@@ -23,7 +25,7 @@ constexpr int CHUNKS_PER_WARP = 8;                       // 8 x 32 items per war
 constexpr int TILE = SORT_THREADS * CHUNKS_PER_WARP;     // 2048 items per block
 constexpr unsigned FULL = 0xffffffffu;
 
-inline size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
+constexpr size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 __device__ __forceinline__ int digit_of(uint64_t key, int shift) {
   return (int)((key >> shift) & (RADIX - 1));
@@ -286,7 +288,7 @@ struct SortWs {
   int32_t* scal;  // 4 int32
 };
 
-size_t sort_ws_bytes(int64_t n) {
+constexpr size_t sort_ws_bytes(int64_t n) {
   const int64_t nblocks = (n + TILE - 1) / TILE;
   return 2 * up256(n * 8) + 2 * up256(n * 4) + up256(RADIX * nblocks * 4 + 4) +
          2 * up256(n * 4 + 4) + up256((n + 1) * 4) + 256;
@@ -339,6 +341,62 @@ int launch_table_grad(const HeadParams& hp, const int32_t* idx, const float* de,
 }
 
 size_t vocab_ws_bytes(int64_t V) { return sort_ws_bytes(V); }
+
+// ------------------------------------------------- table gradient without allocation
+//
+// For callers that cannot allocate device memory themselves (a host that
+// hands this library a fixed pool, code running inside a CUDA graph capture
+// where allocation calls are not allowed, or a plugin whose host framework
+// owns every allocation), the sparse table gradient can run on a scratch
+// array that is part of the library image: the GPU reserves it when the
+// library's device code is loaded and keeps it until the process exits.  It
+// holds the sort buffers for up to ENGRAM_NOALLOC_MAX_ITEMS (token, head)
+// pairs.  Every call reuses the same array: calls that overlap on the GPU
+// (different streams, or different host threads on one device) race and
+// must be serialised by the caller.  No word of the array has to start at
+// zero: each pass writes everything it reads.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = sort_ws_bytes(ENGRAM_NOALLOC_MAX_ITEMS);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device.  Host code only
+// sees a host-side stand-in under the array's name, so the address is taken
+// once per device with that device current.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+    return ENGRAM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return ENGRAM_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ENGRAM_OK;
+}
+
+}  // namespace
+
+int launch_table_grad_noalloc(const HeadParams& hp, const int32_t* idx, const float* de,
+                              int64_t n_tok, int64_t* keys, float* rows, int32_t* n_unique,
+                              cudaStream_t s) {
+  if (n_tok * hp.J > ENGRAM_NOALLOC_MAX_ITEMS) return ENGRAM_ERR_TOO_LARGE;
+  void* scratch = nullptr;
+  const int rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  return launch_table_grad(hp, idx, de, n_tok, keys, rows, n_unique, scratch, kNoAllocScratchBytes,
+                           s);
+}
 
 int launch_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_c_out, void* ws,
                       size_t ws_bytes, cudaStream_t s) {

@@ -30,12 +30,15 @@ ERRORS = {
     -4: "ENGRAM_ERR_UNSUPPORTED",
     -5: "ENGRAM_ERR_CUDA",
     -6: "ENGRAM_ERR_TIMEOUT",
+    -7: "ENGRAM_ERR_TOO_LARGE",
 }
+NOALLOC_MAX_ITEMS = 131072
 
 EXPORTED = (
     "engram_workspace_size", "engram_saved_size", "engram_build_vocab_proj",
     "engram_hash_indices", "engram_gather", "engram_forward", "engram_backward",
-    "engram_table_grad", "engram_forward_hosttable", "engram_get_status",
+    "engram_table_grad", "engram_table_grad_noalloc", "engram_forward_hosttable",
+    "engram_get_status",
     "engram_device_sm_count",
 )
 
@@ -101,6 +104,7 @@ def lib() -> ctypes.CDLL:
         "engram_backward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                            i32, i32, P, sz, P]),
         "engram_table_grad": (ctypes.c_int, [cfgp, P, P, i64, P, P, P, P, sz, P]),
+        "engram_table_grad_noalloc": (ctypes.c_int, [cfgp, P, P, i64, P, P, P, P]),
         "engram_forward_hosttable": (ctypes.c_int, [cfgp, P, P, i64, P, P, P]),
         "engram_get_status": (ctypes.c_int, [P]),
         "engram_device_sm_count": (ctypes.c_int, []),
@@ -187,6 +191,16 @@ def engram_table_grad(cfg: EngramCfg, idx, de, n_tok: int, dtab_keys, dtab_rows,
     _check("engram_table_grad",
            lib().engram_table_grad(ctypes.byref(cfg), _p(idx), _p(de), n_tok, _p(dtab_keys),
                                    _p(dtab_rows), _p(n_unique), _p(ws), ws_bytes, _s(stream)))
+
+
+def engram_table_grad_noalloc(cfg: EngramCfg, idx, de, n_tok: int, dtab_keys, dtab_rows, n_unique,
+                              stream=None) -> None:
+    """engram_table_grad on the library's built-in scratch array: allocates
+    nothing; n_tok * J must not exceed NOALLOC_MAX_ITEMS."""
+    _check("engram_table_grad_noalloc",
+           lib().engram_table_grad_noalloc(ctypes.byref(cfg), _p(idx), _p(de), n_tok,
+                                           _p(dtab_keys), _p(dtab_rows), _p(n_unique),
+                                           _s(stream)))
 
 
 def engram_forward_hosttable(cfg: EngramCfg, idx, host_table, n_tok: int, e, side_stream=None,

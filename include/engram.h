@@ -61,7 +61,8 @@ enum {
   ENGRAM_ERR_WORKSPACE = -3,   /* ws_bytes below engram_workspace_size */
   ENGRAM_ERR_UNSUPPORTED = -4, /* shape/dtype combination not built */
   ENGRAM_ERR_CUDA = -5,        /* a CUDA runtime call failed */
-  ENGRAM_ERR_TIMEOUT = -6      /* status word reports a pipeline wait that ran out */
+  ENGRAM_ERR_TIMEOUT = -6,     /* status word reports a pipeline wait that ran out */
+  ENGRAM_ERR_TOO_LARGE = -7    /* input larger than a fixed, built-in scratch area */
 };
 
 /* bits of the device status word */
@@ -214,6 +215,28 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
 int engram_table_grad(const engram_cfg_t* cfg, const int32_t* idx, const float* de, int64_t n_tok,
                       int64_t* dtab_keys, float* dtab_rows, int32_t* n_unique, void* ws,
                       size_t ws_bytes, void* stream);
+
+/*
+ * engram_table_grad without a workspace argument, for callers that cannot
+ * allocate device memory: a host framework that owns every allocation and
+ * hands out none for scratch, code recording a CUDA graph where allocation
+ * calls are not allowed, or a runtime with a fixed memory pool.  (The pages
+ * have no counterpart: this is an interface variant, not part of the method.)
+ *   Same arguments, outputs and results as engram_table_grad, minus ws.
+ *   The sort buffers live in a device array built into the library, sized
+ *   for n_tok * J <= ENGRAM_NOALLOC_MAX_ITEMS (token, head) pairs (about
+ *   4.8 MB, held on every GPU that loads the library until the process
+ *   exits).  Larger inputs return ENGRAM_ERR_TOO_LARGE and launch nothing.
+ *   The call allocates nothing.  Its first call on a device looks up the
+ *   array's device address (cudaGetSymbolAddress); make that first call
+ *   before capturing a stream into a graph.
+ *   All calls share the array: calls that overlap on the GPU (other streams,
+ *   other host threads) race and must be serialised by the caller.
+ */
+#define ENGRAM_NOALLOC_MAX_ITEMS 131072
+int engram_table_grad_noalloc(const engram_cfg_t* cfg, const int32_t* idx, const float* de,
+                              int64_t n_tok, int64_t* dtab_keys, float* dtab_rows,
+                              int32_t* n_unique, void* stream);
 
 /*
  * Gather from a table in pinned, mapped host memory over PCIe ([p5 二.2]
