@@ -77,6 +77,12 @@ def rank_seed(base: int, rank: int) -> int:
     return base + 7919 * rank
 
 
+def aggregate_rate(units_per_rank: int, world: int, steps: int, elapsed_ms_max: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time."""
+    return units_per_rank * world * steps / (elapsed_ms_max / 1e3)
+
+
 # ---------------------------------------------------------------- peaks, clocks
 
 def load_peaks():
@@ -260,7 +266,7 @@ def run_ours(args):
         raise RuntimeError("device status word set during timing")
     elapsed_ms = max_over_ranks(elapsed_ms)
     ms_per_step = elapsed_ms / args.steps
-    value = N * ws_ * args.steps / (elapsed_ms / 1e3)
+    value = aggregate_rate(N, ws_, args.steps, elapsed_ms)
 
     # ---- end to end through the public API with host buffers
     ids_h = torch.from_numpy(ids_np).pin_memory()
@@ -290,7 +296,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(s2.elapsed_time(e2))
-    e2e_value = N * ws_ * e2e_steps / (e2e_ms / 1e3)
+    e2e_value = aggregate_rate(N, ws_, e2e_steps, e2e_ms)
     h2d = ids_h.numel() * 4 + h_h.numel() * 2
     d2h = out_h.numel() * 2
 

@@ -5,26 +5,31 @@
 // value, combined by matrix products).  Each runs as one persistent tcgen05
 // GEMM pass with the rest of the layer fused into its epilogue:
 //
-//   pass K:  C = e * W_k^T tile by tile; the epilogue reduces each row of the
-//            tile to (sum k^2, sum h*k, sum h^2) partials -- k never reaches HBM.
-//   pass V:  C = e * W_v^T; the epilogue finishes the gate from the partials,
-//            alpha = sigmoid(<h, k> r_h r_k / sqrt(d)), scales v, runs the
-//            width-4 depthwise causal conv along the rows of the tile, applies
-//            SiLU and adds h + vt + SiLU(y) (sechub.in answer: short depthwise
-//            causal conv; discuss.deepseek.club 二.1 (2): 1-D conv, residual).
+//   pass K:  C = e * W_k^T (tokens on TMEM lanes); the epilogue reduces each
+//            token's row of the tile to (sum k^2, sum h*k, sum h^2) partials --
+//            k never reaches HBM.  A small kernel then forms
+//            alpha = sigmoid(<h, k> r_h r_k / sqrt(d)) per token.
+//   pass V:  C = W_v * e^T (features on TMEM lanes, tokens on columns); each
+//            epilogue thread owns one feature and walks consecutive tokens:
+//            vt = alpha * v, the width-4 depthwise causal conv with the three
+//            previous vt in registers, SiLU, and h + vt + SiLU(y) (sechub.in
+//            answer: short depthwise causal conv; discuss.deepseek.club
+//            二.1 (2): 1-D conv, residual).  h comes in and out goes back in
+//            32-token boxes by TMA.
 //
-// The causal conv needs vt of the three tokens before each row.  Pass V walks
-// the tokens in overlapping tiles of 128 rows that advance by 125: the first
-// three rows of a tile are a recomputed halo and produce no output.  In decode
-// (one token per sequence) the three earlier vt come from the conv state.
+// The conv needs vt of the three tokens before each one.  Pass V's token
+// tiles of 256 overlap by 3: the first three tokens of a tile are a
+// recomputed halo and are not stored.  In decode (one token per sequence) the
+// three earlier vt come from the conv state.
 //
-// Pipeline per CTA (one CTA per SM, 320 threads):
-//   warp 0      one lane issues TMA loads of A (e) and B (W) tiles into a ring
-//               of shared-memory stages (128-byte swizzle, K-major);
+// Pipeline per CTA (one CTA per SM):
+//   warp 0      one lane issues TMA loads of the A and B tiles into a ring of
+//               shared-memory stages (128-byte swizzle, K-major);
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
 //               K=16 per instruction) into one of two TMEM accumulators;
-//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4).. (its rows), half
-//               of the tile's columns each, 32 columns per tcgen05.ld.
+//   epilogue    8 warps: warp w reads TMEM lanes 32*(w%4).. and half of the
+//               tile's columns;
+//   last warp   pass V: one lane streams h into a ring of shared-memory boxes.
 // mbarriers link the roles; every wait is bounded in time and, when it runs
 // out, sets ENGRAM_STATUS_TIMEOUT and winds the CTA down without hanging.
 #include <cuda.h>
@@ -40,9 +45,6 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle row
 constexpr int UMMA_K = 16;
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int HP_WARP = 2 + NUM_EPI_WARPS;  // pass V: warp that streams h tiles in by TMA
-constexpr int NUM_THREADS = 64 + NUM_EPI_WARPS * 32 + 32;
 constexpr int HALO = 3;  // conv width 4 - 1
 constexpr float RMS_EPS = 1e-6f;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
@@ -160,11 +162,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
       "r"(smem_u32(src)), "r"(c0), "r"(c1)
       : "memory");
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// the shared-memory sources of this thread's bulk stores have been read
-__device__ __forceinline__ void tma_store_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void fence_async_shared() {
@@ -299,39 +296,83 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+// Pass V, 16 consecutive tokens of one feature: vt = alpha * v, the width-4
+// causal conv over (s3, s2, s1, vt), out = h + vt + SiLU(y), written over h in
+// place.  CHECK = true when a sequence may start inside the group: the conv
+// history is cleared at position 0.
+template <bool CHECK>
+__device__ __forceinline__ void conv_group16(const uint32_t (&u)[16], const float4* al4,
+                                             uint16_t* hs, const float4 w, float& s1, float& s2,
+                                             float& s3, int& pos, const int T) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 a4 = al4[q];
+    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int jj = q * 4 + r;
+      const float vt = av[r] * __uint_as_float(u[jj]);
+      if (CHECK) {
+        if (pos == 0) s1 = s2 = s3 = 0.f;  // a sequence starts at this token
+        pos = (pos + 1 == T) ? 0 : pos + 1;
+      }
+      const float y = fmaf(w.x, s3, fmaf(w.y, s2, fmaf(w.z, s1, w.w * vt)));
+      s3 = s2;
+      s2 = s1;
+      s1 = vt;
+      const float hv = __uint_as_float(((uint32_t)hs[jj * BM]) << 16);
+      const float o = hv + vt + __fdividef(y, 1.0f + __expf(-y));  // h + vt + SiLU(y)
+      hs[jj * BM] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+    }
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 
 template <int BN, int STAGES, int MODE>
 struct TcShape {
   static constexpr bool VPASS = MODE != MODE_GATE_PARTIAL;
+  // epilogue warps: 2 per TMEM lane quadrant
+  static constexpr int EPI = 8;
+  static constexpr int PARTS = EPI / 4;        // column parts of a tile, one per warp of a quadrant
+  static constexpr int HP_WARP = 2 + EPI;      // pass V: warp that streams h in by TMA
+  static constexpr int NUM_THREADS = 64 + EPI * 32 + 32;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int TMEM_COLS = 2 * BN;
   // pass K (tokens on TMEM lanes, features on columns): each epilogue warp
-  // takes half of the tile's columns, 32 at a time
-  static constexpr int HALF_COLS = BN / 2;
-  static constexpr int NCHUNK = HALF_COLS / 32;
+  // takes one part of the tile's columns, 32 at a time
+  static constexpr int PART_COLS = BN / PARTS;
+  static constexpr int NCHUNK = PART_COLS / 32;
   // pass V (features on TMEM lanes, tokens on columns): each epilogue warp
-  // takes half of the tile's tokens, 32 at a time; h arrives by TMA in slots
-  // of two boxes (one per half) of 32 tokens x 128 features
-  static constexpr int HSLOTS = VPASS ? 4 : 0;
+  // takes one part of the tile's tokens, 32 at a time; h arrives by TMA in
+  // slots of PARTS boxes (one per part) of 32 tokens x 128 features
   static constexpr int HBOX_BYTES = 32 * BM * 2;
-  static constexpr int HSLOT_BYTES = 2 * HBOX_BYTES;
+  static constexpr int HSLOT_BYTES = PARTS * HBOX_BYTES;
   static constexpr int ALPHA_BYTES = VPASS ? 2 * BN * 4 : 0;  // gates of a tile, two tiles
+  // as many h slots (up to 4) as the shared memory left by the operand stages holds
+  static constexpr int HSLOTS_FIT =
+      (232448 - STAGES * (A_BYTES + B_BYTES) - 256 - ALPHA_BYTES) / HSLOT_BYTES;
+  static constexpr int HSLOTS = VPASS ? (HSLOTS_FIT < 4 ? HSLOTS_FIT : 4) : 0;
   static constexpr size_t SMEM = (size_t)STAGES * (A_BYTES + B_BYTES) +
                                  (size_t)HSLOTS * HSLOT_BYTES + 256 + ALPHA_BYTES;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "N tile");
   static_assert(2 * STAGES + 13 <= 30, "barrier area");
   static_assert(SMEM <= 232448, "shared memory");
+  static_assert(!VPASS || HSLOTS >= 2, "h ring");
+  static_assert(PART_COLS % 32 == 0, "parts of whole 32-column chunks");
 };
 
 template <int BN, int STAGES, int MODE>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
     tc_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmO,
                     const __grid_constant__ CUtensorMap tmO29, const __grid_constant__ TcArgs args) {
   using S = TcShape<BN, STAGES, MODE>;
   constexpr bool VPASS = S::VPASS;
+  constexpr int NUM_EPI_WARPS = S::EPI;
+  constexpr int HP_WARP = S::HP_WARP;
+  constexpr int PARTS = S::PARTS;
   constexpr uint32_t STAGE_TX = S::A_BYTES + S::B_BYTES;
   // instruction descriptor: fp32 accumulate, bf16 A and B, both K-major,
   // N >> 3 at bit 17, M >> 4 at bit 24
@@ -391,7 +432,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(drain, 1);
     for (int b = 0; b < S::HSLOTS; ++b) {
       mbar_init(&hfull[b], 1);
-      mbar_init(&hempty[b], 2);  // one release per half, after its output box is stored
+      mbar_init(&hempty[b], PARTS);  // one release per part, after its output box is stored
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -488,7 +529,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == HP_WARP) {
     // ------------------------------------------------------------ h producer (pass V)
     if (VPASS && lane == 0) {
-      constexpr int NCH = (BN / 2) / 32;
+      constexpr int NCH = S::NCHUNK;
       int slot = 0;
       uint32_t ph = 0;
       uint32_t issued = 0;
@@ -503,8 +544,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           mbar_expect_tx(&hfull[slot], S::HSLOT_BYTES);
           uint8_t* dst = hring + slot * S::HSLOT_BYTES;
-          tma_load_2d(dst, &tmH, &hfull[slot], ni * BM, tok0 + c * 32);
-          tma_load_2d(dst + S::HBOX_BYTES, &tmH, &hfull[slot], ni * BM, tok0 + BN / 2 + c * 32);
+#pragma unroll
+          for (int pt = 0; pt < PARTS; ++pt)
+            tma_load_2d(dst + pt * S::HBOX_BYTES, &tmH, &hfull[slot], ni * BM,
+                        tok0 + pt * S::PART_COLS + c * 32);
           ++issued;
           if (++slot == S::HSLOTS) {
             slot = 0;
@@ -522,10 +565,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32 * quad ..
-    const int half = ew >> 2;   // which half of the tile's columns
+    const int part = ew >> 2;   // which part of the tile's columns
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t hslot = 0, hphase = 0;  // pass V: next h ring slot and its phase parity
+    int pending_slot = -1;  // pass V, storing thread: slot whose output store may still read it
     int iter = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
       const int mi = tile / args.num_n_tiles, ni = tile - mi * args.num_n_tiles;
@@ -537,19 +581,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t t_acc = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
 
       if constexpr (!VPASS) {
-        // pass K: this lane's token, half of the tile's features
+        // pass K: this lane's token, one part of the tile's features
         const int64_t n = tok0 + quad * 32 + lane;
         const bool valid = n >= 0 && n < args.N;
-        const int col_base = ni * BN + half * S::HALF_COLS;
-        const uint32_t t_row = t_acc + (uint32_t)(half * S::HALF_COLS);
+        const int col_base = ni * BN + part * S::PART_COLS;
+        const uint32_t t_row = t_acc + (uint32_t)(part * S::PART_COLS);
         {  // pull the next tile's rows of h into L2 while this one is reduced
           const int nxt = tile + (int)gridDim.x;
           if (nxt < num_tiles) {
             const int mi2 = nxt / args.num_n_tiles, ni2 = nxt - mi2 * args.num_n_tiles;
             const int64_t n2 = (int64_t)mi2 * args.m_stride + args.m_offset + quad * 32 + lane;
             if (n2 >= 0 && n2 < args.N) {
-              const __nv_bfloat16* hp2 = args.h + n2 * args.d + ni2 * BN + half * S::HALF_COLS;
-              for (int b = 0; b < S::HALF_COLS * 2; b += 128) prefetch_l2(hp2 + b / 2);
+              const __nv_bfloat16* hp2 = args.h + n2 * args.d + ni2 * BN + part * S::PART_COLS;
+              for (int b = 0; b < S::PART_COLS * 2; b += 128) prefetch_l2(hp2 + b / 2);
             }
           }
         }
@@ -575,14 +619,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        if (valid) args.part[n * args.n_part + ni * 2 + half] = make_float4(kk, hk, hh, 0.f);
+        if (valid) args.part[n * args.n_part + ni * PARTS + part] = make_float4(kk, hk, hh, 0.f);
       } else {
-        // pass V: this lane's feature, half of the tile's tokens.  The causal
+        // pass V: this lane's feature, one part of the tile's tokens.  The causal
         // conv walks the tokens in order with vt of the three previous tokens
         // of the same sequence in registers.
         constexpr bool DECODE = MODE == MODE_VALUE_DECODE;
-        constexpr int HALF_TOK = BN / 2;
-        constexpr int NCH = HALF_TOK / 32;
+        constexpr int NCH = S::NCHUNK;
         const int feat = ni * BM + quad * 32 + lane;
         const int T = args.T;
         // gates of the tile's tokens, staged once by all epilogue warps
@@ -593,12 +636,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         named_bar_sync(1, NUM_EPI_WARPS * 32);
         const float4 w = __ldg(args.conv_w + feat);  // taps: w.x for t-3 .. w.w for t
-        const int j0 = half * HALF_TOK;              // first tile column of this warp
+        const int j0 = part * S::PART_COLS;          // first tile column of this warp
         const int first_out = -args.m_offset;        // halo columns produce no output
         int pos = (int)((((tok0 + j0) % T) + T) % T);  // sequence position of column j0
         float s1 = 0.f, s2 = 0.f, s3 = 0.f;           // vt of tokens t-1, t-2, t-3
         if (!DECODE && j0 > 0) {
-          // the three columns before this half, recomputed from TMEM
+          // the three columns before this part, recomputed from TMEM
           uint32_t u4[16];
           __syncwarp();
           if (got) {
@@ -625,7 +668,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           hgot = __shfl_sync(FULL, hgot, 0);
           // h of token jj and feature f of this box: box[jj * BM + f]; the
           // output of the same element replaces it in place
-          uint8_t* box = hring + hslot * S::HSLOT_BYTES + half * S::HBOX_BYTES;
+          uint8_t* box = hring + hslot * S::HSLOT_BYTES + part * S::HBOX_BYTES;
           uint16_t* hs = reinterpret_cast<uint16_t*>(box) + quad * 32 + lane;
           uint32_t u[16], un[16];
           __syncwarp();
@@ -640,26 +683,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int jb = j0 + c * 32;
           const int64_t nb = tok0 + jb;
           const float4* al4 = reinterpret_cast<const float4*>(al + jb);
-          // no sequence starts inside the chunk: no per-token checks
-          const bool clean = !DECODE && pos + 32 <= T && pos != 0;
+          if (DECODE) {
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (g == 1) {
-              if (got) tmem_wait16(un);
+            for (int g = 0; g < 2; ++g) {
+              if (g == 1 && got) tmem_wait16(un);
 #pragma unroll
-              for (int i = 0; i < 16; ++i) u[i] = un[i];
-            }
+              for (int q = 0; q < 4; ++q) {
+                const float4 a4 = al4[g * 4 + q];
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float4 a4 = al4[g * 4 + q];
-              const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-              for (int r = 0; r < 4; ++r) {
-                const int jj = g * 16 + q * 4 + r;
-                const float vt = av[r] * __uint_as_float(u[q * 4 + r]);
-                float y;
-                if (DECODE) {
+                for (int r = 0; r < 4; ++r) {
+                  const int jj = g * 16 + q * 4 + r;
                   const int64_t n = nb + jj;
+                  const float vt = av[r] * __uint_as_float(g == 0 ? u[q * 4 + r] : un[q * 4 + r]);
                   float a1 = 0.f, a2 = 0.f, a3 = 0.f;
                   if (n < args.N) {
                     float* st = args.conv_state + n * 3 * args.d + feat;
@@ -670,31 +706,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     st[args.d] = a1;
                     st[2 * args.d] = vt;
                   }
-                  y = fmaf(w.x, a3, fmaf(w.y, a2, fmaf(w.z, a1, w.w * vt)));
-                } else {
-                  if (!clean) {
-                    if (pos == 0) s1 = s2 = s3 = 0.f;  // a sequence starts at this token
-                    pos = (pos + 1 == T) ? 0 : pos + 1;
-                  }
-                  y = fmaf(w.x, s3, fmaf(w.y, s2, fmaf(w.z, s1, w.w * vt)));
-                  s3 = s2;
-                  s2 = s1;
-                  s1 = vt;
+                  const float y = fmaf(w.x, a3, fmaf(w.y, a2, fmaf(w.z, a1, w.w * vt)));
+                  const float hv = __uint_as_float(((uint32_t)hs[jj * BM]) << 16);
+                  const float o = hv + vt + __fdividef(y, 1.0f + __expf(-y));
+                  hs[jj * BM] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
                 }
-                const float hv = __uint_as_float(((uint32_t)hs[jj * BM]) << 16);
-                const float o = hv + vt + __fdividef(y, 1.0f + __expf(-y));  // h + vt + SiLU(y)
-                hs[jj * BM] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
               }
             }
-          }
-          if (clean) {
+          } else if (pos + 32 <= T && pos != 0) {
+            // no sequence starts inside the chunk: no per-token checks
+            conv_group16<false>(u, al4, hs, w, s1, s2, s3, pos, T);
+            if (got) tmem_wait16(un);
+            conv_group16<false>(un, al4 + 4, hs + 16 * BM, w, s1, s2, s3, pos, T);
             pos += 32;
             if (pos == T) pos = 0;
+          } else {
+            conv_group16<true>(u, al4, hs, w, s1, s2, s3, pos, T);
+            if (got) tmem_wait16(un);
+            conv_group16<true>(un, al4 + 4, hs + 16 * BM, w, s1, s2, s3, pos, T);
           }
-          // the half's four warps have written the box: one thread stores it
+          // the part's four warps have written the box: one thread stores it
           fence_async_shared();
-          named_bar_sync(2 + half, 128);
-          if (ew == half * 4 && lane == 0) {
+          named_bar_sync(2 + part, 128);
+          if (ew == part * 4 && lane == 0) {
             if (hgot && got) {
               if (jb < first_out) {
                 // the first tokens of the tile are the conv halo of the
@@ -703,9 +737,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               } else {
                 tma_store_2d(&tmO, box, ni * BM, (int)nb);
               }
-              tma_store_wait_read();
+            } else {
+              asm volatile("cp.async.bulk.commit_group;" ::: "memory");  // keep one group per chunk
             }
-            mbar_arrive(&hempty[hslot]);
+            // the previous chunk's store has read its box: release that slot
+            // (this one is released after the next chunk, off the critical path)
+            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            if (pending_slot >= 0) mbar_arrive(&hempty[pending_slot]);
+            pending_slot = (int)hslot;
           }
           if (++hslot == (uint32_t)S::HSLOTS) {
             hslot = 0;
@@ -720,7 +759,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (acc == 0) acc_phase ^= 1u;
     }
     // output boxes of pass V fully written before the CTA exits
-    if (VPASS && ew == half * 4 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (VPASS && ew == part * 4 && lane == 0) {
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+      if (pending_slot >= 0) mbar_arrive(&hempty[pending_slot]);
+    }
   }
 
   __syncthreads();
@@ -809,7 +851,7 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   const int tiles = a.num_m_tiles * a.num_n_tiles;
   const int grid = tiles < sms ? tiles : sms;
   if (grid <= 0) return ENGRAM_OK;
-  kern<<<grid, NUM_THREADS, S::SMEM, s>>>(ta, tb, th, to, to29, a);
+  kern<<<grid, S::NUM_THREADS, S::SMEM, s>>>(ta, tb, th, to, to29, a);
   return ck(cudaGetLastError());
 }
 
@@ -839,7 +881,7 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.N = N;
   a.T = T;
   a.d = d;
-  a.n_part = 2 * (d / BN);
+  a.n_part = TcShape<BN, STAGES_K, MODE_GATE_PARTIAL>::PARTS * (d / BN);
   a.h = h;
   a.out = out;
   a.part = part;

@@ -89,10 +89,10 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HeadP
   }
 }
 
-// Row gather with 16-byte vectors.  The e row of a token is J*CR chunks of 16
-// bytes (CR per head row); consecutive threads take consecutive chunks, so the
-// stores are fully coalesced and each head row is read as CR adjacent
-// vectors.  Every thread keeps UNROLL loads in flight before storing.
+// Row gather with 16-byte vectors, generic shape.  The e row of a token is
+// J*CR chunks of 16 bytes (CR per head row); consecutive threads take
+// consecutive chunks, so the stores are fully coalesced.  Every thread keeps
+// UNROLL loads in flight before storing.
 template <int UNROLL>
 __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ HeadParams hp,
                                                      const int32_t* __restrict__ idx,
@@ -131,6 +131,64 @@ __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ Hea
   }
 }
 
+// Row gather for head count JH and head-row width CR (16-byte pieces) fixed
+// at compile time.  One warp takes TPW tokens at a time: lanes 0..JH-1 read
+// the tokens' slots (one coalesced read per token) and pass them by
+// shuffles; then every lane loads its pieces of all TPW tokens' rows
+// (TPW * JH * CR / 32 loads in flight per lane) before storing them,
+// consecutive lanes on consecutive pieces of e.
+template <int JH, int CR, int TPW>
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant__ HeadParams hp,
+                                                          const int32_t* __restrict__ idx,
+                                                          const uint4* __restrict__ table,
+                                                          int64_t n_tok,
+                                                          uint4* __restrict__ e,
+                                                          unsigned int* status) {
+  constexpr int PER_TOK = JH * CR;             // pieces per token
+  constexpr int PER_LANE = (PER_TOK + 31) / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t t0 = warp * TPW; t0 < n_tok; t0 += nwarps * TPW) {
+    int32_t slot[TPW];
+#pragma unroll
+    for (int k = 0; k < TPW; ++k) {
+      const int64_t n = t0 + k;
+      slot[k] = (lane < JH && n < n_tok) ? __ldg(idx + n * JH + lane) : -1;
+    }
+    uint4 v[TPW][PER_LANE];
+#pragma unroll
+    for (int k = 0; k < TPW; ++k) {
+#pragma unroll
+      for (int p = 0; p < PER_LANE; ++p) {
+        const int piece = p * 32 + lane;
+        const int j = piece / CR;  // head of this piece (>= JH past the row's end)
+        const int c = piece - j * CR;
+        const int32_t s = __shfl_sync(FULL, slot[k], j < JH ? j : 0);
+        v[k][p] = make_uint4(0, 0, 0, 0);
+        if (piece < PER_TOK) {
+          if (s >= 0 && (uint64_t)s < hp.P[j]) {
+            v[k][p] = __ldg(table + (hp.row_base[j] + s) * CR + c);
+          } else if (s != -1) {
+            atomicOr(status, ENGRAM_STATUS_BAD_INDEX);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < TPW; ++k) {
+      const int64_t n = t0 + k;
+      if (n < n_tok) {
+#pragma unroll
+        for (int p = 0; p < PER_LANE; ++p) {
+          const int piece = p * 32 + lane;
+          if (piece < PER_TOK) e[n * PER_TOK + piece] = v[k][p];
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
 
 int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, int B, int T,
@@ -148,19 +206,36 @@ int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, i
                   int elem_bytes, void* e, cudaStream_t s) {
   if (n_tok == 0) return ENGRAM_OK;
   const int CR = hp.D_h * elem_bytes / 16;
-  const int64_t total = n_tok * hp.J * CR;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  constexpr int UNROLL = 8;
+  const uint4* tb = static_cast<const uint4*>(table);
+  uint4* eo = static_cast<uint4*>(e);
+  unsigned int* st = status_ptr();
   const int threads = 256;
+  auto rows = [&](auto kern, int tpw) {
+    const int64_t warps = (n_tok + tpw - 1) / tpw;
+    int64_t blocks = (warps * 32 + threads - 1) / threads;
+    const int64_t cap = (int64_t)sms * 8;  // 8 resident blocks of 256 threads per SM
+    if (blocks > cap) blocks = cap;
+    kern<<<(unsigned)blocks, threads, 0, s>>>(hp, idx, tb, n_tok, eo, st);
+    return ck(cudaGetLastError());
+  };
+  const int key = hp.J * 100 + CR;
+  switch (key) {
+    case 4 * 100 + 4: return rows(gather_rows_kernel<4, 4, 8>, 8);     // fp32 rows of 16, 4 heads
+    case 16 * 100 + 10: return rows(gather_rows_kernel<16, 10, 4>, 4);  // bf16 rows of 80
+    case 16 * 100 + 16: return rows(gather_rows_kernel<16, 16, 2>, 2);  // bf16 rows of 128
+    case 16 * 100 + 20: return rows(gather_rows_kernel<16, 20, 2>, 2);  // bf16 rows of 160
+    default: break;
+  }
+  constexpr int UNROLL = 8;
+  const int64_t total = n_tok * hp.J * CR;
   int64_t blocks = (total + (int64_t)threads * UNROLL - 1) / ((int64_t)threads * UNROLL);
-  const int64_t cap = (int64_t)sms * 8;  // 8 resident blocks of 256 threads per SM
+  const int64_t cap = (int64_t)sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  gather_kernel<UNROLL><<<(unsigned)blocks, threads, 0, s>>>(
-      hp, idx, static_cast<const uint4*>(table), n_tok, CR, static_cast<uint4*>(e),
-      status_ptr());
+  gather_kernel<UNROLL><<<(unsigned)blocks, threads, 0, s>>>(hp, idx, tb, n_tok, CR, eo, st);
   return ck(cudaGetLastError());
 }
 
