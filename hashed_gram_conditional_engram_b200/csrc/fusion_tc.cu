@@ -184,41 +184,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(slot)),
-               "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane.
@@ -269,6 +239,83 @@ __device__ __forceinline__ void tmem_wait16(uint32_t (&u)[16]) {
                  "+r"(u[6]), "+r"(u[7]), "+r"(u[8]), "+r"(u[9]), "+r"(u[10]), "+r"(u[11]),
                  "+r"(u[12]), "+r"(u[13]), "+r"(u[14]), "+r"(u[15])
                :
+               : "memory");
+}
+
+// ---- CTA pairs (a cluster of 2 runs one M = 256 MMA over both SMs)
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on the
+// pair's leader barrier (cluster address); no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// arrive on the barrier at this offset in both CTAs of the pair once the
+// issued MMAs complete
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair_self(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
                : "memory");
 }
 
@@ -337,8 +384,10 @@ struct TcShape {
   static constexpr int PARTS = EPI / 4;        // column parts of a tile, one per warp of a quadrant
   static constexpr int HP_WARP = 2 + EPI;      // pass V: warp that streams h in by TMA
   static constexpr int NUM_THREADS = 64 + EPI * 32 + 32;
+  // a CTA pair computes a (2 * BM) x BN tile: each CTA loads its BM rows of
+  // A and half of the BN rows of B, and holds its BM rows of the accumulator
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;
   static constexpr int TMEM_COLS = 2 * BN;
   // pass K (tokens on TMEM lanes, features on columns): each epilogue warp
   // takes one part of the tile's columns, 32 at a time
@@ -364,7 +413,7 @@ struct TcShape {
 };
 
 template <int BN, int STAGES, int MODE>
-__global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
     tc_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmO,
                     const __grid_constant__ CUtensorMap tmO29, const __grid_constant__ TcArgs args) {
@@ -375,9 +424,9 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
   constexpr int PARTS = S::PARTS;
   constexpr uint32_t STAGE_TX = S::A_BYTES + S::B_BYTES;
   // instruction descriptor: fp32 accumulate, bf16 A and B, both K-major,
-  // N >> 3 at bit 17, M >> 4 at bit 24
+  // N >> 3 at bit 17, M >> 4 at bit 24 (M = 256 over the CTA pair)
   constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                             ((uint32_t)(BM >> 4) << 24);
+                             ((uint32_t)((2 * BM) >> 4) << 24);
 
   // The kernel declares no static shared memory, so the dynamic block starts
   // at the base of the CTA's window.  Addressing everything from the
@@ -404,19 +453,24 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_tiles = args.num_m_tiles * args.num_n_tiles;
+  // CTA pair: rank 0 (the leader) issues the MMAs for both
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = (int)(blockIdx.x >> 1), num_pairs = (int)(gridDim.x >> 1);
 
   // Tile t covers token block t / num_n_tiles and feature block
-  // t % num_n_tiles.  Pass K multiplies e (tokens, A) by W_k (features, B);
-  // pass V multiplies W_v (features, A) by e (tokens, B).
+  // t % num_n_tiles.  Pass K multiplies e (256 tokens, A) by W_k (BN
+  // features, B); pass V multiplies W_v (256 features, A) by e (BN tokens,
+  // B).  This CTA loads its 128 rows of A and its half of B.
   auto operand_rows = [&](int tile, int& arow, int& brow) {
     const int mi = tile / args.num_n_tiles, ni = tile - mi * args.num_n_tiles;
     const int tok0 = mi * args.m_stride + args.m_offset;
     if (VPASS) {
-      arow = ni * BM;
-      brow = tok0;
+      arow = ni * (2 * BM) + (int)rank * BM;
+      brow = tok0 + (int)rank * (BN / 2);
     } else {
-      arow = tok0;
-      brow = ni * BN;
+      arow = tok0 + (int)rank * BM;
+      brow = ni * BN + (int)rank * (BN / 2);
     }
   };
 
@@ -427,7 +481,7 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], NUM_EPI_WARPS);
+      mbar_init(&tempty[a], 2 * NUM_EPI_WARPS);  // epilogue warps of both CTAs
     }
     mbar_init(drain, 1);
     for (int b = 0; b < S::HSLOTS; ++b) {
@@ -447,10 +501,11 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
   }
   if (warp == 1) {
     __syncwarp();
-    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
   }
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -460,7 +515,7 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int tile = pair; tile < num_tiles; tile += num_pairs) {
         int arow, brow;
         operand_rows(tile, arow, brow);
         bool ok = true;
@@ -469,9 +524,11 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
             ok = false;
             break;
           }
-          mbar_expect_tx(&full[stage], STAGE_TX);
-          tma_load_2d(sA + stage * S::A_BYTES, &tmA, &full[stage], kt * BK, arow);
-          tma_load_2d(sB + stage * S::B_BYTES, &tmB, &full[stage], kt * BK, brow);
+          // the leader's full barrier counts the bytes of both CTAs
+          if (leader) mbar_expect_tx(&full[stage], 2 * STAGE_TX);
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          tma_load_2d_pair(sA + stage * S::A_BYTES, &tmA, fb, kt * BK, arow);
+          tma_load_2d_pair(sB + stage * S::B_BYTES, &tmB, fb, kt * BK, brow);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -480,21 +537,24 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
         }
         if (!ok) break;
       }
-      // every issued copy must land before the CTA exits
-      for (int s = 0; s < STAGES; ++s) {
-        const uint32_t n_s = issued > (uint32_t)s ? (issued - 1 - s) / STAGES + 1 : 0;
-        if (n_s > 0) wait_drain(&full[s], (n_s - 1) & 1u);
+      // every issued copy of the pair lands before the leader leaves (the
+      // peer waits for the leader at the closing cluster barrier)
+      if (leader) {
+        for (int s = 0; s < STAGES; ++s) {
+          const uint32_t n_s = issued > (uint32_t)s ? (issued - 1 - s) / STAGES + 1 : 0;
+          if (n_s > 0) wait_drain(&full[s], (n_s - 1) & 1u);
+        }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -508,22 +568,22 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
           const uint32_t b0 = smem_u32(sB + stage * S::B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
-            umma_bf16(d_tmem, sw128_desc(a0 + k * UMMA_K * 2), sw128_desc(b0 + k * UMMA_K * 2),
-                      IDESC, (kt | k) != 0 ? 1u : 0u);
+            umma_bf16_pair(d_tmem, sw128_desc(a0 + k * UMMA_K * 2),
+                           sw128_desc(b0 + k * UMMA_K * 2), IDESC, (kt | k) != 0 ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);
+          umma_commit_pair_both(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        umma_commit_pair_both(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       // all issued MMAs complete before TMEM is released
-      umma_commit(drain);
+      umma_commit_pair_self(drain);
       wait_drain(drain, 0);
     }
   } else if (warp == HP_WARP) {
@@ -533,9 +593,10 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
       int slot = 0;
       uint32_t ph = 0;
       uint32_t issued = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int tile = pair; tile < num_tiles; tile += num_pairs) {
         const int mi = tile / args.num_n_tiles, ni = tile - mi * args.num_n_tiles;
         const int tok0 = mi * args.m_stride + args.m_offset;
+        const int f0 = ni * (2 * BM) + (int)rank * BM;  // this CTA's features
         bool ok = true;
         for (int c = 0; c < NCH; ++c) {
           if (!wait_bounded(&hempty[slot], ph ^ 1u, abort_flag, args.status)) {
@@ -546,7 +607,7 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
           uint8_t* dst = hring + slot * S::HSLOT_BYTES;
 #pragma unroll
           for (int pt = 0; pt < PARTS; ++pt)
-            tma_load_2d(dst + pt * S::HBOX_BYTES, &tmH, &hfull[slot], ni * BM,
+            tma_load_2d(dst + pt * S::HBOX_BYTES, &tmH, &hfull[slot], f0,
                         tok0 + pt * S::PART_COLS + c * 32);
           ++issued;
           if (++slot == S::HSLOTS) {
@@ -571,7 +632,7 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
     uint32_t hslot = 0, hphase = 0;  // pass V: next h ring slot and its phase parity
     int pending_slot = -1;  // pass V, storing thread: slot whose output store may still read it
     int iter = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++iter) {
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++iter) {
       const int mi = tile / args.num_n_tiles, ni = tile - mi * args.num_n_tiles;
       const int64_t tok0 = (int64_t)mi * args.m_stride + args.m_offset;
       int got = 0;
@@ -582,15 +643,16 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
 
       if constexpr (!VPASS) {
         // pass K: this lane's token, one part of the tile's features
-        const int64_t n = tok0 + quad * 32 + lane;
+        const int64_t n = tok0 + (int)rank * BM + quad * 32 + lane;
         const bool valid = n >= 0 && n < args.N;
         const int col_base = ni * BN + part * S::PART_COLS;
         const uint32_t t_row = t_acc + (uint32_t)(part * S::PART_COLS);
         {  // pull the next tile's rows of h into L2 while this one is reduced
-          const int nxt = tile + (int)gridDim.x;
+          const int nxt = tile + num_pairs;
           if (nxt < num_tiles) {
             const int mi2 = nxt / args.num_n_tiles, ni2 = nxt - mi2 * args.num_n_tiles;
-            const int64_t n2 = (int64_t)mi2 * args.m_stride + args.m_offset + quad * 32 + lane;
+            const int64_t n2 = (int64_t)mi2 * args.m_stride + args.m_offset + (int)rank * BM +
+                               quad * 32 + lane;
             if (n2 >= 0 && n2 < args.N) {
               const __nv_bfloat16* hp2 = args.h + n2 * args.d + ni2 * BN + part * S::PART_COLS;
               for (int b = 0; b < S::PART_COLS * 2; b += 128) prefetch_l2(hp2 + b / 2);
@@ -626,7 +688,8 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
         // of the same sequence in registers.
         constexpr bool DECODE = MODE == MODE_VALUE_DECODE;
         constexpr int NCH = S::NCHUNK;
-        const int feat = ni * BM + quad * 32 + lane;
+        const int f0 = ni * (2 * BM) + (int)rank * BM;  // this CTA's features
+        const int feat = f0 + quad * 32 + lane;
         const int T = args.T;
         // gates of the tile's tokens, staged once by all epilogue warps
         float* al = alpha_s + (iter & 1) * BN;
@@ -733,9 +796,9 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
               if (jb < first_out) {
                 // the first tokens of the tile are the conv halo of the
                 // previous tile: store from the first output token on
-                tma_store_2d(&tmO29, box + first_out * BM * 2, ni * BM, (int)(nb + first_out));
+                tma_store_2d(&tmO29, box + first_out * BM * 2, f0, (int)(nb + first_out));
               } else {
-                tma_store_2d(&tmO, box, ni * BM, (int)nb);
+                tma_store_2d(&tmO, box, f0, (int)nb);
               }
             } else {
               asm volatile("cp.async.bulk.commit_group;" ::: "memory");  // keep one group per chunk
@@ -754,7 +817,8 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      // this CTA's accumulator rows are read: release them to the leader's MMA
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -765,11 +829,13 @@ __global__ void __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
     }
   }
 
-  __syncthreads();
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();  // the pair's MMAs, loads and reads are all done
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, S::TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
   }
 }
 
@@ -848,10 +914,11 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   }
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // one CTA pair per two SMs, each pair walking its tiles
   const int tiles = a.num_m_tiles * a.num_n_tiles;
-  const int grid = tiles < sms ? tiles : sms;
-  if (grid <= 0) return ENGRAM_OK;
-  kern<<<grid, S::NUM_THREADS, S::SMEM, s>>>(ta, tb, th, to, to29, a);
+  const int pairs = tiles < sms / 2 ? tiles : sms / 2;
+  if (pairs <= 0) return ENGRAM_OK;
+  kern<<<2 * pairs, S::NUM_THREADS, S::SMEM, s>>>(ta, tb, th, to, to29, a);
   return ck(cudaGetLastError());
 }
 
@@ -861,14 +928,15 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
               float* alpha_saved, int64_t N, int T, int d, int E, float4* part, float* alpha,
               cudaStream_t s) {
   const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
-  // pass K: A = e (128 tokens per tile), B = W_k (BN features per tile)
+  // Each CTA of a pair loads 128 rows of A and BN/2 rows of B per stage.
+  // pass K: A = e (256 tokens per pair tile), B = W_k (BN features)
   CUtensorMap ta_k, tb_k, ta_v, tb_v, th, to, to29;
   if (!make_tmap(&ta_k, e, (uint64_t)E, (uint64_t)N, BK, BM, sw128)) return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&tb_k, Wk, (uint64_t)E, (uint64_t)d, BK, BN, sw128)) return ENGRAM_ERR_CUDA;
-  // pass V: A = W_v (128 features per tile), B = e (BN tokens per tile);
+  if (!make_tmap(&tb_k, Wk, (uint64_t)E, (uint64_t)d, BK, BN / 2, sw128)) return ENGRAM_ERR_CUDA;
+  // pass V: A = W_v (256 features per pair tile), B = e (BN tokens);
   // h in boxes of 32 tokens x 128 features
   if (!make_tmap(&ta_v, Wv, (uint64_t)E, (uint64_t)d, BK, BM, sw128)) return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&tb_v, e, (uint64_t)E, (uint64_t)N, BK, BN, sw128)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap(&tb_v, e, (uint64_t)E, (uint64_t)N, BK, BN / 2, sw128)) return ENGRAM_ERR_CUDA;
   if (!make_tmap(&th, h, (uint64_t)d, (uint64_t)N, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ENGRAM_ERR_CUDA;
   // out in the same boxes; a 29-token box skips the 3 halo tokens of a tile
@@ -890,19 +958,19 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.alpha_out = alpha_saved;
   a.alpha = nullptr;
   a.status = status_ptr();
-  // pass K: gate partials, tiles of 128 tokens x BN features
+  // pass K: gate partials, pair tiles of 256 tokens x BN features
   a.num_n_tiles = d / BN;
-  a.m_stride = BM;
+  a.m_stride = 2 * BM;
   a.m_offset = 0;
-  a.num_m_tiles = (int)((N + BM - 1) / BM);
+  a.num_m_tiles = (int)((N + 2 * BM - 1) / (2 * BM));
   int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL>(ta_k, tb_k, th, to, to29, a, s);
   if (rc) return rc;
   gate_from_partials_kernel<<<(unsigned)((N + 255) / 256), 256, 0, s>>>(part, a.n_part, N, d,
                                                                         alpha, alpha_saved);
   a.alpha = alpha;
-  // pass V: tiles of 128 features x BN tokens.  Whole sequences: the token
-  // tiles overlap by 3 (the conv halo, recomputed); decode: plain tiles.
-  a.num_n_tiles = d / BM;
+  // pass V: pair tiles of 256 features x BN tokens.  Whole sequences: the
+  // token tiles overlap by 3 (the conv halo, recomputed); decode: plain tiles.
+  a.num_n_tiles = d / (2 * BM);
   if (conv_state != nullptr) {
     a.m_stride = BN;
     a.m_offset = 0;
@@ -921,7 +989,7 @@ inline bool use_wide(int64_t N, int d) { return d % 256 == 0 && N > 4096; }
 }  // namespace
 
 int tc_supported(int d, int E, int M) {
-  return M == 1 && E % BK == 0 && E >= BK && d % BM == 0 && d >= BM;
+  return M == 1 && E % BK == 0 && E >= BK && d % (2 * BM) == 0 && d >= 2 * BM;
 }
 
 size_t tc_forward_ws_bytes(int64_t N, int d, int E) {
@@ -943,10 +1011,10 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
   float* alpha = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                           (size_t)N * 2 * (d / BN) * sizeof(float4));
   if (wide)
-    return run_layer<256, 4, 3>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
-                             alpha, s);
+    return run_layer<256, 6, 5>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
+                                alpha, s);
   return run_layer<64, 8, 6>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
-                          alpha, s);
+                             alpha, s);
 }
 
 }  // namespace engram

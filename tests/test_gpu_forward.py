@@ -104,9 +104,9 @@ def _bf16_unit_case(B, T, d, K, D_h, seed, rows=None, decode_steps=0):
 
 
 @pytest.mark.parametrize("B,T,d,K,D_h", [
-    (3, 100, 256, 2, 32),      # narrow tiles (N=64), ragged last M tile
-    (1, 1, 128, 2, 32),        # a single token
-    (4, 2, 128, 2, 16),        # every token within the conv's start-up
+    (3, 100, 256, 2, 32),      # narrow tiles (N=64), ragged last tile
+    (1, 1, 256, 2, 32),        # a single token
+    (4, 2, 256, 2, 16),        # every token within the conv's start-up
     (2, 2500, 512, 2, 32),     # wide tiles (N=256), 40 overlapping V tiles of 125
     (1, 4100, 256, 4, 16),     # wide tiles with several sequences per tile boundary
 ])
@@ -226,8 +226,11 @@ def test_forward_layer27b_sampled():
     base = np.concatenate([[0], np.cumsum(w.rows)[:-1]])
     rng = np.random.default_rng(1)
     sample = set(rng.choice(w.N, size=96, replace=False).tolist())
-    sample |= {0, 1, 2, 3, 124, 125, 126, 127, 128, 129, 249, 250, 4095, 4096, 4097, 4098,
-               w.N - 1, w.N - 2, 125 * 262, 125 * 262 - 1}
+    # sequence starts, and the seams of both passes' tiles (pass K: 256-token
+    # pair tiles; pass V: 256-token tiles advancing by 253 with a 3-token halo)
+    sample |= {0, 1, 2, 3, 124, 125, 126, 127, 128, 129, 249, 250, 251, 252, 253, 254, 255, 256,
+               257, 502, 503, 505, 506, 507, 4095, 4096, 4097, 4098, w.N - 1, w.N - 2,
+               253 * 129, 253 * 129 - 1, 253 * 129 + 2, 253 * 129 + 3}
     errs, aerrs = [], []
     for n in sorted(sample):
         p = n % w.T
