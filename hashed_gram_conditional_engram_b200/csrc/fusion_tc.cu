@@ -319,6 +319,17 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
                : "memory");
 }
 
+// Programmatic dependent launch: the next kernel in the stream may start
+// once every CTA of this one has signalled; wait_prior_grid blocks until the
+// kernel launched before this one has completed and its writes are visible
+// (a no-op when this kernel was launched without the attribute).
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -508,6 +519,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
   cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Pass K reads e, written by the gather launched just before it: wait for
+  // it after the set-up above, then let the gate and pass V launch.  Pass V
+  // starts its operand loads and MMAs at once (e is complete by then) and
+  // waits for the gate only where its epilogue first reads alpha.
+  if (!VPASS) wait_prior_grid();
+  allow_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ operand producer
@@ -691,6 +708,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
         const int f0 = ni * (2 * BM) + (int)rank * BM;  // this CTA's features
         const int feat = f0 + quad * 32 + lane;
         const int T = args.T;
+        if (iter == 0) wait_prior_grid();  // alpha comes from the gate kernel
         // gates of the tile's tokens, staged once by all epilogue warps
         float* al = alpha_s + (iter & 1) * BN;
         for (int i = ew * 32 + lane; i < BN; i += NUM_EPI_WARPS * 32) {
@@ -845,6 +863,8 @@ __global__ void __launch_bounds__(256) gate_from_partials_kernel(const float4* _
                                                                  int n_part, int64_t N, int d,
                                                                  float* __restrict__ alpha,
                                                                  float* __restrict__ alpha_copy) {
+  allow_dependents();
+  wait_prior_grid();  // the partials of pass K
   const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
   const float4* pr = part + n * n_part;
@@ -918,8 +938,17 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   const int tiles = a.num_m_tiles * a.num_n_tiles;
   const int pairs = tiles < sms / 2 ? tiles : sms / 2;
   if (pairs <= 0) return ENGRAM_OK;
-  kern<<<2 * pairs, S::NUM_THREADS, S::SMEM, s>>>(ta, tb, th, to, to29, a);
-  return ck(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(S::NUM_THREADS);
+  cfg.dynamicSmemBytes = S::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return ck(cudaLaunchKernelEx(&cfg, kern, ta, tb, th, to, to29, a));
 }
 
 template <int BN, int STAGES_K, int STAGES_V>
@@ -965,8 +994,20 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.num_m_tiles = (int)((N + 2 * BM - 1) / (2 * BM));
   int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL>(ta_k, tb_k, th, to, to29, a, s);
   if (rc) return rc;
-  gate_from_partials_kernel<<<(unsigned)((N + 255) / 256), 256, 0, s>>>(part, a.n_part, N, d,
-                                                                        alpha, alpha_saved);
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((N + 255) / 256));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    rc = ck(cudaLaunchKernelEx(&cfg, gate_from_partials_kernel, (const float4*)part, a.n_part, N,
+                               d, alpha, alpha_saved));
+    if (rc) return rc;
+  }
   a.alpha = alpha;
   // pass V: pair tiles of 256 features x BN tokens.  Whole sequences: the
   // token tiles overlap by 3 (the conv halo, recomputed); decode: plain tiles.

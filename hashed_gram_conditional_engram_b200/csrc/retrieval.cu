@@ -33,60 +33,66 @@ __device__ __forceinline__ int32_t token_cid(const int32_t* __restrict__ proj,
   return __ldg(proj + x);
 }
 
-// One thread per token in flat order.  c_{t-1} and c_{t-2} travel from the
-// neighbouring lanes by warp shuffles; lanes 0 and 1 fetch the two tokens
-// before the warp themselves.
+// TPT threads per token (J / 4 rounded up to a power of two), four heads
+// each; a warp covers 32 / TPT consecutive tokens in flat order.  c_{t-1} and c_{t-2}
+// travel from the lanes of the previous tokens by warp shuffles; the lanes of
+// a warp's first two tokens fetch the tokens before the warp themselves.
 __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HeadParams hp,
                                                    const int32_t* __restrict__ proj,
                                                    const int32_t* __restrict__ ids, int64_t N,
-                                                   int T, int32_t* __restrict__ ngram_state,
+                                                   int T, int tpt,
+                                                   int32_t* __restrict__ ngram_state,
                                                    int32_t* __restrict__ idx,
                                                    unsigned int* status) {
-  const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
+  const int q = lane % tpt;             // which four heads
+  const int64_t n = gt / tpt;           // token
   const int32_t pad = hp.V_c;
   const bool live = n < N;
 
   int32_t c0 = live ? token_cid(proj, ids, n, hp.V_raw, pad) : pad;
-  int32_t c1 = __shfl_up_sync(FULL, c0, 1);
-  int32_t c2 = __shfl_up_sync(FULL, c0, 2);
+  int32_t c1 = __shfl_up_sync(FULL, c0, tpt);
+  int32_t c2 = __shfl_up_sync(FULL, c0, 2 * tpt);
   if (!live) return;
-  if (lane == 0) c1 = token_cid(proj, ids, n - 1, hp.V_raw, pad);
-  if (lane <= 1) c2 = token_cid(proj, ids, n - 2, hp.V_raw, pad);
+  const int tk = lane / tpt;            // token index within the warp
+  if (tk == 0) c1 = token_cid(proj, ids, n - 1, hp.V_raw, pad);
+  if (tk <= 1) c2 = token_cid(proj, ids, n - 2, hp.V_raw, pad);
 
   if (ngram_state != nullptr) {
     // decode: one token per sequence, history from the rolling state
     c1 = ngram_state[2 * n + 0];
     c2 = ngram_state[2 * n + 1];
-    ngram_state[2 * n + 0] = c0;
-    ngram_state[2 * n + 1] = c1;
+    __syncwarp(__activemask());
+    if (q == 0) {
+      ngram_state[2 * n + 0] = c0;
+      ngram_state[2 * n + 1] = c1;
+    }
   } else {
     const int t = (int)(n % T);
     if (t < 1) c1 = pad;
     if (t < 2) c2 = pad;
   }
-  if (c0 < 0) atomicOr(status, ENGRAM_STATUS_BAD_ID);
+  if (c0 < 0 && q == 0) atomicOr(status, ENGRAM_STATUS_BAD_ID);
   const bool bad2 = (c0 < 0) | (c1 < 0);
   const bool bad3 = bad2 | (c2 < 0);
 
   const uint64_t g0 = (uint64_t)(uint32_t)c0, g1 = (uint64_t)(uint32_t)c1,
                  g2 = (uint64_t)(uint32_t)c2;
-  int32_t* dst = idx + n * hp.J;
-  // J is a multiple of 4 (host check): 16-byte stores of four slots
-  for (int j0 = 0; j0 < hp.J; j0 += 4) {
-    int32_t s[4];
+  const int j0 = 4 * q;
+  if (j0 >= hp.J) return;  // padding lane of a token (J / 4 not a power of two)
+  int32_t s[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = j0 + u;
-      uint64_t x = g0 * hp.mult[j][0];
-      x ^= g1 * hp.mult[j][1];
-      const bool tri = j >= hp.K;
-      if (tri) x ^= g2 * hp.mult[j][2];
-      const bool bad = tri ? bad3 : bad2;
-      s[u] = bad ? -1 : (int32_t)mod_prime(x, hp.P[j], hp.mu[j]);
-    }
-    *reinterpret_cast<int4*>(dst + j0) = make_int4(s[0], s[1], s[2], s[3]);
+  for (int u = 0; u < 4; ++u) {
+    const int j = j0 + u;
+    uint64_t x = g0 * hp.mult[j][0];
+    x ^= g1 * hp.mult[j][1];
+    const bool tri = j >= hp.K;
+    if (tri) x ^= g2 * hp.mult[j][2];
+    const bool bad = tri ? bad3 : bad2;
+    s[u] = bad ? -1 : (int32_t)mod_prime(x, hp.P[j], hp.mu[j]);
   }
+  *reinterpret_cast<int4*>(idx + n * hp.J + j0) = make_int4(s[0], s[1], s[2], s[3]);
 }
 
 // Row gather with 16-byte vectors, generic shape.  The e row of a token is
@@ -195,9 +201,13 @@ int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, i
                 int32_t* ngram_state, int32_t* idx, cudaStream_t s) {
   const int64_t N = (int64_t)B * T;
   if (N == 0) return ENGRAM_OK;
+  // threads per token: J / 4 (four heads each) rounded up to a power of two
+  int tpt = 1;
+  while (tpt < hp.J / 4) tpt *= 2;
   const int threads = 256;
-  const int64_t blocks = (N + threads - 1) / threads;
-  hash_kernel<<<(unsigned)blocks, threads, 0, s>>>(hp, proj, ids, N, T, ngram_state, idx,
+  const int64_t total = N * tpt;
+  const int64_t blocks = (total + threads - 1) / threads;
+  hash_kernel<<<(unsigned)blocks, threads, 0, s>>>(hp, proj, ids, N, T, tpt, ngram_state, idx,
                                                    status_ptr());
   return ck(cudaGetLastError());
 }

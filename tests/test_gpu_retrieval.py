@@ -193,3 +193,23 @@ def test_gather_full_size_sampled():
         assert np.array_equal(bf16_bits(e[n]), want), n
     del table
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 6, 8, 10, 16])
+def test_hash_head_counts(K):
+    """Every head count the configuration allows (J = 2K a multiple of 4 up to
+    32, several heads per thread), on a ragged batch."""
+    if (2 * K) % 4:
+        pytest.skip("J must be a multiple of 4")
+    w = synth.workload("tiny")
+    inp = synth.host_inputs(w)
+    proj_ref, V_c = O.build_vocab_proj(inp["keys"])
+    B, T = 3, 45
+    ids = np.random.default_rng(K).integers(0, w.V, size=(B, T)).astype(np.int32)
+    mult = synth.hash_multipliers(100 + K, 2 * K)
+    rows = np.array(synth.primes_at_most(10007, 2 * K), dtype=np.int64)
+    want = O.hash_indices(proj_ref, ids, mult, rows, K, V_c)
+    proj, _ = gpu_vocab_proj(inp["keys"])
+    cfg = eg.make_cfg(K, 16, 64, 1, w.V, V_c, eg.F32, rows, mult)
+    got = gpu_hash(cfg, proj, dev(ids), B, T)
+    assert np.array_equal(got.cpu().numpy(), want)
