@@ -205,8 +205,14 @@ def engram_table_grad_noalloc(cfg: EngramCfg, idx, de, n_tok: int, dtab_keys, dt
 
 def engram_forward_hosttable(cfg: EngramCfg, idx, host_table, n_tok: int, e, side_stream=None,
                              done_event=None) -> None:
-    ev = None if done_event is None else (done_event if isinstance(done_event, int)
-                                          else done_event.cuda_event)
+    ev = None
+    if isinstance(done_event, int):
+        ev = done_event
+    elif done_event is not None:
+        # a torch.cuda.Event creates its CUDA event on first record only
+        if done_event.cuda_event == 0:
+            done_event.record(side_stream)
+        ev = done_event.cuda_event
     _check("engram_forward_hosttable",
            lib().engram_forward_hosttable(ctypes.byref(cfg), _p(idx), _p(host_table), n_tok, _p(e),
                                           _s(side_stream), ev))

@@ -213,3 +213,39 @@ def test_hash_head_counts(K):
     cfg = eg.make_cfg(K, 16, 64, 1, w.V, V_c, eg.F32, rows, mult)
     got = gpu_hash(cfg, proj, dev(ids), B, T)
     assert np.array_equal(got.cpu().numpy(), want)
+
+
+def test_gather_from_host_table_bit_exact():
+    """Rows gathered over PCIe from a pinned, mapped host table on a side
+    stream; the compute stream waits on the returned event."""
+    rng = np.random.default_rng(21)
+    K, D_h = 8, 160
+    rows = synth.primes_at_most(3001, 16)
+    tables = [rng.standard_normal((P, D_h)).astype(np.float32) for P in rows]
+    N = 2051
+    idx = np.stack([rng.integers(0, P, N) for P in rows], -1).astype(np.int32)
+    tb = [synth.to_bf16_bits(t) for t in tables]
+    want = O.gather(idx, tb)
+    flat = np.concatenate([t.reshape(-1) for t in tb]).view(np.int16)
+    host = torch.from_numpy(flat).pin_memory()       # page-locked, mapped into the GPU's space
+    cfg = eg.make_cfg(K, D_h, 256, 1, 1000, 770, eg.BF16, rows, np.ones((16, 3), np.uint64))
+    e = torch.empty((N, 16 * D_h), dtype=torch.bfloat16, device="cuda")
+    side = torch.cuda.Stream()
+    done = torch.cuda.Event()
+    idx_d = dev(idx)
+    side.wait_stream(torch.cuda.current_stream())
+    eg.engram_forward_hosttable(cfg, idx_d, host.data_ptr(), N, e, side, done)
+    torch.cuda.current_stream().wait_event(done)
+    assert np.array_equal(bf16_bits(e), want)
+    assert eg.engram_get_status() == 0
+
+
+def test_gather_from_host_table_rejects_unmapped_memory():
+    cfg = eg.make_cfg(8, 160, 256, 1, 1000, 770, eg.BF16, synth.primes_at_most(3001, 16),
+                      np.ones((16, 3), np.uint64))
+    plain = np.zeros(1 << 20, dtype=np.int16)          # ordinary pageable host memory
+    idx = dev(np.zeros((4, 16), np.int32))
+    e = torch.empty((4, 16 * 160), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(eg.EngramError) as ex:
+        eg.engram_forward_hosttable(cfg, idx, plain.ctypes.data, 4, e, None, None)
+    assert ex.value.rc == -1
