@@ -260,7 +260,7 @@ int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const 
       cudaGetLastError();
       return ENGRAM_ERR_INVALID_ARG;
     }
-    rc = launch_gather(make_head_params(cfg), idx, dev_ptr, n_tok, elem_bytes(cfg), e, s);
+    rc = launch_gather_host(make_head_params(cfg), idx, dev_ptr, n_tok, elem_bytes(cfg), e, s);
     if (rc) return rc;
   }
   if (done_event != nullptr) return ck(cudaEventRecord((cudaEvent_t)done_event, s));

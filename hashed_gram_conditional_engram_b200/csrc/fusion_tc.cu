@@ -358,6 +358,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // causal conv over (s3, s2, s1, vt), out = h + vt + SiLU(y), written over h in
 // place.  CHECK = true when a sequence may start inside the group: the conv
 // history is cleared at position 0.
+//
+// SiLU(y) = y * sigmoid(y) = y/2 * (1 + tanh(y/2)): one hardware tanh
+// (tanh.approx.f32, relative error about 2^-11) instead of an exponential and
+// a reciprocal; the error stays below the bf16 rounding of the output (2^-9).
+__device__ __forceinline__ float silu_tanh(float y) {
+  const float hy = 0.5f * y;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hy));
+  return fmaf(hy, t, hy);
+}
+
 template <bool CHECK>
 __device__ __forceinline__ void conv_group16(const uint32_t (&u)[16], const float4* al4,
                                              uint16_t* hs, const float4 w, float& s1, float& s2,
@@ -379,7 +390,7 @@ __device__ __forceinline__ void conv_group16(const uint32_t (&u)[16], const floa
       s2 = s1;
       s1 = vt;
       const float hv = __uint_as_float(((uint32_t)hs[jj * BM]) << 16);
-      const float o = hv + vt + __fdividef(y, 1.0f + __expf(-y));  // h + vt + SiLU(y)
+      const float o = hv + vt + silu_tanh(y);  // h + vt + SiLU(y)
       hs[jj * BM] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
     }
   }
@@ -767,6 +778,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
           if (DECODE) {
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
+              // the conv states of 16 tokens, loaded before any of them is
+              // written back, so the loads overlap instead of each waiting
+              // behind the previous token's stores
+              float sa1[16], sa2[16], sa3[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int64_t n = nb + g * 16 + i;
+                sa1[i] = sa2[i] = sa3[i] = 0.f;
+                if (n < args.N) {
+                  const float* st = args.conv_state + n * 3 * args.d + feat;
+                  sa3[i] = st[0];
+                  sa2[i] = st[args.d];
+                  sa1[i] = st[2 * args.d];
+                }
+              }
               if (g == 1 && got) tmem_wait16(un);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
@@ -777,19 +803,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
                   const int jj = g * 16 + q * 4 + r;
                   const int64_t n = nb + jj;
                   const float vt = av[r] * __uint_as_float(g == 0 ? u[q * 4 + r] : un[q * 4 + r]);
-                  float a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                  const float a1 = sa1[q * 4 + r], a2 = sa2[q * 4 + r], a3 = sa3[q * 4 + r];
                   if (n < args.N) {
                     float* st = args.conv_state + n * 3 * args.d + feat;
-                    a3 = st[0];
-                    a2 = st[args.d];
-                    a1 = st[2 * args.d];
                     st[0] = a2;
                     st[args.d] = a1;
                     st[2 * args.d] = vt;
                   }
                   const float y = fmaf(w.x, a3, fmaf(w.y, a2, fmaf(w.z, a1, w.w * vt)));
                   const float hv = __uint_as_float(((uint32_t)hs[jj * BM]) << 16);
-                  const float o = hv + vt + __fdividef(y, 1.0f + __expf(-y));
+                  const float o = hv + vt + silu_tanh(y);
                   hs[jj * BM] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
                 }
               }
@@ -857,24 +880,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
   }
 }
 
-// alpha of every token from the gate partials of pass K (fixed order):
+// alpha of every token from the gate partials of pass K, one warp per token
+// (fixed order: lane-strided sums, then a butterfly over the lanes):
 // alpha = sigmoid(<h, k> r_h r_k / sqrt(d)), r_x = (mean(x^2) + eps)^(-1/2).
-__global__ void __launch_bounds__(256) gate_from_partials_kernel(const float4* __restrict__ part,
-                                                                 int n_part, int64_t N, int d,
-                                                                 float* __restrict__ alpha,
-                                                                 float* __restrict__ alpha_copy) {
+constexpr int GATE_THREADS = 256;
+__global__ void __launch_bounds__(GATE_THREADS) gate_from_partials_kernel(
+    const float4* __restrict__ part, int n_part, int64_t N, int d, float* __restrict__ alpha,
+    float* __restrict__ alpha_copy) {
   allow_dependents();
   wait_prior_grid();  // the partials of pass K
-  const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (int64_t)blockIdx.x * (GATE_THREADS / 32) + (threadIdx.x >> 5);
+  if (n >= N) return;  // whole warps leave together
   const float4* pr = part + n * n_part;
   float kk = 0.f, hk = 0.f, hh = 0.f;
-  for (int i = 0; i < n_part; ++i) {
+  for (int i = lane; i < n_part; i += 32) {
     const float4 q = __ldg(pr + i);
     kk += q.x;
     hk += q.y;
     hh += q.z;
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kk += __shfl_xor_sync(0xffffffffu, kk, o);
+    hk += __shfl_xor_sync(0xffffffffu, hk, o);
+    hh += __shfl_xor_sync(0xffffffffu, hh, o);
+  }
+  if (lane != 0) return;
   const float invd = 1.0f / (float)d;
   const float rh = rsqrtf(hh * invd + RMS_EPS), rk = rsqrtf(kk * invd + RMS_EPS);
   const float a = 1.0f / (1.0f + expf(-(hk * rh * rk * rsqrtf((float)d))));
@@ -996,8 +1028,9 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   if (rc) return rc;
   {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((N + 255) / 256));
-    cfg.blockDim = dim3(256);
+    constexpr int TOK_PER_BLOCK = GATE_THREADS / 32;
+    cfg.gridDim = dim3((unsigned)((N + TOK_PER_BLOCK - 1) / TOK_PER_BLOCK));
+    cfg.blockDim = dim3(GATE_THREADS);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

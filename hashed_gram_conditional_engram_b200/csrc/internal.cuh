@@ -36,6 +36,10 @@ int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, i
                 int32_t* ngram_state, int32_t* idx, cudaStream_t s);
 int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,
                   int elem_bytes, void* e, cudaStream_t s);
+// the same gather from pinned host memory: a small fixed grid, deep per-thread
+// load queues (PCIe latency), the GPU's other SMs left free
+int launch_gather_host(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,
+                       int elem_bytes, void* e, cudaStream_t s);
 
 // fp32 CUDA-core path (small layers)
 struct F32Saved {

@@ -6,10 +6,14 @@ without the rest of the layer's inputs on the device.
         [--tokens 32768] [--d 2560] [--heads 16] [--dh 80] [--seq 4096] [--reps 3]
     python -m hashed_gram_conditional_engram_b200.kernel_cases gather [...]
     python -m hashed_gram_conditional_engram_b200.kernel_cases hash [...]
+    python -m hashed_gram_conditional_engram_b200.kernel_cases decode \
+        --tokens 256 --d 4096 --dh 128 --rows 1000003
 
 `fused` runs engram_forward with table = NULL on random gathered rows, i.e.
 the two tensor-core passes; `gather` gathers from a table of --rows rows per
-head; `hash` runs the compress + n-gram + hash kernel.  Defaults are the
+head; `hash` runs the compress + n-gram + hash kernel; `decode` runs whole
+decode steps (hash with rolling n-gram state, then engram_forward with the
+table and the conv state) for --tokens sequences of one token each.  Defaults are the
 27B-shaped layer's dimensions.  Prints the device time per repetition.
 """
 from __future__ import annotations
@@ -25,7 +29,7 @@ from . import synth
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["fused", "gather", "hash"])
+    ap.add_argument("kernel", choices=["fused", "gather", "hash", "decode"])
     ap.add_argument("--tokens", type=int, default=32768)
     ap.add_argument("--seq", type=int, default=4096)
     ap.add_argument("--d", type=int, default=2560)
@@ -39,6 +43,8 @@ def main(argv=None):
     dev = torch.device("cuda")
     K = a.heads // 2
     E = a.heads * a.dh
+    if a.kernel == "decode":
+        a.seq = 1
     B = a.tokens // a.seq
     T = a.seq
     N = B * T
@@ -72,6 +78,30 @@ def main(argv=None):
 
         def run():
             eg.engram_gather(cfg, idx, table, N, e)
+    elif a.kernel == "decode":
+        table = torch.empty(sum(rows) * a.dh, dtype=torch.bfloat16, device=dev)
+        table.normal_(0.0, 0.02, generator=g)
+        h = torch.randn((N, a.d), generator=g, device=dev).to(torch.bfloat16)
+        Wk = (torch.randn((a.d, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        Wv = (torch.randn((a.d, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        cw = torch.randn((a.d, 4), generator=g, device=dev) * 0.5
+        out = torch.empty_like(h)
+        e = torch.empty((N, E), dtype=torch.bfloat16, device=dev)
+        nb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        _, keys_np = synth.host_ids_keys(synth.workload("layer27b"))
+        keys = torch.from_numpy(keys_np).to(dev)
+        proj = torch.empty(129280, dtype=torch.int32, device=dev)
+        vb = eg.engram_workspace_size(None, eg.WS_VOCAB, 129280)
+        eg.engram_build_vocab_proj(keys, 129280, proj, torch.empty(vb, dtype=torch.uint8, device=dev), vb)
+        ids = torch.randint(0, 129280, (N,), generator=g, device=dev, dtype=torch.int32)
+        state = torch.full((N, 2), cfg.V_c, dtype=torch.int32, device=dev)
+        conv_state = torch.zeros((N, 1, 3, a.d), device=dev)
+        idx = torch.empty((N, 1, a.heads), dtype=torch.int32, device=dev)
+
+        def run():
+            eg.engram_hash_indices(cfg, proj, ids, N, 1, state, idx)
+            eg.engram_forward(cfg, idx, table, e, h, Wk, Wv, cw, conv_state, out, None, N, 1, ws, nb)
     else:
         ids_np, keys_np = synth.host_ids_keys(synth.workload("layer27b"))
         keys = torch.from_numpy(keys_np).to(dev)

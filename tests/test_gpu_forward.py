@@ -250,3 +250,58 @@ def test_forward_layer27b_sampled():
     assert max(aerrs) <= TOL_BF16, max(aerrs)
     del table, dense, L
     torch.cuda.empty_cache()
+
+
+def test_decode_full_size_sampled():
+    """The decode workload at full size (256 sequences x 1 token per step,
+    d 4,096, 16 heads x 128 dims, 13B-parameter table) in the launch
+    configuration of the timed decode step, for 4 steps.  Hash indices of
+    every sequence bit-exact; out, alpha and the conv state of sampled
+    sequences (both CTAs of a pair, tile seams, first and last) against the
+    oracle's decode step carried across the steps."""
+    w = synth.workload("decode")
+    ids, keys = synth.host_ids_keys(w)
+    mult = synth.hash_multipliers(synth.layer_seed(w, 0), w.J)
+    proj_ref, V_c = O.build_vocab_proj(keys)
+    table = synth.device_table(w)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(41)
+    Wk_d = (torch.randn((1, w.d, w.E), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    Wv_d = (torch.randn((w.d, w.E), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    cw_d = torch.randn((w.d, 4), generator=g, device="cuda") * 0.5
+    cfg = cfg_of(w, mult, V_c)
+    proj, _ = gpu_vocab_proj(keys)
+    L = Layer(cfg, w.B, 1, table, None, Wk_d, Wv_d, cw_d, torch.bfloat16)
+    state = torch.full((w.B, 2), V_c, dtype=torch.int32, device="cuda")
+    conv = torch.zeros((w.B, 1, 3, w.d), dtype=torch.float32, device="cuda")
+    Wk = O.bf16_bits_to_f64(bf16_bits(Wk_d))
+    Wv = O.bf16_bits_to_f64(bf16_bits(Wv_d))
+    conv_w = cw_d.cpu().numpy()
+    base = np.concatenate([[0], np.cumsum(w.rows)[:-1]])
+    sample = np.array([0, 1, 31, 32, 33, 63, 64, 65, 127, 128, 129, 191, 192, 254, 255])
+    st_ref = np.full((w.B, 2), V_c, dtype=np.int32)
+    conv_ref = np.zeros((len(sample), 1, 3, w.d))
+    for step in range(4):
+        h_d = torch.randn((w.B, 1, 1, w.d), generator=g, device="cuda").to(torch.bfloat16)
+        L.h = h_d
+        idx = gpu_hash(cfg, proj, dev(ids[step].copy()), w.B, 1, state=state)
+        out = L.forward(idx, conv_state=conv)
+        torch.cuda.synchronize()
+        assert eg.engram_get_status() == 0
+        idx_ref, st_ref = O.hash_indices_decode(proj_ref, ids[step], st_ref, mult,
+                                                np.array(w.rows), w.K)
+        assert np.array_equal(idx.cpu().numpy().reshape(w.B, w.J), idx_ref), step
+        e_bits = np.stack([np.concatenate([
+            bf16_bits(table[(base[j] + idx_ref[b, j]) * w.D_h:(base[j] + idx_ref[b, j] + 1) * w.D_h])
+            for j in range(w.J)]) for b in sample])
+        h_bits = bf16_bits(h_d.view(w.B, w.d)[torch.from_numpy(sample).cuda()])
+        o_ref, a_ref, conv_ref = O.decode_step(
+            O.bf16_bits_to_f64(e_bits), O.bf16_bits_to_f64(h_bits)[:, None, :], Wk, Wv, conv_w,
+            conv_ref)
+        got = O.bf16_bits_to_f64(bf16_bits(out.view(w.B, w.d)))[sample]
+        want = O.bf16_bits_to_f64(O.f64_to_bf16_bits(o_ref[:, 0]))
+        assert max_rel_err(got, want) <= TOL_BF16, step
+        assert max_rel_err(_alpha(L, w.B, 1)[sample], a_ref) <= TOL_BF16, step
+        assert max_rel_err(conv.cpu().numpy()[sample], conv_ref) <= TOL_BF16, step
+    del table, L
+    torch.cuda.empty_cache()
