@@ -169,7 +169,8 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
   return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
                            static_cast<const __nv_bfloat16*>(Wk),
                            static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
-                           static_cast<__nv_bfloat16*>(out), saved, N, T, d, E, ws, ws_bytes, s);
+                           static_cast<__nv_bfloat16*>(out), saved, N, T, d, E, ws, ws_bytes,
+                           table != nullptr, s);
 }
 
 int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,

@@ -273,6 +273,18 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// The same through a 3-D map {64-element K chunk, row, chunk index}: one
+// instruction brings several 128-byte K chunks of a row block (a box per
+// chunk would cost one issue each).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b,
                                                uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -319,19 +331,21 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
                : "memory");
 }
 
-// Programmatic dependent launch: the next kernel in the stream may start
-// once every CTA of this one has signalled; wait_prior_grid blocks until the
-// kernel launched before this one has completed and its writes are visible
-// (a no-op when this kernel was launched without the attribute).
-__device__ __forceinline__ void allow_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void wait_prior_grid() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// 32 bf16 held in 4 x 16 bytes -> fp32
+__device__ __forceinline__ void unpack_bf16x32(const uint4 (&w4)[4], float (&x)[32]) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint32_t ws[4] = {w4[v].x, w4[v].y, w4[v].z, w4[v].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[v * 8 + 2 * i] = __uint_as_float(ws[i] << 16);
+      x[v * 8 + 2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+    }
+  }
 }
 
 // 32 bf16 (64 bytes) -> fp32
@@ -398,18 +412,26 @@ __device__ __forceinline__ void conv_group16(const uint32_t (&u)[16], const floa
 
 // ------------------------------------------------------------------ kernel
 
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, int KCH>
 struct TcShape {
   static constexpr bool VPASS = MODE != MODE_GATE_PARTIAL;
   // epilogue warps: 2 per TMEM lane quadrant
   static constexpr int EPI = 8;
   static constexpr int PARTS = EPI / 4;        // column parts of a tile, one per warp of a quadrant
   static constexpr int HP_WARP = 2 + EPI;      // pass V: warp that streams h in by TMA
-  static constexpr int NUM_THREADS = 64 + EPI * 32 + 32;
+  // B-operand producer: a second issuing thread, since one thread issues
+  // tiled copies at only about one per 150 ns (measured on B200), which would
+  // bound a stage of two boxes at ~300 ns
+  static constexpr int BP_WARP = 3 + EPI;
+  static constexpr int NUM_THREADS = 64 + EPI * 32 + 64;
   // a CTA pair computes a (2 * BM) x BN tile: each CTA loads its BM rows of
   // A and half of the BN rows of B, and holds its BM rows of the accumulator
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = (BN / 2) * BK * 2;
+  // a stage holds KCH chunks of 64 K elements (128 bytes) of each operand,
+  // each chunk a 128-byte-swizzled tile of its rows
+  static constexpr int A_CHUNK = BM * BK * 2;
+  static constexpr int B_CHUNK = (BN / 2) * BK * 2;
+  static constexpr int A_BYTES = A_CHUNK * KCH;
+  static constexpr int B_BYTES = B_CHUNK * KCH;
   static constexpr int TMEM_COLS = 2 * BN;
   // pass K (tokens on TMEM lanes, features on columns): each epilogue warp
   // takes one part of the tile's columns, 32 at a time
@@ -434,12 +456,12 @@ struct TcShape {
   static_assert(PART_COLS % 32 == 0, "parts of whole 32-column chunks");
 };
 
-template <int BN, int STAGES, int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, MODE>::NUM_THREADS, 1)
+template <int BN, int STAGES, int MODE, int KCH>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, MODE, KCH>::NUM_THREADS, 1)
     tc_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmO,
                     const __grid_constant__ CUtensorMap tmO29, const __grid_constant__ TcArgs args) {
-  using S = TcShape<BN, STAGES, MODE>;
+  using S = TcShape<BN, STAGES, MODE, KCH>;
   constexpr bool VPASS = S::VPASS;
   constexpr int NUM_EPI_WARPS = S::EPI;
   constexpr int HP_WARP = S::HP_WARP;
@@ -552,11 +574,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
             ok = false;
             break;
           }
-          // the leader's full barrier counts the bytes of both CTAs
+          // the leader's full barrier counts the bytes of both CTAs' A and B
+          // boxes (B comes from the B producer below)
           if (leader) mbar_expect_tx(&full[stage], 2 * STAGE_TX);
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
-          tma_load_2d_pair(sA + stage * S::A_BYTES, &tmA, fb, kt * BK, arow);
-          tma_load_2d_pair(sB + stage * S::B_BYTES, &tmB, fb, kt * BK, brow);
+          tma_load_3d_pair(sA + stage * S::A_BYTES, &tmA, fb, 0, arow, kt * KCH);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -595,9 +617,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
           const uint32_t a0 = smem_u32(sA + stage * S::A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * S::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            umma_bf16_pair(d_tmem, sw128_desc(a0 + k * UMMA_K * 2),
-                           sw128_desc(b0 + k * UMMA_K * 2), IDESC, (kt | k) != 0 ? 1u : 0u);
+          for (int c = 0; c < KCH; ++c) {
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              umma_bf16_pair(d_tmem, sw128_desc(a0 + c * S::A_CHUNK + k * UMMA_K * 2),
+                             sw128_desc(b0 + c * S::B_CHUNK + k * UMMA_K * 2), IDESC,
+                             (kt | c | k) != 0 ? 1u : 0u);
+            }
           }
           umma_commit_pair_both(&empty[stage]);
           if (++stage == STAGES) {
@@ -613,6 +639,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
       // all issued MMAs complete before TMEM is released
       umma_commit_pair_self(drain);
       wait_drain(drain, 0);
+    }
+  } else if (warp == S::BP_WARP) {
+    // ------------------------------------------------------------ B-operand producer
+    // Same stages and order as the A producer; its bytes count on the
+    // leader's full barrier, whose expected total the A producer posts (a
+    // phase cannot complete before that arrival).
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+        int arow, brow;
+        operand_rows(tile, arow, brow);
+        bool ok = true;
+        for (int kt = 0; kt < args.num_k_tiles; ++kt) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          tma_load_3d_pair(sB + stage * S::B_BYTES, &tmB, fb, 0, brow, kt * KCH);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
     }
   } else if (warp == HP_WARP) {
     // ------------------------------------------------------------ h producer (pass V)
@@ -646,7 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
         if (!ok) break;
       }
       for (int b = 0; b < S::HSLOTS; ++b) {
-        const uint32_t n_b = issued > (uint32_t)b ? (issued - 1 - b) / S::HSLOTS + 1 : 0;
+        const uint32_t n_b = issued > (uint32_t)b ? (issued - 1 - b) / (S::HSLOTS > 0 ? S::HSLOTS : 1) + 1 : 0;
         if (n_b > 0) wait_drain(&hfull[b], (n_b - 1) & 1u);
       }
     }
@@ -663,17 +716,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++iter) {
       const int mi = tile / args.num_n_tiles, ni = tile - mi * args.num_n_tiles;
       const int64_t tok0 = (int64_t)mi * args.m_stride + args.m_offset;
-      int got = 0;
-      if (lane == 0) got = wait_bounded(&tfull[acc], acc_phase, abort_flag, args.status) ? 1 : 0;
-      got = __shfl_sync(FULL, got, 0);
-      tc_fence_after();
+      // while the MMAs of this tile run: pull what the epilogue will read
+      // into L2 (pass K: the first tile's h; decode: the conv state)
+      if constexpr (!VPASS) {
+        if (iter == 0) {
+          const int64_t n0 = tok0 + (int)rank * BM + quad * 32 + lane;
+          if (n0 >= 0 && n0 < args.N) {
+            const __nv_bfloat16* hp0 = args.h + n0 * args.d + ni * BN + part * S::PART_COLS;
+            for (int b = 0; b < S::PART_COLS * 2; b += 128) prefetch_l2(hp0 + b / 2);
+          }
+        }
+      } else if constexpr (MODE == MODE_VALUE_DECODE) {
+        const int64_t n0 = tok0 + part * S::PART_COLS + lane;
+        if (lane < S::PART_COLS && n0 < args.N) {
+          const float* st = args.conv_state + n0 * 3 * args.d + ni * (2 * BM) + (int)rank * BM +
+                            quad * 32;
+          prefetch_l2(st);
+          prefetch_l2(st + args.d);
+          prefetch_l2(st + 2 * args.d);
+        }
+      }
       const uint32_t t_acc = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+      // the tile's accumulator is complete (each branch first issues the
+      // loads that do not depend on it)
+      auto wait_acc = [&]() {
+        int ok = 0;
+        if (lane == 0) ok = wait_bounded(&tfull[acc], acc_phase, abort_flag, args.status) ? 1 : 0;
+        ok = __shfl_sync(FULL, ok, 0);
+        tc_fence_after();
+        return ok;
+      };
 
       if constexpr (!VPASS) {
         // pass K: this lane's token, one part of the tile's features
         const int64_t n = tok0 + (int)rank * BM + quad * 32 + lane;
         const bool valid = n >= 0 && n < args.N;
         const int col_base = ni * BN + part * S::PART_COLS;
+        // h of the first 32 features, fetched while the MMAs finish
+        uint4 h0[4];
+        if (valid) {
+          const uint4* q = reinterpret_cast<const uint4*>(args.h + n * args.d + col_base);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) h0[v] = __ldg(q + v);
+        }
+        const int got = wait_acc();
         const uint32_t t_row = t_acc + (uint32_t)(part * S::PART_COLS);
         {  // pull the next tile's rows of h into L2 while this one is reduced
           const int nxt = tile + num_pairs;
@@ -700,7 +786,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
           }
           if (valid) {
             float hv[32];
-            load_bf16x32(args.h + n * args.d + col_base + c * 32, hv);
+            if (c == 0)
+              unpack_bf16x32(h0, hv);
+            else
+              load_bf16x32(args.h + n * args.d + col_base + c * 32, hv);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               kk = fmaf(v[i], v[i], kk);
@@ -719,16 +808,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
         const int f0 = ni * (2 * BM) + (int)rank * BM;  // this CTA's features
         const int feat = f0 + quad * 32 + lane;
         const int T = args.T;
+        const float4 w = __ldg(args.conv_w + feat);  // taps: w.x for t-3 .. w.w for t
         if (iter == 0) wait_prior_grid();  // alpha comes from the gate kernel
         // gates of the tile's tokens, staged once by all epilogue warps
         float* al = alpha_s + (iter & 1) * BN;
         for (int i = ew * 32 + lane; i < BN; i += NUM_EPI_WARPS * 32) {
           const int64_t n = tok0 + i;
-          al[i] = (n >= 0 && n < args.N) ? __ldg(args.alpha + n) : 0.f;
+          // written by the gate kernel while this grid may already run:
+          // read through L2, not the read-only cache
+          al[i] = (n >= 0 && n < args.N) ? __ldcg(args.alpha + n) : 0.f;
+        }
+        const int j0 = part * S::PART_COLS;          // first tile column of this warp
+        // decode, one chunk per part: the conv states of the first 16 tokens,
+        // fetched while the MMAs finish
+        constexpr bool PRELOAD = DECODE && NCH == 1;
+        float pre1[PRELOAD ? 16 : 1], pre2[PRELOAD ? 16 : 1], pre3[PRELOAD ? 16 : 1];
+        if constexpr (PRELOAD) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int64_t n = tok0 + j0 + i;
+            pre1[i] = pre2[i] = pre3[i] = 0.f;
+            if (n < args.N) {
+              const float* st = args.conv_state + n * 3 * args.d + feat;
+              pre3[i] = st[0];
+              pre2[i] = st[args.d];
+              pre1[i] = st[2 * args.d];
+            }
+          }
         }
         named_bar_sync(1, NUM_EPI_WARPS * 32);
-        const float4 w = __ldg(args.conv_w + feat);  // taps: w.x for t-3 .. w.w for t
-        const int j0 = part * S::PART_COLS;          // first tile column of this warp
+        const int got = wait_acc();
         const int first_out = -args.m_offset;        // halo columns produce no output
         int pos = (int)((((tok0 + j0) % T) + T) % T);  // sequence position of column j0
         float s1 = 0.f, s2 = 0.f, s3 = 0.f;           // vt of tokens t-1, t-2, t-3
@@ -782,15 +891,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
               // written back, so the loads overlap instead of each waiting
               // behind the previous token's stores
               float sa1[16], sa2[16], sa3[16];
+              if (PRELOAD && g == 0) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int64_t n = nb + g * 16 + i;
-                sa1[i] = sa2[i] = sa3[i] = 0.f;
-                if (n < args.N) {
-                  const float* st = args.conv_state + n * 3 * args.d + feat;
-                  sa3[i] = st[0];
-                  sa2[i] = st[args.d];
-                  sa1[i] = st[2 * args.d];
+                for (int i = 0; i < 16; ++i) {
+                  sa1[i] = pre1[PRELOAD ? i : 0];
+                  sa2[i] = pre2[PRELOAD ? i : 0];
+                  sa3[i] = pre3[PRELOAD ? i : 0];
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const int64_t n = nb + g * 16 + i;
+                  sa1[i] = sa2[i] = sa3[i] = 0.f;
+                  if (n < args.N) {
+                    const float* st = args.conv_state + n * 3 * args.d + feat;
+                    sa3[i] = st[0];
+                    sa2[i] = st[args.d];
+                    sa1[i] = st[2 * args.d];
+                  }
                 }
               }
               if (g == 1 && got) tmem_wait16(un);
@@ -865,7 +983,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
     }
     // output boxes of pass V fully written before the CTA exits
     if (VPASS && ew == part * 4 && lane == 0) {
-      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+      // the stores have read their boxes; their writes complete with the grid
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       if (pending_slot >= 0) mbar_arrive(&hempty[pending_slot]);
     }
   }
@@ -895,7 +1014,7 @@ __global__ void __launch_bounds__(GATE_THREADS) gate_from_partials_kernel(
   const float4* pr = part + n * n_part;
   float kk = 0.f, hk = 0.f, hh = 0.f;
   for (int i = lane; i < n_part; i += 32) {
-    const float4 q = __ldg(pr + i);
+    const float4 q = __ldcg(pr + i);  // written by pass K during this grid's lifetime
     kk += q.x;
     hk += q.y;
     hh += q.z;
@@ -949,11 +1068,28 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, int MODE>
+// K-major bf16 operand [rows, K] as a 3-D tensor {64-element chunk, row,
+// chunk index} (strides: a row, 128 bytes), boxes of box_rows rows x kch
+// chunks, 128-byte swizzle: a box lands as kch consecutive swizzled tiles.
+bool make_tmap_k(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows,
+                 uint32_t kch) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)BK, rows, K / BK};
+  const cuuint64_t strides[2] = {K * 2, BK * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, kch};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int MODE, int KCH>
 int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& th,
-                const CUtensorMap& to, const CUtensorMap& to29, const TcArgs& a, cudaStream_t s) {
-  using S = TcShape<BN, STAGES, MODE>;
-  auto kern = tc_fused_kernel<BN, STAGES, MODE>;
+                const CUtensorMap& to, const CUtensorMap& to29, const TcArgs& a, cudaStream_t s,
+                bool pdl) {
+  using S = TcShape<BN, STAGES, MODE, KCH>;
+  auto kern = tc_fused_kernel<BN, STAGES, MODE, KCH>;
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -979,25 +1115,24 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return ck(cudaLaunchKernelEx(&cfg, kern, ta, tb, th, to, to29, a));
 }
 
-template <int BN, int STAGES_K, int STAGES_V>
+template <int BN, int STAGES_K, int STAGES_V, int KCH>
 int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
               float* alpha_saved, int64_t N, int T, int d, int E, float4* part, float* alpha,
-              cudaStream_t s) {
-  const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B;
+              bool chained, cudaStream_t s) {
   // Each CTA of a pair loads 128 rows of A and BN/2 rows of B per stage.
   // pass K: A = e (256 tokens per pair tile), B = W_k (BN features)
   CUtensorMap ta_k, tb_k, ta_v, tb_v, th, to, to29;
-  if (!make_tmap(&ta_k, e, (uint64_t)E, (uint64_t)N, BK, BM, sw128)) return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&tb_k, Wk, (uint64_t)E, (uint64_t)d, BK, BN / 2, sw128)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap_k(&ta_k, e, (uint64_t)E, (uint64_t)N, BM, KCH)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap_k(&tb_k, Wk, (uint64_t)E, (uint64_t)d, BN / 2, KCH)) return ENGRAM_ERR_CUDA;
   // pass V: A = W_v (256 features per pair tile), B = e (BN tokens);
   // h in boxes of 32 tokens x 128 features
-  if (!make_tmap(&ta_v, Wv, (uint64_t)E, (uint64_t)d, BK, BM, sw128)) return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&tb_v, e, (uint64_t)E, (uint64_t)N, BK, BN / 2, sw128)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap_k(&ta_v, Wv, (uint64_t)E, (uint64_t)d, BM, KCH)) return ENGRAM_ERR_CUDA;
+  if (!make_tmap_k(&tb_v, e, (uint64_t)E, (uint64_t)N, BN / 2, KCH)) return ENGRAM_ERR_CUDA;
   if (!make_tmap(&th, h, (uint64_t)d, (uint64_t)N, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ENGRAM_ERR_CUDA;
   // out in the same boxes; a 29-token box skips the 3 halo tokens of a tile
@@ -1006,11 +1141,11 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   if (!make_tmap(&to29, out, (uint64_t)d, (uint64_t)N, BM, 32 - HALO, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ENGRAM_ERR_CUDA;
   TcArgs a;
-  a.num_k_tiles = E / BK;
+  a.num_k_tiles = E / (BK * KCH);
   a.N = N;
   a.T = T;
   a.d = d;
-  a.n_part = TcShape<BN, STAGES_K, MODE_GATE_PARTIAL>::PARTS * (d / BN);
+  a.n_part = TcShape<BN, STAGES_K, MODE_GATE_PARTIAL, KCH>::PARTS * (d / BN);
   a.h = h;
   a.out = out;
   a.part = part;
@@ -1024,7 +1159,9 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.m_stride = 2 * BM;
   a.m_offset = 0;
   a.num_m_tiles = (int)((N + 2 * BM - 1) / (2 * BM));
-  int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL>(ta_k, tb_k, th, to, to29, a, s);
+  // pass K starts early only behind this call's own gather; as the call's
+  // first kernel it keeps plain stream order with the caller's work
+  int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL, KCH>(ta_k, tb_k, th, to, to29, a, s, chained);
   if (rc) return rc;
   {
     cudaLaunchConfig_t cfg = {};
@@ -1054,8 +1191,8 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   }
   a.num_m_tiles = (int)((N + a.m_stride - 1) / a.m_stride);
   if (conv_state != nullptr)
-    return launch_pass<BN, STAGES_V, MODE_VALUE_DECODE>(ta_v, tb_v, th, to, to29, a, s);
-  return launch_pass<BN, STAGES_V, MODE_VALUE_CONV>(ta_v, tb_v, th, to, to29, a, s);
+    return launch_pass<BN, STAGES_V, MODE_VALUE_DECODE, KCH>(ta_v, tb_v, th, to, to29, a, s, true);
+  return launch_pass<BN, STAGES_V, MODE_VALUE_CONV, KCH>(ta_v, tb_v, th, to, to29, a, s, true);
 }
 
 inline bool use_wide(int64_t N, int d) { return d % 256 == 0 && N > 4096; }
@@ -1076,7 +1213,7 @@ size_t tc_forward_ws_bytes(int64_t N, int d, int E) {
 int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
                       __nv_bfloat16* out, float* alpha_saved, int64_t N, int T, int d, int E,
-                      void* ws, size_t ws_bytes, cudaStream_t s) {
+                      void* ws, size_t ws_bytes, bool chained, cudaStream_t s) {
   if (ws_bytes < tc_forward_ws_bytes(N, d, E) || ws == nullptr) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL - 256) return ENGRAM_ERR_UNSUPPORTED;
   const bool wide = use_wide(N, d);
@@ -1085,10 +1222,15 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
   float* alpha = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                           (size_t)N * 2 * (d / BN) * sizeof(float4));
   if (wide)
-    return run_layer<256, 6, 5>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
-                                alpha, s);
-  return run_layer<64, 8, 6>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E, part,
-                             alpha, s);
+    return run_layer<256, 6, 5, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E,
+                                   part, alpha, chained, s);
+  // few tokens: each CTA streams long operand rows at a rate set by how many
+  // bytes one copy instruction brings, so two K chunks go in each box
+  if (E % (2 * BK) == 0)
+    return run_layer<64, 4, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E,
+                                  part, alpha, chained, s);
+  return run_layer<64, 8, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E,
+                                part, alpha, chained, s);
 }
 
 }  // namespace engram

@@ -31,6 +31,38 @@ __device__ __forceinline__ float bfbits2f(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }
 
+// ---------------------------------------------------------------- stream order
+// Programmatic dependent launch.  Every kernel of the library calls
+// wait_prior_grid() before it reads anything that an earlier kernel on its
+// stream wrote: it blocks until the kernel launched before this one has
+// completed and its writes are visible (a no-op for a kernel launched
+// without the attribute).  Since every kernel waits so, completion is
+// transitive along the stream, and allow_dependents() may let the next
+// kernel start its prologue while this one still runs.
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Launch with programmatic stream serialisation allowed (see above).
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+               Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return ck(cudaLaunchKernelEx(&cfg, kern, args...));
+}
+
 // ---------------------------------------------------------------- launches
 int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, int B, int T,
                 int32_t* ngram_state, int32_t* idx, cudaStream_t s);
@@ -79,6 +111,6 @@ int tc_supported(int d, int E, int M);
 int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
                       __nv_bfloat16* out, float* alpha_saved, int64_t N, int T, int d, int E,
-                      void* ws, size_t ws_bytes, cudaStream_t s);
+                      void* ws, size_t ws_bytes, bool chained, cudaStream_t s);
 
 }  // namespace engram

@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HeadP
                                                    int32_t* __restrict__ ngram_state,
                                                    int32_t* __restrict__ idx,
                                                    unsigned int* status) {
+  allow_dependents();  // a programmatically launched successor waits for this grid anyway
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
   const int q = lane % tpt;             // which four heads
@@ -106,6 +107,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ Hea
                                                      int64_t n_tok, int CR,
                                                      uint4* __restrict__ e,
                                                      unsigned int* status) {
+  allow_dependents();
   const int per_tok = hp.J * CR;
   const int64_t total = n_tok * per_tok;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -150,6 +152,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant_
                                                           int64_t n_tok,
                                                           uint4* __restrict__ e,
                                                           unsigned int* status) {
+  allow_dependents();
   constexpr int PER_TOK = JH * CR;             // pieces per token
   constexpr int PER_LANE = (PER_TOK + 31) / 32;
   const int lane = threadIdx.x & 31;
@@ -231,6 +234,17 @@ int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, i
     kern<<<(unsigned)blocks, threads, 0, s>>>(hp, idx, tb, n_tok, eo, st);
     return ck(cudaGetLastError());
   };
+  const int64_t total = n_tok * hp.J * CR;
+  if (n_tok * 32 < (int64_t)sms * threads * 4) {
+    // few tokens (a decode step): warps of tokens would leave most SMs idle;
+    // one 16-byte piece per thread instead, a single round trip each
+    constexpr int UNROLL_SMALL = 2;
+    const int64_t blocks =
+        (total + (int64_t)threads * UNROLL_SMALL - 1) / ((int64_t)threads * UNROLL_SMALL);
+    gather_kernel<UNROLL_SMALL><<<(unsigned)blocks, threads, 0, s>>>(hp, idx, tb, n_tok, CR, eo,
+                                                                     st);
+    return ck(cudaGetLastError());
+  }
   const int key = hp.J * 100 + CR;
   switch (key) {
     case 4 * 100 + 4: return rows(gather_rows_kernel<4, 4, 8>, 8);     // fp32 rows of 16, 4 heads
@@ -240,7 +254,6 @@ int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, i
     default: break;
   }
   constexpr int UNROLL = 8;
-  const int64_t total = n_tok * hp.J * CR;
   int64_t blocks = (total + (int64_t)threads * UNROLL - 1) / ((int64_t)threads * UNROLL);
   const int64_t cap = (int64_t)sms * 8;
   if (blocks > cap) blocks = cap;
