@@ -94,25 +94,76 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def gpu_uuid(local: int):
+    """'GPU-…' identifier of the CUDA device, for nvidia-smi and NVML (whose
+    indices need not follow CUDA_VISIBLE_DEVICES)."""
+    try:
+        import torch
+        return "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:  # noqa: BLE001
+        return None
+
+
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    """SM clocks and clock-event (throttle) reasons during the timed region.
+
+    Two sources: nvidia-smi every 100 ms (the standard record), and an NVML
+    poller every ~2 ms restricted to the window between begin() and end(),
+    which a timed region of tens of milliseconds needs to be sampled at all.
+    """
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {4: "sw_power_cap", 8: "hw_slowdown", 32: "sw_thermal_slowdown",
+               64: "hw_thermal_slowdown", 128: "hw_power_brake_slowdown"}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
+        self.uuid = gpu_uuid(gpu_index)
         self.proc = None
         self.path = None
+        self.nv = []
+        self.window = None
+        self._stop = False
+        self._thread = None
+
+    def _poll(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid
+                 else pynvml.nvmlDeviceGetHandleByIndex(self.gpu))
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            while not self._stop:
+                t = time.perf_counter()
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.nv.append((t, sm, rs, pw))
+                time.sleep(0.002)
+            pynvml.nvmlShutdown()
+        except Exception:  # noqa: BLE001 -- the nvidia-smi record remains
+            pass
+
+    def begin(self):
+        self.window = [time.perf_counter(), None]
+
+    def end(self):
+        if self.window is not None:
+            self.window[1] = time.perf_counter()
 
     def __enter__(self):
+        import threading
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={self.uuid or self.gpu}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
@@ -121,6 +172,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -129,10 +183,10 @@ class ClockSampler:
                 self.proc.kill()
             self.f.close()
 
-    def summary(self):
-        if self.proc is None or self.path is None:
-            return None
+    def _smi_rows(self):
         rows = []
+        if self.proc is None or self.path is None:
+            return rows
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
@@ -145,10 +199,10 @@ class ClockSampler:
                 except ValueError:
                     continue
         os.unlink(self.path)
-        if not rows:
-            return None
-        smax = max(r["smax"] for r in rows)
-        loaded = [r for r in rows if r["power"] > 250.0] or rows
+        return rows
+
+    def summary(self):
+        rows = self._smi_rows()
         reasons = set()
         for r in rows:
             if r["hw"] == "Active":
@@ -159,8 +213,28 @@ class ClockSampler:
                 reasons.add("sw_thermal_slowdown")
             if r["pcap"] == "Active":
                 reasons.add("sw_power_cap")
-        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded)}
+        out = {}
+        if rows:
+            loaded = [r for r in rows if r["power"] > 250.0] or rows
+            out = {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                   "sm_max_mhz": max(r["smax"] for r in rows),
+                   "smi_samples": len(rows), "smi_samples_under_load": len(loaded)}
+        win = [x for x in self.nv if self.window and self.window[1] is not None
+               and self.window[0] <= x[0] <= self.window[1]]
+        if win:
+            for _, _, rs, _ in win:
+                for bit, name in self.REASONS.items():
+                    if rs & bit:
+                        reasons.add(name)
+            sms = [x[1] for x in win]
+            out.update({"sm_mhz": statistics.median(sms), "sm_min_mhz": min(sms),
+                        "sm_max_mhz": getattr(self, "smax", out.get("sm_max_mhz")),
+                        "nvml_samples_in_timed_region": len(win),
+                        "power_w_median": statistics.median(x[3] for x in win)})
+        if not out:
+            return None
+        out["reasons"] = sorted(reasons)
+        return out
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -252,11 +326,20 @@ def run_ours(args):
         if ev is not None:
             ev[3].record(stream)
 
-    for _ in range(args.warmup):
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.warmup):
+        if i == 1:
+            w0.record(stream)
         step()
+    w1.record(stream)
     torch.cuda.synchronize()
+    est_step_ms = w0.elapsed_time(w1) / max(1, args.warmup - 1)
     if eg.engram_get_status(stream) != 0:
         raise RuntimeError("device status word set during warm-up")
+    # a one-warp probe beside the timed steps reads the SM clock they run at
+    probe = torch.zeros(2, dtype=torch.int64, device=dev)
+    probe_stream = torch.cuda.Stream(dev)
+    probe_ns = max(1000, int(0.9 * est_step_ms * args.steps * 1e6))
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
@@ -264,13 +347,30 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         barrier()
         torch.cuda.synchronize()
+        clk.begin()
         start.record(stream)
         for k in range(args.steps):
             step(evs[k])
         end.record(stream)
         torch.cuda.synchronize()
+        clk.end()
         barrier()
-    clocks = clk.summary()
+    clocks = clk.summary() or {}
+    # the same steps once more, untimed, with the clock probe beside them (a
+    # probe inside the timed region would hold one SM away from the
+    # persistent passes)
+    torch.cuda.synchronize()
+    eg.engram_clock_probe(probe, probe_ns, probe_stream)
+    for k in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    pc, pns = probe.cpu().tolist()
+    if pns > 0:
+        clocks["sm_mhz_device"] = 1000.0 * pc / pns
+        clocks["sm_mhz_device_how"] = ("SM cycles / global-timer ns of a one-warp probe over "
+                                       f"{pns / 1e6:.1f} ms of an untimed repeat of the timed "
+                                       "steps (the driver's clock query keeps reading the "
+                                       "maximum while board power management lowers it)")
     elapsed_ms = start.elapsed_time(end)
     t_hash = sum(ev[0].elapsed_time(ev[1]) for ev in evs) / args.steps
     t_gather = sum(ev[1].elapsed_time(ev[2]) for ev in evs) / args.steps
@@ -318,6 +418,7 @@ def run_ours(args):
     flops = 2 * 2.0 * N * w.E * w.d            # k and v projections, algorithmic
     achieved = flops / (t_fuse / 1e3) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     traffic = None
     tp = os.path.join(ROOT, "profiles", "traffic_layer27b.json")
     if os.path.exists(tp):
@@ -361,7 +462,10 @@ def run_ours(args):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "kernel": "engram_forward(table=NULL): tc_fused_kernel pass K, gate kernel, tc_fused_kernel pass V",
-                         "peak_source": f"{peak_src} bf16_tflops (burst)"},
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         # the step loop runs the tensor pipe for tens of ms under the
+                         # 1 kW cap: the sustained figure is the one it can hold
+                         "peak_sustained": peak_sus, "frac_of_sustained": achieved / peak_sus},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": 5 * args.steps,

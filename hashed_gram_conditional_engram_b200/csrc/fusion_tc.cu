@@ -999,33 +999,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
   }
 }
 
-// alpha of every token from the gate partials of pass K, one warp per token
-// (fixed order: lane-strided sums, then a butterfly over the lanes):
+// alpha of every token from the gate partials of pass K, TPT lanes per token
+// (a fixed order: lane-strided sums, then a butterfly over the TPT lanes):
 // alpha = sigmoid(<h, k> r_h r_k / sqrt(d)), r_x = (mean(x^2) + eps)^(-1/2).
+// Few tokens (decode) take a warp each; many take a thread each, which keeps
+// more tokens' loads in flight.
 constexpr int GATE_THREADS = 256;
+template <int TPT>
 __global__ void __launch_bounds__(GATE_THREADS) gate_from_partials_kernel(
     const float4* __restrict__ part, int n_part, int64_t N, int d, float* __restrict__ alpha,
     float* __restrict__ alpha_copy) {
   allow_dependents();
   wait_prior_grid();  // the partials of pass K
-  const int lane = threadIdx.x & 31;
-  const int64_t n = (int64_t)blockIdx.x * (GATE_THREADS / 32) + (threadIdx.x >> 5);
-  if (n >= N) return;  // whole warps leave together
-  const float4* pr = part + n * n_part;
+  const int sub = threadIdx.x % TPT;
+  const int64_t n = (int64_t)blockIdx.x * (GATE_THREADS / TPT) + threadIdx.x / TPT;
   float kk = 0.f, hk = 0.f, hh = 0.f;
-  for (int i = lane; i < n_part; i += 32) {
-    const float4 q = __ldcg(pr + i);  // written by pass K during this grid's lifetime
-    kk += q.x;
-    hk += q.y;
-    hh += q.z;
+  if (n < N) {
+    const float4* pr = part + n * n_part;
+    for (int i = sub; i < n_part; i += TPT) {
+      const float4 q = __ldcg(pr + i);  // written by pass K during this grid's lifetime
+      kk += q.x;
+      hk += q.y;
+      hh += q.z;
+    }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
+  for (int o = TPT / 2; o > 0; o >>= 1) {  // every lane takes part in the shuffles
     kk += __shfl_xor_sync(0xffffffffu, kk, o);
     hk += __shfl_xor_sync(0xffffffffu, hk, o);
     hh += __shfl_xor_sync(0xffffffffu, hh, o);
   }
-  if (lane != 0) return;
+  if (n >= N || sub != 0) return;
   const float invd = 1.0f / (float)d;
   const float rh = rsqrtf(hh * invd + RMS_EPS), rk = rsqrtf(kk * invd + RMS_EPS);
   const float a = 1.0f / (1.0f + expf(-(hk * rh * rk * rsqrtf((float)d))));
@@ -1164,18 +1168,17 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL, KCH>(ta_k, tb_k, th, to, to29, a, s, chained);
   if (rc) return rc;
   {
-    cudaLaunchConfig_t cfg = {};
-    constexpr int TOK_PER_BLOCK = GATE_THREADS / 32;
-    cfg.gridDim = dim3((unsigned)((N + TOK_PER_BLOCK - 1) / TOK_PER_BLOCK));
-    cfg.blockDim = dim3(GATE_THREADS);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    rc = ck(cudaLaunchKernelEx(&cfg, gate_from_partials_kernel, (const float4*)part, a.n_part, N,
-                               d, alpha, alpha_saved));
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const bool warp_per_token = N * 32 <= (int64_t)sms * 2048;  // one wave of the GPU
+    const int tok_per_block = warp_per_token ? GATE_THREADS / 32 : GATE_THREADS;
+    const dim3 grid((unsigned)((N + tok_per_block - 1) / tok_per_block));
+    rc = warp_per_token
+             ? launch_pdl(gate_from_partials_kernel<32>, grid, dim3(GATE_THREADS), 0, s,
+                          (const float4*)part, a.n_part, N, d, alpha, alpha_saved)
+             : launch_pdl(gate_from_partials_kernel<1>, grid, dim3(GATE_THREADS), 0, s,
+                          (const float4*)part, a.n_part, N, d, alpha, alpha_saved);
     if (rc) return rc;
   }
   a.alpha = alpha;

@@ -39,7 +39,7 @@ EXPORTED = (
     "engram_hash_indices", "engram_gather", "engram_forward", "engram_backward",
     "engram_table_grad", "engram_table_grad_noalloc", "engram_forward_hosttable",
     "engram_get_status",
-    "engram_device_sm_count",
+    "engram_device_sm_count", "engram_clock_probe",
 )
 
 
@@ -108,6 +108,7 @@ def lib() -> ctypes.CDLL:
         "engram_forward_hosttable": (ctypes.c_int, [cfgp, P, P, i64, P, P, P]),
         "engram_get_status": (ctypes.c_int, [P]),
         "engram_device_sm_count": (ctypes.c_int, []),
+        "engram_clock_probe": (ctypes.c_int, [P, i64, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -224,3 +225,9 @@ def engram_get_status(stream=None) -> int:
 
 def engram_device_sm_count() -> int:
     return _check("engram_device_sm_count", lib().engram_device_sm_count())
+
+
+def engram_clock_probe(out, spin_ns: int, stream=None) -> None:
+    """out: device uint64/int64 tensor of 2; afterwards out[0] / out[1] is the
+    mean SM clock in GHz over `spin_ns` of the global timer."""
+    _check("engram_clock_probe", lib().engram_clock_probe(_p(out), spin_ns, _s(stream)))
