@@ -23,6 +23,18 @@ __device__ __forceinline__ uint64_t mod_prime(uint64_t x, uint64_t P, uint64_t m
   return r >= P ? r - P : r;
 }
 
+// One 16-byte piece of a table row.  Rows are read once and 160 or 256 bytes
+// long at 32-byte alignment: no L1 allocation, and the L2 asked to fetch
+// 64-byte sector pairs on a miss instead of whole 128-byte lines (a 160-byte
+// row spans two lines: 256 bytes from DRAM at line granularity, 192 at 64).
+__device__ __forceinline__ uint4 ld_row_piece(const uint4* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::64B.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
 // Compressed id of flat token m, PAD for m < 0; -1 for a raw id out of range.
 __device__ __forceinline__ int32_t token_cid(const int32_t* __restrict__ proj,
                                              const int32_t* __restrict__ ids, int64_t m,
@@ -125,7 +137,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ Hea
         const int c = r - j * CR;
         const int32_t s = __ldg(idx + n * hp.J + j);
         if (s >= 0 && (uint64_t)s < hp.P[j]) {
-          v[u] = __ldg(table + (hp.row_base[j] + s) * CR + c);
+          v[u] = ld_row_piece(table + (hp.row_base[j] + s) * CR + c);
         } else if (s != -1) {
           atomicOr(status, ENGRAM_STATUS_BAD_INDEX);
         }
@@ -177,7 +189,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant_
         v[k][p] = make_uint4(0, 0, 0, 0);
         if (piece < PER_TOK) {
           if (s >= 0 && (uint64_t)s < hp.P[j]) {
-            v[k][p] = __ldg(table + (hp.row_base[j] + s) * CR + c);
+            v[k][p] = ld_row_piece(table + (hp.row_base[j] + s) * CR + c);
           } else if (s != -1) {
             atomicOr(status, ENGRAM_STATUS_BAD_INDEX);
           }
@@ -248,7 +260,7 @@ int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, i
   const int key = hp.J * 100 + CR;
   switch (key) {
     case 4 * 100 + 4: return rows(gather_rows_kernel<4, 4, 8>, 8);     // fp32 rows of 16, 4 heads
-    case 16 * 100 + 10: return rows(gather_rows_kernel<16, 10, 4>, 4);  // bf16 rows of 80
+    case 16 * 100 + 10: return rows(gather_rows_kernel<16, 10, 2>, 2);  // bf16 rows of 80
     case 16 * 100 + 16: return rows(gather_rows_kernel<16, 16, 2>, 2);  // bf16 rows of 128
     case 16 * 100 + 20: return rows(gather_rows_kernel<16, 20, 2>, 2);  // bf16 rows of 160
     default: break;
