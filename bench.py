@@ -282,9 +282,9 @@ def run_ours(args):
     from hashed_gram_conditional_engram_b200 import engram as eg
     from hashed_gram_conditional_engram_b200 import synth
 
-    ws_, rank = dist_init("nccl")
     _, _, local = dist_env()
-    torch.cuda.set_device(local)
+    torch.cuda.set_device(local)  # before the process group, so NCCL binds this GPU
+    ws_, rank = dist_init("nccl")
     dev = torch.device("cuda", local)
     w = synth.workload(WORKLOAD)
 

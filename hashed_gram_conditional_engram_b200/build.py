@@ -60,6 +60,17 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return OUT
     os.makedirs(BUILD, exist_ok=True)
+    # several processes (one per GPU) may ask at once: one builds, the others
+    # wait for it and find the library up to date
+    import fcntl
+    with open(os.path.join(BUILD, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        if not force and up_to_date():
+            return OUT
+        return _build_locked(verbose)
+
+
+def _build_locked(verbose: bool) -> str:
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         results = list(ex.map(lambda s: _compile(s, verbose), sources()))
     if verbose:
