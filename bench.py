@@ -381,37 +381,62 @@ def run_ours(args):
     ms_per_step = elapsed_ms / args.steps
     value = aggregate_rate(N, ws_, args.steps, elapsed_ms)
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers.  Each step
+    # uploads its ids and h from pinned host memory, runs hash + forward and
+    # reads its output back.  Steps are double-buffered over three streams
+    # (upload, compute, download), as a serving loop would run them: PCIe is
+    # full duplex, so step k+1's upload, step k's compute and step k-1's
+    # download overlap.
     ids_h = torch.from_numpy(ids_np).pin_memory()
     h_h = dense["h"].cpu().pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    ids_d = torch.empty_like(ids)
-    h_d = torch.empty_like(dense["h"])
+    out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    ids_d = [torch.empty_like(ids) for _ in range(2)]
+    h_d = [torch.empty_like(dense["h"]) for _ in range(2)]
+    out_d = [torch.empty_like(out) for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
+    for k in range(2):  # every event recorded once, so the first waits pass
+        for ev in (ev_comp[k], ev_down[k]):
+            ev.record(stream)
 
-    def e2e_step():
-        ids_d.copy_(ids_h, non_blocking=True)
-        h_d.copy_(h_h, non_blocking=True)
-        eg.engram_hash_indices(cfg, proj, ids_d, w.B, w.T, None, idx, stream)
-        eg.engram_forward(cfg, idx, table, e, h_d, dense["Wk"], dense["Wv"], dense["conv_w"],
-                          None, out, saved, w.B, w.T, fws, fb, stream)
-        out_h.copy_(out, non_blocking=True)
+    def e2e_step(k):
+        b = k % 2
+        up.wait_event(ev_comp[b])         # step k-2's compute has read h_d[b]
+        with torch.cuda.stream(up):
+            ids_d[b].copy_(ids_h, non_blocking=True)
+            h_d[b].copy_(h_h, non_blocking=True)
+        ev_up[b].record(up)
+        stream.wait_event(ev_up[b])
+        stream.wait_event(ev_down[b])     # step k-2's output has left out_d[b]
+        eg.engram_hash_indices(cfg, proj, ids_d[b], w.B, w.T, None, idx, stream)
+        eg.engram_forward(cfg, idx, table, e, h_d[b], dense["Wk"], dense["Wv"], dense["conv_w"],
+                          None, out_d[b], saved, w.B, w.T, fws, fb, stream)
+        ev_comp[b].record(stream)
+        down.wait_event(ev_comp[b])
+        with torch.cuda.stream(down):
+            out_h[b].copy_(out_d[b], non_blocking=True)
+        ev_down[b].record(down)
 
-    for _ in range(2):
-        e2e_step()
-    e2e_steps = max(3, min(args.steps, 20))
+    for k in range(2):
+        e2e_step(k)
+    e2e_steps = max(4, min(args.steps, 20))
     barrier()
     torch.cuda.synchronize()
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e2.record(stream)
+    s2.record(up)
+    for k in range(e2e_steps):
+        e2e_step(k)
+    e2.record(down)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(s2.elapsed_time(e2))
     e2e_value = aggregate_rate(N, ws_, e2e_steps, e2e_ms)
     h2d = ids_h.numel() * 4 + h_h.numel() * 2
-    d2h = out_h.numel() * 2
+    d2h = out_h[0].numel() * 2
+    if not torch.equal(out_d[(e2e_steps - 1) % 2], out):
+        raise RuntimeError("end-to-end output differs from the device-resident step")
 
     # ---- roofline of the dominant kernel (the two fused tensor-core passes)
     peaks, peak_src = load_peaks()
