@@ -92,10 +92,12 @@ __global__ void gate_f32_kernel(const float* __restrict__ h, const double* __res
 // y = sum_i w[c,i] vt_{t-3+i}, out = h + vt + SiLU(y): one thread per (n, m, c).
 // With conv_state (decode, T == 1) the three earlier vt come from the state,
 // which is then shifted by one step.
-__global__ void conv_f32_kernel(const float* __restrict__ h, const double* __restrict__ v,
+// h and out may be the same buffer (each element is read before it is
+// written, by the same thread), so neither is declared __restrict__.
+__global__ void conv_f32_kernel(const float* h, const double* __restrict__ v,
                                 const double* __restrict__ alpha, const float* __restrict__ w,
                                 float* __restrict__ conv_state, float* __restrict__ y_out,
-                                float* __restrict__ out, int64_t N, int T, int M, int d) {
+                                float* out, int64_t N, int T, int M, int d) {
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= N * M * d) return;
   const int c = (int)(g % d);

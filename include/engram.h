@@ -167,7 +167,10 @@ int engram_gather(const engram_cfg_t* cfg, const int32_t* idx, const void* table
  *   conv_state NULL for whole sequences.  Non-NULL selects decode (T == 1):
  *           device fp32 [B, M, 3, d], vt of the three previous steps, oldest
  *           first, zeros at the start; updated in place.
- *   out     device [B, T, M, d] (cfg->dtype).
+ *   out     device [B, T, M, d] (cfg->dtype); may be h itself (the residual
+ *           applied in place): every read of h precedes the write of the same
+ *           element.  engram_backward needs the original h, so a forward that
+ *           will be differentiated keeps them apart.
  *   saved   device, engram_saved_size bytes, or NULL: what engram_backward needs.
  *   ws      device workspace of engram_workspace_size(cfg, ENGRAM_WS_FORWARD, B*T).
  * bf16: tables, e, h, W, out in bf16; products, gate, conv in fp32; the output

@@ -305,3 +305,37 @@ def test_decode_full_size_sampled():
         assert max_rel_err(conv.cpu().numpy()[sample], conv_ref) <= TOL_BF16, step
     del table, L
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,T,d,dtype", [
+    (3, 100, 256, "bf16"),    # narrow tensor-core tiles
+    (2, 2500, 512, "bf16"),   # wide tiles: pass V overwrites h while later tiles still load it
+    (2, 37, 64, "f32"),       # CUDA-core path
+])
+def test_forward_in_place_equals_separate_output(B, T, d, dtype):
+    """out == h (the residual applied in place) gives bit for bit the output of
+    a run with a separate out buffer."""
+    rng = np.random.default_rng(B * 7 + T)
+    K, D_h = 2, 32 if dtype == "bf16" else 16
+    J, E, N = 2 * K, 2 * K * D_h, B * T
+    rows = synth.primes_at_most(2003, J)
+    tables = [rng.standard_normal((P, D_h)).astype(np.float32) for P in rows]
+    Wk = (rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32)
+    Wv = (rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32)
+    h = rng.standard_normal((B, T, 1, d)).astype(np.float32)
+    conv_w = (rng.standard_normal((d, 4)) * 0.5).astype(np.float32)
+    idx = dev(np.stack([rng.integers(0, P, N) for P in rows], -1).astype(np.int32).reshape(B, T, J))
+    t_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+    put = bf16_dev if dtype == "bf16" else dev
+    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16 if dtype == "bf16" else eg.F32, rows,
+                      np.ones((J, 3), np.uint64))
+    L = Layer(cfg, B, T, packed_table(tables, dtype), put(h), put(Wk), put(Wv), dev(conv_w),
+              t_dtype)
+    sep = L.forward(idx).clone()
+    alpha_sep = _alpha(L, N, 1).copy()
+    L.out = L.h                     # out aliases h
+    L.forward(idx)
+    torch.cuda.synchronize()
+    assert torch.equal(L.h, sep)
+    assert np.array_equal(_alpha(L, N, 1), alpha_sep)
+    assert eg.engram_get_status() == 0
