@@ -239,6 +239,17 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def oracle_sample(w, ids, keys, mult, head_rows_fn, dense_host, n_seq: int, n_tok: int):
     """The oracle end to end (hash, gather, fusion) on the first
     `n_tok` tokens of each of the first `n_seq` sequences of the batch.
@@ -465,7 +476,7 @@ def run_ours(args):
         extras = {}
         if ws_ == 1 and not args.no_extras:
             for name, fn in (("decode", bench_decode), ("hosttable", bench_hosttable),
-                             ("fwd_bwd", bench_train_step)):
+                             ("fwd_bwd", bench_train_step), ("tiny", bench_tiny)):
                 try:
                     extras[name] = fn(dev)
                 except Exception as ex:  # noqa: BLE001 -- reported, not hidden
@@ -522,6 +533,7 @@ def cpu_baseline_ours(w, ids_np, keys_np, mult, table, dense):
 
     tok, sec, thr = oracle_sample(w, ids_np, keys_np, mult, rows_fn, dense_host, n_seq, w.T)
     return {"value": tok / sec, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
             "sample": f"first {n_seq} sequences of the batch ({tok} tokens), oracle end to "
                       f"end in fp64 ({sec:.1f} s)"}
 
@@ -552,6 +564,62 @@ def _graph_time(fn, steps, warmup, stream):
     with torch.cuda.graph(g, stream=stream):
         fn()
     return _time_loop(g.replay, steps, warmup, stream)
+
+
+def bench_tiny(dev):
+    """One fp32 layer (1 x 64 tokens, d 64, 4 heads x 16 dims): hash, forward
+    with the gather, backward with the sparse table gradient, per call."""
+    import torch
+    from hashed_gram_conditional_engram_b200 import engram as eg
+    from hashed_gram_conditional_engram_b200 import synth
+    w = synth.workload("tiny")
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    inp = synth.host_inputs(w)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+    keys = t(inp["keys"])
+    proj = torch.empty(w.V, dtype=torch.int32, device=dev)
+    vb = eg.engram_workspace_size(None, eg.WS_VOCAB, w.V)
+    V_c = eg.engram_build_vocab_proj(keys, w.V, proj, torch.empty(vb, dtype=torch.uint8, device=dev), vb)
+    cfg = eg.make_cfg(w.K, w.D_h, w.d, w.M, w.V, V_c, eg.F32, w.rows, inp["mult"])
+    N, E = w.N, w.E
+    ids, table = t(inp["ids"]), t(np.concatenate([x.reshape(-1) for x in inp["tables"]]))
+    h, Wk, Wv, cw, dout = t(inp["h"]), t(inp["Wk"]), t(inp["Wv"]), t(inp["conv_w"]), t(inp["dout"])
+    idx = torch.empty((w.B, w.T, w.J), dtype=torch.int32, device=dev)
+    e = torch.empty((N, E), device=dev)
+    out = torch.empty((N, w.M, w.d), device=dev)
+    saved = torch.empty(eg.engram_saved_size(cfg, N), dtype=torch.uint8, device=dev)
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+    fws = torch.empty(fb, dtype=torch.uint8, device=dev)
+    bb = eg.engram_workspace_size(cfg, eg.WS_BACKWARD, N)
+    bws = torch.empty(bb, dtype=torch.uint8, device=dev)
+    dh = torch.empty((N, w.M, w.d), device=dev)
+    dWk, dWv = torch.empty((w.M, w.d, E), device=dev), torch.empty((w.d, E), device=dev)
+    dcw = torch.empty((w.d, 4), device=dev)
+    keys_out = torch.empty(N * w.J, dtype=torch.int64, device=dev)
+    rows_out = torch.empty((N * w.J, w.D_h), device=dev)
+    nu = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def fwd():
+        eg.engram_hash_indices(cfg, proj, ids, w.B, w.T, None, idx, s)
+        eg.engram_forward(cfg, idx, table, e, h, Wk, Wv, cw, None, out, saved, w.B, w.T, fws, fb, s)
+
+    def step():
+        fwd()
+        eg.engram_backward(cfg, idx, e, h, Wk, Wv, cw, saved, dout, dh, dWk, dWv, dcw, None,
+                           keys_out, rows_out, nu, w.B, w.T, bws, bb, s)
+
+    with torch.cuda.stream(s):
+        f_eager = _time_loop(fwd, 200, 5, s)
+        fb_eager = _time_loop(step, 200, 5, s)
+        fb_graph = _graph_time(step, 500, 5, s)
+    if eg.engram_get_status(s) != 0:
+        raise RuntimeError("device status word set in the tiny layer")
+    return {"workload": "tiny: 1 x 64 tokens, d 64, K 2 x 1,009 x 16, fp32 (fp64 arithmetic), "
+                        "one layer",
+            "us_per_fwd_call_eager": f_eager * 1e3, "us_per_fwd_bwd_call_eager": fb_eager * 1e3,
+            "us_per_fwd_bwd_graph": fb_graph * 1e3,
+            "fwd_bwd_tokens_per_s": w.N / (fb_graph / 1e3)}
 
 
 def bench_train_step(dev):
@@ -721,6 +789,8 @@ def bench_hosttable(dev, params=8_000_000_000):
     idx = torch.empty((w.B, w.T, w.J), dtype=torch.int32, device=dev)
     eg.engram_hash_indices(cfg, proj, torch.from_numpy(ids_np).to(dev), w.B, w.T, None, idx)
     e = torch.empty((w.N, w.E), dtype=torch.bfloat16, device=dev)
+    idx_np = idx.cpu().numpy().reshape(w.N, w.J)
+    unique_rows = int(sum(len(np.unique(idx_np[:, j])) for j in range(w.J)))
     comp = torch.cuda.current_stream(dev)
     side = torch.cuda.Stream(dev)
     A = torch.randn((w.N, w.d), device=dev).to(torch.bfloat16)
@@ -769,7 +839,9 @@ def bench_hosttable(dev, params=8_000_000_000):
         raise RuntimeError("device status word set in host-table gather")
     return {"workload": f"hosttable: 4 x 2,048 tokens, 16 heads x 160 dims, {sum(rows) * w.D_h / 1e9:.1f}B "
                         "bf16 params in pinned host memory (the 100B table does not fit the host)",
-            "rows_bytes_per_batch": rows_bytes, "gather_ms": t_gather,
+            "rows_bytes_per_batch": rows_bytes,
+            "unique_rows_bytes_per_batch": unique_rows * w.D_h * 2,
+            "gather_ms": t_gather,
             "pcie_gbs": rows_bytes / (t_gather / 1e3) / 1e9, "h2d_memcpy_peak_gbs": h2d_peak,
             "frac_of_h2d_peak": rows_bytes / (t_gather / 1e3) / 1e9 / h2d_peak,
             "gemm_ms_alone": t_gemm, "gemm_ms_with_gather": t_both_gemm,
@@ -830,6 +902,7 @@ def run_reference(args):
                                "1,024 tokens per step", "global_batch": n_tok, "seq_len": w.T,
                    "parallelism": "none (host cores)"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                         "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
                          "sample": "first 1,024 tokens of one sequence per step, end to end "
                                    "in fp64"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,

@@ -105,23 +105,93 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_scatter_kernel(
 }
 
 // Exclusive scan of int32 x[0..n) into y (may alias x), total into *total
-// (if non-null).  One block of 1024 threads: each thread owns a contiguous
-// run, the run sums are scanned across the block.
-__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* x, int32_t* y, int64_t n,
-                                                    int32_t* total) {
-  __shared__ int32_t wsum[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t per = (n + 1023) / 1024;
-  const int64_t lo = tid * per;
-  const int64_t hi = lo + per < n ? lo + per : n;
-  int32_t s = 0;
-  for (int64_t i = lo; i < hi; ++i) s += x[i];
-  // inclusive scan of s over the block
-  int32_t incl = s;
+// (if non-null), in three passes over at most SCAN_MAX_BLOCKS chunks: each
+// block sums its chunk, one block scans the chunk sums, each block scans its
+// chunk from its offset.  Loads and stores are 16-byte vectors of a thread's
+// SCAN_ITEMS consecutive elements.
+constexpr int SCAN_THREADS = 256;
+constexpr int SCAN_ITEMS = 16;
+constexpr int SCAN_TILE = SCAN_THREADS * SCAN_ITEMS;  // 4096 elements
+constexpr int SCAN_MAX_BLOCKS = 1024;
+
+constexpr int64_t scan_chunk(int64_t n) {
+  const int64_t tiles = (n + SCAN_TILE - 1) / SCAN_TILE;
+  const int64_t per_block = (tiles + SCAN_MAX_BLOCKS - 1) / SCAN_MAX_BLOCKS;
+  return (per_block > 0 ? per_block : 1) * SCAN_TILE;
+}
+
+__device__ __forceinline__ void scan_load(const int32_t* x, int64_t n, int64_t base,
+                                          int32_t (&v)[SCAN_ITEMS]) {
+  if (base + SCAN_ITEMS <= n) {
+    const int4* q = reinterpret_cast<const int4*>(x + base);
+#pragma unroll
+    for (int u = 0; u < SCAN_ITEMS / 4; ++u) {
+      const int4 t = q[u];
+      v[4 * u] = t.x;
+      v[4 * u + 1] = t.y;
+      v[4 * u + 2] = t.z;
+      v[4 * u + 3] = t.w;
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < SCAN_ITEMS; ++u) v[u] = base + u < n ? x[base + u] : 0;
+  }
+}
+
+// Sum of the block's SCAN_THREADS values `t`, returned to every thread, and
+// the exclusive prefix of `t` within the block in *excl.
+__device__ __forceinline__ int32_t block_scan(int32_t t, int32_t* excl) {
+  __shared__ int32_t wsum[SCAN_THREADS / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t incl = t;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int32_t t = __shfl_up_sync(FULL, incl, o);
-    if (lane >= o) incl += t;
+    const int32_t u = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int32_t before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < SCAN_THREADS / 32; ++w) {
+    const int32_t s = wsum[w];
+    if (w < warp) before += s;
+    all += s;
+  }
+  __syncthreads();  // wsum is reused by the next call
+  *excl = before + incl - t;
+  return all;
+}
+
+__global__ void __launch_bounds__(SCAN_THREADS) scan_reduce_kernel(const int32_t* x, int64_t n,
+                                                                   int64_t chunk,
+                                                                   int32_t* bsum) {
+  const int64_t lo = (int64_t)blockIdx.x * chunk;
+  const int64_t hi = lo + chunk < n ? lo + chunk : n;
+  int32_t s = 0;
+  for (int64_t t0 = lo; t0 < hi; t0 += SCAN_TILE) {
+    int32_t v[SCAN_ITEMS];
+    scan_load(x, hi, t0 + (int64_t)threadIdx.x * SCAN_ITEMS, v);
+#pragma unroll
+    for (int u = 0; u < SCAN_ITEMS; ++u) s += v[u];
+  }
+  int32_t ex;
+  const int32_t all = block_scan(s, &ex);
+  if (threadIdx.x == 0) bsum[blockIdx.x] = all;
+}
+
+// Exclusive scan of the nblk chunk sums in place (nblk <= SCAN_MAX_BLOCKS);
+// the grand total into *total.
+__global__ void __launch_bounds__(SCAN_MAX_BLOCKS) scan_sums_kernel(int32_t* bsum, int nblk,
+                                                                    int32_t* total) {
+  __shared__ int32_t wsum[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t v = tid < nblk ? bsum[tid] : 0;
+  int32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t u = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += u;
   }
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
@@ -129,28 +199,75 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* x, int32_t* y
     int32_t w = wsum[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int32_t t = __shfl_up_sync(FULL, w, o);
-      if (lane >= o) w += t;
+      const int32_t u = __shfl_up_sync(FULL, w, o);
+      if (lane >= o) w += u;
     }
     wsum[lane] = w;
   }
   __syncthreads();
-  int32_t run = incl - s + (warp > 0 ? wsum[warp - 1] : 0);
-  for (int64_t i = lo; i < hi; ++i) {
-    const int32_t t = x[i];
-    y[i] = run;
-    run += t;
+  const int32_t ex = incl - v + (warp > 0 ? wsum[warp - 1] : 0);
+  if (tid < nblk) bsum[tid] = ex;
+  if (total != nullptr && tid == SCAN_MAX_BLOCKS - 1) *total = ex + v;
+}
+
+__global__ void __launch_bounds__(SCAN_THREADS) scan_apply_kernel(const int32_t* x, int32_t* y,
+                                                                  int64_t n, int64_t chunk,
+                                                                  const int32_t* bsum) {
+  const int64_t lo = (int64_t)blockIdx.x * chunk;
+  const int64_t hi = lo + chunk < n ? lo + chunk : n;
+  int32_t carry = bsum[blockIdx.x];
+  for (int64_t t0 = lo; t0 < hi; t0 += SCAN_TILE) {
+    const int64_t base = t0 + (int64_t)threadIdx.x * SCAN_ITEMS;
+    int32_t v[SCAN_ITEMS];
+    scan_load(x, hi, base, v);
+    int32_t s = 0;
+#pragma unroll
+    for (int u = 0; u < SCAN_ITEMS; ++u) s += v[u];
+    int32_t ex;
+    const int32_t all = block_scan(s, &ex);
+    int32_t run = carry + ex;
+#pragma unroll
+    for (int u = 0; u < SCAN_ITEMS; ++u) {
+      const int32_t t = v[u];
+      v[u] = run;
+      run += t;
+    }
+    if (base + SCAN_ITEMS <= hi) {
+      int4* q = reinterpret_cast<int4*>(y + base);
+#pragma unroll
+      for (int u = 0; u < SCAN_ITEMS / 4; ++u)
+        q[u] = make_int4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < SCAN_ITEMS; ++u)
+        if (base + u < hi) y[base + u] = v[u];
+    }
+    carry += all;
   }
-  if (total != nullptr && tid == 1023) *total = run;
+}
+
+constexpr size_t scan_ws_bytes() { return up256((SCAN_MAX_BLOCKS + 1) * 4); }
+
+// x and y 16-byte aligned; bsum: scan_ws_bytes() of workspace.
+int launch_scan(const int32_t* x, int32_t* y, int64_t n, int32_t* total, int32_t* bsum,
+                cudaStream_t s) {
+  if (n <= 0) return total != nullptr ? ck(cudaMemsetAsync(total, 0, sizeof(int32_t), s)) : 0;
+  const int64_t chunk = scan_chunk(n);
+  const int nblk = (int)((n + chunk - 1) / chunk);
+  scan_reduce_kernel<<<nblk, SCAN_THREADS, 0, s>>>(x, n, chunk, bsum);
+  scan_sums_kernel<<<1, SCAN_MAX_BLOCKS, 0, s>>>(bsum, nblk, total);
+  scan_apply_kernel<<<nblk, SCAN_THREADS, 0, s>>>(x, y, n, chunk, bsum);
+  return ck(cudaGetLastError());
 }
 
 int radix_sort_pairs(uint64_t*& keys, uint32_t*& vals, uint64_t* keys_alt, uint32_t* vals_alt,
-                     int64_t n, int key_bits, int32_t* hist, cudaStream_t s) {
+                     int64_t n, int key_bits, int32_t* hist, int32_t* bsum, cudaStream_t s) {
   if (n == 0) return ENGRAM_OK;
   const int64_t nblocks = (n + TILE - 1) / TILE;
   for (int shift = 0; shift < key_bits; shift += RADIX_BITS) {
     radix_hist_kernel<<<(unsigned)nblocks, SORT_THREADS, 0, s>>>(keys, n, shift, hist);
-    scan_kernel<<<1, 1024, 0, s>>>(hist, hist, (int64_t)RADIX * nblocks, nullptr);
+    const int rc = launch_scan(hist, hist, (int64_t)RADIX * nblocks, nullptr, bsum, s);
+    if (rc) return rc;
     radix_scatter_kernel<<<(unsigned)nblocks, SORT_THREADS, 0, s>>>(keys, vals, n, shift, hist,
                                                                     keys_alt, vals_alt);
     uint64_t* tk = keys;
@@ -210,22 +327,71 @@ __global__ void tg_heads_kernel(const uint64_t* __restrict__ keys, int64_t n, ui
   if (last_valid) seg_start[ex[p] + (head ? 1 : 0)] = (int32_t)(p + 1);
 }
 
-// One thread per (row, dimension): fp32 sum from +0 over the row's items in
-// sorted (= ascending token) order.  de of item i = n*J + j starts at
-// i * D_h because E = J * D_h.
+// de of item i = n*J + j starts at i * D_h because E = J * D_h.
+//
+// One thread per (unique row, group of 4 dimensions): the row's de segments
+// added in sorted (= ascending token) order, from +0, in fp32, each of the 4
+// dimensions on its own (16-byte loads; D_h is a multiple of 4).  The order
+// of the adds is fixed; the loads are not: a thread takes TG_U items at once
+// so that their first loads overlap, and walks a long segment (a frequent
+// n-gram) with TG_PF loads issued ahead of the adds.
+constexpr int TG_U = 4;
+constexpr int TG_PF = 8;
+__device__ __forceinline__ void add4(float4& a, const float4 x) {
+  a.x = a.x + x.x;
+  a.y = a.y + x.y;
+  a.z = a.z + x.z;
+  a.w = a.w + x.w;
+}
 __global__ void tg_reduce_kernel(const int32_t* __restrict__ seg_start,
-                                 const uint32_t* __restrict__ vals, const float* __restrict__ de,
-                                 const int32_t* __restrict__ n_unique, int D_h,
-                                 float* __restrict__ rows) {
-  const int64_t total = (int64_t)(*n_unique) * D_h;
+                                 const uint32_t* __restrict__ vals, const float4* __restrict__ de,
+                                 const int32_t* __restrict__ n_unique, int D4,
+                                 float4* __restrict__ rows) {
+  const int64_t total = (int64_t)(*n_unique) * D4;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total; g += stride) {
-    const int64_t u = g / D_h;
-    const int c = (int)(g - u * D_h);
-    const int32_t b = seg_start[u], e = seg_start[u + 1];
-    float acc = 0.0f;
-    for (int32_t p = b; p < e; ++p) acc = acc + __ldg(de + (int64_t)vals[p] * D_h + c);
-    rows[g] = acc;
+  for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g0 < total;
+       g0 += stride * TG_U) {
+    int64_t gg[TG_U];
+    int cc[TG_U];
+    int32_t bb[TG_U], ee[TG_U];
+#pragma unroll
+    for (int k = 0; k < TG_U; ++k) {
+      gg[k] = g0 + k * stride;
+      bb[k] = ee[k] = 0;
+      cc[k] = 0;
+      if (gg[k] < total) {
+        const int64_t u = gg[k] / D4;
+        cc[k] = (int)(gg[k] - u * D4);
+        bb[k] = seg_start[u];
+        ee[k] = seg_start[u + 1];
+      }
+    }
+    uint32_t it[TG_U];
+#pragma unroll
+    for (int k = 0; k < TG_U; ++k) it[k] = bb[k] < ee[k] ? __ldg(vals + bb[k]) : 0u;
+    float4 x[TG_U];
+#pragma unroll
+    for (int k = 0; k < TG_U; ++k)
+      x[k] = bb[k] < ee[k] ? __ldg(de + (int64_t)it[k] * D4 + cc[k]) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < TG_U; ++k) {
+      if (gg[k] >= total) continue;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (bb[k] < ee[k]) add4(acc, x[k]);
+      int32_t p = bb[k] + 1;
+      for (; p + TG_PF <= ee[k]; p += TG_PF) {
+        uint32_t iq[TG_PF];
+#pragma unroll
+        for (int q = 0; q < TG_PF; ++q) iq[q] = __ldg(vals + p + q);
+        float4 xq[TG_PF];
+#pragma unroll
+        for (int q = 0; q < TG_PF; ++q) xq[q] = __ldg(de + (int64_t)iq[q] * D4 + cc[k]);
+#pragma unroll
+        for (int q = 0; q < TG_PF; ++q) add4(acc, xq[q]);
+      }
+      for (; p < ee[k]; ++p) add4(acc, __ldg(de + (int64_t)vals[p] * D4 + cc[k]));
+      rows[gg[k]] = acc;
+    }
   }
 }
 
@@ -285,13 +451,14 @@ struct SortWs {
   int32_t* a;   // n int32
   int32_t* b;   // n int32
   int32_t* c;   // n + 1 int32
+  int32_t* bsum;  // chunk sums of the scans
   int32_t* scal;  // 4 int32
 };
 
 constexpr size_t sort_ws_bytes(int64_t n) {
   const int64_t nblocks = (n + TILE - 1) / TILE;
   return 2 * up256(n * 8) + 2 * up256(n * 4) + up256(RADIX * nblocks * 4 + 4) +
-         2 * up256(n * 4 + 4) + up256((n + 1) * 4) + 256;
+         2 * up256(n * 4 + 4) + up256((n + 1) * 4) + scan_ws_bytes() + 256;
 }
 
 SortWs carve(void* ws, int64_t n) {
@@ -306,11 +473,124 @@ SortWs carve(void* ws, int64_t n) {
   w.a = reinterpret_cast<int32_t*>(p); p += up256(n * 4 + 4);
   w.b = reinterpret_cast<int32_t*>(p); p += up256(n * 4 + 4);
   w.c = reinterpret_cast<int32_t*>(p); p += up256((n + 1) * 4);
+  w.bsum = reinterpret_cast<int32_t*>(p); p += scan_ws_bytes();
   w.scal = reinterpret_cast<int32_t*>(p);
   return w;
 }
 
 }  // namespace
+
+// The whole table gradient in one block for up to TG_SMALL_MAX items (a
+// short sequence, a training step on a small batch): the items' (row id,
+// item) keys are sorted in shared memory by a bitonic network (the item index
+// in the low bits keeps equal rows in ascending token order, as the stable
+// radix sort does), segment heads are counted by a block scan, and each
+// (row, 4 dimensions) sums its segment in that order from +0.  The same sums
+// as the multi-kernel path, bit for bit, in one launch instead of ~27.
+constexpr int TG_SMALL_MAX = 2048;   // 24 KB of static shared memory
+constexpr int TG_SMALL_THREADS = 1024;
+constexpr int TG_ITEM_BITS = 12;  // item index < 2^12
+
+__global__ void __launch_bounds__(TG_SMALL_THREADS) tg_small_kernel(
+    const __grid_constant__ HeadParams hp, const int32_t* __restrict__ idx, int n,
+    uint64_t sentinel, const float4* __restrict__ de, int D4, int64_t* __restrict__ keys_out,
+    float4* __restrict__ rows_out, int32_t* __restrict__ n_unique) {
+  __shared__ uint64_t sk[TG_SMALL_MAX];
+  __shared__ int32_t seg[TG_SMALL_MAX + 1];
+  __shared__ int32_t wsum[TG_SMALL_THREADS / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int np2 = 1;
+  while (np2 < n) np2 <<= 1;
+  for (int i = tid; i < np2; i += TG_SMALL_THREADS) {
+    uint64_t key = ~0ull;  // padding sorts last
+    if (i < n) {
+      const int j = i % hp.J;
+      const int32_t sl = idx[i];
+      const uint64_t row = (sl >= 0 && (uint64_t)sl < hp.P[j]) ? (uint64_t)(hp.row_base[j] + sl)
+                                                                : sentinel;
+      key = (row << TG_ITEM_BITS) | (uint64_t)i;
+    }
+    sk[i] = key;
+  }
+  __syncthreads();
+  for (int k = 2; k <= np2; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = tid; i < np2; i += TG_SMALL_THREADS) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const uint64_t a = sk[i], b = sk[ixj];
+          const bool up = (i & k) == 0;
+          if ((a > b) == up) {
+            sk[i] = b;
+            sk[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // segment heads over sorted positions, 4 consecutive positions per thread
+  constexpr int PER = TG_SMALL_MAX / TG_SMALL_THREADS;
+  int heads = 0, valid = 0;
+  bool hd[PER];
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int p = tid * PER + q;
+    hd[q] = false;
+    if (p < n) {
+      const uint64_t row = sk[p] >> TG_ITEM_BITS;
+      if (row != sentinel) {
+        ++valid;
+        hd[q] = p == 0 || (sk[p - 1] >> TG_ITEM_BITS) != row;
+        heads += hd[q] ? 1 : 0;
+      }
+    }
+  }
+  int incl = heads, vincl = valid;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(FULL, incl, o), b = __shfl_up_sync(FULL, vincl, o);
+    if (lane >= o) {
+      incl += a;
+      vincl += b;
+    }
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int before = 0, all = 0;
+  for (int w = 0; w < TG_SMALL_THREADS / 32; ++w) {
+    if (w < warp) before += wsum[w];
+    all += wsum[w];
+  }
+  __syncthreads();
+  if (lane == 31) wsum[warp] = vincl;
+  __syncthreads();
+  int n_valid = 0;
+  for (int w = 0; w < TG_SMALL_THREADS / 32; ++w) n_valid += wsum[w];
+  int h = before + incl - heads;  // exclusive count of heads before this thread's run
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    if (hd[q]) {
+      const int p = tid * PER + q;
+      seg[h] = p;
+      keys_out[h] = (int64_t)(sk[p] >> TG_ITEM_BITS);
+      ++h;
+    }
+  }
+  if (tid == 0) {
+    seg[all] = n_valid;  // valid items sort first: they end where the sentinel rows begin
+    *n_unique = all;
+  }
+  __syncthreads();
+  constexpr uint64_t ITEM_MASK = (1ull << TG_ITEM_BITS) - 1;
+  for (int g = tid; g < all * D4; g += TG_SMALL_THREADS) {
+    const int u = g / D4, c = g - u * D4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p = seg[u]; p < seg[u + 1]; ++p)
+      add4(acc, __ldg(de + (int64_t)(sk[p] & ITEM_MASK) * D4 + c));
+    rows_out[g] = acc;
+  }
+}
 
 size_t table_grad_ws_bytes(int64_t n_items) { return sort_ws_bytes(n_items); }
 
@@ -320,23 +600,33 @@ int launch_table_grad(const HeadParams& hp, const int32_t* idx, const float* de,
   const int64_t n = n_tok * hp.J;
   if (ws_bytes < sort_ws_bytes(n)) return ENGRAM_ERR_WORKSPACE;
   if (n == 0) return ck(cudaMemsetAsync(n_unique, 0, sizeof(int32_t), s));
-  SortWs w = carve(ws, n);
   const uint64_t sentinel = (uint64_t)(hp.row_base[hp.J - 1] + (int64_t)hp.P[hp.J - 1]);
+  if (n <= TG_SMALL_MAX) {
+    tg_small_kernel<<<1, TG_SMALL_THREADS, 0, s>>>(
+        hp, idx, (int)n, sentinel, reinterpret_cast<const float4*>(de), hp.D_h / 4, keys_out,
+        reinterpret_cast<float4*>(rows_out), n_unique);
+    return ck(cudaGetLastError());
+  }
+  SortWs w = carve(ws, n);
   tg_items_kernel<<<nb(n), 256, 0, s>>>(hp, idx, n, sentinel, w.k0, w.v0);
   uint64_t* k = w.k0;
   uint32_t* v = w.v0;
-  int rc = radix_sort_pairs(k, v, w.k1, w.v1, n, bits_for(sentinel), w.hist, s);
+  int rc = radix_sort_pairs(k, v, w.k1, w.v1, n, bits_for(sentinel), w.hist, w.bsum, s);
   if (rc) return rc;
   tg_flags_kernel<<<nb(n), 256, 0, s>>>(k, n, sentinel, w.a);
-  scan_kernel<<<1, 1024, 0, s>>>(w.a, w.b, n, n_unique);
+  rc = launch_scan(w.a, w.b, n, n_unique, w.bsum, s);
+  if (rc) return rc;
   // seg_start needs n_unique + 1 entries; with no valid item it stays empty
   tg_heads_kernel<<<nb(n), 256, 0, s>>>(k, n, sentinel, w.b, w.c, keys_out);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t blocks = nb(n * hp.D_h);
+  const int D4 = hp.D_h / 4;  // D_h * 4 bytes is a multiple of 16 (checked with the config)
+  int64_t blocks = nb(n * D4);
   if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-  tg_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(w.c, v, de, n_unique, hp.D_h, rows_out);
+  tg_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(w.c, v, reinterpret_cast<const float4*>(de),
+                                                    n_unique, D4,
+                                                    reinterpret_cast<float4*>(rows_out));
   return ck(cudaGetLastError());
 }
 
@@ -405,16 +695,18 @@ int launch_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_
   vb_items_kernel<<<nb(V), 256, 0, s>>>(keys, V, w.k0, w.v0);
   uint64_t* k = w.k0;
   uint32_t* v = w.v0;
-  int rc = radix_sort_pairs(k, v, w.k1, w.v1, V, 64, w.hist, s);
+  int rc = radix_sort_pairs(k, v, w.k1, w.v1, V, 64, w.hist, w.bsum, s);
   if (rc) return rc;
   vb_flags_kernel<<<nb(V), 256, 0, s>>>(k, V, w.a);
-  scan_kernel<<<1, 1024, 0, s>>>(w.a, w.b, V, w.scal);
+  rc = launch_scan(w.a, w.b, V, w.scal, w.bsum, s);
+  if (rc) return rc;
   // w.c: first raw id of each group, then reused below
   vb_first_kernel<<<nb(V), 256, 0, s>>>(k, v, V, w.a, w.b, w.c);
   int32_t* rep = reinterpret_cast<int32_t*>(k == w.k0 ? w.k1 : w.k0);  // free after the sort
   vb_rep_kernel<<<nb(V), 256, 0, s>>>(v, V, w.a, w.b, w.c, rep);
   vb_isfirst_kernel<<<nb(V), 256, 0, s>>>(rep, V, w.a);
-  scan_kernel<<<1, 1024, 0, s>>>(w.a, w.b, V, w.scal + 1);
+  rc = launch_scan(w.a, w.b, V, w.scal + 1, w.bsum, s);
+  if (rc) return rc;
   vb_proj_kernel<<<nb(V), 256, 0, s>>>(rep, w.b, V, proj);
   int32_t vc = 0;
   int e = ck(cudaMemcpyAsync(&vc, w.scal + 1, sizeof(int32_t), cudaMemcpyDeviceToHost, s));

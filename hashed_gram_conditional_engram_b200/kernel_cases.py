@@ -8,12 +8,15 @@ without the rest of the layer's inputs on the device.
     python -m hashed_gram_conditional_engram_b200.kernel_cases hash [...]
     python -m hashed_gram_conditional_engram_b200.kernel_cases decode \
         --tokens 256 --d 4096 --dh 128 --rows 1000003
+    python -m hashed_gram_conditional_engram_b200.kernel_cases tablegrad [...]
 
 `fused` runs engram_forward with table = NULL on random gathered rows, i.e.
 the two tensor-core passes; `gather` gathers from a table of --rows rows per
 head; `hash` runs the compress + n-gram + hash kernel; `decode` runs whole
 decode steps (hash with rolling n-gram state, then engram_forward with the
-table and the conv state) for --tokens sequences of one token each.  Defaults are the
+table and the conv state) for --tokens sequences of one token each;
+`tablegrad` runs the sparse table gradient (sort by row, segment sums) on
+fp32 rows of de for hash indices of Zipf(1.1) token ids.  Defaults are the
 27B-shaped layer's dimensions.  Prints the device time per repetition.
 """
 from __future__ import annotations
@@ -29,7 +32,7 @@ from . import synth
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["fused", "gather", "hash", "decode"])
+    ap.add_argument("kernel", choices=["fused", "gather", "hash", "decode", "tablegrad"])
     ap.add_argument("--tokens", type=int, default=32768)
     ap.add_argument("--seq", type=int, default=4096)
     ap.add_argument("--d", type=int, default=2560)
@@ -78,6 +81,27 @@ def main(argv=None):
 
         def run():
             eg.engram_gather(cfg, idx, table, N, e)
+    elif a.kernel == "tablegrad":
+        ids_np, keys_np = synth.host_ids_keys(synth.workload("layer27b"))
+        keys = torch.from_numpy(keys_np).to(dev)
+        proj = torch.empty(129280, dtype=torch.int32, device=dev)
+        vb = eg.engram_workspace_size(None, eg.WS_VOCAB, 129280)
+        eg.engram_build_vocab_proj(keys, 129280, proj, torch.empty(vb, dtype=torch.uint8, device=dev), vb)
+        cfg32 = eg.make_cfg(K, a.dh, a.d, 1, 129280, synth.compressed_vocab(129280), eg.F32, rows,
+                            mult)
+        ids = torch.from_numpy(ids_np.reshape(-1)[:N].copy()).to(dev)
+        idx = torch.empty((N, a.heads), dtype=torch.int32, device=dev)
+        eg.engram_hash_indices(cfg32, proj, ids, B, T, None, idx)
+        de = torch.randn((N, E), generator=g, device=dev)
+        n_items = N * a.heads
+        keys_out = torch.empty(n_items, dtype=torch.int64, device=dev)
+        rows_out = torch.empty((n_items, a.dh), device=dev)
+        nu = torch.zeros(1, dtype=torch.int32, device=dev)
+        nb = eg.engram_workspace_size(cfg32, eg.WS_TABLE_GRAD, N)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+
+        def run():
+            eg.engram_table_grad(cfg32, idx, de, N, keys_out, rows_out, nu, ws, nb)
     elif a.kernel == "decode":
         table = torch.empty(sum(rows) * a.dh, dtype=torch.bfloat16, device=dev)
         table.normal_(0.0, 0.02, generator=g)

@@ -74,21 +74,32 @@ def test_hash_empty_batch():
 
 
 def test_hash_decode_state_bit_exact():
+    """All 2,000 decode steps of the decode workload (256 sequences): the
+    indices of every step and the rolling n-gram state bit-exact."""
     w = synth.workload("decode")
     ids, keys = synth.host_ids_keys(w)          # [steps, B]
-    steps = 200
+    steps = w.steps
     mult = synth.hash_multipliers(synth.layer_seed(w, 0), w.J)
     proj_ref, V_c = O.build_vocab_proj(keys)
     proj, _ = gpu_vocab_proj(keys)
     cfg = cfg_of(w, mult, V_c)
+    state = dev(np.full((w.B, 2), V_c, dtype=np.int32))
+    ids_d = dev(ids)
+    idx_all = torch.empty((steps, w.B, 1, w.J), dtype=torch.int32, device="cuda")
+    mid_state = None
+    for s in range(steps):
+        eg.engram_hash_indices(cfg, proj, ids_d[s], w.B, 1, state, idx_all[s])
+        if s == steps // 2:
+            mid_state = state.cpu().numpy()
+    got = idx_all.cpu().numpy()[:, :, 0]
     state_ref = np.full((w.B, 2), V_c, dtype=np.int32)
-    state = dev(state_ref.copy())
     for s in range(steps):
         want, state_ref = O.hash_indices_decode(proj_ref, ids[s], state_ref, mult,
                                                 np.array(w.rows), w.K)
-        got = gpu_hash(cfg, proj, dev(ids[s].copy()), w.B, 1, state=state)
-        assert np.array_equal(got.cpu().numpy()[:, 0], want), s
-        assert np.array_equal(state.cpu().numpy(), state_ref), s
+        assert np.array_equal(got[s], want), s
+        if s == steps // 2:
+            assert np.array_equal(mid_state, state_ref)
+    assert np.array_equal(state.cpu().numpy(), state_ref)
 
 
 def test_hash_bad_ids_flag_and_minus_one():
