@@ -9,6 +9,8 @@ without the rest of the layer's inputs on the device.
     python -m hashed_gram_conditional_engram_b200.kernel_cases decode \
         --tokens 256 --d 4096 --dh 128 --rows 1000003
     python -m hashed_gram_conditional_engram_b200.kernel_cases tablegrad [...]
+    python -m hashed_gram_conditional_engram_b200.kernel_cases hostgather \
+        --tokens 8192 --seq 2048 --dh 160 --rows 1000003
 
 `fused` runs engram_forward with table = NULL on random gathered rows, i.e.
 the two tensor-core passes; `gather` gathers from a table of --rows rows per
@@ -16,7 +18,8 @@ head; `hash` runs the compress + n-gram + hash kernel; `decode` runs whole
 decode steps (hash with rolling n-gram state, then engram_forward with the
 table and the conv state) for --tokens sequences of one token each;
 `tablegrad` runs the sparse table gradient (sort by row, segment sums) on
-fp32 rows of de for hash indices of Zipf(1.1) token ids.  Defaults are the
+fp32 rows of de for hash indices of Zipf(1.1) token ids; `hostgather` runs
+engram_forward_hosttable on a table in pinned host memory.  Defaults are the
 27B-shaped layer's dimensions.  Prints the device time per repetition.
 """
 from __future__ import annotations
@@ -32,7 +35,8 @@ from . import synth
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["fused", "gather", "hash", "decode", "tablegrad"])
+    ap.add_argument("kernel", choices=["fused", "gather", "hash", "decode", "tablegrad",
+                                       "hostgather"])
     ap.add_argument("--tokens", type=int, default=32768)
     ap.add_argument("--seq", type=int, default=4096)
     ap.add_argument("--d", type=int, default=2560)
@@ -81,6 +85,23 @@ def main(argv=None):
 
         def run():
             eg.engram_gather(cfg, idx, table, N, e)
+    elif a.kernel == "hostgather":
+        n_el = sum(rows) * a.dh
+        host = torch.empty(n_el, dtype=torch.bfloat16, pin_memory=True)
+        buf = torch.empty(1 << 28, dtype=torch.bfloat16, device=dev)
+        for lo in range(0, n_el, 1 << 28):
+            hi = min(n_el, lo + (1 << 28))
+            buf[: hi - lo].normal_(0.0, 0.02, generator=g)
+            host[lo:hi].copy_(buf[: hi - lo])
+        del buf
+        rng = np.random.default_rng(3)
+        idx = torch.from_numpy(np.stack([rng.integers(0, P, N) for P in rows], -1)
+                               .astype(np.int32)).to(dev)
+        e = torch.empty((N, E), dtype=torch.bfloat16, device=dev)
+        side = torch.cuda.current_stream()
+
+        def run():
+            eg.engram_forward_hosttable(cfg, idx, host.data_ptr(), N, e, side, None)
     elif a.kernel == "tablegrad":
         ids_np, keys_np = synth.host_ids_keys(synth.workload("layer27b"))
         keys = torch.from_numpy(keys_np).to(dev)
