@@ -476,7 +476,8 @@ def run_ours(args):
         extras = {}
         if ws_ == 1 and not args.no_extras:
             for name, fn in (("decode", bench_decode), ("hosttable", bench_hosttable),
-                             ("fwd_bwd", bench_train_step), ("tiny", bench_tiny)):
+                             ("fwd_bwd", bench_train_step), ("tiny", bench_tiny),
+                             ("fwd_bwd_27b", bench_fwd_bwd_27b)):
                 try:
                     extras[name] = fn(dev)
                 except Exception as ex:  # noqa: BLE001 -- reported, not hidden
@@ -564,6 +565,78 @@ def _graph_time(fn, steps, warmup, stream):
     with torch.cuda.graph(g, stream=stream):
         fn()
     return _time_loop(g.replay, steps, warmup, stream)
+
+
+def bench_fwd_bwd_27b(dev, steps=10):
+    """Training step of the 27B-shaped layer (8 x 4,096 tokens, d 2,560, 16 x
+    80 dims, 5.7B-parameter bf16 table): hash, forward (gather, fused passes,
+    alpha saved), backward (bf16: elementwise kernels, cuBLAS GEMMs, sparse
+    table gradient)."""
+    import torch
+    from hashed_gram_conditional_engram_b200 import engram as eg
+    from hashed_gram_conditional_engram_b200 import synth
+    w = synth.workload(WORKLOAD)
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    ids_np, keys_np = synth.host_ids_keys(w)
+    mult = synth.hash_multipliers(synth.layer_seed(w, 0), w.J)
+    table = synth.device_table(w, device=dev)
+    dense = synth.device_dense(w, device=dev)
+    keys = torch.from_numpy(keys_np).to(dev)
+    proj = torch.empty(w.V, dtype=torch.int32, device=dev)
+    vb = eg.engram_workspace_size(None, eg.WS_VOCAB, w.V)
+    V_c = eg.engram_build_vocab_proj(keys, w.V, proj, torch.empty(vb, dtype=torch.uint8, device=dev), vb)
+    cfg = eg.make_cfg(w.K, w.D_h, w.d, 1, w.V, V_c, eg.BF16, w.rows, mult)
+    N, E = w.N, w.E
+    ids = torch.from_numpy(ids_np).to(dev)
+    idx = torch.empty((w.B, w.T, w.J), dtype=torch.int32, device=dev)
+    e = torch.empty((N, E), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((N, 1, w.d), dtype=torch.bfloat16, device=dev)
+    saved = torch.empty(eg.engram_saved_size(cfg, N), dtype=torch.uint8, device=dev)
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+    fws = torch.empty(fb, dtype=torch.uint8, device=dev)
+    bb = eg.engram_workspace_size(cfg, eg.WS_BACKWARD, N)
+    bws = torch.empty(bb, dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(27)
+    dout = torch.randn((N, 1, w.d), generator=g, device=dev)
+    dh = torch.empty((N, 1, w.d), device=dev)
+    dWk, dWv = torch.empty((1, w.d, E), device=dev), torch.empty((w.d, E), device=dev)
+    dcw = torch.empty((w.d, 4), device=dev)
+    keys_out = torch.empty(N * w.J, dtype=torch.int64, device=dev)
+    rows_out = torch.empty((N * w.J, w.D_h), device=dev)
+    nu = torch.zeros(1, dtype=torch.int32, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+
+    def step(mark=False):
+        if mark:
+            ev[0].record(s)
+        eg.engram_hash_indices(cfg, proj, ids, w.B, w.T, None, idx, s)
+        eg.engram_forward(cfg, idx, table, e, dense["h"], dense["Wk"], dense["Wv"],
+                          dense["conv_w"], None, out, saved, w.B, w.T, fws, fb, s)
+        if mark:
+            ev[1].record(s)
+        eg.engram_backward(cfg, idx, e, dense["h"], dense["Wk"], dense["Wv"], dense["conv_w"],
+                           saved, dout, dh, dWk, dWv, dcw, None, keys_out, rows_out, nu,
+                           w.B, w.T, bws, bb, s)
+        if mark:
+            ev[2].record(s)
+
+    with torch.cuda.stream(s):
+        ms = _time_loop(step, steps, 3, s)
+        step(mark=True)
+        torch.cuda.synchronize()
+    if eg.engram_get_status(s) != 0:
+        raise RuntimeError("device status word set in the 27B-shaped training step")
+    bwd_flops = 2.0 * N * E * w.d * 6   # k, v recomputed; dW_k, dW_v; two GEMMs for de
+    t_bwd = ev[1].elapsed_time(ev[2])
+    del table, dense, bws, fws
+    torch.cuda.empty_cache()
+    return {"workload": "layer27b training step: 8 x 4,096 tokens, d 2,560, 16 heads x 80 dims, "
+                        "5.7B bf16 params; forward (hash, gather, fused passes) + bf16 backward",
+            "fwd_bwd_tokens_per_s": N / (ms / 1e3), "ms_per_step": ms,
+            "breakdown_ms": {"forward": ev[0].elapsed_time(ev[1]), "backward": t_bwd},
+            "backward_gemm_tflops": bwd_flops / (t_bwd / 1e3) / 1e12}
 
 
 def bench_tiny(dev):

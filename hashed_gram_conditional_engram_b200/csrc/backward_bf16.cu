@@ -1,0 +1,340 @@
+// Backward of the bf16 layer (one branch) at full scale.
+//
+// The four dense contractions of the backward are plain GEMMs with no work
+// to fuse into them: k and v are recomputed as e W_k^T and e W_v^T, the
+// weight gradients are contractions over tokens (dW = d{k,v}^T e) and the
+// row gradient is de = dk W_k + dv W_v.  They run in cuBLAS (bf16 operands,
+// fp32 accumulation), loaded with dlopen on first use so that the library
+// itself has no load-time dependency on it.  Everything between them -- the
+// conv and SiLU backward, the gate, both RMSNorm backwards -- is in the
+// kernels below, and the table rows' gradient goes through the same
+// deterministic sort-and-segment-sum as the fp32 path.
+//
+// Method: discuss.deepseek.club 二.1 (2) (gate with h as query, e as key and
+// value; 1-D conv; residual); gitcode.csdn.net blog, end-to-end training
+// paragraph (deterministic lookups give consistent gradients to the slots).
+#include <cublas_v2.h>
+#include <dlfcn.h>
+
+#include <mutex>
+
+#include "internal.cuh"
+
+namespace engram {
+
+namespace {
+
+// ------------------------------------------------------------ cuBLAS, loaded late
+
+struct Blas {
+  bool ok = false;
+  cublasStatus_t (*create)(cublasHandle_t*) = nullptr;
+  cublasStatus_t (*set_stream)(cublasHandle_t, cudaStream_t) = nullptr;
+  cublasStatus_t (*set_workspace)(cublasHandle_t, void*, size_t) = nullptr;
+  cublasStatus_t (*gemm_ex)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int,
+                            const void*, const void*, cudaDataType, int, const void*, cudaDataType,
+                            int, const void*, void*, cudaDataType, int, cublasComputeType_t,
+                            cublasGemmAlgo_t) = nullptr;
+};
+
+Blas& blas() {
+  static Blas b;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* h = dlopen("libcublas.so.12", RTLD_NOW | RTLD_LOCAL);
+    if (h == nullptr) return;
+    b.create = reinterpret_cast<decltype(b.create)>(dlsym(h, "cublasCreate_v2"));
+    b.set_stream = reinterpret_cast<decltype(b.set_stream)>(dlsym(h, "cublasSetStream_v2"));
+    b.set_workspace =
+        reinterpret_cast<decltype(b.set_workspace)>(dlsym(h, "cublasSetWorkspace_v2"));
+    b.gemm_ex = reinterpret_cast<decltype(b.gemm_ex)>(dlsym(h, "cublasGemmEx"));
+    b.ok = b.create && b.set_stream && b.set_workspace && b.gemm_ex;
+  });
+  return b;
+}
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kBlasWorkspace = 32u << 20;  // from the caller's workspace
+
+// One handle per device, created on first use and kept for the process.
+int blas_handle(cudaStream_t s, void* workspace, cublasHandle_t* out) {
+  static cublasHandle_t handles[kMaxDevices] = {};
+  static std::mutex mu;
+  Blas& b = blas();
+  if (!b.ok) return ENGRAM_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ENGRAM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(mu);
+  if (handles[dev] == nullptr && b.create(&handles[dev]) != CUBLAS_STATUS_SUCCESS) {
+    handles[dev] = nullptr;
+    return ENGRAM_ERR_CUDA;
+  }
+  if (b.set_stream(handles[dev], s) != CUBLAS_STATUS_SUCCESS ||
+      b.set_workspace(handles[dev], workspace, kBlasWorkspace) != CUBLAS_STATUS_SUCCESS)
+    return ENGRAM_ERR_CUDA;
+  *out = handles[dev];
+  return ENGRAM_OK;
+}
+
+// C[m x n] (row-major, fp32) = alpha * op(A)[m x k] . op(B)[k x n] + beta * C
+// with A, B bf16 row-major: op(A) = A (a_t = false, A is [m x k]) or A^T (A
+// is [k x m]); likewise B.  Row-major C = A.B is column-major C^T = B^T.A^T,
+// which is what cuBLAS is asked for.
+int gemm_rm(cublasHandle_t hd, bool a_t, bool b_t, int m, int n, int k, const void* A,
+            const void* B, float* C, float beta) {
+  const float alpha = 1.0f;
+  const int lda = a_t ? m : k;  // row length of A as stored
+  const int ldb = b_t ? k : n;
+  const cublasOperation_t opB = b_t ? CUBLAS_OP_T : CUBLAS_OP_N;
+  const cublasOperation_t opA = a_t ? CUBLAS_OP_T : CUBLAS_OP_N;
+  const cublasStatus_t st =
+      blas().gemm_ex(hd, opB, opA, n, m, k, &alpha, B, CUDA_R_16BF, ldb, A, CUDA_R_16BF, lda,
+                     &beta, C, CUDA_R_32F, n, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+  return st == CUBLAS_STATUS_SUCCESS ? ENGRAM_OK : ENGRAM_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ elementwise backward
+//
+// Notation per token t and feature f (u = dout):
+//   vt = alpha v, y_t = sum_i w_i vt_{t-3+i} (zero before the sequence start),
+//   out = h + vt + SiLU(y)
+//   dy_t = u_t SiLU'(y_t),  SiLU'(y) = s (1 + y (1 - s)), s = sigmoid(y)
+//   dvt_t = u_t + sum_{s = t..t+3, same sequence} w_{3-(s-t)} dy_s
+//   dalpha = <dvt, v>, dv = alpha dvt, dz = dalpha alpha (1 - alpha)
+//   dh^ = dz k^ / sqrt(d), dk^ = dz h^ / sqrt(d)   (h^ = r_h h, k^ = r_k k)
+//   RMSNorm backward: dx = r dx^ - r^3 x <dx^, x> / d, where
+//   <dh^, h> = dz r_k <k, h> / sqrt(d) and <dk^, k> = dz r_h <h, k> / sqrt(d)
+//   dh = u + r_h dh^ - r_h^3 h <dh^, h> / d,  dk = r_k dk^ - r_k^3 k <dk^, k> / d
+//   dw_i = sum_t dy_t vt_{t-3+i}
+
+__device__ __forceinline__ float silu_grad(float y) {
+  const float sg = 1.0f / (1.0f + __expf(-y));
+  return sg * (1.0f + y * (1.0f - sg));
+}
+
+// dy for every (token, feature); thread per element, features fastest.
+__global__ void bw_dy_kernel(const float* __restrict__ v, const float* __restrict__ alpha,
+                             const float4* __restrict__ conv_w, const float* __restrict__ dout,
+                             int64_t N, int T, int d, float* __restrict__ dy) {
+  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= N * d) return;
+  const int64_t t = g / d;
+  const int f = (int)(g - t * d);
+  const int pos = (int)(t % T);
+  const float4 w = __ldg(conv_w + f);
+  const float taps[4] = {w.x, w.y, w.z, w.w};
+  float y = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int back = 3 - i;  // tap i multiplies vt_{t - back}
+    if (back <= pos) y = fmaf(taps[i], alpha[t - back] * v[(t - back) * d + f], y);
+  }
+  dy[g] = dout[g] * silu_grad(y);
+}
+
+constexpr int ROW_THREADS = 256;
+constexpr float BW_RMS_EPS = 1e-6f;  // the forward's RMSNorm epsilon
+
+// Sum of a value over the block, the same order on every run.
+__device__ __forceinline__ float block_sum(float x, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();  // red is reused
+  if (lane == 0) red[warp] = x;
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < ROW_THREADS / 32; ++i) s += red[i];
+  return s;
+}
+
+// dvt of token t, feature f (the conv's transpose plus the direct residual).
+__device__ __forceinline__ float dvt_of(const float* __restrict__ dout,
+                                        const float* __restrict__ dy, float4 w, int64_t t, int f,
+                                        int d, int left) {
+  // left = tokens after t in its sequence
+  const float taps[4] = {w.x, w.y, w.z, w.w};
+  float g = dout[t * d + f];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)  // s = t + k uses tap 3 - k
+    if (k <= left) g = fmaf(taps[3 - k], dy[(t + k) * d + f], g);
+  return g;
+}
+
+// One block per token: the gate and both RMSNorm backwards, which need
+// whole-row sums, then dv and dk (bf16, for the weight and row GEMMs) and dh.
+__global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
+    const __nv_bfloat16* __restrict__ h, const float* __restrict__ k, const float* __restrict__ v,
+    const float* __restrict__ alpha, const float4* __restrict__ conv_w,
+    const float* __restrict__ dout, const float* __restrict__ dy, int64_t N, int T, int d,
+    float* __restrict__ dh, __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out) {
+  __shared__ float red[ROW_THREADS / 32];
+  const int64_t t = blockIdx.x;
+  if (t >= N) return;
+  const int left = T - 1 - (int)(t % T);
+  const __nv_bfloat16* hr = h + t * d;
+  const float* kr = k + t * d;
+  const float* vr = v + t * d;
+  float shh = 0.f, skk = 0.f, shk = 0.f, sgv = 0.f;
+  for (int f = threadIdx.x; f < d; f += ROW_THREADS) {
+    const float hv = __bfloat162float(hr[f]), kv = kr[f];
+    shh = fmaf(hv, hv, shh);
+    skk = fmaf(kv, kv, skk);
+    shk = fmaf(hv, kv, shk);
+    sgv = fmaf(dvt_of(dout, dy, __ldg(conv_w + f), t, f, d, left), vr[f], sgv);
+  }
+  shh = block_sum(shh, red);
+  skk = block_sum(skk, red);
+  shk = block_sum(shk, red);
+  sgv = block_sum(sgv, red);
+  const float invd = 1.0f / (float)d, isd = rsqrtf((float)d);
+  const float rh = rsqrtf(shh * invd + BW_RMS_EPS), rk = rsqrtf(skk * invd + BW_RMS_EPS);
+  const float a = alpha[t];
+  const float dz = sgv * a * (1.0f - a);
+  const float c = dz * isd;                          // dh^ = c k^, dk^ = c h^
+  const float dot_h = c * rk * shk;                  // <dh^, h>
+  const float dot_k = c * rh * shk;                  // <dk^, k>
+  const float ch = rh * rh * rh * dot_h * invd, ck = rk * rk * rk * dot_k * invd;
+  for (int f = threadIdx.x; f < d; f += ROW_THREADS) {
+    const float hv = __bfloat162float(hr[f]), kv = kr[f];
+    const float g = dvt_of(dout, dy, __ldg(conv_w + f), t, f, d, left);
+    dv_out[t * d + f] = __float2bfloat16_rn(a * g);
+    dk_out[t * d + f] = __float2bfloat16_rn(rk * (c * rh * hv) - ck * kv);
+    dh[t * d + f] = dout[t * d + f] + rh * (c * rk * kv) - ch * hv;
+  }
+}
+
+constexpr int DCONV_TOK = 256;  // tokens per partial
+
+// Partial conv-weight gradients: block (chunk of DCONV_TOK tokens, 128
+// features); each thread walks its feature through the chunk with the three
+// previous vt in registers.  part[chunk][f][i].
+__global__ void __launch_bounds__(128) bw_dconv_partial_kernel(
+    const float* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ dy,
+    int64_t N, int T, int d, float4* __restrict__ part) {
+  const int f = blockIdx.y * 128 + threadIdx.x;
+  if (f >= d) return;
+  const int64_t t0 = (int64_t)blockIdx.x * DCONV_TOK;
+  const int64_t t1 = t0 + DCONV_TOK < N ? t0 + DCONV_TOK : N;
+  float s1 = 0.f, s2 = 0.f, s3 = 0.f;  // vt of t-1, t-2, t-3
+  {
+    const int pos = (int)(t0 % T);
+    if (pos >= 1) s1 = alpha[t0 - 1] * v[(t0 - 1) * d + f];
+    if (pos >= 2) s2 = alpha[t0 - 2] * v[(t0 - 2) * d + f];
+    if (pos >= 3) s3 = alpha[t0 - 3] * v[(t0 - 3) * d + f];
+  }
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  for (int64_t t = t0; t < t1; ++t) {
+    if (t % T == 0) s1 = s2 = s3 = 0.f;
+    const float vt = alpha[t] * v[t * d + f];
+    const float g = dy[t * d + f];
+    a0 = fmaf(g, s3, a0);  // tap 0 multiplies vt_{t-3}
+    a1 = fmaf(g, s2, a1);
+    a2 = fmaf(g, s1, a2);
+    a3 = fmaf(g, vt, a3);
+    s3 = s2;
+    s2 = s1;
+    s1 = vt;
+  }
+  part[(int64_t)blockIdx.x * d + f] = make_float4(a0, a1, a2, a3);
+}
+
+// dconv_w[f] = sum over chunks in order.
+__global__ void bw_dconv_reduce_kernel(const float4* __restrict__ part, int chunks, int d,
+                                       float4* __restrict__ dw) {
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f >= d) return;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = 0; c < chunks; ++c) {
+    const float4 p = part[(int64_t)c * d + f];
+    s.x += p.x;
+    s.y += p.y;
+    s.z += p.z;
+    s.w += p.w;
+  }
+  dw[f] = s;
+}
+
+// Workspace: k, v, dy fp32 [N, d]; dk, dv bf16 [N, d]; de fp32 [N, E] when
+// the caller passes none; conv partials; cuBLAS's workspace; the table
+// gradient's sort buffers.
+struct BwdBf16Ws {
+  float *k, *v, *dy, *de;
+  __nv_bfloat16 *dk, *dv;
+  float4* part;
+  void* blas_ws;
+  void* tg_ws;
+  size_t tg_bytes;
+};
+
+constexpr size_t up256b(size_t b) { return (b + 255) & ~(size_t)255; }
+
+size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, BwdBf16Ws* w) {
+  const int64_t chunks = (N + DCONV_TOK - 1) / DCONV_TOK;
+  const size_t Nd4 = up256b((size_t)N * d * 4), Nd2 = up256b((size_t)N * d * 2);
+  const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
+  const size_t tg = table_grad_ws_bytes(N * J);
+  char* p = static_cast<char*>(base);
+  if (w != nullptr) {
+    w->k = reinterpret_cast<float*>(p);
+    w->v = reinterpret_cast<float*>(p + Nd4);
+    w->dy = reinterpret_cast<float*>(p + 2 * Nd4);
+    w->dk = reinterpret_cast<__nv_bfloat16*>(p + 3 * Nd4);
+    w->dv = reinterpret_cast<__nv_bfloat16*>(p + 3 * Nd4 + Nd2);
+    w->de = reinterpret_cast<float*>(p + 3 * Nd4 + 2 * Nd2);
+    w->part = reinterpret_cast<float4*>(p + 3 * Nd4 + 2 * Nd2 + NE4);
+    w->blas_ws = p + 3 * Nd4 + 2 * Nd2 + NE4 + P;
+    w->tg_ws = p + 3 * Nd4 + 2 * Nd2 + NE4 + P + kBlasWorkspace;
+    w->tg_bytes = tg;
+  }
+  return 3 * Nd4 + 2 * Nd2 + NE4 + P + kBlasWorkspace + tg;
+}
+
+}  // namespace
+
+size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J) {
+  return bwd_bf16_layout(nullptr, N, d, E, J, nullptr);
+}
+
+int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bfloat16* e,
+                         const __nv_bfloat16* h, const __nv_bfloat16* Wk,
+                         const __nv_bfloat16* Wv, const float* conv_w, const float* alpha,
+                         const float* dout, float* dh, float* dWk, float* dWv, float* dconv_w,
+                         float* de, int64_t* dtab_keys, float* dtab_rows, int32_t* n_unique,
+                         int64_t N, int T, int d, void* ws, size_t ws_bytes, cudaStream_t s) {
+  const int E = hp.E;
+  if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J)) return ENGRAM_ERR_WORKSPACE;
+  if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
+  BwdBf16Ws w;
+  bwd_bf16_layout(ws, N, d, E, hp.J, &w);
+  if (de == nullptr) de = w.de;
+  cublasHandle_t hd;
+  int rc = blas_handle(s, w.blas_ws, &hd);
+  if (rc) return rc;
+  const int n = (int)N;
+  // k = e W_k^T, v = e W_v^T (fp32)
+  if ((rc = gemm_rm(hd, false, true, n, d, E, e, Wk, w.k, 0.f))) return rc;
+  if ((rc = gemm_rm(hd, false, true, n, d, E, e, Wv, w.v, 0.f))) return rc;
+  const int64_t Nd = N * d;
+  bw_dy_kernel<<<(unsigned)((Nd + 255) / 256), 256, 0, s>>>(
+      w.v, alpha, reinterpret_cast<const float4*>(conv_w), dout, N, T, d, w.dy);
+  bw_row_kernel<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.k, w.v, alpha,
+                                                    reinterpret_cast<const float4*>(conv_w), dout,
+                                                    w.dy, N, T, d, dh, w.dk, w.dv);
+  const int chunks = (int)((N + DCONV_TOK - 1) / DCONV_TOK);
+  bw_dconv_partial_kernel<<<dim3((unsigned)chunks, (unsigned)((d + 127) / 128)), 128, 0, s>>>(
+      w.v, alpha, w.dy, N, T, d, w.part);
+  bw_dconv_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(
+      w.part, chunks, d, reinterpret_cast<float4*>(dconv_w));
+  if ((rc = ck(cudaGetLastError()))) return rc;
+  // dW_k = dk^T e, dW_v = dv^T e (contractions over tokens); de = dk W_k + dv W_v
+  if ((rc = gemm_rm(hd, true, false, d, E, n, w.dk, e, dWk, 0.f))) return rc;
+  if ((rc = gemm_rm(hd, true, false, d, E, n, w.dv, e, dWv, 0.f))) return rc;
+  if ((rc = gemm_rm(hd, false, false, n, E, d, w.dk, Wk, de, 0.f))) return rc;
+  if ((rc = gemm_rm(hd, false, false, n, E, d, w.dv, Wv, de, 1.f))) return rc;
+  // the table rows' gradient from de, in the deterministic order
+  return launch_table_grad(hp, idx, de, N, dtab_keys, dtab_rows, n_unique, w.tg_ws, w.tg_bytes, s);
+}
+
+}  // namespace engram

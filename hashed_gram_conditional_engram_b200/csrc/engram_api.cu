@@ -105,6 +105,7 @@ size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n) {
       if (cfg->dtype == ENGRAM_F32) return f32_forward_ws_bytes(n, M, d);
       return tc_forward_ws_bytes(n, d, E);
     case ENGRAM_WS_BACKWARD:
+      if (cfg->dtype == ENGRAM_BF16) return backward_bf16_ws_bytes(n, d, E, 2 * cfg->K);
       return backward_f32_ws_bytes(n, M, d, E) + table_grad_ws_bytes(n * 2 * cfg->K);
     case ENGRAM_WS_TABLE_GRAD:
       return table_grad_ws_bytes(n * 2 * cfg->K);
@@ -200,7 +201,8 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                     void* ws, size_t ws_bytes, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (cfg->dtype != ENGRAM_F32) return ENGRAM_ERR_UNSUPPORTED;
+  if (cfg->dtype == ENGRAM_BF16 && (cfg->n_branch != 1 || saved == nullptr))
+    return cfg->n_branch != 1 ? ENGRAM_ERR_UNSUPPORTED : ENGRAM_ERR_INVALID_ARG;
   if (B < 0 || T < 0) return ENGRAM_ERR_INVALID_ARG;
   const int64_t N = (int64_t)B * T;
   if (idx == nullptr || e == nullptr || h == nullptr || Wk == nullptr || Wv == nullptr ||
@@ -218,6 +220,19 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
   cudaStream_t s = (cudaStream_t)stream;
   const HeadParams hp = make_head_params(cfg);
   const int M = cfg->n_branch, d = cfg->d_model, E = hp.E;
+  if (cfg->dtype == ENGRAM_BF16) {
+    if (N == 0) {  // no tokens: zero weight gradients, no rows
+      if ((rc = ck(cudaMemsetAsync(dWk, 0, (size_t)d * E * 4, s)))) return rc;
+      if ((rc = ck(cudaMemsetAsync(dWv, 0, (size_t)d * E * 4, s)))) return rc;
+      if ((rc = ck(cudaMemsetAsync(dconv_w, 0, (size_t)d * 16, s)))) return rc;
+      return ck(cudaMemsetAsync(n_unique, 0, sizeof(int32_t), s));
+    }
+    using bf = __nv_bfloat16;
+    return launch_backward_bf16(hp, idx, static_cast<const bf*>(e), static_cast<const bf*>(h),
+                                static_cast<const bf*>(Wk), static_cast<const bf*>(Wv), conv_w,
+                                saved, dout, dh, dWk, dWv, dconv_w, de, dtab_keys, dtab_rows,
+                                n_unique, N, T, d, ws, ws_bytes, s);
+  }
   const size_t bw = backward_f32_ws_bytes(N, M, d, E);
   // de lives in the dense-backward workspace unless the caller wants it
   float* de_buf = de != nullptr ? de : backward_f32_de_slot(ws, N, M, d, E);

@@ -171,3 +171,146 @@ def test_backward_is_deterministic():
         assert torch.equal(g1[k], g2[k]), k
     assert torch.equal(g1["keys"][:U], g2["keys"][:U])
     assert torch.equal(g1["rows"][:U], g2["rows"][:U])
+
+
+# ---------------------------------------------------------------- bf16 layers
+
+TOL_BF16 = 2e-2
+
+
+def _bf16_backward_case(B, T, d, K, D_h, seed):
+    """A unit-scale bf16 layer (tables N(0,1), W N(0,1/E)): GPU forward then
+    backward, and the oracle's fp64 backward on the same bf16 values."""
+    from tests.engram_cases import bf16_bits, bf16_dev
+    rng = np.random.default_rng(seed)
+    J, E, N = 2 * K, 2 * K * D_h, B * T
+    rows = synth.primes_at_most(2003, J)
+    tables = [rng.standard_normal((P, D_h)).astype(np.float32) for P in rows]
+    Wk = (rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32)
+    Wv = (rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32)
+    h = rng.standard_normal((B, T, 1, d)).astype(np.float32)
+    conv_w = (rng.standard_normal((d, 4)) * 0.5).astype(np.float32)
+    dout = rng.standard_normal((N, 1, d)).astype(np.float32)
+    idx = np.stack([rng.integers(0, P, N) for P in rows], -1).astype(np.int32)
+    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((J, 3), np.uint64))
+    L = Layer(cfg, B, T, packed_table(tables, "bf16"), bf16_dev(h), bf16_dev(Wk), bf16_dev(Wv),
+              dev(conv_w), torch.bfloat16)
+    idx_d = dev(idx.reshape(B, T, J))
+    L.forward(idx_d)
+    g = L.backward(idx_d, dev(dout))
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    f64 = O.bf16_bits_to_f64
+    e_ref = f64(O.gather(idx, [synth.to_bf16_bits(t) for t in tables]))
+    assert np.array_equal(bf16_bits(L.e), O.gather(idx, [synth.to_bf16_bits(t) for t in tables]))
+    ref = O.layer_backward(e_ref, f64(synth.to_bf16_bits(h)).reshape(N, 1, d),
+                           f64(synth.to_bf16_bits(Wk)), f64(synth.to_bf16_bits(Wv)), conv_w, T,
+                           dout)
+    ref["e"] = e_ref
+    ref["Wk_bf"] = f64(synth.to_bf16_bits(Wk))
+    ref["Wv_bf"] = f64(synth.to_bf16_bits(Wv))
+    return g, ref, idx, rows, D_h
+
+
+# The gradients that leave the elementwise kernels (dh, dconv_w) are held to
+# the bf16 forward's metric.  dW_k, dW_v and de come out of GEMMs whose
+# operands dk and dv are rounded to bf16 once (relative error <= 2^-9 each)
+# and accumulated in fp32: an element's error is then bounded by 2^-9 times
+# the sum of the absolute products that form it, not by its own size (which
+# cancellation can make arbitrarily small).  Each element is checked against
+# twice that bound, computed from the oracle's own dk and dv.
+GEMM_REL = 2.0 ** -8
+
+
+def _within_gemm_bound(got, want, bound):
+    excess = np.abs(got - want) - (GEMM_REL * bound + 1e-6 * np.abs(want).max())
+    return float(excess.max()) <= 0.0
+
+
+@pytest.mark.parametrize("B,T,d,K,D_h", [
+    (3, 100, 256, 2, 32),     # narrow forward tiles, sequences of 100
+    (2, 2500, 512, 2, 32),    # wide forward tiles
+])
+def test_backward_bf16_matches_oracle(B, T, d, K, D_h):
+    g, ref, idx, rows, D_h = _bf16_backward_case(B, T, d, K, D_h, seed=B * 31 + T)
+    for name in ("dh", "dconv_w"):
+        err = max_rel_err(g[name].cpu().numpy(), ref[name])
+        assert err <= TOL_BF16, (name, err)
+    adk, adv, ae = np.abs(ref["dk"][:, 0, :]), np.abs(ref["dv"]), np.abs(ref["e"])
+    assert _within_gemm_bound(g["dWk"].cpu().numpy()[0], ref["dWk"][0], adk.T @ ae)
+    assert _within_gemm_bound(g["dWv"].cpu().numpy(), ref["dWv"], adv.T @ ae)
+    assert _within_gemm_bound(g["de"].cpu().numpy(), ref["de"],
+                              adk @ np.abs(ref["Wk_bf"][0]) + adv @ np.abs(ref["Wv_bf"]))
+    # and in norm, all three within the bf16 tolerance
+    for name in ("dWk", "dWv", "de"):
+        a, b = g[name].cpu().numpy().reshape(ref[name].shape), ref[name]
+        assert np.linalg.norm(a - b) <= TOL_BF16 * np.linalg.norm(b), name
+    # the sparse table gradient: keys bit-exact, rows within the bf16
+    # tolerance of the oracle's, and bit-exact against the deterministic
+    # reduction applied to the GPU's own de
+    keys_ref, rows_ref = O.table_grad_segments_fast(idx, ref["de"].astype(np.float32), rows, D_h)
+    U = int(g["n_unique"].item())
+    assert U == keys_ref.size
+    assert np.array_equal(g["keys"][:U].cpu().numpy(), keys_ref)
+    a = g["rows"][:U].cpu().numpy()
+    assert np.linalg.norm(a - rows_ref) <= TOL_BF16 * np.linalg.norm(rows_ref)
+    keys_own, rows_own = O.table_grad_segments_fast(idx, g["de"].cpu().numpy(), rows, D_h)
+    assert np.array_equal(g["rows"][:U].cpu().numpy().view(np.uint32), rows_own.view(np.uint32))
+
+
+def test_backward_bf16_is_deterministic():
+    a, _, _, _, _ = _bf16_backward_case(2, 300, 256, 2, 32, seed=9)
+    b, _, _, _, _ = _bf16_backward_case(2, 300, 256, 2, 32, seed=9)
+    for name in ("dh", "dWk", "dWv", "dconv_w", "de"):
+        assert torch.equal(a[name], b[name]), name
+    U = int(a["n_unique"].item())
+    assert torch.equal(a["rows"][:U], b["rows"][:U])
+
+
+def test_backward_bf16_layer27b_full_size():
+    """The 27B-shaped layer at full size (8 x 4,096 tokens, d 2,560, 16 heads
+    x 80 dims, 5.7B-parameter table): forward then backward on the device,
+    every gradient against the oracle's fp64 backward on the same bf16
+    values, the table gradient's keys bit-exact and its sums bit-exact on the
+    GPU's own de."""
+    from tests.engram_cases import bf16_bits
+    w = synth.workload("layer27b")
+    ids, keys = synth.host_ids_keys(w)
+    mult = synth.hash_multipliers(synth.layer_seed(w, 0), w.J)
+    proj_ref, V_c = O.build_vocab_proj(keys)
+    idx_ref = O.hash_indices(proj_ref, ids, mult, np.array(w.rows), w.K, V_c).reshape(-1, w.J)
+    table = synth.device_table(w)
+    dense = synth.device_dense(w)
+    cfg = cfg_of(w, mult, V_c)
+    proj, _ = gpu_vocab_proj(keys)
+    idx = gpu_hash(cfg, proj, dev(ids), w.B, w.T)
+    L = Layer(cfg, w.B, w.T, table, dense["h"], dense["Wk"], dense["Wv"], dense["conv_w"],
+              torch.bfloat16)
+    L.forward(idx)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(27)
+    dout = torch.randn((w.N, 1, w.d), generator=gen, device="cuda")
+    g = L.backward(idx, dout)
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    f64 = O.bf16_bits_to_f64
+    e = f64(bf16_bits(L.e))
+    Wk, Wv = f64(bf16_bits(dense["Wk"])), f64(bf16_bits(dense["Wv"]))
+    ref = O.layer_backward(e, f64(bf16_bits(dense["h"])).reshape(w.N, 1, w.d), Wk, Wv,
+                           dense["conv_w"].cpu().numpy(), w.T, dout.cpu().numpy())
+    for name in ("dh", "dconv_w"):
+        err = max_rel_err(g[name].cpu().numpy(), ref[name])
+        assert err <= TOL_BF16, (name, err)
+    adk, adv, ae = np.abs(ref["dk"][:, 0, :]), np.abs(ref["dv"]), np.abs(e)
+    assert _within_gemm_bound(g["dWk"].cpu().numpy()[0], ref["dWk"][0], adk.T @ ae)
+    assert _within_gemm_bound(g["dWv"].cpu().numpy(), ref["dWv"], adv.T @ ae)
+    assert _within_gemm_bound(g["de"].cpu().numpy(), ref["de"],
+                              adk @ np.abs(Wk[0]) + adv @ np.abs(Wv))
+    keys_ref, _ = O.table_grad_segments_fast(idx_ref, ref["de"].astype(np.float32), w.rows, w.D_h)
+    U = int(g["n_unique"].item())
+    assert U == keys_ref.size
+    assert np.array_equal(g["keys"][:U].cpu().numpy(), keys_ref)
+    _, rows_own = O.table_grad_segments_fast(idx_ref, g["de"].cpu().numpy(), w.rows, w.D_h)
+    assert np.array_equal(g["rows"][:U].cpu().numpy().view(np.uint32), rows_own.view(np.uint32))
+    del table, dense, L, g
+    torch.cuda.empty_cache()
