@@ -81,7 +81,7 @@ int blas_handle(cudaStream_t s, void* workspace, cublasHandle_t* out) {
 // is [k x m]); likewise B.  Row-major C = A.B is column-major C^T = B^T.A^T,
 // which is what cuBLAS is asked for.
 int gemm_rm(cublasHandle_t hd, bool a_t, bool b_t, int m, int n, int k, const void* A,
-            const void* B, float* C, float beta) {
+            const void* B, void* C, float beta, cudaDataType c_type = CUDA_R_32F) {
   const float alpha = 1.0f;
   const int lda = a_t ? m : k;  // row length of A as stored
   const int ldb = b_t ? k : n;
@@ -89,7 +89,7 @@ int gemm_rm(cublasHandle_t hd, bool a_t, bool b_t, int m, int n, int k, const vo
   const cublasOperation_t opA = a_t ? CUBLAS_OP_T : CUBLAS_OP_N;
   const cublasStatus_t st =
       blas().gemm_ex(hd, opB, opA, n, m, k, &alpha, B, CUDA_R_16BF, ldb, A, CUDA_R_16BF, lda,
-                     &beta, C, CUDA_R_32F, n, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+                     &beta, C, c_type, n, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
   return st == CUBLAS_STATUS_SUCCESS ? ENGRAM_OK : ENGRAM_ERR_CUDA;
 }
 
@@ -112,26 +112,6 @@ __device__ __forceinline__ float silu_grad(float y) {
   return sg * (1.0f + y * (1.0f - sg));
 }
 
-// dy for every (token, feature); thread per element, features fastest.
-__global__ void bw_dy_kernel(const float* __restrict__ v, const float* __restrict__ alpha,
-                             const float4* __restrict__ conv_w, const float* __restrict__ dout,
-                             int64_t N, int T, int d, float* __restrict__ dy) {
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= N * d) return;
-  const int64_t t = g / d;
-  const int f = (int)(g - t * d);
-  const int pos = (int)(t % T);
-  const float4 w = __ldg(conv_w + f);
-  const float taps[4] = {w.x, w.y, w.z, w.w};
-  float y = 0.f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int back = 3 - i;  // tap i multiplies vt_{t - back}
-    if (back <= pos) y = fmaf(taps[i], alpha[t - back] * v[(t - back) * d + f], y);
-  }
-  dy[g] = dout[g] * silu_grad(y);
-}
-
 constexpr int ROW_THREADS = 256;
 constexpr float BW_RMS_EPS = 1e-6f;  // the forward's RMSNorm epsilon
 
@@ -149,40 +129,121 @@ __device__ __forceinline__ float block_sum(float x, float* red) {
   return s;
 }
 
-// dvt of token t, feature f (the conv's transpose plus the direct residual).
-__device__ __forceinline__ float dvt_of(const float* __restrict__ dout,
-                                        const float* __restrict__ dy, float4 w, int64_t t, int f,
-                                        int d, int left) {
-  // left = tokens after t in its sequence
-  const float taps[4] = {w.x, w.y, w.z, w.w};
-  float g = dout[t * d + f];
+constexpr int COL_TOK = 128;      // tokens per column chunk
+constexpr int COL_THREADS = 128;  // features per block
+
+// One thread per (feature, chunk of COL_TOK tokens), walking the chunk in
+// token order with the three previous vt, dy and dout in registers.  At token
+// t it forms y_t and dy_t.  dvt of token t-3 is complete then (its vt enters
+// y_{t-3} .. y_t), or earlier when its sequence ends; the walk runs 3 tokens
+// past the chunk for those dy.  `live` counts the ring's tokens that belong
+// to t's sequence and lie in this chunk's walk.  Also writes the chunk's
+// partial conv-weight gradient part[chunk][f] = sum over its tokens of
+// dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).
+__global__ void __launch_bounds__(COL_THREADS) bw_col_kernel(
+    const float* __restrict__ v, const float* __restrict__ alpha,
+    const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
+    float* __restrict__ dvt, float4* __restrict__ part) {
+  const int f = blockIdx.y * COL_THREADS + threadIdx.x;
+  if (f >= d) return;
+  const int64_t t0 = (int64_t)blockIdx.x * COL_TOK;
+  const int64_t t1 = t0 + COL_TOK < N ? t0 + COL_TOK : N;
+  const int64_t t_stop = t1 + 3 < N ? t1 + 3 : N;
+  const float4 w = __ldg(conv_w + f);
+  int pos = (int)(t0 % T);
+  float s1 = 0.f, s2 = 0.f, s3 = 0.f;  // vt of t-1, t-2, t-3 (zero before the sequence start)
+  if (pos >= 1) s1 = alpha[t0 - 1] * v[(t0 - 1) * d + f];
+  if (pos >= 2) s2 = alpha[t0 - 2] * v[(t0 - 2) * d + f];
+  if (pos >= 3) s3 = alpha[t0 - 3] * v[(t0 - 3) * d + f];
+  float g1 = 0.f, g2 = 0.f, g3 = 0.f;  // dy of t-1, t-2, t-3
+  float u1 = 0.f, u2 = 0.f, u3 = 0.f;  // dout of t-1, t-2, t-3
+  int live = 0;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  // the next PF tokens' v (already times alpha) and dout, loaded ahead of
+  // the walk so that their latency overlaps the steps before them
+  constexpr int PF = 4;
+  float pv[PF], pu[PF];
 #pragma unroll
-  for (int k = 0; k < 4; ++k)  // s = t + k uses tap 3 - k
-    if (k <= left) g = fmaf(taps[3 - k], dy[(t + k) * d + f], g);
-  return g;
+  for (int q = 0; q < PF; ++q) {
+    const int64_t tq = t0 + q;
+    pv[q] = tq < t_stop ? alpha[tq] * v[tq * d + f] : 0.f;
+    pu[q] = tq < t_stop ? dout[tq * d + f] : 0.f;
+  }
+  for (int64_t t = t0; t < t_stop; ++t) {
+    const float vt = pv[0], ut = pu[0];
+#pragma unroll
+    for (int q = 0; q < PF - 1; ++q) {
+      pv[q] = pv[q + 1];
+      pu[q] = pu[q + 1];
+    }
+    const int64_t tn = t + PF;
+    pv[PF - 1] = tn < t_stop ? alpha[tn] * v[tn * d + f] : 0.f;
+    pu[PF - 1] = tn < t_stop ? dout[tn * d + f] : 0.f;
+    if (pos == 0) {  // a sequence starts at t
+      s1 = s2 = s3 = 0.f;
+      live = 0;
+    }
+    const float y = fmaf(w.x, s3, fmaf(w.y, s2, fmaf(w.z, s1, w.w * vt)));
+    const float gt = ut * silu_grad(y);
+    if (t < t1) {
+      a0 = fmaf(gt, s3, a0);
+      a1 = fmaf(gt, s2, a1);
+      a2 = fmaf(gt, s1, a2);
+      a3 = fmaf(gt, vt, a3);
+    }
+    if (live == 3 && t - 3 >= t0)
+      dvt[(t - 3) * d + f] = u3 + w.w * g3 + w.z * g2 + w.y * g1 + w.x * gt;
+    if (pos == T - 1) {  // the sequence ends at t: its last tokens are complete
+      if (live >= 2 && t - 2 >= t0 && t - 2 < t1)
+        dvt[(t - 2) * d + f] = u2 + w.w * g2 + w.z * g1 + w.y * gt;
+      if (live >= 1 && t - 1 >= t0 && t - 1 < t1) dvt[(t - 1) * d + f] = u1 + w.w * g1 + w.z * gt;
+      if (t < t1) dvt[t * d + f] = ut + w.w * gt;
+    }
+    s3 = s2;
+    s2 = s1;
+    s1 = vt;
+    g3 = g2;
+    g2 = g1;
+    g1 = gt;
+    u3 = u2;
+    u2 = u1;
+    u1 = ut;
+    live = live < 3 ? live + 1 : 3;
+    pos = pos + 1 == T ? 0 : pos + 1;
+  }
+  if (t1 > t0) part[(int64_t)blockIdx.x * d + f] = make_float4(a0, a1, a2, a3);
 }
 
-// One block per token: the gate and both RMSNorm backwards, which need
-// whole-row sums, then dv and dk (bf16, for the weight and row GEMMs) and dh.
+constexpr int ROW_MAX_ITEMS = 16;  // d <= ROW_THREADS * ROW_MAX_ITEMS = 4,096
+
+// One block per token: the gate and both RMSNorm backwards need whole-row
+// sums; the row's h, k, v, dvt are read once into registers, summed, then
+// dv and dk (bf16, for the GEMMs) and dh are written.
 __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
-    const __nv_bfloat16* __restrict__ h, const float* __restrict__ k, const float* __restrict__ v,
-    const float* __restrict__ alpha, const float4* __restrict__ conv_w,
-    const float* __restrict__ dout, const float* __restrict__ dy, int64_t N, int T, int d,
-    float* __restrict__ dh, __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out) {
+    const __nv_bfloat16* __restrict__ h, const float* __restrict__ k,
+    const float* __restrict__ v, const float* __restrict__ alpha,
+    const float* __restrict__ dout, const float* __restrict__ dvt, int64_t N, int d,
+    float* __restrict__ dh,
+    __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out) {
   __shared__ float red[ROW_THREADS / 32];
   const int64_t t = blockIdx.x;
   if (t >= N) return;
-  const int left = T - 1 - (int)(t % T);
-  const __nv_bfloat16* hr = h + t * d;
-  const float* kr = k + t * d;
-  const float* vr = v + t * d;
+  const int64_t r0 = t * d;
+  float hv[ROW_MAX_ITEMS], kv[ROW_MAX_ITEMS], gv[ROW_MAX_ITEMS];
   float shh = 0.f, skk = 0.f, shk = 0.f, sgv = 0.f;
-  for (int f = threadIdx.x; f < d; f += ROW_THREADS) {
-    const float hv = __bfloat162float(hr[f]), kv = kr[f];
-    shh = fmaf(hv, hv, shh);
-    skk = fmaf(kv, kv, skk);
-    shk = fmaf(hv, kv, shk);
-    sgv = fmaf(dvt_of(dout, dy, __ldg(conv_w + f), t, f, d, left), vr[f], sgv);
+#pragma unroll
+  for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
+    const int f = threadIdx.x + q * ROW_THREADS;
+    hv[q] = kv[q] = gv[q] = 0.f;
+    if (f < d) {
+      hv[q] = __bfloat162float(h[r0 + f]);
+      kv[q] = k[r0 + f];
+      gv[q] = dvt[r0 + f];
+      shh = fmaf(hv[q], hv[q], shh);
+      skk = fmaf(kv[q], kv[q], skk);
+      shk = fmaf(hv[q], kv[q], shk);
+      sgv = fmaf(gv[q], v[r0 + f], sgv);
+    }
   }
   shh = block_sum(shh, red);
   skk = block_sum(skk, red);
@@ -191,53 +252,18 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
   const float invd = 1.0f / (float)d, isd = rsqrtf((float)d);
   const float rh = rsqrtf(shh * invd + BW_RMS_EPS), rk = rsqrtf(skk * invd + BW_RMS_EPS);
   const float a = alpha[t];
-  const float dz = sgv * a * (1.0f - a);
-  const float c = dz * isd;                          // dh^ = c k^, dk^ = c h^
-  const float dot_h = c * rk * shk;                  // <dh^, h>
-  const float dot_k = c * rh * shk;                  // <dk^, k>
-  const float ch = rh * rh * rh * dot_h * invd, ck = rk * rk * rk * dot_k * invd;
-  for (int f = threadIdx.x; f < d; f += ROW_THREADS) {
-    const float hv = __bfloat162float(hr[f]), kv = kr[f];
-    const float g = dvt_of(dout, dy, __ldg(conv_w + f), t, f, d, left);
-    dv_out[t * d + f] = __float2bfloat16_rn(a * g);
-    dk_out[t * d + f] = __float2bfloat16_rn(rk * (c * rh * hv) - ck * kv);
-    dh[t * d + f] = dout[t * d + f] + rh * (c * rk * kv) - ch * hv;
+  const float c = sgv * a * (1.0f - a) * isd;  // dz / sqrt(d): dh^ = c k^, dk^ = c h^
+  const float ch = rh * rh * rh * (c * rk * shk) * invd;   // r_h^3 <dh^, h> / d
+  const float ck = rk * rk * rk * (c * rh * shk) * invd;   // r_k^3 <dk^, k> / d
+#pragma unroll
+  for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
+    const int f = threadIdx.x + q * ROW_THREADS;
+    if (f < d) {
+      dv_out[r0 + f] = __float2bfloat16_rn(a * gv[q]);
+      dk_out[r0 + f] = __float2bfloat16_rn(rk * (c * rh * hv[q]) - ck * kv[q]);
+      dh[r0 + f] = dout[r0 + f] + rh * (c * rk * kv[q]) - ch * hv[q];
+    }
   }
-}
-
-constexpr int DCONV_TOK = 256;  // tokens per partial
-
-// Partial conv-weight gradients: block (chunk of DCONV_TOK tokens, 128
-// features); each thread walks its feature through the chunk with the three
-// previous vt in registers.  part[chunk][f][i].
-__global__ void __launch_bounds__(128) bw_dconv_partial_kernel(
-    const float* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ dy,
-    int64_t N, int T, int d, float4* __restrict__ part) {
-  const int f = blockIdx.y * 128 + threadIdx.x;
-  if (f >= d) return;
-  const int64_t t0 = (int64_t)blockIdx.x * DCONV_TOK;
-  const int64_t t1 = t0 + DCONV_TOK < N ? t0 + DCONV_TOK : N;
-  float s1 = 0.f, s2 = 0.f, s3 = 0.f;  // vt of t-1, t-2, t-3
-  {
-    const int pos = (int)(t0 % T);
-    if (pos >= 1) s1 = alpha[t0 - 1] * v[(t0 - 1) * d + f];
-    if (pos >= 2) s2 = alpha[t0 - 2] * v[(t0 - 2) * d + f];
-    if (pos >= 3) s3 = alpha[t0 - 3] * v[(t0 - 3) * d + f];
-  }
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  for (int64_t t = t0; t < t1; ++t) {
-    if (t % T == 0) s1 = s2 = s3 = 0.f;
-    const float vt = alpha[t] * v[t * d + f];
-    const float g = dy[t * d + f];
-    a0 = fmaf(g, s3, a0);  // tap 0 multiplies vt_{t-3}
-    a1 = fmaf(g, s2, a1);
-    a2 = fmaf(g, s1, a2);
-    a3 = fmaf(g, vt, a3);
-    s3 = s2;
-    s2 = s1;
-    s1 = vt;
-  }
-  part[(int64_t)blockIdx.x * d + f] = make_float4(a0, a1, a2, a3);
 }
 
 // dconv_w[f] = sum over chunks in order.
@@ -256,11 +282,14 @@ __global__ void bw_dconv_reduce_kernel(const float4* __restrict__ part, int chun
   dw[f] = s;
 }
 
-// Workspace: k, v, dy fp32 [N, d]; dk, dv bf16 [N, d]; de fp32 [N, E] when
+// Workspace: k, v, dvt fp32 [N, d]; dk, dv bf16 [N, d]; de fp32 [N, E] when
 // the caller passes none; conv partials; cuBLAS's workspace; the table
 // gradient's sort buffers.
 struct BwdBf16Ws {
-  float *k, *v, *dy, *de;
+  // k and v stay fp32: dh and dalpha are sums whose terms can cancel, so a
+  // bf16 rounding of k or v would show at full size in a small result
+  float *k, *v;
+  float *dvt, *de;
   __nv_bfloat16 *dk, *dv;
   float4* part;
   void* blas_ws;
@@ -271,7 +300,7 @@ struct BwdBf16Ws {
 constexpr size_t up256b(size_t b) { return (b + 255) & ~(size_t)255; }
 
 size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, BwdBf16Ws* w) {
-  const int64_t chunks = (N + DCONV_TOK - 1) / DCONV_TOK;
+  const int64_t chunks = (N + COL_TOK - 1) / COL_TOK;
   const size_t Nd4 = up256b((size_t)N * d * 4), Nd2 = up256b((size_t)N * d * 2);
   const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
   const size_t tg = table_grad_ws_bytes(N * J);
@@ -279,7 +308,7 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, BwdBf16Ws* w)
   if (w != nullptr) {
     w->k = reinterpret_cast<float*>(p);
     w->v = reinterpret_cast<float*>(p + Nd4);
-    w->dy = reinterpret_cast<float*>(p + 2 * Nd4);
+    w->dvt = reinterpret_cast<float*>(p + 2 * Nd4);
     w->dk = reinterpret_cast<__nv_bfloat16*>(p + 3 * Nd4);
     w->dv = reinterpret_cast<__nv_bfloat16*>(p + 3 * Nd4 + Nd2);
     w->de = reinterpret_cast<float*>(p + 3 * Nd4 + 2 * Nd2);
@@ -306,6 +335,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   const int E = hp.E;
   if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J)) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
+  if (d > ROW_THREADS * ROW_MAX_ITEMS) return ENGRAM_ERR_UNSUPPORTED;  // a row in registers
   BwdBf16Ws w;
   bwd_bf16_layout(ws, N, d, E, hp.J, &w);
   if (de == nullptr) de = w.de;
@@ -316,15 +346,12 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   // k = e W_k^T, v = e W_v^T (fp32)
   if ((rc = gemm_rm(hd, false, true, n, d, E, e, Wk, w.k, 0.f))) return rc;
   if ((rc = gemm_rm(hd, false, true, n, d, E, e, Wv, w.v, 0.f))) return rc;
-  const int64_t Nd = N * d;
-  bw_dy_kernel<<<(unsigned)((Nd + 255) / 256), 256, 0, s>>>(
-      w.v, alpha, reinterpret_cast<const float4*>(conv_w), dout, N, T, d, w.dy);
-  bw_row_kernel<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.k, w.v, alpha,
-                                                    reinterpret_cast<const float4*>(conv_w), dout,
-                                                    w.dy, N, T, d, dh, w.dk, w.dv);
-  const int chunks = (int)((N + DCONV_TOK - 1) / DCONV_TOK);
-  bw_dconv_partial_kernel<<<dim3((unsigned)chunks, (unsigned)((d + 127) / 128)), 128, 0, s>>>(
-      w.v, alpha, w.dy, N, T, d, w.part);
+  const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
+  bw_col_kernel<<<dim3((unsigned)chunks, (unsigned)((d + COL_THREADS - 1) / COL_THREADS)),
+                  COL_THREADS, 0, s>>>(w.v, alpha, reinterpret_cast<const float4*>(conv_w), dout,
+                                       N, T, d, w.dvt, w.part);
+  bw_row_kernel<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.k, w.v, alpha, dout, w.dvt, N, d, dh,
+                                                    w.dk, w.dv);
   bw_dconv_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(
       w.part, chunks, d, reinterpret_cast<float4*>(dconv_w));
   if ((rc = ck(cudaGetLastError()))) return rc;
