@@ -133,19 +133,32 @@ constexpr int COL_TOK = 128;      // tokens per column chunk
 constexpr int COL_THREADS = 128;  // features per block
 
 // One thread per (feature, chunk of COL_TOK tokens), walking the chunk in
-// token order with the three previous vt, dy and dout in registers.  At token
-// t it forms y_t and dy_t.  dvt of token t-3 is complete then (its vt enters
-// y_{t-3} .. y_t), or earlier when its sequence ends; the walk runs 3 tokens
-// past the chunk for those dy.  `live` counts the ring's tokens that belong
-// to t's sequence and lie in this chunk's walk.  Also writes the chunk's
+// token order with the three previous tokens' vt, v, alpha, dy and dout in
+// registers.  At token t it forms y_t and dy_t.  dvt of token t-3 is complete
+// then (its vt enters y_{t-3} .. y_t), or earlier when its sequence ends; the
+// walk runs 3 tokens past the chunk for those dy.  `live` counts the ring's
+// tokens that belong to t's sequence and lie in this chunk's walk.  For each
+// completed token the walk writes dv = alpha dvt (bf16, for the GEMMs) and
+// the warp's partial of dalpha = <dvt, v> over its 32 features (fixed
+// butterfly order), dalpha_part[token][f / 32]; and at the end the chunk's
 // partial conv-weight gradient part[chunk][f] = sum over its tokens of
-// dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).
+// dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).  All lanes of a warp walk the
+// same tokens, so the warp-wide sums run on uniform branches.
+__device__ __forceinline__ void col_emit(float r, float v_tok, float a_tok, int64_t tok, int f,
+                                         int d, __nv_bfloat16* __restrict__ dv,
+                                         float* __restrict__ dalpha_part) {
+  dv[tok * d + f] = __float2bfloat16_rn(a_tok * r);
+  float p = r * v_tok;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+  if ((threadIdx.x & 31) == 0) dalpha_part[tok * (d / 32) + f / 32] = p;
+}
+
 __global__ void __launch_bounds__(COL_THREADS) bw_col_kernel(
     const float* __restrict__ v, const float* __restrict__ alpha,
     const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
-    float* __restrict__ dvt, float4* __restrict__ part) {
-  const int f = blockIdx.y * COL_THREADS + threadIdx.x;
-  if (f >= d) return;
+    __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part, float4* __restrict__ part) {
+  const int f = blockIdx.y * COL_THREADS + threadIdx.x;  // d is a multiple of COL_THREADS
   const int64_t t0 = (int64_t)blockIdx.x * COL_TOK;
   const int64_t t1 = t0 + COL_TOK < N ? t0 + COL_TOK : N;
   const int64_t t_stop = t1 + 3 < N ? t1 + 3 : N;
@@ -156,33 +169,38 @@ __global__ void __launch_bounds__(COL_THREADS) bw_col_kernel(
   if (pos >= 2) s2 = alpha[t0 - 2] * v[(t0 - 2) * d + f];
   if (pos >= 3) s3 = alpha[t0 - 3] * v[(t0 - 3) * d + f];
   float g1 = 0.f, g2 = 0.f, g3 = 0.f;  // dy of t-1, t-2, t-3
-  float u1 = 0.f, u2 = 0.f, u3 = 0.f;  // dout of t-1, t-2, t-3
+  float u1 = 0.f, u2 = 0.f, u3 = 0.f;  // dout
+  float v1 = 0.f, v2 = 0.f, v3 = 0.f;  // v
+  float al1 = 0.f, al2 = 0.f, al3 = 0.f;  // alpha
   int live = 0;
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  // the next PF tokens' v (already times alpha) and dout, loaded ahead of
-  // the walk so that their latency overlaps the steps before them
+  // the next PF tokens' v, alpha and dout, loaded ahead of the walk
   constexpr int PF = 4;
-  float pv[PF], pu[PF];
+  float pv[PF], pa[PF], pu[PF];
 #pragma unroll
   for (int q = 0; q < PF; ++q) {
     const int64_t tq = t0 + q;
-    pv[q] = tq < t_stop ? alpha[tq] * v[tq * d + f] : 0.f;
+    pv[q] = tq < t_stop ? v[tq * d + f] : 0.f;
+    pa[q] = tq < t_stop ? alpha[tq] : 0.f;
     pu[q] = tq < t_stop ? dout[tq * d + f] : 0.f;
   }
   for (int64_t t = t0; t < t_stop; ++t) {
-    const float vt = pv[0], ut = pu[0];
+    const float vr = pv[0], at = pa[0], ut = pu[0];
 #pragma unroll
     for (int q = 0; q < PF - 1; ++q) {
       pv[q] = pv[q + 1];
+      pa[q] = pa[q + 1];
       pu[q] = pu[q + 1];
     }
     const int64_t tn = t + PF;
-    pv[PF - 1] = tn < t_stop ? alpha[tn] * v[tn * d + f] : 0.f;
+    pv[PF - 1] = tn < t_stop ? v[tn * d + f] : 0.f;
+    pa[PF - 1] = tn < t_stop ? alpha[tn] : 0.f;
     pu[PF - 1] = tn < t_stop ? dout[tn * d + f] : 0.f;
     if (pos == 0) {  // a sequence starts at t
       s1 = s2 = s3 = 0.f;
       live = 0;
     }
+    const float vt = at * vr;
     const float y = fmaf(w.x, s3, fmaf(w.y, s2, fmaf(w.z, s1, w.w * vt)));
     const float gt = ut * silu_grad(y);
     if (t < t1) {
@@ -192,12 +210,14 @@ __global__ void __launch_bounds__(COL_THREADS) bw_col_kernel(
       a3 = fmaf(gt, vt, a3);
     }
     if (live == 3 && t - 3 >= t0)
-      dvt[(t - 3) * d + f] = u3 + w.w * g3 + w.z * g2 + w.y * g1 + w.x * gt;
+      col_emit(u3 + w.w * g3 + w.z * g2 + w.y * g1 + w.x * gt, v3, al3, t - 3, f, d, dv,
+               dalpha_part);
     if (pos == T - 1) {  // the sequence ends at t: its last tokens are complete
       if (live >= 2 && t - 2 >= t0 && t - 2 < t1)
-        dvt[(t - 2) * d + f] = u2 + w.w * g2 + w.z * g1 + w.y * gt;
-      if (live >= 1 && t - 1 >= t0 && t - 1 < t1) dvt[(t - 1) * d + f] = u1 + w.w * g1 + w.z * gt;
-      if (t < t1) dvt[t * d + f] = ut + w.w * gt;
+        col_emit(u2 + w.w * g2 + w.z * g1 + w.y * gt, v2, al2, t - 2, f, d, dv, dalpha_part);
+      if (live >= 1 && t - 1 >= t0 && t - 1 < t1)
+        col_emit(u1 + w.w * g1 + w.z * gt, v1, al1, t - 1, f, d, dv, dalpha_part);
+      if (t < t1) col_emit(ut + w.w * gt, vr, at, t, f, d, dv, dalpha_part);
     }
     s3 = s2;
     s2 = s1;
@@ -208,6 +228,12 @@ __global__ void __launch_bounds__(COL_THREADS) bw_col_kernel(
     u3 = u2;
     u2 = u1;
     u1 = ut;
+    v3 = v2;
+    v2 = v1;
+    v1 = vr;
+    al3 = al2;
+    al2 = al1;
+    al1 = at;
     live = live < 3 ? live + 1 : 3;
     pos = pos + 1 == T ? 0 : pos + 1;
   }
@@ -217,33 +243,38 @@ __global__ void __launch_bounds__(COL_THREADS) bw_col_kernel(
 constexpr int ROW_MAX_ITEMS = 16;  // d <= ROW_THREADS * ROW_MAX_ITEMS = 4,096
 
 // One block per token: the gate and both RMSNorm backwards need whole-row
-// sums; the row's h, k, v, dvt are read once into registers, summed, then
-// dv and dk (bf16, for the GEMMs) and dh are written.
+// sums; the row's h and k are read once into registers, dalpha is the sum of
+// the column walk's d/32 partials (in order), then dk (bf16, for the GEMMs)
+// and dh are written.
 __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     const __nv_bfloat16* __restrict__ h, const float* __restrict__ k,
-    const float* __restrict__ v, const float* __restrict__ alpha,
-    const float* __restrict__ dout, const float* __restrict__ dvt, int64_t N, int d,
-    float* __restrict__ dh,
-    __nv_bfloat16* __restrict__ dk_out, __nv_bfloat16* __restrict__ dv_out) {
+    const float* __restrict__ alpha, const float* __restrict__ dout,
+    const float* __restrict__ dalpha_part, int64_t N, int d, float* __restrict__ dh,
+    __nv_bfloat16* __restrict__ dk_out) {
   __shared__ float red[ROW_THREADS / 32];
   const int64_t t = blockIdx.x;
   if (t >= N) return;
   const int64_t r0 = t * d;
-  float hv[ROW_MAX_ITEMS], kv[ROW_MAX_ITEMS], gv[ROW_MAX_ITEMS];
-  float shh = 0.f, skk = 0.f, shk = 0.f, sgv = 0.f;
+  float hv[ROW_MAX_ITEMS], kv[ROW_MAX_ITEMS];
+  float shh = 0.f, skk = 0.f, shk = 0.f;
 #pragma unroll
   for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
     const int f = threadIdx.x + q * ROW_THREADS;
-    hv[q] = kv[q] = gv[q] = 0.f;
+    hv[q] = kv[q] = 0.f;
     if (f < d) {
       hv[q] = __bfloat162float(h[r0 + f]);
       kv[q] = k[r0 + f];
-      gv[q] = dvt[r0 + f];
       shh = fmaf(hv[q], hv[q], shh);
       skk = fmaf(kv[q], kv[q], skk);
       shk = fmaf(hv[q], kv[q], shk);
-      sgv = fmaf(gv[q], v[r0 + f], sgv);
     }
+  }
+  // dalpha: the d/32 warp partials of the column walk, added in order by
+  // the first warp then broadcast
+  float sgv = 0.f;
+  if (threadIdx.x < 32) {
+    const float* pp = dalpha_part + t * (d / 32);
+    for (int i = threadIdx.x; i < d / 32; i += 32) sgv += pp[i];
   }
   shh = block_sum(shh, red);
   skk = block_sum(skk, red);
@@ -259,7 +290,6 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
   for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
     const int f = threadIdx.x + q * ROW_THREADS;
     if (f < d) {
-      dv_out[r0 + f] = __float2bfloat16_rn(a * gv[q]);
       dk_out[r0 + f] = __float2bfloat16_rn(rk * (c * rh * hv[q]) - ck * kv[q]);
       dh[r0 + f] = dout[r0 + f] + rh * (c * rk * kv[q]) - ch * hv[q];
     }
@@ -282,14 +312,14 @@ __global__ void bw_dconv_reduce_kernel(const float4* __restrict__ part, int chun
   dw[f] = s;
 }
 
-// Workspace: k, v, dvt fp32 [N, d]; dk, dv bf16 [N, d]; de fp32 [N, E] when
+// Workspace: k, v fp32 [N, d], dalpha partials (sized [N, d] for simplicity); dk, dv bf16 [N, d]; de fp32 [N, E] when
 // the caller passes none; conv partials; cuBLAS's workspace; the table
 // gradient's sort buffers.
 struct BwdBf16Ws {
   // k and v stay fp32: dh and dalpha are sums whose terms can cancel, so a
   // bf16 rounding of k or v would show at full size in a small result
   float *k, *v;
-  float *dvt, *de;
+  float *dalpha_part, *de;  // [N, d/32] partials of <dvt, v>
   __nv_bfloat16 *dk, *dv;
   float4* part;
   void* blas_ws;
@@ -308,7 +338,7 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, BwdBf16Ws* w)
   if (w != nullptr) {
     w->k = reinterpret_cast<float*>(p);
     w->v = reinterpret_cast<float*>(p + Nd4);
-    w->dvt = reinterpret_cast<float*>(p + 2 * Nd4);
+    w->dalpha_part = reinterpret_cast<float*>(p + 2 * Nd4);
     w->dk = reinterpret_cast<__nv_bfloat16*>(p + 3 * Nd4);
     w->dv = reinterpret_cast<__nv_bfloat16*>(p + 3 * Nd4 + Nd2);
     w->de = reinterpret_cast<float*>(p + 3 * Nd4 + 2 * Nd2);
@@ -335,7 +365,8 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   const int E = hp.E;
   if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J)) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
-  if (d > ROW_THREADS * ROW_MAX_ITEMS) return ENGRAM_ERR_UNSUPPORTED;  // a row in registers
+  if (d > ROW_THREADS * ROW_MAX_ITEMS || d % COL_THREADS != 0)
+    return ENGRAM_ERR_UNSUPPORTED;  // a row in registers; whole column blocks
   BwdBf16Ws w;
   bwd_bf16_layout(ws, N, d, E, hp.J, &w);
   if (de == nullptr) de = w.de;
@@ -347,11 +378,11 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   if ((rc = gemm_rm(hd, false, true, n, d, E, e, Wk, w.k, 0.f))) return rc;
   if ((rc = gemm_rm(hd, false, true, n, d, E, e, Wv, w.v, 0.f))) return rc;
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
-  bw_col_kernel<<<dim3((unsigned)chunks, (unsigned)((d + COL_THREADS - 1) / COL_THREADS)),
-                  COL_THREADS, 0, s>>>(w.v, alpha, reinterpret_cast<const float4*>(conv_w), dout,
-                                       N, T, d, w.dvt, w.part);
-  bw_row_kernel<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.k, w.v, alpha, dout, w.dvt, N, d, dh,
-                                                    w.dk, w.dv);
+  bw_col_kernel<<<dim3((unsigned)chunks, (unsigned)(d / COL_THREADS)), COL_THREADS, 0, s>>>(
+      w.v, alpha, reinterpret_cast<const float4*>(conv_w), dout, N, T, d, w.dv, w.dalpha_part,
+      w.part);
+  bw_row_kernel<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.k, alpha, dout, w.dalpha_part, N, d, dh,
+                                                    w.dk);
   bw_dconv_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(
       w.part, chunks, d, reinterpret_cast<float4*>(dconv_w));
   if ((rc = ck(cudaGetLastError()))) return rc;
