@@ -108,7 +108,7 @@ int gemm_rm(cublasHandle_t hd, bool a_t, bool b_t, int m, int n, int k, const vo
 //   dw_i = sum_t dy_t vt_{t-3+i}
 
 __device__ __forceinline__ float silu_grad(float y) {
-  const float sg = 1.0f / (1.0f + __expf(-y));
+  const float sg = __fdividef(1.0f, 1.0f + __expf(-y));
   return sg * (1.0f + y * (1.0f - sg));
 }
 
@@ -154,7 +154,7 @@ __device__ __forceinline__ void col_emit(float r, float v_tok, float a_tok, int6
   if ((threadIdx.x & 31) == 0) dalpha_part[tok * (d / 32) + f / 32] = p;
 }
 
-__global__ void __launch_bounds__(COL_THREADS) bw_col_kernel(
+__global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
     const float* __restrict__ v, const float* __restrict__ alpha,
     const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
     __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part, float4* __restrict__ part) {
@@ -162,40 +162,54 @@ __global__ void __launch_bounds__(COL_THREADS) bw_col_kernel(
   const int64_t t0 = (int64_t)blockIdx.x * COL_TOK;
   const int64_t t1 = t0 + COL_TOK < N ? t0 + COL_TOK : N;
   const int64_t t_stop = t1 + 3 < N ? t1 + 3 : N;
+  // the gates of the walk's tokens (and the 3 before it), staged once
+  __shared__ float al_s[COL_TOK + 6];
+  for (int i = threadIdx.x; i < COL_TOK + 6; i += COL_THREADS) {
+    const int64_t tt = t0 - 3 + i;
+    al_s[i] = (tt >= 0 && tt < t_stop) ? alpha[tt] : 0.f;
+  }
+  __syncthreads();
+  auto al = [&](int64_t tt) { return al_s[(int)(tt - t0) + 3]; };  // t0 - 3 <= tt < t_stop
   const float4 w = __ldg(conv_w + f);
   int pos = (int)(t0 % T);
   float s1 = 0.f, s2 = 0.f, s3 = 0.f;  // vt of t-1, t-2, t-3 (zero before the sequence start)
-  if (pos >= 1) s1 = alpha[t0 - 1] * v[(t0 - 1) * d + f];
-  if (pos >= 2) s2 = alpha[t0 - 2] * v[(t0 - 2) * d + f];
-  if (pos >= 3) s3 = alpha[t0 - 3] * v[(t0 - 3) * d + f];
+  if (pos >= 1) s1 = al(t0 - 1) * v[(t0 - 1) * d + f];
+  if (pos >= 2) s2 = al(t0 - 2) * v[(t0 - 2) * d + f];
+  if (pos >= 3) s3 = al(t0 - 3) * v[(t0 - 3) * d + f];
   float g1 = 0.f, g2 = 0.f, g3 = 0.f;  // dy of t-1, t-2, t-3
   float u1 = 0.f, u2 = 0.f, u3 = 0.f;  // dout
   float v1 = 0.f, v2 = 0.f, v3 = 0.f;  // v
   float al1 = 0.f, al2 = 0.f, al3 = 0.f;  // alpha
   int live = 0;
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  // the next PF tokens' v, alpha and dout, loaded ahead of the walk
+  // the next PF tokens' v and dout, loaded ahead of the walk; row pointers
+  // advance by d per token (no 64-bit index products in the loop)
   constexpr int PF = 4;
-  float pv[PF], pa[PF], pu[PF];
+  float pv[PF], pu[PF];
+  const float* vp = v + t0 * d + f;
+  const float* up = dout + t0 * d + f;
+  const int n_walk = (int)(t_stop - t0);
 #pragma unroll
   for (int q = 0; q < PF; ++q) {
-    const int64_t tq = t0 + q;
-    pv[q] = tq < t_stop ? v[tq * d + f] : 0.f;
-    pa[q] = tq < t_stop ? alpha[tq] : 0.f;
-    pu[q] = tq < t_stop ? dout[tq * d + f] : 0.f;
+    pv[q] = q < n_walk ? vp[(int64_t)q * d] : 0.f;
+    pu[q] = q < n_walk ? up[(int64_t)q * d] : 0.f;
   }
-  for (int64_t t = t0; t < t_stop; ++t) {
-    const float vr = pv[0], at = pa[0], ut = pu[0];
+  vp += (int64_t)PF * d;
+  up += (int64_t)PF * d;
+#pragma unroll 4
+  for (int i = 0; i < n_walk; ++i) {
+    const int64_t t = t0 + i;
+    const float vr = pv[0], at = al_s[i + 3], ut = pu[0];
 #pragma unroll
     for (int q = 0; q < PF - 1; ++q) {
       pv[q] = pv[q + 1];
-      pa[q] = pa[q + 1];
       pu[q] = pu[q + 1];
     }
-    const int64_t tn = t + PF;
-    pv[PF - 1] = tn < t_stop ? v[tn * d + f] : 0.f;
-    pa[PF - 1] = tn < t_stop ? alpha[tn] : 0.f;
-    pu[PF - 1] = tn < t_stop ? dout[tn * d + f] : 0.f;
+    const bool more = i + PF < n_walk;
+    pv[PF - 1] = more ? *vp : 0.f;
+    pu[PF - 1] = more ? *up : 0.f;
+    vp += d;
+    up += d;
     if (pos == 0) {  // a sequence starts at t
       s1 = s2 = s3 = 0.f;
       live = 0;
