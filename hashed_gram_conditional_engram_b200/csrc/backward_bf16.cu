@@ -144,14 +144,16 @@ constexpr int COL_THREADS = 128;  // features per block
 // partial conv-weight gradient part[chunk][f] = sum over its tokens of
 // dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).  All lanes of a warp walk the
 // same tokens, so the warp-wide sums run on uniform branches.
-__device__ __forceinline__ void col_emit(float r, float v_tok, float a_tok, int64_t tok, int f,
-                                         int d, __nv_bfloat16* __restrict__ dv,
-                                         float* __restrict__ dalpha_part) {
-  dv[tok * d + f] = __float2bfloat16_rn(a_tok * r);
+// j: the token's index within the walk (token t0 + j); dvb, pab point at
+// token t0's dv element and dalpha partial of this thread / warp.
+__device__ __forceinline__ void col_emit(float r, float v_tok, float a_tok, int j, int d,
+                                         __nv_bfloat16* __restrict__ dvb,
+                                         float* __restrict__ pab) {
+  dvb[j * d] = __float2bfloat16_rn(a_tok * r);
   float p = r * v_tok;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-  if ((threadIdx.x & 31) == 0) dalpha_part[tok * (d / 32) + f / 32] = p;
+  if ((threadIdx.x & 31) == 0) pab[j * (d / 32)] = p;
 }
 
 __global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
@@ -182,6 +184,9 @@ __global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
   float al1 = 0.f, al2 = 0.f, al3 = 0.f;  // alpha
   int live = 0;
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  __nv_bfloat16* dvb = dv + t0 * d + f;
+  float* pab = dalpha_part + t0 * (d / 32) + f / 32;
+  const int n_chunk = (int)(t1 - t0);
   // the next PF tokens' v and dout, loaded ahead of the walk; row pointers
   // advance by d per token (no 64-bit index products in the loop)
   constexpr int PF = 4;
@@ -198,7 +203,6 @@ __global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
   up += (int64_t)PF * d;
 #pragma unroll 4
   for (int i = 0; i < n_walk; ++i) {
-    const int64_t t = t0 + i;
     const float vr = pv[0], at = al_s[i + 3], ut = pu[0];
 #pragma unroll
     for (int q = 0; q < PF - 1; ++q) {
@@ -217,21 +221,20 @@ __global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
     const float vt = at * vr;
     const float y = fmaf(w.x, s3, fmaf(w.y, s2, fmaf(w.z, s1, w.w * vt)));
     const float gt = ut * silu_grad(y);
-    if (t < t1) {
+    if (i < n_chunk) {
       a0 = fmaf(gt, s3, a0);
       a1 = fmaf(gt, s2, a1);
       a2 = fmaf(gt, s1, a2);
       a3 = fmaf(gt, vt, a3);
     }
-    if (live == 3 && t - 3 >= t0)
-      col_emit(u3 + w.w * g3 + w.z * g2 + w.y * g1 + w.x * gt, v3, al3, t - 3, f, d, dv,
-               dalpha_part);
-    if (pos == T - 1) {  // the sequence ends at t: its last tokens are complete
-      if (live >= 2 && t - 2 >= t0 && t - 2 < t1)
-        col_emit(u2 + w.w * g2 + w.z * g1 + w.y * gt, v2, al2, t - 2, f, d, dv, dalpha_part);
-      if (live >= 1 && t - 1 >= t0 && t - 1 < t1)
-        col_emit(u1 + w.w * g1 + w.z * gt, v1, al1, t - 1, f, d, dv, dalpha_part);
-      if (t < t1) col_emit(ut + w.w * gt, vr, at, t, f, d, dv, dalpha_part);
+    if (live == 3 && i >= 3)
+      col_emit(u3 + w.w * g3 + w.z * g2 + w.y * g1 + w.x * gt, v3, al3, i - 3, d, dvb, pab);
+    if (pos == T - 1) {  // the sequence ends at token i: its last tokens are complete
+      if (live >= 2 && i >= 2 && i - 2 < n_chunk)
+        col_emit(u2 + w.w * g2 + w.z * g1 + w.y * gt, v2, al2, i - 2, d, dvb, pab);
+      if (live >= 1 && i >= 1 && i - 1 < n_chunk)
+        col_emit(u1 + w.w * g1 + w.z * gt, v1, al1, i - 1, d, dvb, pab);
+      if (i < n_chunk) col_emit(ut + w.w * gt, vr, at, i, d, dvb, pab);
     }
     s3 = s2;
     s2 = s1;
