@@ -230,6 +230,9 @@ def _within_gemm_bound(got, want, bound):
 @pytest.mark.parametrize("B,T,d,K,D_h", [
     (3, 100, 256, 2, 32),     # narrow forward tiles, sequences of 100
     (2, 2500, 512, 2, 32),    # wide forward tiles
+    (64, 1, 256, 2, 32),      # one-token sequences: every token starts and ends one
+    (50, 3, 256, 2, 32),      # sequences shorter than the conv
+    (1, 129, 256, 2, 16),     # one sequence one token past a 128-token column chunk
 ])
 def test_backward_bf16_matches_oracle(B, T, d, K, D_h):
     g, ref, idx, rows, D_h = _bf16_backward_case(B, T, d, K, D_h, seed=B * 31 + T)
