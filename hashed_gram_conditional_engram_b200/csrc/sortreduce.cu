@@ -337,6 +337,7 @@ __global__ void tg_heads_kernel(const uint64_t* __restrict__ keys, int64_t n, ui
 // n-gram) with TG_PF loads issued ahead of the adds.
 constexpr int TG_U = 4;
 constexpr int TG_PF = 8;
+constexpr int TG_LONG = 64;  // longer segments go to tg_long_reduce_kernel
 __device__ __forceinline__ void add4(float4& a, const float4 x) {
   a.x = a.x + x.x;
   a.y = a.y + x.y;
@@ -375,7 +376,7 @@ __global__ void tg_reduce_kernel(const int32_t* __restrict__ seg_start,
       x[k] = bb[k] < ee[k] ? __ldg(de + (int64_t)it[k] * D4 + cc[k]) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < TG_U; ++k) {
-      if (gg[k] >= total) continue;
+      if (gg[k] >= total || ee[k] - bb[k] > TG_LONG) continue;  // long rows: below
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       if (bb[k] < ee[k]) add4(acc, x[k]);
       int32_t p = bb[k] + 1;
@@ -479,6 +480,47 @@ SortWs carve(void* ws, int64_t n) {
 }
 
 }  // namespace
+
+// Rows whose segment is longer than TG_LONG (frequent n-grams; under
+// Zipf-distributed tokens a few run to hundreds of tokens), listed by one
+// thread per row (the list's order is free: each row has its own output slot).
+__global__ void tg_long_list_kernel(const int32_t* __restrict__ seg_start,
+                                    const int32_t* __restrict__ n_unique, int32_t* __restrict__ list,
+                                    int32_t* __restrict__ count) {
+  const int32_t u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= *n_unique) return;
+  if (seg_start[u + 1] - seg_start[u] > TG_LONG) list[atomicAdd(count, 1)] = u;
+}
+
+// One block per long row at a time: the block loads TG_LONG items' rows of de
+// into shared memory together (all their loads in flight at once), then one
+// thread per 4 dimensions adds them in order; the next chunk follows.  The
+// same fp32 sums as tg_reduce_kernel, bit for bit.
+constexpr int TG_LONG_THREADS = 256;
+__global__ void __launch_bounds__(TG_LONG_THREADS) tg_long_reduce_kernel(
+    const int32_t* __restrict__ seg_start, const uint32_t* __restrict__ vals,
+    const float4* __restrict__ de, const int32_t* __restrict__ list,
+    const int32_t* __restrict__ count, int D4, float4* __restrict__ rows) {
+  extern __shared__ float4 chunk[];  // [TG_LONG][D4]
+  const int n = *count;
+  for (int li = blockIdx.x; li < n; li += gridDim.x) {
+    const int32_t u = list[li];
+    const int32_t b = seg_start[u], e = seg_start[u + 1];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int32_t p0 = b; p0 < e; p0 += TG_LONG) {
+      const int m = e - p0 < TG_LONG ? e - p0 : TG_LONG;
+      for (int i = threadIdx.x; i < m * D4; i += TG_LONG_THREADS) {
+        const int it = i / D4, c = i - it * D4;
+        chunk[i] = __ldg(de + (int64_t)__ldg(vals + p0 + it) * D4 + c);
+      }
+      __syncthreads();
+      if (threadIdx.x < D4)
+        for (int it = 0; it < m; ++it) add4(acc, chunk[it * D4 + threadIdx.x]);
+      __syncthreads();
+    }
+    if (threadIdx.x < D4) rows[(int64_t)u * D4 + threadIdx.x] = acc;
+  }
+}
 
 // The whole table gradient in one block for up to TG_SMALL_MAX items (a
 // short sequence, a training step on a small batch): the items' (row id,
@@ -627,6 +669,20 @@ int launch_table_grad(const HeadParams& hp, const int32_t* idx, const float* de,
   tg_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(w.c, v, reinterpret_cast<const float4*>(de),
                                                     n_unique, D4,
                                                     reinterpret_cast<float4*>(rows_out));
+  // long segments: w.a (the flags, free after the heads) holds their list,
+  // w.scal[2] its length
+  int32_t* long_count = w.scal + 2;
+  if ((rc = ck(cudaMemsetAsync(long_count, 0, sizeof(int32_t), s)))) return rc;
+  tg_long_list_kernel<<<nb(n), 256, 0, s>>>(w.c, n_unique, w.a, long_count);
+  const size_t long_smem = (size_t)TG_LONG * D4 * sizeof(float4);
+  if (D4 > TG_LONG_THREADS || long_smem > 227 * 1024) return ENGRAM_ERR_UNSUPPORTED;
+  if (long_smem > 48 * 1024 &&
+      (rc = ck(cudaFuncSetAttribute(tg_long_reduce_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)long_smem))))
+    return rc;
+  tg_long_reduce_kernel<<<(unsigned)sms, TG_LONG_THREADS, long_smem, s>>>(
+      w.c, v, reinterpret_cast<const float4*>(de), w.a, long_count, D4,
+      reinterpret_cast<float4*>(rows_out));
   return ck(cudaGetLastError());
 }
 
