@@ -76,20 +76,18 @@ int blas_handle(cudaStream_t s, void* workspace, cublasHandle_t* out) {
   return ENGRAM_OK;
 }
 
-// C[m x n] (row-major, fp32) = alpha * op(A)[m x k] . op(B)[k x n] + beta * C
-// with A, B bf16 row-major: op(A) = A (a_t = false, A is [m x k]) or A^T (A
-// is [k x m]); likewise B.  Row-major C = A.B is column-major C^T = B^T.A^T,
-// which is what cuBLAS is asked for.
-int gemm_rm(cublasHandle_t hd, bool a_t, bool b_t, int m, int n, int k, const void* A,
-            const void* B, void* C, float beta, cudaDataType c_type = CUDA_R_32F) {
+// C[m x n] (row-major, fp32, row stride ldc) = op(A)[m x k] . op(B)[k x n]
+// + beta * C with A, B bf16 row-major: op(A) = A (a_t = false, A is [m x k])
+// or A^T (A is [k x m]), rows lda apart; likewise B.  Row-major C = A.B is
+// column-major C^T = B^T.A^T, which is what cuBLAS is asked for.
+int gemm_rm(cublasHandle_t hd, bool a_t, bool b_t, int m, int n, int k, const void* A, int lda,
+            const void* B, int ldb, float* C, int ldc, float beta) {
   const float alpha = 1.0f;
-  const int lda = a_t ? m : k;  // row length of A as stored
-  const int ldb = b_t ? k : n;
   const cublasOperation_t opB = b_t ? CUBLAS_OP_T : CUBLAS_OP_N;
   const cublasOperation_t opA = a_t ? CUBLAS_OP_T : CUBLAS_OP_N;
   const cublasStatus_t st =
       blas().gemm_ex(hd, opB, opA, n, m, k, &alpha, B, CUDA_R_16BF, ldb, A, CUDA_R_16BF, lda,
-                     &beta, C, c_type, n, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+                     &beta, C, CUDA_R_32F, ldc, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
   return st == CUBLAS_STATUS_SUCCESS ? ENGRAM_OK : ENGRAM_ERR_CUDA;
 }
 
@@ -146,10 +144,10 @@ constexpr int COL_THREADS = 128;  // features per block
 // same tokens, so the warp-wide sums run on uniform branches.
 // j: the token's index within the walk (token t0 + j); dvb, pab point at
 // token t0's dv element and dalpha partial of this thread / warp.
-__device__ __forceinline__ void col_emit(float r, float v_tok, float a_tok, int j, int d,
+__device__ __forceinline__ void col_emit(float r, float v_tok, float a_tok, int j, int d, int ld,
                                          __nv_bfloat16* __restrict__ dvb,
                                          float* __restrict__ pab) {
-  dvb[j * d] = __float2bfloat16_rn(a_tok * r);
+  dvb[j * ld] = __float2bfloat16_rn(a_tok * r);
   float p = r * v_tok;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
@@ -159,7 +157,9 @@ __device__ __forceinline__ void col_emit(float r, float v_tok, float a_tok, int 
 __global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
     const float* __restrict__ v, const float* __restrict__ alpha,
     const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
-    __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part, float4* __restrict__ part) {
+    int ld, __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part,
+    float4* __restrict__ part) {
+  // v and dv rows are ld apart (they share rows with k and dk), dout rows d
   const int f = blockIdx.y * COL_THREADS + threadIdx.x;  // d is a multiple of COL_THREADS
   const int64_t t0 = (int64_t)blockIdx.x * COL_TOK;
   const int64_t t1 = t0 + COL_TOK < N ? t0 + COL_TOK : N;
@@ -175,31 +175,31 @@ __global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
   const float4 w = __ldg(conv_w + f);
   int pos = (int)(t0 % T);
   float s1 = 0.f, s2 = 0.f, s3 = 0.f;  // vt of t-1, t-2, t-3 (zero before the sequence start)
-  if (pos >= 1) s1 = al(t0 - 1) * v[(t0 - 1) * d + f];
-  if (pos >= 2) s2 = al(t0 - 2) * v[(t0 - 2) * d + f];
-  if (pos >= 3) s3 = al(t0 - 3) * v[(t0 - 3) * d + f];
+  if (pos >= 1) s1 = al(t0 - 1) * v[(t0 - 1) * ld + f];
+  if (pos >= 2) s2 = al(t0 - 2) * v[(t0 - 2) * ld + f];
+  if (pos >= 3) s3 = al(t0 - 3) * v[(t0 - 3) * ld + f];
   float g1 = 0.f, g2 = 0.f, g3 = 0.f;  // dy of t-1, t-2, t-3
   float u1 = 0.f, u2 = 0.f, u3 = 0.f;  // dout
   float v1 = 0.f, v2 = 0.f, v3 = 0.f;  // v
   float al1 = 0.f, al2 = 0.f, al3 = 0.f;  // alpha
   int live = 0;
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  __nv_bfloat16* dvb = dv + t0 * d + f;
+  __nv_bfloat16* dvb = dv + t0 * ld + f;
   float* pab = dalpha_part + t0 * (d / 32) + f / 32;
   const int n_chunk = (int)(t1 - t0);
   // the next PF tokens' v and dout, loaded ahead of the walk; row pointers
   // advance by d per token (no 64-bit index products in the loop)
   constexpr int PF = 4;
   float pv[PF], pu[PF];
-  const float* vp = v + t0 * d + f;
+  const float* vp = v + t0 * ld + f;
   const float* up = dout + t0 * d + f;
   const int n_walk = (int)(t_stop - t0);
 #pragma unroll
   for (int q = 0; q < PF; ++q) {
-    pv[q] = q < n_walk ? vp[(int64_t)q * d] : 0.f;
+    pv[q] = q < n_walk ? vp[(int64_t)q * ld] : 0.f;
     pu[q] = q < n_walk ? up[(int64_t)q * d] : 0.f;
   }
-  vp += (int64_t)PF * d;
+  vp += (int64_t)PF * ld;
   up += (int64_t)PF * d;
 #pragma unroll 4
   for (int i = 0; i < n_walk; ++i) {
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
     const bool more = i + PF < n_walk;
     pv[PF - 1] = more ? *vp : 0.f;
     pu[PF - 1] = more ? *up : 0.f;
-    vp += d;
+    vp += ld;
     up += d;
     if (pos == 0) {  // a sequence starts at t
       s1 = s2 = s3 = 0.f;
@@ -228,13 +228,13 @@ __global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
       a3 = fmaf(gt, vt, a3);
     }
     if (live == 3 && i >= 3)
-      col_emit(u3 + w.w * g3 + w.z * g2 + w.y * g1 + w.x * gt, v3, al3, i - 3, d, dvb, pab);
+      col_emit(u3 + w.w * g3 + w.z * g2 + w.y * g1 + w.x * gt, v3, al3, i - 3, d, ld, dvb, pab);
     if (pos == T - 1) {  // the sequence ends at token i: its last tokens are complete
       if (live >= 2 && i >= 2 && i - 2 < n_chunk)
-        col_emit(u2 + w.w * g2 + w.z * g1 + w.y * gt, v2, al2, i - 2, d, dvb, pab);
+        col_emit(u2 + w.w * g2 + w.z * g1 + w.y * gt, v2, al2, i - 2, d, ld, dvb, pab);
       if (live >= 1 && i >= 1 && i - 1 < n_chunk)
-        col_emit(u1 + w.w * g1 + w.z * gt, v1, al1, i - 1, d, dvb, pab);
-      if (i < n_chunk) col_emit(ut + w.w * gt, vr, at, i, d, dvb, pab);
+        col_emit(u1 + w.w * g1 + w.z * gt, v1, al1, i - 1, d, ld, dvb, pab);
+      if (i < n_chunk) col_emit(ut + w.w * gt, vr, at, i, d, ld, dvb, pab);
     }
     s3 = s2;
     s2 = s1;
@@ -266,8 +266,9 @@ constexpr int ROW_MAX_ITEMS = 16;  // d <= ROW_THREADS * ROW_MAX_ITEMS = 4,096
 __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     const __nv_bfloat16* __restrict__ h, const float* __restrict__ k,
     const float* __restrict__ alpha, const float* __restrict__ dout,
-    const float* __restrict__ dalpha_part, int64_t N, int d, float* __restrict__ dh,
+    const float* __restrict__ dalpha_part, int64_t N, int d, int ld, float* __restrict__ dh,
     __nv_bfloat16* __restrict__ dk_out) {
+  // k and dk rows are ld apart (they share rows with v and dv)
   __shared__ float red[ROW_THREADS / 32];
   const int64_t t = blockIdx.x;
   if (t >= N) return;
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     hv[q] = kv[q] = 0.f;
     if (f < d) {
       hv[q] = __bfloat162float(h[r0 + f]);
-      kv[q] = k[r0 + f];
+      kv[q] = k[t * ld + f];
       shh = fmaf(hv[q], hv[q], shh);
       skk = fmaf(kv[q], kv[q], skk);
       shk = fmaf(hv[q], kv[q], shk);
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
   for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
     const int f = threadIdx.x + q * ROW_THREADS;
     if (f < d) {
-      dk_out[r0 + f] = __float2bfloat16_rn(rk * (c * rh * hv[q]) - ck * kv[q]);
+      dk_out[t * ld + f] = __float2bfloat16_rn(rk * (c * rh * hv[q]) - ck * kv[q]);
       dh[r0 + f] = dout[r0 + f] + rh * (c * rk * kv[q]) - ch * hv[q];
     }
   }
@@ -334,10 +335,14 @@ __global__ void bw_dconv_reduce_kernel(const float4* __restrict__ part, int chun
 // gradient's sort buffers.
 struct BwdBf16Ws {
   // k and v stay fp32: dh and dalpha are sums whose terms can cancel, so a
-  // bf16 rounding of k or v would show at full size in a small result
-  float *k, *v;
+  // bf16 rounding of k or v would show at full size in a small result.
+  // They share rows (kv [N, 2d] = [k | v]), as do dk and dv, and W_k, W_v
+  // are stacked (Wkv [2d, E]), so that each pair of GEMMs is one.
+  float* kv;
+  __nv_bfloat16* dkv;
+  __nv_bfloat16* Wkv;
+  float* dWkv;          // [2d, E], copied out to dWk and dWv
   float *dalpha_part, *de;  // [N, d/32] partials of <dvt, v>
-  __nv_bfloat16 *dk, *dv;
   float4* part;
   void* blas_ws;
   void* tg_ws;
@@ -348,23 +353,32 @@ constexpr size_t up256b(size_t b) { return (b + 255) & ~(size_t)255; }
 
 size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, BwdBf16Ws* w) {
   const int64_t chunks = (N + COL_TOK - 1) / COL_TOK;
-  const size_t Nd4 = up256b((size_t)N * d * 4), Nd2 = up256b((size_t)N * d * 2);
+  const size_t KV = up256b((size_t)N * 2 * d * 4), DKV = up256b((size_t)N * 2 * d * 2);
+  const size_t WKV = up256b((size_t)2 * d * E * 2), DW = up256b((size_t)2 * d * E * 4);
+  const size_t DA = up256b((size_t)N * (d / 32) * 4);
   const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
   const size_t tg = table_grad_ws_bytes(N * J);
-  char* p = static_cast<char*>(base);
+  size_t off[9];
+  const size_t sz[9] = {KV, DKV, WKV, DW, DA, NE4, P, kBlasWorkspace, tg};
+  size_t o = 0;
+  for (int i = 0; i < 9; ++i) {
+    off[i] = o;
+    o += sz[i];
+  }
   if (w != nullptr) {
-    w->k = reinterpret_cast<float*>(p);
-    w->v = reinterpret_cast<float*>(p + Nd4);
-    w->dalpha_part = reinterpret_cast<float*>(p + 2 * Nd4);
-    w->dk = reinterpret_cast<__nv_bfloat16*>(p + 3 * Nd4);
-    w->dv = reinterpret_cast<__nv_bfloat16*>(p + 3 * Nd4 + Nd2);
-    w->de = reinterpret_cast<float*>(p + 3 * Nd4 + 2 * Nd2);
-    w->part = reinterpret_cast<float4*>(p + 3 * Nd4 + 2 * Nd2 + NE4);
-    w->blas_ws = p + 3 * Nd4 + 2 * Nd2 + NE4 + P;
-    w->tg_ws = p + 3 * Nd4 + 2 * Nd2 + NE4 + P + kBlasWorkspace;
+    char* p = static_cast<char*>(base);
+    w->kv = reinterpret_cast<float*>(p + off[0]);
+    w->dkv = reinterpret_cast<__nv_bfloat16*>(p + off[1]);
+    w->Wkv = reinterpret_cast<__nv_bfloat16*>(p + off[2]);
+    w->dWkv = reinterpret_cast<float*>(p + off[3]);
+    w->dalpha_part = reinterpret_cast<float*>(p + off[4]);
+    w->de = reinterpret_cast<float*>(p + off[5]);
+    w->part = reinterpret_cast<float4*>(p + off[6]);
+    w->blas_ws = p + off[7];
+    w->tg_ws = p + off[8];
     w->tg_bytes = tg;
   }
-  return 3 * Nd4 + 2 * Nd2 + NE4 + P + kBlasWorkspace + tg;
+  return o;
 }
 
 }  // namespace
@@ -391,23 +405,29 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   int rc = blas_handle(s, w.blas_ws, &hd);
   if (rc) return rc;
   const int n = (int)N;
-  // k = e W_k^T, v = e W_v^T (fp32)
-  if ((rc = gemm_rm(hd, false, true, n, d, E, e, Wk, w.k, 0.f))) return rc;
-  if ((rc = gemm_rm(hd, false, true, n, d, E, e, Wv, w.v, 0.f))) return rc;
+  // W_k and W_v stacked, then [k | v] = e [W_k; W_v]^T (fp32)
+  const size_t wbytes = (size_t)d * E * 2;
+  if ((rc = ck(cudaMemcpyAsync(w.Wkv, Wk, wbytes, cudaMemcpyDeviceToDevice, s)))) return rc;
+  if ((rc = ck(cudaMemcpyAsync(w.Wkv + (size_t)d * E, Wv, wbytes, cudaMemcpyDeviceToDevice, s))))
+    return rc;
+  if ((rc = gemm_rm(hd, false, true, n, 2 * d, E, e, E, w.Wkv, E, w.kv, 2 * d, 0.f))) return rc;
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
   bw_col_kernel<<<dim3((unsigned)chunks, (unsigned)(d / COL_THREADS)), COL_THREADS, 0, s>>>(
-      w.v, alpha, reinterpret_cast<const float4*>(conv_w), dout, N, T, d, w.dv, w.dalpha_part,
-      w.part);
-  bw_row_kernel<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.k, alpha, dout, w.dalpha_part, N, d, dh,
-                                                    w.dk);
+      w.kv + d, alpha, reinterpret_cast<const float4*>(conv_w), dout, N, T, d, 2 * d, w.dkv + d,
+      w.dalpha_part, w.part);
+  bw_row_kernel<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.kv, alpha, dout, w.dalpha_part, N, d,
+                                                    2 * d, dh, w.dkv);
   bw_dconv_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(
       w.part, chunks, d, reinterpret_cast<float4*>(dconv_w));
   if ((rc = ck(cudaGetLastError()))) return rc;
-  // dW_k = dk^T e, dW_v = dv^T e (contractions over tokens); de = dk W_k + dv W_v
-  if ((rc = gemm_rm(hd, true, false, d, E, n, w.dk, e, dWk, 0.f))) return rc;
-  if ((rc = gemm_rm(hd, true, false, d, E, n, w.dv, e, dWv, 0.f))) return rc;
-  if ((rc = gemm_rm(hd, false, false, n, E, d, w.dk, Wk, de, 0.f))) return rc;
-  if ((rc = gemm_rm(hd, false, false, n, E, d, w.dv, Wv, de, 1.f))) return rc;
+  // [dW_k; dW_v] = [dk | dv]^T e (a contraction over tokens), then split;
+  // de = [dk | dv] [W_k; W_v]
+  if ((rc = gemm_rm(hd, true, false, 2 * d, E, n, w.dkv, 2 * d, e, E, w.dWkv, E, 0.f))) return rc;
+  const size_t gbytes = (size_t)d * E * 4;
+  if ((rc = ck(cudaMemcpyAsync(dWk, w.dWkv, gbytes, cudaMemcpyDeviceToDevice, s)))) return rc;
+  if ((rc = ck(cudaMemcpyAsync(dWv, w.dWkv + (size_t)d * E, gbytes, cudaMemcpyDeviceToDevice, s))))
+    return rc;
+  if ((rc = gemm_rm(hd, false, false, n, E, 2 * d, w.dkv, 2 * d, w.Wkv, E, de, E, 0.f))) return rc;
   // the table rows' gradient from de, in the deterministic order
   return launch_table_grad(hp, idx, de, N, dtab_keys, dtab_rows, n_unique, w.tg_ws, w.tg_bytes, s);
 }
