@@ -110,228 +110,303 @@ __device__ __forceinline__ float silu_grad(float y) {
   return sg * (1.0f + y * (1.0f - sg));
 }
 
-constexpr int ROW_THREADS = 256;
-constexpr float BW_RMS_EPS = 1e-6f;  // the forward's RMSNorm epsilon
+constexpr int COL_TOK = 128;   // tokens per column chunk; one warp walks one chunk
+constexpr int COL_FPT = 2;     // features per lane (float2 loads)
+constexpr int COL_FEAT = 32 * COL_FPT;  // features per warp, one dalpha partial per token
+constexpr int COL_WARPS = 4;   // chunks per block
 
-// Sum of a value over the block, the same order on every run.
-__device__ __forceinline__ float block_sum(float x, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();  // red is reused
-  if (lane == 0) red[warp] = x;
-  __syncthreads();
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < ROW_THREADS / 32; ++i) s += red[i];
-  return s;
+__device__ __forceinline__ float2 ld_f2(const float* p) {
+  return *reinterpret_cast<const float2*>(p);
 }
 
-constexpr int COL_TOK = 128;      // tokens per column chunk
-constexpr int COL_THREADS = 128;  // features per block
-
-// One thread per (feature, chunk of COL_TOK tokens), walking the chunk in
-// token order with the three previous tokens' vt, v, alpha, dy and dout in
-// registers.  At token t it forms y_t and dy_t.  dvt of token t-3 is complete
-// then (its vt enters y_{t-3} .. y_t), or earlier when its sequence ends; the
-// walk runs 3 tokens past the chunk for those dy.  `live` counts the ring's
-// tokens that belong to t's sequence and lie in this chunk's walk.  For each
-// completed token the walk writes dv = alpha dvt (bf16, for the GEMMs) and
-// the warp's partial of dalpha = <dvt, v> over its 32 features (fixed
-// butterfly order), dalpha_part[token][f / 32]; and at the end the chunk's
-// partial conv-weight gradient part[chunk][f] = sum over its tokens of
-// dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).  All lanes of a warp walk the
-// same tokens, so the warp-wide sums run on uniform branches.
-// j: the token's index within the walk (token t0 + j); dvb, pab point at
-// token t0's dv element and dalpha partial of this thread / warp.
-__device__ __forceinline__ void col_emit(float r, float v_tok, float a_tok, int j, int d, int ld,
+// Emit token j of the walk: dv = alpha dvt as two bf16, and the warp's
+// partial of dalpha = <dvt, v> over its 64 features (the lane's pair first,
+// then a fixed butterfly).
+__device__ __forceinline__ void col_emit(float2 r, float2 vv, float a, int j, int ld, int np,
                                          __nv_bfloat16* __restrict__ dvb,
                                          float* __restrict__ pab) {
-  dvb[j * ld] = __float2bfloat16_rn(a_tok * r);
-  float p = r * v_tok;
+  *reinterpret_cast<__nv_bfloat162*>(dvb + j * ld) = __floats2bfloat162_rn(a * r.x, a * r.y);
+  float p = fmaf(r.x, vv.x, r.y * vv.y);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-  if ((threadIdx.x & 31) == 0) pab[j * (d / 32)] = p;
+  if ((threadIdx.x & 31) == 0) pab[j * np] = p;
 }
 
-__global__ void __launch_bounds__(COL_THREADS, 8) bw_col_kernel(
+// One warp per (chunk of COL_TOK tokens, 64 features), each lane holding two
+// adjacent features, walking the chunk in token order.  The warp keeps, for
+// the three previous tokens, vt and v, and the partial sums of their dvt:
+// dvt_s = u_s + w_3 dy_s + w_2 dy_{s+1} + w_1 dy_{s+2} + w_0 dy_{s+3} (terms
+// past the sequence end absent), to which each new dy_t adds its share.  At
+// token t it forms y_t and dy_t; dvt of token t-3 is then complete, and at a
+// sequence end so are t-2, t-1 and t.  The walk runs 3 tokens past the chunk
+// for the last tokens' dy.  `live` counts the ring's tokens that belong to
+// t's sequence and to this chunk's walk (tokens before the chunk are emitted
+// by the previous chunk's walk).  For each completed token it writes dv
+// (bf16, for the GEMMs) and the warp's partial of dalpha,
+// dalpha_part[token][f / 64]; at the end the chunk's partial conv-weight
+// gradient, part[chunk][f] = sum over its tokens of
+// dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).  Warps are independent (all
+// lanes of one walk the same tokens, so the butterflies run on uniform
+// branches); the block only groups COL_WARPS chunks for scheduling.
+__global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     const float* __restrict__ v, const float* __restrict__ alpha,
     const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
-    int ld, __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part,
+    int ld, int chunks, __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part,
     float4* __restrict__ part) {
   // v and dv rows are ld apart (they share rows with k and dk), dout rows d
-  const int f = blockIdx.y * COL_THREADS + threadIdx.x;  // d is a multiple of COL_THREADS
-  const int64_t t0 = (int64_t)blockIdx.x * COL_TOK;
+  __shared__ float al_all[COL_WARPS][COL_TOK + 6];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * COL_WARPS + warp;
+  if (chunk >= chunks) return;  // no block-wide barrier follows
+  const int f = blockIdx.y * COL_FEAT + lane * COL_FPT;
+  const int np = d / COL_FEAT;
+  const int64_t t0 = (int64_t)chunk * COL_TOK;
   const int64_t t1 = t0 + COL_TOK < N ? t0 + COL_TOK : N;
   const int64_t t_stop = t1 + 3 < N ? t1 + 3 : N;
-  // the gates of the walk's tokens (and the 3 before it), staged once
-  __shared__ float al_s[COL_TOK + 6];
-  for (int i = threadIdx.x; i < COL_TOK + 6; i += COL_THREADS) {
+  // the gates of the walk's tokens and the 3 before it: al_s[tt - t0 + 3]
+  float* al_s = al_all[warp];
+  for (int i = lane; i < COL_TOK + 6; i += 32) {
     const int64_t tt = t0 - 3 + i;
     al_s[i] = (tt >= 0 && tt < t_stop) ? alpha[tt] : 0.f;
   }
-  __syncthreads();
-  auto al = [&](int64_t tt) { return al_s[(int)(tt - t0) + 3]; };  // t0 - 3 <= tt < t_stop
-  const float4 w = __ldg(conv_w + f);
+  __syncwarp();
+  const float4 wx = __ldg(conv_w + f), wy = __ldg(conv_w + f + 1);
   int pos = (int)(t0 % T);
-  float s1 = 0.f, s2 = 0.f, s3 = 0.f;  // vt of t-1, t-2, t-3 (zero before the sequence start)
-  if (pos >= 1) s1 = al(t0 - 1) * v[(t0 - 1) * ld + f];
-  if (pos >= 2) s2 = al(t0 - 2) * v[(t0 - 2) * ld + f];
-  if (pos >= 3) s3 = al(t0 - 3) * v[(t0 - 3) * ld + f];
-  float g1 = 0.f, g2 = 0.f, g3 = 0.f;  // dy of t-1, t-2, t-3
-  float u1 = 0.f, u2 = 0.f, u3 = 0.f;  // dout
-  float v1 = 0.f, v2 = 0.f, v3 = 0.f;  // v
-  float al1 = 0.f, al2 = 0.f, al3 = 0.f;  // alpha
+  float2 s1 = make_float2(0.f, 0.f), s2 = s1, s3 = s1;  // vt of t-1, t-2, t-3
+  if (pos >= 1) {
+    const float2 q = ld_f2(v + (t0 - 1) * ld + f);
+    s1 = make_float2(al_s[2] * q.x, al_s[2] * q.y);
+  }
+  if (pos >= 2) {
+    const float2 q = ld_f2(v + (t0 - 2) * ld + f);
+    s2 = make_float2(al_s[1] * q.x, al_s[1] * q.y);
+  }
+  if (pos >= 3) {
+    const float2 q = ld_f2(v + (t0 - 3) * ld + f);
+    s3 = make_float2(al_s[0] * q.x, al_s[0] * q.y);
+  }
+  float2 A1 = make_float2(0.f, 0.f), A2 = A1, A3 = A1;  // partial dvt of t-1, t-2, t-3
+  float2 v1 = A1, v2 = A1, v3 = A1;                      // v of t-1, t-2, t-3
+  float4 cx = make_float4(0.f, 0.f, 0.f, 0.f), cy = cx;  // conv-weight partials
   int live = 0;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   __nv_bfloat16* dvb = dv + t0 * ld + f;
-  float* pab = dalpha_part + t0 * (d / 32) + f / 32;
-  const int n_chunk = (int)(t1 - t0);
-  // the next PF tokens' v and dout, loaded ahead of the walk; row pointers
-  // advance by d per token (no 64-bit index products in the loop)
+  float* pab = dalpha_part + t0 * np + blockIdx.y;
+  const int n_chunk = (int)(t1 - t0), n_walk = (int)(t_stop - t0);
+  // the next PF tokens' v and dout, loaded ahead of the walk
   constexpr int PF = 4;
-  float pv[PF], pu[PF];
+  float2 pv[PF], pu[PF];
   const float* vp = v + t0 * ld + f;
   const float* up = dout + t0 * d + f;
-  const int n_walk = (int)(t_stop - t0);
 #pragma unroll
   for (int q = 0; q < PF; ++q) {
-    pv[q] = q < n_walk ? vp[(int64_t)q * ld] : 0.f;
-    pu[q] = q < n_walk ? up[(int64_t)q * d] : 0.f;
+    pv[q] = q < n_walk ? ld_f2(vp + (int64_t)q * ld) : make_float2(0.f, 0.f);
+    pu[q] = q < n_walk ? ld_f2(up + (int64_t)q * d) : make_float2(0.f, 0.f);
   }
   vp += (int64_t)PF * ld;
   up += (int64_t)PF * d;
 #pragma unroll 4
   for (int i = 0; i < n_walk; ++i) {
-    const float vr = pv[0], at = al_s[i + 3], ut = pu[0];
+    const float2 vr = pv[0], ut = pu[0];
+    const float at = al_s[i + 3];
 #pragma unroll
     for (int q = 0; q < PF - 1; ++q) {
       pv[q] = pv[q + 1];
       pu[q] = pu[q + 1];
     }
     const bool more = i + PF < n_walk;
-    pv[PF - 1] = more ? *vp : 0.f;
-    pu[PF - 1] = more ? *up : 0.f;
+    pv[PF - 1] = more ? ld_f2(vp) : make_float2(0.f, 0.f);
+    pu[PF - 1] = more ? ld_f2(up) : make_float2(0.f, 0.f);
     vp += ld;
     up += d;
     if (pos == 0) {  // a sequence starts at t
-      s1 = s2 = s3 = 0.f;
+      s1 = s2 = s3 = make_float2(0.f, 0.f);
       live = 0;
     }
-    const float vt = at * vr;
-    const float y = fmaf(w.x, s3, fmaf(w.y, s2, fmaf(w.z, s1, w.w * vt)));
-    const float gt = ut * silu_grad(y);
+    const float2 vt = make_float2(at * vr.x, at * vr.y);
+    float2 g;
+    g.x = ut.x * silu_grad(fmaf(wx.x, s3.x, fmaf(wx.y, s2.x, fmaf(wx.z, s1.x, wx.w * vt.x))));
+    g.y = ut.y * silu_grad(fmaf(wy.x, s3.y, fmaf(wy.y, s2.y, fmaf(wy.z, s1.y, wy.w * vt.y))));
     if (i < n_chunk) {
-      a0 = fmaf(gt, s3, a0);
-      a1 = fmaf(gt, s2, a1);
-      a2 = fmaf(gt, s1, a2);
-      a3 = fmaf(gt, vt, a3);
+      cx.x = fmaf(g.x, s3.x, cx.x);
+      cx.y = fmaf(g.x, s2.x, cx.y);
+      cx.z = fmaf(g.x, s1.x, cx.z);
+      cx.w = fmaf(g.x, vt.x, cx.w);
+      cy.x = fmaf(g.y, s3.y, cy.x);
+      cy.y = fmaf(g.y, s2.y, cy.y);
+      cy.z = fmaf(g.y, s1.y, cy.z);
+      cy.w = fmaf(g.y, vt.y, cy.w);
     }
-    if (live == 3 && i >= 3)
-      col_emit(u3 + w.w * g3 + w.z * g2 + w.y * g1 + w.x * gt, v3, al3, i - 3, d, ld, dvb, pab);
-    if (pos == T - 1) {  // the sequence ends at token i: its last tokens are complete
-      if (live >= 2 && i >= 2 && i - 2 < n_chunk)
-        col_emit(u2 + w.w * g2 + w.z * g1 + w.y * gt, v2, al2, i - 2, d, ld, dvb, pab);
-      if (live >= 1 && i >= 1 && i - 1 < n_chunk)
-        col_emit(u1 + w.w * g1 + w.z * gt, v1, al1, i - 1, d, ld, dvb, pab);
-      if (i < n_chunk) col_emit(ut + w.w * gt, vr, at, i, d, ld, dvb, pab);
+    if (live == 3)  // token t-3 is complete
+      col_emit(make_float2(fmaf(wx.x, g.x, A3.x), fmaf(wy.x, g.y, A3.y)), v3, al_s[i], i - 3,
+               ld, np, dvb, pab);
+    const float2 B2 = make_float2(fmaf(wx.y, g.x, A2.x), fmaf(wy.y, g.y, A2.y));
+    const float2 B1 = make_float2(fmaf(wx.z, g.x, A1.x), fmaf(wy.z, g.y, A1.y));
+    const float2 B0 = make_float2(fmaf(wx.w, g.x, ut.x), fmaf(wy.w, g.y, ut.y));
+    if (pos == T - 1) {  // the sequence ends at t: its last tokens are complete
+      if (live >= 2 && i - 2 < n_chunk) col_emit(B2, v2, al_s[i + 1], i - 2, ld, np, dvb, pab);
+      if (live >= 1 && i - 1 < n_chunk) col_emit(B1, v1, al_s[i + 2], i - 1, ld, np, dvb, pab);
+      if (i < n_chunk) col_emit(B0, vr, at, i, ld, np, dvb, pab);
     }
+    A3 = B2;
+    A2 = B1;
+    A1 = B0;
     s3 = s2;
     s2 = s1;
     s1 = vt;
-    g3 = g2;
-    g2 = g1;
-    g1 = gt;
-    u3 = u2;
-    u2 = u1;
-    u1 = ut;
     v3 = v2;
     v2 = v1;
     v1 = vr;
-    al3 = al2;
-    al2 = al1;
-    al1 = at;
     live = live < 3 ? live + 1 : 3;
     pos = pos + 1 == T ? 0 : pos + 1;
   }
-  if (t1 > t0) part[(int64_t)blockIdx.x * d + f] = make_float4(a0, a1, a2, a3);
+  part[(int64_t)chunk * d + f] = cx;
+  part[(int64_t)chunk * d + f + 1] = cy;
 }
 
-constexpr int ROW_MAX_ITEMS = 16;  // d <= ROW_THREADS * ROW_MAX_ITEMS = 4,096
+constexpr int ROW_THREADS = 256;
+constexpr int ROW_VEC = 4;        // features per load
+constexpr int ROW_MAX_ITEMS = 4;  // d <= ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS = 4,096
+constexpr float BW_RMS_EPS = 1e-6f;  // the forward's RMSNorm epsilon
+
+__device__ __forceinline__ float4 bf16x4_to_f4(uint2 u) {
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
 
 // One block per token: the gate and both RMSNorm backwards need whole-row
-// sums; the row's h and k are read once into registers, dalpha is the sum of
-// the column walk's d/32 partials (in order), then dk (bf16, for the GEMMs)
-// and dh are written.
+// sums.  The row's h, k and dout are read once (4 features per load) into
+// registers; <h,h>, <k,k>, <h,k> and dalpha (the column walk's d/64
+// partials, added in order by the first warp) are reduced together in one
+// fixed-order pass; then dk (bf16, for the GEMMs) and dh are written.
 __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     const __nv_bfloat16* __restrict__ h, const float* __restrict__ k,
     const float* __restrict__ alpha, const float* __restrict__ dout,
     const float* __restrict__ dalpha_part, int64_t N, int d, int ld, float* __restrict__ dh,
     __nv_bfloat16* __restrict__ dk_out) {
   // k and dk rows are ld apart (they share rows with v and dv)
-  __shared__ float red[ROW_THREADS / 32];
+  __shared__ float4 red[ROW_THREADS / 32];
   const int64_t t = blockIdx.x;
   if (t >= N) return;
-  const int64_t r0 = t * d;
-  float hv[ROW_MAX_ITEMS], kv[ROW_MAX_ITEMS];
+  const int nv = d / ROW_VEC;
+  const __nv_bfloat16* hr = h + t * d;
+  const float* kr = k + t * ld;
+  const float* ur = dout + t * d;
+  float4 hv[ROW_MAX_ITEMS], kv[ROW_MAX_ITEMS], uv[ROW_MAX_ITEMS];
   float shh = 0.f, skk = 0.f, shk = 0.f;
 #pragma unroll
   for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
-    const int f = threadIdx.x + q * ROW_THREADS;
-    hv[q] = kv[q] = 0.f;
-    if (f < d) {
-      hv[q] = __bfloat162float(h[r0 + f]);
-      kv[q] = k[t * ld + f];
-      shh = fmaf(hv[q], hv[q], shh);
-      skk = fmaf(kv[q], kv[q], skk);
-      shk = fmaf(hv[q], kv[q], shk);
+    const int c = threadIdx.x + q * ROW_THREADS;
+    hv[q] = kv[q] = uv[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c < nv) {
+      hv[q] = bf16x4_to_f4(*reinterpret_cast<const uint2*>(hr + c * ROW_VEC));
+      kv[q] = *reinterpret_cast<const float4*>(kr + c * ROW_VEC);
+      uv[q] = __ldcs(reinterpret_cast<const float4*>(ur + c * ROW_VEC));
     }
   }
-  // dalpha: the d/32 warp partials of the column walk, added in order by
-  // the first warp then broadcast
+#pragma unroll
+  for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
+    shh = fmaf(hv[q].x, hv[q].x, fmaf(hv[q].y, hv[q].y, fmaf(hv[q].z, hv[q].z, fmaf(hv[q].w, hv[q].w, shh))));
+    skk = fmaf(kv[q].x, kv[q].x, fmaf(kv[q].y, kv[q].y, fmaf(kv[q].z, kv[q].z, fmaf(kv[q].w, kv[q].w, skk))));
+    shk = fmaf(hv[q].x, kv[q].x, fmaf(hv[q].y, kv[q].y, fmaf(hv[q].z, kv[q].z, fmaf(hv[q].w, kv[q].w, shk))));
+  }
   float sgv = 0.f;
   if (threadIdx.x < 32) {
-    const float* pp = dalpha_part + t * (d / 32);
-    for (int i = threadIdx.x; i < d / 32; i += 32) sgv += pp[i];
+    const int np = d / COL_FEAT;
+    const float* pp = dalpha_part + t * np;
+    for (int i = threadIdx.x; i < np; i += 32) sgv += pp[i];
   }
-  shh = block_sum(shh, red);
-  skk = block_sum(skk, red);
-  shk = block_sum(shk, red);
-  sgv = block_sum(sgv, red);
+  float4 r = make_float4(shh, skk, shk, sgv);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    r.x += __shfl_xor_sync(0xffffffffu, r.x, o);
+    r.y += __shfl_xor_sync(0xffffffffu, r.y, o);
+    r.z += __shfl_xor_sync(0xffffffffu, r.z, o);
+    r.w += __shfl_xor_sync(0xffffffffu, r.w, o);
+  }
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = r;
+  __syncthreads();
+  r = red[0];
+#pragma unroll
+  for (int i = 1; i < ROW_THREADS / 32; ++i) {
+    r.x += red[i].x;
+    r.y += red[i].y;
+    r.z += red[i].z;
+    r.w += red[i].w;
+  }
+  shh = r.x;
+  skk = r.y;
+  shk = r.z;
   const float invd = 1.0f / (float)d, isd = rsqrtf((float)d);
   const float rh = rsqrtf(shh * invd + BW_RMS_EPS), rk = rsqrtf(skk * invd + BW_RMS_EPS);
   const float a = alpha[t];
-  const float c = sgv * a * (1.0f - a) * isd;  // dz / sqrt(d): dh^ = c k^, dk^ = c h^
+  const float c = r.w * a * (1.0f - a) * isd;  // dz / sqrt(d): dh^ = c k^, dk^ = c h^
   const float ch = rh * rh * rh * (c * rk * shk) * invd;   // r_h^3 <dh^, h> / d
   const float ck = rk * rk * rk * (c * rh * shk) * invd;   // r_k^3 <dk^, k> / d
+  const float crh = c * rh, crk = c * rk;
+  __nv_bfloat16* dkr = dk_out + t * ld;
+  float* dhr = dh + t * d;
 #pragma unroll
   for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
-    const int f = threadIdx.x + q * ROW_THREADS;
-    if (f < d) {
-      dk_out[t * ld + f] = __float2bfloat16_rn(rk * (c * rh * hv[q]) - ck * kv[q]);
-      dh[r0 + f] = dout[r0 + f] + rh * (c * rk * kv[q]) - ch * hv[q];
+    const int c4 = threadIdx.x + q * ROW_THREADS;
+    if (c4 < nv) {
+      const float4 hq = hv[q], kq = kv[q], uq = uv[q];
+      const __nv_bfloat162 k01 = __floats2bfloat162_rn(rk * (crh * hq.x) - ck * kq.x,
+                                                      rk * (crh * hq.y) - ck * kq.y);
+      const __nv_bfloat162 k23 = __floats2bfloat162_rn(rk * (crh * hq.z) - ck * kq.z,
+                                                      rk * (crh * hq.w) - ck * kq.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&k01);
+      pk.y = *reinterpret_cast<const uint32_t*>(&k23);
+      *reinterpret_cast<uint2*>(dkr + c4 * ROW_VEC) = pk;
+      float4 o;
+      o.x = uq.x + rh * (crk * kq.x) - ch * hq.x;
+      o.y = uq.y + rh * (crk * kq.y) - ch * hq.y;
+      o.z = uq.z + rh * (crk * kq.z) - ch * hq.z;
+      o.w = uq.w + rh * (crk * kq.w) - ch * hq.w;
+      __stcs(reinterpret_cast<float4*>(dhr + c4 * ROW_VEC), o);
     }
   }
 }
 
-// dconv_w[f] = sum over chunks in order.
-__global__ void bw_dconv_reduce_kernel(const float4* __restrict__ part, int chunks, int d,
-                                       float4* __restrict__ dw) {
-  const int f = blockIdx.x * blockDim.x + threadIdx.x;
-  if (f >= d) return;
+constexpr int DCONV_WARPS = 8;
+
+// dconv_w[f] = sum over chunks of part[chunk][f]: warp w adds chunks w,
+// w + 8, ... in order, then the 8 warp sums are added in warp order.
+__global__ void __launch_bounds__(32 * DCONV_WARPS) bw_dconv_reduce_kernel(
+    const float4* __restrict__ part, int chunks, int d, float4* __restrict__ dw) {
+  __shared__ float4 red[DCONV_WARPS][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f = blockIdx.x * 32 + lane;
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c = 0; c < chunks; ++c) {
-    const float4 p = part[(int64_t)c * d + f];
-    s.x += p.x;
-    s.y += p.y;
-    s.z += p.z;
-    s.w += p.w;
+  if (f < d) {
+#pragma unroll 4
+    for (int c = warp; c < chunks; c += DCONV_WARPS) {
+      const float4 p = part[(int64_t)c * d + f];
+      s.x += p.x;
+      s.y += p.y;
+      s.z += p.z;
+      s.w += p.w;
+    }
   }
-  dw[f] = s;
+  red[warp][lane] = s;
+  __syncthreads();
+  if (warp == 0 && f < d) {
+    float4 o = red[0][lane];
+#pragma unroll
+    for (int w = 1; w < DCONV_WARPS; ++w) {
+      o.x += red[w][lane].x;
+      o.y += red[w][lane].y;
+      o.z += red[w][lane].z;
+      o.w += red[w][lane].w;
+    }
+    dw[f] = o;
+  }
 }
 
-// Workspace: k, v fp32 [N, d], dalpha partials (sized [N, d] for simplicity); dk, dv bf16 [N, d]; de fp32 [N, E] when
-// the caller passes none; conv partials; cuBLAS's workspace; the table
+// Workspace: [k | v] fp32 [N, 2d]; [dk | dv] bf16 [N, 2d]; [W_k; W_v] bf16
+// and [dW_k; dW_v] fp32 [2d, E]; dalpha partials [N, d/64]; de fp32 [N, E]
+// when the caller passes none; conv partials; cuBLAS's workspace; the table
 // gradient's sort buffers.
 struct BwdBf16Ws {
   // k and v stay fp32: dh and dalpha are sums whose terms can cancel, so a
@@ -342,7 +417,7 @@ struct BwdBf16Ws {
   __nv_bfloat16* dkv;
   __nv_bfloat16* Wkv;
   float* dWkv;          // [2d, E], copied out to dWk and dWv
-  float *dalpha_part, *de;  // [N, d/32] partials of <dvt, v>
+  float *dalpha_part, *de;  // [N, d/64] partials of <dvt, v>
   float4* part;
   void* blas_ws;
   void* tg_ws;
@@ -355,7 +430,7 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, BwdBf16Ws* w)
   const int64_t chunks = (N + COL_TOK - 1) / COL_TOK;
   const size_t KV = up256b((size_t)N * 2 * d * 4), DKV = up256b((size_t)N * 2 * d * 2);
   const size_t WKV = up256b((size_t)2 * d * E * 2), DW = up256b((size_t)2 * d * E * 4);
-  const size_t DA = up256b((size_t)N * (d / 32) * 4);
+  const size_t DA = up256b((size_t)N * (d / COL_FEAT) * 4);
   const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
   const size_t tg = table_grad_ws_bytes(N * J);
   size_t off[9];
@@ -396,7 +471,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   const int E = hp.E;
   if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J)) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
-  if (d > ROW_THREADS * ROW_MAX_ITEMS || d % COL_THREADS != 0)
+  if (d > ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS || d % COL_FEAT != 0)
     return ENGRAM_ERR_UNSUPPORTED;  // a row in registers; whole column blocks
   BwdBf16Ws w;
   bwd_bf16_layout(ws, N, d, E, hp.J, &w);
@@ -412,12 +487,13 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
     return rc;
   if ((rc = gemm_rm(hd, false, true, n, 2 * d, E, e, E, w.Wkv, E, w.kv, 2 * d, 0.f))) return rc;
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
-  bw_col_kernel<<<dim3((unsigned)chunks, (unsigned)(d / COL_THREADS)), COL_THREADS, 0, s>>>(
-      w.kv + d, alpha, reinterpret_cast<const float4*>(conv_w), dout, N, T, d, 2 * d, w.dkv + d,
-      w.dalpha_part, w.part);
+  bw_col_kernel<<<dim3((unsigned)((chunks + COL_WARPS - 1) / COL_WARPS), (unsigned)(d / COL_FEAT)),
+                  32 * COL_WARPS, 0, s>>>(w.kv + d, alpha, reinterpret_cast<const float4*>(conv_w),
+                                          dout, N, T, d, 2 * d, chunks, w.dkv + d,
+                                          w.dalpha_part, w.part);
   bw_row_kernel<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.kv, alpha, dout, w.dalpha_part, N, d,
                                                     2 * d, dh, w.dkv);
-  bw_dconv_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(
+  bw_dconv_reduce_kernel<<<(unsigned)((d + 31) / 32), 32 * DCONV_WARPS, 0, s>>>(
       w.part, chunks, d, reinterpret_cast<float4*>(dconv_w));
   if ((rc = ck(cudaGetLastError()))) return rc;
   // [dW_k; dW_v] = [dk | dv]^T e (a contraction over tokens), then split;

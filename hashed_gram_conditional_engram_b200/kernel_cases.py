@@ -11,6 +11,7 @@ without the rest of the layer's inputs on the device.
     python -m hashed_gram_conditional_engram_b200.kernel_cases tablegrad [...]
     python -m hashed_gram_conditional_engram_b200.kernel_cases hostgather \
         --tokens 8192 --seq 2048 --dh 160 --rows 1000003
+    python -m hashed_gram_conditional_engram_b200.kernel_cases backward [...]
 
 `fused` runs engram_forward with table = NULL on random gathered rows, i.e.
 the two tensor-core passes; `gather` gathers from a table of --rows rows per
@@ -19,7 +20,9 @@ decode steps (hash with rolling n-gram state, then engram_forward with the
 table and the conv state) for --tokens sequences of one token each;
 `tablegrad` runs the sparse table gradient (sort by row, segment sums) on
 fp32 rows of de for hash indices of Zipf(1.1) token ids; `hostgather` runs
-engram_forward_hosttable on a table in pinned host memory.  Defaults are the
+engram_forward_hosttable on a table in pinned host memory; `backward` runs
+the bf16 engram_backward (column walk, row kernel, GEMMs, sparse table
+gradient) on random gathered rows, gates and output gradients.  Defaults are the
 27B-shaped layer's dimensions.  Prints the device time per repetition.
 """
 from __future__ import annotations
@@ -36,7 +39,7 @@ from . import synth
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("kernel", choices=["fused", "gather", "hash", "decode", "tablegrad",
-                                       "hostgather"])
+                                       "hostgather", "backward"])
     ap.add_argument("--tokens", type=int, default=32768)
     ap.add_argument("--seq", type=int, default=4096)
     ap.add_argument("--d", type=int, default=2560)
@@ -75,6 +78,29 @@ def main(argv=None):
 
         def run():
             eg.engram_forward(cfg, None, None, e, h, Wk, Wv, cw, None, out, saved, B, T, ws, nb)
+    elif a.kernel == "backward":
+        e = (torch.randn((N, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        h = torch.randn((N, a.d), generator=g, device=dev).to(torch.bfloat16)
+        Wk = (torch.randn((a.d, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        Wv = (torch.randn((a.d, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        cw = torch.randn((a.d, 4), generator=g, device=dev) * 0.5
+        saved = torch.rand((N,), generator=g, device=dev)
+        dout = torch.randn((N, a.d), generator=g, device=dev)
+        rng = np.random.default_rng(3)
+        idx = torch.from_numpy(np.stack([rng.integers(0, P, N) for P in rows], -1)
+                               .astype(np.int32)).to(dev)
+        dh = torch.empty((N, a.d), device=dev)
+        dWk, dWv = torch.empty((a.d, E), device=dev), torch.empty((a.d, E), device=dev)
+        dcw = torch.empty((a.d, 4), device=dev)
+        keys_out = torch.empty(N * a.heads, dtype=torch.int64, device=dev)
+        rows_out = torch.empty((N * a.heads, a.dh), device=dev)
+        nu = torch.zeros(1, dtype=torch.int32, device=dev)
+        nb = eg.engram_workspace_size(cfg, eg.WS_BACKWARD, N)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+
+        def run():
+            eg.engram_backward(cfg, idx, e, h, Wk, Wv, cw, saved, dout, dh, dWk, dWv, dcw, None,
+                               keys_out, rows_out, nu, B, T, ws, nb)
     elif a.kernel == "gather":
         table = torch.empty(sum(rows) * a.dh, dtype=torch.bfloat16, device=dev)
         table.normal_(0.0, 0.02, generator=g)
