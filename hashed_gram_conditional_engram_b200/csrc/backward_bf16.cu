@@ -105,9 +105,15 @@ int gemm_rm(cublasHandle_t hd, bool a_t, bool b_t, int m, int n, int k, const vo
 //   dh = u + r_h dh^ - r_h^3 h <dh^, h> / d,  dk = r_k dk^ - r_k^3 k <dk^, k> / d
 //   dw_i = sum_t dy_t vt_{t-3+i}
 
-__device__ __forceinline__ float silu_grad(float y) {
-  const float sg = __fdividef(1.0f, 1.0f + __expf(-y));
-  return sg * (1.0f + y * (1.0f - sg));
+// SiLU'(y) = s (1 + y (1 - s)), s = sigmoid(y), for two features at once:
+// the arithmetic around the two exponentials and reciprocals runs on packed
+// fp32 pairs.
+__device__ __forceinline__ float2 silu_grad2(float2 y) {
+  const float2 one = make_float2(1.0f, 1.0f);
+  const float2 den = __fadd2_rn(one, make_float2(__expf(-y.x), __expf(-y.y)));
+  const float2 sg = make_float2(__fdividef(1.0f, den.x), __fdividef(1.0f, den.y));
+  const float2 om = __ffma2_rn(make_float2(-1.0f, -1.0f), sg, one);  // 1 - s
+  return __fmul2_rn(sg, __ffma2_rn(y, om, one));
 }
 
 constexpr int COL_TOK = 128;   // tokens per column chunk; one warp walks one chunk
@@ -115,22 +121,65 @@ constexpr int COL_FPT = 2;     // features per lane (float2 loads)
 constexpr int COL_FEAT = 32 * COL_FPT;  // features per warp, one dalpha partial per token
 constexpr int COL_WARPS = 4;   // chunks per block
 
+constexpr int COL_RING = 16;  // tokens per warp in a shared-memory ring, 15 of them in flight
+
 __device__ __forceinline__ float2 ld_f2(const float* p) {
   return *reinterpret_cast<const float2*>(p);
 }
 
-// Emit token j of the walk: dv = alpha dvt as two bf16, and the warp's
-// partial of dalpha = <dvt, v> over its 64 features (the lane's pair first,
-// then a fixed butterfly).
-__device__ __forceinline__ void col_emit(float2 r, float2 vv, float a, int j, int ld, int np,
-                                         __nv_bfloat16* __restrict__ dvb,
-                                         float* __restrict__ pab) {
-  *reinterpret_cast<__nv_bfloat162*>(dvb + j * ld) = __floats2bfloat162_rn(a * r.x, a * r.y);
-  float p = fmaf(r.x, vv.x, r.y * vv.y);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-  if ((threadIdx.x & 31) == 0) pab[j * np] = p;
+// 8-byte asynchronous copy global -> shared (this thread's own slot).
+__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N_PENDING>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N_PENDING) : "memory");
+}
+
+// The warp's dalpha partials, 32 tokens at a time: lane L's share of token
+// j sits at [j % 32][L] (rows padded to 33 so that both the writes and the
+// row sums below are free of bank conflicts).
+struct ColPartials {
+  float p[32][33];
+};
+
+// Sum rows 0 .. cnt-1 (tokens jbase ..) of the buffer across the 32 lanes,
+// lane r adding row r in lane order, and store them; warp-uniform call.
+__device__ __forceinline__ void col_flush(ColPartials& pb, int jbase, int cnt, int np,
+                                          float* __restrict__ pab) {
+  __syncwarp();
+  const int lane = threadIdx.x & 31;
+  if (lane < cnt) {
+    float sum = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c) sum += pb.p[lane][c];
+    pab[(jbase + lane) * np] = sum;
+  }
+  __syncwarp();
+}
+
+// Emit token j of the walk: dv = alpha dvt as two bf16, and the lane's share
+// of dalpha = <dvt, v> over its two features; every 32nd token flushes the
+// warp's partials.  Tokens are emitted once each, in increasing order.
+__device__ __forceinline__ void col_emit(float2 r, float2 vv, float a, int j, int ld, int np,
+                                         __nv_bfloat16* __restrict__ dvb, ColPartials& pb,
+                                         float* __restrict__ pab) {
+  const float2 dvr = __fmul2_rn(make_float2(a, a), r);
+  *reinterpret_cast<__nv_bfloat162*>(dvb + j * ld) = __floats2bfloat162_rn(dvr.x, dvr.y);
+  pb.p[j & 31][threadIdx.x & 31] = fmaf(r.x, vv.x, r.y * vv.y);
+  if ((j & 31) == 31) col_flush(pb, j - 31, 32, np, pab);
+}
+
+// dynamic shared memory of the column walk: per warp the copy ring, the
+// dalpha partials and the chunk's gates
+constexpr int kColSmem =
+    COL_WARPS * (COL_RING * 2 * 32 * 8 + (int)sizeof(ColPartials) + (COL_TOK + 6) * 4);
 
 // One warp per (chunk of COL_TOK tokens, 64 features), each lane holding two
 // adjacent features, walking the chunk in token order.  The warp keeps, for
@@ -139,23 +188,32 @@ __device__ __forceinline__ void col_emit(float2 r, float2 vv, float a, int j, in
 // past the sequence end absent), to which each new dy_t adds its share.  At
 // token t it forms y_t and dy_t; dvt of token t-3 is then complete, and at a
 // sequence end so are t-2, t-1 and t.  The walk runs 3 tokens past the chunk
-// for the last tokens' dy.  `live` counts the ring's tokens that belong to
+// for the last tokens' dy.  v and dout of the next COL_RING - 1 tokens are
+// in flight into a per-warp shared-memory ring (asynchronous copies, each
+// lane its own 8 bytes), enough bytes in flight per SM to stream at HBM
+// rate with four warps per block.  `live` counts the ring's tokens that belong to
 // t's sequence and to this chunk's walk (tokens before the chunk are emitted
 // by the previous chunk's walk).  For each completed token it writes dv
 // (bf16, for the GEMMs) and the warp's partial of dalpha,
-// dalpha_part[token][f / 64]; at the end the chunk's partial conv-weight
+// dalpha_part[token][f / 64] (the lanes' shares summed per 32 tokens, from
+// shared memory, in lane order); at the end the chunk's partial conv-weight
 // gradient, part[chunk][f] = sum over its tokens of
 // dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).  Warps are independent (all
 // lanes of one walk the same tokens, so the butterflies run on uniform
 // branches); the block only groups COL_WARPS chunks for scheduling.
-__global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
+__global__ void __launch_bounds__(32 * COL_WARPS, 4) bw_col_kernel(
     const float* __restrict__ v, const float* __restrict__ alpha,
     const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
     int ld, int chunks, __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part,
     float4* __restrict__ part) {
   // v and dv rows are ld apart (they share rows with k and dk), dout rows d
-  __shared__ float al_all[COL_WARPS][COL_TOK + 6];
+  extern __shared__ __align__(16) unsigned char col_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto* ring_all = reinterpret_cast<float2(*)[COL_RING][2][32]>(col_smem);  // [slot][v, dout][lane]
+  auto* pb_all = reinterpret_cast<ColPartials*>(col_smem + COL_WARPS * COL_RING * 2 * 32 * 8);
+  auto* al_all = reinterpret_cast<float(*)[COL_TOK + 6]>(col_smem + COL_WARPS * COL_RING * 2 * 32 * 8 +
+                                                          COL_WARPS * sizeof(ColPartials));
+  ColPartials& pb = pb_all[warp];
   const int chunk = blockIdx.x * COL_WARPS + warp;
   if (chunk >= chunks) return;  // no block-wide barrier follows
   const int f = blockIdx.y * COL_FEAT + lane * COL_FPT;
@@ -171,6 +229,9 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
   }
   __syncwarp();
   const float4 wx = __ldg(conv_w + f), wy = __ldg(conv_w + f + 1);
+  // the weights as (feature x, feature y) pairs: W0 multiplies vt_{t-3}, W3 vt_t
+  const float2 W0 = make_float2(wx.x, wy.x), W1 = make_float2(wx.y, wy.y);
+  const float2 W2 = make_float2(wx.z, wy.z), W3 = make_float2(wx.w, wy.w);
   int pos = (int)(t0 % T);
   float2 s1 = make_float2(0.f, 0.f), s2 = s1, s3 = s1;  // vt of t-1, t-2, t-3
   if (pos >= 1) {
@@ -187,65 +248,63 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
   }
   float2 A1 = make_float2(0.f, 0.f), A2 = A1, A3 = A1;  // partial dvt of t-1, t-2, t-3
   float2 v1 = A1, v2 = A1, v3 = A1;                      // v of t-1, t-2, t-3
-  float4 cx = make_float4(0.f, 0.f, 0.f, 0.f), cy = cx;  // conv-weight partials
+  // conv-weight partials, (x, y) pairs for w_0 .. w_3
+  float2 C0 = make_float2(0.f, 0.f), C1 = C0, C2 = C0, C3 = C0;
   int live = 0;
   __nv_bfloat16* dvb = dv + t0 * ld + f;
   float* pab = dalpha_part + t0 * np + blockIdx.y;
   const int n_chunk = (int)(t1 - t0), n_walk = (int)(t_stop - t0);
-  // the next PF tokens' v and dout, loaded ahead of the walk
-  constexpr int PF = 4;
-  float2 pv[PF], pu[PF];
+  // token q's v and dout go to ring slot q % COL_RING; the slot refilled at
+  // step i held token i - 1, whose values step i - 1 has already used
+  float2 (*ring)[2][32] = ring_all[warp];
   const float* vp = v + t0 * ld + f;
   const float* up = dout + t0 * d + f;
 #pragma unroll
-  for (int q = 0; q < PF; ++q) {
-    pv[q] = q < n_walk ? ld_f2(vp + (int64_t)q * ld) : make_float2(0.f, 0.f);
-    pu[q] = q < n_walk ? ld_f2(up + (int64_t)q * d) : make_float2(0.f, 0.f);
+  for (int q = 0; q < COL_RING - 1; ++q) {
+    if (q < n_walk) {
+      cp_async8(&ring[q][0][lane], vp);
+      cp_async8(&ring[q][1][lane], up);
+    }
+    cp_async_commit();
+    vp += ld;
+    up += d;
   }
-  vp += (int64_t)PF * ld;
-  up += (int64_t)PF * d;
 #pragma unroll 4
   for (int i = 0; i < n_walk; ++i) {
-    const float2 vr = pv[0], ut = pu[0];
+    cp_async_wait<COL_RING - 2>();  // token i's copies have landed
+    const int slot = i % COL_RING;
+    const float2 vr = ring[slot][0][lane], ut = ring[slot][1][lane];
     const float at = al_s[i + 3];
-#pragma unroll
-    for (int q = 0; q < PF - 1; ++q) {
-      pv[q] = pv[q + 1];
-      pu[q] = pu[q + 1];
+    if (i + COL_RING - 1 < n_walk) {
+      const int refill = (i + COL_RING - 1) % COL_RING;
+      cp_async8(&ring[refill][0][lane], vp);
+      cp_async8(&ring[refill][1][lane], up);
     }
-    const bool more = i + PF < n_walk;
-    pv[PF - 1] = more ? ld_f2(vp) : make_float2(0.f, 0.f);
-    pu[PF - 1] = more ? ld_f2(up) : make_float2(0.f, 0.f);
+    cp_async_commit();
     vp += ld;
     up += d;
     if (pos == 0) {  // a sequence starts at t
       s1 = s2 = s3 = make_float2(0.f, 0.f);
       live = 0;
     }
-    const float2 vt = make_float2(at * vr.x, at * vr.y);
-    float2 g;
-    g.x = ut.x * silu_grad(fmaf(wx.x, s3.x, fmaf(wx.y, s2.x, fmaf(wx.z, s1.x, wx.w * vt.x))));
-    g.y = ut.y * silu_grad(fmaf(wy.x, s3.y, fmaf(wy.y, s2.y, fmaf(wy.z, s1.y, wy.w * vt.y))));
+    const float2 vt = __fmul2_rn(make_float2(at, at), vr);
+    const float2 y = __ffma2_rn(W0, s3, __ffma2_rn(W1, s2, __ffma2_rn(W2, s1, __fmul2_rn(W3, vt))));
+    const float2 g = __fmul2_rn(ut, silu_grad2(y));
     if (i < n_chunk) {
-      cx.x = fmaf(g.x, s3.x, cx.x);
-      cx.y = fmaf(g.x, s2.x, cx.y);
-      cx.z = fmaf(g.x, s1.x, cx.z);
-      cx.w = fmaf(g.x, vt.x, cx.w);
-      cy.x = fmaf(g.y, s3.y, cy.x);
-      cy.y = fmaf(g.y, s2.y, cy.y);
-      cy.z = fmaf(g.y, s1.y, cy.z);
-      cy.w = fmaf(g.y, vt.y, cy.w);
+      C0 = __ffma2_rn(g, s3, C0);
+      C1 = __ffma2_rn(g, s2, C1);
+      C2 = __ffma2_rn(g, s1, C2);
+      C3 = __ffma2_rn(g, vt, C3);
     }
     if (live == 3)  // token t-3 is complete
-      col_emit(make_float2(fmaf(wx.x, g.x, A3.x), fmaf(wy.x, g.y, A3.y)), v3, al_s[i], i - 3,
-               ld, np, dvb, pab);
-    const float2 B2 = make_float2(fmaf(wx.y, g.x, A2.x), fmaf(wy.y, g.y, A2.y));
-    const float2 B1 = make_float2(fmaf(wx.z, g.x, A1.x), fmaf(wy.z, g.y, A1.y));
-    const float2 B0 = make_float2(fmaf(wx.w, g.x, ut.x), fmaf(wy.w, g.y, ut.y));
+      col_emit(__ffma2_rn(W0, g, A3), v3, al_s[i], i - 3, ld, np, dvb, pb, pab);
+    const float2 B2 = __ffma2_rn(W1, g, A2);
+    const float2 B1 = __ffma2_rn(W2, g, A1);
+    const float2 B0 = __ffma2_rn(W3, g, ut);
     if (pos == T - 1) {  // the sequence ends at t: its last tokens are complete
-      if (live >= 2 && i - 2 < n_chunk) col_emit(B2, v2, al_s[i + 1], i - 2, ld, np, dvb, pab);
-      if (live >= 1 && i - 1 < n_chunk) col_emit(B1, v1, al_s[i + 2], i - 1, ld, np, dvb, pab);
-      if (i < n_chunk) col_emit(B0, vr, at, i, ld, np, dvb, pab);
+      if (live >= 2 && i - 2 < n_chunk) col_emit(B2, v2, al_s[i + 1], i - 2, ld, np, dvb, pb, pab);
+      if (live >= 1 && i - 1 < n_chunk) col_emit(B1, v1, al_s[i + 2], i - 1, ld, np, dvb, pb, pab);
+      if (i < n_chunk) col_emit(B0, vr, at, i, ld, np, dvb, pb, pab);
     }
     A3 = B2;
     A2 = B1;
@@ -259,8 +318,9 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     live = live < 3 ? live + 1 : 3;
     pos = pos + 1 == T ? 0 : pos + 1;
   }
-  part[(int64_t)chunk * d + f] = cx;
-  part[(int64_t)chunk * d + f + 1] = cy;
+  if (n_chunk & 31) col_flush(pb, n_chunk & ~31, n_chunk & 31, np, pab);
+  part[(int64_t)chunk * d + f] = make_float4(C0.x, C1.x, C2.x, C3.x);
+  part[(int64_t)chunk * d + f + 1] = make_float4(C0.y, C1.y, C2.y, C3.y);
 }
 
 constexpr int ROW_THREADS = 256;
@@ -279,7 +339,8 @@ __device__ __forceinline__ float4 bf16x4_to_f4(uint2 u) {
 // registers; <h,h>, <k,k>, <h,k> and dalpha (the column walk's d/64
 // partials, added in order by the first warp) are reduced together in one
 // fixed-order pass; then dk (bf16, for the GEMMs) and dh are written.
-__global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
+template <int ITEMS>  // ceil(d / (ROW_THREADS * ROW_VEC)) <= ROW_MAX_ITEMS
+__global__ void __launch_bounds__(ROW_THREADS, 4) bw_row_kernel(
     const __nv_bfloat16* __restrict__ h, const float* __restrict__ k,
     const float* __restrict__ alpha, const float* __restrict__ dout,
     const float* __restrict__ dalpha_part, int64_t N, int d, int ld, float* __restrict__ dh,
@@ -292,20 +353,24 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
   const __nv_bfloat16* hr = h + t * d;
   const float* kr = k + t * ld;
   const float* ur = dout + t * d;
-  float4 hv[ROW_MAX_ITEMS], kv[ROW_MAX_ITEMS], uv[ROW_MAX_ITEMS];
+  uint2 hb[ITEMS];  // h kept as bf16 (4 per item) until used
+  float4 kv[ITEMS], uv[ITEMS];
   float shh = 0.f, skk = 0.f, shk = 0.f;
 #pragma unroll
-  for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
+  for (int q = 0; q < ITEMS; ++q) {
     const int c = threadIdx.x + q * ROW_THREADS;
-    hv[q] = kv[q] = uv[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    hb[q] = make_uint2(0u, 0u);
+    kv[q] = uv[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (c < nv) {
-      hv[q] = bf16x4_to_f4(*reinterpret_cast<const uint2*>(hr + c * ROW_VEC));
+      hb[q] = *reinterpret_cast<const uint2*>(hr + c * ROW_VEC);
       kv[q] = *reinterpret_cast<const float4*>(kr + c * ROW_VEC);
       uv[q] = __ldcs(reinterpret_cast<const float4*>(ur + c * ROW_VEC));
     }
   }
+  float4 hv[ITEMS];
 #pragma unroll
-  for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
+  for (int q = 0; q < ITEMS; ++q) {
+    hv[q] = bf16x4_to_f4(hb[q]);
     shh = fmaf(hv[q].x, hv[q].x, fmaf(hv[q].y, hv[q].y, fmaf(hv[q].z, hv[q].z, fmaf(hv[q].w, hv[q].w, shh))));
     skk = fmaf(kv[q].x, kv[q].x, fmaf(kv[q].y, kv[q].y, fmaf(kv[q].z, kv[q].z, fmaf(kv[q].w, kv[q].w, skk))));
     shk = fmaf(hv[q].x, kv[q].x, fmaf(hv[q].y, kv[q].y, fmaf(hv[q].z, kv[q].z, fmaf(hv[q].w, kv[q].w, shk))));
@@ -347,10 +412,10 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
   __nv_bfloat16* dkr = dk_out + t * ld;
   float* dhr = dh + t * d;
 #pragma unroll
-  for (int q = 0; q < ROW_MAX_ITEMS; ++q) {
+  for (int q = 0; q < ITEMS; ++q) {
     const int c4 = threadIdx.x + q * ROW_THREADS;
     if (c4 < nv) {
-      const float4 hq = hv[q], kq = kv[q], uq = uv[q];
+      const float4 hq = bf16x4_to_f4(hb[q]), kq = kv[q], uq = uv[q];
       const __nv_bfloat162 k01 = __floats2bfloat162_rn(rk * (crh * hq.x) - ck * kq.x,
                                                       rk * (crh * hq.y) - ck * kq.y);
       const __nv_bfloat162 k23 = __floats2bfloat162_rn(rk * (crh * hq.z) - ck * kq.z,
@@ -487,12 +552,21 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
     return rc;
   if ((rc = gemm_rm(hd, false, true, n, 2 * d, E, e, E, w.Wkv, E, w.kv, 2 * d, 0.f))) return rc;
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
+  if ((rc = ck(cudaFuncSetAttribute(bw_col_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kColSmem))))
+    return rc;
   bw_col_kernel<<<dim3((unsigned)((chunks + COL_WARPS - 1) / COL_WARPS), (unsigned)(d / COL_FEAT)),
-                  32 * COL_WARPS, 0, s>>>(w.kv + d, alpha, reinterpret_cast<const float4*>(conv_w),
+                  32 * COL_WARPS, kColSmem, s>>>(w.kv + d, alpha, reinterpret_cast<const float4*>(conv_w),
                                           dout, N, T, d, 2 * d, chunks, w.dkv + d,
                                           w.dalpha_part, w.part);
-  bw_row_kernel<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.kv, alpha, dout, w.dalpha_part, N, d,
-                                                    2 * d, dh, w.dkv);
+  {
+    const int items = (d / ROW_VEC + ROW_THREADS - 1) / ROW_THREADS;
+    auto row = items == 1 ? bw_row_kernel<1>
+             : items == 2 ? bw_row_kernel<2>
+             : items == 3 ? bw_row_kernel<3> : bw_row_kernel<4>;
+    row<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.kv, alpha, dout, w.dalpha_part, N, d, 2 * d, dh,
+                                           w.dkv);
+  }
   bw_dconv_reduce_kernel<<<(unsigned)((d + 31) / 32), 32 * DCONV_WARPS, 0, s>>>(
       w.part, chunks, d, reinterpret_cast<float4*>(dconv_w));
   if ((rc = ck(cudaGetLastError()))) return rc;
