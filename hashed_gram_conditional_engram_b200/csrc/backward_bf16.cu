@@ -16,6 +16,7 @@
 #include <cublas_v2.h>
 #include <dlfcn.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "internal.cuh"
@@ -334,102 +335,195 @@ __device__ __forceinline__ float4 bf16x4_to_f4(uint2 u) {
   return make_float4(a.x, a.y, b.x, b.y);
 }
 
-// One block per token: the gate and both RMSNorm backwards need whole-row
-// sums.  The row's h, k and dout are read once (4 features per load) into
-// registers; <h,h>, <k,k>, <h,k> and dalpha (the column walk's d/64
+constexpr int ROW_STAGES = 2;
+constexpr uint64_t ROW_WAIT_NS = 2000000000ull;  // 2 s: a copy that has not landed by then never will
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from global to this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Wait for the phase of `bar` with the given parity; false after ROW_WAIT_NS.
+__device__ __forceinline__ bool row_wait(uint64_t* bar, uint32_t parity) {
+  uint64_t t0 = 0;
+  for (int spin = 0;; ++spin) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    if (ok) return true;
+    uint64_t now;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+    if (spin == 0) t0 = now;
+    else if (now - t0 > ROW_WAIT_NS) return false;
+  }
+}
+
+// Shared memory of one stage of the row kernel: the token's h (bf16), k and
+// dout (fp32) rows and its d/64 dalpha partials; all offsets are multiples of
+// 16 bytes because d is a multiple of 256.
+__host__ __device__ constexpr size_t row_stage_bytes(int d) {
+  return (size_t)d * 2 + (size_t)d * 4 + (size_t)d * 4 + (size_t)(d / COL_FEAT) * 4;
+}
+
+// The gate and both RMSNorm backwards need whole-row sums, so each token is
+// one step of one block: a persistent block walks tokens blockIdx.x,
+// + gridDim.x, ..., with the next token's rows already in flight into the
+// other shared-memory stage (bulk copies issued by one thread, completing on
+// an mbarrier).  Each thread takes 4 features per item from shared memory
+// into registers; <h,h>, <k,k>, <h,k> and dalpha (the column walk's d/64
 // partials, added in order by the first warp) are reduced together in one
-// fixed-order pass; then dk (bf16, for the GEMMs) and dh are written.
+// fixed-order pass, whose barrier also frees the stage for the token after
+// next; then dk (bf16, for the GEMMs) and dh are written.  A copy that never
+// lands sets ENGRAM_STATUS_TIMEOUT and the block stops.
 template <int ITEMS>  // ceil(d / (ROW_THREADS * ROW_VEC)) <= ROW_MAX_ITEMS
-__global__ void __launch_bounds__(ROW_THREADS, 4) bw_row_kernel(
+__global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     const __nv_bfloat16* __restrict__ h, const float* __restrict__ k,
     const float* __restrict__ alpha, const float* __restrict__ dout,
     const float* __restrict__ dalpha_part, int64_t N, int d, int ld, float* __restrict__ dh,
-    __nv_bfloat16* __restrict__ dk_out) {
+    __nv_bfloat16* __restrict__ dk_out, unsigned int* status) {
   // k and dk rows are ld apart (they share rows with v and dv)
-  __shared__ float4 red[ROW_THREADS / 32];
-  const int64_t t = blockIdx.x;
-  if (t >= N) return;
+  extern __shared__ __align__(128) unsigned char row_smem[];
+  __shared__ uint64_t full[ROW_STAGES];
+  __shared__ float4 red[2][ROW_THREADS / 32];
+  __shared__ int abort_flag;
+  const int np = d / COL_FEAT;
+  const size_t SB = row_stage_bytes(d);
+  const uint32_t hb_bytes = (uint32_t)d * 2, f_bytes = (uint32_t)d * 4, p_bytes = (uint32_t)np * 4;
+  const int64_t G = gridDim.x;
+  unsigned pend = 0;  // thread 0: stages with a copy issued and not yet seen landed
+  auto issue = [&](int64_t t, int st) {  // thread 0
+    pend |= 1u << st;
+    unsigned char* base = row_smem + st * SB;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&full[st])),
+                 "r"(hb_bytes + 2 * f_bytes + p_bytes)
+                 : "memory");
+    bulk_load(base, h + t * d, hb_bytes, &full[st]);
+    bulk_load(base + hb_bytes, k + t * ld, f_bytes, &full[st]);
+    bulk_load(base + hb_bytes + f_bytes, dout + t * d, f_bytes, &full[st]);
+    bulk_load(base + hb_bytes + 2 * f_bytes, dalpha_part + t * np, p_bytes, &full[st]);
+  };
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < ROW_STAGES; ++st)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[st])));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    abort_flag = 0;
+    for (int st = 0; st < ROW_STAGES; ++st)
+      if (blockIdx.x + st * G < N) issue(blockIdx.x + st * G, st);
+  }
+  __syncthreads();
   const int nv = d / ROW_VEC;
-  const __nv_bfloat16* hr = h + t * d;
-  const float* kr = k + t * ld;
-  const float* ur = dout + t * d;
-  uint2 hb[ITEMS];  // h kept as bf16 (4 per item) until used
-  float4 kv[ITEMS], uv[ITEMS];
-  float shh = 0.f, skk = 0.f, shk = 0.f;
+  const float invd = 1.0f / (float)d, isd = rsqrtf((float)d);
+  int it = 0;
+  for (int64_t t = blockIdx.x; t < N; t += G, ++it) {
+    const int st = it % ROW_STAGES;
+    const unsigned char* base = row_smem + st * SB;
+    if (row_wait(&full[st], (uint32_t)(it / ROW_STAGES) & 1u)) {
+      pend &= ~(1u << st);
+    } else {
+      abort_flag = 1;  // every thread reaches the barrier below, then all stop
+      atomicOr(status, ENGRAM_STATUS_TIMEOUT);
+    }
+    const __nv_bfloat16* hs = reinterpret_cast<const __nv_bfloat16*>(base);
+    const float* ks = reinterpret_cast<const float*>(base + hb_bytes);
+    const float* us = reinterpret_cast<const float*>(base + hb_bytes + f_bytes);
+    const float* ps = reinterpret_cast<const float*>(base + hb_bytes + 2 * f_bytes);
+    uint2 hb[ITEMS];  // h kept as bf16 (4 per item) until used
+    float4 kv[ITEMS], uv[ITEMS];
+    float shh = 0.f, skk = 0.f, shk = 0.f;
 #pragma unroll
-  for (int q = 0; q < ITEMS; ++q) {
-    const int c = threadIdx.x + q * ROW_THREADS;
-    hb[q] = make_uint2(0u, 0u);
-    kv[q] = uv[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (c < nv) {
-      hb[q] = *reinterpret_cast<const uint2*>(hr + c * ROW_VEC);
-      kv[q] = *reinterpret_cast<const float4*>(kr + c * ROW_VEC);
-      uv[q] = __ldcs(reinterpret_cast<const float4*>(ur + c * ROW_VEC));
+    for (int q = 0; q < ITEMS; ++q) {
+      const int c = threadIdx.x + q * ROW_THREADS;
+      hb[q] = make_uint2(0u, 0u);
+      kv[q] = uv[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c < nv) {
+        hb[q] = *reinterpret_cast<const uint2*>(hs + c * ROW_VEC);
+        kv[q] = *reinterpret_cast<const float4*>(ks + c * ROW_VEC);
+        uv[q] = *reinterpret_cast<const float4*>(us + c * ROW_VEC);
+      }
+      const float4 hq = bf16x4_to_f4(hb[q]), kq = kv[q];
+      shh = fmaf(hq.x, hq.x, fmaf(hq.y, hq.y, fmaf(hq.z, hq.z, fmaf(hq.w, hq.w, shh))));
+      skk = fmaf(kq.x, kq.x, fmaf(kq.y, kq.y, fmaf(kq.z, kq.z, fmaf(kq.w, kq.w, skk))));
+      shk = fmaf(hq.x, kq.x, fmaf(hq.y, kq.y, fmaf(hq.z, kq.z, fmaf(hq.w, kq.w, shk))));
+    }
+    float sgv = 0.f;
+    if (threadIdx.x < 32)
+      for (int i = threadIdx.x; i < np; i += 32) sgv += ps[i];
+    float4 r = make_float4(shh, skk, shk, sgv);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      r.x += __shfl_xor_sync(0xffffffffu, r.x, o);
+      r.y += __shfl_xor_sync(0xffffffffu, r.y, o);
+      r.z += __shfl_xor_sync(0xffffffffu, r.z, o);
+      r.w += __shfl_xor_sync(0xffffffffu, r.w, o);
+    }
+    float4* rb = red[it & 1];  // two buffers: a fast thread's next write never meets a slow read
+    if ((threadIdx.x & 31) == 0) rb[threadIdx.x >> 5] = r;
+    __syncthreads();  // all reads of this stage are done: it can be refilled
+    if (abort_flag) break;
+    if (threadIdx.x == 0 && t + ROW_STAGES * G < N) issue(t + ROW_STAGES * G, st);
+    r = rb[0];
+#pragma unroll
+    for (int i = 1; i < ROW_THREADS / 32; ++i) {
+      r.x += rb[i].x;
+      r.y += rb[i].y;
+      r.z += rb[i].z;
+      r.w += rb[i].w;
+    }
+    const float rh = rsqrtf(r.x * invd + BW_RMS_EPS), rk = rsqrtf(r.y * invd + BW_RMS_EPS);
+    const float shk_all = r.z;
+    const float a = __ldg(alpha + t);
+    const float c = r.w * a * (1.0f - a) * isd;  // dz / sqrt(d): dh^ = c k^, dk^ = c h^
+    const float ch = rh * rh * rh * (c * rk * shk_all) * invd;  // r_h^3 <dh^, h> / d
+    const float ck = rk * rk * rk * (c * rh * shk_all) * invd;  // r_k^3 <dk^, k> / d
+    const float crh = c * rh, crk = c * rk;
+    __nv_bfloat16* dkr = dk_out + t * ld;
+    float* dhr = dh + t * d;
+#pragma unroll
+    for (int q = 0; q < ITEMS; ++q) {
+      const int c4 = threadIdx.x + q * ROW_THREADS;
+      if (c4 < nv) {
+        const float4 hq = bf16x4_to_f4(hb[q]), kq = kv[q], uq = uv[q];
+        const __nv_bfloat162 k01 = __floats2bfloat162_rn(rk * (crh * hq.x) - ck * kq.x,
+                                                        rk * (crh * hq.y) - ck * kq.y);
+        const __nv_bfloat162 k23 = __floats2bfloat162_rn(rk * (crh * hq.z) - ck * kq.z,
+                                                        rk * (crh * hq.w) - ck * kq.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&k01);
+        pk.y = *reinterpret_cast<const uint32_t*>(&k23);
+        *reinterpret_cast<uint2*>(dkr + c4 * ROW_VEC) = pk;
+        float4 o;
+        o.x = uq.x + rh * (crk * kq.x) - ch * hq.x;
+        o.y = uq.y + rh * (crk * kq.y) - ch * hq.y;
+        o.z = uq.z + rh * (crk * kq.z) - ch * hq.z;
+        o.w = uq.w + rh * (crk * kq.w) - ch * hq.w;
+        __stcs(reinterpret_cast<float4*>(dhr + c4 * ROW_VEC), o);
+      }
     }
   }
-  float4 hv[ITEMS];
-#pragma unroll
-  for (int q = 0; q < ITEMS; ++q) {
-    hv[q] = bf16x4_to_f4(hb[q]);
-    shh = fmaf(hv[q].x, hv[q].x, fmaf(hv[q].y, hv[q].y, fmaf(hv[q].z, hv[q].z, fmaf(hv[q].w, hv[q].w, shh))));
-    skk = fmaf(kv[q].x, kv[q].x, fmaf(kv[q].y, kv[q].y, fmaf(kv[q].z, kv[q].z, fmaf(kv[q].w, kv[q].w, skk))));
-    shk = fmaf(hv[q].x, kv[q].x, fmaf(hv[q].y, kv[q].y, fmaf(hv[q].z, kv[q].z, fmaf(hv[q].w, kv[q].w, shk))));
-  }
-  float sgv = 0.f;
-  if (threadIdx.x < 32) {
-    const int np = d / COL_FEAT;
-    const float* pp = dalpha_part + t * np;
-    for (int i = threadIdx.x; i < np; i += 32) sgv += pp[i];
-  }
-  float4 r = make_float4(shh, skk, shk, sgv);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    r.x += __shfl_xor_sync(0xffffffffu, r.x, o);
-    r.y += __shfl_xor_sync(0xffffffffu, r.y, o);
-    r.z += __shfl_xor_sync(0xffffffffu, r.z, o);
-    r.w += __shfl_xor_sync(0xffffffffu, r.w, o);
-  }
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = r;
-  __syncthreads();
-  r = red[0];
-#pragma unroll
-  for (int i = 1; i < ROW_THREADS / 32; ++i) {
-    r.x += red[i].x;
-    r.y += red[i].y;
-    r.z += red[i].z;
-    r.w += red[i].w;
-  }
-  shh = r.x;
-  skk = r.y;
-  shk = r.z;
-  const float invd = 1.0f / (float)d, isd = rsqrtf((float)d);
-  const float rh = rsqrtf(shh * invd + BW_RMS_EPS), rk = rsqrtf(skk * invd + BW_RMS_EPS);
-  const float a = alpha[t];
-  const float c = r.w * a * (1.0f - a) * isd;  // dz / sqrt(d): dh^ = c k^, dk^ = c h^
-  const float ch = rh * rh * rh * (c * rk * shk) * invd;   // r_h^3 <dh^, h> / d
-  const float ck = rk * rk * rk * (c * rh * shk) * invd;   // r_k^3 <dk^, k> / d
-  const float crh = c * rh, crk = c * rk;
-  __nv_bfloat16* dkr = dk_out + t * ld;
-  float* dhr = dh + t * d;
-#pragma unroll
-  for (int q = 0; q < ITEMS; ++q) {
-    const int c4 = threadIdx.x + q * ROW_THREADS;
-    if (c4 < nv) {
-      const float4 hq = bf16x4_to_f4(hb[q]), kq = kv[q], uq = uv[q];
-      const __nv_bfloat162 k01 = __floats2bfloat162_rn(rk * (crh * hq.x) - ck * kq.x,
-                                                      rk * (crh * hq.y) - ck * kq.y);
-      const __nv_bfloat162 k23 = __floats2bfloat162_rn(rk * (crh * hq.z) - ck * kq.z,
-                                                      rk * (crh * hq.w) - ck * kq.w);
-      uint2 pk;
-      pk.x = *reinterpret_cast<const uint32_t*>(&k01);
-      pk.y = *reinterpret_cast<const uint32_t*>(&k23);
-      *reinterpret_cast<uint2*>(dkr + c4 * ROW_VEC) = pk;
-      float4 o;
-      o.x = uq.x + rh * (crk * kq.x) - ch * hq.x;
-      o.y = uq.y + rh * (crk * kq.y) - ch * hq.y;
-      o.z = uq.z + rh * (crk * kq.z) - ch * hq.z;
-      o.w = uq.w + rh * (crk * kq.w) - ch * hq.w;
-      __stcs(reinterpret_cast<float4*>(dhr + c4 * ROW_VEC), o);
+  // on a timeout, let copies still in flight land (bounded) before the
+  // block's shared memory is released; a stage holds at most one, of the
+  // phase after the last one waited for
+  if (threadIdx.x == 0 && pend != 0) {
+    const int done = it;  // uses waited for: stage s had uses j < done with j % ROW_STAGES == s
+    for (int st = 0; st < ROW_STAGES; ++st) {
+      if (!(pend & (1u << st))) continue;
+      const int use = done / ROW_STAGES + (st < done % ROW_STAGES ? 1 : 0);
+      row_wait(&full[st], (uint32_t)use & 1u);
     }
   }
 }
@@ -536,8 +630,8 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   const int E = hp.E;
   if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J)) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
-  if (d > ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS || d % COL_FEAT != 0)
-    return ENGRAM_ERR_UNSUPPORTED;  // a row in registers; whole column blocks
+  // a row in registers; whole column blocks; 16-byte multiples for the row copies
+  if (d > ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS || d % 256 != 0) return ENGRAM_ERR_UNSUPPORTED;
   BwdBf16Ws w;
   bwd_bf16_layout(ws, N, d, E, hp.J, &w);
   if (de == nullptr) de = w.de;
@@ -564,8 +658,16 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
     auto row = items == 1 ? bw_row_kernel<1>
              : items == 2 ? bw_row_kernel<2>
              : items == 3 ? bw_row_kernel<3> : bw_row_kernel<4>;
-    row<<<(unsigned)N, ROW_THREADS, 0, s>>>(h, w.kv, alpha, dout, w.dalpha_part, N, d, 2 * d, dh,
-                                           w.dkv);
+    const int smem = (int)(ROW_STAGES * row_stage_bytes(d));
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((rc = ck(cudaFuncSetAttribute(row, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) ||
+        (rc = ck(cudaGetDevice(&dev))) ||
+        (rc = ck(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))) ||
+        (rc = ck(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, row, ROW_THREADS, smem))))
+      return rc;
+    const int64_t grid = std::min<int64_t>(N, (int64_t)sms * std::max(per_sm, 1));
+    row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, w.kv, alpha, dout, w.dalpha_part, N, d,
+                                                  2 * d, dh, w.dkv, status_ptr());
   }
   bw_dconv_reduce_kernel<<<(unsigned)((d + 31) / 32), 32 * DCONV_WARPS, 0, s>>>(
       w.part, chunks, d, reinterpret_cast<float4*>(dconv_w));

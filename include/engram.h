@@ -201,12 +201,15 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
  * Each table row's gradient is summed in fp32 over its tokens in ascending
  * token order (see engram_table_grad), so it is reproducible bit for bit.
  * ENGRAM_F32: any branch count; the arithmetic runs in fp64.
- * ENGRAM_BF16: one branch, d_model <= 4,096; e, h, Wk, Wv bf16 as in the forward, `saved`
+ * ENGRAM_BF16: one branch, d_model a multiple of 256 and <= 4,096 (else
+ * ENGRAM_ERR_UNSUPPORTED); e, h, Wk, Wv bf16 as in the forward, `saved`
  * (the forward's alpha) required; dout and every gradient fp32.  The
- * elementwise part runs in fp32; the four plain GEMMs (k and v recomputed in
- * fp32, dW_k and dW_v, de) run in cuBLAS with bf16 operands (dk and dv
- * rounded to bf16 once) and fp32 accumulation, loaded on first use
- * (ENGRAM_ERR_UNSUPPORTED if libcublas.so.12 cannot be loaded).
+ * elementwise part runs in fp32; the plain GEMMs (k and v recomputed in fp32
+ * as one GEMM against [W_k; W_v], [dW_k; dW_v] as one, de as one with
+ * K = 2 d_model) run in cuBLAS with bf16 operands (dk and dv rounded to bf16
+ * once) and fp32 accumulation, loaded on first use (ENGRAM_ERR_UNSUPPORTED
+ * if libcublas.so.12 cannot be loaded).  A device-side wait that runs out
+ * sets ENGRAM_STATUS_TIMEOUT.
  */
 int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,
                     const void* Wk, const void* Wv, const float* conv_w, const float* saved,
