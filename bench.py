@@ -570,8 +570,17 @@ def _graph_time(fn, steps, warmup, stream):
 def bench_fwd_bwd_27b(dev, steps=10):
     """Training step of the 27B-shaped layer (8 x 4,096 tokens, d 2,560, 16 x
     80 dims, 5.7B-parameter bf16 table): hash, forward (gather, fused passes,
-    alpha saved), backward (bf16: elementwise kernels, cuBLAS GEMMs, sparse
-    table gradient)."""
+    alpha, k and v saved), backward (bf16: elementwise kernels, cuBLAS GEMMs,
+    sparse table gradient); and the same with k and v recomputed in the
+    backward instead of saved."""
+    kept = _fwd_bwd_27b_run(dev, steps, save_kv=True)
+    recomputed = _fwd_bwd_27b_run(dev, steps, save_kv=False)
+    kept["recompute_kv"] = {k: recomputed[k] for k in ("ms_per_step", "fwd_bwd_tokens_per_s",
+                                                       "breakdown_ms")}
+    return kept
+
+
+def _fwd_bwd_27b_run(dev, steps, save_kv):
     import torch
     from hashed_gram_conditional_engram_b200 import engram as eg
     from hashed_gram_conditional_engram_b200 import synth
@@ -586,7 +595,8 @@ def bench_fwd_bwd_27b(dev, steps=10):
     proj = torch.empty(w.V, dtype=torch.int32, device=dev)
     vb = eg.engram_workspace_size(None, eg.WS_VOCAB, w.V)
     V_c = eg.engram_build_vocab_proj(keys, w.V, proj, torch.empty(vb, dtype=torch.uint8, device=dev), vb)
-    cfg = eg.make_cfg(w.K, w.D_h, w.d, 1, w.V, V_c, eg.BF16, w.rows, mult)
+    cfg = eg.make_cfg(w.K, w.D_h, w.d, 1, w.V, V_c, eg.BF16, w.rows, mult,
+                      flags=eg.SAVE_KV if save_kv else 0)
     N, E = w.N, w.E
     ids = torch.from_numpy(ids_np).to(dev)
     idx = torch.empty((w.B, w.T, w.J), dtype=torch.int32, device=dev)
@@ -628,12 +638,14 @@ def bench_fwd_bwd_27b(dev, steps=10):
         torch.cuda.synchronize()
     if eg.engram_get_status(s) != 0:
         raise RuntimeError("device status word set in the 27B-shaped training step")
-    bwd_flops = 2.0 * N * E * w.d * 6   # k, v recomputed; dW_k, dW_v; two GEMMs for de
+    # GEMMs: [k | v] recomputed unless saved; [dW_k; dW_v]; de with K = 2d
+    bwd_flops = 2.0 * N * E * (2 * w.d) * (2 if save_kv else 3)
     t_bwd = ev[1].elapsed_time(ev[2])
     del table, dense, bws, fws
     torch.cuda.empty_cache()
     return {"workload": "layer27b training step: 8 x 4,096 tokens, d 2,560, 16 heads x 80 dims, "
-                        "5.7B bf16 params; forward (hash, gather, fused passes) + bf16 backward",
+                        "5.7B bf16 params; forward (hash, gather, fused passes"
+                        + (", k and v saved" if save_kv else "") + ") + bf16 backward",
             "fwd_bwd_tokens_per_s": N / (ms / 1e3), "ms_per_step": ms,
             "breakdown_ms": {"forward": ev[0].elapsed_time(ev[1]), "backward": t_bwd},
             "backward_gemm_tflops": bwd_flops / (t_bwd / 1e3) / 1e12}

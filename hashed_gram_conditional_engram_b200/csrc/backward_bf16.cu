@@ -572,7 +572,7 @@ struct BwdBf16Ws {
   // bf16 rounding of k or v would show at full size in a small result.
   // They share rows (kv [N, 2d] = [k | v]), as do dk and dv, and W_k, W_v
   // are stacked (Wkv [2d, E]), so that each pair of GEMMs is one.
-  float* kv;
+  float* kv;  // recomputed here, or NULL when the forward saved them
   __nv_bfloat16* dkv;
   __nv_bfloat16* Wkv;
   float* dWkv;          // [2d, E], copied out to dWk and dWv
@@ -585,9 +585,10 @@ struct BwdBf16Ws {
 
 constexpr size_t up256b(size_t b) { return (b + 255) & ~(size_t)255; }
 
-size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, BwdBf16Ws* w) {
+size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved, BwdBf16Ws* w) {
   const int64_t chunks = (N + COL_TOK - 1) / COL_TOK;
-  const size_t KV = up256b((size_t)N * 2 * d * 4), DKV = up256b((size_t)N * 2 * d * 2);
+  const size_t KV = kv_saved ? 0 : up256b((size_t)N * 2 * d * 4);
+  const size_t DKV = up256b((size_t)N * 2 * d * 2);
   const size_t WKV = up256b((size_t)2 * d * E * 2), DW = up256b((size_t)2 * d * E * 4);
   const size_t DA = up256b((size_t)N * (d / COL_FEAT) * 4);
   const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
@@ -601,7 +602,7 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, BwdBf16Ws* w)
   }
   if (w != nullptr) {
     char* p = static_cast<char*>(base);
-    w->kv = reinterpret_cast<float*>(p + off[0]);
+    w->kv = kv_saved ? nullptr : reinterpret_cast<float*>(p + off[0]);
     w->dkv = reinterpret_cast<__nv_bfloat16*>(p + off[1]);
     w->Wkv = reinterpret_cast<__nv_bfloat16*>(p + off[2]);
     w->dWkv = reinterpret_cast<float*>(p + off[3]);
@@ -617,40 +618,45 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, BwdBf16Ws* w)
 
 }  // namespace
 
-size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J) {
-  return bwd_bf16_layout(nullptr, N, d, E, J, nullptr);
+size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved) {
+  return bwd_bf16_layout(nullptr, N, d, E, J, kv_saved, nullptr);
 }
 
 int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bfloat16* e,
                          const __nv_bfloat16* h, const __nv_bfloat16* Wk,
                          const __nv_bfloat16* Wv, const float* conv_w, const float* alpha,
-                         const float* dout, float* dh, float* dWk, float* dWv, float* dconv_w,
-                         float* de, int64_t* dtab_keys, float* dtab_rows, int32_t* n_unique,
-                         int64_t N, int T, int d, void* ws, size_t ws_bytes, cudaStream_t s) {
+                         const float* kv_saved, const float* dout, float* dh, float* dWk,
+                         float* dWv, float* dconv_w, float* de, int64_t* dtab_keys,
+                         float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, void* ws,
+                         size_t ws_bytes, cudaStream_t s) {
   const int E = hp.E;
-  if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J)) return ENGRAM_ERR_WORKSPACE;
+  const bool have_kv = kv_saved != nullptr;
+  if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J, have_kv)) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
   // a row in registers; whole column blocks; 16-byte multiples for the row copies
   if (d > ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS || d % 256 != 0) return ENGRAM_ERR_UNSUPPORTED;
   BwdBf16Ws w;
-  bwd_bf16_layout(ws, N, d, E, hp.J, &w);
+  bwd_bf16_layout(ws, N, d, E, hp.J, have_kv, &w);
   if (de == nullptr) de = w.de;
   cublasHandle_t hd;
   int rc = blas_handle(s, w.blas_ws, &hd);
   if (rc) return rc;
   const int n = (int)N;
-  // W_k and W_v stacked, then [k | v] = e [W_k; W_v]^T (fp32)
+  // W_k and W_v stacked (for de), then, unless the forward saved them,
+  // [k | v] = e [W_k; W_v]^T (fp32)
   const size_t wbytes = (size_t)d * E * 2;
   if ((rc = ck(cudaMemcpyAsync(w.Wkv, Wk, wbytes, cudaMemcpyDeviceToDevice, s)))) return rc;
   if ((rc = ck(cudaMemcpyAsync(w.Wkv + (size_t)d * E, Wv, wbytes, cudaMemcpyDeviceToDevice, s))))
     return rc;
-  if ((rc = gemm_rm(hd, false, true, n, 2 * d, E, e, E, w.Wkv, E, w.kv, 2 * d, 0.f))) return rc;
+  if (!have_kv && (rc = gemm_rm(hd, false, true, n, 2 * d, E, e, E, w.Wkv, E, w.kv, 2 * d, 0.f)))
+    return rc;
+  const float* kv = have_kv ? kv_saved : w.kv;
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
   if ((rc = ck(cudaFuncSetAttribute(bw_col_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     kColSmem))))
     return rc;
   bw_col_kernel<<<dim3((unsigned)((chunks + COL_WARPS - 1) / COL_WARPS), (unsigned)(d / COL_FEAT)),
-                  32 * COL_WARPS, kColSmem, s>>>(w.kv + d, alpha, reinterpret_cast<const float4*>(conv_w),
+                  32 * COL_WARPS, kColSmem, s>>>(kv + d, alpha, reinterpret_cast<const float4*>(conv_w),
                                           dout, N, T, d, 2 * d, chunks, w.dkv + d,
                                           w.dalpha_part, w.part);
   {
@@ -666,7 +672,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
         (rc = ck(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, row, ROW_THREADS, smem))))
       return rc;
     const int64_t grid = std::min<int64_t>(N, (int64_t)sms * std::max(per_sm, 1));
-    row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, w.kv, alpha, dout, w.dalpha_part, N, d,
+    row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, kv, alpha, dout, w.dalpha_part, N, d,
                                                   2 * d, dh, w.dkv, status_ptr());
   }
   bw_dconv_reduce_kernel<<<(unsigned)((d + 31) / 32), 32 * DCONV_WARPS, 0, s>>>(

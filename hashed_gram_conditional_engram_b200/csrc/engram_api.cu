@@ -23,6 +23,7 @@ int check_cfg(const engram_cfg_t* c) {
   if (c->D_h < 1 || c->d_model < 1 || c->n_branch < 1) return ENGRAM_ERR_INVALID_ARG;
   if (c->V_raw < 1 || c->V_c < 1 || c->V_c > c->V_raw) return ENGRAM_ERR_INVALID_ARG;
   if (c->dtype != ENGRAM_F32 && c->dtype != ENGRAM_BF16) return ENGRAM_ERR_INVALID_ARG;
+  if ((c->flags & ~ENGRAM_SAVE_KV) != 0) return ENGRAM_ERR_INVALID_ARG;
   const int es = c->dtype == ENGRAM_F32 ? 4 : 2;
   if ((c->D_h * es) % 16 != 0) return ENGRAM_ERR_MISALIGNED;
   for (int j = 0; j < 2 * c->K; ++j) {
@@ -34,6 +35,12 @@ int check_cfg(const engram_cfg_t* c) {
 }
 
 inline int elem_bytes(const engram_cfg_t* c) { return c->dtype == ENGRAM_F32 ? 4 : 2; }
+
+// bf16 layers with ENGRAM_SAVE_KV keep k and v after alpha in `saved`
+inline bool saves_kv(const engram_cfg_t* c) {
+  return c->dtype == ENGRAM_BF16 && (c->flags & ENGRAM_SAVE_KV) != 0;
+}
+inline size_t alpha_bytes_padded(int64_t n_tok) { return ((size_t)n_tok * 4 + 255) & ~(size_t)255; }
 
 }  // namespace
 
@@ -105,7 +112,8 @@ size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n) {
       if (cfg->dtype == ENGRAM_F32) return f32_forward_ws_bytes(n, M, d);
       return tc_forward_ws_bytes(n, d, E);
     case ENGRAM_WS_BACKWARD:
-      if (cfg->dtype == ENGRAM_BF16) return backward_bf16_ws_bytes(n, d, E, 2 * cfg->K);
+      if (cfg->dtype == ENGRAM_BF16)
+        return backward_bf16_ws_bytes(n, d, E, 2 * cfg->K, saves_kv(cfg));
       return backward_f32_ws_bytes(n, M, d, E) + table_grad_ws_bytes(n * 2 * cfg->K);
     case ENGRAM_WS_TABLE_GRAD:
       return table_grad_ws_bytes(n * 2 * cfg->K);
@@ -117,6 +125,8 @@ size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n) {
 size_t engram_saved_size(const engram_cfg_t* cfg, int64_t n_tok) {
   if (check_cfg(cfg) != ENGRAM_OK || n_tok < 0) return 0;
   if (cfg->dtype == ENGRAM_F32) return f32_saved_bytes(n_tok, cfg->n_branch, cfg->d_model);
+  if (saves_kv(cfg))  // alpha, then k and v from the 256-byte boundary on
+    return alpha_bytes_padded(n_tok) + (size_t)n_tok * 2 * cfg->d_model * sizeof(float);
   return (size_t)n_tok * cfg->n_branch * sizeof(float);  // alpha
 }
 
@@ -187,11 +197,15 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
     return launch_forward_f32(static_cast<const float*>(e), static_cast<const float*>(h),
                               static_cast<const float*>(Wk), static_cast<const float*>(Wv), conv_w,
                               conv_state, static_cast<float*>(out), saved, N, T, M, d, E, ws, s);
+  float* kv_save = saved != nullptr && conv_state == nullptr && saves_kv(cfg)
+                       ? reinterpret_cast<float*>(reinterpret_cast<char*>(saved) +
+                                                  alpha_bytes_padded(N))
+                       : nullptr;
   return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
                            static_cast<const __nv_bfloat16*>(Wk),
                            static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
-                           static_cast<__nv_bfloat16*>(out), saved, N, T, d, E, ws, ws_bytes,
-                           table != nullptr, s);
+                           static_cast<__nv_bfloat16*>(out), saved, kv_save, N, T, d, E, ws,
+                           ws_bytes, table != nullptr, s);
 }
 
 int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,
@@ -228,10 +242,14 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
       return ck(cudaMemsetAsync(n_unique, 0, sizeof(int32_t), s));
     }
     using bf = __nv_bfloat16;
+    const float* kv_saved =
+        saves_kv(cfg) ? reinterpret_cast<const float*>(reinterpret_cast<const char*>(saved) +
+                                                       alpha_bytes_padded(N))
+                      : nullptr;
     return launch_backward_bf16(hp, idx, static_cast<const bf*>(e), static_cast<const bf*>(h),
                                 static_cast<const bf*>(Wk), static_cast<const bf*>(Wv), conv_w,
-                                saved, dout, dh, dWk, dWv, dconv_w, de, dtab_keys, dtab_rows,
-                                n_unique, N, T, d, ws, ws_bytes, s);
+                                saved, kv_saved, dout, dh, dWk, dWv, dconv_w, de, dtab_keys,
+                                dtab_rows, n_unique, N, T, d, ws, ws_bytes, s);
   }
   const size_t bw = backward_f32_ws_bytes(N, M, d, E);
   // de lives in the dense-backward workspace unless the caller wants it

@@ -68,6 +68,7 @@ struct TcArgs {
   float* conv_state;
   float* alpha_out;     // pass V: optional copy of alpha for the caller
   const float* alpha;   // pass V: gate of every token, from the gate kernel
+  float* kv_save;       // optional fp32 [N, 2d]: k (pass K) then v (pass V) of each token
   unsigned int* status;
 };
 
@@ -443,12 +444,15 @@ struct TcShape {
   static constexpr int HBOX_BYTES = 32 * BM * 2;
   static constexpr int HSLOT_BYTES = PARTS * HBOX_BYTES;
   static constexpr int ALPHA_BYTES = VPASS ? 2 * BN * 4 : 0;  // gates of a tile, two tiles
+  // pass K, when k is kept: each epilogue warp stages its 32 tokens x 32
+  // features (fp32, 128-byte swizzled) for one tiled store
+  static constexpr int KVBUF_BYTES = VPASS ? 0 : EPI * 32 * 32 * 4;
   // as many h slots (up to 4) as the shared memory left by the operand stages holds
   static constexpr int HSLOTS_FIT =
       (232448 - STAGES * (A_BYTES + B_BYTES) - 256 - ALPHA_BYTES) / HSLOT_BYTES;
   static constexpr int HSLOTS = VPASS ? (HSLOTS_FIT < 4 ? HSLOTS_FIT : 4) : 0;
   static constexpr size_t SMEM = (size_t)STAGES * (A_BYTES + B_BYTES) +
-                                 (size_t)HSLOTS * HSLOT_BYTES + 256 + ALPHA_BYTES;
+                                 (size_t)HSLOTS * HSLOT_BYTES + KVBUF_BYTES + 256 + ALPHA_BYTES;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "N tile");
   static_assert(2 * STAGES + 13 <= 30, "barrier area");
   static_assert(SMEM <= 232448, "shared memory");
@@ -483,7 +487,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::A_BYTES;
   uint8_t* hring = sB + STAGES * S::B_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(hring + S::HSLOTS * S::HSLOT_BYTES);
+  uint8_t* kvbuf = hring + S::HSLOTS * S::HSLOT_BYTES;  // pass K only
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kvbuf + S::KVBUF_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -784,6 +789,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.f;
           }
+          if (args.kv_save != nullptr && got) {
+            // k itself, for the backward: the warp's 32 x 32 block goes
+            // through its staging buffer (row = token, 16-byte chunks
+            // swizzled by the row) and out in one tiled store; rows past N
+            // are not written
+            uint8_t* kb = kvbuf + ew * (32 * 32 * 4);
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();  // the previous store has read the buffer
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<float4*>(kb + lane * 128 + ((q ^ (lane & 7)) * 16)) =
+                  make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            fence_async_shared();
+            __syncwarp();
+            if (lane == 0)
+              tma_store_2d(&tmO, kb, col_base + c * 32, (int)(tok0 + (int)rank * BM + quad * 32));
+          }
           if (valid) {
             float hv[32];
             if (c == 0)
@@ -799,6 +821,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
           }
         }
         if (valid) args.part[n * args.n_part + ni * PARTS + part] = make_float4(kk, hk, hh, 0.f);
+        if (args.kv_save != nullptr && tile + num_pairs >= num_tiles && lane == 0)
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // before the CTA exits
       } else {
         // pass V: this lane's feature, one part of the tile's tokens.  The causal
         // conv walks the tokens in order with vt of the three previous tokens
@@ -947,6 +971,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
             if (got) tmem_wait16(un);
             conv_group16<true>(un, al4 + 4, hs + 16 * BM, w, s1, s2, s3, pos, T);
           }
+          if (!DECODE && args.kv_save != nullptr && got) {
+            // v itself, for the backward: token by token, the warp's 32
+            // features side by side (one 128-byte line per token); halo
+            // columns are stored by the tile that owns them
+            float* vp = args.kv_save + nb * 2 * args.d + args.d + feat;
+            const int64_t ld = 2 * (int64_t)args.d;
+            if (jb >= first_out && nb + 32 <= args.N) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                __stcs(vp, __uint_as_float(i < 16 ? u[i] : un[i - 16]));
+                vp += ld;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                if (jb + i >= first_out && nb + i < args.N)
+                  vp[i * ld] = __uint_as_float(i < 16 ? u[i] : un[i - 16]);
+              }
+            }
+          }
           // the part's four warps have written the box: one thread stores it
           fence_async_shared();
           named_bar_sync(2 + part, 128);
@@ -1072,6 +1116,21 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 [rows, cols] matrix, rows `cols` elements apart, in boxes of
+// box_cols x box_rows.
+bool make_tmap_f32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                   uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 4};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // K-major bf16 operand [rows, K] as a 3-D tensor {64-element chunk, row,
 // chunk index} (strides: a row, 128 bytes), boxes of box_rows rows x kch
 // chunks, 128-byte swizzle: a box lands as kch consecutive swizzled tiles.
@@ -1126,8 +1185,8 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
 template <int BN, int STAGES_K, int STAGES_V, int KCH>
 int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
-              float* alpha_saved, int64_t N, int T, int d, int E, float4* part, float* alpha,
-              bool chained, cudaStream_t s) {
+              float* alpha_saved, float* kv_save, int64_t N, int T, int d, int E, float4* part,
+              float* alpha, bool chained, cudaStream_t s) {
   // Each CTA of a pair loads 128 rows of A and BN/2 rows of B per stage.
   // pass K: A = e (256 tokens per pair tile), B = W_k (BN features)
   CUtensorMap ta_k, tb_k, ta_v, tb_v, th, to, to29;
@@ -1157,6 +1216,7 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.conv_state = conv_state;
   a.alpha_out = alpha_saved;
   a.alpha = nullptr;
+  a.kv_save = conv_state == nullptr ? kv_save : nullptr;
   a.status = status_ptr();
   // pass K: gate partials, pair tiles of 256 tokens x BN features
   a.num_n_tiles = d / BN;
@@ -1165,7 +1225,15 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.num_m_tiles = (int)((N + 2 * BM - 1) / (2 * BM));
   // pass K starts early only behind this call's own gather; as the call's
   // first kernel it keeps plain stream order with the caller's work
-  int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL, KCH>(ta_k, tb_k, th, to, to29, a, s, chained);
+  // pass K writes no output; when k is kept, the output-map slot carries the
+  // map of the saved k (fp32 [N, 2d], boxes of 32 x 32, 128-byte swizzled)
+  CUtensorMap tkv = to;
+  if (a.kv_save != nullptr &&
+      !make_tmap_f32(&tkv, a.kv_save, (uint64_t)(2 * d), (uint64_t)N, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+    return ENGRAM_ERR_CUDA;
+  int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL, KCH>(ta_k, tb_k, th, tkv, to29, a, s,
+                                                             chained);
   if (rc) return rc;
   {
     int dev = 0, sms = 148;
@@ -1215,8 +1283,8 @@ size_t tc_forward_ws_bytes(int64_t N, int d, int E) {
 
 int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
-                      __nv_bfloat16* out, float* alpha_saved, int64_t N, int T, int d, int E,
-                      void* ws, size_t ws_bytes, bool chained, cudaStream_t s) {
+                      __nv_bfloat16* out, float* alpha_saved, float* kv_save, int64_t N, int T,
+                      int d, int E, void* ws, size_t ws_bytes, bool chained, cudaStream_t s) {
   if (ws_bytes < tc_forward_ws_bytes(N, d, E) || ws == nullptr) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL - 256) return ENGRAM_ERR_UNSUPPORTED;
   const bool wide = use_wide(N, d);
@@ -1225,15 +1293,15 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
   float* alpha = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                           (size_t)N * 2 * (d / BN) * sizeof(float4));
   if (wide)
-    return run_layer<256, 6, 5, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E,
-                                   part, alpha, chained, s);
+    return run_layer<256, 6, 5, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, N,
+                                   T, d, E, part, alpha, chained, s);
   // few tokens: each CTA streams long operand rows at a rate set by how many
   // bytes one copy instruction brings, so two K chunks go in each box
   if (E % (2 * BK) == 0)
-    return run_layer<64, 4, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E,
-                                  part, alpha, chained, s);
-  return run_layer<64, 8, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, N, T, d, E,
-                                part, alpha, chained, s);
+    return run_layer<64, 4, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, N,
+                                  T, d, E, part, alpha, chained, s);
+  return run_layer<64, 8, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, N, T,
+                                d, E, part, alpha, chained, s);
 }
 
 }  // namespace engram

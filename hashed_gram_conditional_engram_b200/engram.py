@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libengram_b200.so")
 MAX_HEADS = 32
 F32, BF16 = 0, 1
 WS_VOCAB, WS_FORWARD, WS_BACKWARD, WS_TABLE_GRAD = 0, 1, 2, 3
+SAVE_KV = 1  # EngramCfg.flags
 STATUS_BAD_ID, STATUS_BAD_INDEX, STATUS_TIMEOUT = 1, 2, 4
 
 ERRORS = {
@@ -53,7 +54,7 @@ class EngramCfg(ctypes.Structure):
     _fields_ = [
         ("K", ctypes.c_int32), ("D_h", ctypes.c_int32), ("d_model", ctypes.c_int32),
         ("n_branch", ctypes.c_int32), ("V_raw", ctypes.c_int32), ("V_c", ctypes.c_int32),
-        ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32),
         ("rows", ctypes.c_int64 * MAX_HEADS),
         ("mult", (ctypes.c_uint64 * 3) * MAX_HEADS),
     ]
@@ -68,10 +69,10 @@ class EngramCfg(ctypes.Structure):
 
 
 def make_cfg(K: int, D_h: int, d_model: int, n_branch: int, V_raw: int, V_c: int, dtype: int,
-             rows: Sequence[int], mult) -> EngramCfg:
+             rows: Sequence[int], mult, flags: int = 0) -> EngramCfg:
     c = EngramCfg()
     c.K, c.D_h, c.d_model, c.n_branch = K, D_h, d_model, n_branch
-    c.V_raw, c.V_c, c.dtype, c.reserved = V_raw, V_c, dtype, 0
+    c.V_raw, c.V_c, c.dtype, c.flags = V_raw, V_c, dtype, flags
     mult = np.asarray(mult, dtype=np.uint64)
     for j in range(2 * K):
         c.rows[j] = int(rows[j])

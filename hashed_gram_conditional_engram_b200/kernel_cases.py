@@ -47,6 +47,8 @@ def main(argv=None):
     ap.add_argument("--dh", type=int, default=80)
     ap.add_argument("--rows", type=int, default=4_450_001)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--save-kv", action="store_true",
+                    help="fused, backward: the forward keeps k and v for the backward")
     a = ap.parse_args(argv)
     from . import build
     build.build()
@@ -60,7 +62,8 @@ def main(argv=None):
     N = B * T
     rows = synth.primes_at_most(a.rows, a.heads)
     mult = synth.hash_multipliers(12345, a.heads)
-    cfg = eg.make_cfg(K, a.dh, a.d, 1, 129280, synth.compressed_vocab(129280), eg.BF16, rows, mult)
+    cfg = eg.make_cfg(K, a.dh, a.d, 1, 129280, synth.compressed_vocab(129280), eg.BF16, rows, mult,
+                      flags=eg.SAVE_KV if a.save_kv else 0)
     g = torch.Generator(device=dev)
     g.manual_seed(7)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -74,7 +77,7 @@ def main(argv=None):
         out = torch.empty_like(h)
         nb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
         ws = torch.empty(nb, dtype=torch.uint8, device=dev)
-        saved = torch.empty(N, dtype=torch.float32, device=dev)
+        saved = torch.empty(eg.engram_saved_size(cfg, N), dtype=torch.uint8, device=dev)
 
         def run():
             eg.engram_forward(cfg, None, None, e, h, Wk, Wv, cw, None, out, saved, B, T, ws, nb)
@@ -84,7 +87,12 @@ def main(argv=None):
         Wk = (torch.randn((a.d, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
         Wv = (torch.randn((a.d, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
         cw = torch.randn((a.d, 4), generator=g, device=dev) * 0.5
-        saved = torch.rand((N,), generator=g, device=dev)
+        saved = torch.empty(eg.engram_saved_size(cfg, N), dtype=torch.uint8, device=dev)
+        saved[: N * 4].view(torch.float32).copy_(torch.rand((N,), generator=g, device=dev))
+        if a.save_kv:  # k and v as a forward would have kept them
+            off = (N * 4 + 255) // 256 * 256
+            kv = saved[off: off + N * 2 * a.d * 4].view(torch.float32)
+            kv.copy_((e.float() @ torch.cat([Wk, Wv]).float().T).reshape(-1))
         dout = torch.randn((N, a.d), generator=g, device=dev)
         rng = np.random.default_rng(3)
         idx = torch.from_numpy(np.stack([rng.integers(0, P, N) for P in rows], -1)

@@ -54,6 +54,9 @@ extern "C" {
 
 enum { ENGRAM_F32 = 0, ENGRAM_BF16 = 1 };
 
+/* engram_cfg_t.flags */
+#define ENGRAM_SAVE_KV 1
+
 enum {
   ENGRAM_OK = 0,
   ENGRAM_ERR_INVALID_ARG = -1, /* null pointer, bad size or bad config */
@@ -80,6 +83,13 @@ enum {
  *            table, W_v and conv weights are shared ([p5 二.2] 多分支架构集成).
  *   V_raw    raw vocabulary size; V_c compressed size; PAD id = V_c.
  *   dtype    ENGRAM_F32 or ENGRAM_BF16: storage of table, e, h, W_k, W_v, out.
+ *   flags    0, or ENGRAM_SAVE_KV (bf16 layers; fp32 layers ignore it): a
+ *            forward with whole sequences and a `saved` buffer also stores
+ *            k = W_k e and v = W_v e there (fp32 [n_tok, 2 d_model], each
+ *            token's k then its v, after alpha from the next 256-byte
+ *            boundary), and the backward reads them instead of recomputing
+ *            them: 8 * n_tok * d_model more bytes of `saved` for one GEMM
+ *            less in the backward.  Any other bit is ENGRAM_ERR_INVALID_ARG.
  *   rows[j]  P_j, row count (a prime) of head j's table.  Head j's rows sit
  *            in one packed table after those of heads 0..j-1.
  *   mult[j]  odd 64-bit multipliers of head j for n-gram positions 0, 1, 2
@@ -94,7 +104,7 @@ typedef struct engram_cfg {
   int32_t V_raw;
   int32_t V_c;
   int32_t dtype;
-  int32_t reserved;
+  int32_t flags; /* 0, or ENGRAM_SAVE_KV */
   int64_t rows[ENGRAM_MAX_HEADS];
   uint64_t mult[ENGRAM_MAX_HEADS][3];
 } engram_cfg_t;
@@ -111,7 +121,8 @@ enum {
  * 0 as well for an invalid configuration (the call itself then reports it). */
 size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n);
 
-/* Bytes of the `saved` buffer engram_forward fills for engram_backward. */
+/* Bytes of the `saved` buffer engram_forward fills for engram_backward
+ * (bf16: alpha, fp32 [n_tok], and with ENGRAM_SAVE_KV k and v as well). */
 size_t engram_saved_size(const engram_cfg_t* cfg, int64_t n_tok);
 
 /*

@@ -44,6 +44,15 @@ def test_workspace_sizes_host_only():
     # bf16: gate partials (2 per 256-column tile per token) and the gate itself
     assert eg.engram_workspace_size(b, eg.WS_FORWARD, 32768) == 32768 * 20 * 16 + 32768 * 4
     assert eg.engram_saved_size(b, 32768) == 32768 * 4
+    # keeping k and v: alpha up to the next 256 bytes, then fp32 [N, 2d]; the
+    # backward then needs no room of its own for them
+    bk = _cfg(K=8, D_h=80, d_model=2560, dtype=eg.BF16, rows=[4449997] * 16,
+              mult=np.ones((16, 3), np.uint64), flags=eg.SAVE_KV)
+    assert eg.engram_saved_size(bk, 1000) == 4096 + 1000 * 2 * 2560 * 4
+    assert (eg.engram_workspace_size(b, eg.WS_BACKWARD, 32768)
+            - eg.engram_workspace_size(bk, eg.WS_BACKWARD, 32768)) >= 32768 * 2 * 2560 * 4
+    # fp32 layers keep their own intermediates and ignore the flag
+    assert eg.engram_saved_size(_cfg(flags=eg.SAVE_KV), 64) == eg.engram_saved_size(c, 64)
 
 
 def test_invalid_configurations_rejected_before_any_launch():
@@ -52,7 +61,7 @@ def test_invalid_configurations_rejected_before_any_launch():
         _cfg(D_h=6),                     # 24-byte rows: not a multiple of 16 bytes
         _cfg(rows=[1009, 1009, 1008, 1009]),  # even row count
         _cfg(rows=[1009, 1009, 1, 1009]),
-        _cfg(V_c=1001), _cfg(dtype=7), _cfg(K=3, rows=[1009] * 6,
+        _cfg(V_c=1001), _cfg(dtype=7), _cfg(flags=2), _cfg(K=3, rows=[1009] * 6,
                                             mult=np.ones((6, 3), np.uint64)),  # J % 4 != 0
     ]
     big = _cfg()

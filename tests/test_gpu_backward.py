@@ -178,9 +178,10 @@ def test_backward_is_deterministic():
 TOL_BF16 = 2e-2
 
 
-def _bf16_backward_case(B, T, d, K, D_h, seed):
+def _bf16_backward_case(B, T, d, K, D_h, seed, flags=0, with_layer=False):
     """A unit-scale bf16 layer (tables N(0,1), W N(0,1/E)): GPU forward then
-    backward, and the oracle's fp64 backward on the same bf16 values."""
+    backward, and the oracle's fp64 backward on the same bf16 values.  flags
+    = eg.SAVE_KV has the forward keep k and v for the backward."""
     from tests.engram_cases import bf16_bits, bf16_dev
     rng = np.random.default_rng(seed)
     J, E, N = 2 * K, 2 * K * D_h, B * T
@@ -192,7 +193,8 @@ def _bf16_backward_case(B, T, d, K, D_h, seed):
     conv_w = (rng.standard_normal((d, 4)) * 0.5).astype(np.float32)
     dout = rng.standard_normal((N, 1, d)).astype(np.float32)
     idx = np.stack([rng.integers(0, P, N) for P in rows], -1).astype(np.int32)
-    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((J, 3), np.uint64))
+    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((J, 3), np.uint64),
+                      flags=flags)
     L = Layer(cfg, B, T, packed_table(tables, "bf16"), bf16_dev(h), bf16_dev(Wk), bf16_dev(Wv),
               dev(conv_w), torch.bfloat16)
     idx_d = dev(idx.reshape(B, T, J))
@@ -209,6 +211,8 @@ def _bf16_backward_case(B, T, d, K, D_h, seed):
     ref["e"] = e_ref
     ref["Wk_bf"] = f64(synth.to_bf16_bits(Wk))
     ref["Wv_bf"] = f64(synth.to_bf16_bits(Wv))
+    if with_layer:
+        return g, ref, idx, rows, D_h, L
     return g, ref, idx, rows, D_h
 
 
@@ -235,7 +239,23 @@ def _within_gemm_bound(got, want, bound):
     (1, 129, 256, 2, 16),     # one sequence one token past a 128-token column chunk
 ])
 def test_backward_bf16_matches_oracle(B, T, d, K, D_h):
-    g, ref, idx, rows, D_h = _bf16_backward_case(B, T, d, K, D_h, seed=B * 31 + T)
+    _check_bf16_backward(*_bf16_backward_case(B, T, d, K, D_h, seed=B * 31 + T))
+
+
+@pytest.mark.parametrize("B,T,d,K,D_h", [
+    (3, 100, 256, 2, 32),     # narrow forward tiles
+    (2, 2500, 512, 2, 32),    # wide forward tiles, tiles overlapping by the conv halo
+    (50, 3, 256, 2, 32),      # sequences shorter than the conv
+])
+def test_backward_bf16_saved_kv_matches_oracle(B, T, d, K, D_h):
+    """With ENGRAM_SAVE_KV the forward's k and v (fp32 accumulations of the
+    bf16 products) replace the backward's recomputation: the same bounds
+    hold."""
+    _check_bf16_backward(*_bf16_backward_case(B, T, d, K, D_h, seed=B * 17 + T,
+                                              flags=eg.SAVE_KV))
+
+
+def _check_bf16_backward(g, ref, idx, rows, D_h):
     for name in ("dh", "dconv_w"):
         err = max_rel_err(g[name].cpu().numpy(), ref[name])
         assert err <= TOL_BF16, (name, err)
@@ -317,3 +337,48 @@ def test_backward_bf16_layer27b_full_size():
     assert np.array_equal(g["rows"][:U].cpu().numpy().view(np.uint32), rows_own.view(np.uint32))
     del table, dense, L, g
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,T,d,E_heads", [(3, 100, 256, 2), (2, 2500, 512, 2)])
+def test_forward_saved_kv(B, T, d, E_heads):
+    """ENGRAM_SAVE_KV leaves out, alpha and e bit for bit as they are without
+    it, and the saved k = W_k e and v = W_v e are the fp32 accumulations of
+    the bf16 products (exact in fp32): within the worst-case error of an
+    E-term fp32 sum, E 2^-24 times the sum of the absolute products, of the
+    oracle's fp64 contractions."""
+    from tests.engram_cases import bf16_bits, bf16_dev
+    rng = np.random.default_rng(B * 7 + T)
+    K, D_h = E_heads, 32
+    J, E, N = 2 * K, 2 * K * D_h, B * T
+    rows = synth.primes_at_most(2003, J)
+    tables = [rng.standard_normal((P, D_h)).astype(np.float32) for P in rows]
+    Wk = (rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32)
+    Wv = (rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32)
+    h = rng.standard_normal((B, T, 1, d)).astype(np.float32)
+    conv_w = (rng.standard_normal((d, 4)) * 0.5).astype(np.float32)
+    idx = dev(np.stack([rng.integers(0, P, N) for P in rows], -1).astype(np.int32).reshape(B, T, J))
+    outs = []
+    for flags in (0, eg.SAVE_KV):
+        cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((J, 3), np.uint64),
+                          flags=flags)
+        L = Layer(cfg, B, T, packed_table(tables, "bf16"), bf16_dev(h), bf16_dev(Wk),
+                  bf16_dev(Wv), dev(conv_w), torch.bfloat16)
+        L.forward(idx)
+        torch.cuda.synchronize()
+        assert eg.engram_get_status() == 0
+        outs.append(L)
+    plain, kept = outs
+    assert eg.engram_saved_size(kept.cfg, N) == ((N * 4 + 255) // 256) * 256 + N * 2 * d * 4
+    assert torch.equal(plain.out, kept.out)
+    assert torch.equal(plain.e, kept.e)
+    assert torch.equal(plain.saved[: N * 4], kept.saved[: N * 4])
+    off = ((N * 4 + 255) // 256) * 256
+    kv = kept.saved[off: off + N * 2 * d * 4].view(torch.float32).reshape(N, 2 * d).cpu().numpy()
+    f64 = O.bf16_bits_to_f64
+    e64 = f64(bf16_bits(kept.e))
+    wk64 = f64(synth.to_bf16_bits(Wk))[0]
+    wv64 = f64(synth.to_bf16_bits(Wv))
+    for got, W in ((kv[:, :d], wk64), (kv[:, d:], wv64)):
+        want = e64 @ W.T
+        bound = np.abs(e64) @ np.abs(W).T
+        assert float(np.max(np.abs(got - want) - E * 2.0 ** -24 * bound)) <= 0.0
