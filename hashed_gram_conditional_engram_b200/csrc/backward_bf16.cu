@@ -528,10 +528,11 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
   }
 }
 
-constexpr int DCONV_WARPS = 8;
+constexpr int DCONV_WARPS = 32;
 
 // dconv_w[f] = sum over chunks of part[chunk][f]: warp w adds chunks w,
-// w + 8, ... in order, then the 8 warp sums are added in warp order.
+// w + 32, ... in order (its loads all in flight at once for up to 256
+// chunks), then the 32 warp sums are added in warp order.
 __global__ void __launch_bounds__(32 * DCONV_WARPS) bw_dconv_reduce_kernel(
     const float4* __restrict__ part, int chunks, int d, float4* __restrict__ dw) {
   __shared__ float4 red[DCONV_WARPS][32];
@@ -539,7 +540,7 @@ __global__ void __launch_bounds__(32 * DCONV_WARPS) bw_dconv_reduce_kernel(
   const int f = blockIdx.x * 32 + lane;
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
   if (f < d) {
-#pragma unroll 4
+#pragma unroll 8
     for (int c = warp; c < chunks; c += DCONV_WARPS) {
       const float4 p = part[(int64_t)c * d + f];
       s.x += p.x;
