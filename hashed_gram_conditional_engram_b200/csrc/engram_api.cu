@@ -117,6 +117,10 @@ size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n) {
       return backward_f32_ws_bytes(n, M, d, E) + table_grad_ws_bytes(n * 2 * cfg->K);
     case ENGRAM_WS_TABLE_GRAD:
       return table_grad_ws_bytes(n * 2 * cfg->K);
+    case ENGRAM_WS_HOSTCACHE_RANK:
+      return hot_rows_ws_bytes(n * 2 * cfg->K);
+    case ENGRAM_WS_HOSTCACHE_GATHER:
+      return cached_gather_ws_bytes(n, 2 * cfg->K);
     default:
       return 0;
   }
@@ -317,6 +321,85 @@ int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const 
     rc = launch_gather_host(make_head_params(cfg), idx, dev_ptr, n_tok, elem_bytes(cfg), e, s);
     if (rc) return rc;
   }
+  if (done_event != nullptr) return ck(cudaEventRecord((cudaEvent_t)done_event, s));
+  return ENGRAM_OK;
+}
+
+int64_t engram_table_rows(const engram_cfg_t* cfg) {
+  if (check_cfg(cfg) != ENGRAM_OK) return 0;
+  int64_t t = 0;
+  for (int j = 0; j < 2 * cfg->K; ++j) t += cfg->rows[j];
+  return t;
+}
+
+int engram_hostcache_rank(const engram_cfg_t* cfg, const int32_t* idx, int64_t n_tok, int64_t C,
+                          int64_t* rows_out, int32_t* n_out, void* ws, size_t ws_bytes,
+                          void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (n_tok < 0 || C < 0 || n_out == nullptr || (C > 0 && rows_out == nullptr) ||
+      (n_tok > 0 && (idx == nullptr || ws == nullptr)))
+    return ENGRAM_ERR_INVALID_ARG;
+  if (n_tok * 2 * cfg->K >= 0x7fffffffLL || C >= 0x7fffffffLL) return ENGRAM_ERR_UNSUPPORTED;
+  if (!aligned16(idx) || !aligned16(rows_out) || !aligned16(ws)) return ENGRAM_ERR_MISALIGNED;
+  if (ws_bytes < engram_workspace_size(cfg, ENGRAM_WS_HOSTCACHE_RANK, n_tok))
+    return ENGRAM_ERR_WORKSPACE;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  return launch_hot_rows(make_head_params(cfg), idx, n_tok, C, rows_out, n_out, ws, ws_bytes,
+                         (cudaStream_t)stream);
+}
+
+namespace {
+// the device-side address of a pinned host range (equal to the host address
+// under unified addressing; fails if the memory is not mapped)
+int mapped_host(const void* host, void** dev) {
+  if (cudaHostGetDevicePointer(dev, const_cast<void*>(host), 0) != cudaSuccess) {
+    cudaGetLastError();
+    return ENGRAM_ERR_INVALID_ARG;
+  }
+  return ENGRAM_OK;
+}
+}  // namespace
+
+int engram_hostcache_fill(const engram_cfg_t* cfg, const void* host_table, const int64_t* rows,
+                          int64_t C, void* cache, int32_t* map, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (C < 0 || host_table == nullptr || map == nullptr ||
+      (C > 0 && (rows == nullptr || cache == nullptr)))
+    return ENGRAM_ERR_INVALID_ARG;
+  if (C >= 0x7fffffffLL) return ENGRAM_ERR_UNSUPPORTED;
+  if (!aligned16(host_table) || !aligned16(rows) || !aligned16(cache) || !aligned16(map))
+    return ENGRAM_ERR_MISALIGNED;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  void* dev_ptr = nullptr;
+  if ((rc = mapped_host(host_table, &dev_ptr))) return rc;
+  return launch_cache_fill(make_head_params(cfg), dev_ptr, rows, C, elem_bytes(cfg), cache, map,
+                           (cudaStream_t)stream);
+}
+
+int engram_forward_hostcache(const engram_cfg_t* cfg, const int32_t* idx, const void* host_table,
+                             const void* cache, const int32_t* map, int64_t n_tok, void* e,
+                             int32_t* n_miss, void* ws, size_t ws_bytes, void* side_stream,
+                             void* done_event) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (n_tok < 0 || host_table == nullptr || map == nullptr || ws == nullptr ||
+      (n_tok > 0 && (idx == nullptr || e == nullptr)))
+    return ENGRAM_ERR_INVALID_ARG;
+  if (n_tok * 2 * cfg->K >= 0x7fffffffLL) return ENGRAM_ERR_UNSUPPORTED;
+  if (!aligned16(idx) || !aligned16(host_table) || !aligned16(cache) || !aligned16(map) ||
+      !aligned16(e) || !aligned16(ws))
+    return ENGRAM_ERR_MISALIGNED;
+  if (ws_bytes < engram_workspace_size(cfg, ENGRAM_WS_HOSTCACHE_GATHER, n_tok))
+    return ENGRAM_ERR_WORKSPACE;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  void* dev_ptr = nullptr;
+  if ((rc = mapped_host(host_table, &dev_ptr))) return rc;
+  cudaStream_t s = (cudaStream_t)side_stream;
+  rc = launch_gather_cached(make_head_params(cfg), idx, dev_ptr, cache, map, n_tok,
+                            elem_bytes(cfg), e, n_miss, ws, s);
+  if (rc) return rc;
   if (done_event != nullptr) return ck(cudaEventRecord((cudaEvent_t)done_event, s));
   return ENGRAM_OK;
 }

@@ -99,6 +99,18 @@ int launch_table_grad(const HeadParams& hp, const int32_t* idx, const float* de,
                       int64_t* keys, float* rows, int32_t* n_unique, void* ws, size_t ws_bytes,
                       cudaStream_t s);
 size_t vocab_ws_bytes(int64_t V);
+// HBM cache of host-table rows: fill the cache and its row -> slot map; gather
+// e from the cache (hits) and host memory (the listed misses)
+int launch_cache_fill(const HeadParams& hp, const void* host, const int64_t* rows, int64_t C,
+                      int elem_bytes, void* cache, int32_t* map, cudaStream_t s);
+size_t cached_gather_ws_bytes(int64_t n_tok, int J);
+int launch_gather_cached(const HeadParams& hp, const int32_t* idx, const void* host,
+                         const void* cache, const int32_t* map, int64_t n_tok, int elem_bytes,
+                         void* e, int32_t* n_miss_out, void* ws, cudaStream_t s);
+// the C rows a sample of indices addresses most often (ties: lower row id)
+size_t hot_rows_ws_bytes(int64_t n_items);
+int launch_hot_rows(const HeadParams& hp, const int32_t* idx, int64_t n_tok, int64_t C,
+                    int64_t* rows_out, int32_t* n_out, void* ws, size_t ws_bytes, cudaStream_t s);
 int launch_table_grad_noalloc(const HeadParams& hp, const int32_t* idx, const float* de,
                               int64_t n_tok, int64_t* keys, float* rows, int32_t* n_unique,
                               cudaStream_t s);

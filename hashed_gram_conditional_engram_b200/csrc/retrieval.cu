@@ -299,4 +299,181 @@ int launch_gather_host(const HeadParams& hp, const int32_t* idx, const void* tab
   return ck(cudaGetLastError());
 }
 
+// ------------------------------------------------------- HBM cache of host rows
+//
+// The pages' multi-level cache: the rows of frequent n-grams (Zipfian
+// frequencies) stay in HBM, the long tail in host memory.  A dense map gives
+// each packed-table row its cache slot (-1: not cached), so a lookup is one
+// 4-byte read.
+
+namespace {
+
+// Cache slot i <- host row rows[i] (rows[i] < 0 leaves the slot empty), and
+// map[rows[i]] = i.  A warp per slot, lanes over the row's 16-byte pieces.
+__global__ void cache_fill_kernel(const uint4* __restrict__ host, const int64_t* __restrict__ rows,
+                                  int64_t C, int CR, int64_t total_rows, uint4* __restrict__ cache,
+                                  int32_t* __restrict__ map, unsigned int* status) {
+  const int64_t slot = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (slot >= C) return;
+  const int64_t r = rows[slot];
+  if (r < 0) return;
+  if (r >= total_rows) {
+    if (lane == 0) atomicOr(status, ENGRAM_STATUS_BAD_INDEX);
+    return;
+  }
+  for (int c = lane; c < CR; c += 32) cache[slot * CR + c] = ld_row_piece(host + r * CR + c);
+  if (lane == 0) map[r] = (int32_t)slot;
+}
+
+// Pass 1 of a cached gather: one thread per (token, head) looks its row up.
+// item_slot = the cache slot, -1 for a row left in host memory (appended to
+// the miss list, one atomic per warp), -2 for an invalid slot (zeros).
+__global__ void cache_probe_kernel(const __grid_constant__ HeadParams hp,
+                                   const int32_t* __restrict__ idx,
+                                   const int32_t* __restrict__ map, int64_t n_items,
+                                   int32_t* __restrict__ item_slot, int32_t* __restrict__ miss_list,
+                                   int32_t* __restrict__ n_miss, unsigned int* status) {
+  const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  bool miss = false;
+  if (item < n_items) {
+    const int j = (int)(item % hp.J);
+    const int32_t s = __ldg(idx + item);
+    int32_t slot = -2;
+    if (s >= 0 && (uint64_t)s < hp.P[j]) {
+      slot = __ldg(map + hp.row_base[j] + s);
+      miss = slot < 0;
+      if (miss) slot = -1;
+    } else if (s != -1) {
+      atomicOr(status, ENGRAM_STATUS_BAD_INDEX);
+    }
+    item_slot[item] = slot;
+  }
+  const unsigned ballot = __ballot_sync(FULL, miss);
+  if (ballot == 0) return;
+  int32_t base = 0;
+  if (lane == __ffs(ballot) - 1) base = atomicAdd(n_miss, __popc(ballot));
+  base = __shfl_sync(FULL, base, __ffs(ballot) - 1);
+  if (miss) miss_list[base + __popc(ballot & ((1u << lane) - 1u))] = (int32_t)item;
+}
+
+// Pass 2, on the whole GPU: the pieces of cached rows from HBM, zeros for
+// invalid slots; rows left in host memory are pass 3's.
+template <int UNROLL>
+__global__ void __launch_bounds__(256) gather_hits_kernel(
+    int J, const int32_t* __restrict__ item_slot, const uint4* __restrict__ cache, int64_t n_tok,
+    int CR, uint4* __restrict__ e) {
+  const int per_tok = J * CR;
+  const int64_t total = n_tok * per_tok;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < total;
+       base += stride * UNROLL) {
+    uint4 v[UNROLL];
+    bool own[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t g = base + u * stride;
+      v[u] = make_uint4(0, 0, 0, 0);
+      own[u] = false;
+      if (g < total) {
+        const int64_t item = g / CR;
+        const int c = (int)(g - item * CR);
+        const int32_t slot = __ldg(item_slot + item);
+        own[u] = slot != -1;
+        if (slot >= 0) v[u] = ld_row_piece(cache + (int64_t)slot * CR + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u)
+      if (own[u]) e[base + u * stride] = v[u];
+  }
+}
+
+// Pass 3, on a few CTAs (the reads cross PCIe): the listed (token, head)
+// rows from host memory.
+template <int UNROLL>
+__global__ void __launch_bounds__(128) gather_misses_kernel(
+    const __grid_constant__ HeadParams hp, const int32_t* __restrict__ idx,
+    const uint4* __restrict__ host, const int32_t* __restrict__ miss_list,
+    const int32_t* __restrict__ n_miss, int CR, uint4* __restrict__ e) {
+  const int64_t total = (int64_t)(*n_miss) * CR;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < total;
+       base += stride * UNROLL) {
+    uint4 v[UNROLL];
+    int64_t dst[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t g = base + u * stride;
+      dst[u] = -1;
+      if (g < total) {
+        const int64_t m = g / CR;
+        const int c = (int)(g - m * CR);
+        const int32_t item = miss_list[m];  // n * J + j
+        const int j = item % hp.J;
+        const int32_t s = __ldg(idx + item);  // valid: the probe checked it
+        v[u] = ld_row_piece(host + (hp.row_base[j] + s) * CR + c);
+        dst[u] = (int64_t)item * CR + c;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u)
+      if (dst[u] >= 0) e[dst[u]] = v[u];
+  }
+}
+
+}  // namespace
+
+int launch_cache_fill(const HeadParams& hp, const void* host, const int64_t* rows, int64_t C,
+                      int elem_bytes, void* cache, int32_t* map, cudaStream_t s) {
+  const int64_t total_rows = hp.row_base[hp.J - 1] + (int64_t)hp.P[hp.J - 1];
+  int rc = ck(cudaMemsetAsync(map, 0xff, (size_t)total_rows * sizeof(int32_t), s));  // all -1
+  if (rc || C == 0) return rc;
+  const int CR = hp.D_h * elem_bytes / 16;
+  const int64_t threads = 256;
+  const int64_t blocks = (C * 32 + threads - 1) / threads;
+  cache_fill_kernel<<<(unsigned)blocks, (unsigned)threads, 0, s>>>(
+      static_cast<const uint4*>(host), rows, C, CR, total_rows, static_cast<uint4*>(cache), map,
+      status_ptr());
+  return ck(cudaGetLastError());
+}
+
+size_t cached_gather_ws_bytes(int64_t n_tok, int J) {
+  const size_t list = ((size_t)n_tok * J * 4 + 255) & ~(size_t)255;
+  return 2 * list + 256;  // item slots, miss list, miss count
+}
+
+int launch_gather_cached(const HeadParams& hp, const int32_t* idx, const void* host,
+                         const void* cache, const int32_t* map, int64_t n_tok, int elem_bytes,
+                         void* e, int32_t* n_miss_out, void* ws, cudaStream_t s) {
+  const size_t list = ((size_t)n_tok * hp.J * 4 + 255) & ~(size_t)255;
+  int32_t* item_slot = static_cast<int32_t*>(ws);
+  int32_t* miss_list = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + list);
+  int32_t* n_miss = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + 2 * list);
+  int rc = ck(cudaMemsetAsync(n_miss, 0, sizeof(int32_t), s));
+  if (rc) return rc;
+  if (n_tok > 0) {
+    const int CR = hp.D_h * elem_bytes / 16;
+    const int64_t n_items = n_tok * hp.J;
+    cache_probe_kernel<<<(unsigned)((n_items + 255) / 256), 256, 0, s>>>(
+        hp, idx, map, n_items, item_slot, miss_list, n_miss, status_ptr());
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    constexpr int UNROLL = 4;
+    const int64_t total = n_items * CR;
+    int64_t blocks = (total + 256 * UNROLL - 1) / (256 * UNROLL);
+    if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+    gather_hits_kernel<UNROLL><<<(unsigned)blocks, 256, 0, s>>>(
+        hp.J, item_slot, static_cast<const uint4*>(cache), n_tok, CR, static_cast<uint4*>(e));
+    gather_misses_kernel<8><<<ENGRAM_HOST_GATHER_CTAS, 128, 0, s>>>(
+        hp, idx, static_cast<const uint4*>(host), miss_list, n_miss, CR, static_cast<uint4*>(e));
+    if ((rc = ck(cudaGetLastError()))) return rc;
+  }
+  if (n_miss_out != nullptr)
+    return ck(cudaMemcpyAsync(n_miss_out, n_miss, sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+  return ENGRAM_OK;
+}
+
 }  // namespace engram

@@ -688,6 +688,80 @@ int launch_table_grad(const HeadParams& hp, const int32_t* idx, const float* de,
 
 size_t vocab_ws_bytes(int64_t V) { return sort_ws_bytes(V); }
 
+// ------------------------------------------------------- hot rows of a sample
+//
+// The rows a sample of hash indices addresses most often: the candidates for
+// an HBM cache in front of a host-memory table (the pages' multi-level cache
+// keeps the frequent n-grams' rows near the GPU, relying on their Zipfian
+// frequencies).  Rows are ranked by how many (token, head) pairs address
+// them, ties by ascending row id, so the ranking is a pure function of the
+// sample.  The same sort as the table gradient finds each distinct row and
+// its count; a second stable sort by descending count keeps ascending row
+// order among equal counts.
+
+namespace {
+
+// key of distinct row u: a count-descending order; past n_unique: last
+__global__ void hot_count_kernel(const int32_t* __restrict__ seg_start,
+                                 const int32_t* __restrict__ n_unique, int64_t n,
+                                 uint64_t* __restrict__ keys, uint32_t* __restrict__ vals) {
+  const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= n) return;
+  const int32_t U = *n_unique;
+  const uint32_t cnt = u < U ? (uint32_t)(seg_start[u + 1] - seg_start[u]) : 0u;
+  keys[u] = 0xffffffffull - cnt;  // cnt >= 1 for every distinct row
+  vals[u] = (uint32_t)u;
+}
+
+__global__ void hot_out_kernel(const int64_t* __restrict__ ukeys, const uint32_t* __restrict__ order,
+                               const int32_t* __restrict__ n_unique, int64_t C,
+                               int64_t* __restrict__ rows_out, int32_t* __restrict__ n_out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int32_t U = *n_unique;
+  if (i == 0) *n_out = (int32_t)(C < U ? C : U);
+  if (i >= C) return;
+  rows_out[i] = i < U ? ukeys[order[i]] : -1;
+}
+
+}  // namespace
+
+size_t hot_rows_ws_bytes(int64_t n_items) { return sort_ws_bytes(n_items) + up256(n_items * 8); }
+
+int launch_hot_rows(const HeadParams& hp, const int32_t* idx, int64_t n_tok, int64_t C,
+                    int64_t* rows_out, int32_t* n_out, void* ws, size_t ws_bytes, cudaStream_t s) {
+  const int64_t n = n_tok * hp.J;
+  if (ws_bytes < hot_rows_ws_bytes(n)) return ENGRAM_ERR_WORKSPACE;
+  if (n == 0 || C == 0) {
+    int rc = ck(cudaMemsetAsync(n_out, 0, sizeof(int32_t), s));
+    if (rc || C == 0) return rc;
+    return ck(cudaMemsetAsync(rows_out, 0xff, (size_t)C * sizeof(int64_t), s));  // all -1
+  }
+  const uint64_t sentinel = (uint64_t)(hp.row_base[hp.J - 1] + (int64_t)hp.P[hp.J - 1]);
+  SortWs w = carve(ws, n);
+  int64_t* ukeys = reinterpret_cast<int64_t*>(static_cast<char*>(ws) + sort_ws_bytes(n));
+  int32_t* n_unique = w.scal + 3;
+  tg_items_kernel<<<nb(n), 256, 0, s>>>(hp, idx, n, sentinel, w.k0, w.v0);
+  uint64_t* k = w.k0;
+  uint32_t* v = w.v0;
+  uint64_t* k_alt = w.k1;
+  uint32_t* v_alt = w.v1;
+  int rc = radix_sort_pairs(k, v, k_alt, v_alt, n, bits_for(sentinel), w.hist, w.bsum, s);
+  if (rc) return rc;
+  tg_flags_kernel<<<nb(n), 256, 0, s>>>(k, n, sentinel, w.a);
+  if ((rc = launch_scan(w.a, w.b, n, n_unique, w.bsum, s))) return rc;
+  tg_heads_kernel<<<nb(n), 256, 0, s>>>(k, n, sentinel, w.b, w.c, ukeys);
+  // the sorted items are no longer needed: their buffers take the second sort
+  uint64_t* k2 = w.k0;
+  uint32_t* v2 = w.v0;
+  uint64_t* k2_alt = w.k1;
+  uint32_t* v2_alt = w.v1;
+  hot_count_kernel<<<nb(n), 256, 0, s>>>(w.c, n_unique, n, k2, v2);
+  if ((rc = radix_sort_pairs(k2, v2, k2_alt, v2_alt, n, 32, w.hist, w.bsum, s))) return rc;
+  hot_out_kernel<<<nb(C > 0 ? C : 1), 256, 0, s>>>(ukeys, v2, n_unique, C, rows_out, n_out);
+  return ck(cudaGetLastError());
+}
+
+
 // ------------------------------------------------- table gradient without allocation
 //
 // For callers that cannot allocate device memory themselves (a host that

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libengram_b200.so")
 MAX_HEADS = 32
 F32, BF16 = 0, 1
 WS_VOCAB, WS_FORWARD, WS_BACKWARD, WS_TABLE_GRAD = 0, 1, 2, 3
+WS_HOSTCACHE_RANK, WS_HOSTCACHE_GATHER = 4, 5
 SAVE_KV = 1  # EngramCfg.flags
 STATUS_BAD_ID, STATUS_BAD_INDEX, STATUS_TIMEOUT = 1, 2, 4
 
@@ -40,7 +41,8 @@ EXPORTED = (
     "engram_hash_indices", "engram_gather", "engram_forward", "engram_backward",
     "engram_table_grad", "engram_table_grad_noalloc", "engram_forward_hosttable",
     "engram_get_status",
-    "engram_device_sm_count", "engram_clock_probe",
+    "engram_device_sm_count", "engram_clock_probe", "engram_table_rows",
+    "engram_hostcache_rank", "engram_hostcache_fill", "engram_forward_hostcache",
 )
 
 
@@ -110,6 +112,10 @@ def lib() -> ctypes.CDLL:
         "engram_get_status": (ctypes.c_int, [P]),
         "engram_device_sm_count": (ctypes.c_int, []),
         "engram_clock_probe": (ctypes.c_int, [P, i64, P]),
+        "engram_table_rows": (ctypes.c_int64, [cfgp]),
+        "engram_hostcache_rank": (ctypes.c_int, [cfgp, P, i64, i64, P, P, P, sz, P]),
+        "engram_hostcache_fill": (ctypes.c_int, [cfgp, P, P, i64, P, P, P]),
+        "engram_forward_hostcache": (ctypes.c_int, [cfgp, P, P, P, P, i64, P, P, P, sz, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -218,6 +224,40 @@ def engram_forward_hosttable(cfg: EngramCfg, idx, host_table, n_tok: int, e, sid
     _check("engram_forward_hosttable",
            lib().engram_forward_hosttable(ctypes.byref(cfg), _p(idx), _p(host_table), n_tok, _p(e),
                                           _s(side_stream), ev))
+
+
+def _event_handle(done_event, side_stream):
+    if done_event is None or isinstance(done_event, int):
+        return done_event
+    # a torch.cuda.Event creates its CUDA event on first record only
+    if done_event.cuda_event == 0:
+        done_event.record(side_stream)
+    return done_event.cuda_event
+
+
+def engram_table_rows(cfg: EngramCfg) -> int:
+    return int(lib().engram_table_rows(ctypes.byref(cfg)))
+
+
+def engram_hostcache_rank(cfg: EngramCfg, idx, n_tok: int, C: int, rows_out, n_out, ws,
+                          ws_bytes: int, stream=None) -> None:
+    _check("engram_hostcache_rank",
+           lib().engram_hostcache_rank(ctypes.byref(cfg), _p(idx), n_tok, C, _p(rows_out),
+                                       _p(n_out), _p(ws), ws_bytes, _s(stream)))
+
+
+def engram_hostcache_fill(cfg: EngramCfg, host_table, rows, C: int, cache, map_, stream=None):
+    _check("engram_hostcache_fill",
+           lib().engram_hostcache_fill(ctypes.byref(cfg), _p(host_table), _p(rows), C, _p(cache),
+                                       _p(map_), _s(stream)))
+
+
+def engram_forward_hostcache(cfg: EngramCfg, idx, host_table, cache, map_, n_tok: int, e, n_miss,
+                             ws, ws_bytes: int, side_stream=None, done_event=None) -> None:
+    _check("engram_forward_hostcache",
+           lib().engram_forward_hostcache(ctypes.byref(cfg), _p(idx), _p(host_table), _p(cache),
+                                          _p(map_), n_tok, _p(e), _p(n_miss), _p(ws), ws_bytes,
+                                          _s(side_stream), _event_handle(done_event, side_stream)))
 
 
 def engram_get_status(stream=None) -> int:

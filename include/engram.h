@@ -114,7 +114,9 @@ enum {
   ENGRAM_WS_VOCAB = 0,     /* engram_build_vocab_proj, n = V */
   ENGRAM_WS_FORWARD = 1,   /* engram_forward, n = tokens */
   ENGRAM_WS_BACKWARD = 2,  /* engram_backward, n = tokens */
-  ENGRAM_WS_TABLE_GRAD = 3 /* engram_table_grad, n = tokens */
+  ENGRAM_WS_TABLE_GRAD = 3, /* engram_table_grad, n = tokens */
+  ENGRAM_WS_HOSTCACHE_RANK = 4,  /* engram_hostcache_rank, n = tokens of the sample */
+  ENGRAM_WS_HOSTCACHE_GATHER = 5 /* engram_forward_hostcache, n = tokens */
 };
 
 /* Bytes of device workspace the call needs for n items (0 = none).  Returns
@@ -274,6 +276,66 @@ int engram_table_grad_noalloc(const engram_cfg_t* cfg, const int32_t* idx, const
  */
 int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const void* host_table,
                              int64_t n_tok, void* e, void* side_stream, void* done_event);
+
+/*
+ * HBM cache of hot host-table rows ([p1 系统效率优化] / [p2] 多级缓存设计: the
+ * n-grams' Zipfian frequencies let the rows of frequent n-grams stay in GPU
+ * memory and the long tail in host memory).  Three calls:
+ *   engram_hostcache_rank  the C rows a sample of hash indices addresses most
+ *                          often (the cache's contents);
+ *   engram_hostcache_fill  copies them from the host table into the cache and
+ *                          builds the row -> slot map;
+ *   engram_forward_hostcache  gathers e like engram_forward_hosttable, the
+ *                          cached rows from HBM and only the others over PCIe.
+ * The gathered e is identical to engram_forward_hosttable's whatever the
+ * cache holds; the cache changes where rows are read from, never what.
+ */
+
+/* Packed-table rows of the configuration: sum of rows[j] over the J heads
+ * (the entries of the hostcache map); 0 for an invalid configuration. */
+int64_t engram_table_rows(const engram_cfg_t* cfg);
+
+/*
+ *   idx      device int32 [n_tok, J]: a sample of hash indices (e.g. earlier
+ *            batches); invalid slots (-1) count for no row.
+ *   C        rows wanted (>= 0).
+ *   rows_out device int64 [C], out: packed-table row ids (row_base_j + slot),
+ *            most addressed first, ties by ascending row id; -1 past n_out.
+ *   n_out    device int32, out: min(C, distinct rows addressed).
+ *   ws       engram_workspace_size(cfg, ENGRAM_WS_HOSTCACHE_RANK, n_tok) bytes.
+ * n_tok * J must stay below 2^31.  Asynchronous on `stream`.
+ */
+int engram_hostcache_rank(const engram_cfg_t* cfg, const int32_t* idx, int64_t n_tok, int64_t C,
+                          int64_t* rows_out, int32_t* n_out, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/*
+ *   host_table pinned, mapped host memory as in engram_forward_hosttable.
+ *   rows       device int64 [C]: packed-table rows to cache (-1: slot unused);
+ *              a row out of range sets ENGRAM_STATUS_BAD_INDEX.
+ *   cache      device [C, D_h] (cfg->dtype), out: cache slot i = rows[i].
+ *   map        device int32 [engram_table_rows(cfg)], out: the cache slot of
+ *              each packed-table row, -1 for rows not cached.
+ * Asynchronous on `stream` (reads C rows over PCIe).
+ */
+int engram_hostcache_fill(const engram_cfg_t* cfg, const void* host_table, const int64_t* rows,
+                          int64_t C, void* cache, int32_t* map, void* stream);
+
+/*
+ *   idx, host_table, n_tok, e, side_stream, done_event as in
+ *   engram_forward_hosttable; cache and map from engram_hostcache_fill.
+ *   n_miss   device int32, out (may be NULL): (token, head) pairs whose row
+ *            came from host memory.
+ *   ws       engram_workspace_size(cfg, ENGRAM_WS_HOSTCACHE_GATHER, n_tok).
+ * Three kernels on side_stream: a probe (one thread per (token, head):
+ * the row's slot, misses appended to a list), the cached rows' pieces from
+ * HBM on the whole GPU, then the listed rows from host memory on a few CTAs.
+ * n_tok * J must stay below 2^31.
+ */
+int engram_forward_hostcache(const engram_cfg_t* cfg, const int32_t* idx, const void* host_table,
+                             const void* cache, const int32_t* map, int64_t n_tok, void* e,
+                             int32_t* n_miss, void* ws, size_t ws_bytes, void* side_stream,
+                             void* done_event);
 
 /* Synchronises `stream`, then returns the device status word of the current
  * device (bits ENGRAM_STATUS_*) and clears it; a negative value is an

@@ -166,9 +166,41 @@ def gather(idx: np.ndarray, tables) -> np.ndarray:
     """e_t = concatenation over heads j of T_j[idx_j] ([p5 二.1 (1)] 拼接检索结果).
 
     tables: list of J arrays [P_j, D_h].  idx: [..., J].  Returns [..., J*D_h]
-    in the tables' dtype (an exact copy)."""
-    parts = [np.asarray(tables[j])[idx[..., j]] for j in range(len(tables))]
+    in the tables' dtype (an exact copy).  A slot of -1 (a token whose n-gram
+    holds an invalid id) reads no row: its D_h entries are zero."""
+    parts = []
+    for j in range(len(tables)):
+        t = np.asarray(tables[j])
+        ij = idx[..., j]
+        part = t[np.where(ij >= 0, ij, 0)]
+        part[ij < 0] = 0
+        parts.append(part)
     return np.concatenate(parts, axis=-1)
+
+
+def hot_rows(idx: np.ndarray, rows, C: int):
+    """The C packed-table rows that a sample of hash indices addresses most
+    often: the rows a GPU-memory cache in front of a host-memory table keeps
+    ([p1] 系统效率优化 / [p2] 多级缓存设计: by the Zipfian frequencies of
+    n-grams, frequent rows near the GPU, the long tail further away).
+
+    idx [..., J]; rows = P_j.  Head j's slot s is packed row
+    P_0 + .. + P_{j-1} + s; slots outside [0, P_j) address no row.  Rows are
+    ranked by how many (token, head) pairs address them, ties by ascending
+    row id.  Returns (top: int64 [C], the ranked rows then -1, n_out =
+    min(C, distinct rows))."""
+    rows = np.asarray(rows, dtype=np.int64)
+    J = rows.size
+    idx = np.asarray(idx, dtype=np.int64).reshape(-1, J)
+    base = np.concatenate([[0], np.cumsum(rows)[:-1]])
+    valid = (idx >= 0) & (idx < rows[None, :])
+    packed = (base[None, :] + idx)[valid]
+    uniq, counts = np.unique(packed, return_counts=True)
+    order = np.lexsort((uniq, -counts))  # by count descending, then row ascending
+    top = uniq[order][:C]
+    out = np.full(C, -1, dtype=np.int64)
+    out[: top.size] = top
+    return out, int(top.size)
 
 
 # ----------------------------------------------------------------------------
