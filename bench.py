@@ -922,6 +922,8 @@ def bench_hosttable(dev, params=8_000_000_000):
     t_both_gather = ev[4].elapsed_time(ev[5]) / 10
     if eg.engram_get_status(comp) != 0:
         raise RuntimeError("device status word set in host-table gather")
+    cached = _hosttable_cached(dev, w, cfg, proj, host, idx, e, side, comp, gemm, t_gemm,
+                               rows_bytes)
     return {"workload": f"hosttable: 4 x 2,048 tokens, 16 heads x 160 dims, {sum(rows) * w.D_h / 1e9:.1f}B "
                         "bf16 params in pinned host memory (the 100B table does not fit the host)",
             "rows_bytes_per_batch": rows_bytes,
@@ -931,7 +933,94 @@ def bench_hosttable(dev, params=8_000_000_000):
             "frac_of_h2d_peak": rows_bytes / (t_gather / 1e3) / 1e9 / h2d_peak,
             "gemm_ms_alone": t_gemm, "gemm_ms_with_gather": t_both_gemm,
             "gather_ms_with_gemm": t_both_gather,
-            "gemm_slowdown": t_both_gemm / t_gemm - 1.0}
+            "gemm_slowdown": t_both_gemm / t_gemm - 1.0,
+            "hbm_cache": cached}
+
+
+def _hosttable_cached(dev, w, cfg, proj, host, idx, e, side, comp, gemm, t_gemm, rows_bytes,
+                      history_batches=256, C=1 << 24):
+    """The same batch through an HBM cache of the rows that earlier batches
+    of the same distribution (history_batches x 8,192 Zipf(1.1) tokens) hit
+    most: ranked on the device, copied in once, then gathered (probe, hits
+    from HBM, misses over PCIe) on the side stream.  Hit rates for smaller
+    caches (prefixes of the same ranking) beside it."""
+    import torch
+    from hashed_gram_conditional_engram_b200 import engram as eg
+    from hashed_gram_conditional_engram_b200 import synth
+    e_plain = e.clone()  # the uncached gather's result, to compare with
+    n_hist = history_batches * w.N
+    hist_ids = synth.zipf_ids(np.random.default_rng(w.seed + 1000), w.V, 1.1, n_hist,
+                              perm=synth.host_ids_perm(w))
+    hist_idx = torch.empty((history_batches * w.B, w.T, w.J), dtype=torch.int32, device=dev)
+    eg.engram_hash_indices(cfg, proj, torch.from_numpy(hist_ids.astype(np.int32)).to(dev)
+                           .reshape(history_batches * w.B, w.T), history_batches * w.B, w.T, None,
+                           hist_idx)
+    nb = eg.engram_workspace_size(cfg, eg.WS_HOSTCACHE_RANK, n_hist)
+    rows_d = torch.empty(C, dtype=torch.int64, device=dev)
+    n_out = torch.zeros(1, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    eg.engram_hostcache_rank(cfg, hist_idx, n_hist, C, rows_d, n_out,
+                             torch.empty(nb, dtype=torch.uint8, device=dev), nb)
+    torch.cuda.synchronize()
+    t_rank = time.perf_counter() - t0
+    n_cached = int(n_out.item())
+    cache = torch.empty((max(n_cached, 1), w.D_h), dtype=torch.bfloat16, device=dev)
+    cmap = torch.empty(eg.engram_table_rows(cfg), dtype=torch.int32, device=dev)
+    gb = eg.engram_workspace_size(cfg, eg.WS_HOSTCACHE_GATHER, w.N)
+    gws = torch.empty(gb, dtype=torch.uint8, device=dev)
+    n_miss = torch.zeros(1, dtype=torch.int32, device=dev)
+    valid = int((idx >= 0).sum().item())
+    hit_by_size = {}
+    for c in (1 << 16, 1 << 18, 1 << 20, 1 << 22):
+        if c >= n_cached:
+            break
+        eg.engram_hostcache_fill(cfg, host.data_ptr(), rows_d, c, cache, cmap)
+        eg.engram_forward_hostcache(cfg, idx, host.data_ptr(), cache, cmap, w.N, e, n_miss, gws,
+                                    gb, None, None)
+        hit_by_size[str(c)] = 1.0 - int(n_miss.item()) / max(valid, 1)
+    t0 = time.perf_counter()
+    eg.engram_hostcache_fill(cfg, host.data_ptr(), rows_d, n_cached, cache, cmap)
+    torch.cuda.synchronize()
+    t_fill = time.perf_counter() - t0
+    del hist_idx
+
+    def gather():
+        eg.engram_forward_hostcache(cfg, idx, host.data_ptr(), cache, cmap, w.N, e, n_miss, gws,
+                                    gb, side, None)
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for _ in range(3):
+        gather()
+    torch.cuda.synchronize()
+    if not torch.equal(e, e_plain):
+        raise RuntimeError("cached gather differs from the uncached one")
+    ev[0].record(side)
+    for _ in range(10):
+        gather()
+    ev[1].record(side)
+    torch.cuda.synchronize()
+    t_gather = ev[0].elapsed_time(ev[1]) / 10
+    side.wait_stream(comp)
+    torch.cuda.synchronize()
+    ev[2].record(comp)
+    ev[4].record(side)
+    for _ in range(10):
+        gather()
+        gemm()
+    ev[3].record(comp)
+    ev[5].record(side)
+    torch.cuda.synchronize()
+    t_both_gemm = ev[2].elapsed_time(ev[3]) / 10
+    misses = int(n_miss.item())
+    if eg.engram_get_status(comp) != 0:
+        raise RuntimeError("device status word set in the cached host-table gather")
+    return {"cache_rows": n_cached, "cache_bytes": n_cached * w.D_h * 2,
+            "history_tokens": n_hist, "rank_s": t_rank, "fill_s": t_fill,
+            "hit_rate": 1.0 - misses / max(valid, 1), "hit_rate_by_cache_rows": hit_by_size,
+            "pcie_row_bytes_per_batch": misses * w.D_h * 2,
+            "gather_ms": t_gather, "rows_gbs_effective": rows_bytes / (t_gather / 1e3) / 1e9,
+            "gemm_ms_with_gather": t_both_gemm, "gemm_slowdown": t_both_gemm / t_gemm - 1.0}
 
 
 # ---------------------------------------------------------------- reference arm

@@ -458,6 +458,9 @@ int launch_gather_cached(const HeadParams& hp, const int32_t* idx, const void* h
     const int64_t n_items = n_tok * hp.J;
     cache_probe_kernel<<<(unsigned)((n_items + 255) / 256), 256, 0, s>>>(
         hp, idx, map, n_items, item_slot, miss_list, n_miss, status_ptr());
+    // the cached rows come from HBM on the whole GPU, briefly (measured with
+    // a GEMM on the compute stream: 32 CTAs here ran longer and delayed the
+    // GEMM more than a full grid)
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

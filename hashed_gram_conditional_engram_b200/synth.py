@@ -80,15 +80,19 @@ def primes_at_most(x: int, count: int) -> List[int]:
     return out
 
 
-def zipf_ids(rng: np.random.Generator, V: int, s: float, n: int) -> np.ndarray:
+def zipf_ids(rng: np.random.Generator, V: int, s: float, n: int,
+             perm: Optional[np.ndarray] = None) -> np.ndarray:
     """n raw token ids, rank r (1-based) drawn with p(r) ~ r^-s by inverse CDF,
-    then sent through a random permutation of the vocabulary."""
+    then sent through a random permutation of the vocabulary (drawn from rng
+    after the ranks, unless `perm` gives it: more text of the same
+    distribution)."""
     p = np.arange(1, V + 1, dtype=np.float64) ** (-s)
     cdf = np.cumsum(p)
     cdf /= cdf[-1]
     r = np.searchsorted(cdf, rng.random(n), side="right")
     r = np.minimum(r, V - 1)
-    perm = rng.permutation(V)
+    if perm is None:
+        perm = rng.permutation(V)
     return perm[r].astype(np.int32)
 
 
@@ -246,6 +250,14 @@ def device_dense(w: Workload, layer: int = 0, device="cuda"):
     Wv = (torch.randn((w.d, w.E), generator=g, device=device) * 0.02).to(torch.bfloat16)
     conv_w = torch.randn((w.d, 4), generator=g, device=device) * 0.5
     return dict(h=h, Wk=Wk, Wv=Wv, conv_w=conv_w)
+
+
+def host_ids_perm(w: Workload) -> np.ndarray:
+    """The vocabulary permutation behind host_ids_keys(w)'s ids (its draws
+    replayed), so that more ids of the same distribution can be drawn."""
+    base = np.random.default_rng(w.seed)
+    base.random(w.N * w.steps)
+    return base.permutation(w.V)
 
 
 def host_ids_keys(w: Workload):

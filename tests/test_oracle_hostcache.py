@@ -86,3 +86,15 @@ def test_gather_zero_rows_for_invalid_slots():
     e = O.gather(idx, tables)
     assert e.tolist() == [[8, 9, 10, 11, 0, 0, 0, 0],
                           [0, 0, 0, 0, 100, 101, 102, 103]]
+
+
+def test_history_ids_share_the_batch_vocabulary_permutation():
+    """More text of the host-table workload's distribution (the history a
+    cache is ranked on) maps ranks through the batch's own permutation:
+    replaying the batch's draws with it reproduces the batch exactly."""
+    from hashed_gram_conditional_engram_b200 import synth
+    w = synth.workload("hosttable")
+    ids, _ = synth.host_ids_keys(w)
+    perm = synth.host_ids_perm(w)
+    again = synth.zipf_ids(np.random.default_rng(w.seed), w.V, 1.1, w.N * w.steps, perm=perm)
+    assert np.array_equal(again.reshape(ids.shape), ids)
