@@ -353,6 +353,177 @@ def layer_backward(e, h, Wk, Wv, conv_w, T, dout, fwd=None):
     return dict(dh=dh, dWk=dWk, dWv=dWv, dconv_w=dconv_w, de=de, dk=dk, dv=dv)
 
 
+# ----------------------------------------------------------------------------
+# formulation variants: the pages fix neither the conv's dilation, nor a norm
+# before it, nor whether branches share it, nor learnable norm scales
+# ([p2]: short depthwise causal conv; [p5 二.1 (2)] 一维卷积增强 then the
+# residual; [p5 二.2] branches share table and W_v).  Each is a flag; with no
+# flag the layer is the one above.
+# ----------------------------------------------------------------------------
+
+CONV_DILATED = 2      # taps at t, t-3, t-6, t-9 (dilation = the largest n-gram order)
+CONV_PRENORM = 4      # the conv reads RMSNorm(vt) (times g_v with NORM_SCALES)
+CONV_PER_BRANCH = 8   # conv weights per branch: [M, d, 4]
+NORM_SCALES = 16      # learnable RMSNorm scales g_h, g_k (and g_v with CONV_PRENORM)
+
+
+def param_count(flags: int, M: int, d: int) -> int:
+    """Floats of the small-parameter block: conv weights ([M or 1] x d x 4),
+    then with NORM_SCALES g_h [M, d], g_k [M, d] and, with CONV_PRENORM,
+    g_v [M, d]."""
+    n = (M if flags & CONV_PER_BRANCH else 1) * d * CONV_K
+    if flags & NORM_SCALES:
+        n += (3 if flags & CONV_PRENORM else 2) * M * d
+    return n
+
+
+def unpack_params(block, flags: int, M: int, d: int) -> dict:
+    """The block's parts as fp64 arrays: w [M, d, 4] (a shared conv repeated
+    over branches), g_h, g_k, g_v [M, d] (ones where absent)."""
+    b = np.asarray(block, np.float64).reshape(-1)
+    assert b.size == param_count(flags, M, d)
+    Mc = M if flags & CONV_PER_BRANCH else 1
+    w = b[: Mc * d * CONV_K].reshape(Mc, d, CONV_K)
+    if Mc == 1:
+        w = np.repeat(w, M, axis=0)
+    off = Mc * d * CONV_K
+    ones = np.ones((M, d))
+    g_h = g_k = g_v = ones
+    if flags & NORM_SCALES:
+        g_h = b[off: off + M * d].reshape(M, d)
+        g_k = b[off + M * d: off + 2 * M * d].reshape(M, d)
+        if flags & CONV_PRENORM:
+            g_v = b[off + 2 * M * d: off + 3 * M * d].reshape(M, d)
+    return dict(w=w, g_h=g_h, g_k=g_k, g_v=g_v, Mc=Mc)
+
+
+def dilation_of(flags: int) -> int:
+    return 3 if flags & CONV_DILATED else 1
+
+
+def causal_conv_v(c: np.ndarray, w: np.ndarray, T: int, dil: int) -> np.ndarray:
+    """y_t = sum_i w[m, :, i] * c_{t-(3-i)*dil} per branch m, zero across
+    sequence starts.  c: [N, M, d]; w: [M, d, 4]."""
+    N = c.shape[0]
+    pos = np.arange(N) % T
+    y = np.zeros_like(c)
+    for i in range(CONV_K):
+        lag = (CONV_K - 1 - i) * dil
+        src = np.arange(N) - lag
+        ok = pos >= lag
+        y[ok] += w[None, :, :, i] * c[src[ok]]
+    return y
+
+
+def layer_forward_v(e, h, Wk, Wv, block, T, flags):
+    """The layer with the formulation variants of `flags`, fp64.
+
+    z = <RMSNorm(h) g_h, RMSNorm(k) g_k> / sqrt(d), alpha = sigmoid(z),
+    vt = alpha v, c = RMSNorm(vt) g_v with CONV_PRENORM else vt,
+    y_t = sum_i w_i c_{t-(3-i) dil}, out = h + vt + SiLU(y)."""
+    e = np.asarray(e, np.float64)
+    h = np.asarray(h, np.float64)
+    Wk = np.asarray(Wk, np.float64)
+    Wv = np.asarray(Wv, np.float64)
+    N, M, d = h.shape
+    P = unpack_params(block, flags, M, d)
+    k = np.stack([e @ Wk[m].T for m in range(M)], axis=1)
+    v = e @ Wv.T
+    z = np.sum(rmsnorm(h) * P["g_h"][None] * rmsnorm(k) * P["g_k"][None], axis=-1) / math.sqrt(d)
+    alpha = sigmoid(z)
+    vt = alpha[..., None] * v[:, None, :]
+    c = rmsnorm(vt) * P["g_v"][None] if flags & CONV_PRENORM else vt
+    y = causal_conv_v(c, P["w"], T, dilation_of(flags))
+    out = h + vt + silu(y)
+    return dict(out=out, k=k, v=v, z=z, alpha=alpha, vt=vt, c=c, y=y)
+
+
+def decode_step_v(e, h, Wk, Wv, block, conv_state, flags):
+    """One token per sequence with the variants of `flags`.  conv_state
+    [B, M, 3 dil, d] holds the conv inputs c of the 3 dil previous steps,
+    oldest first (zeros at the start).  Returns (out, alpha, new_state)."""
+    e = np.asarray(e, np.float64)
+    h = np.asarray(h, np.float64)
+    Wk = np.asarray(Wk, np.float64)
+    Wv = np.asarray(Wv, np.float64)
+    st = np.asarray(conv_state, np.float64)
+    B, M, d = h.shape
+    dil = dilation_of(flags)
+    P = unpack_params(block, flags, M, d)
+    k = np.stack([e @ Wk[m].T for m in range(M)], axis=1)
+    v = e @ Wv.T
+    z = np.sum(rmsnorm(h) * P["g_h"][None] * rmsnorm(k) * P["g_k"][None], axis=-1) / math.sqrt(d)
+    alpha = sigmoid(z)
+    vt = alpha[..., None] * v[:, None, :]
+    c = rmsnorm(vt) * P["g_v"][None] if flags & CONV_PRENORM else vt
+    w = P["w"]
+    y = w[None, :, :, 3] * c
+    for i in range(3):
+        lag = (3 - i) * dil                  # state index 3 dil - lag
+        y = y + w[None, :, :, i] * st[:, :, 3 * dil - lag, :]
+    out = h + vt + silu(y)
+    new_state = np.concatenate([st[:, :, 1:, :], c[:, :, None, :]], axis=2)
+    return out, alpha, new_state
+
+
+def layer_backward_v(e, h, Wk, Wv, block, T, dout, flags):
+    """All gradients of L = sum(dout * out) for the variant layer, fp64:
+    dh, dWk, dWv, de and dblock (the small-parameter block's gradient, in
+    the block's layout)."""
+    e = np.asarray(e, np.float64)
+    h = np.asarray(h, np.float64)
+    Wk = np.asarray(Wk, np.float64)
+    Wv = np.asarray(Wv, np.float64)
+    u = np.asarray(dout, np.float64)
+    N, M, d = h.shape
+    P = unpack_params(block, flags, M, d)
+    f = layer_forward_v(e, h, Wk, Wv, block, T, flags)
+    k, v, alpha, vt, c, y = f["k"], f["v"], f["alpha"], f["vt"], f["c"], f["y"]
+    w, dil = P["w"], dilation_of(flags)
+    pos = np.arange(N) % T
+    sy = sigmoid(y)
+    dy = u * sy * (1.0 + y * (1.0 - sy))
+    dc = np.zeros_like(c)
+    dw = np.zeros((M, d, CONV_K))
+    for i in range(CONV_K):
+        lag = (CONV_K - 1 - i) * dil
+        tgt = np.arange(N) + lag               # y_{t+lag} reads c_t through tap i
+        ok = (pos + lag) < T
+        dc[ok] += w[None, :, :, i] * dy[tgt[ok]]
+        src = np.arange(N) - lag
+        ok2 = pos >= lag
+        dw[:, :, i] = np.sum(dy[ok2] * c[src[ok2]], axis=0)
+    dg_v = np.zeros((M, d))
+    if flags & CONV_PRENORM:
+        ch = rmsnorm(vt)
+        dg_v = np.sum(dc * ch, axis=0)
+        dvt = u + rmsnorm_backward(vt, dc * P["g_v"][None])
+    else:
+        dvt = u + dc
+    dalpha = np.sum(dvt * v[:, None, :], axis=-1)
+    dv = np.sum(alpha[..., None] * dvt, axis=1)
+    dz = dalpha * alpha * (1.0 - alpha)
+    hh, kh = rmsnorm(h), rmsnorm(k)
+    gh, gk = P["g_h"][None], P["g_k"][None]
+    dhh = dz[..., None] * gh * gk * kh / math.sqrt(d)
+    dkh = dz[..., None] * gh * gk * hh / math.sqrt(d)
+    dg_h = np.sum(dz[..., None] * hh * kh * gk, axis=0) / math.sqrt(d)
+    dg_k = np.sum(dz[..., None] * hh * kh * gh, axis=0) / math.sqrt(d)
+    dh = u + rmsnorm_backward(h, dhh)
+    dk = rmsnorm_backward(k, dkh)
+    dWk = np.stack([dk[:, m, :].T @ e for m in range(M)], axis=0)
+    dWv = dv.T @ e
+    de = dv @ Wv
+    for m in range(M):
+        de = de + dk[:, m, :] @ Wk[m]
+    parts = [(dw if P["Mc"] == M else dw.sum(axis=0, keepdims=True)).reshape(-1)]
+    if flags & NORM_SCALES:
+        parts += [dg_h.reshape(-1), dg_k.reshape(-1)]
+        if flags & CONV_PRENORM:
+            parts.append(dg_v.reshape(-1))
+    return dict(dh=dh, dWk=dWk, dWv=dWv, de=de, dblock=np.concatenate(parts), dk=dk, dv=dv)
+
+
 def table_grad_f64(idx, de, rows, D_h):
     """Dense fp64 table gradient: dT_j[s] = sum of de_t[j-th segment] over the
     tokens t with idx[t, j] = s.  Returns a list of J arrays [P_j, D_h]."""
