@@ -23,7 +23,7 @@ int check_cfg(const engram_cfg_t* c) {
   if (c->D_h < 1 || c->d_model < 1 || c->n_branch < 1) return ENGRAM_ERR_INVALID_ARG;
   if (c->V_raw < 1 || c->V_c < 1 || c->V_c > c->V_raw) return ENGRAM_ERR_INVALID_ARG;
   if (c->dtype != ENGRAM_F32 && c->dtype != ENGRAM_BF16) return ENGRAM_ERR_INVALID_ARG;
-  if ((c->flags & ~ENGRAM_SAVE_KV) != 0) return ENGRAM_ERR_INVALID_ARG;
+  if ((c->flags & ~(ENGRAM_SAVE_KV | ENGRAM_VARIANT_FLAGS)) != 0) return ENGRAM_ERR_INVALID_ARG;
   const int es = c->dtype == ENGRAM_F32 ? 4 : 2;
   if ((c->D_h * es) % 16 != 0) return ENGRAM_ERR_MISALIGNED;
   for (int j = 0; j < 2 * c->K; ++j) {
@@ -192,7 +192,9 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
   cudaStream_t s = (cudaStream_t)stream;
   const HeadParams hp = make_head_params(cfg);
   const int M = cfg->n_branch, d = cfg->d_model, E = hp.E;
-  if (cfg->dtype == ENGRAM_BF16 && !tc_supported(d, E, M)) return ENGRAM_ERR_UNSUPPORTED;
+  if (cfg->dtype == ENGRAM_BF16 &&
+      (!tc_supported(d, E, M) || (cfg->flags & ENGRAM_VARIANT_FLAGS) != 0))
+    return ENGRAM_ERR_UNSUPPORTED;
   if (table != nullptr) {
     rc = launch_gather(hp, idx, table, N, elem_bytes(cfg), e, s);
     if (rc) return rc;
@@ -200,7 +202,8 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
   if (cfg->dtype == ENGRAM_F32)
     return launch_forward_f32(static_cast<const float*>(e), static_cast<const float*>(h),
                               static_cast<const float*>(Wk), static_cast<const float*>(Wv), conv_w,
-                              conv_state, static_cast<float*>(out), saved, N, T, M, d, E, ws, s);
+                              cfg->flags, conv_state, static_cast<float*>(out), saved, N, T, M, d,
+                              E, ws, s);
   float* kv_save = saved != nullptr && conv_state == nullptr && saves_kv(cfg)
                        ? reinterpret_cast<float*>(reinterpret_cast<char*>(saved) +
                                                   alpha_bytes_padded(N))
@@ -219,8 +222,11 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                     void* ws, size_t ws_bytes, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (cfg->dtype == ENGRAM_BF16 && (cfg->n_branch != 1 || saved == nullptr))
-    return cfg->n_branch != 1 ? ENGRAM_ERR_UNSUPPORTED : ENGRAM_ERR_INVALID_ARG;
+  if (cfg->dtype == ENGRAM_BF16 &&
+      (cfg->n_branch != 1 || saved == nullptr || (cfg->flags & ENGRAM_VARIANT_FLAGS) != 0))
+    return saved == nullptr && cfg->n_branch == 1 && (cfg->flags & ENGRAM_VARIANT_FLAGS) == 0
+               ? ENGRAM_ERR_INVALID_ARG
+               : ENGRAM_ERR_UNSUPPORTED;
   if (B < 0 || T < 0) return ENGRAM_ERR_INVALID_ARG;
   const int64_t N = (int64_t)B * T;
   if (idx == nullptr || e == nullptr || h == nullptr || Wk == nullptr || Wv == nullptr ||
@@ -261,7 +267,8 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
   F32Saved sv = f32_saved_layout(saved != nullptr ? const_cast<float*>(saved) : ws, N, M, d);
   rc = launch_backward_f32(static_cast<const float*>(e), static_cast<const float*>(h),
                            static_cast<const float*>(Wk), static_cast<const float*>(Wv), conv_w,
-                           sv, dout, dh, dWk, dWv, dconv_w, de_buf, N, T, M, d, E, ws, s);
+                           cfg->flags, sv, dout, dh, dWk, dWv, dconv_w, de_buf, N, T, M, d, E, ws,
+                           s);
   if (rc) return rc;
   return launch_table_grad(hp, idx, de_buf, N, dtab_keys, dtab_rows, n_unique,
                            static_cast<char*>(ws) + bw, ws_bytes - bw, s);
@@ -323,6 +330,12 @@ int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const 
   }
   if (done_event != nullptr) return ck(cudaEventRecord((cudaEvent_t)done_event, s));
   return ENGRAM_OK;
+}
+
+int64_t engram_param_floats(const engram_cfg_t* cfg) {
+  if (check_cfg(cfg) != ENGRAM_OK) return 0;
+  if (cfg->dtype == ENGRAM_BF16) return (int64_t)cfg->d_model * 4;
+  return f32_param_floats(cfg->flags, cfg->n_branch, cfg->d_model);
 }
 
 int64_t engram_table_rows(const engram_cfg_t* cfg) {

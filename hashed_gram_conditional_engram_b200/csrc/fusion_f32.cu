@@ -23,6 +23,32 @@ __device__ __forceinline__ float warp_sum(float x) {
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// The formulation variants of the layer's flags, and where their parameters
+// sit in the small-parameter block: conv weights ([M or 1][d][4]), then with
+// ENGRAM_NORM_SCALES g_h [M][d], g_k [M][d] and, with ENGRAM_CONV_PRENORM,
+// g_v [M][d].
+struct F32Var {
+  int dil;         // conv dilation: 1, or 3 with ENGRAM_CONV_DILATED
+  int prenorm;     // the conv reads RMSNorm(vt) (times g_v)
+  int per_branch;  // conv weights per branch
+  const float* w;
+  const float *gh, *gk, *gv;  // NULL when absent (scale 1)
+  __device__ const float* taps(int m, int d, int c) const {
+    return w + ((int64_t)(per_branch ? m : 0) * d + c) * 4;
+  }
+  // g_h g_k of branch m, feature c
+  __device__ double gg(int m, int d, int c) const {
+    return gh != nullptr ? (double)gh[m * d + c] * (double)gk[m * d + c] : 1.0;
+  }
+  // the conv input of token n, branch m, feature c
+  __device__ double conv_in(const double* alpha, const double* v, const double* rc, int64_t n,
+                            int m, int M, int d, int c) const {
+    const double vt = alpha[n * M + m] * v[n * d + c];
+    if (!prenorm) return vt;
+    return vt * rc[n * M + m] * (gv != nullptr ? (double)gv[m * d + c] : 1.0);
+  }
+};
+
 // The forward keeps every product and sum in fp64 and rounds each stored
 // value (out, and alpha, k, v, y in `saved`) to fp32 once.
 
@@ -61,66 +87,74 @@ __global__ void proj_f32_kernel(const float* __restrict__ e, const float* __rest
   }
 }
 
-// alpha[n,m] = sigmoid(<RMSNorm(h), RMSNorm(k)> / sqrt(d)): one warp per (n, m).
+// alpha[n,m] = sigmoid(<RMSNorm(h) g_h, RMSNorm(k) g_k> / sqrt(d)): one warp
+// per (n, m).  With the pre-conv norm it also keeps
+// r_c[n,m] = (mean(vt^2) + eps)^(-1/2), vt = alpha v.
 __global__ void gate_f32_kernel(const float* __restrict__ h, const double* __restrict__ k,
+                                const double* __restrict__ v, const F32Var var,
                                 double* __restrict__ alpha, float* __restrict__ alpha32,
-                                int64_t NM, int d) {
+                                double* __restrict__ rc, int64_t NM, int M, int d) {
   const int lane = threadIdx.x & 31;
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (w >= NM) return;
+  const int m = (int)(w % M);
   const float* hr = h + w * d;
   const double* kr = k + w * d;
-  double hh = 0.0, kk = 0.0, hk = 0.0;
+  const double* vr = v + (w / M) * d;
+  double hh = 0.0, kk = 0.0, hk = 0.0, vv = 0.0;
   for (int c = lane; c < d; c += 32) {
     const double a = hr[c], b = kr[c];
     hh = fma(a, a, hh);
     kk = fma(b, b, kk);
-    hk = fma(a, b, hk);
+    hk = fma(a * b, var.gg(m, d, c), hk);
+    if (var.prenorm) vv = fma(vr[c], vr[c], vv);
   }
   hh = warp_sum_fd(hh);
   kk = warp_sum_fd(kk);
   hk = warp_sum_fd(hk);
+  vv = warp_sum_fd(vv);
   if (lane == 0) {
     const double rh = 1.0 / sqrt(hh / d + (double)RMS_EPS);
     const double rk = 1.0 / sqrt(kk / d + (double)RMS_EPS);
     const double a = 1.0 / (1.0 + exp(-(hk * rh * rk / sqrt((double)d))));
     alpha[w] = a;
     alpha32[w] = (float)a;
+    if (var.prenorm) rc[w] = 1.0 / sqrt(a * a * vv / d + (double)RMS_EPS);
   }
 }
 
-// y = sum_i w[c,i] vt_{t-3+i}, out = h + vt + SiLU(y): one thread per (n, m, c).
-// With conv_state (decode, T == 1) the three earlier vt come from the state,
-// which is then shifted by one step.
-// h and out may be the same buffer (each element is read before it is
-// written, by the same thread), so neither is declared __restrict__.
+// y = sum_i w[c,i] c_{t-(3-i) dil}, out = h + vt + SiLU(y): one thread per
+// (n, m, c); the conv input c is vt, or RMSNorm(vt) g_v with the pre-conv
+// norm.  With conv_state (decode, T == 1) the earlier inputs come from the
+// state ([3 dil][d] per (n, m), oldest first), which is then shifted by one
+// step.  h and out may be the same buffer (each element is read before it
+// is written, by the same thread), so neither is declared __restrict__.
 __global__ void conv_f32_kernel(const float* h, const double* __restrict__ v,
-                                const double* __restrict__ alpha, const float* __restrict__ w,
-                                float* __restrict__ conv_state, float* __restrict__ y_out,
-                                float* out, int64_t N, int T, int M, int d) {
+                                const double* __restrict__ alpha, const double* __restrict__ rc,
+                                const F32Var var, float* __restrict__ conv_state,
+                                float* __restrict__ y_out, float* out, int64_t N, int T, int M,
+                                int d) {
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= N * M * d) return;
   const int c = (int)(g % d);
   const int m = (int)((g / d) % M);
   const int64_t n = g / ((int64_t)d * M);
-  const float4 wc = *reinterpret_cast<const float4*>(w + 4 * c);
-  const double taps[4] = {wc.x, wc.y, wc.z, wc.w};
+  const float* wp = var.taps(m, d, c);
+  const double taps[4] = {wp[0], wp[1], wp[2], wp[3]};
   const double vt = alpha[n * M + m] * v[n * d + c];
-  double y = taps[3] * vt;
+  const double cin = var.conv_in(alpha, v, rc, n, m, M, d, c);
+  double y = taps[3] * cin;
+  const int dil = var.dil;
   if (conv_state != nullptr) {
-    float* st = conv_state + ((n * M + m) * 3) * d + c;  // [3][d] oldest first
-    const double s0 = st[0], s1 = st[d], s2 = st[2 * d];
-    y = fma(taps[0], s0, fma(taps[1], s1, fma(taps[2], s2, y)));
-    st[0] = (float)s1;
-    st[d] = (float)s2;
-    st[2 * d] = (float)vt;
+    float* st = conv_state + ((n * M + m) * 3 * dil) * d + c;  // [3 dil][d] oldest first
+    for (int L = 3; L >= 1; --L) y = fma(taps[3 - L], (double)st[(3 * dil - L * dil) * d], y);
+    for (int q = 0; q + 1 < 3 * dil; ++q) st[q * d] = st[(q + 1) * d];
+    st[(3 * dil - 1) * d] = (float)cin;
   } else {
     const int t = (int)(n % T);
-    for (int lag = 1; lag <= 3; ++lag) {
-      if (t >= lag) {
-        const int64_t p = n - lag;
-        y = fma(taps[3 - lag], alpha[p * M + m] * v[p * d + c], y);
-      }
+    for (int L = 1; L <= 3; ++L) {
+      const int lag = L * dil;
+      if (t >= lag) y = fma(taps[3 - L], var.conv_in(alpha, v, rc, n - lag, m, M, d, c), y);
     }
   }
   y_out[g] = (float)y;
@@ -162,62 +196,75 @@ __global__ void rec_proj_kernel(const float* __restrict__ e, const float* __rest
   }
 }
 
-// alpha64[n,m] and the row sums the gate backward needs: one warp per (n, m)
+// alpha64[n,m] and the row sums the gate backward needs (r_h, r_k,
+// <h g_h g_k, k>; r_c of the pre-conv norm in rc): one warp per (n, m)
 __global__ void rec_gate_kernel(const float* __restrict__ h, const double* __restrict__ k,
+                                const double* __restrict__ v, const F32Var var,
                                 double* __restrict__ alpha, double* __restrict__ sums,
-                                int64_t NM, int d) {
+                                double* __restrict__ rc, int64_t NM, int M, int d) {
   const int lane = threadIdx.x & 31;
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (w >= NM) return;
-  double hh = 0.0, kk = 0.0, hk = 0.0;
+  const int m = (int)(w % M);
+  const double* vr = v + (w / M) * d;
+  double hh = 0.0, kk = 0.0, hk = 0.0, vv = 0.0;
   for (int c = lane; c < d; c += 32) {
     const double a = h[w * d + c], b = k[w * d + c];
     hh = fma(a, a, hh);
     kk = fma(b, b, kk);
-    hk = fma(a, b, hk);
+    hk = fma(a * b, var.gg(m, d, c), hk);
+    if (var.prenorm) vv = fma(vr[c], vr[c], vv);
   }
   hh = warp_sum_d(hh);
   kk = warp_sum_d(kk);
   hk = warp_sum_d(hk);
+  vv = warp_sum_d(vv);
   if (lane == 0) {
     const double rh = 1.0 / sqrt(hh / d + (double)RMS_EPS);
     const double rk = 1.0 / sqrt(kk / d + (double)RMS_EPS);
-    alpha[w] = sigmoid_d(hk * rh * rk / sqrt((double)d));
+    const double a = sigmoid_d(hk * rh * rk / sqrt((double)d));
+    alpha[w] = a;
     sums[3 * w + 0] = rh;
     sums[3 * w + 1] = rk;
     sums[3 * w + 2] = hk;
+    if (var.prenorm) rc[w] = 1.0 / sqrt(a * a * vv / d + (double)RMS_EPS);
   }
 }
 
 // y64 and dy64 = dout * SiLU'(y): one thread per (n, m, c)
 __global__ void rec_conv_dsilu_kernel(const double* __restrict__ v, const double* __restrict__ alpha,
-                                      const float* __restrict__ w, const float* __restrict__ dout,
-                                      double* __restrict__ dy, int64_t N, int T, int M, int d) {
+                                      const double* __restrict__ rc, const F32Var var,
+                                      const float* __restrict__ dout, double* __restrict__ dy,
+                                      int64_t N, int T, int M, int d) {
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= N * M * d) return;
   const int c = (int)(g % d);
   const int m = (int)((g / d) % M);
   const int64_t n = g / ((int64_t)d * M);
   const int t = (int)(n % T);
+  const float* wp = var.taps(m, d, c);
   double y = 0.0;
-  for (int lag = 0; lag <= 3; ++lag) {
-    if (t >= lag) {
-      const int64_t p = n - lag;
-      y = fma((double)w[4 * c + 3 - lag], alpha[p * M + m] * v[p * d + c], y);
-    }
+  for (int L = 0; L <= 3; ++L) {
+    const int lag = L * var.dil;
+    if (t >= lag) y = fma((double)wp[3 - L], var.conv_in(alpha, v, rc, n - lag, m, M, d, c), y);
   }
   const double s = sigmoid_d(y);
   dy[g] = (double)dout[g] * s * (1.0 + y * (1.0 - s));
 }
 
-// One warp per (n, m): dvt = dout + sum_i w[:,i] dy_{t+3-i}; dalpha = <dvt, v>;
-// dz = dalpha a (1 - a); RMSNorm backward for h and k:
-//   dx = r dxh - r^3 x <dxh, x> / d, with dh^ = dz k^ / sqrt(d), dk^ = dz h^ / sqrt(d).
+// One warp per (n, m).  dc = sum_i w[:,i] dy_{t+(3-i) dil} (the gradient of
+// the conv input); dvt = dout + dc, or with the pre-conv norm
+// dout + r_c dc^ - r_c^3 vt <dc^, vt> / d with dc^ = dc g_v; dalpha =
+// <dvt, v>; dz = dalpha a (1 - a); the gate's RMSNorm backwards:
+//   dx = r dxh - r^3 x <dxh, x> / d, with dh^ = dz g_h g_k k^ / sqrt(d) and
+//   dk^ = dz g_h g_k h^ / sqrt(d).
+// dc (for g_v's gradient) and dz (for g_h's and g_k's) are kept when asked.
 __global__ void gate_bwd_kernel(const float* __restrict__ dout, const double* __restrict__ dy,
                                 const float* __restrict__ h, const double* __restrict__ k,
                                 const double* __restrict__ v, const double* __restrict__ alpha,
-                                const double* __restrict__ sums, const float* __restrict__ w,
-                                double* __restrict__ dvt, float* __restrict__ dh,
+                                const double* __restrict__ sums, const double* __restrict__ rc,
+                                const F32Var var, double* __restrict__ dvt, double* __restrict__ dc_keep,
+                                double* __restrict__ dz_keep, float* __restrict__ dh,
                                 double* __restrict__ dk, int64_t N, int T, int M, int d) {
   const int lane = threadIdx.x & 31;
   const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -225,27 +272,49 @@ __global__ void gate_bwd_kernel(const float* __restrict__ dout, const double* __
   const int m = (int)(wid % M);
   const int64_t n = wid / M;
   const int t = (int)(n % T);
+  const double al = alpha[wid];
+  // dc into dvt; with the pre-conv norm also <dc^, vt>
+  double cv = 0.0;
+  for (int c = lane; c < d; c += 32) {
+    const float* wp = var.taps(m, d, c);
+    double g = 0.0;
+    for (int L = 0; L <= 3; ++L) {
+      const int lag = L * var.dil;
+      if (t + lag < T) g = fma((double)wp[3 - L], dy[((n + lag) * M + m) * d + c], g);
+    }
+    dvt[wid * d + c] = g;
+    if (dc_keep != nullptr) dc_keep[wid * d + c] = g;
+    if (var.prenorm) {
+      const double gvc = var.gv != nullptr ? (double)var.gv[m * d + c] : 1.0;
+      cv = fma(g * gvc, al * v[n * d + c], cv);
+    }
+  }
+  cv = warp_sum_d(cv);
+  const double r = var.prenorm ? rc[wid] : 0.0;
   double da = 0.0;
   for (int c = lane; c < d; c += 32) {
-    double g = dout[wid * d + c];
-    for (int lag = 0; lag <= 3; ++lag) {
-      if (t + lag < T) g = fma((double)w[4 * c + 3 - lag], dy[((n + lag) * M + m) * d + c], g);
+    double g = dvt[wid * d + c];
+    if (var.prenorm) {
+      const double gvc = var.gv != nullptr ? (double)var.gv[m * d + c] : 1.0;
+      g = r * (g * gvc) - r * r * r * (al * v[n * d + c]) * cv / d;
     }
+    g += (double)dout[wid * d + c];
     dvt[wid * d + c] = g;
     da = fma(g, v[n * d + c], da);
   }
   da = warp_sum_d(da);
-  const double al = alpha[wid];
   const double dz = da * al * (1.0 - al);
+  if (dz_keep != nullptr && lane == 0) dz_keep[wid] = dz;
   const double rh = sums[3 * wid], rk = sums[3 * wid + 1], hk = sums[3 * wid + 2];
   const double isd = 1.0 / sqrt((double)d);
-  // <dh^, h> = dz/sqrt(d) * rk * <k, h>, <dk^, k> = dz/sqrt(d) * rh * <h, k>
+  // <dh^, h> = dz/sqrt(d) * rk * <h g g, k>, <dk^, k> = dz/sqrt(d) * rh * <h g g, k>
   const double dot_hh = dz * isd * rk * hk;
   const double dot_kk = dz * isd * rh * hk;
   for (int c = lane; c < d; c += 32) {
     const double a = h[wid * d + c], b = k[wid * d + c];
-    const double dhh = dz * isd * rk * b;
-    const double dkh = dz * isd * rh * a;
+    const double gg = var.gg(m, d, c);
+    const double dhh = dz * isd * rk * gg * b;
+    const double dkh = dz * isd * rh * gg * a;
     dh[wid * d + c] = (float)((double)dout[wid * d + c] + rh * dhh - rh * rh * rh * a * dot_hh / d);
     dk[wid * d + c] = rk * dkh - rk * rk * rk * b * dot_kk / d;
   }
@@ -263,20 +332,53 @@ __global__ void dv_kernel(const double* __restrict__ dvt, const double* __restri
   dv[g] = acc;
 }
 
-// dconv_w[c,i] = sum_n sum_m dy[n,m,c] vt_{n-3+i}[m,c] (tokens, then branches, ascending)
+// dconv_w[mc,c,i] = sum_n sum_m dy[n,m,c] c_{n-(3-i) dil}[m,c] over the
+// branches m that conv mc serves (all of them for a shared conv): tokens,
+// then branches, ascending
 __global__ void dconv_kernel(const double* __restrict__ dy, const double* __restrict__ v,
-                             const double* __restrict__ alpha, float* __restrict__ dw, int64_t N,
-                             int T, int M, int d) {
+                             const double* __restrict__ alpha, const double* __restrict__ rc,
+                             const F32Var var, float* __restrict__ dw, int64_t N, int T, int M,
+                             int d) {
+  const int Mc = var.per_branch ? M : 1;
   const int g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= d * 4) return;
-  const int c = g >> 2, i = g & 3, lag = 3 - i;
+  if (g >= Mc * d * 4) return;
+  const int i = g & 3, c = (g >> 2) % d, mc = (g >> 2) / d;
+  const int lag = (3 - i) * var.dil;
+  const int m0 = var.per_branch ? mc : 0, m1 = var.per_branch ? mc + 1 : M;
   double acc = 0.0;
   for (int64_t n = 0; n < N; ++n) {
     if ((int)(n % T) < lag) continue;
-    const int64_t p = n - lag;
-    for (int m = 0; m < M; ++m) acc = fma(dy[(n * M + m) * d + c], alpha[p * M + m] * v[p * d + c], acc);
+    for (int m = m0; m < m1; ++m)
+      acc = fma(dy[(n * M + m) * d + c], var.conv_in(alpha, v, rc, n - lag, m, M, d, c), acc);
   }
   dw[g] = (float)acc;
+}
+
+// The learnable norm scales' gradients, one thread per (m, c), tokens in
+// ascending order:
+//   dg_h = sum_n dz h^ k^ g_k / sqrt(d),  dg_k = sum_n dz h^ k^ g_h / sqrt(d),
+//   dg_v = sum_n dc c^ (c^ = RMSNorm(vt), with the pre-conv norm).
+__global__ void dscale_kernel(const float* __restrict__ h, const double* __restrict__ k,
+                              const double* __restrict__ v, const double* __restrict__ alpha,
+                              const double* __restrict__ sums, const double* __restrict__ rc,
+                              const double* __restrict__ dz, const double* __restrict__ dc,
+                              const F32Var var, float* __restrict__ dgh, float* __restrict__ dgk,
+                              float* __restrict__ dgv, int64_t N, int M, int d) {
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= M * d) return;
+  const int m = g / d, c = g % d;
+  const double isd = 1.0 / sqrt((double)d);
+  double ah = 0.0, ak = 0.0, avv = 0.0;
+  for (int64_t n = 0; n < N; ++n) {
+    const int64_t w = n * M + m;
+    const double hk = (double)h[w * d + c] * sums[3 * w] * k[w * d + c] * sums[3 * w + 1];
+    ah = fma(dz[w] * hk, (double)var.gk[g] * isd, ah);
+    ak = fma(dz[w] * hk, (double)var.gh[g] * isd, ak);
+    if (var.prenorm) avv = fma(dc[w * d + c], alpha[w] * v[n * d + c] * rc[w], avv);
+  }
+  dgh[g] = (float)ah;
+  dgk[g] = (float)ak;
+  if (var.prenorm) dgv[g] = (float)avv;
 }
 
 // dWk[m,c,i] = sum_n dk[n,m,c] e[n,i]; dWv[c,i] = sum_n dv[n,c] e[n,i]
@@ -319,6 +421,22 @@ inline unsigned blocks_for(int64_t threads_total, int per_block) {
   return (unsigned)((threads_total + per_block - 1) / per_block);
 }
 
+// the variants of `flags` over a small-parameter block (or its gradient)
+F32Var make_var(int flags, const float* block, int M, int d) {
+  F32Var v;
+  v.dil = (flags & ENGRAM_CONV_DILATED) ? 3 : 1;
+  v.prenorm = (flags & ENGRAM_CONV_PRENORM) ? 1 : 0;
+  v.per_branch = (flags & ENGRAM_CONV_PER_BRANCH) ? 1 : 0;
+  v.w = block;
+  v.gh = v.gk = v.gv = nullptr;
+  if (flags & ENGRAM_NORM_SCALES) {
+    v.gh = block + (int64_t)(v.per_branch ? M : 1) * d * 4;
+    v.gk = v.gh + (int64_t)M * d;
+    if (v.prenorm) v.gv = v.gk + (int64_t)M * d;
+  }
+  return v;
+}
+
 }  // namespace
 
 size_t f32_saved_bytes(int64_t N, int M, int d) {
@@ -342,13 +460,20 @@ F32Saved f32_saved_layout(void* base, int64_t N, int M, int d) {
 
 size_t f32_forward_ws_bytes(int64_t N, int M, int d) {
   auto up = [](size_t b) { return (b + 255) & ~(size_t)255; };
-  return up((size_t)N * M * d * 8) + up((size_t)N * d * 8) + up((size_t)N * M * 8) +
+  return up((size_t)N * M * d * 8) + up((size_t)N * d * 8) + 2 * up((size_t)N * M * 8) +
          f32_saved_bytes(N, M, d);
 }
 
+int64_t f32_param_floats(int flags, int M, int d) {
+  int64_t n = (int64_t)((flags & ENGRAM_CONV_PER_BRANCH) ? M : 1) * d * 4;
+  if (flags & ENGRAM_NORM_SCALES) n += (int64_t)((flags & ENGRAM_CONV_PRENORM) ? 3 : 2) * M * d;
+  return n;
+}
+
 int launch_forward_f32(const float* e, const float* h, const float* Wk, const float* Wv,
-                       const float* conv_w, float* conv_state, float* out, float* saved, int64_t N,
-                       int T, int M, int d, int E, void* ws, cudaStream_t s) {
+                       const float* params, int flags, float* conv_state, float* out,
+                       float* saved, int64_t N, int T, int M, int d, int E, void* ws,
+                       cudaStream_t s) {
   if (N == 0) return ENGRAM_OK;
   auto up = [](size_t b) { return (b + 255) & ~(size_t)255; };
   char* p = static_cast<char*>(ws);
@@ -358,19 +483,23 @@ int launch_forward_f32(const float* e, const float* h, const float* Wk, const fl
   p += up((size_t)N * d * 8);
   double* a64 = reinterpret_cast<double*>(p);
   p += up((size_t)N * M * 8);
+  double* rc64 = reinterpret_cast<double*>(p);
+  p += up((size_t)N * M * 8);
   F32Saved sv = f32_saved_layout(saved != nullptr ? static_cast<void*>(saved) : p, N, M, d);
+  const F32Var var = make_var(flags, params, M, d);
   const int tb = 256;
   proj_f32_kernel<<<blocks_for(N * (M + 1) * d * 32, tb), tb, 0, s>>>(e, Wk, Wv, k64, v64, sv.k,
                                                                       sv.v, N, M, d, E);
-  gate_f32_kernel<<<blocks_for(N * M * 32, tb), tb, 0, s>>>(h, k64, a64, sv.alpha, N * M, d);
-  conv_f32_kernel<<<blocks_for(N * M * d, tb), tb, 0, s>>>(h, v64, a64, conv_w, conv_state, sv.y,
-                                                           out, N, T, M, d);
+  gate_f32_kernel<<<blocks_for(N * M * 32, tb), tb, 0, s>>>(h, k64, v64, var, a64, sv.alpha,
+                                                            rc64, N * M, M, d);
+  conv_f32_kernel<<<blocks_for(N * M * d, tb), tb, 0, s>>>(h, v64, a64, rc64, var, conv_state,
+                                                           sv.y, out, N, T, M, d);
   return ck(cudaGetLastError());
 }
 
 namespace {
 struct BwdWs {
-  double *k, *v, *alpha, *sums, *dy, *dvt, *dk, *dv;
+  double *k, *v, *alpha, *sums, *rc, *dz, *dy, *dvt, *dc, *dk, *dv;
   float* de;
 };
 size_t bwd_layout(void* base, int64_t N, int M, int d, int E, BwdWs* out) {
@@ -383,8 +512,11 @@ size_t bwd_layout(void* base, int64_t N, int M, int d, int E, BwdWs* out) {
   w.v = reinterpret_cast<double*>(p + off); off += up(Nd * 8);
   w.alpha = reinterpret_cast<double*>(p + off); off += up(NM * 8);
   w.sums = reinterpret_cast<double*>(p + off); off += up(NM * 3 * 8);
+  w.rc = reinterpret_cast<double*>(p + off); off += up(NM * 8);
+  w.dz = reinterpret_cast<double*>(p + off); off += up(NM * 8);
   w.dy = reinterpret_cast<double*>(p + off); off += up(NMd * 8);
   w.dvt = reinterpret_cast<double*>(p + off); off += up(NMd * 8);
+  w.dc = reinterpret_cast<double*>(p + off); off += up(NMd * 8);
   w.dk = reinterpret_cast<double*>(p + off); off += up(NMd * 8);
   w.dv = reinterpret_cast<double*>(p + off); off += up(Nd * 8);
   w.de = reinterpret_cast<float*>(p + off); off += up((size_t)N * E * 4);
@@ -404,26 +536,42 @@ float* backward_f32_de_slot(void* ws, int64_t N, int M, int d, int E) {
 }
 
 int launch_backward_f32(const float* e, const float* h, const float* Wk, const float* Wv,
-                        const float* conv_w, F32Saved sv, const float* dout, float* dh, float* dWk,
-                        float* dWv, float* dconv_w, float* de, int64_t N, int T, int M, int d,
-                        int E, void* ws, cudaStream_t s) {
+                        const float* params, int flags, F32Saved sv, const float* dout, float* dh,
+                        float* dWk, float* dWv, float* dparams, float* de, int64_t N, int T, int M,
+                        int d, int E, void* ws, cudaStream_t s) {
   (void)sv;
   BwdWs w;
   bwd_layout(ws, N, M, d, E, &w);
+  const F32Var var = make_var(flags, params, M, d);
+  const F32Var dvar = make_var(flags, dparams, M, d);  // where each gradient goes
+  const bool scales = (flags & ENGRAM_NORM_SCALES) != 0;
   const int tb = 256;
   if (N > 0) {
     rec_proj_kernel<<<blocks_for(N * (M + 1) * d * 32, tb), tb, 0, s>>>(e, Wk, Wv, w.k, w.v, N, M,
                                                                         d, E);
-    rec_gate_kernel<<<blocks_for(N * M * 32, tb), tb, 0, s>>>(h, w.k, w.alpha, w.sums, N * M, d);
-    rec_conv_dsilu_kernel<<<blocks_for(N * M * d, tb), tb, 0, s>>>(w.v, w.alpha, conv_w, dout,
+    rec_gate_kernel<<<blocks_for(N * M * 32, tb), tb, 0, s>>>(h, w.k, w.v, var, w.alpha, w.sums,
+                                                              w.rc, N * M, M, d);
+    rec_conv_dsilu_kernel<<<blocks_for(N * M * d, tb), tb, 0, s>>>(w.v, w.alpha, w.rc, var, dout,
                                                                    w.dy, N, T, M, d);
-    gate_bwd_kernel<<<blocks_for(N * M * 32, tb), tb, 0, s>>>(dout, w.dy, h, w.k, w.v, w.alpha,
-                                                              w.sums, conv_w, w.dvt, dh, w.dk, N,
-                                                              T, M, d);
+    gate_bwd_kernel<<<blocks_for(N * M * 32, tb), tb, 0, s>>>(
+        dout, w.dy, h, w.k, w.v, w.alpha, w.sums, w.rc, var, w.dvt, scales ? w.dc : nullptr,
+        scales ? w.dz : nullptr, dh, w.dk, N, T, M, d);
     dv_kernel<<<blocks_for(N * d, tb), tb, 0, s>>>(w.dvt, w.alpha, w.dv, N, M, d);
   }
-  dconv_kernel<<<blocks_for((int64_t)d * 4, tb), tb, 0, s>>>(w.dy, w.v, w.alpha, dconv_w, N, T, M,
-                                                             d);
+  const int Mc = var.per_branch ? M : 1;
+  dconv_kernel<<<blocks_for((int64_t)Mc * d * 4, tb), tb, 0, s>>>(w.dy, w.v, w.alpha, w.rc, var,
+                                                                  dparams, N, T, M, d);
+  if (scales) {
+    if (N > 0) {
+      dscale_kernel<<<blocks_for((int64_t)M * d, tb), tb, 0, s>>>(
+          h, w.k, w.v, w.alpha, w.sums, w.rc, w.dz, w.dc, var, const_cast<float*>(dvar.gh),
+          const_cast<float*>(dvar.gk), const_cast<float*>(dvar.gv), N, M, d);
+    } else {  // no tokens: zero gradients
+      const size_t nb = (size_t)(f32_param_floats(flags, M, d) - (int64_t)Mc * d * 4) * 4;
+      const int rc = ck(cudaMemsetAsync(const_cast<float*>(dvar.gh), 0, nb, s));
+      if (rc) return rc;
+    }
+  }
   dweight_kernel<<<blocks_for((int64_t)(M + 1) * d * E, tb), tb, 0, s>>>(w.dk, w.dv, e, dWk, dWv,
                                                                          N, M, d, E);
   if (N > 0)

@@ -83,15 +83,19 @@ struct F32Saved {
 F32Saved f32_saved_layout(void* base, int64_t N, int M, int d);
 size_t f32_saved_bytes(int64_t N, int M, int d);
 size_t f32_forward_ws_bytes(int64_t N, int M, int d);
+// params: the small-parameter block of the layer's flags (conv weights,
+// then the norm scales); dparams its gradient in the same layout
+int64_t f32_param_floats(int flags, int M, int d);
 int launch_forward_f32(const float* e, const float* h, const float* Wk, const float* Wv,
-                       const float* conv_w, float* conv_state, float* out, float* saved, int64_t N,
-                       int T, int M, int d, int E, void* ws, cudaStream_t s);
+                       const float* params, int flags, float* conv_state, float* out,
+                       float* saved, int64_t N, int T, int M, int d, int E, void* ws,
+                       cudaStream_t s);
 size_t backward_f32_ws_bytes(int64_t N, int M, int d, int E);
 float* backward_f32_de_slot(void* ws, int64_t N, int M, int d, int E);
 int launch_backward_f32(const float* e, const float* h, const float* Wk, const float* Wv,
-                        const float* conv_w, F32Saved sv, const float* dout, float* dh, float* dWk,
-                        float* dWv, float* dconv_w, float* de, int64_t N, int T, int M, int d,
-                        int E, void* ws, cudaStream_t s);
+                        const float* params, int flags, F32Saved sv, const float* dout, float* dh,
+                        float* dWk, float* dWv, float* dparams, float* de, int64_t N, int T, int M,
+                        int d, int E, void* ws, cudaStream_t s);
 
 // sort / scan / segmented reduce
 size_t table_grad_ws_bytes(int64_t n_items);

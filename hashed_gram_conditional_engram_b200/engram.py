@@ -23,6 +23,8 @@ F32, BF16 = 0, 1
 WS_VOCAB, WS_FORWARD, WS_BACKWARD, WS_TABLE_GRAD = 0, 1, 2, 3
 WS_HOSTCACHE_RANK, WS_HOSTCACHE_GATHER = 4, 5
 SAVE_KV = 1  # EngramCfg.flags
+# formulation variants (fp32 layers)
+CONV_DILATED, CONV_PRENORM, CONV_PER_BRANCH, NORM_SCALES = 2, 4, 8, 16
 STATUS_BAD_ID, STATUS_BAD_INDEX, STATUS_TIMEOUT = 1, 2, 4
 
 ERRORS = {
@@ -41,7 +43,7 @@ EXPORTED = (
     "engram_hash_indices", "engram_gather", "engram_forward", "engram_backward",
     "engram_table_grad", "engram_table_grad_noalloc", "engram_forward_hosttable",
     "engram_get_status",
-    "engram_device_sm_count", "engram_clock_probe", "engram_table_rows",
+    "engram_device_sm_count", "engram_clock_probe", "engram_table_rows", "engram_param_floats",
     "engram_hostcache_rank", "engram_hostcache_fill", "engram_forward_hostcache",
 )
 
@@ -113,6 +115,7 @@ def lib() -> ctypes.CDLL:
         "engram_device_sm_count": (ctypes.c_int, []),
         "engram_clock_probe": (ctypes.c_int, [P, i64, P]),
         "engram_table_rows": (ctypes.c_int64, [cfgp]),
+        "engram_param_floats": (ctypes.c_int64, [cfgp]),
         "engram_hostcache_rank": (ctypes.c_int, [cfgp, P, i64, i64, P, P, P, sz, P]),
         "engram_hostcache_fill": (ctypes.c_int, [cfgp, P, P, i64, P, P, P]),
         "engram_forward_hostcache": (ctypes.c_int, [cfgp, P, P, P, P, i64, P, P, P, sz, P, P]),
@@ -233,6 +236,10 @@ def _event_handle(done_event, side_stream):
     if done_event.cuda_event == 0:
         done_event.record(side_stream)
     return done_event.cuda_event
+
+
+def engram_param_floats(cfg: EngramCfg) -> int:
+    return int(lib().engram_param_floats(ctypes.byref(cfg)))
 
 
 def engram_table_rows(cfg: EngramCfg) -> int:

@@ -56,6 +56,16 @@ enum { ENGRAM_F32 = 0, ENGRAM_BF16 = 1 };
 
 /* engram_cfg_t.flags */
 #define ENGRAM_SAVE_KV 1
+/* formulation variants (fp32 layers; a bf16 layer with any of them is
+ * ENGRAM_ERR_UNSUPPORTED): the pages fix neither the conv's dilation, nor a
+ * norm before it, nor whether branches share it, nor learnable norm scales
+ * ([p2] short depthwise causal conv; [p5 二.1 (2)] 一维卷积; [p5 二.2]) */
+#define ENGRAM_CONV_DILATED 2     /* taps at t, t-3, t-6, t-9 (dilation 3 = the largest order) */
+#define ENGRAM_CONV_PRENORM 4     /* the conv reads RMSNorm(vt) (times g_v with NORM_SCALES) */
+#define ENGRAM_CONV_PER_BRANCH 8  /* conv weights per branch */
+#define ENGRAM_NORM_SCALES 16     /* learnable RMSNorm scales g_h, g_k (and g_v) */
+#define ENGRAM_VARIANT_FLAGS \
+  (ENGRAM_CONV_DILATED | ENGRAM_CONV_PRENORM | ENGRAM_CONV_PER_BRANCH | ENGRAM_NORM_SCALES)
 
 enum {
   ENGRAM_OK = 0,
@@ -89,7 +99,16 @@ enum {
  *            token's k then its v, after alpha from the next 256-byte
  *            boundary), and the backward reads them instead of recomputing
  *            them: 8 * n_tok * d_model more bytes of `saved` for one GEMM
- *            less in the backward.  Any other bit is ENGRAM_ERR_INVALID_ARG.
+ *            less in the backward.
+ *            ENGRAM_CONV_DILATED, ENGRAM_CONV_PRENORM, ENGRAM_CONV_PER_BRANCH,
+ *            ENGRAM_NORM_SCALES (fp32 layers): formulation variants, any
+ *            combination.  z = <RMSNorm(h) g_h, RMSNorm(k) g_k> / sqrt(d),
+ *            vt = alpha v, c = RMSNorm(vt) g_v (PRENORM) or vt,
+ *            y_t = sum_i w[:, i] c_{t-(3-i) dil} (dil 3 with DILATED, else 1),
+ *            out = h + vt + SiLU(y); each branch m has its own w (PER_BRANCH)
+ *            and its own g_h, g_k, g_v (NORM_SCALES).  Their parameters form
+ *            the conv_w block (engram_param_floats floats).
+ *            Any other bit is ENGRAM_ERR_INVALID_ARG.
  *   rows[j]  P_j, row count (a prime) of head j's table.  Head j's rows sit
  *            in one packed table after those of heads 0..j-1.
  *   mult[j]  odd 64-bit multipliers of head j for n-gram positions 0, 1, 2
@@ -176,10 +195,12 @@ int engram_gather(const engram_cfg_t* cfg, const int32_t* idx, const void* table
  *   Wk      device [M, d, E] key projections, Wv device [d, E] value
  *           projection (cfg->dtype; k = W_k e, v = W_v e: the contraction runs
  *           along the contiguous axis).
- *   conv_w  device fp32 [d, 4]: y_t = sum_i conv_w[:, i] * vt_{t-3+i}.
+ *   conv_w  device fp32 [d, 4]: y_t = sum_i conv_w[:, i] * vt_{t-3+i}; with
+ *           variant flags the small-parameter block (engram_param_floats).
  *   conv_state NULL for whole sequences.  Non-NULL selects decode (T == 1):
- *           device fp32 [B, M, 3, d], vt of the three previous steps, oldest
- *           first, zeros at the start; updated in place.
+ *           device fp32 [B, M, 3 dil, d], the conv inputs (vt, or the
+ *           normalised vt with ENGRAM_CONV_PRENORM) of the 3 dil previous
+ *           steps, oldest first, zeros at the start; updated in place.
  *   out     device [B, T, M, d] (cfg->dtype); may be h itself (the residual
  *           applied in place): every read of h precedes the write of the same
  *           element.  engram_backward needs the original h, so a forward that
@@ -206,7 +227,8 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
  * carries one fp32 rounding) and
  *   dout     device fp32 [B, T, M, d].
  * Outputs (device fp32, overwritten):
- *   dh [B, T, M, d], dWk [M, d, E], dWv [d, E], dconv_w [d, 4],
+ *   dh [B, T, M, d], dWk [M, d, E], dWv [d, E], dconv_w [d, 4] (the
+ *   gradient of the whole small-parameter block with variant flags),
  *   de       [B*T, E] or NULL,
  *   dtab_keys int64 [<= B*T*J]: packed-table row ids, ascending, unique,
  *   dtab_rows [<= B*T*J, D_h]: gradient of those rows,
@@ -290,6 +312,13 @@ int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const 
  * The gathered e is identical to engram_forward_hosttable's whatever the
  * cache holds; the cache changes where rows are read from, never what.
  */
+
+/* Floats of the small-parameter block `conv_w` (and of its gradient
+ * `dconv_w`): the conv weights, [d, 4], or [M, d, 4] with
+ * ENGRAM_CONV_PER_BRANCH; then, with ENGRAM_NORM_SCALES, g_h [M, d], g_k
+ * [M, d] and, with ENGRAM_CONV_PRENORM as well, g_v [M, d].  0 for an
+ * invalid configuration. */
+int64_t engram_param_floats(const engram_cfg_t* cfg);
 
 /* Packed-table rows of the configuration: sum of rows[j] over the J heads
  * (the entries of the hostcache map); 0 for an invalid configuration. */

@@ -55,13 +55,24 @@ def test_workspace_sizes_host_only():
     assert eg.engram_saved_size(_cfg(flags=eg.SAVE_KV), 64) == eg.engram_saved_size(c, 64)
 
 
+def test_small_parameter_block_sizes():
+    """conv weights [d, 4] or [M, d, 4], then g_h, g_k (and g_v) of [M, d]."""
+    d, M = 64, 3
+    for flags, want in [(0, 4 * d), (eg.CONV_DILATED | eg.CONV_PRENORM, 4 * d),
+                        (eg.CONV_PER_BRANCH, 4 * d * M), (eg.NORM_SCALES, 4 * d + 2 * M * d),
+                        (eg.NORM_SCALES | eg.CONV_PRENORM | eg.CONV_PER_BRANCH,
+                         4 * d * M + 3 * M * d)]:
+        assert eg.engram_param_floats(_cfg(n_branch=M, flags=flags)) == want, flags
+    assert eg.engram_param_floats(_cfg(flags=64)) == 0  # not a flag: invalid configuration
+
+
 def test_invalid_configurations_rejected_before_any_launch():
     bad = [
         _cfg(K=0),
         _cfg(D_h=6),                     # 24-byte rows: not a multiple of 16 bytes
         _cfg(rows=[1009, 1009, 1008, 1009]),  # even row count
         _cfg(rows=[1009, 1009, 1, 1009]),
-        _cfg(V_c=1001), _cfg(dtype=7), _cfg(flags=2), _cfg(K=3, rows=[1009] * 6,
+        _cfg(V_c=1001), _cfg(dtype=7), _cfg(flags=32), _cfg(K=3, rows=[1009] * 6,
                                             mult=np.ones((6, 3), np.uint64)),  # J % 4 != 0
     ]
     big = _cfg()

@@ -1,0 +1,125 @@
+"""Parity of the formulation variants (conv dilation 3, pre-conv RMSNorm,
+per-branch conv, learnable RMSNorm scales) of the fp32 layer with the
+oracle: forward, decode streaming and every gradient, including the
+small-parameter block's, within the fp32 tolerance (1e-5 max relative
+error with a 1e-3 RMS floor); bf16 layers refuse the variants."""
+import numpy as np
+import pytest
+import torch
+
+from hashed_gram_conditional_engram_b200 import engram as eg
+from hashed_gram_conditional_engram_b200 import synth
+from oracle import engram_oracle as O
+from tests.engram_cases import dev, max_rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-5
+DIL, PRE, BR, SC = eg.CONV_DILATED, eg.CONV_PRENORM, eg.CONV_PER_BRANCH, eg.NORM_SCALES
+FLAG_SETS = [DIL, PRE, BR, SC, PRE | SC, DIL | PRE | BR | SC]
+
+
+def _ws(nbytes):
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device="cuda")
+
+
+def _layer(seed, flags, B=2, T=13, M=2, d=64, K=2, D_h=8):
+    rng = np.random.default_rng(seed)
+    J, E, N = 2 * K, 2 * K * D_h, B * T
+    rows = synth.primes_at_most(101, J)
+    cfg = eg.make_cfg(K, D_h, d, M, 1000, 770, eg.F32, rows, np.ones((J, 3), np.uint64),
+                      flags=flags)
+    n_par = eg.engram_param_floats(cfg)
+    assert n_par == O.param_count(flags, M, d)
+    block = (rng.standard_normal(n_par) * 0.5).astype(np.float32)
+    if flags & SC:
+        n_conv = (M if flags & BR else 1) * d * 4
+        block[n_conv:] = (1.0 + 0.3 * rng.standard_normal(n_par - n_conv)).astype(np.float32)
+    x = dict(
+        e=rng.standard_normal((N, E)).astype(np.float32),
+        h=rng.standard_normal((N, M, d)).astype(np.float32),
+        Wk=(rng.standard_normal((M, d, E)) / np.sqrt(E)).astype(np.float32),
+        Wv=(rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32),
+        block=block,
+        dout=rng.standard_normal((N, M, d)).astype(np.float32),
+        idx=np.stack([rng.integers(0, P, N) for P in rows], -1).astype(np.int32),
+    )
+    return cfg, x, B, T, M, d, E, J, D_h
+
+
+@pytest.mark.parametrize("flags", FLAG_SETS)
+def test_variant_forward_and_backward_match_oracle(flags):
+    cfg, x, B, T, M, d, E, J, D_h = _layer(100 + flags, flags)
+    N = B * T
+    e, h = dev(x["e"]), dev(x["h"])
+    Wk, Wv, block = dev(x["Wk"]), dev(x["Wv"]), dev(x["block"])
+    out = torch.empty((N, M, d), device="cuda")
+    saved = _ws(eg.engram_saved_size(cfg, N))
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+    eg.engram_forward(cfg, None, None, e, h, Wk, Wv, block, None, out, saved, B, T, _ws(fb), fb)
+    ref = O.layer_forward_v(x["e"], x["h"], x["Wk"], x["Wv"], x["block"], T, flags)
+    assert max_rel_err(out.cpu().numpy(), ref["out"]) <= TOL
+    g = dict(dh=torch.empty((N, M, d), device="cuda"), dWk=torch.empty((M, d, E), device="cuda"),
+             dWv=torch.empty((d, E), device="cuda"),
+             dblock=torch.full((block.numel(),), 7.0, device="cuda"),
+             de=torch.empty((N, E), device="cuda"))
+    keys = torch.empty(N * J, dtype=torch.int64, device="cuda")
+    rows_out = torch.empty((N * J, D_h), device="cuda")
+    nu = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bb = eg.engram_workspace_size(cfg, eg.WS_BACKWARD, N)
+    eg.engram_backward(cfg, dev(x["idx"]), e, h, Wk, Wv, block, saved, dev(x["dout"]), g["dh"],
+                       g["dWk"], g["dWv"], g["dblock"], g["de"], keys, rows_out, nu, B, T,
+                       _ws(bb), bb)
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    want = O.layer_backward_v(x["e"], x["h"], x["Wk"], x["Wv"], x["block"], T, x["dout"], flags)
+    for name in ("dh", "dWk", "dWv", "de", "dblock"):
+        err = max_rel_err(g[name].cpu().numpy(), want[name])
+        assert err <= TOL, (name, err)
+
+
+@pytest.mark.parametrize("flags", FLAG_SETS)
+def test_variant_decode_streaming_matches_whole_sequences(flags):
+    cfg, x, B, T, M, d, E, J, D_h = _layer(200 + flags, flags, T=12)
+    dil = 3 if flags & DIL else 1
+    ref = O.layer_forward_v(x["e"], x["h"], x["Wk"], x["Wv"], x["block"], T, flags)
+    eb = x["e"].reshape(B, T, E)
+    hb = x["h"].reshape(B, T, M, d)
+    state = torch.zeros((B, M, 3 * dil, d), device="cuda")
+    Wk, Wv, block = dev(x["Wk"]), dev(x["Wv"]), dev(x["block"])
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, B)
+    ws = _ws(fb)
+    out = torch.empty((B, 1, M, d), device="cuda")
+    got = []
+    for t in range(T):
+        eg.engram_forward(cfg, None, None, dev(np.ascontiguousarray(eb[:, t])),
+                          dev(np.ascontiguousarray(hb[:, t])), Wk, Wv, block, state, out, None,
+                          B, 1, ws, fb)
+        got.append(out[:, 0].cpu().numpy().copy())
+    got = np.stack(got, axis=1).reshape(B * T, M, d)
+    # The state carries the conv inputs between steps in fp32 (the API's state
+    # type): each is rounded once (relative 2^-24), so out differs from the
+    # whole-sequence forward by at most SiLU' (< 1.1) times the conv of those
+    # roundings, plus out's own rounding; twice that is allowed.
+    P = O.unpack_params(x["block"], flags, M, d)
+    conv_abs = O.causal_conv_v(np.abs(ref["c"]), np.abs(P["w"]), T, dil)
+    bound = 2.0 ** -23 * (np.abs(ref["out"]) + 1.1 * conv_abs)
+    assert np.all(np.abs(got - ref["out"]) <= bound), float(np.max(np.abs(got - ref["out"]) - bound))
+    assert eg.engram_get_status() == 0
+
+
+def test_bf16_layers_refuse_the_variants():
+    K, D_h, d = 2, 32, 256
+    rows = synth.primes_at_most(1009, 2 * K)
+    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
+                      flags=eg.CONV_DILATED)
+    N, E = 4, 2 * K * D_h
+    e = torch.zeros((N, E), dtype=torch.bfloat16, device="cuda")
+    h = torch.zeros((N, d), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((d, E), dtype=torch.bfloat16, device="cuda")
+    cw = torch.zeros((d, 4), device="cuda")
+    out = torch.empty_like(h)
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+    with pytest.raises(eg.EngramError) as ex:
+        eg.engram_forward(cfg, None, None, e, h, W, W, cw, None, out, None, 1, N, _ws(fb), fb)
+    assert eg.ERRORS[ex.value.rc] == "ENGRAM_ERR_UNSUPPORTED"
