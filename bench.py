@@ -477,6 +477,8 @@ def run_ours(args):
         if ws_ == 1 and not args.no_extras:
             for name, fn in (("decode", bench_decode), ("hosttable", bench_hosttable),
                              ("fwd_bwd", bench_train_step), ("tiny", bench_tiny),
+                             ("tiny_all_variants",
+                              lambda d_: bench_tiny(d_, flags=30)),  # dilated, prenorm, per-branch, scales
                              ("fwd_bwd_27b", bench_fwd_bwd_27b)):
                 try:
                     extras[name] = fn(dev)
@@ -651,9 +653,11 @@ def _fwd_bwd_27b_run(dev, steps, save_kv):
             "backward_gemm_tflops": bwd_flops / (t_bwd / 1e3) / 1e12}
 
 
-def bench_tiny(dev):
+def bench_tiny(dev, flags=0):
     """One fp32 layer (1 x 64 tokens, d 64, 4 heads x 16 dims): hash, forward
-    with the gather, backward with the sparse table gradient, per call."""
+    with the gather, backward with the sparse table gradient, per call; with
+    `flags`, the formulation variants (their extra parameters: conv weights
+    repeated per branch, norm scales 1 + N(0, 0.1))."""
     import torch
     from hashed_gram_conditional_engram_b200 import engram as eg
     from hashed_gram_conditional_engram_b200 import synth
@@ -666,10 +670,17 @@ def bench_tiny(dev):
     proj = torch.empty(w.V, dtype=torch.int32, device=dev)
     vb = eg.engram_workspace_size(None, eg.WS_VOCAB, w.V)
     V_c = eg.engram_build_vocab_proj(keys, w.V, proj, torch.empty(vb, dtype=torch.uint8, device=dev), vb)
-    cfg = eg.make_cfg(w.K, w.D_h, w.d, w.M, w.V, V_c, eg.F32, w.rows, inp["mult"])
+    cfg = eg.make_cfg(w.K, w.D_h, w.d, w.M, w.V, V_c, eg.F32, w.rows, inp["mult"], flags=flags)
     N, E = w.N, w.E
     ids, table = t(inp["ids"]), t(np.concatenate([x.reshape(-1) for x in inp["tables"]]))
-    h, Wk, Wv, cw, dout = t(inp["h"]), t(inp["Wk"]), t(inp["Wv"]), t(inp["conv_w"]), t(inp["dout"])
+    block = np.asarray(inp["conv_w"], np.float32).reshape(-1)
+    if flags & eg.CONV_PER_BRANCH:
+        block = np.tile(block, w.M)
+    n_par = eg.engram_param_floats(cfg)
+    if n_par > block.size:
+        rng = np.random.default_rng(w.seed + 9)
+        block = np.r_[block, 1.0 + 0.1 * rng.standard_normal(n_par - block.size)].astype(np.float32)
+    h, Wk, Wv, cw, dout = t(inp["h"]), t(inp["Wk"]), t(inp["Wv"]), t(block), t(inp["dout"])
     idx = torch.empty((w.B, w.T, w.J), dtype=torch.int32, device=dev)
     e = torch.empty((N, E), device=dev)
     out = torch.empty((N, w.M, w.d), device=dev)
@@ -680,7 +691,7 @@ def bench_tiny(dev):
     bws = torch.empty(bb, dtype=torch.uint8, device=dev)
     dh = torch.empty((N, w.M, w.d), device=dev)
     dWk, dWv = torch.empty((w.M, w.d, E), device=dev), torch.empty((w.d, E), device=dev)
-    dcw = torch.empty((w.d, 4), device=dev)
+    dcw = torch.empty(n_par, device=dev)
     keys_out = torch.empty(N * w.J, dtype=torch.int64, device=dev)
     rows_out = torch.empty((N * w.J, w.D_h), device=dev)
     nu = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -701,7 +712,7 @@ def bench_tiny(dev):
     if eg.engram_get_status(s) != 0:
         raise RuntimeError("device status word set in the tiny layer")
     return {"workload": "tiny: 1 x 64 tokens, d 64, K 2 x 1,009 x 16, fp32 (fp64 arithmetic), "
-                        "one layer",
+                        "one layer" + (f", variant flags {flags}" if flags else ""),
             "us_per_fwd_call_eager": f_eager * 1e3, "us_per_fwd_bwd_call_eager": fb_eager * 1e3,
             "us_per_fwd_bwd_graph": fb_graph * 1e3,
             "fwd_bwd_tokens_per_s": w.N / (fb_graph / 1e3)}
