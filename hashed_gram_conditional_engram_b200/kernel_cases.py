@@ -12,6 +12,8 @@ without the rest of the layer's inputs on the device.
     python -m hashed_gram_conditional_engram_b200.kernel_cases hostgather \
         --tokens 8192 --seq 2048 --dh 160 --rows 1000003
     python -m hashed_gram_conditional_engram_b200.kernel_cases backward [...]
+    python -m hashed_gram_conditional_engram_b200.kernel_cases hostcache \
+        --tokens 8192 --seq 2048 --dh 160 --rows 1000003 [--cache-rows 1048576]
 
 `fused` runs engram_forward with table = NULL on random gathered rows, i.e.
 the two tensor-core passes; `gather` gathers from a table of --rows rows per
@@ -22,7 +24,10 @@ table and the conv state) for --tokens sequences of one token each;
 fp32 rows of de for hash indices of Zipf(1.1) token ids; `hostgather` runs
 engram_forward_hosttable on a table in pinned host memory; `backward` runs
 the bf16 engram_backward (column walk, row kernel, GEMMs, sparse table
-gradient) on random gathered rows, gates and output gradients.  Defaults are the
+gradient) on random gathered rows, gates and output gradients; `hostcache`
+runs engram_forward_hostcache with an HBM cache of the rows a second sample
+of the same skewed (Zipf 1.2 per head) slot distribution addresses most.
+Defaults are the
 27B-shaped layer's dimensions.  Prints the device time per repetition.
 """
 from __future__ import annotations
@@ -39,7 +44,7 @@ from . import synth
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("kernel", choices=["fused", "gather", "hash", "decode", "tablegrad",
-                                       "hostgather", "backward"])
+                                       "hostgather", "backward", "hostcache"])
     ap.add_argument("--tokens", type=int, default=32768)
     ap.add_argument("--seq", type=int, default=4096)
     ap.add_argument("--d", type=int, default=2560)
@@ -47,6 +52,7 @@ def main(argv=None):
     ap.add_argument("--dh", type=int, default=80)
     ap.add_argument("--rows", type=int, default=4_450_001)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--cache-rows", type=int, default=1 << 20)
     ap.add_argument("--save-kv", action="store_true",
                     help="fused, backward: the forward keeps k and v for the backward")
     a = ap.parse_args(argv)
@@ -136,6 +142,41 @@ def main(argv=None):
 
         def run():
             eg.engram_forward_hosttable(cfg, idx, host.data_ptr(), N, e, side, None)
+    elif a.kernel == "hostcache":
+        n_el = sum(rows) * a.dh
+        host = torch.empty(n_el, dtype=torch.bfloat16, pin_memory=True)
+        buf = torch.empty(1 << 28, dtype=torch.bfloat16, device=dev)
+        for lo in range(0, n_el, 1 << 28):
+            hi = min(n_el, lo + (1 << 28))
+            buf[: hi - lo].normal_(0.0, 0.02, generator=g)
+            host[lo:hi].copy_(buf[: hi - lo])
+        del buf
+        rng = np.random.default_rng(3)
+
+        def skewed(n):
+            return np.stack([(rng.zipf(1.2, n) - 1) % P for P in rows], -1).astype(np.int32)
+
+        idx = torch.from_numpy(skewed(N)).to(dev)
+        sample = torch.from_numpy(skewed(8 * N)).to(dev)
+        C = a.cache_rows
+        rb = eg.engram_workspace_size(cfg, eg.WS_HOSTCACHE_RANK, 8 * N)
+        crow = torch.empty(C, dtype=torch.int64, device=dev)
+        n_out = torch.zeros(1, dtype=torch.int32, device=dev)
+        eg.engram_hostcache_rank(cfg, sample, 8 * N, C, crow, n_out,
+                                 torch.empty(rb, dtype=torch.uint8, device=dev), rb)
+        n_c = int(n_out.item())
+        cache = torch.empty((max(n_c, 1), a.dh), dtype=torch.bfloat16, device=dev)
+        cmap = torch.empty(eg.engram_table_rows(cfg), dtype=torch.int32, device=dev)
+        eg.engram_hostcache_fill(cfg, host.data_ptr(), crow, n_c, cache, cmap)
+        e = torch.empty((N, E), dtype=torch.bfloat16, device=dev)
+        gb = eg.engram_workspace_size(cfg, eg.WS_HOSTCACHE_GATHER, N)
+        gws = torch.empty(gb, dtype=torch.uint8, device=dev)
+        n_miss = torch.zeros(1, dtype=torch.int32, device=dev)
+        side = torch.cuda.current_stream()
+
+        def run():
+            eg.engram_forward_hostcache(cfg, idx, host.data_ptr(), cache, cmap, N, e, n_miss, gws,
+                                        gb, side, None)
     elif a.kernel == "tablegrad":
         ids_np, keys_np = synth.host_ids_keys(synth.workload("layer27b"))
         keys = torch.from_numpy(keys_np).to(dev)
@@ -200,6 +241,9 @@ def main(argv=None):
         ev1.record()
         torch.cuda.synchronize()
         print(f"{a.kernel} rep {r}: {ev0.elapsed_time(ev1) * 1e3:.1f} us")
+    if a.kernel == "hostcache":
+        print(f"hostcache: {n_c} cached rows, {int(n_miss.item())} of {N * a.heads} "
+              "(token, head) rows from host memory")
     st = eg.engram_get_status()
     if st != 0:
         raise SystemExit(f"device status word {st}")
