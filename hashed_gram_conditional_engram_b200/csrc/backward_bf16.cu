@@ -390,12 +390,18 @@ __host__ __device__ constexpr size_t row_stage_bytes(int d) {
 // fixed-order pass, whose barrier also frees the stage for the token after
 // next; then dk (bf16, for the GEMMs) and dh are written.  A copy that never
 // lands sets ENGRAM_STATUS_TIMEOUT and the block stops.
-template <int ITEMS>  // ceil(d / (ROW_THREADS * ROW_VEC)) <= ROW_MAX_ITEMS
+// With learnable norm scales (SCALED) the gate reads <RMSNorm(h) g_h,
+// RMSNorm(k) g_k>: h k is weighted by gg = g_h g_k in the sums and in dk, dh,
+// and each thread adds up, over the block's tokens, c (r_h h)(r_k k) for its
+// features (c = dz / sqrt(d)); the block's sums go to spart[block][f] for
+// the scales' gradients (dg_h = S g_k, dg_k = S g_h).
+template <int ITEMS, bool SCALED>  // ITEMS = ceil(d / (ROW_THREADS * ROW_VEC)) <= ROW_MAX_ITEMS
 __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     const __nv_bfloat16* __restrict__ h, const float* __restrict__ k,
     const float* __restrict__ alpha, const float* __restrict__ dout,
-    const float* __restrict__ dalpha_part, int64_t N, int d, int ld, float* __restrict__ dh,
-    __nv_bfloat16* __restrict__ dk_out, unsigned int* status) {
+    const float* __restrict__ dalpha_part, const float* __restrict__ gscale, int64_t N, int d,
+    int ld, float* __restrict__ dh, __nv_bfloat16* __restrict__ dk_out,
+    float* __restrict__ spart, unsigned int* status) {
   // k and dk rows are ld apart (they share rows with v and dv)
   extern __shared__ __align__(128) unsigned char row_smem[];
   __shared__ uint64_t full[ROW_STAGES];
@@ -428,6 +434,20 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
   __syncthreads();
   const int nv = d / ROW_VEC;
   const float invd = 1.0f / (float)d, isd = rsqrtf((float)d);
+  // SCALED: g_h g_k of the thread's features, and its running sums
+  float4 ggv[SCALED ? ITEMS : 1], sacc[SCALED ? ITEMS : 1];
+  if constexpr (SCALED) {
+#pragma unroll
+    for (int q = 0; q < ITEMS; ++q) {
+      const int c4 = threadIdx.x + q * ROW_THREADS;
+      ggv[q] = sacc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c4 < nv) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(gscale) + c4);
+        const float4 b = __ldg(reinterpret_cast<const float4*>(gscale + d) + c4);
+        ggv[q] = make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+      }
+    }
+  }
   int it = 0;
   for (int64_t t = blockIdx.x; t < N; t += G, ++it) {
     const int st = it % ROW_STAGES;
@@ -458,7 +478,13 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
       const float4 hq = bf16x4_to_f4(hb[q]), kq = kv[q];
       shh = fmaf(hq.x, hq.x, fmaf(hq.y, hq.y, fmaf(hq.z, hq.z, fmaf(hq.w, hq.w, shh))));
       skk = fmaf(kq.x, kq.x, fmaf(kq.y, kq.y, fmaf(kq.z, kq.z, fmaf(kq.w, kq.w, skk))));
-      shk = fmaf(hq.x, kq.x, fmaf(hq.y, kq.y, fmaf(hq.z, kq.z, fmaf(hq.w, kq.w, shk))));
+      if constexpr (SCALED) {
+        const float4 g = ggv[q];
+        shk = fmaf(hq.x * g.x, kq.x,
+                   fmaf(hq.y * g.y, kq.y, fmaf(hq.z * g.z, kq.z, fmaf(hq.w * g.w, kq.w, shk))));
+      } else {
+        shk = fmaf(hq.x, kq.x, fmaf(hq.y, kq.y, fmaf(hq.z, kq.z, fmaf(hq.w, kq.w, shk))));
+      }
     }
     float sgv = 0.f;
     if (threadIdx.x < 32)
@@ -497,22 +523,41 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     for (int q = 0; q < ITEMS; ++q) {
       const int c4 = threadIdx.x + q * ROW_THREADS;
       if (c4 < nv) {
-        const float4 hq = bf16x4_to_f4(hb[q]), kq = kv[q], uq = uv[q];
-        const __nv_bfloat162 k01 = __floats2bfloat162_rn(rk * (crh * hq.x) - ck * kq.x,
-                                                        rk * (crh * hq.y) - ck * kq.y);
-        const __nv_bfloat162 k23 = __floats2bfloat162_rn(rk * (crh * hq.z) - ck * kq.z,
-                                                        rk * (crh * hq.w) - ck * kq.w);
+        const float4 hq = bf16x4_to_f4(hb[q]), kq0 = kv[q], uq = uv[q];
+        float4 hg = hq, kg = kq0;  // h, k weighted by g_h g_k where they cross
+        if constexpr (SCALED) {
+          const float4 g = ggv[q];
+          hg = make_float4(hq.x * g.x, hq.y * g.y, hq.z * g.z, hq.w * g.w);
+          kg = make_float4(kq0.x * g.x, kq0.y * g.y, kq0.z * g.z, kq0.w * g.w);
+          const float cr = c * rh * rk;
+          sacc[q].x = fmaf(cr * hq.x, kq0.x, sacc[q].x);
+          sacc[q].y = fmaf(cr * hq.y, kq0.y, sacc[q].y);
+          sacc[q].z = fmaf(cr * hq.z, kq0.z, sacc[q].z);
+          sacc[q].w = fmaf(cr * hq.w, kq0.w, sacc[q].w);
+        }
+        const float4 kq = kq0;
+        const __nv_bfloat162 k01 = __floats2bfloat162_rn(rk * (crh * hg.x) - ck * kq.x,
+                                                        rk * (crh * hg.y) - ck * kq.y);
+        const __nv_bfloat162 k23 = __floats2bfloat162_rn(rk * (crh * hg.z) - ck * kq.z,
+                                                        rk * (crh * hg.w) - ck * kq.w);
         uint2 pk;
         pk.x = *reinterpret_cast<const uint32_t*>(&k01);
         pk.y = *reinterpret_cast<const uint32_t*>(&k23);
         *reinterpret_cast<uint2*>(dkr + c4 * ROW_VEC) = pk;
         float4 o;
-        o.x = uq.x + rh * (crk * kq.x) - ch * hq.x;
-        o.y = uq.y + rh * (crk * kq.y) - ch * hq.y;
-        o.z = uq.z + rh * (crk * kq.z) - ch * hq.z;
-        o.w = uq.w + rh * (crk * kq.w) - ch * hq.w;
+        o.x = uq.x + rh * (crk * kg.x) - ch * hq.x;
+        o.y = uq.y + rh * (crk * kg.y) - ch * hq.y;
+        o.z = uq.z + rh * (crk * kg.z) - ch * hq.z;
+        o.w = uq.w + rh * (crk * kg.w) - ch * hq.w;
         __stcs(reinterpret_cast<float4*>(dhr + c4 * ROW_VEC), o);
       }
+    }
+  }
+  if constexpr (SCALED) {
+#pragma unroll
+    for (int q = 0; q < ITEMS; ++q) {
+      const int c4 = threadIdx.x + q * ROW_THREADS;
+      if (c4 < nv) reinterpret_cast<float4*>(spart + (int64_t)blockIdx.x * d)[c4] = sacc[q];
     }
   }
   // on a timeout, let copies still in flight land (bounded) before the
@@ -526,6 +571,20 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
       row_wait(&full[st], (uint32_t)use & 1u);
     }
   }
+}
+
+// dg_h[f] = S[f] g_k[f], dg_k[f] = S[f] g_h[f], S[f] = the row blocks' sums
+// added in block order
+__global__ void bw_scale_reduce_kernel(const float* __restrict__ spart, int blocks, int d,
+                                       const float* __restrict__ gscale,
+                                       float* __restrict__ dgscale) {
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f >= d) return;
+  float S = 0.f;
+#pragma unroll 8
+  for (int b = 0; b < blocks; ++b) S += spart[(int64_t)b * d + f];
+  dgscale[f] = S * gscale[d + f];      // d/dg_h
+  dgscale[d + f] = S * gscale[f];      // d/dg_k
 }
 
 constexpr int DCONV_WARPS = 32;
@@ -579,6 +638,7 @@ struct BwdBf16Ws {
   float* dWkv;          // [2d, E], copied out to dWk and dWv
   float *dalpha_part, *de;  // [N, d/64] partials of <dvt, v>
   float4* part;
+  float* spart;  // with norm scales: [kMaxRowBlocks][d] sums of the row blocks
   void* blas_ws;
   void* tg_ws;
   size_t tg_bytes;
@@ -586,7 +646,10 @@ struct BwdBf16Ws {
 
 constexpr size_t up256b(size_t b) { return (b + 255) & ~(size_t)255; }
 
-size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved, BwdBf16Ws* w) {
+constexpr int kMaxRowBlocks = 1024;  // row-kernel blocks when the scales' sums are kept
+
+size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved, bool scaled,
+                       BwdBf16Ws* w) {
   const int64_t chunks = (N + COL_TOK - 1) / COL_TOK;
   const size_t KV = kv_saved ? 0 : up256b((size_t)N * 2 * d * 4);
   const size_t DKV = up256b((size_t)N * 2 * d * 2);
@@ -594,10 +657,11 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
   const size_t DA = up256b((size_t)N * (d / COL_FEAT) * 4);
   const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
   const size_t tg = table_grad_ws_bytes(N * J);
-  size_t off[9];
-  const size_t sz[9] = {KV, DKV, WKV, DW, DA, NE4, P, kBlasWorkspace, tg};
+  const size_t SP = scaled ? up256b((size_t)kMaxRowBlocks * d * 4) : 0;
+  size_t off[10];
+  const size_t sz[10] = {KV, DKV, WKV, DW, DA, NE4, P, kBlasWorkspace, tg, SP};
   size_t o = 0;
-  for (int i = 0; i < 9; ++i) {
+  for (int i = 0; i < 10; ++i) {
     off[i] = o;
     o += sz[i];
   }
@@ -613,31 +677,35 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
     w->blas_ws = p + off[7];
     w->tg_ws = p + off[8];
     w->tg_bytes = tg;
+    w->spart = scaled ? reinterpret_cast<float*>(p + off[9]) : nullptr;
   }
   return o;
 }
 
 }  // namespace
 
-size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved) {
-  return bwd_bf16_layout(nullptr, N, d, E, J, kv_saved, nullptr);
+size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved, bool scaled) {
+  return bwd_bf16_layout(nullptr, N, d, E, J, kv_saved, scaled, nullptr);
 }
 
 int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bfloat16* e,
                          const __nv_bfloat16* h, const __nv_bfloat16* Wk,
-                         const __nv_bfloat16* Wv, const float* conv_w, const float* alpha,
-                         const float* kv_saved, const float* dout, float* dh, float* dWk,
+                         const __nv_bfloat16* Wv, const float* conv_w, const float* gscale,
+                         const float* alpha, const float* kv_saved, const float* dout, float* dh,
+                         float* dWk,
                          float* dWv, float* dconv_w, float* de, int64_t* dtab_keys,
                          float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, void* ws,
                          size_t ws_bytes, cudaStream_t s) {
   const int E = hp.E;
   const bool have_kv = kv_saved != nullptr;
-  if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J, have_kv)) return ENGRAM_ERR_WORKSPACE;
+  const bool scaled = gscale != nullptr;
+  if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J, have_kv, scaled))
+    return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
   // a row in registers; whole column blocks; 16-byte multiples for the row copies
   if (d > ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS || d % 256 != 0) return ENGRAM_ERR_UNSUPPORTED;
   BwdBf16Ws w;
-  bwd_bf16_layout(ws, N, d, E, hp.J, have_kv, &w);
+  bwd_bf16_layout(ws, N, d, E, hp.J, have_kv, scaled, &w);
   if (de == nullptr) de = w.de;
   cublasHandle_t hd;
   int rc = blas_handle(s, w.blas_ws, &hd);
@@ -662,9 +730,12 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
                                           w.dalpha_part, w.part);
   {
     const int items = (d / ROW_VEC + ROW_THREADS - 1) / ROW_THREADS;
-    auto row = items == 1 ? bw_row_kernel<1>
-             : items == 2 ? bw_row_kernel<2>
-             : items == 3 ? bw_row_kernel<3> : bw_row_kernel<4>;
+    auto row = scaled ? (items == 1 ? bw_row_kernel<1, true>
+                         : items == 2 ? bw_row_kernel<2, true>
+                         : items == 3 ? bw_row_kernel<3, true> : bw_row_kernel<4, true>)
+                      : (items == 1 ? bw_row_kernel<1, false>
+                         : items == 2 ? bw_row_kernel<2, false>
+                         : items == 3 ? bw_row_kernel<3, false> : bw_row_kernel<4, false>);
     const int smem = (int)(ROW_STAGES * row_stage_bytes(d));
     int dev = 0, sms = 0, per_sm = 0;
     if ((rc = ck(cudaFuncSetAttribute(row, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) ||
@@ -672,9 +743,13 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
         (rc = ck(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))) ||
         (rc = ck(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, row, ROW_THREADS, smem))))
       return rc;
-    const int64_t grid = std::min<int64_t>(N, (int64_t)sms * std::max(per_sm, 1));
-    row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, kv, alpha, dout, w.dalpha_part, N, d,
-                                                  2 * d, dh, w.dkv, status_ptr());
+    int64_t grid = std::min<int64_t>(N, (int64_t)sms * std::max(per_sm, 1));
+    if (scaled) grid = std::min<int64_t>(grid, kMaxRowBlocks);
+    row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, kv, alpha, dout, w.dalpha_part, gscale, N, d,
+                                                  2 * d, dh, w.dkv, w.spart, status_ptr());
+    if (scaled)
+      bw_scale_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(
+          w.spart, (int)grid, d, gscale, dconv_w + 4 * (int64_t)d);
   }
   bw_dconv_reduce_kernel<<<(unsigned)((d + 31) / 32), 32 * DCONV_WARPS, 0, s>>>(
       w.part, chunks, d, reinterpret_cast<float4*>(dconv_w));

@@ -36,6 +36,16 @@ int check_cfg(const engram_cfg_t* c) {
 
 inline int elem_bytes(const engram_cfg_t* c) { return c->dtype == ENGRAM_F32 ? 4 : 2; }
 
+// variants the bf16 path implements: learnable norm scales, and per-branch
+// conv weights (with one branch, the same as shared ones)
+constexpr int kBf16Variants = ENGRAM_NORM_SCALES | ENGRAM_CONV_PER_BRANCH;
+inline bool bf16_variant_ok(const engram_cfg_t* c) {
+  return (c->flags & ENGRAM_VARIANT_FLAGS & ~kBf16Variants) == 0;
+}
+inline bool bf16_scaled(const engram_cfg_t* c) {
+  return c->dtype == ENGRAM_BF16 && (c->flags & ENGRAM_NORM_SCALES) != 0;
+}
+
 // bf16 layers with ENGRAM_SAVE_KV keep k and v after alpha in `saved`
 inline bool saves_kv(const engram_cfg_t* c) {
   return c->dtype == ENGRAM_BF16 && (c->flags & ENGRAM_SAVE_KV) != 0;
@@ -110,10 +120,11 @@ size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n) {
   switch (call) {
     case ENGRAM_WS_FORWARD:
       if (cfg->dtype == ENGRAM_F32) return f32_forward_ws_bytes(n, M, d);
-      return tc_forward_ws_bytes(n, d, E);
+      // with norm scales, their product g_h g_k after the passes' buffers
+      return tc_forward_ws_bytes(n, d, E) + (bf16_scaled(cfg) ? ((size_t)d * 4 + 255) & ~(size_t)255 : 0);
     case ENGRAM_WS_BACKWARD:
       if (cfg->dtype == ENGRAM_BF16)
-        return backward_bf16_ws_bytes(n, d, E, 2 * cfg->K, saves_kv(cfg));
+        return backward_bf16_ws_bytes(n, d, E, 2 * cfg->K, saves_kv(cfg), bf16_scaled(cfg));
       return backward_f32_ws_bytes(n, M, d, E) + table_grad_ws_bytes(n * 2 * cfg->K);
     case ENGRAM_WS_TABLE_GRAD:
       return table_grad_ws_bytes(n * 2 * cfg->K);
@@ -192,8 +203,7 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
   cudaStream_t s = (cudaStream_t)stream;
   const HeadParams hp = make_head_params(cfg);
   const int M = cfg->n_branch, d = cfg->d_model, E = hp.E;
-  if (cfg->dtype == ENGRAM_BF16 &&
-      (!tc_supported(d, E, M) || (cfg->flags & ENGRAM_VARIANT_FLAGS) != 0))
+  if (cfg->dtype == ENGRAM_BF16 && (!tc_supported(d, E, M) || !bf16_variant_ok(cfg)))
     return ENGRAM_ERR_UNSUPPORTED;
   if (table != nullptr) {
     rc = launch_gather(hp, idx, table, N, elem_bytes(cfg), e, s);
@@ -208,10 +218,15 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
                        ? reinterpret_cast<float*>(reinterpret_cast<char*>(saved) +
                                                   alpha_bytes_padded(N))
                        : nullptr;
+  float* gg = nullptr;  // g_h g_k, after the passes' workspace
+  if (bf16_scaled(cfg)) {
+    gg = reinterpret_cast<float*>(static_cast<char*>(ws) + tc_forward_ws_bytes(N, d, E));
+    if ((rc = launch_scale_product(conv_w + 4 * d, conv_w + 5 * d, d, gg, s))) return rc;
+  }
   return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
                            static_cast<const __nv_bfloat16*>(Wk),
                            static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
-                           static_cast<__nv_bfloat16*>(out), saved, kv_save, N, T, d, E, ws,
+                           static_cast<__nv_bfloat16*>(out), saved, kv_save, gg, N, T, d, E, ws,
                            ws_bytes, table != nullptr, s);
 }
 
@@ -222,11 +237,9 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                     void* ws, size_t ws_bytes, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (cfg->dtype == ENGRAM_BF16 &&
-      (cfg->n_branch != 1 || saved == nullptr || (cfg->flags & ENGRAM_VARIANT_FLAGS) != 0))
-    return saved == nullptr && cfg->n_branch == 1 && (cfg->flags & ENGRAM_VARIANT_FLAGS) == 0
-               ? ENGRAM_ERR_INVALID_ARG
-               : ENGRAM_ERR_UNSUPPORTED;
+  if (cfg->dtype == ENGRAM_BF16 && (cfg->n_branch != 1 || !bf16_variant_ok(cfg)))
+    return ENGRAM_ERR_UNSUPPORTED;
+  if (cfg->dtype == ENGRAM_BF16 && saved == nullptr) return ENGRAM_ERR_INVALID_ARG;
   if (B < 0 || T < 0) return ENGRAM_ERR_INVALID_ARG;
   const int64_t N = (int64_t)B * T;
   if (idx == nullptr || e == nullptr || h == nullptr || Wk == nullptr || Wv == nullptr ||
@@ -248,7 +261,8 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
     if (N == 0) {  // no tokens: zero weight gradients, no rows
       if ((rc = ck(cudaMemsetAsync(dWk, 0, (size_t)d * E * 4, s)))) return rc;
       if ((rc = ck(cudaMemsetAsync(dWv, 0, (size_t)d * E * 4, s)))) return rc;
-      if ((rc = ck(cudaMemsetAsync(dconv_w, 0, (size_t)d * 16, s)))) return rc;
+      if ((rc = ck(cudaMemsetAsync(dconv_w, 0, (size_t)engram_param_floats(cfg) * 4, s))))
+        return rc;
       return ck(cudaMemsetAsync(n_unique, 0, sizeof(int32_t), s));
     }
     using bf = __nv_bfloat16;
@@ -258,8 +272,9 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                       : nullptr;
     return launch_backward_bf16(hp, idx, static_cast<const bf*>(e), static_cast<const bf*>(h),
                                 static_cast<const bf*>(Wk), static_cast<const bf*>(Wv), conv_w,
-                                saved, kv_saved, dout, dh, dWk, dWv, dconv_w, de, dtab_keys,
-                                dtab_rows, n_unique, N, T, d, ws, ws_bytes, s);
+                                bf16_scaled(cfg) ? conv_w + 4 * d : nullptr, saved, kv_saved,
+                                dout, dh, dWk, dWv, dconv_w, de, dtab_keys, dtab_rows, n_unique,
+                                N, T, d, ws, ws_bytes, s);
   }
   const size_t bw = backward_f32_ws_bytes(N, M, d, E);
   // de lives in the dense-backward workspace unless the caller wants it
@@ -334,7 +349,8 @@ int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const 
 
 int64_t engram_param_floats(const engram_cfg_t* cfg) {
   if (check_cfg(cfg) != ENGRAM_OK) return 0;
-  if (cfg->dtype == ENGRAM_BF16) return (int64_t)cfg->d_model * 4;
+  if (cfg->dtype == ENGRAM_BF16)
+    return (int64_t)cfg->d_model * ((cfg->flags & ENGRAM_NORM_SCALES) ? 6 : 4);
   return f32_param_floats(cfg->flags, cfg->n_branch, cfg->d_model);
 }
 

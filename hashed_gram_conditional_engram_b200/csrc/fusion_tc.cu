@@ -52,7 +52,8 @@ constexpr unsigned FULL = 0xffffffffu;
 
 // pass K; pass V over whole sequences (conv history from the rows above);
 // pass V in decode (one token per sequence, conv history from the state)
-enum { MODE_GATE_PARTIAL = 0, MODE_VALUE_CONV = 1, MODE_VALUE_DECODE = 2 };
+// pass K (MODE_GATE_SCALED: with learnable norm scales) and pass V
+enum { MODE_GATE_PARTIAL = 0, MODE_VALUE_CONV = 1, MODE_VALUE_DECODE = 2, MODE_GATE_SCALED = 3 };
 
 struct TcArgs {
   int num_m_tiles, num_n_tiles, num_k_tiles;
@@ -69,6 +70,7 @@ struct TcArgs {
   float* alpha_out;     // pass V: optional copy of alpha for the caller
   const float* alpha;   // pass V: gate of every token, from the gate kernel
   float* kv_save;       // optional fp32 [N, 2d]: k (pass K) then v (pass V) of each token
+  const float* gg;      // optional [d]: g_h * g_k, the learnable norm scales' product (pass K)
   unsigned int* status;
 };
 
@@ -415,7 +417,7 @@ __device__ __forceinline__ void conv_group16(const uint32_t (&u)[16], const floa
 
 template <int BN, int STAGES, int MODE, int KCH>
 struct TcShape {
-  static constexpr bool VPASS = MODE != MODE_GATE_PARTIAL;
+  static constexpr bool VPASS = MODE == MODE_VALUE_CONV || MODE == MODE_VALUE_DECODE;
   // epilogue warps: 2 per TMEM lane quadrant
   static constexpr int EPI = 8;
   static constexpr int PARTS = EPI / 4;        // column parts of a tile, one per warp of a quadrant
@@ -812,11 +814,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
               unpack_bf16x32(h0, hv);
             else
               load_bf16x32(args.h + n * args.d + col_base + c * 32, hv);
+            if constexpr (MODE == MODE_GATE_SCALED) {
+              // <RMSNorm(h) g_h, RMSNorm(k) g_k>: weight h k by g_h g_k
+              const float4* gq = reinterpret_cast<const float4*>(args.gg + col_base + c * 32);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              kk = fmaf(v[i], v[i], kk);
-              hk = fmaf(hv[i], v[i], hk);
-              hh = fmaf(hv[i], hv[i], hh);
+              for (int q = 0; q < 8; ++q) {
+                const float4 g4 = __ldg(gq + q);
+                const float gw[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                  const int i = 4 * q + r;
+                  kk = fmaf(v[i], v[i], kk);
+                  hk = fmaf(hv[i] * gw[r], v[i], hk);
+                  hh = fmaf(hv[i], hv[i], hh);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                kk = fmaf(v[i], v[i], kk);
+                hk = fmaf(hv[i], v[i], hk);
+                hh = fmaf(hv[i], hv[i], hh);
+              }
             }
           }
         }
@@ -1185,8 +1204,8 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
 template <int BN, int STAGES_K, int STAGES_V, int KCH>
 int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
-              float* alpha_saved, float* kv_save, int64_t N, int T, int d, int E, float4* part,
-              float* alpha, bool chained, cudaStream_t s) {
+              float* alpha_saved, float* kv_save, const float* gg, int64_t N, int T, int d, int E,
+              float4* part, float* alpha, bool chained, cudaStream_t s) {
   // Each CTA of a pair loads 128 rows of A and BN/2 rows of B per stage.
   // pass K: A = e (256 tokens per pair tile), B = W_k (BN features)
   CUtensorMap ta_k, tb_k, ta_v, tb_v, th, to, to29;
@@ -1217,6 +1236,7 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.alpha_out = alpha_saved;
   a.alpha = nullptr;
   a.kv_save = conv_state == nullptr ? kv_save : nullptr;
+  a.gg = gg;
   a.status = status_ptr();
   // pass K: gate partials, pair tiles of 256 tokens x BN features
   a.num_n_tiles = d / BN;
@@ -1232,8 +1252,11 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
       !make_tmap_f32(&tkv, a.kv_save, (uint64_t)(2 * d), (uint64_t)N, 32, 32,
                      CU_TENSOR_MAP_SWIZZLE_128B))
     return ENGRAM_ERR_CUDA;
-  int rc = launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL, KCH>(ta_k, tb_k, th, tkv, to29, a, s,
-                                                             chained);
+  int rc = gg != nullptr
+               ? launch_pass<BN, STAGES_K, MODE_GATE_SCALED, KCH>(ta_k, tb_k, th, tkv, to29, a, s,
+                                                                  chained)
+               : launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL, KCH>(ta_k, tb_k, th, tkv, to29, a, s,
+                                                                   chained);
   if (rc) return rc;
   {
     int dev = 0, sms = 148;
@@ -1270,6 +1293,19 @@ inline bool use_wide(int64_t N, int d) { return d % 256 == 0 && N > 4096; }
 
 }  // namespace
 
+namespace {
+__global__ void scale_product_kernel(const float* __restrict__ gh, const float* __restrict__ gk,
+                                     int d, float* __restrict__ gg) {
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f < d) gg[f] = gh[f] * gk[f];
+}
+}  // namespace
+
+int launch_scale_product(const float* gh, const float* gk, int d, float* gg, cudaStream_t s) {
+  scale_product_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(gh, gk, d, gg);
+  return ck(cudaGetLastError());
+}
+
 int tc_supported(int d, int E, int M) {
   return M == 1 && E % BK == 0 && E >= BK && d % (2 * BM) == 0 && d >= 2 * BM;
 }
@@ -1283,8 +1319,9 @@ size_t tc_forward_ws_bytes(int64_t N, int d, int E) {
 
 int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
-                      __nv_bfloat16* out, float* alpha_saved, float* kv_save, int64_t N, int T,
-                      int d, int E, void* ws, size_t ws_bytes, bool chained, cudaStream_t s) {
+                      __nv_bfloat16* out, float* alpha_saved, float* kv_save, const float* gg,
+                      int64_t N, int T, int d, int E, void* ws, size_t ws_bytes, bool chained,
+                      cudaStream_t s) {
   if (ws_bytes < tc_forward_ws_bytes(N, d, E) || ws == nullptr) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL - 256) return ENGRAM_ERR_UNSUPPORTED;
   const bool wide = use_wide(N, d);
@@ -1293,15 +1330,15 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
   float* alpha = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                           (size_t)N * 2 * (d / BN) * sizeof(float4));
   if (wide)
-    return run_layer<256, 6, 5, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, N,
-                                   T, d, E, part, alpha, chained, s);
+    return run_layer<256, 6, 5, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
+                                   gg, N, T, d, E, part, alpha, chained, s);
   // few tokens: each CTA streams long operand rows at a rate set by how many
   // bytes one copy instruction brings, so two K chunks go in each box
   if (E % (2 * BK) == 0)
-    return run_layer<64, 4, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, N,
-                                  T, d, E, part, alpha, chained, s);
-  return run_layer<64, 8, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, N, T,
-                                d, E, part, alpha, chained, s);
+    return run_layer<64, 4, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
+                                  gg, N, T, d, E, part, alpha, chained, s);
+  return run_layer<64, 8, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, gg,
+                                N, T, d, E, part, alpha, chained, s);
 }
 
 }  // namespace engram

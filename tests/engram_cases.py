@@ -90,7 +90,10 @@ class Layer:
             dh=torch.empty((N, M, d), dtype=torch.float32, device="cuda"),
             dWk=torch.empty((M, d, E), dtype=torch.float32, device="cuda"),
             dWv=torch.empty((d, E), dtype=torch.float32, device="cuda"),
-            dconv_w=torch.empty((d, 4), dtype=torch.float32, device="cuda"),
+            # the small-parameter block's gradient: conv weights [d, 4], then
+            # any learnable norm scales'
+            dconv_w=torch.empty(eg.engram_param_floats(cfg), dtype=torch.float32,
+                                device="cuda"),
             de=torch.empty((N, E), dtype=torch.float32, device="cuda"),
             keys=torch.empty(max(N * cfg.J, 1), dtype=torch.int64, device="cuda"),
             rows=torch.empty((max(N * cfg.J, 1), cfg.D_h), dtype=torch.float32, device="cuda"),

@@ -195,8 +195,11 @@ def _bf16_backward_case(B, T, d, K, D_h, seed, flags=0, with_layer=False):
     idx = np.stack([rng.integers(0, P, N) for P in rows], -1).astype(np.int32)
     cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((J, 3), np.uint64),
                       flags=flags)
+    block = conv_w.reshape(-1)
+    if flags & eg.NORM_SCALES:  # learnable g_h, g_k after the conv weights
+        block = np.r_[block, 1.0 + 0.3 * rng.standard_normal(2 * d)].astype(np.float32)
     L = Layer(cfg, B, T, packed_table(tables, "bf16"), bf16_dev(h), bf16_dev(Wk), bf16_dev(Wv),
-              dev(conv_w), torch.bfloat16)
+              dev(block), torch.bfloat16)
     idx_d = dev(idx.reshape(B, T, J))
     L.forward(idx_d)
     g = L.backward(idx_d, dev(dout))
@@ -205,9 +208,15 @@ def _bf16_backward_case(B, T, d, K, D_h, seed, flags=0, with_layer=False):
     f64 = O.bf16_bits_to_f64
     e_ref = f64(O.gather(idx, [synth.to_bf16_bits(t) for t in tables]))
     assert np.array_equal(bf16_bits(L.e), O.gather(idx, [synth.to_bf16_bits(t) for t in tables]))
-    ref = O.layer_backward(e_ref, f64(synth.to_bf16_bits(h)).reshape(N, 1, d),
-                           f64(synth.to_bf16_bits(Wk)), f64(synth.to_bf16_bits(Wv)), conv_w, T,
-                           dout)
+    if flags & eg.NORM_SCALES:
+        ref = O.layer_backward_v(e_ref, f64(synth.to_bf16_bits(h)).reshape(N, 1, d),
+                                 f64(synth.to_bf16_bits(Wk)), f64(synth.to_bf16_bits(Wv)), block,
+                                 T, dout, O.NORM_SCALES)
+        ref["dconv_w"] = ref["dblock"]
+    else:
+        ref = O.layer_backward(e_ref, f64(synth.to_bf16_bits(h)).reshape(N, 1, d),
+                               f64(synth.to_bf16_bits(Wk)), f64(synth.to_bf16_bits(Wv)), conv_w,
+                               T, dout)
     ref["e"] = e_ref
     ref["Wk_bf"] = f64(synth.to_bf16_bits(Wk))
     ref["Wv_bf"] = f64(synth.to_bf16_bits(Wv))
@@ -253,6 +262,19 @@ def test_backward_bf16_saved_kv_matches_oracle(B, T, d, K, D_h):
     hold."""
     _check_bf16_backward(*_bf16_backward_case(B, T, d, K, D_h, seed=B * 17 + T,
                                               flags=eg.SAVE_KV))
+
+
+@pytest.mark.parametrize("B,T,d,flags", [
+    (3, 100, 256, eg.NORM_SCALES),                 # narrow forward tiles
+    (2, 2500, 512, eg.NORM_SCALES),                # wide forward tiles
+    (2, 700, 256, eg.NORM_SCALES | eg.SAVE_KV),    # with k and v kept by the forward
+])
+def test_backward_bf16_norm_scales_match_oracle(B, T, d, flags):
+    """Learnable RMSNorm scales on a bf16 layer: the gate weights h k by
+    g_h g_k in the forward's pass K and in the backward's row kernel; the
+    scales' gradients (after the conv weights' in dconv_w) are held with dh
+    to the bf16 metric."""
+    _check_bf16_backward(*_bf16_backward_case(B, T, d, 2, 32, seed=B * 7 + T, flags=flags))
 
 
 def _check_bf16_backward(g, ref, idx, rows, D_h):

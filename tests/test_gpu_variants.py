@@ -123,3 +123,36 @@ def test_bf16_layers_refuse_the_variants():
     with pytest.raises(eg.EngramError) as ex:
         eg.engram_forward(cfg, None, None, e, h, W, W, cw, None, out, None, 1, N, _ws(fb), fb)
     assert eg.ERRORS[ex.value.rc] == "ENGRAM_ERR_UNSUPPORTED"
+
+
+@pytest.mark.parametrize("N,T", [(300, 100), (5000, 2500)])
+def test_bf16_norm_scales_forward_matches_oracle(N, T):
+    """bf16 layer with learnable RMSNorm scales: out within the bf16 metric
+    of the oracle's fp64 forward on the same bf16 values, alpha to 1e-5."""
+    from tests.engram_cases import bf16_dev
+    rng = np.random.default_rng(N)
+    K, D_h, d = 2, 32, 256
+    E = 2 * K * D_h
+    rows = synth.primes_at_most(1009, 2 * K)
+    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
+                      flags=eg.NORM_SCALES)
+    e = rng.standard_normal((N, E)).astype(np.float32)
+    h = rng.standard_normal((N, 1, d)).astype(np.float32)
+    Wk = (rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32)
+    Wv = (rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32)
+    block = np.r_[(rng.standard_normal(4 * d) * 0.5), 1.0 + 0.3 * rng.standard_normal(2 * d)]
+    block = block.astype(np.float32)
+    assert eg.engram_param_floats(cfg) == block.size
+    out = torch.empty((N, 1, d), dtype=torch.bfloat16, device="cuda")
+    saved = _ws(eg.engram_saved_size(cfg, N))
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+    eg.engram_forward(cfg, None, None, bf16_dev(e), bf16_dev(h), bf16_dev(Wk), bf16_dev(Wv),
+                      dev(block), None, out, saved, N // T, T, _ws(fb), fb)
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    f64 = O.bf16_bits_to_f64
+    b = synth.to_bf16_bits
+    ref = O.layer_forward_v(f64(b(e)), f64(b(h)), f64(b(Wk)), f64(b(Wv)), block, T, eg.NORM_SCALES)
+    assert max_rel_err(out.float().cpu().numpy(), ref["out"]) <= 2e-2
+    alpha = saved[: N * 4].view(torch.float32).cpu().numpy()
+    assert np.max(np.abs(alpha - ref["alpha"].reshape(-1))) <= 1e-5
