@@ -15,14 +15,6 @@ namespace {
 
 constexpr float RMS_EPS = 1e-6f;
 
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
-}
-
-__device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
-
 // The formulation variants of the layer's flags, and where their parameters
 // sit in the small-parameter block: conv weights ([M or 1][d][4]), then with
 // ENGRAM_NORM_SCALES g_h [M][d], g_k [M][d] and, with ENGRAM_CONV_PRENORM,

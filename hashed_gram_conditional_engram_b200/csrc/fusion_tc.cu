@@ -217,10 +217,6 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }
 
-__device__ __forceinline__ void prefetch_l1(const void* p) {
-  asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
-}
-
 // 16 consecutive fp32 columns of this thread's TMEM lane, without waiting:
 // the registers are valid only after tmem_wait16 on the same array.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&u)[16]) {
@@ -266,19 +262,10 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // TMA load into this CTA's shared memory whose completion is counted on the
-// pair's leader barrier (cluster address); no multicast.
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
-                                                 uint32_t bar_cluster, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-// The same through a 3-D map {64-element K chunk, row, chunk index}: one
-// instruction brings several 128-byte K chunks of a row block (a box per
-// chunk would cost one issue each).
+// pair's leader barrier (cluster address), no multicast, through a 3-D map
+// {64-element K chunk, row, chunk index}: one instruction brings several
+// 128-byte K chunks of a row block (a box per chunk would cost one issue
+// each).
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map,
                                                  uint32_t bar_cluster, int c0, int c1, int c2) {
   asm volatile(
@@ -364,11 +351,6 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, float (&x)[
       x[v * 8 + 2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
     }
   }
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&b);
 }
 
 // Pass V, 16 consecutive tokens of one feature: vt = alpha * v, the width-4
