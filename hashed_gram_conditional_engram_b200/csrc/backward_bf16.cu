@@ -118,22 +118,46 @@ __device__ __forceinline__ float2 silu_grad2(float2 y) {
 }
 
 constexpr int COL_TOK = 128;   // tokens per column chunk; one warp walks one chunk
-constexpr int COL_FPT = 2;     // features per lane (float2 loads)
-constexpr int COL_FEAT = 32 * COL_FPT;  // features per warp, one dalpha partial per token
+constexpr int COL_NP = 2;      // feature pairs per lane (2 pairs: one 16-byte load per row)
+constexpr int COL_FEAT = 64 * COL_NP;  // features per warp, one dalpha partial per token
 constexpr int COL_WARPS = 4;   // chunks per block
 
-constexpr int COL_RING = 16;  // tokens per warp in a shared-memory ring, 15 of them in flight
+constexpr int COL_RING = 12;  // tokens per warp in a shared-memory ring, 11 of them in flight
 
-__device__ __forceinline__ float2 ld_f2(const float* p) {
-  return *reinterpret_cast<const float2*>(p);
+// dalpha partials per token, padded to 16 bytes for the row kernel's copies
+__host__ __device__ constexpr int col_partials(int d) { return ((d / COL_FEAT) + 3) & ~3; }
+
+// A lane's features: COL_NP pairs of adjacent ones.
+struct FPairs {
+  float2 p[COL_NP];
+};
+
+__device__ __forceinline__ FPairs ld_pairs(const float* q) {
+  FPairs r;
+  if constexpr (COL_NP == 2) {
+    const float4 t = *reinterpret_cast<const float4*>(q);
+    r.p[0] = make_float2(t.x, t.y);
+    r.p[COL_NP - 1] = make_float2(t.z, t.w);
+  } else {
+    r.p[0] = *reinterpret_cast<const float2*>(q);
+  }
+  return r;
 }
 
-// 8-byte asynchronous copy global -> shared (this thread's own slot).
-__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
-                   (uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src)
-               : "memory");
+// Asynchronous copy of a lane's features (8 * COL_NP bytes), global -> its
+// own shared-memory slot.
+__device__ __forceinline__ void cp_async_pairs(void* dst, const void* src) {
+  if constexpr (COL_NP == 2) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+  } else {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+  }
 }
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
@@ -165,44 +189,59 @@ __device__ __forceinline__ void col_flush(ColPartials& pb, int jbase, int cnt, i
   __syncwarp();
 }
 
-// Emit token j of the walk: dv = alpha dvt as two bf16, and the lane's share
-// of dalpha = <dvt, v> over its two features; every 32nd token flushes the
-// warp's partials.  Tokens are emitted once each, in increasing order.
-__device__ __forceinline__ void col_emit(float2 r, float2 vv, float a, int j, int ld, int np,
-                                         __nv_bfloat16* __restrict__ dvb, ColPartials& pb,
+// Emit token j of the walk: dv = alpha dvt (the lane's features, bf16), and
+// the lane's share of dalpha = <dvt, v>; every 32nd token flushes the warp's
+// partials.  Tokens are emitted once each, in increasing order.
+__device__ __forceinline__ void col_emit(const FPairs& r, const FPairs& vv, float a, int j, int ld,
+                                         int np, __nv_bfloat16* __restrict__ dvb, ColPartials& pb,
                                          float* __restrict__ pab) {
-  const float2 dvr = __fmul2_rn(make_float2(a, a), r);
-  *reinterpret_cast<__nv_bfloat162*>(dvb + j * ld) = __floats2bfloat162_rn(dvr.x, dvr.y);
-  pb.p[j & 31][threadIdx.x & 31] = fmaf(r.x, vv.x, r.y * vv.y);
+  __nv_bfloat162 o[COL_NP];
+  float dot = 0.f;
+#pragma unroll
+  for (int q = 0; q < COL_NP; ++q) {
+    const float2 dvr = __fmul2_rn(make_float2(a, a), r.p[q]);
+    o[q] = __floats2bfloat162_rn(dvr.x, dvr.y);
+    dot = fmaf(r.p[q].x, vv.p[q].x, fmaf(r.p[q].y, vv.p[q].y, dot));
+  }
+  if constexpr (COL_NP == 2) {
+    uint2 w;
+    w.x = *reinterpret_cast<const uint32_t*>(&o[0]);
+    w.y = *reinterpret_cast<const uint32_t*>(&o[COL_NP - 1]);
+    *reinterpret_cast<uint2*>(dvb + j * ld) = w;
+  } else {
+    *reinterpret_cast<__nv_bfloat162*>(dvb + j * ld) = o[0];
+  }
+  pb.p[j & 31][threadIdx.x & 31] = dot;
   if ((j & 31) == 31) col_flush(pb, j - 31, 32, np, pab);
 }
 
 // dynamic shared memory of the column walk: per warp the copy ring, the
 // dalpha partials and the chunk's gates
-constexpr int kColSmem =
-    COL_WARPS * (COL_RING * 2 * 32 * 8 + (int)sizeof(ColPartials) + (COL_TOK + 6) * 4);
+constexpr int kColSmem = COL_WARPS * (COL_RING * 2 * 32 * (int)sizeof(FPairs) +
+                                      (int)sizeof(ColPartials) + (COL_TOK + 6) * 4);
 
-// One warp per (chunk of COL_TOK tokens, 64 features), each lane holding two
-// adjacent features, walking the chunk in token order.  The warp keeps, for
-// the three previous tokens, vt and v, and the partial sums of their dvt:
-// dvt_s = u_s + w_3 dy_s + w_2 dy_{s+1} + w_1 dy_{s+2} + w_0 dy_{s+3} (terms
-// past the sequence end absent), to which each new dy_t adds its share.  At
-// token t it forms y_t and dy_t; dvt of token t-3 is then complete, and at a
-// sequence end so are t-2, t-1 and t.  The walk runs 3 tokens past the chunk
-// for the last tokens' dy.  v and dout of the next COL_RING - 1 tokens are
-// in flight into a per-warp shared-memory ring (asynchronous copies, each
-// lane its own 8 bytes), enough bytes in flight per SM to stream at HBM
-// rate with four warps per block.  `live` counts the ring's tokens that belong to
-// t's sequence and to this chunk's walk (tokens before the chunk are emitted
-// by the previous chunk's walk).  For each completed token it writes dv
-// (bf16, for the GEMMs) and the warp's partial of dalpha,
-// dalpha_part[token][f / 64] (the lanes' shares summed per 32 tokens, from
-// shared memory, in lane order); at the end the chunk's partial conv-weight
-// gradient, part[chunk][f] = sum over its tokens of
-// dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).  Warps are independent (all
-// lanes of one walk the same tokens, so the butterflies run on uniform
-// branches); the block only groups COL_WARPS chunks for scheduling.
-__global__ void __launch_bounds__(32 * COL_WARPS, 4) bw_col_kernel(
+// One warp per (chunk of COL_TOK tokens, COL_FEAT features), each lane
+// holding COL_NP pairs of adjacent features, walking the chunk in token
+// order.  The warp keeps, for the three previous tokens, vt and v, and the
+// partial sums of their dvt: dvt_s = u_s + w_3 dy_s + w_2 dy_{s+1} +
+// w_1 dy_{s+2} + w_0 dy_{s+3} (terms past the sequence end absent), to which
+// each new dy_t adds its share.  At token t it forms y_t and dy_t; dvt of
+// token t-3 is then complete, and at a sequence end so are t-2, t-1 and t.
+// The walk runs 3 tokens past the chunk for the last tokens' dy.  v and dout
+// of the next COL_RING - 1 tokens are in flight into a per-warp
+// shared-memory ring (asynchronous copies, each lane its own bytes), enough
+// bytes in flight per SM to stream at HBM rate.  `live` counts the ring's
+// tokens that belong to t's sequence and to this chunk's walk (tokens before
+// the chunk are emitted by the previous chunk's walk).  For each completed
+// token it writes dv (bf16, for the GEMMs) and the warp's partial of dalpha,
+// dalpha_part[token][f / COL_FEAT] (the lanes' shares summed per 32 tokens,
+// from shared memory, in lane order); at the end the chunk's partial
+// conv-weight gradient, part[chunk][f] = sum over its tokens of
+// dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).  The arithmetic runs on packed
+// fp32 pairs.  Warps are independent (all lanes of one walk the same tokens,
+// so the branches are uniform); the block only groups COL_WARPS chunks for
+// scheduling.
+__global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     const float* __restrict__ v, const float* __restrict__ alpha,
     const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
     int ld, int chunks, __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part,
@@ -210,15 +249,16 @@ __global__ void __launch_bounds__(32 * COL_WARPS, 4) bw_col_kernel(
   // v and dv rows are ld apart (they share rows with k and dk), dout rows d
   extern __shared__ __align__(16) unsigned char col_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  auto* ring_all = reinterpret_cast<float2(*)[COL_RING][2][32]>(col_smem);  // [slot][v, dout][lane]
-  auto* pb_all = reinterpret_cast<ColPartials*>(col_smem + COL_WARPS * COL_RING * 2 * 32 * 8);
-  auto* al_all = reinterpret_cast<float(*)[COL_TOK + 6]>(col_smem + COL_WARPS * COL_RING * 2 * 32 * 8 +
+  constexpr int RING_BYTES = COL_RING * 2 * 32 * (int)sizeof(FPairs);
+  auto* ring_all = reinterpret_cast<FPairs(*)[COL_RING][2][32]>(col_smem);  // [slot][v, dout][lane]
+  auto* pb_all = reinterpret_cast<ColPartials*>(col_smem + COL_WARPS * RING_BYTES);
+  auto* al_all = reinterpret_cast<float(*)[COL_TOK + 6]>(col_smem + COL_WARPS * RING_BYTES +
                                                           COL_WARPS * sizeof(ColPartials));
   ColPartials& pb = pb_all[warp];
   const int chunk = blockIdx.x * COL_WARPS + warp;
   if (chunk >= chunks) return;  // no block-wide barrier follows
-  const int f = blockIdx.y * COL_FEAT + lane * COL_FPT;
-  const int np = d / COL_FEAT;
+  const int f = blockIdx.y * COL_FEAT + lane * 2 * COL_NP;
+  const int np = col_partials(d);
   const int64_t t0 = (int64_t)chunk * COL_TOK;
   const int64_t t1 = t0 + COL_TOK < N ? t0 + COL_TOK : N;
   const int64_t t_stop = t1 + 3 < N ? t1 + 3 : N;
@@ -229,42 +269,45 @@ __global__ void __launch_bounds__(32 * COL_WARPS, 4) bw_col_kernel(
     al_s[i] = (tt >= 0 && tt < t_stop) ? alpha[tt] : 0.f;
   }
   __syncwarp();
-  const float4 wx = __ldg(conv_w + f), wy = __ldg(conv_w + f + 1);
   // the weights as (feature x, feature y) pairs: W0 multiplies vt_{t-3}, W3 vt_t
-  const float2 W0 = make_float2(wx.x, wy.x), W1 = make_float2(wx.y, wy.y);
-  const float2 W2 = make_float2(wx.z, wy.z), W3 = make_float2(wx.w, wy.w);
+  FPairs W0, W1, W2, W3;
+#pragma unroll
+  for (int q = 0; q < COL_NP; ++q) {
+    const float4 wx = __ldg(conv_w + f + 2 * q), wy = __ldg(conv_w + f + 2 * q + 1);
+    W0.p[q] = make_float2(wx.x, wy.x);
+    W1.p[q] = make_float2(wx.y, wy.y);
+    W2.p[q] = make_float2(wx.z, wy.z);
+    W3.p[q] = make_float2(wx.w, wy.w);
+  }
+  const FPairs zero = {};
   int pos = (int)(t0 % T);
-  float2 s1 = make_float2(0.f, 0.f), s2 = s1, s3 = s1;  // vt of t-1, t-2, t-3
-  if (pos >= 1) {
-    const float2 q = ld_f2(v + (t0 - 1) * ld + f);
-    s1 = make_float2(al_s[2] * q.x, al_s[2] * q.y);
-  }
-  if (pos >= 2) {
-    const float2 q = ld_f2(v + (t0 - 2) * ld + f);
-    s2 = make_float2(al_s[1] * q.x, al_s[1] * q.y);
-  }
-  if (pos >= 3) {
-    const float2 q = ld_f2(v + (t0 - 3) * ld + f);
-    s3 = make_float2(al_s[0] * q.x, al_s[0] * q.y);
-  }
-  float2 A1 = make_float2(0.f, 0.f), A2 = A1, A3 = A1;  // partial dvt of t-1, t-2, t-3
-  float2 v1 = A1, v2 = A1, v3 = A1;                      // v of t-1, t-2, t-3
-  // conv-weight partials, (x, y) pairs for w_0 .. w_3
-  float2 C0 = make_float2(0.f, 0.f), C1 = C0, C2 = C0, C3 = C0;
+  FPairs s1 = zero, s2 = zero, s3 = zero;  // vt of t-1, t-2, t-3
+  auto vt_of = [&](int64_t tt, float a) {
+    FPairs q = ld_pairs(v + tt * ld + f);
+#pragma unroll
+    for (int k = 0; k < COL_NP; ++k) q.p[k] = __fmul2_rn(make_float2(a, a), q.p[k]);
+    return q;
+  };
+  if (pos >= 1) s1 = vt_of(t0 - 1, al_s[2]);
+  if (pos >= 2) s2 = vt_of(t0 - 2, al_s[1]);
+  if (pos >= 3) s3 = vt_of(t0 - 3, al_s[0]);
+  FPairs A1 = zero, A2 = zero, A3 = zero;  // partial dvt of t-1, t-2, t-3
+  FPairs v1 = zero, v2 = zero, v3 = zero;  // v of t-1, t-2, t-3
+  FPairs C0 = zero, C1 = zero, C2 = zero, C3 = zero;  // conv-weight partials for w_0 .. w_3
   int live = 0;
   __nv_bfloat16* dvb = dv + t0 * ld + f;
   float* pab = dalpha_part + t0 * np + blockIdx.y;
   const int n_chunk = (int)(t1 - t0), n_walk = (int)(t_stop - t0);
   // token q's v and dout go to ring slot q % COL_RING; the slot refilled at
   // step i held token i - 1, whose values step i - 1 has already used
-  float2 (*ring)[2][32] = ring_all[warp];
+  FPairs (*ring)[2][32] = ring_all[warp];
   const float* vp = v + t0 * ld + f;
   const float* up = dout + t0 * d + f;
 #pragma unroll
   for (int q = 0; q < COL_RING - 1; ++q) {
     if (q < n_walk) {
-      cp_async8(&ring[q][0][lane], vp);
-      cp_async8(&ring[q][1][lane], up);
+      cp_async_pairs(&ring[q][0][lane], vp);
+      cp_async_pairs(&ring[q][1][lane], up);
     }
     cp_async_commit();
     vp += ld;
@@ -274,34 +317,44 @@ __global__ void __launch_bounds__(32 * COL_WARPS, 4) bw_col_kernel(
   for (int i = 0; i < n_walk; ++i) {
     cp_async_wait<COL_RING - 2>();  // token i's copies have landed
     const int slot = i % COL_RING;
-    const float2 vr = ring[slot][0][lane], ut = ring[slot][1][lane];
+    const FPairs vr = ring[slot][0][lane], ut = ring[slot][1][lane];
     const float at = al_s[i + 3];
     if (i + COL_RING - 1 < n_walk) {
       const int refill = (i + COL_RING - 1) % COL_RING;
-      cp_async8(&ring[refill][0][lane], vp);
-      cp_async8(&ring[refill][1][lane], up);
+      cp_async_pairs(&ring[refill][0][lane], vp);
+      cp_async_pairs(&ring[refill][1][lane], up);
     }
     cp_async_commit();
     vp += ld;
     up += d;
     if (pos == 0) {  // a sequence starts at t
-      s1 = s2 = s3 = make_float2(0.f, 0.f);
+      s1 = s2 = s3 = zero;
       live = 0;
     }
-    const float2 vt = __fmul2_rn(make_float2(at, at), vr);
-    const float2 y = __ffma2_rn(W0, s3, __ffma2_rn(W1, s2, __ffma2_rn(W2, s1, __fmul2_rn(W3, vt))));
-    const float2 g = __fmul2_rn(ut, silu_grad2(y));
-    if (i < n_chunk) {
-      C0 = __ffma2_rn(g, s3, C0);
-      C1 = __ffma2_rn(g, s2, C1);
-      C2 = __ffma2_rn(g, s1, C2);
-      C3 = __ffma2_rn(g, vt, C3);
+    FPairs vt, g, E3, B2, B1, B0;
+#pragma unroll
+    for (int q = 0; q < COL_NP; ++q) {
+      vt.p[q] = __fmul2_rn(make_float2(at, at), vr.p[q]);
+      const float2 y = __ffma2_rn(W0.p[q], s3.p[q],
+                                  __ffma2_rn(W1.p[q], s2.p[q],
+                                             __ffma2_rn(W2.p[q], s1.p[q],
+                                                        __fmul2_rn(W3.p[q], vt.p[q]))));
+      g.p[q] = __fmul2_rn(ut.p[q], silu_grad2(y));
+      E3.p[q] = __ffma2_rn(W0.p[q], g.p[q], A3.p[q]);  // dvt of t-3, complete
+      B2.p[q] = __ffma2_rn(W1.p[q], g.p[q], A2.p[q]);
+      B1.p[q] = __ffma2_rn(W2.p[q], g.p[q], A1.p[q]);
+      B0.p[q] = __ffma2_rn(W3.p[q], g.p[q], ut.p[q]);
     }
-    if (live == 3)  // token t-3 is complete
-      col_emit(__ffma2_rn(W0, g, A3), v3, al_s[i], i - 3, ld, np, dvb, pb, pab);
-    const float2 B2 = __ffma2_rn(W1, g, A2);
-    const float2 B1 = __ffma2_rn(W2, g, A1);
-    const float2 B0 = __ffma2_rn(W3, g, ut);
+    if (i < n_chunk) {
+#pragma unroll
+      for (int q = 0; q < COL_NP; ++q) {
+        C0.p[q] = __ffma2_rn(g.p[q], s3.p[q], C0.p[q]);
+        C1.p[q] = __ffma2_rn(g.p[q], s2.p[q], C1.p[q]);
+        C2.p[q] = __ffma2_rn(g.p[q], s1.p[q], C2.p[q]);
+        C3.p[q] = __ffma2_rn(g.p[q], vt.p[q], C3.p[q]);
+      }
+    }
+    if (live == 3) col_emit(E3, v3, al_s[i], i - 3, ld, np, dvb, pb, pab);  // token t-3
     if (pos == T - 1) {  // the sequence ends at t: its last tokens are complete
       if (live >= 2 && i - 2 < n_chunk) col_emit(B2, v2, al_s[i + 1], i - 2, ld, np, dvb, pb, pab);
       if (live >= 1 && i - 1 < n_chunk) col_emit(B1, v1, al_s[i + 2], i - 1, ld, np, dvb, pb, pab);
@@ -320,8 +373,13 @@ __global__ void __launch_bounds__(32 * COL_WARPS, 4) bw_col_kernel(
     pos = pos + 1 == T ? 0 : pos + 1;
   }
   if (n_chunk & 31) col_flush(pb, n_chunk & ~31, n_chunk & 31, np, pab);
-  part[(int64_t)chunk * d + f] = make_float4(C0.x, C1.x, C2.x, C3.x);
-  part[(int64_t)chunk * d + f + 1] = make_float4(C0.y, C1.y, C2.y, C3.y);
+#pragma unroll
+  for (int q = 0; q < COL_NP; ++q) {
+    part[(int64_t)chunk * d + f + 2 * q] =
+        make_float4(C0.p[q].x, C1.p[q].x, C2.p[q].x, C3.p[q].x);
+    part[(int64_t)chunk * d + f + 2 * q + 1] =
+        make_float4(C0.p[q].y, C1.p[q].y, C2.p[q].y, C3.p[q].y);
+  }
 }
 
 constexpr int ROW_THREADS = 256;
@@ -374,10 +432,10 @@ __device__ __forceinline__ bool row_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Shared memory of one stage of the row kernel: the token's h (bf16), k and
-// dout (fp32) rows and its d/64 dalpha partials; all offsets are multiples of
-// 16 bytes because d is a multiple of 256.
+// dout (fp32) rows and its dalpha partials (d/128, padded to a multiple of
+// 4); all offsets are multiples of 16 bytes because d is a multiple of 256.
 __host__ __device__ constexpr size_t row_stage_bytes(int d) {
-  return (size_t)d * 2 + (size_t)d * 4 + (size_t)d * 4 + (size_t)(d / COL_FEAT) * 4;
+  return (size_t)d * 2 + (size_t)d * 4 + (size_t)d * 4 + (size_t)col_partials(d) * 4;
 }
 
 // The gate and both RMSNorm backwards need whole-row sums, so each token is
@@ -385,7 +443,7 @@ __host__ __device__ constexpr size_t row_stage_bytes(int d) {
 // + gridDim.x, ..., with the next token's rows already in flight into the
 // other shared-memory stage (bulk copies issued by one thread, completing on
 // an mbarrier).  Each thread takes 4 features per item from shared memory
-// into registers; <h,h>, <k,k>, <h,k> and dalpha (the column walk's d/64
+// into registers; <h,h>, <k,k>, <h,k> and dalpha (the column walk's d/128
 // partials, added in order by the first warp) are reduced together in one
 // fixed-order pass, whose barrier also frees the stage for the token after
 // next; then dk (bf16, for the GEMMs) and dh are written.  A copy that never
@@ -407,9 +465,10 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
   __shared__ uint64_t full[ROW_STAGES];
   __shared__ float4 red[2][ROW_THREADS / 32];
   __shared__ int abort_flag;
-  const int np = d / COL_FEAT;
+  const int np = d / COL_FEAT, np_pad = col_partials(d);
   const size_t SB = row_stage_bytes(d);
-  const uint32_t hb_bytes = (uint32_t)d * 2, f_bytes = (uint32_t)d * 4, p_bytes = (uint32_t)np * 4;
+  const uint32_t hb_bytes = (uint32_t)d * 2, f_bytes = (uint32_t)d * 4,
+                 p_bytes = (uint32_t)np_pad * 4;
   const int64_t G = gridDim.x;
   unsigned pend = 0;  // thread 0: stages with a copy issued and not yet seen landed
   auto issue = [&](int64_t t, int st) {  // thread 0
@@ -421,7 +480,7 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     bulk_load(base, h + t * d, hb_bytes, &full[st]);
     bulk_load(base + hb_bytes, k + t * ld, f_bytes, &full[st]);
     bulk_load(base + hb_bytes + f_bytes, dout + t * d, f_bytes, &full[st]);
-    bulk_load(base + hb_bytes + 2 * f_bytes, dalpha_part + t * np, p_bytes, &full[st]);
+    bulk_load(base + hb_bytes + 2 * f_bytes, dalpha_part + t * np_pad, p_bytes, &full[st]);
   };
   if (threadIdx.x == 0) {
     for (int st = 0; st < ROW_STAGES; ++st)
@@ -624,7 +683,7 @@ __global__ void __launch_bounds__(32 * DCONV_WARPS) bw_dconv_reduce_kernel(
 }
 
 // Workspace: [k | v] fp32 [N, 2d]; [dk | dv] bf16 [N, 2d]; [W_k; W_v] bf16
-// and [dW_k; dW_v] fp32 [2d, E]; dalpha partials [N, d/64]; de fp32 [N, E]
+// and [dW_k; dW_v] fp32 [2d, E]; dalpha partials [N, d/128 padded to 4]; de fp32 [N, E]
 // when the caller passes none; conv partials; cuBLAS's workspace; the table
 // gradient's sort buffers.
 struct BwdBf16Ws {
@@ -636,7 +695,7 @@ struct BwdBf16Ws {
   __nv_bfloat16* dkv;
   __nv_bfloat16* Wkv;
   float* dWkv;          // [2d, E], copied out to dWk and dWv
-  float *dalpha_part, *de;  // [N, d/64] partials of <dvt, v>
+  float *dalpha_part, *de;  // partials of <dvt, v>, padded rows
   float4* part;
   float* spart;  // with norm scales: [kMaxRowBlocks][d] sums of the row blocks
   void* blas_ws;
@@ -654,7 +713,7 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
   const size_t KV = kv_saved ? 0 : up256b((size_t)N * 2 * d * 4);
   const size_t DKV = up256b((size_t)N * 2 * d * 2);
   const size_t WKV = up256b((size_t)2 * d * E * 2), DW = up256b((size_t)2 * d * E * 4);
-  const size_t DA = up256b((size_t)N * (d / COL_FEAT) * 4);
+  const size_t DA = up256b((size_t)N * col_partials(d) * 4);
   const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
   const size_t tg = table_grad_ws_bytes(N * J);
   const size_t SP = scaled ? up256b((size_t)kMaxRowBlocks * d * 4) : 0;
