@@ -53,7 +53,14 @@ constexpr unsigned FULL = 0xffffffffu;
 // pass K; pass V over whole sequences (conv history from the rows above);
 // pass V in decode (one token per sequence, conv history from the state)
 // pass K (MODE_GATE_SCALED: with learnable norm scales) and pass V
-enum { MODE_GATE_PARTIAL = 0, MODE_VALUE_CONV = 1, MODE_VALUE_DECODE = 2, MODE_GATE_SCALED = 3 };
+// (MODE_VALUE_CONV_KV: also storing v for the backward)
+enum {
+  MODE_GATE_PARTIAL = 0,
+  MODE_VALUE_CONV = 1,
+  MODE_VALUE_DECODE = 2,
+  MODE_GATE_SCALED = 3,
+  MODE_VALUE_CONV_KV = 4
+};
 
 struct TcArgs {
   int num_m_tiles, num_n_tiles, num_k_tiles;
@@ -399,7 +406,9 @@ __device__ __forceinline__ void conv_group16(const uint32_t (&u)[16], const floa
 
 template <int BN, int STAGES, int MODE, int KCH>
 struct TcShape {
-  static constexpr bool VPASS = MODE == MODE_VALUE_CONV || MODE == MODE_VALUE_DECODE;
+  static constexpr bool VPASS =
+      MODE == MODE_VALUE_CONV || MODE == MODE_VALUE_DECODE || MODE == MODE_VALUE_CONV_KV;
+  static constexpr bool KEEP_V = MODE == MODE_VALUE_CONV_KV;
   // epilogue warps: 2 per TMEM lane quadrant
   static constexpr int EPI = 8;
   static constexpr int PARTS = EPI / 4;        // column parts of a tile, one per warp of a quadrant
@@ -429,11 +438,12 @@ struct TcShape {
   static constexpr int HSLOT_BYTES = PARTS * HBOX_BYTES;
   static constexpr int ALPHA_BYTES = VPASS ? 2 * BN * 4 : 0;  // gates of a tile, two tiles
   // pass K, when k is kept: each epilogue warp stages its 32 tokens x 32
-  // features (fp32, 128-byte swizzled) for one tiled store
-  static constexpr int KVBUF_BYTES = VPASS ? 0 : EPI * 32 * 32 * 4;
+  // features (fp32, 128-byte swizzled) for one tiled store; pass V keeping v
+  // stages its 32 tokens x 32 features (token rows) the same way
+  static constexpr int KVBUF_BYTES = (VPASS && !KEEP_V) ? 0 : EPI * 32 * 32 * 4;
   // as many h slots (up to 4) as the shared memory left by the operand stages holds
   static constexpr int HSLOTS_FIT =
-      (232448 - STAGES * (A_BYTES + B_BYTES) - 256 - ALPHA_BYTES) / HSLOT_BYTES;
+      (232448 - STAGES * (A_BYTES + B_BYTES) - KVBUF_BYTES - 256 - ALPHA_BYTES) / HSLOT_BYTES;
   static constexpr int HSLOTS = VPASS ? (HSLOTS_FIT < 4 ? HSLOTS_FIT : 4) : 0;
   static constexpr size_t SMEM = (size_t)STAGES * (A_BYTES + B_BYTES) +
                                  (size_t)HSLOTS * HSLOT_BYTES + KVBUF_BYTES + 256 + ALPHA_BYTES;
@@ -448,7 +458,8 @@ template <int BN, int STAGES, int MODE, int KCH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, MODE, KCH>::NUM_THREADS, 1)
     tc_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmO,
-                    const __grid_constant__ CUtensorMap tmO29, const __grid_constant__ TcArgs args) {
+                    const __grid_constant__ CUtensorMap tmO29, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmV29, const __grid_constant__ TcArgs args) {
   using S = TcShape<BN, STAGES, MODE, KCH>;
   constexpr bool VPASS = S::VPASS;
   constexpr int NUM_EPI_WARPS = S::EPI;
@@ -471,7 +482,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::A_BYTES;
   uint8_t* hring = sB + STAGES * S::B_BYTES;
-  uint8_t* kvbuf = hring + S::HSLOTS * S::HSLOT_BYTES;  // pass K only
+  uint8_t* kvbuf = hring + S::HSLOTS * S::HSLOT_BYTES;  // pass K, and pass V keeping v
   uint64_t* bars = reinterpret_cast<uint64_t*>(kvbuf + S::KVBUF_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
@@ -530,6 +541,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
       prefetch_tmap(&tmH);
       prefetch_tmap(&tmO);
       prefetch_tmap(&tmO29);
+      if constexpr (S::KEEP_V) {
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmV29);
+      }
     }
   }
   if (warp == 1) {
@@ -972,24 +987,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
             if (got) tmem_wait16(un);
             conv_group16<true>(un, al4 + 4, hs + 16 * BM, w, s1, s2, s3, pos, T);
           }
-          if (!DECODE && args.kv_save != nullptr && got) {
-            // v itself, for the backward: token by token, the warp's 32
-            // features side by side (one 128-byte line per token); halo
-            // columns are stored by the tile that owns them
-            float* vp = args.kv_save + nb * 2 * args.d + args.d + feat;
-            const int64_t ld = 2 * (int64_t)args.d;
-            if (jb >= first_out && nb + 32 <= args.N) {
+          if constexpr (S::KEEP_V) {
+            // v itself, for the backward: the warp's 32 tokens x 32 features
+            // go through its staging buffer (row = token) and out in one
+            // tiled store by lane 1 (its own bulk groups); the halo tokens of
+            // a tile are stored by the tile that owns them
+            uint8_t* vb = kvbuf + ew * (32 * 32 * 4);
+            if (lane == 1) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();  // the previous store has read the buffer
+            float* vrow = reinterpret_cast<float*>(vb) + lane;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                __stcs(vp, __uint_as_float(i < 16 ? u[i] : un[i - 16]));
-                vp += ld;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                if (jb + i >= first_out && nb + i < args.N)
-                  vp[i * ld] = __uint_as_float(i < 16 ? u[i] : un[i - 16]);
-              }
+            for (int i = 0; i < 32; ++i) vrow[i * 32] = __uint_as_float(i < 16 ? u[i] : un[i - 16]);
+            fence_async_shared();
+            __syncwarp();
+            if (lane == 1 && got) {
+              const int vx = args.d + f0 + quad * 32;
+              if (jb < first_out)
+                tma_store_2d(&tmV29, vb + first_out * 128, vx, (int)(nb + first_out));
+              else
+                tma_store_2d(&tmV, vb, vx, (int)nb);
             }
           }
           // the part's four warps have written the box: one thread stores it
@@ -1025,6 +1041,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
+    }
+    if constexpr (S::KEEP_V) {  // v's staging buffers read before the CTA exits
+      if (lane == 1) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
     // output boxes of pass V fully written before the CTA exits
     if (VPASS && ew == part * 4 && lane == 0) {
@@ -1150,8 +1169,8 @@ bool make_tmap_k(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, ui
 
 template <int BN, int STAGES, int MODE, int KCH>
 int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& th,
-                const CUtensorMap& to, const CUtensorMap& to29, const TcArgs& a, cudaStream_t s,
-                bool pdl) {
+                const CUtensorMap& to, const CUtensorMap& to29, const CUtensorMap& tv,
+                const CUtensorMap& tv29, const TcArgs& a, cudaStream_t s, bool pdl) {
   using S = TcShape<BN, STAGES, MODE, KCH>;
   auto kern = tc_fused_kernel<BN, STAGES, MODE, KCH>;
   static bool configured[64] = {false};
@@ -1180,10 +1199,12 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return ck(cudaLaunchKernelEx(&cfg, kern, ta, tb, th, to, to29, a));
+  return ck(cudaLaunchKernelEx(&cfg, kern, ta, tb, th, to, to29, tv, tv29, a));
 }
 
-template <int BN, int STAGES_K, int STAGES_V, int KCH>
+// STAGES_VKV: operand stages of pass V when it also keeps v (its staging
+// buffers take the room of one stage on the wide tiles)
+template <int BN, int STAGES_K, int STAGES_V, int STAGES_VKV, int KCH>
 int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
               float* alpha_saved, float* kv_save, const float* gg, int64_t N, int T, int d, int E,
@@ -1235,10 +1256,10 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
                      CU_TENSOR_MAP_SWIZZLE_128B))
     return ENGRAM_ERR_CUDA;
   int rc = gg != nullptr
-               ? launch_pass<BN, STAGES_K, MODE_GATE_SCALED, KCH>(ta_k, tb_k, th, tkv, to29, a, s,
-                                                                  chained)
-               : launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL, KCH>(ta_k, tb_k, th, tkv, to29, a, s,
-                                                                   chained);
+               ? launch_pass<BN, STAGES_K, MODE_GATE_SCALED, KCH>(ta_k, tb_k, th, tkv, to29, to,
+                                                                  to29, a, s, chained)
+               : launch_pass<BN, STAGES_K, MODE_GATE_PARTIAL, KCH>(ta_k, tb_k, th, tkv, to29, to,
+                                                                   to29, a, s, chained);
   if (rc) return rc;
   {
     int dev = 0, sms = 148;
@@ -1267,8 +1288,22 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   }
   a.num_m_tiles = (int)((N + a.m_stride - 1) / a.m_stride);
   if (conv_state != nullptr)
-    return launch_pass<BN, STAGES_V, MODE_VALUE_DECODE, KCH>(ta_v, tb_v, th, to, to29, a, s, true);
-  return launch_pass<BN, STAGES_V, MODE_VALUE_CONV, KCH>(ta_v, tb_v, th, to, to29, a, s, true);
+    return launch_pass<BN, STAGES_V, MODE_VALUE_DECODE, KCH>(ta_v, tb_v, th, to, to29, to, to29, a,
+                                                             s, true);
+  if (a.kv_save != nullptr) {
+    // v into the saved [k | v] rows: boxes of 32 features x 32 tokens, and a
+    // 29-token box that skips a tile's conv halo
+    CUtensorMap tv, tv29;
+    if (!make_tmap_f32(&tv, a.kv_save, (uint64_t)(2 * d), (uint64_t)N, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tmap_f32(&tv29, a.kv_save, (uint64_t)(2 * d), (uint64_t)N, 32, 32 - HALO,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+      return ENGRAM_ERR_CUDA;
+    return launch_pass<BN, STAGES_VKV, MODE_VALUE_CONV_KV, KCH>(ta_v, tb_v, th, to, to29, tv, tv29,
+                                                                a, s, true);
+  }
+  return launch_pass<BN, STAGES_V, MODE_VALUE_CONV, KCH>(ta_v, tb_v, th, to, to29, to, to29, a, s,
+                                                         true);
 }
 
 inline bool use_wide(int64_t N, int d) { return d % 256 == 0 && N > 4096; }
@@ -1312,14 +1347,14 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
   float* alpha = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                           (size_t)N * 2 * (d / BN) * sizeof(float4));
   if (wide)
-    return run_layer<256, 6, 5, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
+    return run_layer<256, 6, 5, 4, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
                                    gg, N, T, d, E, part, alpha, chained, s);
   // few tokens: each CTA streams long operand rows at a rate set by how many
   // bytes one copy instruction brings, so two K chunks go in each box
   if (E % (2 * BK) == 0)
-    return run_layer<64, 4, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
+    return run_layer<64, 4, 3, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
                                   gg, N, T, d, E, part, alpha, chained, s);
-  return run_layer<64, 8, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, gg,
+  return run_layer<64, 8, 6, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, gg,
                                 N, T, d, E, part, alpha, chained, s);
 }
 
