@@ -36,9 +36,9 @@ int check_cfg(const engram_cfg_t* c) {
 
 inline int elem_bytes(const engram_cfg_t* c) { return c->dtype == ENGRAM_F32 ? 4 : 2; }
 
-// variants the bf16 path implements: learnable norm scales, and per-branch
-// conv weights (with one branch, the same as shared ones)
-constexpr int kBf16Variants = ENGRAM_NORM_SCALES | ENGRAM_CONV_PER_BRANCH;
+// variants the bf16 path implements: learnable norm scales, the dilated
+// conv, and per-branch conv weights (with one branch, the same as shared ones)
+constexpr int kBf16Variants = ENGRAM_NORM_SCALES | ENGRAM_CONV_PER_BRANCH | ENGRAM_CONV_DILATED;
 inline bool bf16_variant_ok(const engram_cfg_t* c) {
   return (c->flags & ENGRAM_VARIANT_FLAGS & ~kBf16Variants) == 0;
 }
@@ -226,8 +226,9 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
   return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
                            static_cast<const __nv_bfloat16*>(Wk),
                            static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
-                           static_cast<__nv_bfloat16*>(out), saved, kv_save, gg, N, T, d, E, ws,
-                           ws_bytes, table != nullptr, s);
+                           static_cast<__nv_bfloat16*>(out), saved, kv_save, gg,
+                           (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1, N, T, d, E, ws, ws_bytes,
+                           table != nullptr, s);
 }
 
 int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,
@@ -237,7 +238,8 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                     void* ws, size_t ws_bytes, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (cfg->dtype == ENGRAM_BF16 && (cfg->n_branch != 1 || !bf16_variant_ok(cfg)))
+  if (cfg->dtype == ENGRAM_BF16 && (cfg->n_branch != 1 || !bf16_variant_ok(cfg) ||
+                                    (cfg->flags & ENGRAM_CONV_DILATED) != 0))
     return ENGRAM_ERR_UNSUPPORTED;
   if (cfg->dtype == ENGRAM_BF16 && saved == nullptr) return ENGRAM_ERR_INVALID_ARG;
   if (B < 0 || T < 0) return ENGRAM_ERR_INVALID_ARG;

@@ -45,21 +45,25 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle row
 constexpr int UMMA_K = 16;
-constexpr int HALO = 3;  // conv width 4 - 1
 constexpr float RMS_EPS = 1e-6f;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 constexpr unsigned FULL = 0xffffffffu;
 
 // pass K; pass V over whole sequences (conv history from the rows above);
 // pass V in decode (one token per sequence, conv history from the state)
-// pass K (MODE_GATE_SCALED: with learnable norm scales) and pass V
-// (MODE_VALUE_CONV_KV: also storing v for the backward)
+// Kernel modes, as bits: pass K (MODE_GATE_SCALED: with learnable norm
+// scales) or pass V (MODE_V_PASS) with its options: decode steps, v also
+// stored for the backward, the conv dilated by 3.
 enum {
   MODE_GATE_PARTIAL = 0,
-  MODE_VALUE_CONV = 1,
-  MODE_VALUE_DECODE = 2,
-  MODE_GATE_SCALED = 3,
-  MODE_VALUE_CONV_KV = 4
+  MODE_GATE_SCALED = 1,
+  MODE_V_PASS = 16,
+  MODE_V_DECODE = 2,
+  MODE_V_KEEP = 4,
+  MODE_V_DILATED = 8,
+  MODE_VALUE_CONV = MODE_V_PASS,
+  MODE_VALUE_DECODE = MODE_V_PASS | MODE_V_DECODE,
+  MODE_VALUE_CONV_KV = MODE_V_PASS | MODE_V_KEEP
 };
 
 struct TcArgs {
@@ -375,10 +379,11 @@ __device__ __forceinline__ float silu_tanh(float y) {
   return fmaf(hy, t, hy);
 }
 
-template <bool CHECK>
+// sh[q] holds vt of token t-1-q (the conv's 3 * DIL tokens of history).
+template <bool CHECK, int DIL>
 __device__ __forceinline__ void conv_group16(const uint32_t (&u)[16], const float4* al4,
-                                             uint16_t* hs, const float4 w, float& s1, float& s2,
-                                             float& s3, int& pos, const int T) {
+                                             uint16_t* hs, const float4 w, float (&sh)[3 * DIL],
+                                             int& pos, const int T) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const float4 a4 = al4[q];
@@ -388,13 +393,17 @@ __device__ __forceinline__ void conv_group16(const uint32_t (&u)[16], const floa
       const int jj = q * 4 + r;
       const float vt = av[r] * __uint_as_float(u[jj]);
       if (CHECK) {
-        if (pos == 0) s1 = s2 = s3 = 0.f;  // a sequence starts at this token
+        if (pos == 0) {  // a sequence starts at this token
+#pragma unroll
+          for (int k = 0; k < 3 * DIL; ++k) sh[k] = 0.f;
+        }
         pos = (pos + 1 == T) ? 0 : pos + 1;
       }
-      const float y = fmaf(w.x, s3, fmaf(w.y, s2, fmaf(w.z, s1, w.w * vt)));
-      s3 = s2;
-      s2 = s1;
-      s1 = vt;
+      const float y =
+          fmaf(w.x, sh[3 * DIL - 1], fmaf(w.y, sh[2 * DIL - 1], fmaf(w.z, sh[DIL - 1], w.w * vt)));
+#pragma unroll
+      for (int k = 3 * DIL - 1; k > 0; --k) sh[k] = sh[k - 1];
+      sh[0] = vt;
       const float hv = __uint_as_float(((uint32_t)hs[jj * BM]) << 16);
       const float o = hv + vt + silu_tanh(y);  // h + vt + SiLU(y)
       hs[jj * BM] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
@@ -406,9 +415,12 @@ __device__ __forceinline__ void conv_group16(const uint32_t (&u)[16], const floa
 
 template <int BN, int STAGES, int MODE, int KCH>
 struct TcShape {
-  static constexpr bool VPASS =
-      MODE == MODE_VALUE_CONV || MODE == MODE_VALUE_DECODE || MODE == MODE_VALUE_CONV_KV;
-  static constexpr bool KEEP_V = MODE == MODE_VALUE_CONV_KV;
+  static constexpr bool VPASS = (MODE & MODE_V_PASS) != 0;
+  static constexpr bool DECODE = VPASS && (MODE & MODE_V_DECODE) != 0;
+  static constexpr bool KEEP_V = VPASS && (MODE & MODE_V_KEEP) != 0;
+  static constexpr bool SCALED = !VPASS && (MODE & MODE_GATE_SCALED) != 0;
+  static constexpr int DIL = (VPASS && (MODE & MODE_V_DILATED) != 0) ? 3 : 1;  // conv dilation
+  static constexpr int HALO_T = 3 * DIL;  // tokens of conv history a token needs
   // epilogue warps: 2 per TMEM lane quadrant
   static constexpr int EPI = 8;
   static constexpr int PARTS = EPI / 4;        // column parts of a tile, one per warp of a quadrant
@@ -730,7 +742,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
             for (int b = 0; b < S::PART_COLS * 2; b += 128) prefetch_l2(hp0 + b / 2);
           }
         }
-      } else if constexpr (MODE == MODE_VALUE_DECODE) {
+      } else if constexpr (S::DECODE) {
         const int64_t n0 = tok0 + part * S::PART_COLS + lane;
         if (lane < S::PART_COLS && n0 < args.N) {
           const float* st = args.conv_state + n0 * 3 * args.d + ni * (2 * BM) + (int)rank * BM +
@@ -811,7 +823,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
               unpack_bf16x32(h0, hv);
             else
               load_bf16x32(args.h + n * args.d + col_base + c * 32, hv);
-            if constexpr (MODE == MODE_GATE_SCALED) {
+            if constexpr (S::SCALED) {
               // <RMSNorm(h) g_h, RMSNorm(k) g_k>: weight h k by g_h g_k
               const float4* gq = reinterpret_cast<const float4*>(args.gg + col_base + c * 32);
 #pragma unroll
@@ -843,7 +855,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
         // pass V: this lane's feature, one part of the tile's tokens.  The causal
         // conv walks the tokens in order with vt of the three previous tokens
         // of the same sequence in registers.
-        constexpr bool DECODE = MODE == MODE_VALUE_DECODE;
+        constexpr bool DECODE = S::DECODE;
         constexpr int NCH = S::NCHUNK;
         const int f0 = ni * (2 * BM) + (int)rank * BM;  // this CTA's features
         const int feat = f0 + quad * 32 + lane;
@@ -861,7 +873,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
         const int j0 = part * S::PART_COLS;          // first tile column of this warp
         // decode, one chunk per part: the conv states of the first 16 tokens,
         // fetched while the MMAs finish
-        constexpr bool PRELOAD = DECODE && NCH == 1;
+        constexpr bool PRELOAD = DECODE && NCH == 1 && S::DIL == 1;
         float pre1[PRELOAD ? 16 : 1], pre2[PRELOAD ? 16 : 1], pre3[PRELOAD ? 16 : 1];
         if constexpr (PRELOAD) {
 #pragma unroll
@@ -880,9 +892,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
         const int got = wait_acc();
         const int first_out = -args.m_offset;        // halo columns produce no output
         int pos = (int)((((tok0 + j0) % T) + T) % T);  // sequence position of column j0
-        float s1 = 0.f, s2 = 0.f, s3 = 0.f;           // vt of tokens t-1, t-2, t-3
+        constexpr int NH = S::HALO_T;                 // tokens of conv history
+        float sh[NH];                                 // sh[q]: vt of token t-1-q
+#pragma unroll
+        for (int k = 0; k < NH; ++k) sh[k] = 0.f;
         if (!DECODE && j0 > 0) {
-          // the three columns before this part, recomputed from TMEM
+          // the NH columns before this part, recomputed from TMEM
           uint32_t u4[16];
           __syncwarp();
           if (got) {
@@ -893,13 +908,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
             for (int i = 0; i < 16; ++i) u4[i] = 0u;
           }
 #pragma unroll
-          for (int i = 13; i < 16; ++i) {
+          for (int i = 16 - NH; i < 16; ++i) {
             const int pq = (((pos - (16 - i)) % T) + T) % T;
             const float vt = al[j0 - 16 + i] * __uint_as_float(u4[i]);
-            if (pq == 0) s1 = s2 = s3 = 0.f;
-            s3 = s2;
-            s2 = s1;
-            s1 = vt;
+            if (pq == 0) {
+#pragma unroll
+              for (int k = 0; k < NH; ++k) sh[k] = 0.f;
+            }
+#pragma unroll
+            for (int k = NH - 1; k > 0; --k) sh[k] = sh[k - 1];
+            sh[0] = vt;
           }
         }
 #pragma unroll 1
@@ -924,7 +942,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
           const int jb = j0 + c * 32;
           const int64_t nb = tok0 + jb;
           const float4* al4 = reinterpret_cast<const float4*>(al + jb);
-          if (DECODE) {
+          if constexpr (DECODE && S::DIL > 1) {
+            // dilated conv: the state holds vt of the 3 dil previous steps
+            // (oldest first); 4 tokens' states are loaded before any of them
+            // is written back
+            constexpr int NS = S::HALO_T;
+#pragma unroll
+            for (int g4 = 0; g4 < 8; ++g4) {
+              if (g4 == 4 && got) tmem_wait16(un);
+              float sq[4][NS];
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                const int64_t n = nb + g4 * 4 + r;
+#pragma unroll
+                for (int k = 0; k < NS; ++k) sq[r][k] = 0.f;
+                if (n < args.N) {
+                  const float* st = args.conv_state + n * NS * args.d + feat;
+#pragma unroll
+                  for (int k = 0; k < NS; ++k) sq[r][k] = st[k * args.d];
+                }
+              }
+              const float4 a4 = al4[g4];
+              const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+              for (int r = 0; r < 4; ++r) {
+                const int jj = g4 * 4 + r;
+                const int64_t n = nb + jj;
+                const float vt = av[r] * __uint_as_float(jj < 16 ? u[jj] : un[jj - 16]);
+                if (n < args.N) {
+                  float* st = args.conv_state + n * NS * args.d + feat;
+#pragma unroll
+                  for (int k = 0; k + 1 < NS; ++k) st[k * args.d] = sq[r][k + 1];
+                  st[(NS - 1) * args.d] = vt;
+                }
+                const float y = fmaf(w.x, sq[r][0], fmaf(w.y, sq[r][S::DIL],
+                                                         fmaf(w.z, sq[r][2 * S::DIL], w.w * vt)));
+                const float hv = __uint_as_float(((uint32_t)hs[jj * BM]) << 16);
+                const float o = hv + vt + silu_tanh(y);
+                hs[jj * BM] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+              }
+            }
+          } else if (DECODE) {
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
               // the conv states of 16 tokens, loaded before any of them is
@@ -977,15 +1035,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
             }
           } else if (pos + 32 <= T && pos != 0) {
             // no sequence starts inside the chunk: no per-token checks
-            conv_group16<false>(u, al4, hs, w, s1, s2, s3, pos, T);
+            conv_group16<false, S::DIL>(u, al4, hs, w, sh, pos, T);
             if (got) tmem_wait16(un);
-            conv_group16<false>(un, al4 + 4, hs + 16 * BM, w, s1, s2, s3, pos, T);
+            conv_group16<false, S::DIL>(un, al4 + 4, hs + 16 * BM, w, sh, pos, T);
             pos += 32;
             if (pos == T) pos = 0;
           } else {
-            conv_group16<true>(u, al4, hs, w, s1, s2, s3, pos, T);
+            conv_group16<true, S::DIL>(u, al4, hs, w, sh, pos, T);
             if (got) tmem_wait16(un);
-            conv_group16<true>(un, al4 + 4, hs + 16 * BM, w, s1, s2, s3, pos, T);
+            conv_group16<true, S::DIL>(un, al4 + 4, hs + 16 * BM, w, sh, pos, T);
           }
           if constexpr (S::KEEP_V) {
             // v itself, for the backward: the warp's 32 tokens x 32 features
@@ -1207,8 +1265,8 @@ int launch_pass(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
 template <int BN, int STAGES_K, int STAGES_V, int STAGES_VKV, int KCH>
 int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
-              float* alpha_saved, float* kv_save, const float* gg, int64_t N, int T, int d, int E,
-              float4* part, float* alpha, bool chained, cudaStream_t s) {
+              float* alpha_saved, float* kv_save, const float* gg, int dil, int64_t N, int T,
+              int d, int E, float4* part, float* alpha, bool chained, cudaStream_t s) {
   // Each CTA of a pair loads 128 rows of A and BN/2 rows of B per stage.
   // pass K: A = e (256 tokens per pair tile), B = W_k (BN features)
   CUtensorMap ta_k, tb_k, ta_v, tb_v, th, to, to29;
@@ -1220,10 +1278,12 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   if (!make_tmap_k(&tb_v, e, (uint64_t)E, (uint64_t)N, BN / 2, KCH)) return ENGRAM_ERR_CUDA;
   if (!make_tmap(&th, h, (uint64_t)d, (uint64_t)N, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ENGRAM_ERR_CUDA;
-  // out in the same boxes; a 29-token box skips the 3 halo tokens of a tile
+  // out in the same boxes; a shorter box skips the halo tokens of a tile
+  // (3 dil: the conv's history)
+  const int halo = 3 * dil;
   if (!make_tmap(&to, out, (uint64_t)d, (uint64_t)N, BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ENGRAM_ERR_CUDA;
-  if (!make_tmap(&to29, out, (uint64_t)d, (uint64_t)N, BM, 32 - HALO, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!make_tmap(&to29, out, (uint64_t)d, (uint64_t)N, BM, 32 - halo, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ENGRAM_ERR_CUDA;
   TcArgs a;
   a.num_k_tiles = E / (BK * KCH);
@@ -1277,33 +1337,41 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   }
   a.alpha = alpha;
   // pass V: pair tiles of 256 features x BN tokens.  Whole sequences: the
-  // token tiles overlap by 3 (the conv halo, recomputed); decode: plain tiles.
+  // token tiles overlap by the conv's history (recomputed); decode: plain
+  // tiles.
   a.num_n_tiles = d / (2 * BM);
   if (conv_state != nullptr) {
     a.m_stride = BN;
     a.m_offset = 0;
   } else {
-    a.m_stride = BN - HALO;
-    a.m_offset = -HALO;
+    a.m_stride = BN - halo;
+    a.m_offset = -halo;
   }
   a.num_m_tiles = (int)((N + a.m_stride - 1) / a.m_stride);
+  constexpr int D3 = MODE_V_DILATED;
   if (conv_state != nullptr)
-    return launch_pass<BN, STAGES_V, MODE_VALUE_DECODE, KCH>(ta_v, tb_v, th, to, to29, to, to29, a,
-                                                             s, true);
+    return dil == 3 ? launch_pass<BN, STAGES_V, MODE_VALUE_DECODE | D3, KCH>(
+                          ta_v, tb_v, th, to, to29, to, to29, a, s, true)
+                    : launch_pass<BN, STAGES_V, MODE_VALUE_DECODE, KCH>(ta_v, tb_v, th, to, to29, to,
+                                                                        to29, a, s, true);
   if (a.kv_save != nullptr) {
     // v into the saved [k | v] rows: boxes of 32 features x 32 tokens, and a
-    // 29-token box that skips a tile's conv halo
+    // shorter box that skips a tile's conv halo
     CUtensorMap tv, tv29;
     if (!make_tmap_f32(&tv, a.kv_save, (uint64_t)(2 * d), (uint64_t)N, 32, 32,
                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_tmap_f32(&tv29, a.kv_save, (uint64_t)(2 * d), (uint64_t)N, 32, 32 - HALO,
+        !make_tmap_f32(&tv29, a.kv_save, (uint64_t)(2 * d), (uint64_t)N, 32, 32 - halo,
                        CU_TENSOR_MAP_SWIZZLE_NONE))
       return ENGRAM_ERR_CUDA;
-    return launch_pass<BN, STAGES_VKV, MODE_VALUE_CONV_KV, KCH>(ta_v, tb_v, th, to, to29, tv, tv29,
-                                                                a, s, true);
+    return dil == 3 ? launch_pass<BN, STAGES_VKV, MODE_VALUE_CONV_KV | D3, KCH>(
+                          ta_v, tb_v, th, to, to29, tv, tv29, a, s, true)
+                    : launch_pass<BN, STAGES_VKV, MODE_VALUE_CONV_KV, KCH>(ta_v, tb_v, th, to, to29,
+                                                                           tv, tv29, a, s, true);
   }
-  return launch_pass<BN, STAGES_V, MODE_VALUE_CONV, KCH>(ta_v, tb_v, th, to, to29, to, to29, a, s,
-                                                         true);
+  return dil == 3 ? launch_pass<BN, STAGES_V, MODE_VALUE_CONV | D3, KCH>(ta_v, tb_v, th, to, to29,
+                                                                         to, to29, a, s, true)
+                  : launch_pass<BN, STAGES_V, MODE_VALUE_CONV, KCH>(ta_v, tb_v, th, to, to29, to,
+                                                                    to29, a, s, true);
 }
 
 inline bool use_wide(int64_t N, int d) { return d % 256 == 0 && N > 4096; }
@@ -1337,8 +1405,8 @@ size_t tc_forward_ws_bytes(int64_t N, int d, int E) {
 int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
                       __nv_bfloat16* out, float* alpha_saved, float* kv_save, const float* gg,
-                      int64_t N, int T, int d, int E, void* ws, size_t ws_bytes, bool chained,
-                      cudaStream_t s) {
+                      int dil, int64_t N, int T, int d, int E, void* ws, size_t ws_bytes,
+                      bool chained, cudaStream_t s) {
   if (ws_bytes < tc_forward_ws_bytes(N, d, E) || ws == nullptr) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL - 256) return ENGRAM_ERR_UNSUPPORTED;
   const bool wide = use_wide(N, d);
@@ -1348,14 +1416,14 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
                                           (size_t)N * 2 * (d / BN) * sizeof(float4));
   if (wide)
     return run_layer<256, 6, 5, 4, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
-                                   gg, N, T, d, E, part, alpha, chained, s);
+                                   gg, dil, N, T, d, E, part, alpha, chained, s);
   // few tokens: each CTA streams long operand rows at a rate set by how many
   // bytes one copy instruction brings, so two K chunks go in each box
   if (E % (2 * BK) == 0)
     return run_layer<64, 4, 3, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
-                                  gg, N, T, d, E, part, alpha, chained, s);
+                                  gg, dil, N, T, d, E, part, alpha, chained, s);
   return run_layer<64, 8, 6, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, gg,
-                                N, T, d, E, part, alpha, chained, s);
+                                dil, N, T, d, E, part, alpha, chained, s);
 }
 
 }  // namespace engram

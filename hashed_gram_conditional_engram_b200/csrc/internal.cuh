@@ -142,7 +142,7 @@ int launch_scale_product(const float* gh, const float* gk, int d, float* gg, cud
 int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
                       __nv_bfloat16* out, float* alpha_saved, float* kv_save, const float* gg,
-                      int64_t N, int T, int d, int E, void* ws, size_t ws_bytes, bool chained,
-                      cudaStream_t s);
+                      int dil, int64_t N, int T, int d, int E, void* ws, size_t ws_bytes,
+                      bool chained, cudaStream_t s);
 
 }  // namespace engram

@@ -2,7 +2,8 @@
 per-branch conv, learnable RMSNorm scales) of the fp32 layer with the
 oracle: forward, decode streaming and every gradient, including the
 small-parameter block's, within the fp32 tolerance (1e-5 max relative
-error with a 1e-3 RMS floor); bf16 layers refuse the variants."""
+error with a 1e-3 RMS floor); bf16 layers with the scales and the dilated
+conv against the bf16 metric; bf16 layers refuse the pre-conv norm."""
 import numpy as np
 import pytest
 import torch
@@ -112,7 +113,7 @@ def test_bf16_layers_refuse_the_variants():
     K, D_h, d = 2, 32, 256
     rows = synth.primes_at_most(1009, 2 * K)
     cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
-                      flags=eg.CONV_DILATED)
+                      flags=eg.CONV_PRENORM)
     N, E = 4, 2 * K * D_h
     e = torch.zeros((N, E), dtype=torch.bfloat16, device="cuda")
     h = torch.zeros((N, d), dtype=torch.bfloat16, device="cuda")
@@ -156,3 +157,69 @@ def test_bf16_norm_scales_forward_matches_oracle(N, T):
     assert max_rel_err(out.float().cpu().numpy(), ref["out"]) <= 2e-2
     alpha = saved[: N * 4].view(torch.float32).cpu().numpy()
     assert np.max(np.abs(alpha - ref["alpha"].reshape(-1))) <= 1e-5
+
+
+@pytest.mark.parametrize("B,T,d", [(3, 100, 256), (2, 2500, 512), (40, 7, 256), (1, 4100, 256)])
+def test_bf16_dilated_forward_matches_oracle(B, T, d):
+    """bf16 layer with the dilated conv (taps at t, t-3, t-6, t-9): out within
+    the bf16 metric of the oracle; narrow and wide tiles, sequences shorter
+    than the conv's 9-token history, tile seams (tiles overlap by 9)."""
+    from tests.engram_cases import bf16_dev
+    rng = np.random.default_rng(B * 13 + T)
+    K, D_h = 2, 32
+    E, N = 2 * K * D_h, B * T
+    rows = synth.primes_at_most(1009, 2 * K)
+    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
+                      flags=eg.CONV_DILATED)
+    e = rng.standard_normal((N, E)).astype(np.float32)
+    h = rng.standard_normal((N, 1, d)).astype(np.float32)
+    Wk = (rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32)
+    Wv = (rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32)
+    block = (rng.standard_normal(4 * d) * 0.5).astype(np.float32)
+    out = torch.empty((N, 1, d), dtype=torch.bfloat16, device="cuda")
+    saved = _ws(eg.engram_saved_size(cfg, N))
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+    eg.engram_forward(cfg, None, None, bf16_dev(e), bf16_dev(h), bf16_dev(Wk), bf16_dev(Wv),
+                      dev(block), None, out, saved, B, T, _ws(fb), fb)
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    f64 = O.bf16_bits_to_f64
+    b = synth.to_bf16_bits
+    ref = O.layer_forward_v(f64(b(e)), f64(b(h)), f64(b(Wk)), f64(b(Wv)), block, T,
+                            eg.CONV_DILATED)
+    assert max_rel_err(out.float().cpu().numpy(), ref["out"]) <= 2e-2
+
+
+def test_bf16_dilated_decode_matches_whole_sequences():
+    """Decode steps of a dilated bf16 layer (conv state [B, 1, 9, d], vt of
+    the nine previous steps) against the oracle's whole-sequence forward,
+    each step within the bf16 metric."""
+    from tests.engram_cases import bf16_dev
+    rng = np.random.default_rng(77)
+    B, T, K, D_h, d = 24, 14, 2, 32, 256
+    E = 2 * K * D_h
+    rows = synth.primes_at_most(1009, 2 * K)
+    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
+                      flags=eg.CONV_DILATED)
+    e = rng.standard_normal((B, T, E)).astype(np.float32)
+    h = rng.standard_normal((B, T, 1, d)).astype(np.float32)
+    Wk = (rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32)
+    Wv = (rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32)
+    block = (rng.standard_normal(4 * d) * 0.5).astype(np.float32)
+    f64 = O.bf16_bits_to_f64
+    b = synth.to_bf16_bits
+    ref = O.layer_forward_v(f64(b(e)).reshape(B * T, E), f64(b(h)).reshape(B * T, 1, d),
+                            f64(b(Wk)), f64(b(Wv)), block, T, eg.CONV_DILATED)
+    ref_out = ref["out"].reshape(B, T, 1, d)
+    state = torch.zeros((B, 1, 9, d), device="cuda")
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, B)
+    ws = _ws(fb)
+    Wk_d, Wv_d, blk = bf16_dev(Wk), bf16_dev(Wv), dev(block)
+    out = torch.empty((B, 1, 1, d), dtype=torch.bfloat16, device="cuda")
+    for t in range(T):
+        eg.engram_forward(cfg, None, None, bf16_dev(np.ascontiguousarray(e[:, t])),
+                          bf16_dev(np.ascontiguousarray(h[:, t])), Wk_d, Wv_d, blk, state, out,
+                          None, B, 1, ws, fb)
+        got = out[:, 0].float().cpu().numpy()
+        assert max_rel_err(got, ref_out[:, t]) <= 2e-2, t
+    assert eg.engram_get_status() == 0
