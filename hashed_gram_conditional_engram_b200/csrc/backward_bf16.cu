@@ -118,36 +118,41 @@ __device__ __forceinline__ float2 silu_grad2(float2 y) {
 }
 
 constexpr int COL_TOK = 128;   // tokens per column chunk; one warp walks one chunk
-constexpr int COL_NP = 2;      // feature pairs per lane (2 pairs: one 16-byte load per row)
-constexpr int COL_FEAT = 64 * COL_NP;  // features per warp, one dalpha partial per token
 constexpr int COL_WARPS = 4;   // chunks per block
+constexpr int COL_RING = 12;   // tokens per warp in a shared-memory ring, 11 of them in flight
 
-constexpr int COL_RING = 12;  // tokens per warp in a shared-memory ring, 11 of them in flight
-
+// Features per warp of the walk: NP pairs per lane, 2 for the plain conv, 1
+// for the dilated one (whose 9-token history takes the registers).
+__host__ __device__ constexpr int col_feat(int np_lane) { return 64 * np_lane; }
 // dalpha partials per token, padded to 16 bytes for the row kernel's copies
-__host__ __device__ constexpr int col_partials(int d) { return ((d / COL_FEAT) + 3) & ~3; }
+__host__ __device__ constexpr int col_partials(int d, int np_lane) {
+  return ((d / col_feat(np_lane)) + 3) & ~3;
+}
 
-// A lane's features: COL_NP pairs of adjacent ones.
+// A lane's features: NP pairs of adjacent ones.
+template <int NP>
 struct FPairs {
-  float2 p[COL_NP];
+  float2 p[NP];
 };
 
-__device__ __forceinline__ FPairs ld_pairs(const float* q) {
-  FPairs r;
-  if constexpr (COL_NP == 2) {
+template <int NP>
+__device__ __forceinline__ FPairs<NP> ld_pairs(const float* q) {
+  FPairs<NP> r;
+  if constexpr (NP == 2) {
     const float4 t = *reinterpret_cast<const float4*>(q);
     r.p[0] = make_float2(t.x, t.y);
-    r.p[COL_NP - 1] = make_float2(t.z, t.w);
+    r.p[NP - 1] = make_float2(t.z, t.w);
   } else {
     r.p[0] = *reinterpret_cast<const float2*>(q);
   }
   return r;
 }
 
-// Asynchronous copy of a lane's features (8 * COL_NP bytes), global -> its
-// own shared-memory slot.
+// Asynchronous copy of a lane's features (8 NP bytes), global -> its own
+// shared-memory slot.
+template <int NP>
 __device__ __forceinline__ void cp_async_pairs(void* dst, const void* src) {
-  if constexpr (COL_NP == 2) {
+  if constexpr (NP == 2) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
                      (uint32_t)__cvta_generic_to_shared(dst)),
                  "l"(src)
@@ -192,21 +197,22 @@ __device__ __forceinline__ void col_flush(ColPartials& pb, int jbase, int cnt, i
 // Emit token j of the walk: dv = alpha dvt (the lane's features, bf16), and
 // the lane's share of dalpha = <dvt, v>; every 32nd token flushes the warp's
 // partials.  Tokens are emitted once each, in increasing order.
-__device__ __forceinline__ void col_emit(const FPairs& r, const FPairs& vv, float a, int j, int ld,
-                                         int np, __nv_bfloat16* __restrict__ dvb, ColPartials& pb,
-                                         float* __restrict__ pab) {
-  __nv_bfloat162 o[COL_NP];
+template <int NP>
+__device__ __forceinline__ void col_emit(const FPairs<NP>& r, const FPairs<NP>& vv, float a,
+                                         int j, int ld, int np, __nv_bfloat16* __restrict__ dvb,
+                                         ColPartials& pb, float* __restrict__ pab) {
+  __nv_bfloat162 o[NP];
   float dot = 0.f;
 #pragma unroll
-  for (int q = 0; q < COL_NP; ++q) {
+  for (int q = 0; q < NP; ++q) {
     const float2 dvr = __fmul2_rn(make_float2(a, a), r.p[q]);
     o[q] = __floats2bfloat162_rn(dvr.x, dvr.y);
     dot = fmaf(r.p[q].x, vv.p[q].x, fmaf(r.p[q].y, vv.p[q].y, dot));
   }
-  if constexpr (COL_NP == 2) {
+  if constexpr (NP == 2) {
     uint2 w;
     w.x = *reinterpret_cast<const uint32_t*>(&o[0]);
-    w.y = *reinterpret_cast<const uint32_t*>(&o[COL_NP - 1]);
+    w.y = *reinterpret_cast<const uint32_t*>(&o[NP - 1]);
     *reinterpret_cast<uint2*>(dvb + j * ld) = w;
   } else {
     *reinterpret_cast<__nv_bfloat162*>(dvb + j * ld) = o[0];
@@ -216,98 +222,105 @@ __device__ __forceinline__ void col_emit(const FPairs& r, const FPairs& vv, floa
 }
 
 // dynamic shared memory of the column walk: per warp the copy ring, the
-// dalpha partials and the chunk's gates
-constexpr int kColSmem = COL_WARPS * (COL_RING * 2 * 32 * (int)sizeof(FPairs) +
-                                      (int)sizeof(ColPartials) + (COL_TOK + 6) * 4);
+// dalpha partials and the chunk's gates (with DIL * 3 tokens on each side)
+template <int DIL, int NP>
+constexpr int col_smem_bytes() {
+  return COL_WARPS * (COL_RING * 2 * 32 * (int)sizeof(FPairs<NP>) + (int)sizeof(ColPartials) +
+                      (COL_TOK + 6 * DIL) * 4);
+}
 
-// One warp per (chunk of COL_TOK tokens, COL_FEAT features), each lane
-// holding COL_NP pairs of adjacent features, walking the chunk in token
-// order.  The warp keeps, for the three previous tokens, vt and v, and the
-// partial sums of their dvt: dvt_s = u_s + w_3 dy_s + w_2 dy_{s+1} +
-// w_1 dy_{s+2} + w_0 dy_{s+3} (terms past the sequence end absent), to which
-// each new dy_t adds its share.  At token t it forms y_t and dy_t; dvt of
-// token t-3 is then complete, and at a sequence end so are t-2, t-1 and t.
-// The walk runs 3 tokens past the chunk for the last tokens' dy.  v and dout
-// of the next COL_RING - 1 tokens are in flight into a per-warp
-// shared-memory ring (asynchronous copies, each lane its own bytes), enough
-// bytes in flight per SM to stream at HBM rate.  `live` counts the ring's
+// One warp per (chunk of COL_TOK tokens, 64 NP features), each lane holding
+// NP pairs of adjacent features, walking the chunk in token order; the conv
+// reads y_t = sum_i w_i vt_{t-(3-i) DIL}.  The warp keeps, for the NH = 3 DIL
+// previous tokens, vt and v, and the partial sums of their dvt:
+// dvt_s = u_s + w_3 dy_s + w_2 dy_{s+DIL} + w_1 dy_{s+2 DIL} + w_0 dy_{s+3 DIL}
+// (terms past the sequence end absent), to which each new dy_t adds its
+// share.  At token t it forms y_t and dy_t; dvt of token t-NH is then
+// complete, and at a sequence end so are all later ones.  The walk runs NH
+// tokens past the chunk for the last tokens' dy.  v and dout of the next
+// COL_RING - 1 tokens are in flight into a per-warp shared-memory ring
+// (asynchronous copies, each lane its own bytes).  `live` counts the ring's
 // tokens that belong to t's sequence and to this chunk's walk (tokens before
 // the chunk are emitted by the previous chunk's walk).  For each completed
 // token it writes dv (bf16, for the GEMMs) and the warp's partial of dalpha,
-// dalpha_part[token][f / COL_FEAT] (the lanes' shares summed per 32 tokens,
+// dalpha_part[token][f / (64 NP)] (the lanes' shares summed per 32 tokens,
 // from shared memory, in lane order); at the end the chunk's partial
 // conv-weight gradient, part[chunk][f] = sum over its tokens of
-// dy_t * (vt_{t-3}, vt_{t-2}, vt_{t-1}, vt_t).  The arithmetic runs on packed
-// fp32 pairs.  Warps are independent (all lanes of one walk the same tokens,
-// so the branches are uniform); the block only groups COL_WARPS chunks for
-// scheduling.
+// dy_t * (vt_{t-3 DIL}, vt_{t-2 DIL}, vt_{t-DIL}, vt_t).  The arithmetic runs
+// on packed fp32 pairs.  Warps are independent (all lanes of one walk the
+// same tokens, so the branches are uniform); the block only groups COL_WARPS
+// chunks for scheduling.
+template <int DIL, int NP>
 __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     const float* __restrict__ v, const float* __restrict__ alpha,
     const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
     int ld, int chunks, __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part,
     float4* __restrict__ part) {
   // v and dv rows are ld apart (they share rows with k and dk), dout rows d
+  using FP = FPairs<NP>;
+  constexpr int NH = 3 * DIL;
   extern __shared__ __align__(16) unsigned char col_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int RING_BYTES = COL_RING * 2 * 32 * (int)sizeof(FPairs);
-  auto* ring_all = reinterpret_cast<FPairs(*)[COL_RING][2][32]>(col_smem);  // [slot][v, dout][lane]
+  constexpr int RING_BYTES = COL_RING * 2 * 32 * (int)sizeof(FP);
+  auto* ring_all = reinterpret_cast<FP(*)[COL_RING][2][32]>(col_smem);  // [slot][v, dout][lane]
   auto* pb_all = reinterpret_cast<ColPartials*>(col_smem + COL_WARPS * RING_BYTES);
-  auto* al_all = reinterpret_cast<float(*)[COL_TOK + 6]>(col_smem + COL_WARPS * RING_BYTES +
-                                                          COL_WARPS * sizeof(ColPartials));
+  auto* al_all = reinterpret_cast<float(*)[COL_TOK + 2 * NH]>(col_smem + COL_WARPS * RING_BYTES +
+                                                               COL_WARPS * sizeof(ColPartials));
   ColPartials& pb = pb_all[warp];
   const int chunk = blockIdx.x * COL_WARPS + warp;
   if (chunk >= chunks) return;  // no block-wide barrier follows
-  const int f = blockIdx.y * COL_FEAT + lane * 2 * COL_NP;
-  const int np = col_partials(d);
+  const int f = blockIdx.y * col_feat(NP) + lane * 2 * NP;
+  const int np = col_partials(d, NP);
   const int64_t t0 = (int64_t)chunk * COL_TOK;
   const int64_t t1 = t0 + COL_TOK < N ? t0 + COL_TOK : N;
-  const int64_t t_stop = t1 + 3 < N ? t1 + 3 : N;
-  // the gates of the walk's tokens and the 3 before it: al_s[tt - t0 + 3]
+  const int64_t t_stop = t1 + NH < N ? t1 + NH : N;
+  // the gates of the walk's tokens and the NH before it: al_s[tt - t0 + NH]
   float* al_s = al_all[warp];
-  for (int i = lane; i < COL_TOK + 6; i += 32) {
-    const int64_t tt = t0 - 3 + i;
+  for (int i = lane; i < COL_TOK + 2 * NH; i += 32) {
+    const int64_t tt = t0 - NH + i;
     al_s[i] = (tt >= 0 && tt < t_stop) ? alpha[tt] : 0.f;
   }
   __syncwarp();
-  // the weights as (feature x, feature y) pairs: W0 multiplies vt_{t-3}, W3 vt_t
-  FPairs W0, W1, W2, W3;
+  // the weights as (feature x, feature y) pairs: W0 multiplies vt_{t-NH}, W3 vt_t
+  FP W0, W1, W2, W3;
 #pragma unroll
-  for (int q = 0; q < COL_NP; ++q) {
+  for (int q = 0; q < NP; ++q) {
     const float4 wx = __ldg(conv_w + f + 2 * q), wy = __ldg(conv_w + f + 2 * q + 1);
     W0.p[q] = make_float2(wx.x, wy.x);
     W1.p[q] = make_float2(wx.y, wy.y);
     W2.p[q] = make_float2(wx.z, wy.z);
     W3.p[q] = make_float2(wx.w, wy.w);
   }
-  const FPairs zero = {};
+  const FP zero = {};
   int pos = (int)(t0 % T);
-  FPairs s1 = zero, s2 = zero, s3 = zero;  // vt of t-1, t-2, t-3
-  auto vt_of = [&](int64_t tt, float a) {
-    FPairs q = ld_pairs(v + tt * ld + f);
+  // rings over the NH previous tokens: index k holds token t-1-k
+  FP sr[NH], ar[NH], vr_[NH];  // vt, partial dvt, v
 #pragma unroll
-    for (int k = 0; k < COL_NP; ++k) q.p[k] = __fmul2_rn(make_float2(a, a), q.p[k]);
-    return q;
-  };
-  if (pos >= 1) s1 = vt_of(t0 - 1, al_s[2]);
-  if (pos >= 2) s2 = vt_of(t0 - 2, al_s[1]);
-  if (pos >= 3) s3 = vt_of(t0 - 3, al_s[0]);
-  FPairs A1 = zero, A2 = zero, A3 = zero;  // partial dvt of t-1, t-2, t-3
-  FPairs v1 = zero, v2 = zero, v3 = zero;  // v of t-1, t-2, t-3
-  FPairs C0 = zero, C1 = zero, C2 = zero, C3 = zero;  // conv-weight partials for w_0 .. w_3
+  for (int k = 0; k < NH; ++k) {
+    sr[k] = ar[k] = vr_[k] = zero;
+    if (pos >= k + 1) {  // the token lies in this sequence
+      FP q = ld_pairs<NP>(v + (t0 - 1 - k) * ld + f);
+      const float a = al_s[NH - 1 - k];
+#pragma unroll
+      for (int j = 0; j < NP; ++j) q.p[j] = __fmul2_rn(make_float2(a, a), q.p[j]);
+      sr[k] = q;
+    }
+  }
+  FP C0 = zero, C1 = zero, C2 = zero, C3 = zero;  // conv-weight partials for w_0 .. w_3
   int live = 0;
   __nv_bfloat16* dvb = dv + t0 * ld + f;
   float* pab = dalpha_part + t0 * np + blockIdx.y;
   const int n_chunk = (int)(t1 - t0), n_walk = (int)(t_stop - t0);
   // token q's v and dout go to ring slot q % COL_RING; the slot refilled at
   // step i held token i - 1, whose values step i - 1 has already used
-  FPairs (*ring)[2][32] = ring_all[warp];
+  FP (*ring)[2][32] = ring_all[warp];
   const float* vp = v + t0 * ld + f;
   const float* up = dout + t0 * d + f;
 #pragma unroll
   for (int q = 0; q < COL_RING - 1; ++q) {
     if (q < n_walk) {
-      cp_async_pairs(&ring[q][0][lane], vp);
-      cp_async_pairs(&ring[q][1][lane], up);
+      cp_async_pairs<NP>(&ring[q][0][lane], vp);
+      cp_async_pairs<NP>(&ring[q][1][lane], up);
     }
     cp_async_commit();
     vp += ld;
@@ -317,64 +330,67 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
   for (int i = 0; i < n_walk; ++i) {
     cp_async_wait<COL_RING - 2>();  // token i's copies have landed
     const int slot = i % COL_RING;
-    const FPairs vr = ring[slot][0][lane], ut = ring[slot][1][lane];
-    const float at = al_s[i + 3];
+    const FP vr = ring[slot][0][lane], ut = ring[slot][1][lane];
+    const float at = al_s[i + NH];
     if (i + COL_RING - 1 < n_walk) {
       const int refill = (i + COL_RING - 1) % COL_RING;
-      cp_async_pairs(&ring[refill][0][lane], vp);
-      cp_async_pairs(&ring[refill][1][lane], up);
+      cp_async_pairs<NP>(&ring[refill][0][lane], vp);
+      cp_async_pairs<NP>(&ring[refill][1][lane], up);
     }
     cp_async_commit();
     vp += ld;
     up += d;
     if (pos == 0) {  // a sequence starts at t
-      s1 = s2 = s3 = zero;
+#pragma unroll
+      for (int k = 0; k < NH; ++k) sr[k] = zero;
       live = 0;
     }
-    FPairs vt, g, E3, B2, B1, B0;
+    FP vt, g, E, A0;
 #pragma unroll
-    for (int q = 0; q < COL_NP; ++q) {
+    for (int q = 0; q < NP; ++q) {
       vt.p[q] = __fmul2_rn(make_float2(at, at), vr.p[q]);
-      const float2 y = __ffma2_rn(W0.p[q], s3.p[q],
-                                  __ffma2_rn(W1.p[q], s2.p[q],
-                                             __ffma2_rn(W2.p[q], s1.p[q],
-                                                        __fmul2_rn(W3.p[q], vt.p[q]))));
+      const float2 y =
+          __ffma2_rn(W0.p[q], sr[NH - 1].p[q],
+                     __ffma2_rn(W1.p[q], sr[2 * DIL - 1].p[q],
+                                __ffma2_rn(W2.p[q], sr[DIL - 1].p[q], __fmul2_rn(W3.p[q], vt.p[q]))));
       g.p[q] = __fmul2_rn(ut.p[q], silu_grad2(y));
-      E3.p[q] = __ffma2_rn(W0.p[q], g.p[q], A3.p[q]);  // dvt of t-3, complete
-      B2.p[q] = __ffma2_rn(W1.p[q], g.p[q], A2.p[q]);
-      B1.p[q] = __ffma2_rn(W2.p[q], g.p[q], A1.p[q]);
-      B0.p[q] = __ffma2_rn(W3.p[q], g.p[q], ut.p[q]);
+      E.p[q] = __ffma2_rn(W0.p[q], g.p[q], ar[NH - 1].p[q]);  // dvt of t-NH, complete
+      ar[2 * DIL - 1].p[q] = __ffma2_rn(W1.p[q], g.p[q], ar[2 * DIL - 1].p[q]);
+      ar[DIL - 1].p[q] = __ffma2_rn(W2.p[q], g.p[q], ar[DIL - 1].p[q]);
+      A0.p[q] = __ffma2_rn(W3.p[q], g.p[q], ut.p[q]);
     }
     if (i < n_chunk) {
 #pragma unroll
-      for (int q = 0; q < COL_NP; ++q) {
-        C0.p[q] = __ffma2_rn(g.p[q], s3.p[q], C0.p[q]);
-        C1.p[q] = __ffma2_rn(g.p[q], s2.p[q], C1.p[q]);
-        C2.p[q] = __ffma2_rn(g.p[q], s1.p[q], C2.p[q]);
+      for (int q = 0; q < NP; ++q) {
+        C0.p[q] = __ffma2_rn(g.p[q], sr[NH - 1].p[q], C0.p[q]);
+        C1.p[q] = __ffma2_rn(g.p[q], sr[2 * DIL - 1].p[q], C1.p[q]);
+        C2.p[q] = __ffma2_rn(g.p[q], sr[DIL - 1].p[q], C2.p[q]);
         C3.p[q] = __ffma2_rn(g.p[q], vt.p[q], C3.p[q]);
       }
     }
-    if (live == 3) col_emit(E3, v3, al_s[i], i - 3, ld, np, dvb, pb, pab);  // token t-3
-    if (pos == T - 1) {  // the sequence ends at t: its last tokens are complete
-      if (live >= 2 && i - 2 < n_chunk) col_emit(B2, v2, al_s[i + 1], i - 2, ld, np, dvb, pb, pab);
-      if (live >= 1 && i - 1 < n_chunk) col_emit(B1, v1, al_s[i + 2], i - 1, ld, np, dvb, pb, pab);
-      if (i < n_chunk) col_emit(B0, vr, at, i, ld, np, dvb, pb, pab);
+    if (live == NH) col_emit<NP>(E, vr_[NH - 1], al_s[i], i - NH, ld, np, dvb, pb, pab);
+    if (pos == T - 1) {  // the sequence ends at t: its later tokens are complete
+#pragma unroll
+      for (int k = NH - 1; k >= 1; --k)  // tokens t-k, oldest first
+        if (live >= k && i - k < n_chunk)
+          col_emit<NP>(ar[k - 1], vr_[k - 1], al_s[i + NH - k], i - k, ld, np, dvb, pb, pab);
+      if (i < n_chunk) col_emit<NP>(A0, vr, at, i, ld, np, dvb, pb, pab);
     }
-    A3 = B2;
-    A2 = B1;
-    A1 = B0;
-    s3 = s2;
-    s2 = s1;
-    s1 = vt;
-    v3 = v2;
-    v2 = v1;
-    v1 = vr;
-    live = live < 3 ? live + 1 : 3;
+#pragma unroll
+    for (int k = NH - 1; k > 0; --k) {
+      ar[k] = ar[k - 1];
+      sr[k] = sr[k - 1];
+      vr_[k] = vr_[k - 1];
+    }
+    ar[0] = A0;
+    sr[0] = vt;
+    vr_[0] = vr;
+    live = live < NH ? live + 1 : NH;
     pos = pos + 1 == T ? 0 : pos + 1;
   }
   if (n_chunk & 31) col_flush(pb, n_chunk & ~31, n_chunk & 31, np, pab);
 #pragma unroll
-  for (int q = 0; q < COL_NP; ++q) {
+  for (int q = 0; q < NP; ++q) {
     part[(int64_t)chunk * d + f + 2 * q] =
         make_float4(C0.p[q].x, C1.p[q].x, C2.p[q].x, C3.p[q].x);
     part[(int64_t)chunk * d + f + 2 * q + 1] =
@@ -432,10 +448,10 @@ __device__ __forceinline__ bool row_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Shared memory of one stage of the row kernel: the token's h (bf16), k and
-// dout (fp32) rows and its dalpha partials (d/128, padded to a multiple of
-// 4); all offsets are multiples of 16 bytes because d is a multiple of 256.
-__host__ __device__ constexpr size_t row_stage_bytes(int d) {
-  return (size_t)d * 2 + (size_t)d * 4 + (size_t)d * 4 + (size_t)col_partials(d) * 4;
+// dout (fp32) rows and its np_pad dalpha partials (a multiple of 4); all
+// offsets are multiples of 16 bytes because d is a multiple of 256.
+__host__ __device__ constexpr size_t row_stage_bytes(int d, int np_pad) {
+  return (size_t)d * 2 + (size_t)d * 4 + (size_t)d * 4 + (size_t)np_pad * 4;
 }
 
 // The gate and both RMSNorm backwards need whole-row sums, so each token is
@@ -443,8 +459,8 @@ __host__ __device__ constexpr size_t row_stage_bytes(int d) {
 // + gridDim.x, ..., with the next token's rows already in flight into the
 // other shared-memory stage (bulk copies issued by one thread, completing on
 // an mbarrier).  Each thread takes 4 features per item from shared memory
-// into registers; <h,h>, <k,k>, <h,k> and dalpha (the column walk's d/128
-// partials, added in order by the first warp) are reduced together in one
+// into registers; <h,h>, <k,k>, <h,k> and dalpha (the column walk's np
+// partials per token, rows np_pad apart, added by the first warp) are reduced together in one
 // fixed-order pass, whose barrier also frees the stage for the token after
 // next; then dk (bf16, for the GEMMs) and dh are written.  A copy that never
 // lands sets ENGRAM_STATUS_TIMEOUT and the block stops.
@@ -457,16 +473,15 @@ template <int ITEMS, bool SCALED>  // ITEMS = ceil(d / (ROW_THREADS * ROW_VEC)) 
 __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     const __nv_bfloat16* __restrict__ h, const float* __restrict__ k,
     const float* __restrict__ alpha, const float* __restrict__ dout,
-    const float* __restrict__ dalpha_part, const float* __restrict__ gscale, int64_t N, int d,
-    int ld, float* __restrict__ dh, __nv_bfloat16* __restrict__ dk_out,
+    const float* __restrict__ dalpha_part, int np, int np_pad, const float* __restrict__ gscale,
+    int64_t N, int d, int ld, float* __restrict__ dh, __nv_bfloat16* __restrict__ dk_out,
     float* __restrict__ spart, unsigned int* status) {
   // k and dk rows are ld apart (they share rows with v and dv)
   extern __shared__ __align__(128) unsigned char row_smem[];
   __shared__ uint64_t full[ROW_STAGES];
   __shared__ float4 red[2][ROW_THREADS / 32];
   __shared__ int abort_flag;
-  const int np = d / COL_FEAT, np_pad = col_partials(d);
-  const size_t SB = row_stage_bytes(d);
+  const size_t SB = row_stage_bytes(d, np_pad);
   const uint32_t hb_bytes = (uint32_t)d * 2, f_bytes = (uint32_t)d * 4,
                  p_bytes = (uint32_t)np_pad * 4;
   const int64_t G = gridDim.x;
@@ -683,7 +698,7 @@ __global__ void __launch_bounds__(32 * DCONV_WARPS) bw_dconv_reduce_kernel(
 }
 
 // Workspace: [k | v] fp32 [N, 2d]; [dk | dv] bf16 [N, 2d]; [W_k; W_v] bf16
-// and [dW_k; dW_v] fp32 [2d, E]; dalpha partials [N, d/128 padded to 4]; de fp32 [N, E]
+// and [dW_k; dW_v] fp32 [2d, E]; dalpha partials [N, up to d/64 padded to 4]; de fp32 [N, E]
 // when the caller passes none; conv partials; cuBLAS's workspace; the table
 // gradient's sort buffers.
 struct BwdBf16Ws {
@@ -713,7 +728,7 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
   const size_t KV = kv_saved ? 0 : up256b((size_t)N * 2 * d * 4);
   const size_t DKV = up256b((size_t)N * 2 * d * 2);
   const size_t WKV = up256b((size_t)2 * d * E * 2), DW = up256b((size_t)2 * d * E * 4);
-  const size_t DA = up256b((size_t)N * col_partials(d) * 4);
+  const size_t DA = up256b((size_t)N * col_partials(d, 1) * 4);  // the most partials
   const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
   const size_t tg = table_grad_ws_bytes(N * J);
   const size_t SP = scaled ? up256b((size_t)kMaxRowBlocks * d * 4) : 0;
@@ -753,8 +768,8 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
                          const float* alpha, const float* kv_saved, const float* dout, float* dh,
                          float* dWk,
                          float* dWv, float* dconv_w, float* de, int64_t* dtab_keys,
-                         float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, void* ws,
-                         size_t ws_bytes, cudaStream_t s) {
+                         float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, int dil,
+                         void* ws, size_t ws_bytes, cudaStream_t s) {
   const int E = hp.E;
   const bool have_kv = kv_saved != nullptr;
   const bool scaled = gscale != nullptr;
@@ -762,7 +777,8 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
     return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
   // a row in registers; whole column blocks; 16-byte multiples for the row copies
-  if (d > ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS || d % 256 != 0) return ENGRAM_ERR_UNSUPPORTED;
+  if (d > ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS || d % 256 != 0 || (dil != 1 && dil != 3))
+    return ENGRAM_ERR_UNSUPPORTED;
   BwdBf16Ws w;
   bwd_bf16_layout(ws, N, d, E, hp.J, have_kv, scaled, &w);
   if (de == nullptr) de = w.de;
@@ -780,13 +796,19 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
     return rc;
   const float* kv = have_kv ? kv_saved : w.kv;
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
-  if ((rc = ck(cudaFuncSetAttribute(bw_col_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kColSmem))))
-    return rc;
-  bw_col_kernel<<<dim3((unsigned)((chunks + COL_WARPS - 1) / COL_WARPS), (unsigned)(d / COL_FEAT)),
-                  32 * COL_WARPS, kColSmem, s>>>(kv + d, alpha, reinterpret_cast<const float4*>(conv_w),
-                                          dout, N, T, d, 2 * d, chunks, w.dkv + d,
-                                          w.dalpha_part, w.part);
+  // the plain conv walks two feature pairs per lane, the dilated one (nine
+  // tokens of history in registers) one
+  const int np_lane = dil == 1 ? 2 : 1;
+  const int np = d / col_feat(np_lane), np_pad = col_partials(d, np_lane);
+  {
+    auto col = dil == 1 ? bw_col_kernel<1, 2> : bw_col_kernel<3, 1>;
+    const int smem = dil == 1 ? col_smem_bytes<1, 2>() : col_smem_bytes<3, 1>();
+    if ((rc = ck(cudaFuncSetAttribute(col, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))))
+      return rc;
+    col<<<dim3((unsigned)((chunks + COL_WARPS - 1) / COL_WARPS), (unsigned)np), 32 * COL_WARPS,
+          smem, s>>>(kv + d, alpha, reinterpret_cast<const float4*>(conv_w), dout, N, T, d, 2 * d,
+                     chunks, w.dkv + d, w.dalpha_part, w.part);
+  }
   {
     const int items = (d / ROW_VEC + ROW_THREADS - 1) / ROW_THREADS;
     auto row = scaled ? (items == 1 ? bw_row_kernel<1, true>
@@ -795,7 +817,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
                       : (items == 1 ? bw_row_kernel<1, false>
                          : items == 2 ? bw_row_kernel<2, false>
                          : items == 3 ? bw_row_kernel<3, false> : bw_row_kernel<4, false>);
-    const int smem = (int)(ROW_STAGES * row_stage_bytes(d));
+    const int smem = (int)(ROW_STAGES * row_stage_bytes(d, np_pad));
     int dev = 0, sms = 0, per_sm = 0;
     if ((rc = ck(cudaFuncSetAttribute(row, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) ||
         (rc = ck(cudaGetDevice(&dev))) ||
@@ -804,8 +826,9 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
       return rc;
     int64_t grid = std::min<int64_t>(N, (int64_t)sms * std::max(per_sm, 1));
     if (scaled) grid = std::min<int64_t>(grid, kMaxRowBlocks);
-    row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, kv, alpha, dout, w.dalpha_part, gscale, N, d,
-                                                  2 * d, dh, w.dkv, w.spart, status_ptr());
+    row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, kv, alpha, dout, w.dalpha_part, np, np_pad,
+                                                  gscale, N, d, 2 * d, dh, w.dkv, w.spart,
+                                                  status_ptr());
     if (scaled)
       bw_scale_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(
           w.spart, (int)grid, d, gscale, dconv_w + 4 * (int64_t)d);

@@ -238,8 +238,7 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                     void* ws, size_t ws_bytes, void* stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (cfg->dtype == ENGRAM_BF16 && (cfg->n_branch != 1 || !bf16_variant_ok(cfg) ||
-                                    (cfg->flags & ENGRAM_CONV_DILATED) != 0))
+  if (cfg->dtype == ENGRAM_BF16 && (cfg->n_branch != 1 || !bf16_variant_ok(cfg)))
     return ENGRAM_ERR_UNSUPPORTED;
   if (cfg->dtype == ENGRAM_BF16 && saved == nullptr) return ENGRAM_ERR_INVALID_ARG;
   if (B < 0 || T < 0) return ENGRAM_ERR_INVALID_ARG;
@@ -276,7 +275,8 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                                 static_cast<const bf*>(Wk), static_cast<const bf*>(Wv), conv_w,
                                 bf16_scaled(cfg) ? conv_w + 4 * d : nullptr, saved, kv_saved,
                                 dout, dh, dWk, dWv, dconv_w, de, dtab_keys, dtab_rows, n_unique,
-                                N, T, d, ws, ws_bytes, s);
+                                N, T, d, (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1, ws,
+                                ws_bytes, s);
   }
   const size_t bw = backward_f32_ws_bytes(N, M, d, E);
   // de lives in the dense-backward workspace unless the caller wants it

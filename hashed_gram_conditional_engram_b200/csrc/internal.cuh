@@ -125,14 +125,14 @@ int launch_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_
 // kv_saved: the forward's fp32 [N, 2d] k and v, or NULL to recompute them
 size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved, bool scaled);
 // gscale: the learnable norm scales g_h [d], g_k [d] (NULL: none); their
-// gradients go to dconv_w + 4 d
+// gradients go to dconv_w + 4 d.  dil: the conv's dilation, 1 or 3
 int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bfloat16* e,
                          const __nv_bfloat16* h, const __nv_bfloat16* Wk,
                          const __nv_bfloat16* Wv, const float* conv_w, const float* gscale,
                          const float* alpha, const float* kv_saved, const float* dout, float* dh,
                          float* dWk, float* dWv, float* dconv_w, float* de, int64_t* dtab_keys,
-                         float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, void* ws,
-                         size_t ws_bytes, cudaStream_t s);
+                         float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, int dil,
+                         void* ws, size_t ws_bytes, cudaStream_t s);
 
 // bf16 tensor-core path (sm_100a tcgen05)
 size_t tc_forward_ws_bytes(int64_t N, int d, int E);

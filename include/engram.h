@@ -59,9 +59,10 @@ enum { ENGRAM_F32 = 0, ENGRAM_BF16 = 1 };
 /* formulation variants: the pages fix neither the conv's dilation, nor a
  * norm before it, nor whether branches share it, nor learnable norm scales
  * ([p2] short depthwise causal conv; [p5 二.1 (2)] 一维卷积; [p5 二.2]).  fp32
- * layers take any combination; bf16 layers take ENGRAM_NORM_SCALES and
- * ENGRAM_CONV_PER_BRANCH (with their one branch the same as a shared conv)
- * and return ENGRAM_ERR_UNSUPPORTED for the other two. */
+ * layers take any combination; bf16 layers take ENGRAM_CONV_DILATED,
+ * ENGRAM_NORM_SCALES and ENGRAM_CONV_PER_BRANCH (with their one branch the
+ * same as a shared conv) and return ENGRAM_ERR_UNSUPPORTED for
+ * ENGRAM_CONV_PRENORM. */
 #define ENGRAM_CONV_DILATED 2     /* taps at t, t-3, t-6, t-9 (dilation 3 = the largest order) */
 #define ENGRAM_CONV_PRENORM 4     /* the conv reads RMSNorm(vt) (times g_v with NORM_SCALES) */
 #define ENGRAM_CONV_PER_BRANCH 8  /* conv weights per branch */
@@ -104,7 +105,8 @@ enum {
  *            less in the backward.
  *            ENGRAM_CONV_DILATED, ENGRAM_CONV_PRENORM, ENGRAM_CONV_PER_BRANCH,
  *            ENGRAM_NORM_SCALES: formulation variants (fp32 layers: any
- *            combination; bf16 layers: the last two).  z = <RMSNorm(h) g_h, RMSNorm(k) g_k> / sqrt(d),
+ *            combination; bf16 layers: all but PRENORM).
+ *            z = <RMSNorm(h) g_h, RMSNorm(k) g_k> / sqrt(d),
  *            vt = alpha v, c = RMSNorm(vt) g_v (PRENORM) or vt,
  *            y_t = sum_i w[:, i] c_{t-(3-i) dil} (dil 3 with DILATED, else 1),
  *            out = h + vt + SiLU(y); each branch m has its own w (PER_BRANCH)

@@ -208,10 +208,12 @@ def _bf16_backward_case(B, T, d, K, D_h, seed, flags=0, with_layer=False):
     f64 = O.bf16_bits_to_f64
     e_ref = f64(O.gather(idx, [synth.to_bf16_bits(t) for t in tables]))
     assert np.array_equal(bf16_bits(L.e), O.gather(idx, [synth.to_bf16_bits(t) for t in tables]))
-    if flags & eg.NORM_SCALES:
+    vflags = ((O.NORM_SCALES if flags & eg.NORM_SCALES else 0) |
+              (O.CONV_DILATED if flags & eg.CONV_DILATED else 0))
+    if vflags:
         ref = O.layer_backward_v(e_ref, f64(synth.to_bf16_bits(h)).reshape(N, 1, d),
                                  f64(synth.to_bf16_bits(Wk)), f64(synth.to_bf16_bits(Wv)), block,
-                                 T, dout, O.NORM_SCALES)
+                                 T, dout, vflags)
         ref["dconv_w"] = ref["dblock"]
     else:
         ref = O.layer_backward(e_ref, f64(synth.to_bf16_bits(h)).reshape(N, 1, d),
@@ -275,6 +277,22 @@ def test_backward_bf16_norm_scales_match_oracle(B, T, d, flags):
     scales' gradients (after the conv weights' in dconv_w) are held with dh
     to the bf16 metric."""
     _check_bf16_backward(*_bf16_backward_case(B, T, d, 2, 32, seed=B * 7 + T, flags=flags))
+
+
+@pytest.mark.parametrize("B,T,d,flags", [
+    (3, 100, 256, eg.CONV_DILATED),                 # narrow forward tiles
+    (2, 2500, 512, eg.CONV_DILATED),                # wide forward tiles, chunks inside sequences
+    (40, 7, 256, eg.CONV_DILATED),                  # sequences shorter than the dilated taps
+    (1, 300, 256, eg.CONV_DILATED | eg.SAVE_KV),    # one sequence over three column chunks
+    (3, 129, 768, eg.CONV_DILATED | eg.NORM_SCALES),
+    (64, 1, 256, eg.CONV_DILATED),                  # one-token sequences
+])
+def test_backward_bf16_dilated_matches_oracle(B, T, d, flags):
+    """The dilated conv (taps 3, 6 and 9 tokens back) on a bf16 layer: the
+    column walk keeps nine tokens of history per feature and completes a
+    token's dvt 9 tokens later (or at its sequence's end); every gradient is
+    held to the same bounds as the plain conv's."""
+    _check_bf16_backward(*_bf16_backward_case(B, T, d, 2, 32, seed=B * 5 + T, flags=flags))
 
 
 def _check_bf16_backward(g, ref, idx, rows, D_h):
