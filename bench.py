@@ -573,16 +573,20 @@ def bench_fwd_bwd_27b(dev, steps=10):
     """Training step of the 27B-shaped layer (8 x 4,096 tokens, d 2,560, 16 x
     80 dims, 5.7B-parameter bf16 table): hash, forward (gather, fused passes,
     alpha, k and v saved), backward (bf16: elementwise kernels, cuBLAS GEMMs,
-    sparse table gradient); and the same with k and v recomputed in the
-    backward instead of saved."""
+    sparse table gradient); the same with k and v recomputed in the
+    backward instead of saved; and with the dilated conv (taps 3, 6 and 9
+    tokens back)."""
+    keys = ("ms_per_step", "fwd_bwd_tokens_per_s", "breakdown_ms")
     kept = _fwd_bwd_27b_run(dev, steps, save_kv=True)
     recomputed = _fwd_bwd_27b_run(dev, steps, save_kv=False)
-    kept["recompute_kv"] = {k: recomputed[k] for k in ("ms_per_step", "fwd_bwd_tokens_per_s",
-                                                       "breakdown_ms")}
+    kept["recompute_kv"] = {k: recomputed[k] for k in keys}
+    from hashed_gram_conditional_engram_b200 import engram as eg
+    dilated = _fwd_bwd_27b_run(dev, steps, save_kv=True, variant=eg.CONV_DILATED)
+    kept["dilated_conv"] = {k: dilated[k] for k in keys}
     return kept
 
 
-def _fwd_bwd_27b_run(dev, steps, save_kv):
+def _fwd_bwd_27b_run(dev, steps, save_kv, variant=0):
     import torch
     from hashed_gram_conditional_engram_b200 import engram as eg
     from hashed_gram_conditional_engram_b200 import synth
@@ -598,7 +602,7 @@ def _fwd_bwd_27b_run(dev, steps, save_kv):
     vb = eg.engram_workspace_size(None, eg.WS_VOCAB, w.V)
     V_c = eg.engram_build_vocab_proj(keys, w.V, proj, torch.empty(vb, dtype=torch.uint8, device=dev), vb)
     cfg = eg.make_cfg(w.K, w.D_h, w.d, 1, w.V, V_c, eg.BF16, w.rows, mult,
-                      flags=eg.SAVE_KV if save_kv else 0)
+                      flags=(eg.SAVE_KV if save_kv else 0) | variant)
     N, E = w.N, w.E
     ids = torch.from_numpy(ids_np).to(dev)
     idx = torch.empty((w.B, w.T, w.J), dtype=torch.int32, device=dev)

@@ -55,6 +55,8 @@ def main(argv=None):
     ap.add_argument("--cache-rows", type=int, default=1 << 20)
     ap.add_argument("--save-kv", action="store_true",
                     help="fused, backward: the forward keeps k and v for the backward")
+    ap.add_argument("--dilated", action="store_true",
+                    help="fused, backward, decode: the dilated conv (taps 3, 6, 9 tokens back)")
     a = ap.parse_args(argv)
     from . import build
     build.build()
@@ -69,7 +71,8 @@ def main(argv=None):
     rows = synth.primes_at_most(a.rows, a.heads)
     mult = synth.hash_multipliers(12345, a.heads)
     cfg = eg.make_cfg(K, a.dh, a.d, 1, 129280, synth.compressed_vocab(129280), eg.BF16, rows, mult,
-                      flags=eg.SAVE_KV if a.save_kv else 0)
+                      flags=(eg.SAVE_KV if a.save_kv else 0) |
+                      (eg.CONV_DILATED if a.dilated else 0))
     g = torch.Generator(device=dev)
     g.manual_seed(7)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -216,7 +219,7 @@ def main(argv=None):
         eg.engram_build_vocab_proj(keys, 129280, proj, torch.empty(vb, dtype=torch.uint8, device=dev), vb)
         ids = torch.randint(0, 129280, (N,), generator=g, device=dev, dtype=torch.int32)
         state = torch.full((N, 2), cfg.V_c, dtype=torch.int32, device=dev)
-        conv_state = torch.zeros((N, 1, 3, a.d), device=dev)
+        conv_state = torch.zeros((N, 1, 9 if a.dilated else 3, a.d), device=dev)
         idx = torch.empty((N, 1, a.heads), dtype=torch.int32, device=dev)
 
         def run():
