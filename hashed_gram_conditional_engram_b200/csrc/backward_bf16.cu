@@ -55,7 +55,6 @@ Blas& blas() {
 }
 
 constexpr int kMaxDevices = 64;
-constexpr size_t kBlasWorkspace = 32u << 20;  // from the caller's workspace
 
 // One handle per device, created on first use and kept for the process.
 int blas_handle(cudaStream_t s, void* workspace, cublasHandle_t* out) {
@@ -221,12 +220,50 @@ __device__ __forceinline__ void col_emit(const FPairs<NP>& r, const FPairs<NP>& 
   if ((j & 31) == 31) col_flush(pb, j - 31, 32, np, pab);
 }
 
+// With the pre-conv norm the walk's result for token j is dc (the conv
+// input's gradient, fp32, the lane's features at dcb + j d) instead of dv:
+// the lane's share of <g_v dc, vt> (vt = alpha v) goes to the partials, which
+// the pre-norm row kernel adds up for the norm's backward, and dc rc vt
+// (= dc q v, q = alpha rc) is added to gacc for g_v's gradient.
+template <int NP>
+__device__ __forceinline__ void col_emit_pre(const FPairs<NP>& r, const FPairs<NP>& vv, float a,
+                                             float qa, const FPairs<NP>& gv, FPairs<NP>& gacc,
+                                             int j, int d, int np, float* __restrict__ dcb,
+                                             ColPartials& pb, float* __restrict__ pab) {
+  float dot = 0.f;
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    const float2 gr = __fmul2_rn(gv.p[q], r.p[q]);
+    dot = fmaf(gr.x, a * vv.p[q].x, fmaf(gr.y, a * vv.p[q].y, dot));
+    gacc.p[q] = __ffma2_rn(r.p[q], __fmul2_rn(make_float2(qa, qa), vv.p[q]), gacc.p[q]);
+  }
+  if constexpr (NP == 2) {
+    *reinterpret_cast<float4*>(dcb + (int64_t)j * d) =
+        make_float4(r.p[0].x, r.p[0].y, r.p[NP - 1].x, r.p[NP - 1].y);
+  } else {
+    *reinterpret_cast<float2*>(dcb + (int64_t)j * d) = r.p[0];
+  }
+  pb.p[j & 31][threadIdx.x & 31] = dot;
+  if ((j & 31) == 31) col_flush(pb, j - 31, 32, np, pab);
+}
+
+// The pre-conv norm's inputs and outputs of the walk (unused without it):
+// rc[t] = (alpha_t^2 <v_t, v_t> / d + eps)^(-1/2), g_v (NULL: ones), dc
+// [N, d] fp32 and the chunks' partial sums of dc rc vt, gvpart [chunks, d].
+struct ColPre {
+  const float* rc;
+  const float* gv;
+  float* dc;
+  float* gvpart;
+};
+
 // dynamic shared memory of the column walk: per warp the copy ring, the
-// dalpha partials and the chunk's gates (with DIL * 3 tokens on each side)
-template <int DIL, int NP>
+// dalpha partials and the chunk's gates (with DIL * 3 tokens on each side),
+// and with the pre-conv norm the tokens' alpha rc likewise
+template <int DIL, int NP, bool PRE>
 constexpr int col_smem_bytes() {
   return COL_WARPS * (COL_RING * 2 * 32 * (int)sizeof(FPairs<NP>) + (int)sizeof(ColPartials) +
-                      (COL_TOK + 6 * DIL) * 4);
+                      (PRE ? 2 : 1) * (COL_TOK + 6 * DIL) * 4);
 }
 
 // One warp per (chunk of COL_TOK tokens, 64 NP features), each lane holding
@@ -250,12 +287,17 @@ constexpr int col_smem_bytes() {
 // on packed fp32 pairs.  Warps are independent (all lanes of one walk the
 // same tokens, so the branches are uniform); the block only groups COL_WARPS
 // chunks for scheduling.
-template <int DIL, int NP>
+// With the pre-conv norm (PRE) the conv reads c = alpha rc g_v v instead of
+// vt, the running sums are those of dc (dvt without u and without the norm's
+// backward, which needs whole rows and is left to the pre-norm row kernel),
+// and each completed token's dc goes out as col_emit_pre describes; part then
+// holds the sums of dy_t * (c_{t-3 DIL}, ..., c_t).
+template <int DIL, int NP, bool PRE>
 __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     const float* __restrict__ v, const float* __restrict__ alpha,
     const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
     int ld, int chunks, __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part,
-    float4* __restrict__ part) {
+    float4* __restrict__ part, ColPre pre) {
   // v and dv rows are ld apart (they share rows with k and dk), dout rows d
   using FP = FPairs<NP>;
   constexpr int NH = 3 * DIL;
@@ -267,6 +309,8 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
   auto* al_all = reinterpret_cast<float(*)[COL_TOK + 2 * NH]>(col_smem + COL_WARPS * RING_BYTES +
                                                                COL_WARPS * sizeof(ColPartials));
   ColPartials& pb = pb_all[warp];
+  // PRE: q_s[i] = alpha rc of the token al_s[i] belongs to
+  float* q_s = PRE ? al_all[COL_WARPS + warp] : nullptr;
   const int chunk = blockIdx.x * COL_WARPS + warp;
   if (chunk >= chunks) return;  // no block-wide barrier follows
   const int f = blockIdx.y * col_feat(NP) + lane * 2 * NP;
@@ -279,8 +323,17 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
   for (int i = lane; i < COL_TOK + 2 * NH; i += 32) {
     const int64_t tt = t0 - NH + i;
     al_s[i] = (tt >= 0 && tt < t_stop) ? alpha[tt] : 0.f;
+    if constexpr (PRE) q_s[i] = (tt >= 0 && tt < t_stop) ? alpha[tt] * pre.rc[tt] : 0.f;
   }
   __syncwarp();
+  // PRE: g_v of the lane's features, and its gradient's running sum
+  FPairs<NP> Gv, Gacc;
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    Gv.p[q] = make_float2(1.f, 1.f);
+    Gacc.p[q] = make_float2(0.f, 0.f);
+  }
+  if (PRE && pre.gv != nullptr) Gv = ld_pairs<NP>(pre.gv + blockIdx.y * col_feat(NP) + lane * 2 * NP);
   // the weights as (feature x, feature y) pairs: W0 multiplies vt_{t-NH}, W3 vt_t
   FP W0, W1, W2, W3;
 #pragma unroll
@@ -300,16 +353,27 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     sr[k] = ar[k] = vr_[k] = zero;
     if (pos >= k + 1) {  // the token lies in this sequence
       FP q = ld_pairs<NP>(v + (t0 - 1 - k) * ld + f);
-      const float a = al_s[NH - 1 - k];
+      const float a = PRE ? q_s[NH - 1 - k] : al_s[NH - 1 - k];
 #pragma unroll
-      for (int j = 0; j < NP; ++j) q.p[j] = __fmul2_rn(make_float2(a, a), q.p[j]);
+      for (int j = 0; j < NP; ++j) {
+        q.p[j] = __fmul2_rn(make_float2(a, a), q.p[j]);
+        if constexpr (PRE) q.p[j] = __fmul2_rn(Gv.p[j], q.p[j]);
+      }
       sr[k] = q;
     }
   }
   FP C0 = zero, C1 = zero, C2 = zero, C3 = zero;  // conv-weight partials for w_0 .. w_3
   int live = 0;
   __nv_bfloat16* dvb = dv + t0 * ld + f;
+  float* dcb = PRE ? pre.dc + t0 * d + f : nullptr;
   float* pab = dalpha_part + t0 * np + blockIdx.y;
+  // emit the token whose gate and alpha rc sit at al_s[ia], q_s[ia]
+  auto emit = [&](const FP& r, const FP& vv, int ia, int j) {
+    if constexpr (PRE)
+      col_emit_pre<NP>(r, vv, al_s[ia], q_s[ia], Gv, Gacc, j, d, np, dcb, pb, pab);
+    else
+      col_emit<NP>(r, vv, al_s[ia], j, ld, np, dvb, pb, pab);
+  };
   const int n_chunk = (int)(t1 - t0), n_walk = (int)(t_stop - t0);
   // token q's v and dout go to ring slot q % COL_RING; the slot refilled at
   // step i held token i - 1, whose values step i - 1 has already used
@@ -345,10 +409,12 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
       for (int k = 0; k < NH; ++k) sr[k] = zero;
       live = 0;
     }
-    FP vt, g, E, A0;
+    FP vt, g, E, A0;  // vt: the conv's input at t (c with PRE)
+    const float ct = PRE ? q_s[i + NH] : at;
 #pragma unroll
     for (int q = 0; q < NP; ++q) {
-      vt.p[q] = __fmul2_rn(make_float2(at, at), vr.p[q]);
+      vt.p[q] = __fmul2_rn(make_float2(ct, ct), vr.p[q]);
+      if constexpr (PRE) vt.p[q] = __fmul2_rn(Gv.p[q], vt.p[q]);
       const float2 y =
           __ffma2_rn(W0.p[q], sr[NH - 1].p[q],
                      __ffma2_rn(W1.p[q], sr[2 * DIL - 1].p[q],
@@ -357,7 +423,7 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
       E.p[q] = __ffma2_rn(W0.p[q], g.p[q], ar[NH - 1].p[q]);  // dvt of t-NH, complete
       ar[2 * DIL - 1].p[q] = __ffma2_rn(W1.p[q], g.p[q], ar[2 * DIL - 1].p[q]);
       ar[DIL - 1].p[q] = __ffma2_rn(W2.p[q], g.p[q], ar[DIL - 1].p[q]);
-      A0.p[q] = __ffma2_rn(W3.p[q], g.p[q], ut.p[q]);
+      A0.p[q] = PRE ? __fmul2_rn(W3.p[q], g.p[q]) : __ffma2_rn(W3.p[q], g.p[q], ut.p[q]);
     }
     if (i < n_chunk) {
 #pragma unroll
@@ -368,13 +434,12 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
         C3.p[q] = __ffma2_rn(g.p[q], vt.p[q], C3.p[q]);
       }
     }
-    if (live == NH) col_emit<NP>(E, vr_[NH - 1], al_s[i], i - NH, ld, np, dvb, pb, pab);
+    if (live == NH) emit(E, vr_[NH - 1], i, i - NH);
     if (pos == T - 1) {  // the sequence ends at t: its later tokens are complete
 #pragma unroll
       for (int k = NH - 1; k >= 1; --k)  // tokens t-k, oldest first
-        if (live >= k && i - k < n_chunk)
-          col_emit<NP>(ar[k - 1], vr_[k - 1], al_s[i + NH - k], i - k, ld, np, dvb, pb, pab);
-      if (i < n_chunk) col_emit<NP>(A0, vr, at, i, ld, np, dvb, pb, pab);
+        if (live >= k && i - k < n_chunk) emit(ar[k - 1], vr_[k - 1], i + NH - k, i - k);
+      if (i < n_chunk) emit(A0, vr, i + NH, i);
     }
 #pragma unroll
     for (int k = NH - 1; k > 0; --k) {
@@ -395,6 +460,11 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
         make_float4(C0.p[q].x, C1.p[q].x, C2.p[q].x, C3.p[q].x);
     part[(int64_t)chunk * d + f + 2 * q + 1] =
         make_float4(C0.p[q].y, C1.p[q].y, C2.p[q].y, C3.p[q].y);
+  }
+  if constexpr (PRE) {
+#pragma unroll
+    for (int q = 0; q < NP; ++q)
+      *reinterpret_cast<float2*>(pre.gvpart + (int64_t)chunk * d + f + 2 * q) = Gacc.p[q];
   }
 }
 
@@ -661,6 +731,84 @@ __global__ void bw_scale_reduce_kernel(const float* __restrict__ spart, int bloc
   dgscale[d + f] = S * gscale[f];      // d/dg_k
 }
 
+// The pre-conv norm's backward, one token per block step (persistent blocks,
+// 256 threads): S = <g_v dc, vt> from the column walk's partials (added in
+// order by the first warp), then per feature
+//   dvt = u + rc g_v dc - rc^3 vt S / d   (vt = alpha v; RMSNorm backward)
+// dv = alpha dvt (bf16, for the GEMMs) and dalpha = <dvt, v> (a fixed-order
+// block reduction), written as the one dalpha partial of the token's row of
+// da (rows 4 floats apart) for the gate's row kernel.
+constexpr int PN_ROW_THREADS = 256;
+__global__ void __launch_bounds__(PN_ROW_THREADS) bw_prenorm_row_kernel(
+    const float* __restrict__ dc, const float* __restrict__ v, int ld,
+    const float* __restrict__ dout, const float* __restrict__ alpha,
+    const float* __restrict__ rc, const float* __restrict__ gv, const float* __restrict__ ppart,
+    int np, int np_pad, int64_t N, int d, __nv_bfloat16* __restrict__ dv,
+    float* __restrict__ da) {
+  __shared__ float Ssh;
+  __shared__ float red[2][PN_ROW_THREADS / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nv = d / 4;
+  const float invd = 1.0f / (float)d;
+  int it = 0;
+  for (int64_t t = blockIdx.x; t < N; t += gridDim.x, ++it) {
+    if (warp == 0) {
+      float S = 0.f;
+      for (int i = lane; i < np; i += 32) S += ppart[t * np_pad + i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+      if (lane == 0) Ssh = S;
+    }
+    __syncthreads();
+    const float S = Ssh;
+    const float a = alpha[t], r = rc[t];
+    const float cS = r * r * r * a * S * invd;  // rc^3 S / d, times alpha for vt = alpha v
+    const float4* dcr = reinterpret_cast<const float4*>(dc + t * d);
+    const float4* vr = reinterpret_cast<const float4*>(v + t * ld);
+    const float4* ur = reinterpret_cast<const float4*>(dout + t * d);
+    const float4* gr = reinterpret_cast<const float4*>(gv);
+    float dot = 0.f;
+    for (int c4 = threadIdx.x; c4 < nv; c4 += PN_ROW_THREADS) {
+      const float4 x = dcr[c4], vv = vr[c4], u = ur[c4];
+      const float4 g = gv != nullptr ? gr[c4] : make_float4(1.f, 1.f, 1.f, 1.f);
+      float4 o;
+      o.x = u.x + r * g.x * x.x - cS * vv.x;
+      o.y = u.y + r * g.y * x.y - cS * vv.y;
+      o.z = u.z + r * g.z * x.z - cS * vv.z;
+      o.w = u.w + r * g.w * x.w - cS * vv.w;
+      dot = fmaf(o.x, vv.x, fmaf(o.y, vv.y, fmaf(o.z, vv.z, fmaf(o.w, vv.w, dot))));
+      const __nv_bfloat162 p01 = __floats2bfloat162_rn(a * o.x, a * o.y);
+      const __nv_bfloat162 p23 = __floats2bfloat162_rn(a * o.z, a * o.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&p01);
+      pk.y = *reinterpret_cast<const uint32_t*>(&p23);
+      *reinterpret_cast<uint2*>(dv + t * ld + c4 * 4) = pk;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    float* rb = red[it & 1];  // two buffers: a fast warp's next write never meets a slow read
+    if (lane == 0) rb[warp] = dot;
+    __syncthreads();  // also: every thread has read Ssh before the next token's write
+    if (threadIdx.x == 0) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < PN_ROW_THREADS / 32; ++w) sum += rb[w];
+      *reinterpret_cast<float4*>(da + t * 4) = make_float4(sum, 0.f, 0.f, 0.f);
+    }
+  }
+}
+
+// dg_v[f] = sum over chunks, in order, of gvpart[chunk][f]
+__global__ void bw_gv_reduce_kernel(const float* __restrict__ gvpart, int chunks, int d,
+                                    float* __restrict__ dgv) {
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f >= d) return;
+  float S = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < chunks; ++c) S += gvpart[(int64_t)c * d + f];
+  dgv[f] = S;
+}
+
 constexpr int DCONV_WARPS = 32;
 
 // dconv_w[f] = sum over chunks of part[chunk][f]: warp w adds chunks w,
@@ -713,6 +861,9 @@ struct BwdBf16Ws {
   float *dalpha_part, *de;  // partials of <dvt, v>, padded rows
   float4* part;
   float* spart;  // with norm scales: [kMaxRowBlocks][d] sums of the row blocks
+  // with the pre-conv norm: rc [N], dc [N, d], dalpha rows [N, 4], the
+  // chunks' g_v sums [chunks, d]
+  float *rc, *dc, *da, *gvpart;
   void* blas_ws;
   void* tg_ws;
   size_t tg_bytes;
@@ -723,7 +874,7 @@ constexpr size_t up256b(size_t b) { return (b + 255) & ~(size_t)255; }
 constexpr int kMaxRowBlocks = 1024;  // row-kernel blocks when the scales' sums are kept
 
 size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved, bool scaled,
-                       BwdBf16Ws* w) {
+                       bool prenorm, BwdBf16Ws* w) {
   const int64_t chunks = (N + COL_TOK - 1) / COL_TOK;
   const size_t KV = kv_saved ? 0 : up256b((size_t)N * 2 * d * 4);
   const size_t DKV = up256b((size_t)N * 2 * d * 2);
@@ -732,10 +883,14 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
   const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
   const size_t tg = table_grad_ws_bytes(N * J);
   const size_t SP = scaled ? up256b((size_t)kMaxRowBlocks * d * 4) : 0;
-  size_t off[10];
-  const size_t sz[10] = {KV, DKV, WKV, DW, DA, NE4, P, kBlasWorkspace, tg, SP};
+  const size_t RC = prenorm ? up256b((size_t)N * 4) : 0;
+  const size_t DC = prenorm ? up256b((size_t)N * d * 4) : 0;
+  const size_t DA1 = prenorm ? up256b((size_t)N * 16) : 0;
+  const size_t GVP = prenorm ? up256b((size_t)chunks * d * 4) : 0;
+  size_t off[14];
+  const size_t sz[14] = {KV, DKV, WKV, DW, DA, NE4, P, kBlasWorkspace, tg, SP, RC, DC, DA1, GVP};
   size_t o = 0;
-  for (int i = 0; i < 10; ++i) {
+  for (int i = 0; i < 14; ++i) {
     off[i] = o;
     o += sz[i];
   }
@@ -752,14 +907,27 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
     w->tg_ws = p + off[8];
     w->tg_bytes = tg;
     w->spart = scaled ? reinterpret_cast<float*>(p + off[9]) : nullptr;
+    w->rc = prenorm ? reinterpret_cast<float*>(p + off[10]) : nullptr;
+    w->dc = prenorm ? reinterpret_cast<float*>(p + off[11]) : nullptr;
+    w->da = prenorm ? reinterpret_cast<float*>(p + off[12]) : nullptr;
+    w->gvpart = prenorm ? reinterpret_cast<float*>(p + off[13]) : nullptr;
   }
   return o;
 }
 
 }  // namespace
 
-size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved, bool scaled) {
-  return bwd_bf16_layout(nullptr, N, d, E, J, kv_saved, scaled, nullptr);
+size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved, bool scaled,
+                              bool prenorm) {
+  return bwd_bf16_layout(nullptr, N, d, E, J, kv_saved, scaled, prenorm, nullptr);
+}
+
+int blas_gemm_bf16(cudaStream_t s, void* blas_ws, bool a_t, bool b_t, int m, int n, int k,
+                   const void* A, int lda, const void* B, int ldb, float* C, int ldc, float beta) {
+  cublasHandle_t hd;
+  const int rc = blas_handle(s, blas_ws, &hd);
+  if (rc) return rc;
+  return gemm_rm(hd, a_t, b_t, m, n, k, A, lda, B, ldb, C, ldc, beta);
 }
 
 int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bfloat16* e,
@@ -769,18 +937,19 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
                          float* dWk,
                          float* dWv, float* dconv_w, float* de, int64_t* dtab_keys,
                          float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, int dil,
-                         void* ws, size_t ws_bytes, cudaStream_t s) {
+                         bool prenorm, const float* gv, void* ws, size_t ws_bytes,
+                         cudaStream_t s) {
   const int E = hp.E;
   const bool have_kv = kv_saved != nullptr;
   const bool scaled = gscale != nullptr;
-  if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J, have_kv, scaled))
+  if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J, have_kv, scaled, prenorm))
     return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
   // a row in registers; whole column blocks; 16-byte multiples for the row copies
   if (d > ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS || d % 256 != 0 || (dil != 1 && dil != 3))
     return ENGRAM_ERR_UNSUPPORTED;
   BwdBf16Ws w;
-  bwd_bf16_layout(ws, N, d, E, hp.J, have_kv, scaled, &w);
+  bwd_bf16_layout(ws, N, d, E, hp.J, have_kv, scaled, prenorm, &w);
   if (de == nullptr) de = w.de;
   cublasHandle_t hd;
   int rc = blas_handle(s, w.blas_ws, &hd);
@@ -800,14 +969,39 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   // tokens of history in registers) one
   const int np_lane = dil == 1 ? 2 : 1;
   const int np = d / col_feat(np_lane), np_pad = col_partials(d, np_lane);
+  const ColPre pre{w.rc, gv, w.dc, w.gvpart};
+  // with the pre-conv norm: rc of every token first (the walk's conv input
+  // is alpha rc g_v v)
+  if (prenorm && (rc = launch_prenorm_rc(kv + d, 2 * d, alpha, N, d, w.rc, s))) return rc;
   {
-    auto col = dil == 1 ? bw_col_kernel<1, 2> : bw_col_kernel<3, 1>;
-    const int smem = dil == 1 ? col_smem_bytes<1, 2>() : col_smem_bytes<3, 1>();
+    auto col = dil == 1 ? (prenorm ? bw_col_kernel<1, 2, true> : bw_col_kernel<1, 2, false>)
+                        : (prenorm ? bw_col_kernel<3, 1, true> : bw_col_kernel<3, 1, false>);
+    const int smem = dil == 1 ? (prenorm ? col_smem_bytes<1, 2, true>() : col_smem_bytes<1, 2, false>())
+                              : (prenorm ? col_smem_bytes<3, 1, true>() : col_smem_bytes<3, 1, false>());
     if ((rc = ck(cudaFuncSetAttribute(col, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))))
       return rc;
     col<<<dim3((unsigned)((chunks + COL_WARPS - 1) / COL_WARPS), (unsigned)np), 32 * COL_WARPS,
           smem, s>>>(kv + d, alpha, reinterpret_cast<const float4*>(conv_w), dout, N, T, d, 2 * d,
-                     chunks, w.dkv + d, w.dalpha_part, w.part);
+                     chunks, w.dkv + d, w.dalpha_part, w.part, pre);
+  }
+  // the pre-conv norm's backward per token: dv and dalpha (one partial per row)
+  const float* da_rows = w.dalpha_part;
+  int da_np = np, da_np_pad = np_pad;
+  if (prenorm) {
+    int dev = 0, sms = 0;
+    if ((rc = ck(cudaGetDevice(&dev))) ||
+        (rc = ck(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))))
+      return rc;
+    const int64_t grid = std::min<int64_t>(N, (int64_t)sms * 8);
+    bw_prenorm_row_kernel<<<(unsigned)grid, PN_ROW_THREADS, 0, s>>>(
+        w.dc, kv + d, 2 * d, dout, alpha, w.rc, gv, w.dalpha_part, np, np_pad, N, d, w.dkv + d,
+        w.da);
+    if (scaled)  // dg_v after dg_h, dg_k
+      bw_gv_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(w.gvpart, chunks, d,
+                                                                      dconv_w + 6 * (int64_t)d);
+    da_rows = w.da;
+    da_np = 1;
+    da_np_pad = 4;
   }
   {
     const int items = (d / ROW_VEC + ROW_THREADS - 1) / ROW_THREADS;
@@ -817,7 +1011,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
                       : (items == 1 ? bw_row_kernel<1, false>
                          : items == 2 ? bw_row_kernel<2, false>
                          : items == 3 ? bw_row_kernel<3, false> : bw_row_kernel<4, false>);
-    const int smem = (int)(ROW_STAGES * row_stage_bytes(d, np_pad));
+    const int smem = (int)(ROW_STAGES * row_stage_bytes(d, da_np_pad));
     int dev = 0, sms = 0, per_sm = 0;
     if ((rc = ck(cudaFuncSetAttribute(row, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))) ||
         (rc = ck(cudaGetDevice(&dev))) ||
@@ -826,7 +1020,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
       return rc;
     int64_t grid = std::min<int64_t>(N, (int64_t)sms * std::max(per_sm, 1));
     if (scaled) grid = std::min<int64_t>(grid, kMaxRowBlocks);
-    row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, kv, alpha, dout, w.dalpha_part, np, np_pad,
+    row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, kv, alpha, dout, da_rows, da_np, da_np_pad,
                                                   gscale, N, d, 2 * d, dh, w.dkv, w.spart,
                                                   status_ptr());
     if (scaled)

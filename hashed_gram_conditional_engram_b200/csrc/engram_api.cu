@@ -37,8 +37,10 @@ int check_cfg(const engram_cfg_t* c) {
 inline int elem_bytes(const engram_cfg_t* c) { return c->dtype == ENGRAM_F32 ? 4 : 2; }
 
 // variants the bf16 path implements: learnable norm scales, the dilated
-// conv, and per-branch conv weights (with one branch, the same as shared ones)
-constexpr int kBf16Variants = ENGRAM_NORM_SCALES | ENGRAM_CONV_PER_BRANCH | ENGRAM_CONV_DILATED;
+// conv, the pre-conv norm, and per-branch conv weights (with one branch, the
+// same as shared ones)
+constexpr int kBf16Variants = ENGRAM_NORM_SCALES | ENGRAM_CONV_PER_BRANCH | ENGRAM_CONV_DILATED |
+                              ENGRAM_CONV_PRENORM;
 inline bool bf16_variant_ok(const engram_cfg_t* c) {
   return (c->flags & ENGRAM_VARIANT_FLAGS & ~kBf16Variants) == 0;
 }
@@ -51,6 +53,27 @@ inline bool saves_kv(const engram_cfg_t* c) {
   return c->dtype == ENGRAM_BF16 && (c->flags & ENGRAM_SAVE_KV) != 0;
 }
 inline size_t alpha_bytes_padded(int64_t n_tok) { return ((size_t)n_tok * 4 + 255) & ~(size_t)255; }
+inline bool bf16_prenorm(const engram_cfg_t* c) {
+  return c->dtype == ENGRAM_BF16 && (c->flags & ENGRAM_CONV_PRENORM) != 0;
+}
+inline size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// bf16 forward workspace: the passes' buffers, then g_h g_k (norm scales),
+// then with the pre-conv norm v [N, d] fp32, rc [N] and cuBLAS's workspace
+struct Bf16FwdWs {
+  size_t gg, vbuf, rc, blas, total;
+};
+inline Bf16FwdWs bf16_fwd_ws(const engram_cfg_t* c, int64_t n) {
+  const int d = c->d_model, E = 2 * c->K * c->D_h;
+  Bf16FwdWs w;
+  w.gg = tc_forward_ws_bytes(n, d, E);
+  w.vbuf = w.gg + (bf16_scaled(c) ? up256((size_t)d * 4) : 0);
+  const bool pn = bf16_prenorm(c);
+  w.rc = w.vbuf + (pn ? up256((size_t)n * d * 4) : 0);
+  w.blas = w.rc + (pn ? up256((size_t)n * 4) : 0);
+  w.total = w.blas + (pn ? kBlasWorkspace : 0);
+  return w;
+}
 
 }  // namespace
 
@@ -120,11 +143,11 @@ size_t engram_workspace_size(const engram_cfg_t* cfg, int32_t call, int64_t n) {
   switch (call) {
     case ENGRAM_WS_FORWARD:
       if (cfg->dtype == ENGRAM_F32) return f32_forward_ws_bytes(n, M, d);
-      // with norm scales, their product g_h g_k after the passes' buffers
-      return tc_forward_ws_bytes(n, d, E) + (bf16_scaled(cfg) ? ((size_t)d * 4 + 255) & ~(size_t)255 : 0);
+      return bf16_fwd_ws(cfg, n).total;
     case ENGRAM_WS_BACKWARD:
       if (cfg->dtype == ENGRAM_BF16)
-        return backward_bf16_ws_bytes(n, d, E, 2 * cfg->K, saves_kv(cfg), bf16_scaled(cfg));
+        return backward_bf16_ws_bytes(n, d, E, 2 * cfg->K, saves_kv(cfg), bf16_scaled(cfg),
+                                      bf16_prenorm(cfg));
       return backward_f32_ws_bytes(n, M, d, E) + table_grad_ws_bytes(n * 2 * cfg->K);
     case ENGRAM_WS_TABLE_GRAD:
       return table_grad_ws_bytes(n * 2 * cfg->K);
@@ -218,17 +241,24 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
                        ? reinterpret_cast<float*>(reinterpret_cast<char*>(saved) +
                                                   alpha_bytes_padded(N))
                        : nullptr;
+  const Bf16FwdWs wl = bf16_fwd_ws(cfg, N);
+  char* wsb = static_cast<char*>(ws);
   float* gg = nullptr;  // g_h g_k, after the passes' workspace
   if (bf16_scaled(cfg)) {
-    gg = reinterpret_cast<float*>(static_cast<char*>(ws) + tc_forward_ws_bytes(N, d, E));
+    gg = reinterpret_cast<float*>(wsb + wl.gg);
     if ((rc = launch_scale_product(conv_w + 4 * d, conv_w + 5 * d, d, gg, s))) return rc;
   }
+  // the pre-conv norm: v into the kept [k | v] rows when there are any
+  PrenormFwd pn{bf16_scaled(cfg) ? conv_w + 6 * d : nullptr,
+                kv_save != nullptr ? kv_save + d : reinterpret_cast<float*>(wsb + wl.vbuf),
+                kv_save != nullptr ? 2 * d : d, reinterpret_cast<float*>(wsb + wl.rc),
+                wsb + wl.blas};
   return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
                            static_cast<const __nv_bfloat16*>(Wk),
                            static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
                            static_cast<__nv_bfloat16*>(out), saved, kv_save, gg,
                            (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1, N, T, d, E, ws, ws_bytes,
-                           table != nullptr, s);
+                           table != nullptr, bf16_prenorm(cfg) ? &pn : nullptr, s);
 }
 
 int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,
@@ -275,8 +305,10 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                                 static_cast<const bf*>(Wk), static_cast<const bf*>(Wv), conv_w,
                                 bf16_scaled(cfg) ? conv_w + 4 * d : nullptr, saved, kv_saved,
                                 dout, dh, dWk, dWv, dconv_w, de, dtab_keys, dtab_rows, n_unique,
-                                N, T, d, (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1, ws,
-                                ws_bytes, s);
+                                N, T, d, (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1,
+                                bf16_prenorm(cfg),
+                                bf16_scaled(cfg) && bf16_prenorm(cfg) ? conv_w + 6 * d : nullptr,
+                                ws, ws_bytes, s);
   }
   const size_t bw = backward_f32_ws_bytes(N, M, d, E);
   // de lives in the dense-backward workspace unless the caller wants it
@@ -351,8 +383,9 @@ int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const 
 
 int64_t engram_param_floats(const engram_cfg_t* cfg) {
   if (check_cfg(cfg) != ENGRAM_OK) return 0;
-  if (cfg->dtype == ENGRAM_BF16)
-    return (int64_t)cfg->d_model * ((cfg->flags & ENGRAM_NORM_SCALES) ? 6 : 4);
+  if (cfg->dtype == ENGRAM_BF16)  // conv weights, then g_h, g_k (and g_v with the pre-conv norm)
+    return (int64_t)cfg->d_model *
+           (4 + ((cfg->flags & ENGRAM_NORM_SCALES) ? ((cfg->flags & ENGRAM_CONV_PRENORM) ? 3 : 2) : 0));
   return f32_param_floats(cfg->flags, cfg->n_branch, cfg->d_model);
 }
 

@@ -1266,7 +1266,8 @@ template <int BN, int STAGES_K, int STAGES_V, int STAGES_VKV, int KCH>
 int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
               float* alpha_saved, float* kv_save, const float* gg, int dil, int64_t N, int T,
-              int d, int E, float4* part, float* alpha, bool chained, cudaStream_t s) {
+              int d, int E, float4* part, float* alpha, bool chained, bool gate_only,
+              cudaStream_t s) {
   // Each CTA of a pair loads 128 rows of A and BN/2 rows of B per stage.
   // pass K: A = e (256 tokens per pair tile), B = W_k (BN features)
   CUtensorMap ta_k, tb_k, ta_v, tb_v, th, to, to29;
@@ -1335,6 +1336,7 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
                           (const float4*)part, a.n_part, N, d, alpha, alpha_saved);
     if (rc) return rc;
   }
+  if (gate_only) return ENGRAM_OK;  // the pre-conv norm's path takes over from alpha
   a.alpha = alpha;
   // pass V: pair tiles of 256 features x BN tokens.  Whole sequences: the
   // token tiles overlap by the conv's history (recomputed); decode: plain
@@ -1406,7 +1408,7 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
                       __nv_bfloat16* out, float* alpha_saved, float* kv_save, const float* gg,
                       int dil, int64_t N, int T, int d, int E, void* ws, size_t ws_bytes,
-                      bool chained, cudaStream_t s) {
+                      bool chained, const PrenormFwd* pn, cudaStream_t s) {
   if (ws_bytes < tc_forward_ws_bytes(N, d, E) || ws == nullptr) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL - 256) return ENGRAM_ERR_UNSUPPORTED;
   const bool wide = use_wide(N, d);
@@ -1414,16 +1416,22 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
   float4* part = static_cast<float4*>(ws);
   float* alpha = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                           (size_t)N * 2 * (d / BN) * sizeof(float4));
+  // with the pre-conv norm the passes stop at the gate (pass K and alpha)
+  const bool gate_only = pn != nullptr;
+  int rc;
   if (wide)
-    return run_layer<256, 6, 5, 4, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
-                                   gg, dil, N, T, d, E, part, alpha, chained, s);
+    rc = run_layer<256, 6, 5, 4, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
+                                    gg, dil, N, T, d, E, part, alpha, chained, gate_only, s);
   // few tokens: each CTA streams long operand rows at a rate set by how many
   // bytes one copy instruction brings, so two K chunks go in each box
-  if (E % (2 * BK) == 0)
-    return run_layer<64, 4, 3, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
-                                  gg, dil, N, T, d, E, part, alpha, chained, s);
-  return run_layer<64, 8, 6, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save, gg,
-                                dil, N, T, d, E, part, alpha, chained, s);
+  else if (E % (2 * BK) == 0)
+    rc = run_layer<64, 4, 3, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
+                                   gg, dil, N, T, d, E, part, alpha, chained, gate_only, s);
+  else
+    rc = run_layer<64, 8, 6, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
+                                   gg, dil, N, T, d, E, part, alpha, chained, gate_only, s);
+  if (rc || pn == nullptr) return rc;
+  return launch_prenorm_tail(*pn, e, Wv, h, conv_w, alpha, conv_state, out, dil, N, T, d, E, s);
 }
 
 }  // namespace engram

@@ -121,18 +121,47 @@ int launch_table_grad_noalloc(const HeadParams& hp, const int32_t* idx, const fl
 int launch_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_c_out, void* ws,
                       size_t ws_bytes, cudaStream_t s);
 
+// cuBLAS, loaded on first use: C [m x n] (row-major fp32, rows ldc apart) =
+// op(A) op(B) + beta C with bf16 row-major operands (op = transpose when
+// a_t / b_t), on stream s with kBlasWorkspace bytes of blas_ws
+constexpr size_t kBlasWorkspace = 32u << 20;
+int blas_gemm_bf16(cudaStream_t s, void* blas_ws, bool a_t, bool b_t, int m, int n, int k,
+                   const void* A, int lda, const void* B, int ldb, float* C, int ldc, float beta);
+
+// pre-conv RMSNorm of bf16 layers: rc[t] = (alpha_t^2 <v_t, v_t> / d + eps)^(-1/2)
+int launch_prenorm_rc(const float* v, int ldv, const float* alpha, int64_t N, int d, float* rc,
+                      cudaStream_t s);
+// after the gate: v = e W_v^T into vbuf (fp32, rows ldv apart), rc, then the
+// conv over c = alpha rc g_v v with out = h + alpha v + SiLU(y) (decode when
+// conv_state is given)
+struct PrenormFwd {
+  const float* gv;  // g_v [d], or NULL (ones)
+  float* vbuf;
+  int ldv;
+  float* rc;        // [N]
+  void* blas_ws;    // kBlasWorkspace bytes
+};
+int launch_prenorm_tail(const PrenormFwd& p, const __nv_bfloat16* e, const __nv_bfloat16* Wv,
+                        const __nv_bfloat16* h, const float* conv_w, const float* alpha,
+                        float* conv_state, __nv_bfloat16* out, int dil, int64_t N, int T, int d,
+                        int E, cudaStream_t s);
+
 // bf16 backward (one branch): elementwise kernels here, plain GEMMs in cuBLAS
 // kv_saved: the forward's fp32 [N, 2d] k and v, or NULL to recompute them
-size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved, bool scaled);
+size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved, bool scaled,
+                              bool prenorm);
 // gscale: the learnable norm scales g_h [d], g_k [d] (NULL: none); their
-// gradients go to dconv_w + 4 d.  dil: the conv's dilation, 1 or 3
+// gradients go to dconv_w + 4 d.  dil: the conv's dilation, 1 or 3.
+// prenorm: the conv reads RMSNorm(vt) g_v (gv = g_v, or NULL for ones; its
+// gradient goes to dconv_w + 6 d when gscale is given)
 int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bfloat16* e,
                          const __nv_bfloat16* h, const __nv_bfloat16* Wk,
                          const __nv_bfloat16* Wv, const float* conv_w, const float* gscale,
                          const float* alpha, const float* kv_saved, const float* dout, float* dh,
                          float* dWk, float* dWv, float* dconv_w, float* de, int64_t* dtab_keys,
                          float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, int dil,
-                         void* ws, size_t ws_bytes, cudaStream_t s);
+                         bool prenorm, const float* gv, void* ws, size_t ws_bytes,
+                         cudaStream_t s);
 
 // bf16 tensor-core path (sm_100a tcgen05)
 size_t tc_forward_ws_bytes(int64_t N, int d, int E);
@@ -143,6 +172,6 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
                       __nv_bfloat16* out, float* alpha_saved, float* kv_save, const float* gg,
                       int dil, int64_t N, int T, int d, int E, void* ws, size_t ws_bytes,
-                      bool chained, cudaStream_t s);
+                      bool chained, const PrenormFwd* pn, cudaStream_t s);
 
 }  // namespace engram

@@ -64,6 +64,27 @@ def test_small_parameter_block_sizes():
                          4 * d * M + 3 * M * d)]:
         assert eg.engram_param_floats(_cfg(n_branch=M, flags=flags)) == want, flags
     assert eg.engram_param_floats(_cfg(flags=64)) == 0  # not a flag: invalid configuration
+    # bf16 layers (one branch): conv weights, then g_h, g_k, and g_v with the
+    # pre-conv norm
+    d = 256
+    for flags, want in [(0, 4 * d), (eg.CONV_PRENORM, 4 * d), (eg.NORM_SCALES, 6 * d),
+                        (eg.NORM_SCALES | eg.CONV_PRENORM | eg.CONV_DILATED, 7 * d)]:
+        c = _cfg(d_model=d, K=2, D_h=32, dtype=eg.BF16, flags=flags)
+        assert eg.engram_param_floats(c) == want, flags
+
+
+def test_prenorm_workspace_holds_v_rc_and_blas():
+    """With the pre-conv norm a bf16 forward also needs v (fp32 [N, d]), rc
+    [N] and cuBLAS's 32 MB; the backward dc (fp32 [N, d]) and more."""
+    N, d = 32768, 2560
+    kw = dict(K=8, D_h=80, d_model=d, dtype=eg.BF16, rows=[4449997] * 16,
+              mult=np.ones((16, 3), np.uint64))
+    b, p = _cfg(**kw), _cfg(flags=eg.CONV_PRENORM, **kw)
+    extra = eg.engram_workspace_size(p, eg.WS_FORWARD, N) - eg.engram_workspace_size(
+        b, eg.WS_FORWARD, N)
+    assert extra == N * d * 4 + N * 4 + (32 << 20)
+    assert (eg.engram_workspace_size(p, eg.WS_BACKWARD, N)
+            - eg.engram_workspace_size(b, eg.WS_BACKWARD, N)) >= N * d * 4 + N * 20
 
 
 def test_invalid_configurations_rejected_before_any_launch():

@@ -196,8 +196,9 @@ def _bf16_backward_case(B, T, d, K, D_h, seed, flags=0, with_layer=False):
     cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((J, 3), np.uint64),
                       flags=flags)
     block = conv_w.reshape(-1)
-    if flags & eg.NORM_SCALES:  # learnable g_h, g_k after the conv weights
-        block = np.r_[block, 1.0 + 0.3 * rng.standard_normal(2 * d)].astype(np.float32)
+    n_scales = eg.engram_param_floats(cfg) - 4 * d
+    if n_scales:  # learnable g_h, g_k (and g_v) after the conv weights
+        block = np.r_[block, 1.0 + 0.3 * rng.standard_normal(n_scales)].astype(np.float32)
     L = Layer(cfg, B, T, packed_table(tables, "bf16"), bf16_dev(h), bf16_dev(Wk), bf16_dev(Wv),
               dev(block), torch.bfloat16)
     idx_d = dev(idx.reshape(B, T, J))
@@ -209,7 +210,8 @@ def _bf16_backward_case(B, T, d, K, D_h, seed, flags=0, with_layer=False):
     e_ref = f64(O.gather(idx, [synth.to_bf16_bits(t) for t in tables]))
     assert np.array_equal(bf16_bits(L.e), O.gather(idx, [synth.to_bf16_bits(t) for t in tables]))
     vflags = ((O.NORM_SCALES if flags & eg.NORM_SCALES else 0) |
-              (O.CONV_DILATED if flags & eg.CONV_DILATED else 0))
+              (O.CONV_DILATED if flags & eg.CONV_DILATED else 0) |
+              (O.CONV_PRENORM if flags & eg.CONV_PRENORM else 0))
     if vflags:
         ref = O.layer_backward_v(e_ref, f64(synth.to_bf16_bits(h)).reshape(N, 1, d),
                                  f64(synth.to_bf16_bits(Wk)), f64(synth.to_bf16_bits(Wv)), block,
@@ -293,6 +295,23 @@ def test_backward_bf16_dilated_matches_oracle(B, T, d, flags):
     token's dvt 9 tokens later (or at its sequence's end); every gradient is
     held to the same bounds as the plain conv's."""
     _check_bf16_backward(*_bf16_backward_case(B, T, d, 2, 32, seed=B * 5 + T, flags=flags))
+
+
+@pytest.mark.parametrize("B,T,d,flags", [
+    (3, 100, 256, eg.CONV_PRENORM),                                 # narrow forward tiles
+    (2, 2500, 512, eg.CONV_PRENORM | eg.NORM_SCALES),               # g_v's gradient too
+    (40, 7, 256, eg.CONV_PRENORM | eg.CONV_DILATED),                # short sequences, dilated
+    (1, 300, 256, eg.CONV_PRENORM | eg.SAVE_KV),                    # kept k and v
+    (3, 129, 768, eg.CONV_PRENORM | eg.CONV_DILATED | eg.NORM_SCALES),
+    (64, 1, 256, eg.CONV_PRENORM),                                  # one-token sequences
+])
+def test_backward_bf16_prenorm_matches_oracle(B, T, d, flags):
+    """The pre-conv RMSNorm on a bf16 layer: the column walk carries dc (the
+    conv input's gradient) and the partial sums of <g_v dc, vt>; a row
+    kernel forms dvt through the norm's backward, dv and dalpha; every
+    gradient, g_v's included, is held to the same bounds as the plain
+    conv's."""
+    _check_bf16_backward(*_bf16_backward_case(B, T, d, 2, 32, seed=B * 3 + T, flags=flags))
 
 
 def _check_bf16_backward(g, ref, idx, rows, D_h):

@@ -2,8 +2,9 @@
 per-branch conv, learnable RMSNorm scales) of the fp32 layer with the
 oracle: forward, decode streaming and every gradient, including the
 small-parameter block's, within the fp32 tolerance (1e-5 max relative
-error with a 1e-3 RMS floor); bf16 layers with the scales and the dilated
-conv against the bf16 metric; bf16 layers refuse the pre-conv norm."""
+error with a 1e-3 RMS floor); bf16 layers with the scales, the dilated conv
+and the pre-conv norm against the bf16 metric; bf16 layers refuse more than
+one branch."""
 import numpy as np
 import pytest
 import torch
@@ -109,10 +110,10 @@ def test_variant_decode_streaming_matches_whole_sequences(flags):
     assert eg.engram_get_status() == 0
 
 
-def test_bf16_layers_refuse_the_variants():
+def test_bf16_layers_refuse_two_branches():
     K, D_h, d = 2, 32, 256
     rows = synth.primes_at_most(1009, 2 * K)
-    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
+    cfg = eg.make_cfg(K, D_h, d, 2, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
                       flags=eg.CONV_PRENORM)
     N, E = 4, 2 * K * D_h
     e = torch.zeros((N, E), dtype=torch.bfloat16, device="cuda")
@@ -190,28 +191,84 @@ def test_bf16_dilated_forward_matches_oracle(B, T, d):
     assert max_rel_err(out.float().cpu().numpy(), ref["out"]) <= 2e-2
 
 
-def test_bf16_dilated_decode_matches_whole_sequences():
-    """Decode steps of a dilated bf16 layer (conv state [B, 1, 9, d], vt of
-    the nine previous steps) against the oracle's whole-sequence forward,
-    each step within the bf16 metric."""
+def _bf16_block(rng, cfg, d):
+    """conv weights N(0, 0.5^2), then the norm scales 1 + N(0, 0.3^2)."""
+    n = eg.engram_param_floats(cfg)
+    block = rng.standard_normal(n) * 0.5
+    block[4 * d:] = 1.0 + 0.3 * rng.standard_normal(n - 4 * d)
+    return block.astype(np.float32)
+
+
+@pytest.mark.parametrize("B,T,d,flags", [
+    (3, 100, 256, PRE),              # narrow forward tiles
+    (2, 2500, 512, PRE | SC),        # wide tiles, g_v with the other scales
+    (40, 7, 256, PRE | DIL),         # sequences shorter than the dilated taps
+    (1, 4100, 256, PRE | DIL | SC),  # one sequence over many conv chunks
+    (2, 700, 256, PRE | eg.SAVE_KV), # v written into the kept [k | v] rows
+])
+def test_bf16_prenorm_forward_matches_oracle(B, T, d, flags):
+    """bf16 layer with the pre-conv RMSNorm (c = RMSNorm(alpha v) g_v): out
+    within the bf16 metric of the oracle's fp64 forward on the same bf16
+    values, alpha to 1e-5, and with ENGRAM_SAVE_KV the kept k and v against
+    the oracle's."""
     from tests.engram_cases import bf16_dev
-    rng = np.random.default_rng(77)
+    rng = np.random.default_rng(B * 11 + T + flags)
+    K, D_h = 2, 32
+    E, N = 2 * K * D_h, B * T
+    rows = synth.primes_at_most(1009, 2 * K)
+    cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
+                      flags=flags)
+    e = rng.standard_normal((N, E)).astype(np.float32)
+    h = rng.standard_normal((N, 1, d)).astype(np.float32)
+    Wk = (rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32)
+    Wv = (rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32)
+    block = _bf16_block(rng, cfg, d)
+    vflags = flags & (PRE | DIL | SC)
+    assert block.size == O.param_count(vflags, 1, d)
+    out = torch.empty((N, 1, d), dtype=torch.bfloat16, device="cuda")
+    saved = _ws(eg.engram_saved_size(cfg, N))
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+    eg.engram_forward(cfg, None, None, bf16_dev(e), bf16_dev(h), bf16_dev(Wk), bf16_dev(Wv),
+                      dev(block), None, out, saved, B, T, _ws(fb), fb)
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    f64 = O.bf16_bits_to_f64
+    b = synth.to_bf16_bits
+    ref = O.layer_forward_v(f64(b(e)), f64(b(h)), f64(b(Wk)), f64(b(Wv)), block, T, vflags)
+    assert max_rel_err(out.float().cpu().numpy(), ref["out"]) <= 2e-2
+    alpha = saved[: N * 4].view(torch.float32).cpu().numpy()
+    assert np.max(np.abs(alpha - ref["alpha"].reshape(-1))) <= 1e-5
+    if flags & eg.SAVE_KV:
+        off = (N * 4 + 255) // 256 * 256
+        kv = saved[off: off + N * 2 * d * 4].view(torch.float32).reshape(N, 2 * d).cpu().numpy()
+        assert max_rel_err(kv[:, :d], ref["k"][:, 0]) <= 1e-3
+        assert max_rel_err(kv[:, d:], ref["v"]) <= 1e-3
+
+
+@pytest.mark.parametrize("flags", [DIL, PRE, PRE | DIL | SC])
+def test_bf16_decode_matches_whole_sequences(flags):
+    """Decode steps of a bf16 layer (conv state [B, 1, 3 dil, d], the conv
+    inputs of the previous steps: vt, or RMSNorm(vt) g_v with the pre-conv
+    norm) against the oracle's whole-sequence forward, each step within the
+    bf16 metric."""
+    from tests.engram_cases import bf16_dev
+    rng = np.random.default_rng(70 + flags)
     B, T, K, D_h, d = 24, 14, 2, 32, 256
     E = 2 * K * D_h
     rows = synth.primes_at_most(1009, 2 * K)
     cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
-                      flags=eg.CONV_DILATED)
+                      flags=flags)
     e = rng.standard_normal((B, T, E)).astype(np.float32)
     h = rng.standard_normal((B, T, 1, d)).astype(np.float32)
     Wk = (rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32)
     Wv = (rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32)
-    block = (rng.standard_normal(4 * d) * 0.5).astype(np.float32)
+    block = _bf16_block(rng, cfg, d)
     f64 = O.bf16_bits_to_f64
     b = synth.to_bf16_bits
     ref = O.layer_forward_v(f64(b(e)).reshape(B * T, E), f64(b(h)).reshape(B * T, 1, d),
-                            f64(b(Wk)), f64(b(Wv)), block, T, eg.CONV_DILATED)
+                            f64(b(Wk)), f64(b(Wv)), block, T, flags)
     ref_out = ref["out"].reshape(B, T, 1, d)
-    state = torch.zeros((B, 1, 9, d), device="cuda")
+    state = torch.zeros((B, 1, 3 * O.dilation_of(flags), d), device="cuda")
     fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, B)
     ws = _ws(fb)
     Wk_d, Wv_d, blk = bf16_dev(Wk), bf16_dev(Wv), dev(block)
