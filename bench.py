@@ -574,8 +574,8 @@ def bench_fwd_bwd_27b(dev, steps=10):
     80 dims, 5.7B-parameter bf16 table): hash, forward (gather, fused passes,
     alpha, k and v saved), backward (bf16: elementwise kernels, cuBLAS GEMMs,
     sparse table gradient); the same with k and v recomputed in the
-    backward instead of saved; and with the dilated conv (taps 3, 6 and 9
-    tokens back)."""
+    backward instead of saved; with the dilated conv (taps 3, 6 and 9
+    tokens back); and with the pre-conv RMSNorm."""
     keys = ("ms_per_step", "fwd_bwd_tokens_per_s", "breakdown_ms")
     kept = _fwd_bwd_27b_run(dev, steps, save_kv=True)
     recomputed = _fwd_bwd_27b_run(dev, steps, save_kv=False)
@@ -583,6 +583,8 @@ def bench_fwd_bwd_27b(dev, steps=10):
     from hashed_gram_conditional_engram_b200 import engram as eg
     dilated = _fwd_bwd_27b_run(dev, steps, save_kv=True, variant=eg.CONV_DILATED)
     kept["dilated_conv"] = {k: dilated[k] for k in keys}
+    prenorm = _fwd_bwd_27b_run(dev, steps, save_kv=True, variant=eg.CONV_PRENORM)
+    kept["prenorm_conv"] = {k: prenorm[k] for k in keys}
     return kept
 
 

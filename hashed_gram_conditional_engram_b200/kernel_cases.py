@@ -57,6 +57,8 @@ def main(argv=None):
                     help="fused, backward: the forward keeps k and v for the backward")
     ap.add_argument("--dilated", action="store_true",
                     help="fused, backward, decode: the dilated conv (taps 3, 6, 9 tokens back)")
+    ap.add_argument("--prenorm", action="store_true",
+                    help="fused, backward, decode: the pre-conv RMSNorm (no learnable g_v)")
     a = ap.parse_args(argv)
     from . import build
     build.build()
@@ -72,7 +74,8 @@ def main(argv=None):
     mult = synth.hash_multipliers(12345, a.heads)
     cfg = eg.make_cfg(K, a.dh, a.d, 1, 129280, synth.compressed_vocab(129280), eg.BF16, rows, mult,
                       flags=(eg.SAVE_KV if a.save_kv else 0) |
-                      (eg.CONV_DILATED if a.dilated else 0))
+                      (eg.CONV_DILATED if a.dilated else 0) |
+                      (eg.CONV_PRENORM if a.prenorm else 0))
     g = torch.Generator(device=dev)
     g.manual_seed(7)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -59,10 +59,11 @@ enum { ENGRAM_F32 = 0, ENGRAM_BF16 = 1 };
 /* formulation variants: the pages fix neither the conv's dilation, nor a
  * norm before it, nor whether branches share it, nor learnable norm scales
  * ([p2] short depthwise causal conv; [p5 二.1 (2)] 一维卷积; [p5 二.2]).  fp32
- * layers take any combination; bf16 layers take ENGRAM_CONV_DILATED,
- * ENGRAM_NORM_SCALES and ENGRAM_CONV_PER_BRANCH (with their one branch the
- * same as a shared conv) and return ENGRAM_ERR_UNSUPPORTED for
- * ENGRAM_CONV_PRENORM. */
+ * layers take any combination; bf16 layers (one branch) too, where
+ * ENGRAM_CONV_PER_BRANCH is the same as a shared conv.  With
+ * ENGRAM_CONV_PRENORM a bf16 layer computes v = e W_v^T with cuBLAS (fp32)
+ * after the gate, and its forward workspace holds v, a per-token scale and
+ * cuBLAS's 32 MB. */
 #define ENGRAM_CONV_DILATED 2     /* taps at t, t-3, t-6, t-9 (dilation 3 = the largest order) */
 #define ENGRAM_CONV_PRENORM 4     /* the conv reads RMSNorm(vt) (times g_v with NORM_SCALES) */
 #define ENGRAM_CONV_PER_BRANCH 8  /* conv weights per branch */
@@ -105,7 +106,7 @@ enum {
  *            less in the backward.
  *            ENGRAM_CONV_DILATED, ENGRAM_CONV_PRENORM, ENGRAM_CONV_PER_BRANCH,
  *            ENGRAM_NORM_SCALES: formulation variants (fp32 layers: any
- *            combination; bf16 layers: all but PRENORM).
+ *            combination on fp32 and on bf16 layers).
  *            z = <RMSNorm(h) g_h, RMSNorm(k) g_k> / sqrt(d),
  *            vt = alpha v, c = RMSNorm(vt) g_v (PRENORM) or vt,
  *            y_t = sum_i w[:, i] c_{t-(3-i) dil} (dil 3 with DILATED, else 1),
