@@ -120,8 +120,7 @@ constexpr int COL_TOK = 128;   // tokens per column chunk; one warp walks one ch
 constexpr int COL_WARPS = 4;   // chunks per block
 constexpr int COL_RING = 12;   // tokens per warp in a shared-memory ring, 11 of them in flight
 
-// Features per warp of the walk: NP pairs per lane, 2 for the plain conv, 1
-// for the dilated one (whose 9-token history takes the registers).
+// Features per warp of the walk: NP pairs per lane
 __host__ __device__ constexpr int col_feat(int np_lane) { return 64 * np_lane; }
 // dalpha partials per token, padded to 16 bytes for the row kernel's copies
 __host__ __device__ constexpr int col_partials(int d, int np_lane) {
@@ -171,16 +170,16 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N_PENDING) : "memory");
 }
 
-// The warp's dalpha partials, 32 tokens at a time: lane L's share of token
-// j sits at [j % 32][L] (rows padded to 33 so that both the writes and the
-// row sums below are free of bank conflicts).
+// The warp's dalpha partials, 32 emitted tokens at a time: lane L's share of
+// the warp's e-th emitted token sits at [e % 32][L] (rows padded to 33 so
+// that both the writes and the row sums below are free of bank conflicts).
 struct ColPartials {
   float p[32][33];
 };
 
-// Sum rows 0 .. cnt-1 (tokens jbase ..) of the buffer across the 32 lanes,
-// lane r adding row r in lane order, and store them; warp-uniform call.
-__device__ __forceinline__ void col_flush(ColPartials& pb, int jbase, int cnt, int np,
+// Sum rows 0 .. cnt-1 of the buffer across the 32 lanes, lane r adding row r
+// in lane order, and store row r as token jbase + r * stride; warp-uniform.
+__device__ __forceinline__ void col_flush(ColPartials& pb, int jbase, int stride, int cnt, int np,
                                           float* __restrict__ pab) {
   __syncwarp();
   const int lane = threadIdx.x & 31;
@@ -188,18 +187,20 @@ __device__ __forceinline__ void col_flush(ColPartials& pb, int jbase, int cnt, i
     float sum = 0.f;
 #pragma unroll 8
     for (int c = 0; c < 32; ++c) sum += pb.p[lane][c];
-    pab[(jbase + lane) * np] = sum;
+    pab[(jbase + lane * stride) * np] = sum;
   }
   __syncwarp();
 }
 
-// Emit token j of the walk: dv = alpha dvt (the lane's features, bf16), and
-// the lane's share of dalpha = <dvt, v>; every 32nd token flushes the warp's
-// partials.  Tokens are emitted once each, in increasing order.
+// Emit the warp's e-th token, token j = r + e S of its chunk (a walk emits
+// the tokens r, r + S, r + 2 S, ... of its chunk, each once and in order):
+// dv = alpha dvt (the lane's features, bf16), and the lane's share of
+// dalpha = <dvt, v>; every 32nd token flushes the warp's partials.
 template <int NP>
 __device__ __forceinline__ void col_emit(const FPairs<NP>& r, const FPairs<NP>& vv, float a,
-                                         int j, int ld, int np, __nv_bfloat16* __restrict__ dvb,
-                                         ColPartials& pb, float* __restrict__ pab) {
+                                         int j, int e, int S, int ld, int np,
+                                         __nv_bfloat16* __restrict__ dvb, ColPartials& pb,
+                                         float* __restrict__ pab) {
   __nv_bfloat162 o[NP];
   float dot = 0.f;
 #pragma unroll
@@ -216,8 +217,8 @@ __device__ __forceinline__ void col_emit(const FPairs<NP>& r, const FPairs<NP>& 
   } else {
     *reinterpret_cast<__nv_bfloat162*>(dvb + j * ld) = o[0];
   }
-  pb.p[j & 31][threadIdx.x & 31] = dot;
-  if ((j & 31) == 31) col_flush(pb, j - 31, 32, np, pab);
+  pb.p[e & 31][threadIdx.x & 31] = dot;
+  if ((e & 31) == 31) col_flush(pb, j - 31 * S, S, 32, np, pab);
 }
 
 // With the pre-conv norm the walk's result for token j is dc (the conv
@@ -228,8 +229,9 @@ __device__ __forceinline__ void col_emit(const FPairs<NP>& r, const FPairs<NP>& 
 template <int NP>
 __device__ __forceinline__ void col_emit_pre(const FPairs<NP>& r, const FPairs<NP>& vv, float a,
                                              float qa, const FPairs<NP>& gv, FPairs<NP>& gacc,
-                                             int j, int d, int np, float* __restrict__ dcb,
-                                             ColPartials& pb, float* __restrict__ pab) {
+                                             int j, int e, int S, int d, int np,
+                                             float* __restrict__ dcb, ColPartials& pb,
+                                             float* __restrict__ pab) {
   float dot = 0.f;
 #pragma unroll
   for (int q = 0; q < NP; ++q) {
@@ -243,13 +245,13 @@ __device__ __forceinline__ void col_emit_pre(const FPairs<NP>& r, const FPairs<N
   } else {
     *reinterpret_cast<float2*>(dcb + (int64_t)j * d) = r.p[0];
   }
-  pb.p[j & 31][threadIdx.x & 31] = dot;
-  if ((j & 31) == 31) col_flush(pb, j - 31, 32, np, pab);
+  pb.p[e & 31][threadIdx.x & 31] = dot;
+  if ((e & 31) == 31) col_flush(pb, j - 31 * S, S, 32, np, pab);
 }
 
 // The pre-conv norm's inputs and outputs of the walk (unused without it):
 // rc[t] = (alpha_t^2 <v_t, v_t> / d + eps)^(-1/2), g_v (NULL: ones), dc
-// [N, d] fp32 and the chunks' partial sums of dc rc vt, gvpart [chunks, d].
+// [N, d] fp32 and the walks' partial sums of dc rc vt, gvpart [units, d].
 struct ColPre {
   const float* rc;
   const float* gv;
@@ -266,62 +268,67 @@ constexpr int col_smem_bytes() {
                       (PRE ? 2 : 1) * (COL_TOK + 6 * DIL) * 4);
 }
 
-// One warp per (chunk of COL_TOK tokens, 64 NP features), each lane holding
-// NP pairs of adjacent features, walking the chunk in token order; the conv
-// reads y_t = sum_i w_i vt_{t-(3-i) DIL}.  The warp keeps, for the NH = 3 DIL
-// previous tokens, vt and v, and the partial sums of their dvt:
-// dvt_s = u_s + w_3 dy_s + w_2 dy_{s+DIL} + w_1 dy_{s+2 DIL} + w_0 dy_{s+3 DIL}
+// One warp per (chunk of COL_TOK tokens, chain, 64 NP features), each lane
+// holding NP pairs of adjacent features.  The conv reads
+// y_t = sum_i w_i vt_{t-(3-i) DIL}, so the tokens of a chunk fall into DIL
+// chains (token index mod DIL, S = DIL apart), each an independent conv of
+// dilation 1 along the chain; a warp walks one chain in token order.  The
+// warp keeps, for the chain's three previous tokens, vt and v, and the
+// partial sums of their dvt:
+// dvt_s = u_s + w_3 dy_s + w_2 dy_{s+S} + w_1 dy_{s+2 S} + w_0 dy_{s+3 S}
 // (terms past the sequence end absent), to which each new dy_t adds its
-// share.  At token t it forms y_t and dy_t; dvt of token t-NH is then
-// complete, and at a sequence end so are all later ones.  The walk runs NH
-// tokens past the chunk for the last tokens' dy.  v and dout of the next
-// COL_RING - 1 tokens are in flight into a per-warp shared-memory ring
-// (asynchronous copies, each lane its own bytes).  `live` counts the ring's
-// tokens that belong to t's sequence and to this chunk's walk (tokens before
-// the chunk are emitted by the previous chunk's walk).  For each completed
-// token it writes dv (bf16, for the GEMMs) and the warp's partial of dalpha,
-// dalpha_part[token][f / (64 NP)] (the lanes' shares summed per 32 tokens,
-// from shared memory, in lane order); at the end the chunk's partial
-// conv-weight gradient, part[chunk][f] = sum over its tokens of
-// dy_t * (vt_{t-3 DIL}, vt_{t-2 DIL}, vt_{t-DIL}, vt_t).  The arithmetic runs
-// on packed fp32 pairs.  Warps are independent (all lanes of one walk the
-// same tokens, so the branches are uniform); the block only groups COL_WARPS
-// chunks for scheduling.
+// share.  At token t it forms y_t and dy_t; dvt of token t-3S is then
+// complete, and at a sequence end so are the chain's later ones.  The walk
+// runs three chain steps past the chunk for the last tokens' dy.  v and dout
+// of the next COL_RING - 1 chain tokens are in flight into a per-warp
+// shared-memory ring (asynchronous copies, each lane its own bytes).  `live`
+// counts the history's tokens that belong to t's sequence and to this
+// walk (tokens before the chunk are emitted by the previous chunk's walks).
+// For each completed token it writes dv (bf16, for the GEMMs) and the warp's
+// partial of dalpha, dalpha_part[token][f / (64 NP)] (the lanes' shares
+// summed per 32 tokens, from shared memory, in lane order); at the end the
+// walk's partial conv-weight gradient, part[unit][f] = sum over its chain's
+// tokens in the chunk of dy_t * (vt_{t-3 S}, vt_{t-2 S}, vt_{t-S}, vt_t).
+// The arithmetic runs on packed fp32 pairs.  Warps are independent (all
+// lanes of one walk the same tokens, so the branches are uniform); the block
+// only groups COL_WARPS walks for scheduling.
 // With the pre-conv norm (PRE) the conv reads c = alpha rc g_v v instead of
 // vt, the running sums are those of dc (dvt without u and without the norm's
 // backward, which needs whole rows and is left to the pre-norm row kernel),
 // and each completed token's dc goes out as col_emit_pre describes; part then
-// holds the sums of dy_t * (c_{t-3 DIL}, ..., c_t).
+// holds the sums of dy_t * (c_{t-3 S}, ..., c_t).
 template <int DIL, int NP, bool PRE>
 __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     const float* __restrict__ v, const float* __restrict__ alpha,
     const float4* __restrict__ conv_w, const float* __restrict__ dout, int64_t N, int T, int d,
-    int ld, int chunks, __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part,
+    int ld, int units, __nv_bfloat16* __restrict__ dv, float* __restrict__ dalpha_part,
     float4* __restrict__ part, ColPre pre) {
   // v and dv rows are ld apart (they share rows with k and dk), dout rows d
   using FP = FPairs<NP>;
-  constexpr int NH = 3 * DIL;
+  constexpr int S = DIL;       // token stride of a chain
+  constexpr int HT = 3 * DIL;  // tokens of conv history
   extern __shared__ __align__(16) unsigned char col_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int RING_BYTES = COL_RING * 2 * 32 * (int)sizeof(FP);
   auto* ring_all = reinterpret_cast<FP(*)[COL_RING][2][32]>(col_smem);  // [slot][v, dout][lane]
   auto* pb_all = reinterpret_cast<ColPartials*>(col_smem + COL_WARPS * RING_BYTES);
-  auto* al_all = reinterpret_cast<float(*)[COL_TOK + 2 * NH]>(col_smem + COL_WARPS * RING_BYTES +
+  auto* al_all = reinterpret_cast<float(*)[COL_TOK + 2 * HT]>(col_smem + COL_WARPS * RING_BYTES +
                                                                COL_WARPS * sizeof(ColPartials));
   ColPartials& pb = pb_all[warp];
   // PRE: q_s[i] = alpha rc of the token al_s[i] belongs to
   float* q_s = PRE ? al_all[COL_WARPS + warp] : nullptr;
-  const int chunk = blockIdx.x * COL_WARPS + warp;
-  if (chunk >= chunks) return;  // no block-wide barrier follows
+  const int unit = blockIdx.x * COL_WARPS + warp;
+  if (unit >= units) return;  // no block-wide barrier follows
+  const int chunk = unit / S, r0 = unit - chunk * S;  // the chain: tokens r0, r0 + S, ...
   const int f = blockIdx.y * col_feat(NP) + lane * 2 * NP;
   const int np = col_partials(d, NP);
   const int64_t t0 = (int64_t)chunk * COL_TOK;
   const int64_t t1 = t0 + COL_TOK < N ? t0 + COL_TOK : N;
-  const int64_t t_stop = t1 + NH < N ? t1 + NH : N;
-  // the gates of the walk's tokens and the NH before it: al_s[tt - t0 + NH]
+  const int64_t t_stop = t1 + HT < N ? t1 + HT : N;
+  // the gates of the chunk's tokens and the HT on each side: al_s[tt - t0 + HT]
   float* al_s = al_all[warp];
-  for (int i = lane; i < COL_TOK + 2 * NH; i += 32) {
-    const int64_t tt = t0 - NH + i;
+  for (int i = lane; i < COL_TOK + 2 * HT; i += 32) {
+    const int64_t tt = t0 - HT + i;
     al_s[i] = (tt >= 0 && tt < t_stop) ? alpha[tt] : 0.f;
     if constexpr (PRE) q_s[i] = (tt >= 0 && tt < t_stop) ? alpha[tt] * pre.rc[tt] : 0.f;
   }
@@ -333,8 +340,8 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     Gv.p[q] = make_float2(1.f, 1.f);
     Gacc.p[q] = make_float2(0.f, 0.f);
   }
-  if (PRE && pre.gv != nullptr) Gv = ld_pairs<NP>(pre.gv + blockIdx.y * col_feat(NP) + lane * 2 * NP);
-  // the weights as (feature x, feature y) pairs: W0 multiplies vt_{t-NH}, W3 vt_t
+  if (PRE && pre.gv != nullptr) Gv = ld_pairs<NP>(pre.gv + f);
+  // the weights as (feature x, feature y) pairs: W0 multiplies vt_{t-3S}, W3 vt_t
   FP W0, W1, W2, W3;
 #pragma unroll
   for (int q = 0; q < NP; ++q) {
@@ -345,15 +352,20 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     W3.p[q] = make_float2(wx.w, wy.w);
   }
   const FP zero = {};
-  int pos = (int)(t0 % T);
-  // rings over the NH previous tokens: index k holds token t-1-k
-  FP sr[NH], ar[NH], vr_[NH];  // vt, partial dvt, v
+  // chain steps: step i is token r0 + S i of the chunk
+  const int span = (int)(t1 - t0), wspan = (int)(t_stop - t0);
+  const int n_chunk = span > r0 ? (span - r0 + S - 1) / S : 0;
+  const int n_walk = wspan > r0 ? (wspan - r0 + S - 1) / S : 0;
+  int pos = (int)((t0 + r0) % T);
+  // rings over the three previous chain tokens: index k holds token t-(k+1)S
+  FP sr[3], ar[3], vr_[3];  // vt, partial dvt, v
 #pragma unroll
-  for (int k = 0; k < NH; ++k) {
+  for (int k = 0; k < 3; ++k) {
     sr[k] = ar[k] = vr_[k] = zero;
-    if (pos >= k + 1) {  // the token lies in this sequence
-      FP q = ld_pairs<NP>(v + (t0 - 1 - k) * ld + f);
-      const float a = PRE ? q_s[NH - 1 - k] : al_s[NH - 1 - k];
+    if (pos >= S * (k + 1)) {  // the token lies in this sequence
+      const int jk = r0 - S * (k + 1);
+      FP q = ld_pairs<NP>(v + (t0 + jk) * ld + f);
+      const float a = PRE ? q_s[jk + HT] : al_s[jk + HT];
 #pragma unroll
       for (int j = 0; j < NP; ++j) {
         q.p[j] = __fmul2_rn(make_float2(a, a), q.p[j]);
@@ -367,19 +379,19 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
   __nv_bfloat16* dvb = dv + t0 * ld + f;
   float* dcb = PRE ? pre.dc + t0 * d + f : nullptr;
   float* pab = dalpha_part + t0 * np + blockIdx.y;
-  // emit the token whose gate and alpha rc sit at al_s[ia], q_s[ia]
-  auto emit = [&](const FP& r, const FP& vv, int ia, int j) {
+  // emit the chain's e-th token
+  auto emit = [&](const FP& rr, const FP& vv, int e) {
+    const int j = r0 + S * e;
     if constexpr (PRE)
-      col_emit_pre<NP>(r, vv, al_s[ia], q_s[ia], Gv, Gacc, j, d, np, dcb, pb, pab);
+      col_emit_pre<NP>(rr, vv, al_s[j + HT], q_s[j + HT], Gv, Gacc, j, e, S, d, np, dcb, pb, pab);
     else
-      col_emit<NP>(r, vv, al_s[ia], j, ld, np, dvb, pb, pab);
+      col_emit<NP>(rr, vv, al_s[j + HT], j, e, S, ld, np, dvb, pb, pab);
   };
-  const int n_chunk = (int)(t1 - t0), n_walk = (int)(t_stop - t0);
-  // token q's v and dout go to ring slot q % COL_RING; the slot refilled at
-  // step i held token i - 1, whose values step i - 1 has already used
+  // step q's v and dout go to ring slot q % COL_RING; the slot refilled at
+  // step i held step i - 1, whose values step i - 1 has already used
   FP (*ring)[2][32] = ring_all[warp];
-  const float* vp = v + t0 * ld + f;
-  const float* up = dout + t0 * d + f;
+  const float* vp = v + (t0 + r0) * ld + f;
+  const float* up = dout + (t0 + r0) * d + f;
 #pragma unroll
   for (int q = 0; q < COL_RING - 1; ++q) {
     if (q < n_walk) {
@@ -387,62 +399,62 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
       cp_async_pairs<NP>(&ring[q][1][lane], up);
     }
     cp_async_commit();
-    vp += ld;
-    up += d;
+    vp += S * ld;
+    up += S * d;
   }
 #pragma unroll 4
   for (int i = 0; i < n_walk; ++i) {
-    cp_async_wait<COL_RING - 2>();  // token i's copies have landed
+    cp_async_wait<COL_RING - 2>();  // step i's copies have landed
     const int slot = i % COL_RING;
     const FP vr = ring[slot][0][lane], ut = ring[slot][1][lane];
-    const float at = al_s[i + NH];
+    const int ia = r0 + S * i + HT;  // the token's gate at al_s[ia]
+    const float at = al_s[ia];
     if (i + COL_RING - 1 < n_walk) {
       const int refill = (i + COL_RING - 1) % COL_RING;
       cp_async_pairs<NP>(&ring[refill][0][lane], vp);
       cp_async_pairs<NP>(&ring[refill][1][lane], up);
     }
     cp_async_commit();
-    vp += ld;
-    up += d;
-    if (pos == 0) {  // a sequence starts at t
+    vp += S * ld;
+    up += S * d;
+    if (pos < S) {  // the chain's previous token lies in an earlier sequence
 #pragma unroll
-      for (int k = 0; k < NH; ++k) sr[k] = zero;
+      for (int k = 0; k < 3; ++k) sr[k] = zero;
       live = 0;
     }
     FP vt, g, E, A0;  // vt: the conv's input at t (c with PRE)
-    const float ct = PRE ? q_s[i + NH] : at;
+    const float ct = PRE ? q_s[ia] : at;
 #pragma unroll
     for (int q = 0; q < NP; ++q) {
       vt.p[q] = __fmul2_rn(make_float2(ct, ct), vr.p[q]);
       if constexpr (PRE) vt.p[q] = __fmul2_rn(Gv.p[q], vt.p[q]);
-      const float2 y =
-          __ffma2_rn(W0.p[q], sr[NH - 1].p[q],
-                     __ffma2_rn(W1.p[q], sr[2 * DIL - 1].p[q],
-                                __ffma2_rn(W2.p[q], sr[DIL - 1].p[q], __fmul2_rn(W3.p[q], vt.p[q]))));
+      const float2 y = __ffma2_rn(
+          W0.p[q], sr[2].p[q],
+          __ffma2_rn(W1.p[q], sr[1].p[q], __ffma2_rn(W2.p[q], sr[0].p[q], __fmul2_rn(W3.p[q], vt.p[q]))));
       g.p[q] = __fmul2_rn(ut.p[q], silu_grad2(y));
-      E.p[q] = __ffma2_rn(W0.p[q], g.p[q], ar[NH - 1].p[q]);  // dvt of t-NH, complete
-      ar[2 * DIL - 1].p[q] = __ffma2_rn(W1.p[q], g.p[q], ar[2 * DIL - 1].p[q]);
-      ar[DIL - 1].p[q] = __ffma2_rn(W2.p[q], g.p[q], ar[DIL - 1].p[q]);
+      E.p[q] = __ffma2_rn(W0.p[q], g.p[q], ar[2].p[q]);  // dvt of t-3S, complete
+      ar[1].p[q] = __ffma2_rn(W1.p[q], g.p[q], ar[1].p[q]);
+      ar[0].p[q] = __ffma2_rn(W2.p[q], g.p[q], ar[0].p[q]);
       A0.p[q] = PRE ? __fmul2_rn(W3.p[q], g.p[q]) : __ffma2_rn(W3.p[q], g.p[q], ut.p[q]);
     }
     if (i < n_chunk) {
 #pragma unroll
       for (int q = 0; q < NP; ++q) {
-        C0.p[q] = __ffma2_rn(g.p[q], sr[NH - 1].p[q], C0.p[q]);
-        C1.p[q] = __ffma2_rn(g.p[q], sr[2 * DIL - 1].p[q], C1.p[q]);
-        C2.p[q] = __ffma2_rn(g.p[q], sr[DIL - 1].p[q], C2.p[q]);
+        C0.p[q] = __ffma2_rn(g.p[q], sr[2].p[q], C0.p[q]);
+        C1.p[q] = __ffma2_rn(g.p[q], sr[1].p[q], C1.p[q]);
+        C2.p[q] = __ffma2_rn(g.p[q], sr[0].p[q], C2.p[q]);
         C3.p[q] = __ffma2_rn(g.p[q], vt.p[q], C3.p[q]);
       }
     }
-    if (live == NH) emit(E, vr_[NH - 1], i, i - NH);
-    if (pos == T - 1) {  // the sequence ends at t: its later tokens are complete
+    if (live == 3) emit(E, vr_[2], i - 3);
+    if (pos + S >= T) {  // the chain's sequence ends at t: its later tokens are complete
 #pragma unroll
-      for (int k = NH - 1; k >= 1; --k)  // tokens t-k, oldest first
-        if (live >= k && i - k < n_chunk) emit(ar[k - 1], vr_[k - 1], i + NH - k, i - k);
-      if (i < n_chunk) emit(A0, vr, i + NH, i);
+      for (int k = 2; k >= 1; --k)  // steps i-k, oldest first
+        if (live >= k && i - k < n_chunk) emit(ar[k - 1], vr_[k - 1], i - k);
+      if (i < n_chunk) emit(A0, vr, i);
     }
 #pragma unroll
-    for (int k = NH - 1; k > 0; --k) {
+    for (int k = 2; k > 0; --k) {
       ar[k] = ar[k - 1];
       sr[k] = sr[k - 1];
       vr_[k] = vr_[k - 1];
@@ -450,21 +462,22 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
     ar[0] = A0;
     sr[0] = vt;
     vr_[0] = vr;
-    live = live < NH ? live + 1 : NH;
-    pos = pos + 1 == T ? 0 : pos + 1;
+    live = live < 3 ? live + 1 : 3;
+    pos += S;
+    while (pos >= T) pos -= T;  // at most S / T + 1 times
   }
-  if (n_chunk & 31) col_flush(pb, n_chunk & ~31, n_chunk & 31, np, pab);
+  if (n_chunk & 31) col_flush(pb, r0 + S * (n_chunk & ~31), S, n_chunk & 31, np, pab);
 #pragma unroll
   for (int q = 0; q < NP; ++q) {
-    part[(int64_t)chunk * d + f + 2 * q] =
+    part[(int64_t)unit * d + f + 2 * q] =
         make_float4(C0.p[q].x, C1.p[q].x, C2.p[q].x, C3.p[q].x);
-    part[(int64_t)chunk * d + f + 2 * q + 1] =
+    part[(int64_t)unit * d + f + 2 * q + 1] =
         make_float4(C0.p[q].y, C1.p[q].y, C2.p[q].y, C3.p[q].y);
   }
   if constexpr (PRE) {
 #pragma unroll
     for (int q = 0; q < NP; ++q)
-      *reinterpret_cast<float2*>(pre.gvpart + (int64_t)chunk * d + f + 2 * q) = Gacc.p[q];
+      *reinterpret_cast<float2*>(pre.gvpart + (int64_t)unit * d + f + 2 * q) = Gacc.p[q];
   }
 }
 
@@ -798,31 +811,31 @@ __global__ void __launch_bounds__(PN_ROW_THREADS) bw_prenorm_row_kernel(
   }
 }
 
-// dg_v[f] = sum over chunks, in order, of gvpart[chunk][f]
-__global__ void bw_gv_reduce_kernel(const float* __restrict__ gvpart, int chunks, int d,
+// dg_v[f] = sum over the walks, in order, of gvpart[unit][f]
+__global__ void bw_gv_reduce_kernel(const float* __restrict__ gvpart, int units, int d,
                                     float* __restrict__ dgv) {
   const int f = blockIdx.x * blockDim.x + threadIdx.x;
   if (f >= d) return;
   float S = 0.f;
 #pragma unroll 8
-  for (int c = 0; c < chunks; ++c) S += gvpart[(int64_t)c * d + f];
+  for (int c = 0; c < units; ++c) S += gvpart[(int64_t)c * d + f];
   dgv[f] = S;
 }
 
 constexpr int DCONV_WARPS = 32;
 
-// dconv_w[f] = sum over chunks of part[chunk][f]: warp w adds chunks w,
+// dconv_w[f] = sum over the walks of part[unit][f]: warp w adds units w,
 // w + 32, ... in order (its loads all in flight at once for up to 256
-// chunks), then the 32 warp sums are added in warp order.
+// units), then the 32 warp sums are added in warp order.
 __global__ void __launch_bounds__(32 * DCONV_WARPS) bw_dconv_reduce_kernel(
-    const float4* __restrict__ part, int chunks, int d, float4* __restrict__ dw) {
+    const float4* __restrict__ part, int units, int d, float4* __restrict__ dw) {
   __shared__ float4 red[DCONV_WARPS][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int f = blockIdx.x * 32 + lane;
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
   if (f < d) {
 #pragma unroll 8
-    for (int c = warp; c < chunks; c += DCONV_WARPS) {
+    for (int c = warp; c < units; c += DCONV_WARPS) {
       const float4 p = part[(int64_t)c * d + f];
       s.x += p.x;
       s.y += p.y;
@@ -880,13 +893,14 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
   const size_t DKV = up256b((size_t)N * 2 * d * 2);
   const size_t WKV = up256b((size_t)2 * d * E * 2), DW = up256b((size_t)2 * d * E * 4);
   const size_t DA = up256b((size_t)N * col_partials(d, 1) * 4);  // the most partials
-  const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * d * 16);
+  // conv partials of up to three walks (chains) per chunk
+  const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * 3 * d * 16);
   const size_t tg = table_grad_ws_bytes(N * J);
   const size_t SP = scaled ? up256b((size_t)kMaxRowBlocks * d * 4) : 0;
   const size_t RC = prenorm ? up256b((size_t)N * 4) : 0;
   const size_t DC = prenorm ? up256b((size_t)N * d * 4) : 0;
   const size_t DA1 = prenorm ? up256b((size_t)N * 16) : 0;
-  const size_t GVP = prenorm ? up256b((size_t)chunks * d * 4) : 0;
+  const size_t GVP = prenorm ? up256b((size_t)chunks * 3 * d * 4) : 0;
   size_t off[14];
   const size_t sz[14] = {KV, DKV, WKV, DW, DA, NE4, P, kBlasWorkspace, tg, SP, RC, DC, DA1, GVP};
   size_t o = 0;
@@ -965,24 +979,23 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
     return rc;
   const float* kv = have_kv ? kv_saved : w.kv;
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
-  // the plain conv walks two feature pairs per lane, the dilated one (nine
-  // tokens of history in registers) one
-  const int np_lane = dil == 1 ? 2 : 1;
-  const int np = d / col_feat(np_lane), np_pad = col_partials(d, np_lane);
+  // one walk per (chunk, chain): the dilated conv's chunks hold three chains
+  const int units = chunks * dil;
+  const int np = d / col_feat(2), np_pad = col_partials(d, 2);
   const ColPre pre{w.rc, gv, w.dc, w.gvpart};
   // with the pre-conv norm: rc of every token first (the walk's conv input
   // is alpha rc g_v v)
   if (prenorm && (rc = launch_prenorm_rc(kv + d, 2 * d, alpha, N, d, w.rc, s))) return rc;
   {
     auto col = dil == 1 ? (prenorm ? bw_col_kernel<1, 2, true> : bw_col_kernel<1, 2, false>)
-                        : (prenorm ? bw_col_kernel<3, 1, true> : bw_col_kernel<3, 1, false>);
+                        : (prenorm ? bw_col_kernel<3, 2, true> : bw_col_kernel<3, 2, false>);
     const int smem = dil == 1 ? (prenorm ? col_smem_bytes<1, 2, true>() : col_smem_bytes<1, 2, false>())
-                              : (prenorm ? col_smem_bytes<3, 1, true>() : col_smem_bytes<3, 1, false>());
+                              : (prenorm ? col_smem_bytes<3, 2, true>() : col_smem_bytes<3, 2, false>());
     if ((rc = ck(cudaFuncSetAttribute(col, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))))
       return rc;
-    col<<<dim3((unsigned)((chunks + COL_WARPS - 1) / COL_WARPS), (unsigned)np), 32 * COL_WARPS,
+    col<<<dim3((unsigned)((units + COL_WARPS - 1) / COL_WARPS), (unsigned)np), 32 * COL_WARPS,
           smem, s>>>(kv + d, alpha, reinterpret_cast<const float4*>(conv_w), dout, N, T, d, 2 * d,
-                     chunks, w.dkv + d, w.dalpha_part, w.part, pre);
+                     units, w.dkv + d, w.dalpha_part, w.part, pre);
   }
   // the pre-conv norm's backward per token: dv and dalpha (one partial per row)
   const float* da_rows = w.dalpha_part;
@@ -997,7 +1010,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
         w.dc, kv + d, 2 * d, dout, alpha, w.rc, gv, w.dalpha_part, np, np_pad, N, d, w.dkv + d,
         w.da);
     if (scaled)  // dg_v after dg_h, dg_k
-      bw_gv_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(w.gvpart, chunks, d,
+      bw_gv_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(w.gvpart, units, d,
                                                                       dconv_w + 6 * (int64_t)d);
     da_rows = w.da;
     da_np = 1;
@@ -1028,7 +1041,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
           w.spart, (int)grid, d, gscale, dconv_w + 4 * (int64_t)d);
   }
   bw_dconv_reduce_kernel<<<(unsigned)((d + 31) / 32), 32 * DCONV_WARPS, 0, s>>>(
-      w.part, chunks, d, reinterpret_cast<float4*>(dconv_w));
+      w.part, units, d, reinterpret_cast<float4*>(dconv_w));
   if ((rc = ck(cudaGetLastError()))) return rc;
   // [dW_k; dW_v] = [dk | dv]^T e (a contraction over tokens), then split;
   // de = [dk | dv] [W_k; W_v]
