@@ -17,8 +17,11 @@ namespace engram {
 
 namespace {
 
-constexpr int RADIX_BITS = 8;
-constexpr int RADIX = 1 << RADIX_BITS;
+// digits of up to RADIX_MAX_BITS bits: a sort of b key bits takes
+// ceil(b / 10) passes, the bits spread evenly over them (27-bit row ids: 3
+// passes of 9 bits)
+constexpr int RADIX_MAX_BITS = 10;
+constexpr int RADIX_MAX = 1 << RADIX_MAX_BITS;
 constexpr int SORT_THREADS = 256;
 constexpr int SORT_WARPS = SORT_THREADS / 32;
 constexpr int CHUNKS_PER_WARP = 8;                       // 8 x 32 items per warp
@@ -27,24 +30,25 @@ constexpr unsigned FULL = 0xffffffffu;
 
 constexpr size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
 
-__device__ __forceinline__ int digit_of(uint64_t key, int shift) {
-  return (int)((key >> shift) & (RADIX - 1));
+__device__ __forceinline__ int digit_of(uint64_t key, int shift, int radix) {
+  return (int)((key >> shift) & (uint64_t)(radix - 1));
 }
 
-// Counts of each digit in this block's tile -> hist[digit * nblocks + block].
+// Counts of each of the radix digits in this block's tile ->
+// hist[digit * nblocks + block].
 __global__ void __launch_bounds__(SORT_THREADS) radix_hist_kernel(const uint64_t* __restrict__ keys,
-                                                                  int64_t n, int shift,
+                                                                  int64_t n, int shift, int radix,
                                                                   int32_t* __restrict__ hist) {
-  __shared__ int32_t cnt[RADIX];
-  for (int i = threadIdx.x; i < RADIX; i += SORT_THREADS) cnt[i] = 0;
+  __shared__ int32_t cnt[RADIX_MAX];
+  for (int i = threadIdx.x; i < radix; i += SORT_THREADS) cnt[i] = 0;
   __syncthreads();
   const int64_t base = (int64_t)blockIdx.x * TILE;
   for (int i = threadIdx.x; i < TILE; i += SORT_THREADS) {
     const int64_t p = base + i;
-    if (p < n) atomicAdd(&cnt[digit_of(keys[p], shift)], 1);
+    if (p < n) atomicAdd(&cnt[digit_of(keys[p], shift, radix)], 1);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < RADIX; i += SORT_THREADS)
+  for (int i = threadIdx.x; i < radix; i += SORT_THREADS)
     hist[(int64_t)i * gridDim.x + blockIdx.x] = cnt[i];
 }
 
@@ -53,13 +57,14 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_hist_kernel(const uint64_t
 // digit before it in that order.
 __global__ void __launch_bounds__(SORT_THREADS) radix_scatter_kernel(
     const uint64_t* __restrict__ keys_in, const uint32_t* __restrict__ vals_in, int64_t n,
-    int shift, const int32_t* __restrict__ offsets, uint64_t* __restrict__ keys_out,
+    int shift, int radix, const int32_t* __restrict__ offsets, uint64_t* __restrict__ keys_out,
     uint32_t* __restrict__ vals_out) {
-  __shared__ int32_t wcnt[SORT_WARPS][RADIX];
-  __shared__ int32_t boff[RADIX];
+  __shared__ int32_t wcnt[SORT_WARPS][RADIX_MAX];
+  __shared__ int32_t boff[RADIX_MAX];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < SORT_WARPS * RADIX; i += SORT_THREADS) (&wcnt[0][0])[i] = 0;
-  for (int i = threadIdx.x; i < RADIX; i += SORT_THREADS)
+  for (int w = 0; w < SORT_WARPS; ++w)
+    for (int i = threadIdx.x; i < radix; i += SORT_THREADS) wcnt[w][i] = 0;
+  for (int i = threadIdx.x; i < radix; i += SORT_THREADS)
     boff[i] = offsets[(int64_t)i * gridDim.x + blockIdx.x];
   __syncthreads();
 
@@ -74,18 +79,18 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_scatter_kernel(
     const bool ok = p < n;
     k[c] = ok ? keys_in[p] : 0;
     v[c] = ok ? vals_in[p] : 0;
-    const int d = ok ? digit_of(k[c], shift) : RADIX;  // RADIX marks "no item"
+    const int d = ok ? digit_of(k[c], shift, radix) : radix;  // radix marks "no item"
     dg[c] = d;
     const unsigned peers = __match_any_sync(FULL, d);
-    const int before = (d < RADIX) ? wcnt[warp][d] : 0;
+    const int before = (d < radix) ? wcnt[warp][d] : 0;
     rk[c] = before + __popc(peers & lt_mask);
     __syncwarp();
-    if (d < RADIX && (peers & lt_mask) == 0) wcnt[warp][d] = before + __popc(peers);
+    if (d < radix && (peers & lt_mask) == 0) wcnt[warp][d] = before + __popc(peers);
     __syncwarp();
   }
   __syncthreads();
   // exclusive prefix over warps, per digit
-  for (int d = threadIdx.x; d < RADIX; d += SORT_THREADS) {
+  for (int d = threadIdx.x; d < radix; d += SORT_THREADS) {
     int run = 0;
     for (int w = 0; w < SORT_WARPS; ++w) {
       const int t = wcnt[w][d];
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_scatter_kernel(
   __syncthreads();
 #pragma unroll
   for (int c = 0; c < CHUNKS_PER_WARP; ++c) {
-    if (dg[c] < RADIX) {
+    if (dg[c] < radix) {
       const int64_t dst = (int64_t)boff[dg[c]] + wcnt[warp][dg[c]] + rk[c];
       keys_out[dst] = k[c];
       vals_out[dst] = v[c];
@@ -264,12 +269,15 @@ int radix_sort_pairs(uint64_t*& keys, uint32_t*& vals, uint64_t* keys_alt, uint3
                      int64_t n, int key_bits, int32_t* hist, int32_t* bsum, cudaStream_t s) {
   if (n == 0) return ENGRAM_OK;
   const int64_t nblocks = (n + TILE - 1) / TILE;
-  for (int shift = 0; shift < key_bits; shift += RADIX_BITS) {
-    radix_hist_kernel<<<(unsigned)nblocks, SORT_THREADS, 0, s>>>(keys, n, shift, hist);
-    const int rc = launch_scan(hist, hist, (int64_t)RADIX * nblocks, nullptr, bsum, s);
+  const int passes = (key_bits + RADIX_MAX_BITS - 1) / RADIX_MAX_BITS;
+  const int bits = (key_bits + passes - 1) / passes;
+  const int radix = 1 << bits;
+  for (int shift = 0; shift < key_bits; shift += bits) {
+    radix_hist_kernel<<<(unsigned)nblocks, SORT_THREADS, 0, s>>>(keys, n, shift, radix, hist);
+    const int rc = launch_scan(hist, hist, (int64_t)radix * nblocks, nullptr, bsum, s);
     if (rc) return rc;
-    radix_scatter_kernel<<<(unsigned)nblocks, SORT_THREADS, 0, s>>>(keys, vals, n, shift, hist,
-                                                                    keys_alt, vals_alt);
+    radix_scatter_kernel<<<(unsigned)nblocks, SORT_THREADS, 0, s>>>(keys, vals, n, shift, radix,
+                                                                    hist, keys_alt, vals_alt);
     uint64_t* tk = keys;
     keys = keys_alt;
     keys_alt = tk;
@@ -458,7 +466,7 @@ struct SortWs {
 
 constexpr size_t sort_ws_bytes(int64_t n) {
   const int64_t nblocks = (n + TILE - 1) / TILE;
-  return 2 * up256(n * 8) + 2 * up256(n * 4) + up256(RADIX * nblocks * 4 + 4) +
+  return 2 * up256(n * 8) + 2 * up256(n * 4) + up256(RADIX_MAX * nblocks * 4 + 4) +
          2 * up256(n * 4 + 4) + up256((n + 1) * 4) + scan_ws_bytes() + 256;
 }
 
@@ -470,7 +478,7 @@ SortWs carve(void* ws, int64_t n) {
   w.k1 = reinterpret_cast<uint64_t*>(p); p += up256(n * 8);
   w.v0 = reinterpret_cast<uint32_t*>(p); p += up256(n * 4);
   w.v1 = reinterpret_cast<uint32_t*>(p); p += up256(n * 4);
-  w.hist = reinterpret_cast<int32_t*>(p); p += up256(RADIX * nblocks * 4 + 4);
+  w.hist = reinterpret_cast<int32_t*>(p); p += up256(RADIX_MAX * nblocks * 4 + 4);
   w.a = reinterpret_cast<int32_t*>(p); p += up256(n * 4 + 4);
   w.b = reinterpret_cast<int32_t*>(p); p += up256(n * 4 + 4);
   w.c = reinterpret_cast<int32_t*>(p); p += up256((n + 1) * 4);
