@@ -118,7 +118,12 @@ __device__ __forceinline__ float2 silu_grad2(float2 y) {
 
 constexpr int COL_TOK = 128;   // tokens per column chunk; one warp walks one chunk
 constexpr int COL_WARPS = 4;   // chunks per block
-constexpr int COL_RING = 12;   // tokens per warp in a shared-memory ring, 11 of them in flight
+// tokens per warp in a shared-memory ring (all but one in flight): 12, or 8
+// with four pairs per lane, whose slots are twice as large
+template <int NP>
+__host__ __device__ constexpr int col_ring() {
+  return NP >= 4 ? 8 : 12;
+}
 
 // Features per warp of the walk: NP pairs per lane
 __host__ __device__ constexpr int col_feat(int np_lane) { return 64 * np_lane; }
@@ -136,10 +141,13 @@ struct FPairs {
 template <int NP>
 __device__ __forceinline__ FPairs<NP> ld_pairs(const float* q) {
   FPairs<NP> r;
-  if constexpr (NP == 2) {
-    const float4 t = *reinterpret_cast<const float4*>(q);
-    r.p[0] = make_float2(t.x, t.y);
-    r.p[NP - 1] = make_float2(t.z, t.w);
+  if constexpr (NP >= 2) {
+#pragma unroll
+    for (int h = 0; h < NP / 2; ++h) {
+      const float4 t = *reinterpret_cast<const float4*>(q + 4 * h);
+      r.p[2 * h] = make_float2(t.x, t.y);
+      r.p[2 * h + 1] = make_float2(t.z, t.w);
+    }
   } else {
     r.p[0] = *reinterpret_cast<const float2*>(q);
   }
@@ -150,11 +158,13 @@ __device__ __forceinline__ FPairs<NP> ld_pairs(const float* q) {
 // shared-memory slot.
 template <int NP>
 __device__ __forceinline__ void cp_async_pairs(void* dst, const void* src) {
-  if constexpr (NP == 2) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                     (uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src)
-                 : "memory");
+  if constexpr (NP >= 2) {
+#pragma unroll
+    for (int h = 0; h < NP / 2; ++h)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                       (uint32_t)__cvta_generic_to_shared(dst) + 16u * h),
+                   "l"(static_cast<const float*>(src) + 4 * h)
+                   : "memory");
   } else {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
                      (uint32_t)__cvta_generic_to_shared(dst)),
@@ -209,7 +219,14 @@ __device__ __forceinline__ void col_emit(const FPairs<NP>& r, const FPairs<NP>& 
     o[q] = __floats2bfloat162_rn(dvr.x, dvr.y);
     dot = fmaf(r.p[q].x, vv.p[q].x, fmaf(r.p[q].y, vv.p[q].y, dot));
   }
-  if constexpr (NP == 2) {
+  if constexpr (NP == 4) {
+    uint4 w;
+    w.x = *reinterpret_cast<const uint32_t*>(&o[0]);
+    w.y = *reinterpret_cast<const uint32_t*>(&o[1 % NP]);
+    w.z = *reinterpret_cast<const uint32_t*>(&o[2 % NP]);
+    w.w = *reinterpret_cast<const uint32_t*>(&o[3 % NP]);
+    *reinterpret_cast<uint4*>(dvb + j * ld) = w;
+  } else if constexpr (NP == 2) {
     uint2 w;
     w.x = *reinterpret_cast<const uint32_t*>(&o[0]);
     w.y = *reinterpret_cast<const uint32_t*>(&o[NP - 1]);
@@ -239,9 +256,11 @@ __device__ __forceinline__ void col_emit_pre(const FPairs<NP>& r, const FPairs<N
     dot = fmaf(gr.x, a * vv.p[q].x, fmaf(gr.y, a * vv.p[q].y, dot));
     gacc.p[q] = __ffma2_rn(r.p[q], __fmul2_rn(make_float2(qa, qa), vv.p[q]), gacc.p[q]);
   }
-  if constexpr (NP == 2) {
-    *reinterpret_cast<float4*>(dcb + (int64_t)j * d) =
-        make_float4(r.p[0].x, r.p[0].y, r.p[NP - 1].x, r.p[NP - 1].y);
+  if constexpr (NP >= 2) {
+#pragma unroll
+    for (int h = 0; h < NP / 2; ++h)
+      *reinterpret_cast<float4*>(dcb + (int64_t)j * d + 4 * h) =
+          make_float4(r.p[2 * h].x, r.p[2 * h].y, r.p[2 * h + 1].x, r.p[2 * h + 1].y);
   } else {
     *reinterpret_cast<float2*>(dcb + (int64_t)j * d) = r.p[0];
   }
@@ -264,7 +283,7 @@ struct ColPre {
 // and with the pre-conv norm the tokens' alpha rc likewise
 template <int DIL, int NP, bool PRE>
 constexpr int col_smem_bytes() {
-  return COL_WARPS * (COL_RING * 2 * 32 * (int)sizeof(FPairs<NP>) + (int)sizeof(ColPartials) +
+  return COL_WARPS * (col_ring<NP>() * 2 * 32 * (int)sizeof(FPairs<NP>) + (int)sizeof(ColPartials) +
                       (PRE ? 2 : 1) * (COL_TOK + 6 * DIL) * 4);
 }
 
@@ -280,7 +299,7 @@ constexpr int col_smem_bytes() {
 // share.  At token t it forms y_t and dy_t; dvt of token t-3S is then
 // complete, and at a sequence end so are the chain's later ones.  The walk
 // runs three chain steps past the chunk for the last tokens' dy.  v and dout
-// of the next COL_RING - 1 chain tokens are in flight into a per-warp
+// of the next col_ring - 1 chain tokens are in flight into a per-warp
 // shared-memory ring (asynchronous copies, each lane its own bytes).  `live`
 // counts the history's tokens that belong to t's sequence and to this
 // walk (tokens before the chunk are emitted by the previous chunk's walks).
@@ -309,6 +328,7 @@ __global__ void __launch_bounds__(32 * COL_WARPS) bw_col_kernel(
   constexpr int HT = 3 * DIL;  // tokens of conv history
   extern __shared__ __align__(16) unsigned char col_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int COL_RING = col_ring<NP>();
   constexpr int RING_BYTES = COL_RING * 2 * 32 * (int)sizeof(FP);
   auto* ring_all = reinterpret_cast<FP(*)[COL_RING][2][32]>(col_smem);  // [slot][v, dout][lane]
   auto* pb_all = reinterpret_cast<ColPartials*>(col_smem + COL_WARPS * RING_BYTES);
@@ -981,16 +1001,17 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
   // one walk per (chunk, chain): the dilated conv's chunks hold three chains
   const int units = chunks * dil;
-  const int np = d / col_feat(2), np_pad = col_partials(d, 2);
+  constexpr int CP = 2;  // feature pairs per lane of the walk
+  const int np = d / col_feat(CP), np_pad = col_partials(d, CP);
   const ColPre pre{w.rc, gv, w.dc, w.gvpart};
   // with the pre-conv norm: rc of every token first (the walk's conv input
   // is alpha rc g_v v)
   if (prenorm && (rc = launch_prenorm_rc(kv + d, 2 * d, alpha, N, d, w.rc, s))) return rc;
   {
-    auto col = dil == 1 ? (prenorm ? bw_col_kernel<1, 2, true> : bw_col_kernel<1, 2, false>)
-                        : (prenorm ? bw_col_kernel<3, 2, true> : bw_col_kernel<3, 2, false>);
-    const int smem = dil == 1 ? (prenorm ? col_smem_bytes<1, 2, true>() : col_smem_bytes<1, 2, false>())
-                              : (prenorm ? col_smem_bytes<3, 2, true>() : col_smem_bytes<3, 2, false>());
+    auto col = dil == 1 ? (prenorm ? bw_col_kernel<1, CP, true> : bw_col_kernel<1, CP, false>)
+                        : (prenorm ? bw_col_kernel<3, CP, true> : bw_col_kernel<3, CP, false>);
+    const int smem = dil == 1 ? (prenorm ? col_smem_bytes<1, CP, true>() : col_smem_bytes<1, CP, false>())
+                              : (prenorm ? col_smem_bytes<3, CP, true>() : col_smem_bytes<3, CP, false>());
     if ((rc = ck(cudaFuncSetAttribute(col, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))))
       return rc;
     col<<<dim3((unsigned)((units + COL_WARPS - 1) / COL_WARPS), (unsigned)np), 32 * COL_WARPS,
