@@ -70,6 +70,26 @@ def test_dilated_conv_taps_and_short_sequences():
     assert not y[others].any()
 
 
+@pytest.mark.parametrize("T", [1, 2, 3, 7, 12, 20])
+def test_dilated_conv_is_three_interleaved_plain_convs(T):
+    """Taps 3, 6 and 9 tokens back only ever read tokens of the same residue
+    mod 3 within a sequence, so the dilated conv equals three independent
+    dilation-1 convs, one over each residue's subsequence (bit for bit: the
+    same terms in the same order)."""
+    rng = np.random.default_rng(T)
+    B, d = 3, 5
+    c = rng.standard_normal((B * T, 1, d))
+    w = rng.standard_normal((1, d, 4))
+    y = O.causal_conv_v(c, w, T, 3)
+    for b in range(B):
+        for r in range(3):
+            rows = np.arange(b * T + r, (b + 1) * T, 3)
+            if rows.size == 0:
+                continue
+            sub = O.causal_conv_v(c[rows], w, rows.size, 1)
+            assert np.array_equal(y[rows], sub), (b, r)
+
+
 @pytest.mark.parametrize("flags", FLAG_SETS)
 def test_decode_streaming_equals_whole_sequences(flags):
     B, T, M, d = 2, 12, 2, 8
