@@ -572,7 +572,7 @@ def _graph_time(fn, steps, warmup, stream):
 def bench_fwd_bwd_27b(dev, steps=10):
     """Training step of the 27B-shaped layer (8 x 4,096 tokens, d 2,560, 16 x
     80 dims, 5.7B-parameter bf16 table): hash, forward (gather, fused passes,
-    alpha, k and v saved), backward (bf16: elementwise kernels, cuBLAS GEMMs,
+    alpha, k and v saved), backward (bf16: elementwise kernels, tensor-core GEMMs,
     sparse table gradient); the same with k and v recomputed in the
     backward instead of saved; with the dilated conv (taps 3, 6 and 9
     tokens back); and with the pre-conv RMSNorm."""

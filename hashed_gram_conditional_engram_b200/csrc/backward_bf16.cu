@@ -1,21 +1,18 @@
 // Backward of the bf16 layer (one branch) at full scale.
 //
-// The four dense contractions of the backward are plain GEMMs with no work
-// to fuse into them: k and v are recomputed as e W_k^T and e W_v^T, the
-// weight gradients are contractions over tokens (dW = d{k,v}^T e) and the
-// row gradient is de = dk W_k + dv W_v.  They run in cuBLAS (bf16 operands,
-// fp32 accumulation), loaded with dlopen on first use so that the library
-// itself has no load-time dependency on it.  Everything between them -- the
-// conv and SiLU backward, the gate, both RMSNorm backwards -- is in the
-// kernels below, and the table rows' gradient goes through the same
-// deterministic sort-and-segment-sum as the fp32 path.
+// The dense contractions of the backward are plain GEMMs with no work to
+// fuse into them: k and v are recomputed as e W_k^T and e W_v^T (unless the
+// forward kept them), the weight gradients are contractions over tokens
+// (dW = d{k,v}^T e) and the row gradient is de = dk W_k + dv W_v.  They run
+// on the tensor cores (gemm_tc.cu: tcgen05, bf16 operands, fp32
+// accumulation).  Everything between them -- the conv and SiLU backward, the
+// gate, both RMSNorm backwards -- is in the kernels below, and the table
+// rows' gradient goes through the same deterministic sort-and-segment-sum as
+// the fp32 path.
 //
 // Method: discuss.deepseek.club 二.1 (2) (gate with h as query, e as key and
 // value; 1-D conv; residual); gitcode.csdn.net blog, end-to-end training
 // paragraph (deterministic lookups give consistent gradients to the slots).
-#include <cublas_v2.h>
-#include <dlfcn.h>
-
 #include <algorithm>
 #include <mutex>
 
@@ -24,72 +21,6 @@
 namespace engram {
 
 namespace {
-
-// ------------------------------------------------------------ cuBLAS, loaded late
-
-struct Blas {
-  bool ok = false;
-  cublasStatus_t (*create)(cublasHandle_t*) = nullptr;
-  cublasStatus_t (*set_stream)(cublasHandle_t, cudaStream_t) = nullptr;
-  cublasStatus_t (*set_workspace)(cublasHandle_t, void*, size_t) = nullptr;
-  cublasStatus_t (*gemm_ex)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int,
-                            const void*, const void*, cudaDataType, int, const void*, cudaDataType,
-                            int, const void*, void*, cudaDataType, int, cublasComputeType_t,
-                            cublasGemmAlgo_t) = nullptr;
-};
-
-Blas& blas() {
-  static Blas b;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* h = dlopen("libcublas.so.12", RTLD_NOW | RTLD_LOCAL);
-    if (h == nullptr) return;
-    b.create = reinterpret_cast<decltype(b.create)>(dlsym(h, "cublasCreate_v2"));
-    b.set_stream = reinterpret_cast<decltype(b.set_stream)>(dlsym(h, "cublasSetStream_v2"));
-    b.set_workspace =
-        reinterpret_cast<decltype(b.set_workspace)>(dlsym(h, "cublasSetWorkspace_v2"));
-    b.gemm_ex = reinterpret_cast<decltype(b.gemm_ex)>(dlsym(h, "cublasGemmEx"));
-    b.ok = b.create && b.set_stream && b.set_workspace && b.gemm_ex;
-  });
-  return b;
-}
-
-constexpr int kMaxDevices = 64;
-
-// One handle per device, created on first use and kept for the process.
-int blas_handle(cudaStream_t s, void* workspace, cublasHandle_t* out) {
-  static cublasHandle_t handles[kMaxDevices] = {};
-  static std::mutex mu;
-  Blas& b = blas();
-  if (!b.ok) return ENGRAM_ERR_UNSUPPORTED;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ENGRAM_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(mu);
-  if (handles[dev] == nullptr && b.create(&handles[dev]) != CUBLAS_STATUS_SUCCESS) {
-    handles[dev] = nullptr;
-    return ENGRAM_ERR_CUDA;
-  }
-  if (b.set_stream(handles[dev], s) != CUBLAS_STATUS_SUCCESS ||
-      b.set_workspace(handles[dev], workspace, kBlasWorkspace) != CUBLAS_STATUS_SUCCESS)
-    return ENGRAM_ERR_CUDA;
-  *out = handles[dev];
-  return ENGRAM_OK;
-}
-
-// C[m x n] (row-major, fp32, row stride ldc) = op(A)[m x k] . op(B)[k x n]
-// + beta * C with A, B bf16 row-major: op(A) = A (a_t = false, A is [m x k])
-// or A^T (A is [k x m]), rows lda apart; likewise B.  Row-major C = A.B is
-// column-major C^T = B^T.A^T, which is what cuBLAS is asked for.
-int gemm_rm(cublasHandle_t hd, bool a_t, bool b_t, int m, int n, int k, const void* A, int lda,
-            const void* B, int ldb, float* C, int ldc, float beta) {
-  const float alpha = 1.0f;
-  const cublasOperation_t opB = b_t ? CUBLAS_OP_T : CUBLAS_OP_N;
-  const cublasOperation_t opA = a_t ? CUBLAS_OP_T : CUBLAS_OP_N;
-  const cublasStatus_t st =
-      blas().gemm_ex(hd, opB, opA, n, m, k, &alpha, B, CUDA_R_16BF, ldb, A, CUDA_R_16BF, lda,
-                     &beta, C, CUDA_R_32F, ldc, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-  return st == CUBLAS_STATUS_SUCCESS ? ENGRAM_OK : ENGRAM_ERR_CUDA;
-}
 
 // ------------------------------------------------------------ elementwise backward
 //
@@ -878,26 +809,24 @@ __global__ void __launch_bounds__(32 * DCONV_WARPS) bw_dconv_reduce_kernel(
   }
 }
 
-// Workspace: [k | v] fp32 [N, 2d]; [dk | dv] bf16 [N, 2d]; [W_k; W_v] bf16
-// and [dW_k; dW_v] fp32 [2d, E]; dalpha partials [N, up to d/64 padded to 4]; de fp32 [N, E]
-// when the caller passes none; conv partials; cuBLAS's workspace; the table
+// Workspace: [k | v] fp32 [N, 2d]; [dk | dv] bf16 [N, 2d]; dalpha partials
+// [N, up to d/64 padded to 4]; de fp32 [N, E] when the caller passes none;
+// conv partials; the weight-gradient GEMM's tile counters; the table
 // gradient's sort buffers.
 struct BwdBf16Ws {
   // k and v stay fp32: dh and dalpha are sums whose terms can cancel, so a
   // bf16 rounding of k or v would show at full size in a small result.
   // They share rows (kv [N, 2d] = [k | v]), as do dk and dv, and W_k, W_v
-  // are stacked (Wkv [2d, E]), so that each pair of GEMMs is one.
+  // are read as one stacked operand, so that each pair of GEMMs is one.
   float* kv;  // recomputed here, or NULL when the forward saved them
   __nv_bfloat16* dkv;
-  __nv_bfloat16* Wkv;
-  float* dWkv;          // [2d, E], copied out to dWk and dWv
   float *dalpha_part, *de;  // partials of <dvt, v>, padded rows
   float4* part;
   float* spart;  // with norm scales: [kMaxRowBlocks][d] sums of the row blocks
   // with the pre-conv norm: rc [N], dc [N, d], dalpha rows [N, 4], the
   // chunks' g_v sums [chunks, d]
   float *rc, *dc, *da, *gvpart;
-  void* blas_ws;
+  void* gemm_ws;
   void* tg_ws;
   size_t tg_bytes;
 };
@@ -911,7 +840,6 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
   const int64_t chunks = (N + COL_TOK - 1) / COL_TOK;
   const size_t KV = kv_saved ? 0 : up256b((size_t)N * 2 * d * 4);
   const size_t DKV = up256b((size_t)N * 2 * d * 2);
-  const size_t WKV = up256b((size_t)2 * d * E * 2), DW = up256b((size_t)2 * d * E * 4);
   const size_t DA = up256b((size_t)N * col_partials(d, 1) * 4);  // the most partials
   // conv partials of up to three walks (chains) per chunk
   const size_t NE4 = up256b((size_t)N * E * 4), P = up256b((size_t)chunks * 3 * d * 16);
@@ -921,10 +849,11 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
   const size_t DC = prenorm ? up256b((size_t)N * d * 4) : 0;
   const size_t DA1 = prenorm ? up256b((size_t)N * 16) : 0;
   const size_t GVP = prenorm ? up256b((size_t)chunks * 3 * d * 4) : 0;
-  size_t off[14];
-  const size_t sz[14] = {KV, DKV, WKV, DW, DA, NE4, P, kBlasWorkspace, tg, SP, RC, DC, DA1, GVP};
+  const size_t GF = gemm_dw_ws_bytes(d, E);
+  size_t off[12];
+  const size_t sz[12] = {KV, DKV, DA, NE4, P, GF, tg, SP, RC, DC, DA1, GVP};
   size_t o = 0;
-  for (int i = 0; i < 14; ++i) {
+  for (int i = 0; i < 12; ++i) {
     off[i] = o;
     o += sz[i];
   }
@@ -932,19 +861,17 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
     char* p = static_cast<char*>(base);
     w->kv = kv_saved ? nullptr : reinterpret_cast<float*>(p + off[0]);
     w->dkv = reinterpret_cast<__nv_bfloat16*>(p + off[1]);
-    w->Wkv = reinterpret_cast<__nv_bfloat16*>(p + off[2]);
-    w->dWkv = reinterpret_cast<float*>(p + off[3]);
-    w->dalpha_part = reinterpret_cast<float*>(p + off[4]);
-    w->de = reinterpret_cast<float*>(p + off[5]);
-    w->part = reinterpret_cast<float4*>(p + off[6]);
-    w->blas_ws = p + off[7];
-    w->tg_ws = p + off[8];
+    w->dalpha_part = reinterpret_cast<float*>(p + off[2]);
+    w->de = reinterpret_cast<float*>(p + off[3]);
+    w->part = reinterpret_cast<float4*>(p + off[4]);
+    w->gemm_ws = p + off[5];
+    w->tg_ws = p + off[6];
     w->tg_bytes = tg;
-    w->spart = scaled ? reinterpret_cast<float*>(p + off[9]) : nullptr;
-    w->rc = prenorm ? reinterpret_cast<float*>(p + off[10]) : nullptr;
-    w->dc = prenorm ? reinterpret_cast<float*>(p + off[11]) : nullptr;
-    w->da = prenorm ? reinterpret_cast<float*>(p + off[12]) : nullptr;
-    w->gvpart = prenorm ? reinterpret_cast<float*>(p + off[13]) : nullptr;
+    w->spart = scaled ? reinterpret_cast<float*>(p + off[7]) : nullptr;
+    w->rc = prenorm ? reinterpret_cast<float*>(p + off[8]) : nullptr;
+    w->dc = prenorm ? reinterpret_cast<float*>(p + off[9]) : nullptr;
+    w->da = prenorm ? reinterpret_cast<float*>(p + off[10]) : nullptr;
+    w->gvpart = prenorm ? reinterpret_cast<float*>(p + off[11]) : nullptr;
   }
   return o;
 }
@@ -954,14 +881,6 @@ size_t bwd_bf16_layout(void* base, int64_t N, int d, int E, int J, bool kv_saved
 size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved, bool scaled,
                               bool prenorm) {
   return bwd_bf16_layout(nullptr, N, d, E, J, kv_saved, scaled, prenorm, nullptr);
-}
-
-int blas_gemm_bf16(cudaStream_t s, void* blas_ws, bool a_t, bool b_t, int m, int n, int k,
-                   const void* A, int lda, const void* B, int ldb, float* C, int ldc, float beta) {
-  cublasHandle_t hd;
-  const int rc = blas_handle(s, blas_ws, &hd);
-  if (rc) return rc;
-  return gemm_rm(hd, a_t, b_t, m, n, k, A, lda, B, ldb, C, ldc, beta);
 }
 
 int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bfloat16* e,
@@ -978,25 +897,16 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   const bool scaled = gscale != nullptr;
   if (ws_bytes < backward_bf16_ws_bytes(N, d, E, hp.J, have_kv, scaled, prenorm))
     return ENGRAM_ERR_WORKSPACE;
-  if (N > 0x7fffffffLL / 8) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
+  if (!gemm_supported(N, d, E)) return ENGRAM_ERR_UNSUPPORTED;
   // a row in registers; whole column blocks; 16-byte multiples for the row copies
   if (d > ROW_THREADS * ROW_VEC * ROW_MAX_ITEMS || d % 256 != 0 || (dil != 1 && dil != 3))
     return ENGRAM_ERR_UNSUPPORTED;
   BwdBf16Ws w;
   bwd_bf16_layout(ws, N, d, E, hp.J, have_kv, scaled, prenorm, &w);
   if (de == nullptr) de = w.de;
-  cublasHandle_t hd;
-  int rc = blas_handle(s, w.blas_ws, &hd);
-  if (rc) return rc;
-  const int n = (int)N;
-  // W_k and W_v stacked (for de), then, unless the forward saved them,
-  // [k | v] = e [W_k; W_v]^T (fp32)
-  const size_t wbytes = (size_t)d * E * 2;
-  if ((rc = ck(cudaMemcpyAsync(w.Wkv, Wk, wbytes, cudaMemcpyDeviceToDevice, s)))) return rc;
-  if ((rc = ck(cudaMemcpyAsync(w.Wkv + (size_t)d * E, Wv, wbytes, cudaMemcpyDeviceToDevice, s))))
-    return rc;
-  if (!have_kv && (rc = gemm_rm(hd, false, true, n, 2 * d, E, e, E, w.Wkv, E, w.kv, 2 * d, 0.f)))
-    return rc;
+  int rc;
+  // unless the forward saved them, [k | v] = e [W_k; W_v]^T (fp32)
+  if (!have_kv && (rc = launch_gemm_kv(e, Wk, Wv, N, d, E, w.kv, 2 * d, s))) return rc;
   const float* kv = have_kv ? kv_saved : w.kv;
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
   // one walk per (chunk, chain): the dilated conv's chunks hold three chains
@@ -1064,14 +974,10 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   bw_dconv_reduce_kernel<<<(unsigned)((d + 31) / 32), 32 * DCONV_WARPS, 0, s>>>(
       w.part, units, d, reinterpret_cast<float4*>(dconv_w));
   if ((rc = ck(cudaGetLastError()))) return rc;
-  // [dW_k; dW_v] = [dk | dv]^T e (a contraction over tokens), then split;
-  // de = [dk | dv] [W_k; W_v]
-  if ((rc = gemm_rm(hd, true, false, 2 * d, E, n, w.dkv, 2 * d, e, E, w.dWkv, E, 0.f))) return rc;
-  const size_t gbytes = (size_t)d * E * 4;
-  if ((rc = ck(cudaMemcpyAsync(dWk, w.dWkv, gbytes, cudaMemcpyDeviceToDevice, s)))) return rc;
-  if ((rc = ck(cudaMemcpyAsync(dWv, w.dWkv + (size_t)d * E, gbytes, cudaMemcpyDeviceToDevice, s))))
-    return rc;
-  if ((rc = gemm_rm(hd, false, false, n, E, 2 * d, w.dkv, 2 * d, w.Wkv, E, de, E, 0.f))) return rc;
+  // [dW_k; dW_v] = [dk | dv]^T e (a contraction over tokens, rows d.. into
+  // dW_v); de = [dk | dv] [W_k; W_v]
+  if ((rc = launch_gemm_dw(w.dkv, e, N, d, E, dWk, dWv, w.gemm_ws, s))) return rc;
+  if ((rc = launch_gemm_de(w.dkv, Wk, Wv, N, d, E, de, s))) return rc;
   // the table rows' gradient from de, in the deterministic order
   return launch_table_grad(hp, idx, de, N, dtab_keys, dtab_rows, n_unique, w.tg_ws, w.tg_bytes, s);
 }

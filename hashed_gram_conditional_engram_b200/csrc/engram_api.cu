@@ -59,9 +59,9 @@ inline bool bf16_prenorm(const engram_cfg_t* c) {
 inline size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 // bf16 forward workspace: the passes' buffers, then g_h g_k (norm scales),
-// then with the pre-conv norm v [N, d] fp32, rc [N] and cuBLAS's workspace
+// then with the pre-conv norm v [N, d] fp32 and rc [N]
 struct Bf16FwdWs {
-  size_t gg, vbuf, rc, blas, total;
+  size_t gg, vbuf, rc, total;
 };
 inline Bf16FwdWs bf16_fwd_ws(const engram_cfg_t* c, int64_t n) {
   const int d = c->d_model, E = 2 * c->K * c->D_h;
@@ -70,8 +70,7 @@ inline Bf16FwdWs bf16_fwd_ws(const engram_cfg_t* c, int64_t n) {
   w.vbuf = w.gg + (bf16_scaled(c) ? up256((size_t)d * 4) : 0);
   const bool pn = bf16_prenorm(c);
   w.rc = w.vbuf + (pn ? up256((size_t)n * d * 4) : 0);
-  w.blas = w.rc + (pn ? up256((size_t)n * 4) : 0);
-  w.total = w.blas + (pn ? kBlasWorkspace : 0);
+  w.total = w.rc + (pn ? up256((size_t)n * 4) : 0);
   return w;
 }
 
@@ -251,8 +250,7 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
   // the pre-conv norm: v into the kept [k | v] rows when there are any
   PrenormFwd pn{bf16_scaled(cfg) ? conv_w + 6 * d : nullptr,
                 kv_save != nullptr ? kv_save + d : reinterpret_cast<float*>(wsb + wl.vbuf),
-                kv_save != nullptr ? 2 * d : d, reinterpret_cast<float*>(wsb + wl.rc),
-                wsb + wl.blas};
+                kv_save != nullptr ? 2 * d : d, reinterpret_cast<float*>(wsb + wl.rc)};
   return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
                            static_cast<const __nv_bfloat16*>(Wk),
                            static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,

@@ -121,12 +121,21 @@ int launch_table_grad_noalloc(const HeadParams& hp, const int32_t* idx, const fl
 int launch_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_c_out, void* ws,
                       size_t ws_bytes, cudaStream_t s);
 
-// cuBLAS, loaded on first use: C [m x n] (row-major fp32, rows ldc apart) =
-// op(A) op(B) + beta C with bf16 row-major operands (op = transpose when
-// a_t / b_t), on stream s with kBlasWorkspace bytes of blas_ws
-constexpr size_t kBlasWorkspace = 32u << 20;
-int blas_gemm_bf16(cudaStream_t s, void* blas_ws, bool a_t, bool b_t, int m, int n, int k,
-                   const void* A, int lda, const void* B, int ldb, float* C, int ldc, float beta);
+// bf16 tensor-core GEMMs with fp32 output (gemm_tc.cu); shapes: d a
+// multiple of 256, E of 64, W_k and W_v [d, E], token rows for the rest.
+int gemm_supported(int64_t N, int d, int E);
+// C [N, 2d] (rows ldc floats apart) = e [W_k; W_v]^T, or C [N, d] = e W_v^T
+// when Wk is NULL
+int launch_gemm_kv(const __nv_bfloat16* e, const __nv_bfloat16* Wk, const __nv_bfloat16* Wv,
+                   int64_t N, int d, int E, float* C, int64_t ldc, cudaStream_t s);
+// dW_k [d, E] and dW_v [d, E] = [dk | dv]^T e over the N tokens (dkv bf16
+// [N, 2d]); ws: gemm_dw_ws_bytes of tile counters
+size_t gemm_dw_ws_bytes(int d, int E);
+int launch_gemm_dw(const __nv_bfloat16* dkv, const __nv_bfloat16* e, int64_t N, int d, int E,
+                   float* dWk, float* dWv, void* ws, cudaStream_t s);
+// de [N, E] = [dk | dv] [W_k; W_v]
+int launch_gemm_de(const __nv_bfloat16* dkv, const __nv_bfloat16* Wk, const __nv_bfloat16* Wv,
+                   int64_t N, int d, int E, float* de, cudaStream_t s);
 
 // pre-conv RMSNorm of bf16 layers: rc[t] = (alpha_t^2 <v_t, v_t> / d + eps)^(-1/2)
 int launch_prenorm_rc(const float* v, int ldv, const float* alpha, int64_t N, int d, float* rc,
@@ -139,14 +148,13 @@ struct PrenormFwd {
   float* vbuf;
   int ldv;
   float* rc;        // [N]
-  void* blas_ws;    // kBlasWorkspace bytes
 };
 int launch_prenorm_tail(const PrenormFwd& p, const __nv_bfloat16* e, const __nv_bfloat16* Wv,
                         const __nv_bfloat16* h, const float* conv_w, const float* alpha,
                         float* conv_state, __nv_bfloat16* out, int dil, int64_t N, int T, int d,
                         int E, cudaStream_t s);
 
-// bf16 backward (one branch): elementwise kernels here, plain GEMMs in cuBLAS
+// bf16 backward (one branch): elementwise kernels and the tensor-core GEMMs
 // kv_saved: the forward's fp32 [N, 2d] k and v, or NULL to recompute them
 size_t backward_bf16_ws_bytes(int64_t N, int d, int E, int J, bool kv_saved, bool scaled,
                               bool prenorm);

@@ -4,7 +4,7 @@
 // The norm needs, per token, the sum of squares over all d features of vt,
 // while the tensor-core pass V spreads a token's features over the CTAs of
 // its tile.  So with this variant the layer runs pass K and the gate as
-// usual, then v = e W_v^T as a plain GEMM (cuBLAS, fp32 out), one warp per
+// usual, then v = e W_v^T as a plain tensor-core GEMM (fp32 out), one warp per
 // token for rc = (alpha^2 <v, v> / d + eps)^(-1/2) (RMSNorm(vt) = rc vt),
 // and a walk along each feature over the tokens for the conv, SiLU and
 // residual: out = h + vt + SiLU(y), y_t = sum_i w_i c_{t-(3-i) dil}.
@@ -143,9 +143,8 @@ int launch_prenorm_tail(const PrenormFwd& p, const __nv_bfloat16* e, const __nv_
                         const __nv_bfloat16* h, const float* conv_w, const float* alpha,
                         float* conv_state, __nv_bfloat16* out, int dil, int64_t N, int T, int d,
                         int E, cudaStream_t s) {
-  if (N > 0x7fffffffLL) return ENGRAM_ERR_UNSUPPORTED;  // cuBLAS takes int sizes
   // v = e W_v^T, fp32, rows ldv apart
-  int rc = blas_gemm_bf16(s, p.blas_ws, false, true, (int)N, d, E, e, E, Wv, E, p.vbuf, p.ldv, 0.f);
+  int rc = launch_gemm_kv(e, nullptr, Wv, N, d, E, p.vbuf, p.ldv, s);
   if (rc) return rc;
   if ((rc = launch_prenorm_rc(p.vbuf, p.ldv, alpha, N, d, p.rc, s))) return rc;
   const float4* w = reinterpret_cast<const float4*>(conv_w);

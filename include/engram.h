@@ -61,9 +61,9 @@ enum { ENGRAM_F32 = 0, ENGRAM_BF16 = 1 };
  * ([p2] short depthwise causal conv; [p5 二.1 (2)] 一维卷积; [p5 二.2]).  fp32
  * layers take any combination; bf16 layers (one branch) too, where
  * ENGRAM_CONV_PER_BRANCH is the same as a shared conv.  With
- * ENGRAM_CONV_PRENORM a bf16 layer computes v = e W_v^T with cuBLAS (fp32)
- * after the gate, and its forward workspace holds v, a per-token scale and
- * cuBLAS's 32 MB. */
+ * ENGRAM_CONV_PRENORM a bf16 layer computes v = e W_v^T as a tensor-core
+ * GEMM (fp32 out) after the gate, and its forward workspace holds v and a
+ * per-token scale. */
 #define ENGRAM_CONV_DILATED 2     /* taps at t, t-3, t-6, t-9 (dilation 3 = the largest order) */
 #define ENGRAM_CONV_PRENORM 4     /* the conv reads RMSNorm(vt) (times g_v with NORM_SCALES) */
 #define ENGRAM_CONV_PER_BRANCH 8  /* conv weights per branch */
@@ -246,9 +246,10 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
  * (the forward's alpha) required; dout and every gradient fp32.  The
  * elementwise part runs in fp32; the plain GEMMs (k and v recomputed in fp32
  * as one GEMM against [W_k; W_v], [dW_k; dW_v] as one, de as one with
- * K = 2 d_model) run in cuBLAS with bf16 operands (dk and dv rounded to bf16
- * once) and fp32 accumulation, loaded on first use (ENGRAM_ERR_UNSUPPORTED
- * if libcublas.so.12 cannot be loaded).  A device-side wait that runs out
+ * K = 2 d_model) run on the tensor cores with bf16 operands (dk and dv
+ * rounded to bf16 once) and fp32 accumulation.  The weight gradients are
+ * summed over the tokens in an order fixed by the launch configuration, so
+ * they are reproducible from call to call.  A device-side wait that runs out
  * sets ENGRAM_STATUS_TIMEOUT.
  */
 int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,
