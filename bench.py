@@ -337,20 +337,11 @@ def run_ours(args):
         if ev is not None:
             ev[3].record(stream)
 
-    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for i in range(args.warmup):
-        if i == 1:
-            w0.record(stream)
         step()
-    w1.record(stream)
     torch.cuda.synchronize()
-    est_step_ms = w0.elapsed_time(w1) / max(1, args.warmup - 1)
     if eg.engram_get_status(stream) != 0:
         raise RuntimeError("device status word set during warm-up")
-    # a one-warp probe beside the timed steps reads the SM clock they run at
-    probe = torch.zeros(2, dtype=torch.int64, device=dev)
-    probe_stream = torch.cuda.Stream(dev)
-    probe_ns = max(1000, int(0.9 * est_step_ms * args.steps * 1e6))
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
@@ -367,21 +358,6 @@ def run_ours(args):
         clk.end()
         barrier()
     clocks = clk.summary() or {}
-    # the same steps once more, untimed, with the clock probe beside them (a
-    # probe inside the timed region would hold one SM away from the
-    # persistent passes)
-    torch.cuda.synchronize()
-    eg.engram_clock_probe(probe, probe_ns, probe_stream)
-    for k in range(args.steps):
-        step()
-    torch.cuda.synchronize()
-    pc, pns = probe.cpu().tolist()
-    if pns > 0:
-        clocks["sm_mhz_device"] = 1000.0 * pc / pns
-        clocks["sm_mhz_device_how"] = ("SM cycles / global-timer ns of a one-warp probe over "
-                                       f"{pns / 1e6:.1f} ms of an untimed repeat of the timed "
-                                       "steps (the driver's clock query keeps reading the "
-                                       "maximum while board power management lowers it)")
     elapsed_ms = start.elapsed_time(end)
     t_hash = sum(ev[0].elapsed_time(ev[1]) for ev in evs) / args.steps
     t_gather = sum(ev[1].elapsed_time(ev[2]) for ev in evs) / args.steps

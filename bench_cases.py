@@ -2,17 +2,17 @@
 shape, a few times, for profiling a kernel alone (e.g. under Nsight Compute)
 without the rest of the layer's inputs on the device.
 
-    python -m hashed_gram_conditional_engram_b200.kernel_cases fused \
+    python bench_cases.py fused \
         [--tokens 32768] [--d 2560] [--heads 16] [--dh 80] [--seq 4096] [--reps 3]
-    python -m hashed_gram_conditional_engram_b200.kernel_cases gather [...]
-    python -m hashed_gram_conditional_engram_b200.kernel_cases hash [...]
-    python -m hashed_gram_conditional_engram_b200.kernel_cases decode \
+    python bench_cases.py gather [...]
+    python bench_cases.py hash [...]
+    python bench_cases.py decode \
         --tokens 256 --d 4096 --dh 128 --rows 1000003
-    python -m hashed_gram_conditional_engram_b200.kernel_cases tablegrad [...]
-    python -m hashed_gram_conditional_engram_b200.kernel_cases hostgather \
+    python bench_cases.py tablegrad [...]
+    python bench_cases.py hostgather \
         --tokens 8192 --seq 2048 --dh 160 --rows 1000003
-    python -m hashed_gram_conditional_engram_b200.kernel_cases backward [...]
-    python -m hashed_gram_conditional_engram_b200.kernel_cases hostcache \
+    python bench_cases.py backward [...]
+    python bench_cases.py hostcache \
         --tokens 8192 --seq 2048 --dh 160 --rows 1000003 [--cache-rows 1048576]
 
 `fused` runs engram_forward with table = NULL on random gathered rows, i.e.
@@ -37,8 +37,8 @@ import argparse
 import numpy as np
 import torch
 
-from . import engram as eg
-from . import synth
+from hashed_gram_conditional_engram_b200 import engram as eg
+from hashed_gram_conditional_engram_b200 import synth
 
 
 def main(argv=None):
@@ -60,7 +60,7 @@ def main(argv=None):
     ap.add_argument("--prenorm", action="store_true",
                     help="fused, backward, decode: the pre-conv RMSNorm (no learnable g_v)")
     a = ap.parse_args(argv)
-    from . import build
+    from hashed_gram_conditional_engram_b200 import build
     build.build()
     dev = torch.device("cuda")
     K = a.heads // 2

@@ -112,25 +112,6 @@ HeadParams make_head_params(const engram_cfg_t* cfg) {
 
 using namespace engram;
 
-namespace engram {
-namespace {
-// One warp: SM cycles against the global timer over a window of spin_ns.
-__global__ void clock_probe_kernel(unsigned long long spin_ns, unsigned long long* out) {
-  if (threadIdx.x != 0) return;
-  unsigned long long g0, g;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g0));
-  const long long c0 = clock64();
-  g = g0;
-  while (g - g0 < spin_ns) {
-    __nanosleep(2000);
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g));
-  }
-  const long long c1 = clock64();
-  out[0] = (unsigned long long)(c1 - c0);
-  out[1] = g - g0;
-}
-}  // namespace
-}  // namespace engram
 
 extern "C" {
 
@@ -477,18 +458,6 @@ int engram_get_status(void* stream) {
   if (cudaMemsetAsync(p, 0, sizeof(v), s) != cudaSuccess) return ENGRAM_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return ENGRAM_ERR_CUDA;
   return (int)(v & 0x7fffffffu);
-}
-
-int engram_clock_probe(uint64_t* out, int64_t spin_ns, void* stream) {
-  if (out == nullptr || spin_ns < 1 || spin_ns > 10000000000LL) return ENGRAM_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(out) & 7u) != 0) return ENGRAM_ERR_MISALIGNED;
-  // the SM it lands on keeps the largest shared-memory split, so kernels that
-  // need it can still share that SM
-  cudaFuncSetAttribute(clock_probe_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                       (int)cudaSharedmemCarveoutMaxShared);
-  clock_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((unsigned long long)spin_ns,
-                                                          reinterpret_cast<unsigned long long*>(out));
-  return ck(cudaGetLastError());
 }
 
 int engram_device_sm_count(void) {

@@ -25,17 +25,18 @@
 //               TMA store (fp32), or plain stores for split tiles (below);
 //   warp 10     B producer: this CTA's half of the tile's 256 columns.
 //
-// Scheduling.  With many tiles each pair takes whole tiles p, p + P, ...
-// The weight gradient has few output tiles (2d/256 x E/256 = 100 at the
-// 27B shape) and a long K (one row per token), so there each pair takes an
-// equal share of the (tile, k step) iterations instead (stream-K).  A tile
-// whose iterations fall to several pairs is summed in a fixed order: the
-// pair holding the tile's last k steps stores its partial first (it reaches
-// it first: a pair's range starts there), then each pair below it, once the
-// counter of the tile shows that all 16 epilogue warps of the pair above
-// have stored, loads the sum so far, adds its own partial and stores.  So
-// the result does not depend on timing.  Every wait is bounded in time; one
-// that runs out sets ENGRAM_STATUS_TIMEOUT and the CTA winds down.
+// Scheduling.  Each pair takes units p, p + P, ... of the output's pair
+// tiles.  The weight gradient has few output tiles (2d/256 x E/256 = 100 at
+// the 27B shape) and a long K (one row per token), so there the k steps of
+// every tile are cut into S parts and unit u is part u / tiles of tile
+// u % tiles: the pairs at work at any moment all read the same stretch of
+// tokens, which stays in L2 while every tile takes its turn on it.  A tile's
+// parts are summed in a fixed order: part 0 stores its sum, then part s,
+// once the tile's counter shows that all 16 epilogue warps of part s - 1
+// have stored, loads the sum so far, adds its own and stores (part s - 1
+// ran about one round of units earlier, so the wait is rarely felt).  The
+// result therefore does not depend on timing.  Every wait is bounded in
+// time; one that runs out sets ENGRAM_STATUS_TIMEOUT and the CTA winds down.
 #include "tc_ptx.cuh"
 
 namespace engram {
@@ -48,11 +49,13 @@ constexpr int GN = 256;                       // columns of a pair tile (N of on
 constexpr int G_EPI = 8;                      // epilogue warps
 constexpr int G_BP_WARP = 2 + G_EPI;          // B-operand producer
 constexpr int G_THREADS = (3 + G_EPI) * 32;
-constexpr int G_STAGES = 5;
+constexpr int G_STAGES = 6;
 constexpr int G_A_BYTES = BM * BK * 2;        // 128 rows x 64 k
 constexpr int G_B_BYTES = (GN / 2) * BK * 2;  // this CTA's 128 of the tile's columns x 64 k
 constexpr int G_STG = 32 * 32 * 4;            // a warp's 32 x 32 fp32 staging block
-constexpr int G_BUFS = 2;                     // staging blocks per warp
+constexpr int G_BUFS = 1;                     // staging blocks per warp (a seventh operand
+                                              // stage would not fit; six stages and one
+                                              // block measured faster than five and two)
 constexpr int G_MN_LBO = BK * 128;            // MN-major tiles: next 64 M/N elements
 constexpr size_t G_SMEM =
     (size_t)G_STAGES * (G_A_BYTES + G_B_BYTES) + (size_t)G_EPI * G_BUFS * G_STG + 256;
@@ -63,73 +66,42 @@ struct GemmArgs {
   int k_iters;           // K in steps of 64
   int b_split;           // B map row (K-major: n; MN-major: k) where the second map takes over
   int c_split;           // output row where the second output block takes over
-  int stream_k;          // 0: whole tiles p, p + P, ...; 1: equal shares of tiles x k_iters
+  int splits;            // parts S of each tile's k steps (1: whole tiles)
   float* c0;             // output blocks (row-major, ldc floats per row) for the plain stores
   float* c1;
   int64_t ldc;
   int64_t c_rows;        // output rows over both blocks
   int c_cols;            // output columns (a multiple of 32)
-  int* flags;            // stream-K: a counter per tile, zero at launch
+  int* flags;            // S > 1: a counter per tile, zero at launch
   unsigned int* status;
 };
 
-// One stretch of a pair's work: k steps [kb, ke) of a tile.
+// One unit of a pair's work: part `split` of a tile, k steps [kb, ke).
 struct GUnit {
-  int tile, kb, ke;
+  int tile, split, kb, ke;
 };
 
-// The pair's stretches in order, the same walk in every role.  Stream-K:
-// pair q's share starts at iteration q W / P of W = tiles x k_iters.
+// The pair's units in order, the same walk in every role.
 struct GWalk {
-  int64_t cur, end;
-  int step, KT, tiles;
-  bool sk;
+  int cur, end, step, tiles, KT, S;
   __device__ GWalk(const GemmArgs& a, int pair, int npairs) {
-    KT = a.k_iters;
     tiles = a.m_tiles * a.n_tiles;
-    sk = a.stream_k != 0;
+    KT = a.k_iters;
+    S = a.splits;
+    cur = pair;
+    end = tiles * S;
     step = npairs;
-    if (sk) {
-      const int64_t W = (int64_t)tiles * KT;
-      cur = W * pair / npairs;
-      end = W * (pair + 1) / npairs;
-    } else {
-      cur = pair;
-      end = tiles;
-    }
   }
   __device__ bool next(GUnit& u) {
     if (cur >= end) return false;
-    if (sk) {
-      const int t = (int)(cur / KT);
-      const int64_t t0 = (int64_t)t * KT;
-      const int64_t te = t0 + KT < end ? t0 + KT : end;
-      u.tile = t;
-      u.kb = (int)(cur - t0);
-      u.ke = (int)(te - t0);
-      cur = te;
-    } else {
-      u.tile = (int)cur;
-      u.kb = 0;
-      u.ke = KT;
-      cur += step;
-    }
+    u.split = cur / tiles;
+    u.tile = cur - u.split * tiles;
+    u.kb = (int)((int64_t)u.split * KT / S);
+    u.ke = (int)((int64_t)(u.split + 1) * KT / S);
+    cur += step;
     return true;
   }
 };
-
-// How many pairs above `pair` hold k steps of `tile` after this pair's
-// stretch, which ends at iteration g_end inside the tile (stream-K).
-__device__ int later_stretches(const GemmArgs& a, int pair, int npairs, int tile) {
-  const int64_t W = (int64_t)a.m_tiles * a.n_tiles * a.k_iters;
-  const int64_t tile_end = (int64_t)(tile + 1) * a.k_iters;
-  int n = 0;
-  for (int q = pair + 1; q < npairs; ++q) {
-    if (W * q / npairs >= tile_end) break;
-    ++n;
-  }
-  return n;
-}
 
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   int v;
@@ -321,7 +293,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
       if (!ok) break;
       const uint32_t t_row =
           tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * GN + part * (GN / 2));
-      if (u.kb == 0 && u.ke == a.k_iters) {
+      if (a.splits == 1) {
         // the whole tile: 32 x 32 blocks through the staging buffers, one
         // tiled store each (rows and columns outside C are not written)
         int rr = r0;
@@ -334,9 +306,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
         for (int c = 0; c < GN / 2 / 32; ++c) {
           float v[32];
           tmem_ld32(t_row + c * 32, v);
-          uint8_t* buf = my_stg + (nstore & 1u) * G_STG;
-          // the store issued two blocks ago has read this buffer
-          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          uint8_t* buf = my_stg + (nstore % G_BUFS) * G_STG;
+          // the store issued G_BUFS blocks ago has read this buffer
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(G_BUFS - 1) : "memory");
           __syncwarp();
 #pragma unroll
           for (int q = 0; q < 8; ++q)
@@ -348,13 +320,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
           ++nstore;
         }
       } else {
-        // a stretch of a split tile (stream-K): this lane's row, plain
-        // stores in the fixed order described at the top
-        const int later = u.ke == a.k_iters ? 0 : later_stretches(a, pair, npairs, u.tile);
+        // part s of a split tile: wait for part s - 1 of this tile, then for
+        // each 32 x 32 block, stage it (the same swizzled layout as above)
+        // and move it in 16-byte pieces, four 128-byte rows per instruction:
+        // loaded (the sum so far), added to, stored
         int good = 1;
-        if (later > 0) {
+        if (u.split > 0) {
           if (lane == 0) {
-            const int want = 2 * G_EPI * later;
+            const int want = 2 * G_EPI * u.split;
             const uint64_t t0 = global_ns();
             while (ld_acquire_gpu(a.flags + u.tile) < want) {
               if (*abort_flag) {
@@ -372,30 +345,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
           }
           good = __shfl_sync(FULL, good, 0);
         }
-        const int64_t row = (int64_t)r0 + lane;
-        float* crow = nullptr;
-        if (row < a.c_rows)
-          crow = row < a.c_split ? a.c0 + row * a.ldc : a.c1 + (row - a.c_split) * a.ldc;
+        uint8_t* buf = my_stg;
 #pragma unroll 1
         for (int c = 0; c < GN / 2 / 32; ++c) {
           float v[32];
           tmem_ld32(t_row + c * 32, v);
-          const int col = col0 + c * 32;
-          if (good && crow != nullptr && col < a.c_cols) {
-            float4* p = reinterpret_cast<float4*>(crow + col);
-            if (later > 0) {
+          __syncwarp();  // the previous block's reads of buf are done
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 o = __ldcg(p + q);  // the sum of the stretches after this one
-                v[4 * q] = o.x + v[4 * q];
-                v[4 * q + 1] = o.y + v[4 * q + 1];
-                v[4 * q + 2] = o.z + v[4 * q + 2];
-                v[4 * q + 3] = o.w + v[4 * q + 3];
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(buf + lane * 128 + ((q ^ (lane & 7)) * 16)) =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          __syncwarp();
+          // lane: 4 columns (16-byte chunk cg) of rows rg, rg + 4, ..., rg + 28
+          const int cg = lane & 7, rg = lane >> 3;
+          const int col = col0 + c * 32 + cg * 4;
+          if (good && col < a.c_cols) {
+            float4* gp[8];
+            float4 x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = 4 * i + rg;
+              const int64_t row = (int64_t)r0 + r;
+              gp[i] = row < a.c_rows
+                          ? reinterpret_cast<float4*>(
+                                (row < a.c_split ? a.c0 + row * a.ldc
+                                                 : a.c1 + (row - a.c_split) * a.ldc) + col)
+                          : nullptr;
+              x[i] = *reinterpret_cast<const float4*>(buf + r * 128 + ((cg ^ (r & 7)) << 4));
+            }
+            if (u.split > 0) {
+              // the sum of parts 0 .. s-1: all eight loads in flight, then the adds
+              float4 o[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                o[i] = gp[i] != nullptr ? __ldcg(gp[i]) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                x[i].x = o[i].x + x[i].x;
+                x[i].y = o[i].y + x[i].y;
+                x[i].z = o[i].z + x[i].z;
+                x[i].w = o[i].w + x[i].w;
               }
             }
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              __stcg(p + q, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+            for (int i = 0; i < 8; ++i)
+              if (gp[i] != nullptr) __stcg(gp[i], x[i]);
           }
         }
         // publish: all lanes' stores, then one count for this warp
@@ -438,7 +432,7 @@ int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& t
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G_SMEM) !=
         cudaSuccess)
       return ENGRAM_ERR_CUDA;
-    // pairs that fit on the GPU at once: stream-K waits between pairs, so
+    // pairs that fit on the GPU at once: split tiles wait between pairs, so
     // all of them must be resident
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -461,17 +455,29 @@ int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& t
     configured[dev] = true;
   }
   const int tiles = a.m_tiles * a.n_tiles;
-  int pairs;
-  if (a.stream_k) {
-    // at least 8 k steps per pair, so that a tile is not cut into slivers
-    const int64_t W = (int64_t)tiles * a.k_iters;
-    const int64_t want = W / 8 > 0 ? W / 8 : 1;
-    pairs = (int)(want < max_pairs[dev] ? want : max_pairs[dev]);
-    if (cudaMemsetAsync(a.flags, 0, (size_t)tiles * sizeof(int), s) != cudaSuccess)
-      return ENGRAM_ERR_CUDA;
-  } else {
-    pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+  const int P = max_pairs[dev];
+  if (a.splits == 0) {
+    // parts per tile: the fewest rounds of units per part of the work
+    // (rounds / S), each part charged 2% for the extra partial sums it
+    // moves through L2 (measured at the 27B shape: S = 5 and 8 equal, 4 and
+    // 6 slower, 11 slower still), with at least 8 k steps in a part
+    int best = 1;
+    double best_cost = (double)((tiles + P - 1) / P) * 1.02;
+    const int s_max = a.k_iters / 8 < 32 ? a.k_iters / 8 : 32;
+    for (int S = 2; S <= s_max; ++S) {
+      const double cost = (double)(((int64_t)S * tiles + P - 1) / P) / S * (1.0 + 0.02 * S);
+      if (cost < best_cost - 1e-9) {
+        best_cost = cost;
+        best = S;
+      }
+    }
+    a.splits = best;
   }
+  if (a.splits > 1 &&
+      cudaMemsetAsync(a.flags, 0, (size_t)tiles * sizeof(int), s) != cudaSuccess)
+    return ENGRAM_ERR_CUDA;
+  const int64_t units = (int64_t)tiles * a.splits;
+  const int pairs = (int)(units < P ? units : P);
   if (pairs <= 0) return ENGRAM_OK;
   kern<<<dim3(2 * pairs), dim3(G_THREADS), G_SMEM, s>>>(ta, tb0, tb1, tc0, tc1, a);
   return ck(cudaGetLastError());
@@ -484,6 +490,7 @@ GemmArgs gemm_args(int64_t M, int64_t Nc, int64_t K) {
   a.k_iters = (int)((K + BK - 1) / BK);
   a.b_split = 0x7fffffff;
   a.c_split = 0x7fffffff;
+  a.splits = 1;
   a.status = status_ptr();
   return a;
 }
@@ -540,7 +547,7 @@ int launch_gemm_dw(const __nv_bfloat16* dkv, const __nv_bfloat16* e, int64_t N, 
     return ENGRAM_ERR_CUDA;
   GemmArgs a = gemm_args(2 * d, E, N);
   a.c_split = d;  // rows d.. are dW_v
-  a.stream_k = 1;
+  a.splits = 0;   // chosen at launch
   a.c0 = dWk;
   a.c1 = dWv;
   a.ldc = E;

@@ -43,7 +43,7 @@ EXPORTED = (
     "engram_hash_indices", "engram_gather", "engram_forward", "engram_backward",
     "engram_table_grad", "engram_table_grad_noalloc", "engram_forward_hosttable",
     "engram_get_status",
-    "engram_device_sm_count", "engram_clock_probe", "engram_table_rows", "engram_param_floats",
+    "engram_device_sm_count", "engram_table_rows", "engram_param_floats",
     "engram_hostcache_rank", "engram_hostcache_fill", "engram_forward_hostcache",
 )
 
@@ -113,7 +113,6 @@ def lib() -> ctypes.CDLL:
         "engram_forward_hosttable": (ctypes.c_int, [cfgp, P, P, i64, P, P, P]),
         "engram_get_status": (ctypes.c_int, [P]),
         "engram_device_sm_count": (ctypes.c_int, []),
-        "engram_clock_probe": (ctypes.c_int, [P, i64, P]),
         "engram_table_rows": (ctypes.c_int64, [cfgp]),
         "engram_param_floats": (ctypes.c_int64, [cfgp]),
         "engram_hostcache_rank": (ctypes.c_int, [cfgp, P, i64, i64, P, P, P, sz, P]),
@@ -273,9 +272,3 @@ def engram_get_status(stream=None) -> int:
 
 def engram_device_sm_count() -> int:
     return _check("engram_device_sm_count", lib().engram_device_sm_count())
-
-
-def engram_clock_probe(out, spin_ns: int, stream=None) -> None:
-    """out: device uint64/int64 tensor of 2; afterwards out[0] / out[1] is the
-    mean SM clock in GHz over `spin_ns` of the global timer."""
-    _check("engram_clock_probe", lib().engram_clock_probe(_p(out), spin_ns, _s(stream)))

@@ -380,21 +380,6 @@ int engram_get_status(void* stream);
 /* Multiprocessor count of the current device, or a negative ENGRAM_ERR_*. */
 int engram_device_sm_count(void);
 
-/* Measurement aid (no counterpart on the pages): the SM clock as the device
- * itself sees it.  One warp on one SM sleeps in 2 us steps until `spin_ns`
- * nanoseconds of the global timer have passed and writes
- *   out[0] = SM cycles elapsed (clock64), out[1] = global-timer ns elapsed,
- * so out[0] / out[1] is the mean SM clock in GHz over the window.  Launched
- * on a side stream next to other work it reports the clock that work ran at
- * (board power management lowers it under sustained tensor load while the
- * driver's clock query still reads the maximum).  It holds a block slot on
- * one SM for the whole window, so a persistent grid sized to every SM can be
- * delayed by it: take the reading beside an untimed repeat of the work.
- *   out      device uint64 [2], 8-byte aligned.
- *   spin_ns  1 .. 10,000,000,000 (10 s), else ENGRAM_ERR_INVALID_ARG.
- * Asynchronous on `stream`. */
-int engram_clock_probe(uint64_t* out, int64_t spin_ns, void* stream);
-
 #ifdef __cplusplus
 }
 #endif

@@ -108,11 +108,3 @@ def test_invalid_configurations_rejected_before_any_launch():
 def test_error_names():
     e = eg.EngramError("engram_forward", -4)
     assert "UNSUPPORTED" in str(e)
-
-
-def test_clock_probe_argument_checks_without_a_launch():
-    L = eg.lib()
-    assert L.engram_clock_probe(None, 1000, None) == -1          # no output buffer
-    assert L.engram_clock_probe(4096, 0, None) == -1             # empty window
-    assert L.engram_clock_probe(4096, 10_000_000_001, None) == -1  # beyond 10 s
-    assert L.engram_clock_probe(4100, 1000, None) == -2          # not 8-byte aligned

@@ -260,14 +260,3 @@ def test_gather_from_host_table_rejects_unmapped_memory():
     with pytest.raises(eg.EngramError) as ex:
         eg.engram_forward_hosttable(cfg, idx, plain.ctypes.data, 4, e, None, None)
     assert ex.value.rc == -1
-
-
-def test_clock_probe_reports_a_plausible_sm_clock():
-    """The measurement aid: SM cycles over global-timer nanoseconds of a 2 ms
-    window on an otherwise idle GPU lie between 0.3 and 2.5 GHz, and the
-    window is at least as long as asked."""
-    out = torch.zeros(2, dtype=torch.int64, device="cuda")
-    eg.engram_clock_probe(out, 2_000_000)
-    c, ns = out.cpu().tolist()
-    assert ns >= 2_000_000
-    assert 0.3 < c / ns < 2.5, c / ns
