@@ -250,9 +250,50 @@ def cpu_model() -> str:
     return "unknown"
 
 
+class single_thread:
+    """The oracle runs single-threaded: numpy's BLAS pool is held to one
+    thread for the duration (threadpoolctl)."""
+
+    def __enter__(self):
+        try:
+            from threadpoolctl import threadpool_limits
+            self._lim = threadpool_limits(limits=1)
+        except Exception:  # noqa: BLE001 -- numpy without a BLAS pool runs on one thread
+            self._lim = None
+        return self
+
+    def __exit__(self, *a):
+        if self._lim is not None:
+            self._lim.unregister()
+
+
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def time_oracle(fn, min_s: float = 1.0):
+    """Seconds per call of `fn` on one thread: one untimed call, then calls
+    until min_s has passed."""
+    with single_thread():
+        fn()
+        n, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= min_s:
+                break
+        return el / n, oracle_threads()
+
+
 def oracle_sample(w, ids, keys, mult, head_rows_fn, dense_host, n_seq: int, n_tok: int):
     """The oracle end to end (hash, gather, fusion) on the first
-    `n_tok` tokens of each of the first `n_seq` sequences of the batch.
+    `n_tok` tokens of each of the first `n_seq` sequences of the batch, on
+    one thread.
 
     `head_rows_fn(j, slots)` supplies rows `slots` of head j's table as
     [len(slots), D_h] float64; the oracle then gathers from a compact table
@@ -260,27 +301,41 @@ def oracle_sample(w, ids, keys, mult, head_rows_fn, dense_host, n_seq: int, n_to
     movement, not the method, and stays outside the timed spans.
     Returns (tokens, seconds, threads)."""
     from oracle import engram_oracle as O
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:  # noqa: BLE001
-        threads = 1
     proj, V_c = O.build_vocab_proj(keys)     # one-time set-up, untimed on both sides
-    t0 = time.perf_counter()
-    sub = np.ascontiguousarray(ids[:n_seq, :n_tok])
-    idx = O.hash_indices(proj, sub, mult, np.array(w.rows), w.K, V_c).reshape(-1, w.J)
-    sec = time.perf_counter() - t0
-    tables, local = [], np.empty_like(idx)
-    for j in range(w.J):
-        u, inv = np.unique(idx[:, j], return_inverse=True)
-        tables.append(head_rows_fn(j, u))
-        local[:, j] = inv.reshape(-1)
-    h = dense_host["h"][: n_seq * n_tok]
-    t1 = time.perf_counter()
-    e = O.gather(local, tables)
-    O.layer_forward(e, h, dense_host["Wk"], dense_host["Wv"], dense_host["conv_w"], n_tok)
-    sec += time.perf_counter() - t1
+    with single_thread():
+        threads = oracle_threads()
+        t0 = time.perf_counter()
+        sub = np.ascontiguousarray(ids[:n_seq, :n_tok])
+        idx = O.hash_indices(proj, sub, mult, np.array(w.rows), w.K, V_c).reshape(-1, w.J)
+        sec = time.perf_counter() - t0
+        tables, local = [], np.empty_like(idx)
+        for j in range(w.J):
+            u, inv = np.unique(idx[:, j], return_inverse=True)
+            tables.append(head_rows_fn(j, u))
+            local[:, j] = inv.reshape(-1)
+        h = dense_host["h"][: n_seq * n_tok]
+        t1 = time.perf_counter()
+        e = O.gather(local, tables)
+        O.layer_forward(e, h, dense_host["Wk"], dense_host["Wv"], dense_host["conv_w"], n_tok)
+        sec += time.perf_counter() - t1
     return n_seq * n_tok, sec, threads
+
+
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured graph (kept with keep_graph=True), or None."""
+    try:
+        from cuda.bindings import runtime as rt
+        graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(graph, numNodes=0)
+        err, nodes, n = rt.cudaGraphGetNodes(graph, numNodes=n)
+        k = 0
+        for nd in nodes:
+            err, t = rt.cudaGraphNodeGetType(nd)
+            if t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                k += 1
+        return k
+    except Exception:  # noqa: BLE001 -- reported as unknown
+        return None
 
 
 # ---------------------------------------------------------------- our path
@@ -493,12 +548,11 @@ def run_ours(args):
 
 
 def cpu_baseline_ours(w, ids_np, keys_np, mult, table, dense):
-    """The oracle on a bounded sample of the same workload (the whole batch,
-    about 6 s of CPU work on this machine's cores)."""
+    """The oracle on a bounded sample of the same workload: the first
+    sequence of the batch (4,096 tokens), end to end, on one thread."""
     import torch
-    from oracle import engram_oracle as O
     base = np.concatenate([[0], np.cumsum(w.rows)[:-1]])
-    n_seq = w.B
+    n_seq = 1
     dense_host = {
         "h": dense["h"][:n_seq].reshape(-1, 1, w.d).double().cpu().numpy(),
         "Wk": dense["Wk"].double().cpu().numpy(),
@@ -513,8 +567,8 @@ def cpu_baseline_ours(w, ids_np, keys_np, mult, table, dense):
     tok, sec, thr = oracle_sample(w, ids_np, keys_np, mult, rows_fn, dense_host, n_seq, w.T)
     return {"value": tok / sec, "unit": "tokens/s", "cores": thr, "kind": "oracle",
             "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
-            "sample": f"first {n_seq} sequences of the batch ({tok} tokens), oracle end to "
-                      f"end in fp64 ({sec:.1f} s)"}
+            "sample": f"first sequence of the batch ({tok} tokens), oracle end to end in fp64 "
+                      f"on one thread ({sec:.1f} s)"}
 
 
 # ---------------------------------------------------------------- other workloads
@@ -533,27 +587,65 @@ def _time_loop(fn, steps, warmup, stream):
     return a.elapsed_time(b) / steps
 
 
-def _graph_time(fn, steps, warmup, stream):
-    """The same step captured once into a CUDA graph and replayed."""
+def _graph_time(fn, steps, warmup, stream, nodes=None):
+    """The same step captured once into a CUDA graph and replayed; with a
+    list `nodes`, the graph's kernel-node count is appended to it."""
     import torch
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
+    g = torch.cuda.CUDAGraph(keep_graph=True)
     with torch.cuda.graph(g, stream=stream):
         fn()
+    if nodes is not None:
+        nodes.append(graph_kernel_nodes(g))
+    g.instantiate()
     return _time_loop(g.replay, steps, warmup, stream)
+
+
+_FLOOR = {}
+
+
+def launch_floor_us(dev, stream):
+    """Device time per kernel node of a graph of 200 one-element kernels:
+    the floor a chain of dependent launches cannot go below."""
+    import torch
+    if "us" not in _FLOOR:
+        x = torch.zeros(1, device=dev)
+
+        def chain():
+            for _ in range(200):
+                x.add_(1.0)
+
+        with torch.cuda.stream(stream):
+            _FLOOR["us"] = _graph_time(chain, 20, 2, stream) * 1e3 / 200
+    return _FLOOR["us"]
+
+
+def latency_roofline(dev, stream, us_per_call, kernels):
+    """Launch-latency roofline of a small step: its kernel count times the
+    per-kernel floor of a graph, against the measured time."""
+    floor = launch_floor_us(dev, stream)
+    if not kernels:
+        return {"bound": "latency", "achieved": us_per_call, "peak": None, "unit": "us",
+                "frac": None, "kernels_per_step": kernels, "floor_us_per_kernel": floor}
+    peak = kernels * floor
+    return {"bound": "latency", "achieved": us_per_call, "peak": peak, "unit": "us",
+            "frac": peak / us_per_call, "traffic": None, "kernels_per_step": kernels,
+            "floor_us_per_kernel": floor,
+            "how": "peak = kernels in the step's CUDA graph x device time per node of a graph of "
+                   "200 one-element kernels; frac = peak / measured (1.0 = launch-bound floor)"}
 
 
 def bench_fwd_bwd_27b(dev, steps=10):
     """Training step of the 27B-shaped layer (8 x 4,096 tokens, d 2,560, 16 x
     80 dims, 5.7B-parameter bf16 table): hash, forward (gather, fused passes,
-    alpha, k and v saved), backward (bf16: elementwise kernels, tensor-core GEMMs,
-    sparse table gradient); the same with k and v recomputed in the
+    alpha, k and v saved), backward (bf16: elementwise kernels, tensor-core
+    GEMMs, sparse table gradient); the same with k and v recomputed in the
     backward instead of saved; with the dilated conv (taps 3, 6 and 9
     tokens back); and with the pre-conv RMSNorm."""
-    keys = ("ms_per_step", "fwd_bwd_tokens_per_s", "breakdown_ms")
-    kept = _fwd_bwd_27b_run(dev, steps, save_kv=True)
+    keys = ("ms_per_step", "fwd_bwd_tokens_per_s", "breakdown_ms", "roofline")
+    kept = _fwd_bwd_27b_run(dev, steps, save_kv=True, cpu=True)
     recomputed = _fwd_bwd_27b_run(dev, steps, save_kv=False)
     kept["recompute_kv"] = {k: recomputed[k] for k in keys}
     from hashed_gram_conditional_engram_b200 import engram as eg
@@ -564,7 +656,42 @@ def bench_fwd_bwd_27b(dev, steps=10):
     return kept
 
 
-def _fwd_bwd_27b_run(dev, steps, save_kv, variant=0):
+def cpu_baseline_fwd_bwd_27b(w, ids_np, keys_np, mult, table, dense, dout, n_tok=512):
+    """The oracle's training step on the first n_tok tokens of the first
+    sequence: hash, gather, forward, backward and the table gradient, fp64,
+    one thread (the rows the sample touches are fetched outside the timing)."""
+    import torch
+    from oracle import engram_oracle as O
+    proj, V_c = O.build_vocab_proj(keys_np)
+    base = np.concatenate([[0], np.cumsum(w.rows)[:-1]])
+    ids = np.ascontiguousarray(ids_np[:1, :n_tok])
+    idx = O.hash_indices(proj, ids, mult, np.array(w.rows), w.K, V_c).reshape(-1, w.J)
+    tables, local = [], np.empty_like(idx)
+    for j in range(w.J):
+        u, inv = np.unique(idx[:, j], return_inverse=True)
+        r = torch.from_numpy(base[j] + u.astype(np.int64)).to(table.device)
+        tables.append(table.view(-1, w.D_h).index_select(0, r).double().cpu().numpy())
+        local[:, j] = inv.reshape(-1)
+    h = dense["h"][:1, :n_tok].reshape(n_tok, 1, w.d).double().cpu().numpy()
+    Wk, Wv = dense["Wk"].double().cpu().numpy(), dense["Wv"].double().cpu().numpy()
+    cw = dense["conv_w"].double().cpu().numpy()
+    u = dout[:n_tok].double().cpu().numpy()
+
+    def run():
+        O.hash_indices(proj, ids, mult, np.array(w.rows), w.K, V_c)
+        e = O.gather(local, tables)
+        g = O.layer_backward(e, h, Wk, Wv, cw, n_tok, u)
+        O.table_grad_segments_fast(local, g["de"].astype(np.float32),
+                                   [t.shape[0] for t in tables], w.D_h)
+
+    sec, thr = time_oracle(run, min_s=3.0)
+    return {"value": n_tok / sec, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+            "sample": f"first {n_tok} tokens of sequence 0: hash, gather, forward, backward, "
+                      f"table gradient in fp64 on one thread ({sec:.2f} s per call)"}
+
+
+def _fwd_bwd_27b_run(dev, steps, save_kv, variant=0, cpu=False):
     import torch
     from hashed_gram_conditional_engram_b200 import engram as eg
     from hashed_gram_conditional_engram_b200 import synth
@@ -622,17 +749,36 @@ def _fwd_bwd_27b_run(dev, steps, save_kv, variant=0):
         torch.cuda.synchronize()
     if eg.engram_get_status(s) != 0:
         raise RuntimeError("device status word set in the 27B-shaped training step")
-    # GEMMs: [k | v] recomputed unless saved; [dW_k; dW_v]; de with K = 2d
-    bwd_flops = 2.0 * N * E * (2 * w.d) * (2 if save_kv else 3)
+    # dense contractions of one step: forward k and v; backward [dW_k; dW_v]
+    # and de (K = 2d), and [k | v] again unless the forward kept them
+    flops = 2.0 * N * E * w.d * 2 + 2.0 * N * E * (2 * w.d) * (2 if save_kv else 3)
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    achieved = flops / (ms / 1e3) / 1e12
+    cpu_line = None
+    if cpu:
+        cpu_line = cpu_baseline_fwd_bwd_27b(w, ids_np, keys_np, mult, table, dense, dout)
     t_bwd = ev[1].elapsed_time(ev[2])
     del table, dense, bws, fws
     torch.cuda.empty_cache()
-    return {"workload": "layer27b training step: 8 x 4,096 tokens, d 2,560, 16 heads x 80 dims, "
-                        "5.7B bf16 params; forward (hash, gather, fused passes"
-                        + (", k and v saved" if save_kv else "") + ") + bf16 backward",
-            "fwd_bwd_tokens_per_s": N / (ms / 1e3), "ms_per_step": ms,
-            "breakdown_ms": {"forward": ev[0].elapsed_time(ev[1]), "backward": t_bwd},
-            "backward_gemm_tflops": bwd_flops / (t_bwd / 1e3) / 1e12}
+    out_line = {
+        "workload": "layer27b training step: 8 x 4,096 tokens, d 2,560, 16 heads x 80 dims, "
+                    "5.7B bf16 params; forward (hash, gather, fused passes"
+                    + (", k and v saved" if save_kv else "") + ") + bf16 backward",
+        "fwd_bwd_tokens_per_s": N / (ms / 1e3), "ms_per_step": ms,
+        "breakdown_ms": {"forward": ev[0].elapsed_time(ev[1]), "backward": t_bwd},
+        # the step's dense flops over the whole step's time (the elementwise
+        # kernels between the GEMMs included): a floor on the GEMMs' own rate,
+        # whose kernel times are in the committed launch list
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "what": "all dense GEMM flops of the step / whole step time",
+                     "flops_per_step": flops,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained"},
+    }
+    if cpu_line is not None:
+        out_line["cpu_baseline"] = cpu_line
+    return out_line
 
 
 def bench_tiny(dev, flags=0):
@@ -687,17 +833,42 @@ def bench_tiny(dev, flags=0):
         eg.engram_backward(cfg, idx, e, h, Wk, Wv, cw, saved, dout, dh, dWk, dWv, dcw, None,
                            keys_out, rows_out, nu, w.B, w.T, bws, bb, s)
 
+    nodes = []
     with torch.cuda.stream(s):
         f_eager = _time_loop(fwd, 200, 5, s)
         fb_eager = _time_loop(step, 200, 5, s)
-        fb_graph = _graph_time(step, 500, 5, s)
+        fb_graph = _graph_time(step, 500, 5, s, nodes)
     if eg.engram_get_status(s) != 0:
         raise RuntimeError("device status word set in the tiny layer")
+    from oracle import engram_oracle as O
+    proj_ref, V_c_ref = O.build_vocab_proj(inp["keys"])
+    tables64 = [np.asarray(x, np.float64) for x in inp["tables"]]
+
+    def oracle_step():
+        idx_r = O.hash_indices(proj_ref, inp["ids"], inp["mult"], inp["rows"], w.K, V_c_ref)
+        e_r = O.gather(idx_r.reshape(-1, w.J), tables64)
+        h_r = inp["h"].reshape(N, w.M, w.d)
+        if flags:
+            g_r = O.layer_backward_v(e_r, h_r, inp["Wk"], inp["Wv"], block, w.T,
+                                     inp["dout"].reshape(N, w.M, w.d), flags)
+        else:
+            g_r = O.layer_backward(e_r, h_r, inp["Wk"], inp["Wv"], inp["conv_w"], w.T,
+                                   inp["dout"].reshape(N, w.M, w.d))
+        O.table_grad_segments_fast(idx_r.reshape(-1, w.J), g_r["de"].astype(np.float32),
+                                   w.rows, w.D_h)
+
+    sec, thr = time_oracle(oracle_step)
     return {"workload": "tiny: 1 x 64 tokens, d 64, K 2 x 1,009 x 16, fp32 (fp64 arithmetic), "
                         "one layer" + (f", variant flags {flags}" if flags else ""),
             "us_per_fwd_call_eager": f_eager * 1e3, "us_per_fwd_bwd_call_eager": fb_eager * 1e3,
             "us_per_fwd_bwd_graph": fb_graph * 1e3,
-            "fwd_bwd_tokens_per_s": w.N / (fb_graph / 1e3)}
+            "fwd_bwd_tokens_per_s": w.N / (fb_graph / 1e3),
+            "roofline": latency_roofline(dev, s, fb_graph * 1e3, nodes[0] if nodes else None),
+            "cpu_baseline": {"value": w.N / sec, "unit": "tokens/s", "cores": thr,
+                             "kind": "oracle", "cpu_model": cpu_model(),
+                             "sample": "the whole workload (64 tokens): hash, gather, forward, "
+                                       f"backward, table gradient in fp64 ({sec * 1e3:.1f} ms "
+                                       "per call, one thread)"}}
 
 
 def bench_train_step(dev):
@@ -754,28 +925,65 @@ def bench_train_step(dev):
                                L["keys_out"], L["rows_out"], L["nu"], w.B, w.T, L["bws"], L["bb"], s)
             g = L["dh"]
 
+    nodes = []
     with torch.cuda.stream(s):
         eager = _time_loop(step, 50, 5, s)
-        graph = _graph_time(step, 200, 5, s)
+        graph = _graph_time(step, 200, 5, s, nodes)
     if eg.engram_get_status(s) != 0:
         raise RuntimeError("device status word set in the training step")
+    from oracle import engram_oracle as O
+    ref_layers = []
+    for li in (2, 6):
+        inp = synth.host_inputs(w, layer=li)
+        proj_ref, V_c_ref = O.build_vocab_proj(inp["keys"])
+        ref_layers.append((inp, proj_ref, V_c_ref, [np.asarray(x, np.float64) for x in inp["tables"]]))
+    h0_r = synth.host_inputs(w, layer=2)["h"].reshape(w.N, w.M, w.d).astype(np.float64)
+    dout_r = synth.host_inputs(w, layer=2)["dout"].reshape(w.N, w.M, w.d).astype(np.float64)
+
+    def oracle_step():
+        hin, saved_r = h0_r, []
+        for inp, proj_ref, V_c_ref, tabs in ref_layers:
+            idx_r = O.hash_indices(proj_ref, inp["ids"], inp["mult"], inp["rows"], w.K,
+                                   V_c_ref).reshape(-1, w.J)
+            e_r = O.gather(idx_r, tabs)
+            f = O.layer_forward(e_r, hin, inp["Wk"], inp["Wv"], inp["conv_w"], w.T)
+            saved_r.append((inp, idx_r, e_r, hin, f))
+            hin = f["out"]
+        g = dout_r
+        for inp, idx_r, e_r, hin, f in reversed(saved_r):
+            gr = O.layer_backward(e_r, hin, inp["Wk"], inp["Wv"], inp["conv_w"], w.T, g, fwd=f)
+            O.table_grad_segments_fast(idx_r, gr["de"].astype(np.float32), w.rows, w.D_h)
+            g = gr["dh"]
+
+    sec, thr = time_oracle(oracle_step)
     return {"workload": "train: 1 x 64 tokens, d 64, 4 branches, Engram at layers 2 and 6, "
                         "K 2 x 1,009 x 16 per layer, fp32 (fp64 arithmetic)",
             "fwd_bwd_tokens_per_s": w.N / (graph / 1e3), "ms_per_step_graph": graph,
-            "ms_per_step_eager": eager, "fwd_bwd_tokens_per_s_eager": w.N / (eager / 1e3)}
+            "ms_per_step_eager": eager, "fwd_bwd_tokens_per_s_eager": w.N / (eager / 1e3),
+            "roofline": latency_roofline(dev, s, graph * 1e3, nodes[0] if nodes else None),
+            "cpu_baseline": {"value": w.N / sec, "unit": "tokens/s", "cores": thr,
+                             "kind": "oracle", "cpu_model": cpu_model(),
+                             "sample": "the whole workload (64 tokens, both layers): forward "
+                                       "and backward with the table gradients in fp64 "
+                                       f"({sec * 1e3:.1f} ms per step, one thread)"}}
 
 
-def bench_decode(dev, steps=200):
-    """Decode: 256 sequences x 1 token per step, d 4,096, K 8 x ~6.35M rows x
-    128 (13B bf16 parameters, 26 GB on the device), rolling n-gram and conv
-    state; one step = hash with state, gather, fused passes in decode mode."""
+def bench_decode(dev):
+    """Decode: 256 sequences x 1 token per step over the workload's 2,000
+    steps of Zipf(1.1) ids, each step with its own pregenerated hidden state
+    N(0, 1); d 4,096, K 8 x ~6.35M rows x 128 (13B bf16 parameters, 26 GB on
+    the device), rolling n-gram and conv state.  One step = hash with the
+    n-gram state, gather, fused passes in decode mode.  All 2,000 steps are
+    captured into one CUDA graph (each step reading its own ids and h rows),
+    replayed once untimed and once timed from the same initial state."""
     import torch
     from hashed_gram_conditional_engram_b200 import engram as eg
     from hashed_gram_conditional_engram_b200 import synth
     w = synth.workload("decode")
+    S = w.steps
     s = torch.cuda.Stream(dev)
     s.wait_stream(torch.cuda.current_stream(dev))
-    ids_np, keys_np = synth.host_ids_keys(w)
+    ids_np, keys_np = synth.host_ids_keys(w)          # [2000, 256]
     mult = synth.hash_multipliers(synth.layer_seed(w, 0), w.J)
     table = synth.device_table(w, device=dev)
     g = torch.Generator(device=dev)
@@ -783,13 +991,16 @@ def bench_decode(dev, steps=200):
     Wk = (torch.randn((1, w.d, w.E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
     Wv = (torch.randn((w.d, w.E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
     cw = torch.randn((w.d, 4), generator=g, device=dev) * 0.5
-    hs = torch.randn((8, w.B, 1, 1, w.d), generator=g, device=dev).to(torch.bfloat16)
+    hs = torch.empty((S, w.B, 1, 1, w.d), dtype=torch.bfloat16, device=dev)
+    for a in range(0, S, 250):
+        hs[a:a + 250] = torch.randn((min(250, S - a), w.B, 1, 1, w.d), generator=g,
+                                    device=dev).to(torch.bfloat16)
     keys = torch.from_numpy(keys_np).to(dev)
     proj = torch.empty(w.V, dtype=torch.int32, device=dev)
     vb = eg.engram_workspace_size(None, eg.WS_VOCAB, w.V)
     V_c = eg.engram_build_vocab_proj(keys, w.V, proj, torch.empty(vb, dtype=torch.uint8, device=dev), vb)
     cfg = eg.make_cfg(w.K, w.D_h, w.d, 1, w.V, V_c, eg.BF16, w.rows, mult)
-    ids = torch.from_numpy(ids_np).to(dev)          # [steps, B]
+    ids = torch.from_numpy(ids_np).to(dev)
     state = torch.full((w.B, 2), V_c, dtype=torch.int32, device=dev)
     conv_state = torch.zeros((w.B, 1, 3, w.d), device=dev)
     idx = torch.empty((w.B, 1, w.J), dtype=torch.int32, device=dev)
@@ -797,41 +1008,120 @@ def bench_decode(dev, steps=200):
     out = torch.empty((w.B, 1, 1, w.d), dtype=torch.bfloat16, device=dev)
     fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, w.B)
     fws = torch.empty(fb, dtype=torch.uint8, device=dev)
-    # the step reads its token ids and hidden state from fixed buffers, as a
-    # serving loop that replays one captured graph per step would
-    ids_step = ids[0].clone()
-    h_step = hs[0].clone()
 
-    def hash_only():
-        eg.engram_hash_indices(cfg, proj, ids_step, w.B, 1, state, idx, s)
-
-    def forward_only():
-        eg.engram_forward(cfg, idx, table, e, h_step, Wk, Wv, cw, conv_state, out, None, w.B, 1,
+    def step(k):
+        eg.engram_hash_indices(cfg, proj, ids[k], w.B, 1, state, idx, s)
+        eg.engram_forward(cfg, idx, table, e, hs[k], Wk, Wv, cw, conv_state, out, None, w.B, 1,
                           fws, fb, s)
 
-    def step():
-        hash_only()
-        forward_only()
+    def reset():
+        state.fill_(V_c)
+        conv_state.zero_()
+
+    def all_steps():
+        for k in range(S):
+            step(k)
 
     with torch.cuda.stream(s):
-        for i in range(16):                      # a few real steps first
-            ids_step.copy_(ids[i])
-            h_step.copy_(hs[i % 8])
-            step()
-        ms = _time_loop(step, steps, 5, s)
-        ms_hash = _time_loop(hash_only, steps, 5, s)
-        ms_fwd = _time_loop(forward_only, steps, 5, s)
-        ms_graph = _graph_time(step, steps, 5, s)
+        for k in range(8):                       # set-up of the kernels on this device
+            step(k)
+        reset()
+        torch.cuda.synchronize()
+        # eager: one Python call pair per step (host-bound)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        all_steps()
+        b.record(s)
+        torch.cuda.synchronize()
+        ms_eager = a.elapsed_time(b) / S
+        reset()
+        graph = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(graph, stream=s):
+            all_steps()
+        kernels = graph_kernel_nodes(graph)
+        graph.instantiate()
+        graph.replay()                           # untimed
+        torch.cuda.synchronize()
+        reset()
+        torch.cuda.synchronize()
+        a.record(s)
+        graph.replay()
+        b.record(s)
+        torch.cuda.synchronize()
+        ms_graph = a.elapsed_time(b) / S
     if eg.engram_get_status(s) != 0:
         raise RuntimeError("device status word set in decode")
-    del table
+    # algorithmic bytes per step: both weight matrices, the rows and indices,
+    # ids and n-gram state, h and out, and the conv state read and rewritten
+    # (three steps of history per feature, kept oldest first)
+    wbytes = 2 * w.d * w.E * 2
+    rbytes = w.B * w.J * (w.D_h * 2 + 4)
+    sbytes = w.B * (4 + 2 * 4 * 2)
+    hbytes = 2 * w.B * w.d * 2
+    cbytes = 2 * w.B * 3 * w.d * 4
+    step_bytes = wbytes + rbytes + sbytes + hbytes + cbytes
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    achieved = step_bytes / (ms_graph / 1e3) / 1e9
+    cpu = cpu_baseline_decode(w, ids_np, keys_np, mult, table, Wk, Wv, cw, hs, V_c)
+    del table, hs, graph
     torch.cuda.empty_cache()
-    return {"workload": "decode: 256 sequences x 1 token per step, d_model 4,096, K 8 x "
-                        "6.35M rows x 128 (13.0B bf16 params), rolling n-gram and conv state",
+    return {"workload": "decode: 256 sequences x 1 token per step, 2,000 steps of Zipf(1.1) ids "
+                        "with fresh h per step, d_model 4,096, K 8 x 6.35M rows x 128 (13.0B bf16 "
+                        "params), rolling n-gram and conv state",
             "tokens_per_s": w.B / (ms_graph / 1e3), "us_per_step_graph": ms_graph * 1e3,
-            "us_per_step_eager": ms * 1e3, "tokens_per_s_eager": w.B / (ms / 1e3),
-            "eager_breakdown_us": {"hash": ms_hash * 1e3, "forward (gather + fused)": ms_fwd * 1e3},
-            "weight_bytes_per_step": 2 * w.d * w.E * 2, "steps": steps}
+            "us_per_step_eager": ms_eager * 1e3, "tokens_per_s_eager": w.B / (ms_eager / 1e3),
+            "steps_timed": S, "kernels_per_step": (kernels / S) if kernels else None,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "bytes_per_step": step_bytes,
+                         "bytes_split": {"W_k + W_v": wbytes, "rows + idx": rbytes,
+                                         "ids + ngram state": sbytes, "h + out": hbytes,
+                                         "conv state read + write": cbytes},
+                         "peak_source": f"{peak_src} hbm_gbs"},
+            "cpu_baseline": cpu}
+
+
+def cpu_baseline_decode(w, ids_np, keys_np, mult, table, Wk, Wv, cw, hs, V_c, n_steps=4):
+    """The oracle's decode steps 0 .. n_steps-1 for all 256 sequences (hash
+    with the rolling state, gather, gate, conv with the conv state), fp64 on
+    one thread; the touched rows and the step's h are fetched outside the
+    timing."""
+    import torch
+    from oracle import engram_oracle as O
+    proj, V_c_ref = O.build_vocab_proj(keys_np)
+    base = np.concatenate([[0], np.cumsum(w.rows)[:-1]])
+    Wk_h, Wv_h = Wk.double().cpu().numpy(), Wv.double().cpu().numpy()
+    cw_h = cw.double().cpu().numpy()
+    # the rows the sample's steps touch, by a dry run of the hash
+    st = np.full((w.B, 2), V_c_ref, np.int32)
+    rows_of = []
+    for k in range(n_steps):
+        idx_k, st = O.hash_indices_decode(proj, ids_np[k], st, mult, np.array(w.rows), w.K)
+        rows_of.append(idx_k)
+    tabs_of = []
+    for idx_k in rows_of:
+        tabs = []
+        for j in range(w.J):
+            r = torch.from_numpy(base[j] + idx_k[:, j].astype(np.int64)).to(table.device)
+            tabs.append(table.view(-1, w.D_h).index_select(0, r).double().cpu().numpy())
+        tabs_of.append(tabs)
+    h_of = [hs[k].reshape(w.B, 1, w.d).double().cpu().numpy() for k in range(n_steps)]
+    local = np.tile(np.arange(w.B, dtype=np.int64)[:, None], (1, w.J))
+
+    def run():
+        st_r = np.full((w.B, 2), V_c_ref, np.int32)
+        conv = np.zeros((w.B, 1, 3, w.d))
+        for k in range(n_steps):
+            _, st_r = O.hash_indices_decode(proj, ids_np[k], st_r, mult, np.array(w.rows), w.K)
+            e_r = O.gather(local, tabs_of[k])
+            _, _, conv = O.decode_step(e_r, h_of[k], Wk_h, Wv_h, cw_h, conv)
+
+    sec, thr = time_oracle(run, min_s=3.0)
+    return {"value": n_steps * w.B / sec, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+            "sample": f"decode steps 0-{n_steps - 1} of all 256 sequences, fp64 on one thread "
+                      f"({sec:.2f} s per run of {n_steps} steps)"}
 
 
 def bench_hosttable(dev, params=8_000_000_000):
@@ -917,6 +1207,15 @@ def bench_hosttable(dev, params=8_000_000_000):
         raise RuntimeError("device status word set in host-table gather")
     cached = _hosttable_cached(dev, w, cfg, proj, host, idx, e, side, comp, gemm, t_gemm,
                                rows_bytes)
+    # the oracle's gather of the same batch, reading the same pinned host
+    # table in place (rows as bf16 bit patterns: the gather is a copy)
+    from oracle import engram_oracle as O
+    host_bits = host.view(torch.int16).numpy()
+    starts = np.concatenate([[0], np.cumsum(rows)])
+    heads = [host_bits[starts[j] * w.D_h:starts[j + 1] * w.D_h].reshape(rows[j], w.D_h)
+             for j in range(w.J)]
+    sec, thr = time_oracle(lambda: O.gather(idx_np, heads), min_s=2.0)
+    pcie_gbs = rows_bytes / (t_gather / 1e3) / 1e9
     return {"workload": f"hosttable: 4 x 2,048 tokens, 16 heads x 160 dims, {sum(rows) * w.D_h / 1e9:.1f}B "
                         "bf16 params in pinned host memory (the 100B table does not fit the host)",
             "rows_bytes_per_batch": rows_bytes,
@@ -927,6 +1226,16 @@ def bench_hosttable(dev, params=8_000_000_000):
             "gemm_ms_alone": t_gemm, "gemm_ms_with_gather": t_both_gemm,
             "gather_ms_with_gemm": t_both_gather,
             "gemm_slowdown": t_both_gemm / t_gemm - 1.0,
+            "roofline": {"bound": "pcie", "achieved": pcie_gbs, "peak": h2d_peak, "unit": "GB/s",
+                         "frac": pcie_gbs / h2d_peak, "traffic": None,
+                         "bytes_per_batch": rows_bytes,
+                         "peak_source": "pinned host-to-device cudaMemcpy of 1 GiB on this box"},
+            "cpu_baseline": {"value": w.N / sec, "unit": "tokens/s", "cores": thr,
+                             "kind": "oracle", "cpu_model": cpu_model(),
+                             "rows_gbs": rows_bytes / sec / 1e9,
+                             "sample": "the whole batch (8,192 tokens x 16 rows of 160 bf16) "
+                                       "gathered by the oracle from the same pinned host table, "
+                                       f"one thread ({sec * 1e3:.1f} ms per batch)"},
             "hbm_cache": cached}
 
 
@@ -1071,7 +1380,7 @@ def run_reference(args):
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
                          "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
                          "sample": "first 1,024 tokens of one sequence per step, end to end "
-                                   "in fp64"},
+                                   "in fp64 on one thread"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

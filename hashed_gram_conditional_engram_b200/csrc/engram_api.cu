@@ -19,7 +19,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 int check_cfg(const engram_cfg_t* c) {
   if (c == nullptr) return ENGRAM_ERR_INVALID_ARG;
-  if (c->K < 1 || 2 * c->K > ENGRAM_MAX_HEADS || (2 * c->K) % 4 != 0) return ENGRAM_ERR_INVALID_ARG;
+  if (c->K < 1 || 2 * c->K > ENGRAM_MAX_HEADS) return ENGRAM_ERR_INVALID_ARG;
   if (c->D_h < 1 || c->d_model < 1 || c->n_branch < 1) return ENGRAM_ERR_INVALID_ARG;
   if (c->V_raw < 1 || c->V_c < 1 || c->V_c > c->V_raw) return ENGRAM_ERR_INVALID_ARG;
   if (c->dtype != ENGRAM_F32 && c->dtype != ENGRAM_BF16) return ENGRAM_ERR_INVALID_ARG;
@@ -150,6 +150,7 @@ size_t engram_saved_size(const engram_cfg_t* cfg, int64_t n_tok) {
 
 int engram_build_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_c_out,
                             void* ws, size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx("engram_build_vocab_proj");
   if (V < 1 || keys == nullptr || proj == nullptr || V_c_out == nullptr || ws == nullptr)
     return ENGRAM_ERR_INVALID_ARG;
   if (!aligned16(keys) || !aligned16(proj) || !aligned16(ws)) return ENGRAM_ERR_MISALIGNED;
@@ -159,6 +160,7 @@ int engram_build_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32
 
 int engram_hash_indices(const engram_cfg_t* cfg, const int32_t* proj, const int32_t* ids,
                         int32_t B, int32_t T, int32_t* ngram_state, int32_t* idx, void* stream) {
+  const NvtxRange nvtx("engram_hash_indices");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (B < 0 || T < 0 || proj == nullptr || idx == nullptr || (B * (int64_t)T > 0 && ids == nullptr))
@@ -174,6 +176,7 @@ int engram_hash_indices(const engram_cfg_t* cfg, const int32_t* proj, const int3
 
 int engram_gather(const engram_cfg_t* cfg, const int32_t* idx, const void* table, int64_t n_tok,
                   void* e, void* stream) {
+  const NvtxRange nvtx("engram_gather");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (n_tok < 0 || (n_tok > 0 && (idx == nullptr || table == nullptr || e == nullptr)))
@@ -188,6 +191,7 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
                    const void* h, const void* Wk, const void* Wv, const float* conv_w,
                    float* conv_state, void* out, float* saved, int32_t B, int32_t T, void* ws,
                    size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx("engram_forward");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (B < 0 || T < 0) return ENGRAM_ERR_INVALID_ARG;
@@ -245,6 +249,7 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                     const float* dout, float* dh, float* dWk, float* dWv, float* dconv_w, float* de,
                     int64_t* dtab_keys, float* dtab_rows, int32_t* n_unique, int32_t B, int32_t T,
                     void* ws, size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx("engram_backward");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (cfg->dtype == ENGRAM_BF16 && (cfg->n_branch != 1 || !bf16_variant_ok(cfg)))
@@ -305,13 +310,14 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
 int engram_table_grad(const engram_cfg_t* cfg, const int32_t* idx, const float* de, int64_t n_tok,
                       int64_t* dtab_keys, float* dtab_rows, int32_t* n_unique, void* ws,
                       size_t ws_bytes, void* stream) {
+  const NvtxRange nvtx("engram_table_grad");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (n_tok < 0 || n_unique == nullptr) return ENGRAM_ERR_INVALID_ARG;
   if (n_tok > 0 && (idx == nullptr || de == nullptr || dtab_keys == nullptr ||
                     dtab_rows == nullptr || ws == nullptr))
     return ENGRAM_ERR_INVALID_ARG;
-  if ((int64_t)n_tok * 2 * cfg->K >= 0x7fffffffLL) return ENGRAM_ERR_UNSUPPORTED;
+  if (n_tok >= 0x7fffffffLL / (2 * cfg->K)) return ENGRAM_ERR_UNSUPPORTED;
   if (!aligned16(idx) || !aligned16(de) || !aligned16(dtab_keys) || !aligned16(dtab_rows) ||
       !aligned16(ws))
     return ENGRAM_ERR_MISALIGNED;
@@ -323,6 +329,7 @@ int engram_table_grad(const engram_cfg_t* cfg, const int32_t* idx, const float* 
 int engram_table_grad_noalloc(const engram_cfg_t* cfg, const int32_t* idx, const float* de,
                               int64_t n_tok, int64_t* dtab_keys, float* dtab_rows,
                               int32_t* n_unique, void* stream) {
+  const NvtxRange nvtx("engram_table_grad_noalloc");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (n_tok < 0 || n_unique == nullptr) return ENGRAM_ERR_INVALID_ARG;
@@ -330,7 +337,8 @@ int engram_table_grad_noalloc(const engram_cfg_t* cfg, const int32_t* idx, const
     return ENGRAM_ERR_INVALID_ARG;
   if (!aligned16(idx) || !aligned16(de) || !aligned16(dtab_keys) || !aligned16(dtab_rows))
     return ENGRAM_ERR_MISALIGNED;
-  if (n_tok * 2 * cfg->K > ENGRAM_NOALLOC_MAX_ITEMS) return ENGRAM_ERR_TOO_LARGE;
+  // compared before multiplying, so that no n_tok can overflow the product
+  if (n_tok > ENGRAM_NOALLOC_MAX_ITEMS / (2 * cfg->K)) return ENGRAM_ERR_TOO_LARGE;
   if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
   return launch_table_grad_noalloc(make_head_params(cfg), idx, de, n_tok, dtab_keys, dtab_rows,
                                    n_unique, (cudaStream_t)stream);
@@ -338,6 +346,7 @@ int engram_table_grad_noalloc(const engram_cfg_t* cfg, const int32_t* idx, const
 
 int engram_forward_hosttable(const engram_cfg_t* cfg, const int32_t* idx, const void* host_table,
                              int64_t n_tok, void* e, void* side_stream, void* done_event) {
+  const NvtxRange nvtx("engram_forward_hosttable");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (n_tok < 0 || (n_tok > 0 && (idx == nullptr || host_table == nullptr || e == nullptr)))
@@ -378,12 +387,13 @@ int64_t engram_table_rows(const engram_cfg_t* cfg) {
 int engram_hostcache_rank(const engram_cfg_t* cfg, const int32_t* idx, int64_t n_tok, int64_t C,
                           int64_t* rows_out, int32_t* n_out, void* ws, size_t ws_bytes,
                           void* stream) {
+  const NvtxRange nvtx("engram_hostcache_rank");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (n_tok < 0 || C < 0 || n_out == nullptr || (C > 0 && rows_out == nullptr) ||
       (n_tok > 0 && (idx == nullptr || ws == nullptr)))
     return ENGRAM_ERR_INVALID_ARG;
-  if (n_tok * 2 * cfg->K >= 0x7fffffffLL || C >= 0x7fffffffLL) return ENGRAM_ERR_UNSUPPORTED;
+  if (n_tok >= 0x7fffffffLL / (2 * cfg->K) || C >= 0x7fffffffLL) return ENGRAM_ERR_UNSUPPORTED;
   if (!aligned16(idx) || !aligned16(rows_out) || !aligned16(ws)) return ENGRAM_ERR_MISALIGNED;
   if (ws_bytes < engram_workspace_size(cfg, ENGRAM_WS_HOSTCACHE_RANK, n_tok))
     return ENGRAM_ERR_WORKSPACE;
@@ -406,6 +416,7 @@ int mapped_host(const void* host, void** dev) {
 
 int engram_hostcache_fill(const engram_cfg_t* cfg, const void* host_table, const int64_t* rows,
                           int64_t C, void* cache, int32_t* map, void* stream) {
+  const NvtxRange nvtx("engram_hostcache_fill");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (C < 0 || host_table == nullptr || map == nullptr ||
@@ -425,12 +436,13 @@ int engram_forward_hostcache(const engram_cfg_t* cfg, const int32_t* idx, const 
                              const void* cache, const int32_t* map, int64_t n_tok, void* e,
                              int32_t* n_miss, void* ws, size_t ws_bytes, void* side_stream,
                              void* done_event) {
+  const NvtxRange nvtx("engram_forward_hostcache");
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (n_tok < 0 || host_table == nullptr || map == nullptr || ws == nullptr ||
       (n_tok > 0 && (idx == nullptr || e == nullptr)))
     return ENGRAM_ERR_INVALID_ARG;
-  if (n_tok * 2 * cfg->K >= 0x7fffffffLL) return ENGRAM_ERR_UNSUPPORTED;
+  if (n_tok >= 0x7fffffffLL / (2 * cfg->K)) return ENGRAM_ERR_UNSUPPORTED;
   if (!aligned16(idx) || !aligned16(host_table) || !aligned16(cache) || !aligned16(map) ||
       !aligned16(e) || !aligned16(ws))
     return ENGRAM_ERR_MISALIGNED;
@@ -448,6 +460,7 @@ int engram_forward_hostcache(const engram_cfg_t* cfg, const int32_t* idx, const 
 }
 
 int engram_get_status(void* stream) {
+  const NvtxRange nvtx("engram_get_status");
   unsigned int* p = status_ptr();
   if (p == nullptr) return ENGRAM_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;

@@ -5,9 +5,22 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/engram.h"
 
 namespace engram {
+
+// An NVTX range named after the entry point around each call of the C ABI,
+// so a timeline (Nsight Systems, Nsight Compute's NVTX filters) shows which
+// call issued which kernels.  The NVTX header does nothing unless a tool is
+// attached to the process.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Per-head constants handed to kernels by value.
 struct HeadParams {

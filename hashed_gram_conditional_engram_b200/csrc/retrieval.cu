@@ -45,10 +45,13 @@ __device__ __forceinline__ int32_t token_cid(const int32_t* __restrict__ proj,
   return __ldg(proj + x);
 }
 
-// TPT threads per token (J / 4 rounded up to a power of two), four heads
-// each; a warp covers 32 / TPT consecutive tokens in flat order.  c_{t-1} and c_{t-2}
-// travel from the lanes of the previous tokens by warp shuffles; the lanes of
-// a warp's first two tokens fetch the tokens before the warp themselves.
+// TPT threads per token (J / HPT rounded up to a power of two), HPT heads
+// each: four (one 16-byte store) when J is a multiple of 4, else two (an
+// 8-byte store; J = 2K is even); a warp covers 32 / TPT consecutive tokens
+// in flat order.  c_{t-1} and c_{t-2} travel from the lanes of the previous
+// tokens by warp shuffles; the lanes of a warp's first two tokens fetch the
+// tokens before the warp themselves.
+template <int HPT>
 __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HeadParams hp,
                                                    const int32_t* __restrict__ proj,
                                                    const int32_t* __restrict__ ids, int64_t N,
@@ -59,7 +62,7 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HeadP
   allow_dependents();  // a programmatically launched successor waits for this grid anyway
   const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
-  const int q = lane % tpt;             // which four heads
+  const int q = lane % tpt;             // which HPT heads
   const int64_t n = gt / tpt;           // token
   const int32_t pad = hp.V_c;
   const bool live = n < N;
@@ -92,11 +95,11 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HeadP
 
   const uint64_t g0 = (uint64_t)(uint32_t)c0, g1 = (uint64_t)(uint32_t)c1,
                  g2 = (uint64_t)(uint32_t)c2;
-  const int j0 = 4 * q;
-  if (j0 >= hp.J) return;  // padding lane of a token (J / 4 not a power of two)
-  int32_t s[4];
+  const int j0 = HPT * q;
+  if (j0 >= hp.J) return;  // padding lane of a token (J / HPT not a power of two)
+  int32_t s[HPT];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < HPT; ++u) {
     const int j = j0 + u;
     uint64_t x = g0 * hp.mult[j][0];
     x ^= g1 * hp.mult[j][1];
@@ -105,7 +108,10 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HeadP
     const bool bad = tri ? bad3 : bad2;
     s[u] = bad ? -1 : (int32_t)mod_prime(x, hp.P[j], hp.mu[j]);
   }
-  *reinterpret_cast<int4*>(idx + n * hp.J + j0) = make_int4(s[0], s[1], s[2], s[3]);
+  if constexpr (HPT == 4)
+    *reinterpret_cast<int4*>(idx + n * hp.J + j0) = make_int4(s[0], s[1], s[2], s[3]);
+  else
+    *reinterpret_cast<int2*>(idx + n * hp.J + j0) = make_int2(s[0], s[1]);
 }
 
 // Row gather with 16-byte vectors, generic shape.  The e row of a token is
@@ -216,14 +222,19 @@ int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, i
                 int32_t* ngram_state, int32_t* idx, cudaStream_t s) {
   const int64_t N = (int64_t)B * T;
   if (N == 0) return ENGRAM_OK;
-  // threads per token: J / 4 (four heads each) rounded up to a power of two
+  // threads per token: J / HPT (HPT heads each) rounded up to a power of two
+  const int hpt = hp.J % 4 == 0 ? 4 : 2;
   int tpt = 1;
-  while (tpt < hp.J / 4) tpt *= 2;
+  while (tpt < hp.J / hpt) tpt *= 2;
   const int threads = 256;
   const int64_t total = N * tpt;
   const int64_t blocks = (total + threads - 1) / threads;
-  hash_kernel<<<(unsigned)blocks, threads, 0, s>>>(hp, proj, ids, N, T, tpt, ngram_state, idx,
-                                                   status_ptr());
+  if (hpt == 4)
+    hash_kernel<4><<<(unsigned)blocks, threads, 0, s>>>(hp, proj, ids, N, T, tpt, ngram_state,
+                                                        idx, status_ptr());
+  else
+    hash_kernel<2><<<(unsigned)blocks, threads, 0, s>>>(hp, proj, ids, N, T, tpt, ngram_state,
+                                                        idx, status_ptr());
   return ck(cudaGetLastError());
 }
 

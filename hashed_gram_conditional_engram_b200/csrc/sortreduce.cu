@@ -818,7 +818,7 @@ int noalloc_scratch(void** out) {
 int launch_table_grad_noalloc(const HeadParams& hp, const int32_t* idx, const float* de,
                               int64_t n_tok, int64_t* keys, float* rows, int32_t* n_unique,
                               cudaStream_t s) {
-  if (n_tok * hp.J > ENGRAM_NOALLOC_MAX_ITEMS) return ENGRAM_ERR_TOO_LARGE;
+  if (n_tok < 0 || n_tok > ENGRAM_NOALLOC_MAX_ITEMS / hp.J) return ENGRAM_ERR_TOO_LARGE;
   void* scratch = nullptr;
   const int rc = noalloc_scratch(&scratch);
   if (rc) return rc;

@@ -285,6 +285,9 @@ int engram_table_grad(const engram_cfg_t* cfg, const int32_t* idx, const float* 
  *   before capturing a stream into a graph.
  *   All calls share the array: calls that overlap on the GPU (other streams,
  *   other host threads) race and must be serialised by the caller.
+ *   The looked-up address is kept for the life of the process: after a
+ *   cudaDeviceReset the array moves, so the library must not be used on
+ *   that device again (the same holds for the status word of every call).
  */
 #define ENGRAM_NOALLOC_MAX_ITEMS 131072
 int engram_table_grad_noalloc(const engram_cfg_t* cfg, const int32_t* idx, const float* de,

@@ -93,8 +93,7 @@ def test_invalid_configurations_rejected_before_any_launch():
         _cfg(D_h=6),                     # 24-byte rows: not a multiple of 16 bytes
         _cfg(rows=[1009, 1009, 1008, 1009]),  # even row count
         _cfg(rows=[1009, 1009, 1, 1009]),
-        _cfg(V_c=1001), _cfg(dtype=7), _cfg(flags=32), _cfg(K=3, rows=[1009] * 6,
-                                            mult=np.ones((6, 3), np.uint64)),  # J % 4 != 0
+        _cfg(V_c=1001), _cfg(dtype=7), _cfg(flags=32),
     ]
     big = _cfg()
     big.K = 17                             # J = 34 > 32 heads
