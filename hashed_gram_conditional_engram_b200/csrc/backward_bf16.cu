@@ -461,8 +461,10 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// Wait for the phase of `bar` with the given parity; false after ROW_WAIT_NS.
-__device__ __forceinline__ bool row_wait(uint64_t* bar, uint32_t parity) {
+constexpr uint64_t ROW_TEST_WAIT_NS = 1000000ull;  // 1 ms, with ENGRAM_TEST_STALL
+
+// Wait for the phase of `bar` with the given parity; false after limit_ns.
+__device__ __forceinline__ bool row_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   uint64_t t0 = 0;
   for (int spin = 0;; ++spin) {
     uint32_t ok;
@@ -477,7 +479,7 @@ __device__ __forceinline__ bool row_wait(uint64_t* bar, uint32_t parity) {
     uint64_t now;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
     if (spin == 0) t0 = now;
-    else if (now - t0 > ROW_WAIT_NS) return false;
+    else if (now - t0 > limit_ns) return false;
   }
 }
 
@@ -509,7 +511,7 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     const float* __restrict__ alpha, const float* __restrict__ dout,
     const float* __restrict__ dalpha_part, int np, int np_pad, const float* __restrict__ gscale,
     int64_t N, int d, int ld, float* __restrict__ dh, __nv_bfloat16* __restrict__ dk_out,
-    float* __restrict__ spart, unsigned int* status) {
+    float* __restrict__ spart, unsigned int* status, uint64_t wait_ns, int stall) {
   // k and dk rows are ld apart (they share rows with v and dv)
   extern __shared__ __align__(128) unsigned char row_smem[];
   __shared__ uint64_t full[ROW_STAGES];
@@ -526,6 +528,7 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(&full[st])),
                  "r"(hb_bytes + 2 * f_bytes + p_bytes)
                  : "memory");
+    if (stall) return;  // ENGRAM_TEST_STALL: the stage is armed, its copies never issued
     bulk_load(base, h + t * d, hb_bytes, &full[st]);
     bulk_load(base + hb_bytes, k + t * ld, f_bytes, &full[st]);
     bulk_load(base + hb_bytes + f_bytes, dout + t * d, f_bytes, &full[st]);
@@ -560,7 +563,7 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
   for (int64_t t = blockIdx.x; t < N; t += G, ++it) {
     const int st = it % ROW_STAGES;
     const unsigned char* base = row_smem + st * SB;
-    if (row_wait(&full[st], (uint32_t)(it / ROW_STAGES) & 1u)) {
+    if (row_wait(&full[st], (uint32_t)(it / ROW_STAGES) & 1u, wait_ns)) {
       pend &= ~(1u << st);
     } else {
       abort_flag = 1;  // every thread reaches the barrier below, then all stop
@@ -676,7 +679,7 @@ __global__ void __launch_bounds__(ROW_THREADS) bw_row_kernel(
     for (int st = 0; st < ROW_STAGES; ++st) {
       if (!(pend & (1u << st))) continue;
       const int use = done / ROW_STAGES + (st < done % ROW_STAGES ? 1 : 0);
-      row_wait(&full[st], (uint32_t)use & 1u);
+      row_wait(&full[st], (uint32_t)use & 1u, wait_ns);
     }
   }
 }
@@ -890,7 +893,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
                          float* dWk,
                          float* dWv, float* dconv_w, float* de, int64_t* dtab_keys,
                          float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, int dil,
-                         bool prenorm, const float* gv, void* ws, size_t ws_bytes,
+                         bool prenorm, const float* gv, void* ws, size_t ws_bytes, bool stall,
                          cudaStream_t s) {
   const int E = hp.E;
   const bool have_kv = kv_saved != nullptr;
@@ -906,7 +909,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   if (de == nullptr) de = w.de;
   int rc;
   // unless the forward saved them, [k | v] = e [W_k; W_v]^T (fp32)
-  if (!have_kv && (rc = launch_gemm_kv(e, Wk, Wv, N, d, E, w.kv, 2 * d, s))) return rc;
+  if (!have_kv && (rc = launch_gemm_kv(e, Wk, Wv, N, d, E, w.kv, 2 * d, s, stall))) return rc;
   const float* kv = have_kv ? kv_saved : w.kv;
   const int chunks = (int)((N + COL_TOK - 1) / COL_TOK);
   // one walk per (chunk, chain): the dilated conv's chunks hold three chains
@@ -966,7 +969,9 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
     if (scaled) grid = std::min<int64_t>(grid, kMaxRowBlocks);
     row<<<(unsigned)grid, ROW_THREADS, smem, s>>>(h, kv, alpha, dout, da_rows, da_np, da_np_pad,
                                                   gscale, N, d, 2 * d, dh, w.dkv, w.spart,
-                                                  status_ptr());
+                                                  status_ptr(),
+                                                  stall ? ROW_TEST_WAIT_NS : ROW_WAIT_NS,
+                                                  stall ? 1 : 0);
     if (scaled)
       bw_scale_reduce_kernel<<<(unsigned)((d + 255) / 256), 256, 0, s>>>(
           w.spart, (int)grid, d, gscale, dconv_w + 4 * (int64_t)d);
@@ -976,8 +981,8 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
   if ((rc = ck(cudaGetLastError()))) return rc;
   // [dW_k; dW_v] = [dk | dv]^T e (a contraction over tokens, rows d.. into
   // dW_v); de = [dk | dv] [W_k; W_v]
-  if ((rc = launch_gemm_dw(w.dkv, e, N, d, E, dWk, dWv, w.gemm_ws, s))) return rc;
-  if ((rc = launch_gemm_de(w.dkv, Wk, Wv, N, d, E, de, s))) return rc;
+  if ((rc = launch_gemm_dw(w.dkv, e, N, d, E, dWk, dWv, w.gemm_ws, s, stall))) return rc;
+  if ((rc = launch_gemm_de(w.dkv, Wk, Wv, N, d, E, de, s, stall))) return rc;
   // the table rows' gradient from de, in the deterministic order
   return launch_table_grad(hp, idx, de, N, dtab_keys, dtab_rows, n_unique, w.tg_ws, w.tg_bytes, s);
 }

@@ -23,7 +23,8 @@ int check_cfg(const engram_cfg_t* c) {
   if (c->D_h < 1 || c->d_model < 1 || c->n_branch < 1) return ENGRAM_ERR_INVALID_ARG;
   if (c->V_raw < 1 || c->V_c < 1 || c->V_c > c->V_raw) return ENGRAM_ERR_INVALID_ARG;
   if (c->dtype != ENGRAM_F32 && c->dtype != ENGRAM_BF16) return ENGRAM_ERR_INVALID_ARG;
-  if ((c->flags & ~(ENGRAM_SAVE_KV | ENGRAM_VARIANT_FLAGS)) != 0) return ENGRAM_ERR_INVALID_ARG;
+  if ((c->flags & ~(ENGRAM_SAVE_KV | ENGRAM_VARIANT_FLAGS | ENGRAM_TEST_STALL)) != 0)
+    return ENGRAM_ERR_INVALID_ARG;
   const int es = c->dtype == ENGRAM_F32 ? 4 : 2;
   if ((c->D_h * es) % 16 != 0) return ENGRAM_ERR_MISALIGNED;
   for (int j = 0; j < 2 * c->K; ++j) {
@@ -241,7 +242,8 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
                            static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
                            static_cast<__nv_bfloat16*>(out), saved, kv_save, gg,
                            (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1, N, T, d, E, ws, ws_bytes,
-                           table != nullptr, bf16_prenorm(cfg) ? &pn : nullptr, s);
+                           table != nullptr, bf16_prenorm(cfg) ? &pn : nullptr,
+                           (cfg->flags & ENGRAM_TEST_STALL) != 0, s);
 }
 
 int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,
@@ -292,7 +294,7 @@ int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, 
                                 N, T, d, (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1,
                                 bf16_prenorm(cfg),
                                 bf16_scaled(cfg) && bf16_prenorm(cfg) ? conv_w + 6 * d : nullptr,
-                                ws, ws_bytes, s);
+                                ws, ws_bytes, (cfg->flags & ENGRAM_TEST_STALL) != 0, s);
   }
   const size_t bw = backward_f32_ws_bytes(N, M, d, E);
   // de lives in the dense-backward workspace unless the caller wants it

@@ -76,6 +76,8 @@ struct TcArgs {
   float* kv_save;       // optional fp32 [N, 2d]: k (pass K) then v (pass V) of each token
   const float* gg;      // optional [d]: g_h * g_k, the learnable norm scales' product (pass K)
   unsigned int* status;
+  uint64_t wait_ns;     // limit of every bounded wait
+  int stall;            // ENGRAM_TEST_STALL: the B producer issues nothing
 };
 
 
@@ -329,7 +331,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
         operand_rows(tile, arow, brow);
         bool ok = true;
         for (int kt = 0; kt < args.num_k_tiles; ++kt) {
-          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -351,7 +353,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
       if (leader) {
         for (int s = 0; s < STAGES; ++s) {
           const uint32_t n_s = issued > (uint32_t)s ? (issued - 1 - s) / STAGES + 1 : 0;
-          if (n_s > 0) wait_drain(&full[s], (n_s - 1) & 1u);
+          if (n_s > 0) wait_drain(&full[s], (n_s - 1) & 1u, args.wait_ns);
         }
       }
     }
@@ -364,11 +366,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) break;
+        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status, args.wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         for (int kt = 0; kt < args.num_k_tiles; ++kt) {
-          if (!wait_bounded(&full[stage], phase, abort_flag, args.status)) {
+          if (!wait_bounded(&full[stage], phase, abort_flag, args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -397,14 +399,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
       }
       // all issued MMAs complete before TMEM is released
       umma_commit_pair_self(drain);
-      wait_drain(drain, 0);
+      wait_drain(drain, 0, args.wait_ns);
     }
   } else if (warp == S::BP_WARP) {
     // ------------------------------------------------------------ B-operand producer
     // Same stages and order as the A producer; its bytes count on the
     // leader's full barrier, whose expected total the A producer posts (a
-    // phase cannot complete before that arrival).
-    if (lane == 0) {
+    // phase cannot complete before that arrival).  With ENGRAM_TEST_STALL it
+    // issues nothing, so the stages never fill and the waits run out.
+    if (lane == 0 && !args.stall) {
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = pair; tile < num_tiles; tile += num_pairs) {
@@ -412,7 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
         operand_rows(tile, arow, brow);
         bool ok = true;
         for (int kt = 0; kt < args.num_k_tiles; ++kt) {
-          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -439,7 +442,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
         const int f0 = ni * (2 * BM) + (int)rank * BM;  // this CTA's features
         bool ok = true;
         for (int c = 0; c < NCH; ++c) {
-          if (!wait_bounded(&hempty[slot], ph ^ 1u, abort_flag, args.status)) {
+          if (!wait_bounded(&hempty[slot], ph ^ 1u, abort_flag, args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -459,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
       }
       for (int b = 0; b < S::HSLOTS; ++b) {
         const uint32_t n_b = issued > (uint32_t)b ? (issued - 1 - b) / (S::HSLOTS > 0 ? S::HSLOTS : 1) + 1 : 0;
-        if (n_b > 0) wait_drain(&hfull[b], (n_b - 1) & 1u);
+        if (n_b > 0) wait_drain(&hfull[b], (n_b - 1) & 1u, args.wait_ns);
       }
     }
   } else {
@@ -500,7 +503,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
       // loads that do not depend on it)
       auto wait_acc = [&]() {
         int ok = 0;
-        if (lane == 0) ok = wait_bounded(&tfull[acc], acc_phase, abort_flag, args.status) ? 1 : 0;
+        if (lane == 0) ok = wait_bounded(&tfull[acc], acc_phase, abort_flag, args.status, args.wait_ns) ? 1 : 0;
         ok = __shfl_sync(FULL, ok, 0);
         tc_fence_after();
         return ok;
@@ -666,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcShape<BN, STAGES, 
 #pragma unroll 1
         for (int c = 0; c < NCH; ++c) {
           int hgot = 0;
-          if (lane == 0) hgot = wait_bounded(&hfull[hslot], hphase, abort_flag, args.status) ? 1 : 0;
+          if (lane == 0) hgot = wait_bounded(&hfull[hslot], hphase, abort_flag, args.status, args.wait_ns) ? 1 : 0;
           hgot = __shfl_sync(FULL, hgot, 0);
           // h of token jj and feature f of this box: box[jj * BM + f]; the
           // output of the same element replaces it in place
@@ -944,7 +947,7 @@ template <int BN, int STAGES_K, int STAGES_V, int STAGES_VKV, int KCH>
 int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
               const __nv_bfloat16* Wv, const float* conv_w, float* conv_state, __nv_bfloat16* out,
               float* alpha_saved, float* kv_save, const float* gg, int dil, int64_t N, int T,
-              int d, int E, float4* part, float* alpha, bool chained, bool gate_only,
+              int d, int E, float4* part, float* alpha, bool chained, bool gate_only, bool stall,
               cudaStream_t s) {
   // Each CTA of a pair loads 128 rows of A and BN/2 rows of B per stage.
   // pass K: A = e (256 tokens per pair tile), B = W_k (BN features)
@@ -980,6 +983,8 @@ int run_layer(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat1
   a.kv_save = conv_state == nullptr ? kv_save : nullptr;
   a.gg = gg;
   a.status = status_ptr();
+  a.wait_ns = stall ? TEST_WAIT_LIMIT_NS : WAIT_LIMIT_NS;
+  a.stall = stall ? 1 : 0;
   // pass K: gate partials, pair tiles of 256 tokens x BN features
   a.num_n_tiles = d / BN;
   a.m_stride = 2 * BM;
@@ -1086,7 +1091,7 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
                       __nv_bfloat16* out, float* alpha_saved, float* kv_save, const float* gg,
                       int dil, int64_t N, int T, int d, int E, void* ws, size_t ws_bytes,
-                      bool chained, const PrenormFwd* pn, cudaStream_t s) {
+                      bool chained, const PrenormFwd* pn, bool stall, cudaStream_t s) {
   if (ws_bytes < tc_forward_ws_bytes(N, d, E) || ws == nullptr) return ENGRAM_ERR_WORKSPACE;
   if (N > 0x7fffffffLL - 256) return ENGRAM_ERR_UNSUPPORTED;
   const bool wide = use_wide(N, d);
@@ -1099,17 +1104,18 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
   int rc;
   if (wide)
     rc = run_layer<256, 6, 5, 4, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
-                                    gg, dil, N, T, d, E, part, alpha, chained, gate_only, s);
+                                    gg, dil, N, T, d, E, part, alpha, chained, gate_only, stall, s);
   // few tokens: each CTA streams long operand rows at a rate set by how many
   // bytes one copy instruction brings, so two K chunks go in each box
   else if (E % (2 * BK) == 0)
     rc = run_layer<64, 4, 3, 3, 2>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
-                                   gg, dil, N, T, d, E, part, alpha, chained, gate_only, s);
+                                   gg, dil, N, T, d, E, part, alpha, chained, gate_only, stall, s);
   else
     rc = run_layer<64, 8, 6, 6, 1>(e, h, Wk, Wv, conv_w, conv_state, out, alpha_saved, kv_save,
-                                   gg, dil, N, T, d, E, part, alpha, chained, gate_only, s);
+                                   gg, dil, N, T, d, E, part, alpha, chained, gate_only, stall, s);
   if (rc || pn == nullptr) return rc;
-  return launch_prenorm_tail(*pn, e, Wv, h, conv_w, alpha, conv_state, out, dil, N, T, d, E, s);
+  return launch_prenorm_tail(*pn, e, Wv, h, conv_w, alpha, conv_state, out, dil, N, T, d, E,
+                             stall, s);
 }
 
 }  // namespace engram

@@ -74,6 +74,8 @@ struct GemmArgs {
   int c_cols;            // output columns (a multiple of 32)
   int* flags;            // S > 1: a counter per tile, zero at launch
   unsigned int* status;
+  uint64_t wait_ns;      // limit of every bounded wait
+  int stall;             // ENGRAM_TEST_STALL: the B producer issues nothing
 };
 
 // One unit of a pair's work: part `split` of a tile, k steps [kb, ke).
@@ -175,8 +177,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
     // ------------------------------------------------------------ operand producers
     // Warp 0 loads A and posts the stage's expected bytes (both CTAs' A and
     // B boxes count on the leader's barrier); warp 10 loads B into the same
-    // stages in the same order.
-    if (lane == 0) {
+    // stages in the same order (with ENGRAM_TEST_STALL it issues nothing, so
+    // the stages never fill and the waits run out).
+    if (lane == 0 && !(warp == G_BP_WARP && a.stall)) {
       const bool isA = warp == 0;
       GWalk w(a, pair, npairs);
       GUnit u;
@@ -188,7 +191,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
         const int m0 = mi * (2 * BM) + (int)rank * BM;      // this CTA's rows of A
         const int n0 = ni * GN + (int)rank * (GN / 2);      // this CTA's columns of B
         for (int kt = u.kb; kt < u.ke; ++kt) {
-          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.status)) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.status, a.wait_ns)) {
             ok = false;
             break;
           }
@@ -223,7 +226,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
       if (isA && leader) {
         for (int s = 0; s < G_STAGES; ++s) {
           const uint32_t n_s = issued > (uint32_t)s ? (issued - 1 - s) / G_STAGES + 1 : 0;
-          if (n_s > 0) wait_drain(&full[s], (n_s - 1) & 1u);
+          if (n_s > 0) wait_drain(&full[s], (n_s - 1) & 1u, a.wait_ns);
         }
       }
     }
@@ -236,11 +239,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       while (ok && w.next(u)) {
-        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, a.status)) break;
+        if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, a.status, a.wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * GN);
         for (int kt = u.kb; kt < u.ke; ++kt) {
-          if (!wait_bounded(&full[stage], phase, abort_flag, a.status)) {
+          if (!wait_bounded(&full[stage], phase, abort_flag, a.status, a.wait_ns)) {
             ok = false;
             break;
           }
@@ -270,7 +273,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
       }
       // all issued MMAs complete before TMEM is released
       umma_commit_pair_self(drain);
-      wait_drain(drain, 0);
+      wait_drain(drain, 0, a.wait_ns);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -287,7 +290,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
       const int r0 = mi * (2 * BM) + (int)rank * BM + quad * 32;  // the warp's first row
       const int col0 = ni * GN + part * (GN / 2);
       int ok = 0;
-      if (lane == 0) ok = wait_bounded(&tfull[acc], acc_phase, abort_flag, a.status) ? 1 : 0;
+      if (lane == 0) ok = wait_bounded(&tfull[acc], acc_phase, abort_flag, a.status, a.wait_ns) ? 1 : 0;
       ok = __shfl_sync(FULL, ok, 0);
       tc_fence_after();
       if (!ok) break;
@@ -334,7 +337,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(G_THREADS, 1)
                 good = 0;
                 break;
               }
-              if (global_ns() - t0 > WAIT_LIMIT_NS) {
+              if (global_ns() - t0 > a.wait_ns) {
                 *abort_flag = 1;
                 atomicOr(a.status, ENGRAM_STATUS_TIMEOUT);
                 good = 0;
@@ -483,7 +486,7 @@ int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& t
   return ck(cudaGetLastError());
 }
 
-GemmArgs gemm_args(int64_t M, int64_t Nc, int64_t K) {
+GemmArgs gemm_args(int64_t M, int64_t Nc, int64_t K, bool stall) {
   GemmArgs a = {};
   a.m_tiles = (int)((M + 2 * BM - 1) / (2 * BM));
   a.n_tiles = (int)((Nc + GN - 1) / GN);
@@ -492,6 +495,8 @@ GemmArgs gemm_args(int64_t M, int64_t Nc, int64_t K) {
   a.c_split = 0x7fffffff;
   a.splits = 1;
   a.status = status_ptr();
+  a.wait_ns = stall ? TEST_WAIT_LIMIT_NS : WAIT_LIMIT_NS;
+  a.stall = stall ? 1 : 0;
   return a;
 }
 
@@ -502,7 +507,7 @@ int gemm_supported(int64_t N, int d, int E) {
 }
 
 int launch_gemm_kv(const __nv_bfloat16* e, const __nv_bfloat16* Wk, const __nv_bfloat16* Wv,
-                   int64_t N, int d, int E, float* C, int64_t ldc, cudaStream_t s) {
+                   int64_t N, int d, int E, float* C, int64_t ldc, cudaStream_t s, bool stall) {
   if (!gemm_supported(N, d, E) || ldc % 4 != 0) return ENGRAM_ERR_UNSUPPORTED;
   if (N == 0) return ENGRAM_OK;
   const bool both = Wk != nullptr;
@@ -514,7 +519,7 @@ int launch_gemm_kv(const __nv_bfloat16* e, const __nv_bfloat16* Wk, const __nv_b
       !make_tmap_f32_ld(&tc0, C, (uint64_t)cols, (uint64_t)N, (uint64_t)ldc, 32, 32,
                         CU_TENSOR_MAP_SWIZZLE_128B))
     return ENGRAM_ERR_CUDA;
-  GemmArgs a = gemm_args(N, cols, E);
+  GemmArgs a = gemm_args(N, cols, E, stall);
   if (both) a.b_split = d;  // columns d.. of C come from W_v
   a.c0 = C;
   a.ldc = ldc;
@@ -529,7 +534,7 @@ size_t gemm_dw_ws_bytes(int d, int E) {
 }
 
 int launch_gemm_dw(const __nv_bfloat16* dkv, const __nv_bfloat16* e, int64_t N, int d, int E,
-                   float* dWk, float* dWv, void* ws, cudaStream_t s) {
+                   float* dWk, float* dWv, void* ws, cudaStream_t s, bool stall) {
   if (!gemm_supported(N, d, E)) return ENGRAM_ERR_UNSUPPORTED;
   if (N == 0) {  // no tokens: the gradients are zero
     if (cudaMemsetAsync(dWk, 0, (size_t)d * E * 4, s) != cudaSuccess ||
@@ -545,7 +550,7 @@ int launch_gemm_dw(const __nv_bfloat16* dkv, const __nv_bfloat16* e, int64_t N, 
       !make_tmap_f32(&tc0, dWk, (uint64_t)E, (uint64_t)d, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_f32(&tc1, dWv, (uint64_t)E, (uint64_t)d, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return ENGRAM_ERR_CUDA;
-  GemmArgs a = gemm_args(2 * d, E, N);
+  GemmArgs a = gemm_args(2 * d, E, N, stall);
   a.c_split = d;  // rows d.. are dW_v
   a.splits = 0;   // chosen at launch
   a.c0 = dWk;
@@ -558,7 +563,7 @@ int launch_gemm_dw(const __nv_bfloat16* dkv, const __nv_bfloat16* e, int64_t N, 
 }
 
 int launch_gemm_de(const __nv_bfloat16* dkv, const __nv_bfloat16* Wk, const __nv_bfloat16* Wv,
-                   int64_t N, int d, int E, float* de, cudaStream_t s) {
+                   int64_t N, int d, int E, float* de, cudaStream_t s, bool stall) {
   if (!gemm_supported(N, d, E)) return ENGRAM_ERR_UNSUPPORTED;
   if (N == 0) return ENGRAM_OK;
   // A = [dk | dv] (K-major over K = 2d); B = [W_k; W_v]: (f, c) at f * E + c,
@@ -569,7 +574,7 @@ int launch_gemm_de(const __nv_bfloat16* dkv, const __nv_bfloat16* Wk, const __nv
       !make_tmap_mn(&tb1, Wv, (uint64_t)E, (uint64_t)d, (uint64_t)E, BK, GN / 2 / BK) ||
       !make_tmap_f32(&tc0, de, (uint64_t)E, (uint64_t)N, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return ENGRAM_ERR_CUDA;
-  GemmArgs a = gemm_args(N, E, 2 * d);
+  GemmArgs a = gemm_args(N, E, 2 * d, stall);
   a.b_split = d;
   a.c0 = de;
   a.ldc = E;

@@ -139,16 +139,18 @@ int launch_vocab_proj(const int64_t* keys, int32_t V, int32_t* proj, int32_t* V_
 int gemm_supported(int64_t N, int d, int E);
 // C [N, 2d] (rows ldc floats apart) = e [W_k; W_v]^T, or C [N, d] = e W_v^T
 // when Wk is NULL
+// stall: ENGRAM_TEST_STALL (the B producer issues nothing, 1 ms waits)
 int launch_gemm_kv(const __nv_bfloat16* e, const __nv_bfloat16* Wk, const __nv_bfloat16* Wv,
-                   int64_t N, int d, int E, float* C, int64_t ldc, cudaStream_t s);
+                   int64_t N, int d, int E, float* C, int64_t ldc, cudaStream_t s,
+                   bool stall = false);
 // dW_k [d, E] and dW_v [d, E] = [dk | dv]^T e over the N tokens (dkv bf16
 // [N, 2d]); ws: gemm_dw_ws_bytes of tile counters
 size_t gemm_dw_ws_bytes(int d, int E);
 int launch_gemm_dw(const __nv_bfloat16* dkv, const __nv_bfloat16* e, int64_t N, int d, int E,
-                   float* dWk, float* dWv, void* ws, cudaStream_t s);
+                   float* dWk, float* dWv, void* ws, cudaStream_t s, bool stall = false);
 // de [N, E] = [dk | dv] [W_k; W_v]
 int launch_gemm_de(const __nv_bfloat16* dkv, const __nv_bfloat16* Wk, const __nv_bfloat16* Wv,
-                   int64_t N, int d, int E, float* de, cudaStream_t s);
+                   int64_t N, int d, int E, float* de, cudaStream_t s, bool stall = false);
 
 // pre-conv RMSNorm of bf16 layers: rc[t] = (alpha_t^2 <v_t, v_t> / d + eps)^(-1/2)
 int launch_prenorm_rc(const float* v, int ldv, const float* alpha, int64_t N, int d, float* rc,
@@ -165,7 +167,7 @@ struct PrenormFwd {
 int launch_prenorm_tail(const PrenormFwd& p, const __nv_bfloat16* e, const __nv_bfloat16* Wv,
                         const __nv_bfloat16* h, const float* conv_w, const float* alpha,
                         float* conv_state, __nv_bfloat16* out, int dil, int64_t N, int T, int d,
-                        int E, cudaStream_t s);
+                        int E, bool stall, cudaStream_t s);
 
 // bf16 backward (one branch): elementwise kernels and the tensor-core GEMMs
 // kv_saved: the forward's fp32 [N, 2d] k and v, or NULL to recompute them
@@ -181,7 +183,7 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
                          const float* alpha, const float* kv_saved, const float* dout, float* dh,
                          float* dWk, float* dWv, float* dconv_w, float* de, int64_t* dtab_keys,
                          float* dtab_rows, int32_t* n_unique, int64_t N, int T, int d, int dil,
-                         bool prenorm, const float* gv, void* ws, size_t ws_bytes,
+                         bool prenorm, const float* gv, void* ws, size_t ws_bytes, bool stall,
                          cudaStream_t s);
 
 // bf16 tensor-core path (sm_100a tcgen05)
@@ -193,6 +195,6 @@ int launch_forward_tc(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv
                       const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
                       __nv_bfloat16* out, float* alpha_saved, float* kv_save, const float* gg,
                       int dil, int64_t N, int T, int d, int E, void* ws, size_t ws_bytes,
-                      bool chained, const PrenormFwd* pn, cudaStream_t s);
+                      bool chained, const PrenormFwd* pn, bool stall, cudaStream_t s);
 
 }  // namespace engram

@@ -142,9 +142,9 @@ int launch_prenorm_rc(const float* v, int ldv, const float* alpha, int64_t N, in
 int launch_prenorm_tail(const PrenormFwd& p, const __nv_bfloat16* e, const __nv_bfloat16* Wv,
                         const __nv_bfloat16* h, const float* conv_w, const float* alpha,
                         float* conv_state, __nv_bfloat16* out, int dil, int64_t N, int T, int d,
-                        int E, cudaStream_t s) {
+                        int E, bool stall, cudaStream_t s) {
   // v = e W_v^T, fp32, rows ldv apart
-  int rc = launch_gemm_kv(e, nullptr, Wv, N, d, E, p.vbuf, p.ldv, s);
+  int rc = launch_gemm_kv(e, nullptr, Wv, N, d, E, p.vbuf, p.ldv, s, stall);
   if (rc) return rc;
   if ((rc = launch_prenorm_rc(p.vbuf, p.ldv, alpha, N, d, p.rc, s))) return rc;
   const float4* w = reinterpret_cast<const float4*>(conv_w);

@@ -17,6 +17,7 @@ constexpr int BM = 128;     // accumulator rows per CTA (M = 256 over a CTA pair
 constexpr int BK = 64;      // 64 bf16 = 128 bytes: one swizzle row
 constexpr int UMMA_K = 16;  // K of one bf16 MMA instruction
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s
+constexpr uint64_t TEST_WAIT_LIMIT_NS = 1000000ull;  // 1 ms, with ENGRAM_TEST_STALL
 constexpr unsigned FULL = 0xffffffffu;
 
 // ------------------------------------------------------------ PTX wrappers
@@ -65,14 +66,14 @@ __device__ __forceinline__ uint64_t global_ns() {
 // up (returns false) when the CTA is aborting or after WAIT_LIMIT_NS, which
 // starts the abort and flags the status word.
 inline __device__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                             unsigned int* status) {
+                                    unsigned int* status, uint64_t limit_ns = WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((spin & 3u) == 0) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > WAIT_LIMIT_NS) {
+      if (global_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(status, ENGRAM_STATUS_TIMEOUT);
         return false;
@@ -83,10 +84,11 @@ inline __device__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int
 
 // Same, ignoring the abort flag: used to let in-flight copies and MMAs land
 // before the CTA releases its shared memory and TMEM.
-inline __device__ bool wait_drain(uint64_t* bar, uint32_t parity) {
+inline __device__ bool wait_drain(uint64_t* bar, uint32_t parity,
+                                  uint64_t limit_ns = WAIT_LIMIT_NS) {
   const uint64_t t0 = global_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
   return true;
 }

@@ -26,6 +26,8 @@ SAVE_KV = 1  # EngramCfg.flags
 # formulation variants (fp32 layers)
 CONV_DILATED, CONV_PRENORM, CONV_PER_BRANCH, NORM_SCALES = 2, 4, 8, 16
 STATUS_BAD_ID, STATUS_BAD_INDEX, STATUS_TIMEOUT = 1, 2, 4
+# test only: the call's bounded device-side waits run out (see engram.h)
+TEST_STALL = 1 << 30
 
 ERRORS = {
     -1: "ENGRAM_ERR_INVALID_ARG",

@@ -70,6 +70,18 @@ enum { ENGRAM_F32 = 0, ENGRAM_BF16 = 1 };
 #define ENGRAM_NORM_SCALES 16     /* learnable RMSNorm scales g_h, g_k (and g_v) */
 #define ENGRAM_VARIANT_FLAGS \
   (ENGRAM_CONV_DILATED | ENGRAM_CONV_PRENORM | ENGRAM_CONV_PER_BRANCH | ENGRAM_NORM_SCALES)
+/* Test only (the pages have no counterpart): makes a bf16 call run the
+ * wind-down path of its bounded device-side waits.  The producers of the
+ * second operand of every tensor-core kernel (the fused passes of
+ * engram_forward, the GEMMs of engram_backward) issue no copies, and the
+ * backward's row kernel arms its copy ring without issuing the copies, so
+ * the first wait on them cannot complete.  Every bounded wait of the call
+ * gives up after about 1 ms instead of 2 s; the kernels set
+ * ENGRAM_STATUS_TIMEOUT, let what they issued land, release their tensor
+ * memory and return.  The call returns ENGRAM_OK and its outputs are
+ * undefined; later calls without the flag are unaffected.  fp32 layers
+ * (no such waits) ignore it. */
+#define ENGRAM_TEST_STALL (1 << 30)
 
 enum {
   ENGRAM_OK = 0,
