@@ -973,7 +973,8 @@ def bench_decode(dev):
     steps of Zipf(1.1) ids, each step with its own pregenerated hidden state
     N(0, 1); d 4,096, K 8 x ~6.35M rows x 128 (13B bf16 parameters, 26 GB on
     the device), rolling n-gram and conv state.  One step = hash with the
-    n-gram state, gather, fused passes in decode mode.  All 2,000 steps are
+    n-gram state and gather (one kernel), fused passes in decode mode
+    (engram_decode_step).  All 2,000 steps are
     captured into one CUDA graph (each step reading its own ids and h rows),
     replayed once untimed and once timed from the same initial state."""
     import torch
@@ -1003,16 +1004,14 @@ def bench_decode(dev):
     ids = torch.from_numpy(ids_np).to(dev)
     state = torch.full((w.B, 2), V_c, dtype=torch.int32, device=dev)
     conv_state = torch.zeros((w.B, 1, 3, w.d), device=dev)
-    idx = torch.empty((w.B, 1, w.J), dtype=torch.int32, device=dev)
     e = torch.empty((w.B, w.E), dtype=torch.bfloat16, device=dev)
     out = torch.empty((w.B, 1, 1, w.d), dtype=torch.bfloat16, device=dev)
     fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, w.B)
     fws = torch.empty(fb, dtype=torch.uint8, device=dev)
 
-    def step(k):
-        eg.engram_hash_indices(cfg, proj, ids[k], w.B, 1, state, idx, s)
-        eg.engram_forward(cfg, idx, table, e, hs[k], Wk, Wv, cw, conv_state, out, None, w.B, 1,
-                          fws, fb, s)
+    def step(k):  # hash + gather in one kernel, then the fused passes
+        eg.engram_decode_step(cfg, proj, ids[k], state, None, table, e, hs[k], Wk, Wv, cw,
+                              conv_state, out, w.B, fws, fb, s)
 
     def reset():
         state.fill_(V_c)

@@ -109,6 +109,44 @@ HeadParams make_head_params(const engram_cfg_t* cfg) {
   return hp;
 }
 
+// The layer after the gather (gate, value, conv, residual), for engram_forward
+// and engram_decode_step; `chained`: a gather kernel of this call runs just
+// before, so the first pass may start as it ends (programmatic launch).
+int forward_from_e(const engram_cfg_t* cfg, const HeadParams& hp, void* e, const void* h,
+                   const void* Wk, const void* Wv, const float* conv_w, float* conv_state,
+                   void* out, float* saved, int64_t N, int32_t T, void* ws, size_t ws_bytes,
+                   bool chained, cudaStream_t s) {
+  const int M = cfg->n_branch, d = cfg->d_model, E = hp.E;
+  int rc;
+  if (cfg->dtype == ENGRAM_F32)
+    return launch_forward_f32(static_cast<const float*>(e), static_cast<const float*>(h),
+                              static_cast<const float*>(Wk), static_cast<const float*>(Wv), conv_w,
+                              cfg->flags, conv_state, static_cast<float*>(out), saved, N, T, M, d,
+                              E, ws, s);
+  float* kv_save = saved != nullptr && conv_state == nullptr && saves_kv(cfg)
+                       ? reinterpret_cast<float*>(reinterpret_cast<char*>(saved) +
+                                                  alpha_bytes_padded(N))
+                       : nullptr;
+  const Bf16FwdWs wl = bf16_fwd_ws(cfg, N);
+  char* wsb = static_cast<char*>(ws);
+  float* gg = nullptr;  // g_h g_k, after the passes' workspace
+  if (bf16_scaled(cfg)) {
+    gg = reinterpret_cast<float*>(wsb + wl.gg);
+    if ((rc = launch_scale_product(conv_w + 4 * d, conv_w + 5 * d, d, gg, s))) return rc;
+  }
+  // the pre-conv norm: v into the kept [k | v] rows when there are any
+  PrenormFwd pn{bf16_scaled(cfg) ? conv_w + 6 * d : nullptr,
+                kv_save != nullptr ? kv_save + d : reinterpret_cast<float*>(wsb + wl.vbuf),
+                kv_save != nullptr ? 2 * d : d, reinterpret_cast<float*>(wsb + wl.rc)};
+  return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
+                           static_cast<const __nv_bfloat16*>(Wk),
+                           static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
+                           static_cast<__nv_bfloat16*>(out), saved, kv_save, gg,
+                           (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1, N, T, d, E, ws, ws_bytes,
+                           chained, bf16_prenorm(cfg) ? &pn : nullptr,
+                           (cfg->flags & ENGRAM_TEST_STALL) != 0, s);
+}
+
 }  // namespace engram
 
 using namespace engram;
@@ -210,40 +248,47 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
   if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
   const HeadParams hp = make_head_params(cfg);
-  const int M = cfg->n_branch, d = cfg->d_model, E = hp.E;
-  if (cfg->dtype == ENGRAM_BF16 && (!tc_supported(d, E, M) || !bf16_variant_ok(cfg)))
+  if (cfg->dtype == ENGRAM_BF16 &&
+      (!tc_supported(cfg->d_model, hp.E, cfg->n_branch) || !bf16_variant_ok(cfg)))
     return ENGRAM_ERR_UNSUPPORTED;
   if (table != nullptr) {
     rc = launch_gather(hp, idx, table, N, elem_bytes(cfg), e, s);
     if (rc) return rc;
   }
-  if (cfg->dtype == ENGRAM_F32)
-    return launch_forward_f32(static_cast<const float*>(e), static_cast<const float*>(h),
-                              static_cast<const float*>(Wk), static_cast<const float*>(Wv), conv_w,
-                              cfg->flags, conv_state, static_cast<float*>(out), saved, N, T, M, d,
-                              E, ws, s);
-  float* kv_save = saved != nullptr && conv_state == nullptr && saves_kv(cfg)
-                       ? reinterpret_cast<float*>(reinterpret_cast<char*>(saved) +
-                                                  alpha_bytes_padded(N))
-                       : nullptr;
-  const Bf16FwdWs wl = bf16_fwd_ws(cfg, N);
-  char* wsb = static_cast<char*>(ws);
-  float* gg = nullptr;  // g_h g_k, after the passes' workspace
-  if (bf16_scaled(cfg)) {
-    gg = reinterpret_cast<float*>(wsb + wl.gg);
-    if ((rc = launch_scale_product(conv_w + 4 * d, conv_w + 5 * d, d, gg, s))) return rc;
-  }
-  // the pre-conv norm: v into the kept [k | v] rows when there are any
-  PrenormFwd pn{bf16_scaled(cfg) ? conv_w + 6 * d : nullptr,
-                kv_save != nullptr ? kv_save + d : reinterpret_cast<float*>(wsb + wl.vbuf),
-                kv_save != nullptr ? 2 * d : d, reinterpret_cast<float*>(wsb + wl.rc)};
-  return launch_forward_tc(static_cast<const __nv_bfloat16*>(e), static_cast<const __nv_bfloat16*>(h),
-                           static_cast<const __nv_bfloat16*>(Wk),
-                           static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
-                           static_cast<__nv_bfloat16*>(out), saved, kv_save, gg,
-                           (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1, N, T, d, E, ws, ws_bytes,
-                           table != nullptr, bf16_prenorm(cfg) ? &pn : nullptr,
-                           (cfg->flags & ENGRAM_TEST_STALL) != 0, s);
+  return forward_from_e(cfg, hp, e, h, Wk, Wv, conv_w, conv_state, out, saved, N, T, ws, ws_bytes,
+                        table != nullptr, s);
+}
+
+int engram_decode_step(const engram_cfg_t* cfg, const int32_t* proj, const int32_t* ids,
+                       int32_t* ngram_state, int32_t* idx, const void* table, void* e,
+                       const void* h, const void* Wk, const void* Wv, const float* conv_w,
+                       float* conv_state, void* out, int32_t B, void* ws, size_t ws_bytes,
+                       void* stream) {
+  const NvtxRange nvtx("engram_decode_step");
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (B < 0) return ENGRAM_ERR_INVALID_ARG;
+  if (B == 0) return ENGRAM_OK;
+  if (proj == nullptr || ids == nullptr || ngram_state == nullptr || table == nullptr ||
+      e == nullptr || h == nullptr || Wk == nullptr || Wv == nullptr || conv_w == nullptr ||
+      conv_state == nullptr || out == nullptr)
+    return ENGRAM_ERR_INVALID_ARG;
+  if (!aligned16(proj) || !aligned16(ids) || !aligned16(ngram_state) || !aligned16(idx) ||
+      !aligned16(table) || !aligned16(e) || !aligned16(h) || !aligned16(Wk) || !aligned16(Wv) ||
+      !aligned16(conv_w) || !aligned16(conv_state) || !aligned16(out) || !aligned16(ws))
+    return ENGRAM_ERR_MISALIGNED;
+  if (ws_bytes < engram_workspace_size(cfg, ENGRAM_WS_FORWARD, B)) return ENGRAM_ERR_WORKSPACE;
+  if (status_ptr() == nullptr) return ENGRAM_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  const HeadParams hp = make_head_params(cfg);
+  if (cfg->dtype == ENGRAM_BF16 &&
+      (!tc_supported(cfg->d_model, hp.E, cfg->n_branch) || !bf16_variant_ok(cfg)))
+    return ENGRAM_ERR_UNSUPPORTED;
+  if ((rc = launch_hash_gather_decode(hp, proj, ids, B, ngram_state, idx, table, elem_bytes(cfg),
+                                      e, s)))
+    return rc;
+  return forward_from_e(cfg, hp, e, h, Wk, Wv, conv_w, conv_state, out, nullptr, B, 1, ws,
+                        ws_bytes, true, s);
 }
 
 int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,

@@ -81,6 +81,11 @@ int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, i
                 int32_t* ngram_state, int32_t* idx, cudaStream_t s);
 int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,
                   int elem_bytes, void* e, cudaStream_t s);
+// one decode step's hash (rolling n-gram state, idx optional) and gather in
+// one launch, B sequences of one token
+int launch_hash_gather_decode(const HeadParams& hp, const int32_t* proj, const int32_t* ids,
+                              int64_t B, int32_t* ngram_state, int32_t* idx, const void* table,
+                              int elem_bytes, void* e, cudaStream_t s);
 // the same gather from pinned host memory: a small fixed grid, deep per-thread
 // load queues (PCIe latency), the GPU's other SMs left free
 int launch_gather_host(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,

@@ -114,6 +114,58 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HeadP
     *reinterpret_cast<int2*>(idx + n * hp.J + j0) = make_int2(s[0], s[1]);
 }
 
+// One decode step's hash and gather in one launch (one token per sequence,
+// the n-gram history from the rolling state): a block per token.  Thread 0
+// reads the token's compressed id and state; threads 0..J-1 hash one head
+// each; then the block copies the token's J rows in 16-byte pieces, and
+// thread 0 writes the new state (c_t, c_{t-1}) -- only thread 0 reads or
+// writes the state, so no other thread can see it half-updated.
+__global__ void __launch_bounds__(256) hash_gather_decode_kernel(
+    const __grid_constant__ HeadParams hp, const int32_t* __restrict__ proj,
+    const int32_t* __restrict__ ids, int32_t* __restrict__ ngram_state,
+    int32_t* __restrict__ idx, const uint4* __restrict__ table, int CR,
+    uint4* __restrict__ e, unsigned int* status) {
+  allow_dependents();
+  __shared__ int32_t cid[3];
+  __shared__ int32_t slot[ENGRAM_MAX_HEADS];
+  const int64_t n = blockIdx.x;
+  const int J = hp.J;
+  if (threadIdx.x == 0) {
+    const int32_t c0 = token_cid(proj, ids, n, hp.V_raw, hp.V_c);
+    const int32_t c1 = ngram_state[2 * n + 0], c2 = ngram_state[2 * n + 1];
+    if (c0 < 0) atomicOr(status, ENGRAM_STATUS_BAD_ID);
+    cid[0] = c0;
+    cid[1] = c1;
+    cid[2] = c2;
+  }
+  __syncthreads();
+  const int32_t c0 = cid[0], c1 = cid[1], c2 = cid[2];
+  if (threadIdx.x < J) {
+    const int j = threadIdx.x;
+    const bool bad2 = (c0 < 0) | (c1 < 0);
+    const bool bad3 = bad2 | (c2 < 0);
+    uint64_t x = (uint64_t)(uint32_t)c0 * hp.mult[j][0];
+    x ^= (uint64_t)(uint32_t)c1 * hp.mult[j][1];
+    const bool tri = j >= hp.K;
+    if (tri) x ^= (uint64_t)(uint32_t)c2 * hp.mult[j][2];
+    const int32_t sl = (tri ? bad3 : bad2) ? -1 : (int32_t)mod_prime(x, hp.P[j], hp.mu[j]);
+    slot[j] = sl;
+    if (idx != nullptr) idx[n * J + j] = sl;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    ngram_state[2 * n + 0] = c0;
+    ngram_state[2 * n + 1] = c1;
+  }
+  const int per_tok = J * CR;
+  for (int p = threadIdx.x; p < per_tok; p += blockDim.x) {
+    const int j = p / CR, c = p - j * CR;
+    const int32_t sl = slot[j];
+    e[n * per_tok + p] =
+        sl >= 0 ? ld_row_piece(table + (hp.row_base[j] + sl) * CR + c) : make_uint4(0, 0, 0, 0);
+  }
+}
+
 // Row gather with 16-byte vectors, generic shape.  The e row of a token is
 // J*CR chunks of 16 bytes (CR per head row); consecutive threads take
 // consecutive chunks, so the stores are fully coalesced.  Every thread keeps
@@ -285,28 +337,194 @@ int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, i
   return ck(cudaGetLastError());
 }
 
+int launch_hash_gather_decode(const HeadParams& hp, const int32_t* proj, const int32_t* ids,
+                              int64_t B, int32_t* ngram_state, int32_t* idx, const void* table,
+                              int elem_bytes, void* e, cudaStream_t s) {
+  if (B == 0) return ENGRAM_OK;
+  const int CR = hp.D_h * elem_bytes / 16;
+  const int per_tok = hp.J * CR;
+  // at least a warp (threads 0..J-1 hash, J <= 32), at most 256 pieces at a time
+  int threads = ((per_tok + 31) / 32) * 32;
+  if (threads > 256) threads = 256;
+  hash_gather_decode_kernel<<<(unsigned)B, (unsigned)threads, 0, s>>>(
+      hp, proj, ids, ngram_state, idx, static_cast<const uint4*>(table), CR,
+      static_cast<uint4*>(e), status_ptr());
+  return ck(cudaGetLastError());
+}
+
 // Gather from a table in pinned, mapped host memory.  Reads cross PCIe, so
-// the time goes to latency, not to the SMs: a few small CTAs with many loads
-// in flight each (128 threads x 8 x 16 B) leave the rest of the GPU to the
-// work on the compute stream.  Measured on B200 with a bf16 GEMM
-// [8,192 x 2,560] x [2,560 x 10,240] on the compute stream: 16 CTAs keep the
-// GEMM within 9% of its time alone at 17 GB/s of rows; 32 CTAs reach 21 GB/s
-// but slow the GEMM by 46%; a full grid reaches 30 GB/s and serialises it.
+// the time goes to latency and to the size of the link's read requests, not
+// to the SMs: a few CTAs, each with many rows in flight, leave the rest of
+// the GPU to the work on the compute stream.  Each warp walks its own tokens;
+// for a token, lanes 0..J-1 each copy one table row (D_h elements, a multiple
+// of 16 bytes) from host memory into a shared-memory slot with one
+// cp.async.bulk, all completing on the slot's mbarrier, so a row crosses the
+// link as one request stream instead of 16-byte loads.  The warp then writes
+// the slot to e with coalesced 16-byte stores.  HG_SLOTS slots per warp keep
+// that many tokens' rows in flight.  Slots of -1 read nothing and give zero
+// rows; slots outside [0, P_j) also set ENGRAM_STATUS_BAD_INDEX.  A slot
+// whose copies do not land within the wait limit sets
+// ENGRAM_STATUS_TIMEOUT; the warp then stops and lets its copies in flight
+// land (bounded) before the block exits.
+namespace {
+
 #ifndef ENGRAM_HOST_GATHER_CTAS
 #define ENGRAM_HOST_GATHER_CTAS 16
 #endif
+constexpr int HG_WARPS = 8;
+constexpr int HG_SLOTS = 2;  // 1, 2 and 3 slots measured alike (16 CTAs)
+constexpr uint64_t HG_WAIT_NS = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint32_t hg_smem(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ bool hg_wait(uint64_t* bar, uint32_t parity) {
+  uint64_t t0 = 0;
+  for (int spin = 0;; ++spin) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(hg_smem(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    if (ok) return true;
+    uint64_t now;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+    if (spin == 0) t0 = now;
+    else if (now - t0 > HG_WAIT_NS) return false;
+  }
+}
+
+__global__ void __launch_bounds__(HG_WARPS * 32) gather_host_rows_kernel(
+    const __grid_constant__ HeadParams hp, const int32_t* __restrict__ idx,
+    const uint8_t* __restrict__ table, int64_t n_tok, int row_bytes, int slots,
+    uint4* __restrict__ e, unsigned int* status) {
+  extern __shared__ __align__(128) uint8_t hg_ring[];
+  __shared__ uint64_t bars[HG_WARPS][HG_SLOTS];
+  __shared__ uint32_t masks[HG_WARPS][HG_SLOTS];  // rows of the slot's token that were copied
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int J = hp.J;
+  const int tok_bytes = J * row_bytes;
+  const int pieces = tok_bytes / 16, row_pieces = row_bytes / 16;
+  uint8_t* ring = hg_ring + (size_t)warp * slots * tok_bytes;
+  const int64_t first = (int64_t)blockIdx.x * HG_WARPS + warp;
+  const int64_t stride = (int64_t)gridDim.x * HG_WARPS;
+  if (lane < slots) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(hg_smem(&bars[warp][lane])));
+  }
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __syncwarp();
+  unsigned pend = 0;  // lane 0: slots with copies issued and not yet seen landed
+  // Copies of token t's rows into `slot`: lane 0 posts the bytes to expect,
+  // then lanes 0..J-1 issue one row each.
+  auto issue = [&](int64_t t, int slot) {
+    int32_t sl = -1;
+    bool ok = false;
+    if (lane < J) {
+      sl = __ldg(idx + t * J + lane);
+      ok = sl >= 0 && (uint64_t)sl < hp.P[lane];
+      if (!ok && sl != -1) atomicOr(status, ENGRAM_STATUS_BAD_INDEX);
+    }
+    const uint32_t mask = __ballot_sync(0xffffffffu, ok);
+    if (lane == 0) {
+      masks[warp][slot] = mask;
+      pend |= 1u << slot;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                       hg_smem(&bars[warp][slot])),
+                   "r"((uint32_t)__popc(mask) * (uint32_t)row_bytes)
+                   : "memory");
+    }
+    __syncwarp();
+    if (ok) {
+      const uint8_t* src = table + (uint64_t)(hp.row_base[lane] + sl) * (uint64_t)row_bytes;
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+          ::"r"(hg_smem(ring + (size_t)slot * tok_bytes + (size_t)lane * row_bytes)),
+          "l"(src), "r"((uint32_t)row_bytes), "r"(hg_smem(&bars[warp][slot]))
+          : "memory");
+    }
+  };
+  for (int k = 0; k < slots; ++k) {
+    const int64_t t = first + k * stride;
+    if (t < n_tok) issue(t, k);
+  }
+  int k = 0;
+  for (int64_t t = first; t < n_tok; t += stride, ++k) {
+    const int slot = k % slots;
+    int ok = 1;
+    if (lane == 0) ok = hg_wait(&bars[warp][slot], (uint32_t)(k / slots) & 1u) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) {
+      if (lane == 0) atomicOr(status, ENGRAM_STATUS_TIMEOUT);
+      break;
+    }
+    if (lane == 0) pend &= ~(1u << slot);
+    const uint32_t mask = masks[warp][slot];
+    const uint4* src = reinterpret_cast<const uint4*>(ring + (size_t)slot * tok_bytes);
+    uint4* dst = e + t * pieces;
+    for (int p = lane; p < pieces; p += 32) {
+      const int r = p / row_pieces;
+      dst[p] = ((mask >> r) & 1u) ? src[p] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncwarp();  // every lane has read the slot before it is refilled
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    const int64_t nt = t + (int64_t)slots * stride;
+    if (nt < n_tok) issue(nt, slot);
+  }
+  // after a timeout: let the copies still in flight land (bounded) before the
+  // block's shared memory is released; a slot holds at most one use, the one
+  // after the last waited for
+  if (lane == 0 && pend != 0) {
+    for (int sl = 0; sl < slots; ++sl) {
+      if (!(pend & (1u << sl))) continue;
+      const int use = k / slots + (sl < k % slots ? 1 : 0);
+      hg_wait(&bars[warp][sl], (uint32_t)use & 1u);
+    }
+  }
+}
+
+}  // namespace
 
 int launch_gather_host(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,
                        int elem_bytes, void* e, cudaStream_t s) {
   if (n_tok == 0) return ENGRAM_OK;
-  const int CR = hp.D_h * elem_bytes / 16;
-  constexpr int UNROLL = 8;
-  constexpr int threads = 128;
-  const int64_t total = n_tok * hp.J * CR;
-  int64_t blocks = (total + (int64_t)threads * UNROLL - 1) / ((int64_t)threads * UNROLL);
+  const int row_bytes = hp.D_h * elem_bytes;
+  constexpr size_t kRing = 160 * 1024;  // shared memory for the warps' slots
+  const size_t tok_bytes = (size_t)hp.J * row_bytes;
+  int slots = (int)(kRing / (HG_WARPS * tok_bytes));
+  if (slots > HG_SLOTS) slots = HG_SLOTS;
+  if (slots < 1) {
+    // a token's rows exceed a slot: 16-byte loads, eight in flight per thread
+    constexpr int UNROLL = 8;
+    const int CR = row_bytes / 16;
+    const int64_t total = n_tok * hp.J * CR;
+    int64_t blocks = (total + 128 * UNROLL - 1) / (128 * UNROLL);
+    if (blocks > ENGRAM_HOST_GATHER_CTAS) blocks = ENGRAM_HOST_GATHER_CTAS;
+    gather_kernel<UNROLL><<<(unsigned)blocks, 128, 0, s>>>(
+        hp, idx, static_cast<const uint4*>(table), n_tok, CR, static_cast<uint4*>(e),
+        status_ptr());
+    return ck(cudaGetLastError());
+  }
+  const size_t smem = (size_t)HG_WARPS * slots * tok_bytes;
+  static bool configured[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ENGRAM_ERR_CUDA;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(gather_host_rows_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRing) !=
+        cudaSuccess)
+      return ENGRAM_ERR_CUDA;
+    configured[dev] = true;
+  }
+  // one warp per token at most; ENGRAM_HOST_GATHER_CTAS blocks at most
+  int64_t blocks = (n_tok + HG_WARPS - 1) / HG_WARPS;
   if (blocks > ENGRAM_HOST_GATHER_CTAS) blocks = ENGRAM_HOST_GATHER_CTAS;
-  gather_kernel<UNROLL><<<(unsigned)blocks, threads, 0, s>>>(
-      hp, idx, static_cast<const uint4*>(table), n_tok, CR, static_cast<uint4*>(e), status_ptr());
+  gather_host_rows_kernel<<<(unsigned)blocks, HG_WARPS * 32, smem, s>>>(
+      hp, idx, static_cast<const uint8_t*>(table), n_tok, row_bytes, slots,
+      static_cast<uint4*>(e), status_ptr());
   return ck(cudaGetLastError());
 }
 
@@ -402,35 +620,90 @@ __global__ void __launch_bounds__(256) gather_hits_kernel(
 }
 
 // Pass 3, on a few CTAs (the reads cross PCIe): the listed (token, head)
-// rows from host memory.
-template <int UNROLL>
-__global__ void __launch_bounds__(128) gather_misses_kernel(
+// rows from host memory, by bulk copies as in gather_host_rows_kernel: a
+// warp takes grp (up to 32) listed rows at a time, each lane copying one row
+// into the warp's shared-memory slot; the warp then writes the rows to their
+// places in e.  `slots` groups per warp are in flight.
+__global__ void __launch_bounds__(HG_WARPS * 32) gather_misses_kernel(
     const __grid_constant__ HeadParams hp, const int32_t* __restrict__ idx,
-    const uint4* __restrict__ host, const int32_t* __restrict__ miss_list,
-    const int32_t* __restrict__ n_miss, int CR, uint4* __restrict__ e) {
-  const int64_t total = (int64_t)(*n_miss) * CR;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < total;
-       base += stride * UNROLL) {
-    uint4 v[UNROLL];
-    int64_t dst[UNROLL];
-#pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int64_t g = base + u * stride;
-      dst[u] = -1;
-      if (g < total) {
-        const int64_t m = g / CR;
-        const int c = (int)(g - m * CR);
-        const int32_t item = miss_list[m];  // n * J + j
-        const int j = item % hp.J;
-        const int32_t s = __ldg(idx + item);  // valid: the probe checked it
-        v[u] = ld_row_piece(host + (hp.row_base[j] + s) * CR + c);
-        dst[u] = (int64_t)item * CR + c;
-      }
+    const uint8_t* __restrict__ host, const int32_t* __restrict__ miss_list,
+    const int32_t* __restrict__ n_miss, int row_bytes, int grp, int slots,
+    uint8_t* __restrict__ e, unsigned int* status) {
+  extern __shared__ __align__(128) uint8_t hg_ring[];
+  __shared__ uint64_t bars[HG_WARPS][HG_SLOTS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int J = hp.J;
+  const int grp_bytes = grp * row_bytes, row_pieces = row_bytes / 16;
+  uint8_t* ring = hg_ring + (size_t)warp * slots * grp_bytes;
+  const int64_t n = *n_miss;
+  const int64_t groups = (n + grp - 1) / grp;
+  const int64_t first = (int64_t)blockIdx.x * HG_WARPS + warp;
+  const int64_t stride = (int64_t)gridDim.x * HG_WARPS;
+  if (lane < slots) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(hg_smem(&bars[warp][lane])));
+  }
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __syncwarp();
+  unsigned pend = 0;
+  auto issue = [&](int64_t gi, int slot) {
+    const int64_t m = gi * grp + lane;
+    const bool ok = lane < grp && m < n;
+    const uint32_t cnt = __popc(__ballot_sync(0xffffffffu, ok));
+    if (lane == 0) {
+      pend |= 1u << slot;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                       hg_smem(&bars[warp][slot])),
+                   "r"(cnt * (uint32_t)row_bytes)
+                   : "memory");
     }
-#pragma unroll
-    for (int u = 0; u < UNROLL; ++u)
-      if (dst[u] >= 0) e[dst[u]] = v[u];
+    __syncwarp();
+    if (ok) {
+      const int32_t item = miss_list[m];  // n * J + j
+      const int j = item % J;
+      const int32_t sl = __ldg(idx + item);  // valid: the probe checked it
+      const uint8_t* src = host + (uint64_t)(hp.row_base[j] + sl) * (uint64_t)row_bytes;
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+          ::"r"(hg_smem(ring + (size_t)slot * grp_bytes + (size_t)lane * row_bytes)),
+          "l"(src), "r"((uint32_t)row_bytes), "r"(hg_smem(&bars[warp][slot]))
+          : "memory");
+    }
+  };
+  for (int k = 0; k < slots; ++k) {
+    const int64_t gi = first + k * stride;
+    if (gi < groups) issue(gi, k);
+  }
+  int k = 0;
+  for (int64_t gi = first; gi < groups; gi += stride, ++k) {
+    const int slot = k % slots;
+    int ok = 1;
+    if (lane == 0) ok = hg_wait(&bars[warp][slot], (uint32_t)(k / slots) & 1u) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) {
+      if (lane == 0) atomicOr(status, ENGRAM_STATUS_TIMEOUT);
+      break;
+    }
+    if (lane == 0) pend &= ~(1u << slot);
+    const int64_t m0 = gi * grp;
+    const int cnt = (int)(n - m0 < grp ? n - m0 : grp);
+    const uint4* src = reinterpret_cast<const uint4*>(ring + (size_t)slot * grp_bytes);
+    for (int p = lane; p < cnt * row_pieces; p += 32) {
+      const int r = p / row_pieces;
+      const int c = p - r * row_pieces;
+      uint4* dst = reinterpret_cast<uint4*>(e + (int64_t)miss_list[m0 + r] * row_bytes) + c;
+      *dst = src[p];
+    }
+    __syncwarp();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    const int64_t ng = gi + (int64_t)slots * stride;
+    if (ng < groups) issue(ng, slot);
+  }
+  if (lane == 0 && pend != 0) {
+    for (int sl = 0; sl < slots; ++sl) {
+      if (!(pend & (1u << sl))) continue;
+      const int use = k / slots + (sl < k % slots ? 1 : 0);
+      hg_wait(&bars[warp][sl], (uint32_t)use & 1u);
+    }
   }
 }
 
@@ -481,8 +754,27 @@ int launch_gather_cached(const HeadParams& hp, const int32_t* idx, const void* h
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
     gather_hits_kernel<UNROLL><<<(unsigned)blocks, 256, 0, s>>>(
         hp.J, item_slot, static_cast<const uint4*>(cache), n_tok, CR, static_cast<uint4*>(e));
-    gather_misses_kernel<8><<<ENGRAM_HOST_GATHER_CTAS, 128, 0, s>>>(
-        hp, idx, static_cast<const uint4*>(host), miss_list, n_miss, CR, static_cast<uint4*>(e));
+    // groups of up to 32 rows per warp slot, as many slots (up to
+    // HG_SLOTS) as kRing bytes of shared memory hold
+    const int row_bytes = CR * 16;
+    constexpr size_t kRing = 160 * 1024;
+    int grp = (int)(kRing / ((size_t)HG_WARPS * row_bytes));
+    if (grp > 32) grp = 32;
+    if (grp < 1) return ENGRAM_ERR_UNSUPPORTED;  // a row over 20 KB
+    int slots = (int)(kRing / ((size_t)HG_WARPS * grp * row_bytes));
+    if (slots > HG_SLOTS) slots = HG_SLOTS;
+    static bool configured[64] = {false};
+    if (dev < 0 || dev >= 64) return ENGRAM_ERR_CUDA;
+    if (!configured[dev]) {
+      if ((rc = ck(cudaFuncSetAttribute(gather_misses_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRing))))
+        return rc;
+      configured[dev] = true;
+    }
+    gather_misses_kernel<<<ENGRAM_HOST_GATHER_CTAS, HG_WARPS * 32,
+                           (size_t)HG_WARPS * slots * grp * row_bytes, s>>>(
+        hp, idx, static_cast<const uint8_t*>(host), miss_list, n_miss, row_bytes, grp, slots,
+        static_cast<uint8_t*>(e), status_ptr());
     if ((rc = ck(cudaGetLastError()))) return rc;
   }
   if (n_miss_out != nullptr)

@@ -42,7 +42,8 @@ NOALLOC_MAX_ITEMS = 131072
 
 EXPORTED = (
     "engram_workspace_size", "engram_saved_size", "engram_build_vocab_proj",
-    "engram_hash_indices", "engram_gather", "engram_forward", "engram_backward",
+    "engram_hash_indices", "engram_gather", "engram_forward", "engram_decode_step",
+    "engram_backward",
     "engram_table_grad", "engram_table_grad_noalloc", "engram_forward_hosttable",
     "engram_get_status",
     "engram_device_sm_count", "engram_table_rows", "engram_param_floats",
@@ -108,6 +109,8 @@ def lib() -> ctypes.CDLL:
         "engram_hash_indices": (ctypes.c_int, [cfgp, P, P, i32, i32, P, P, P]),
         "engram_gather": (ctypes.c_int, [cfgp, P, P, i64, P, P]),
         "engram_forward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P, i32, i32, P, sz, P]),
+        "engram_decode_step": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, i32, P,
+                                              sz, P]),
         "engram_backward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                            i32, i32, P, sz, P]),
         "engram_table_grad": (ctypes.c_int, [cfgp, P, P, i64, P, P, P, P, sz, P]),
@@ -186,6 +189,15 @@ def engram_forward(cfg: EngramCfg, idx, table, e, h, Wk, Wv, conv_w, conv_state,
            lib().engram_forward(ctypes.byref(cfg), _p(idx), _p(table), _p(e), _p(h), _p(Wk),
                                 _p(Wv), _p(conv_w), _p(conv_state), _p(out), _p(saved), B, T,
                                 _p(ws), ws_bytes, _s(stream)))
+
+
+def engram_decode_step(cfg: EngramCfg, proj, ids, ngram_state, idx, table, e, h, Wk, Wv,
+                       conv_w, conv_state, out, B: int, ws, ws_bytes: int, stream=None) -> None:
+    _check("engram_decode_step",
+           lib().engram_decode_step(ctypes.byref(cfg), _p(proj), _p(ids), _p(ngram_state),
+                                    _p(idx), _p(table), _p(e), _p(h), _p(Wk), _p(Wv),
+                                    _p(conv_w), _p(conv_state), _p(out), B, _p(ws), ws_bytes,
+                                    _s(stream)))
 
 
 def engram_backward(cfg: EngramCfg, idx, e, h, Wk, Wv, conv_w, saved, dout, dh, dWk, dWv,

@@ -236,6 +236,27 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
                    size_t ws_bytes, void* stream);
 
 /*
+ * One decode step in one call: for B sequences of one new token each,
+ * steps 1-3 with the n-gram history from the rolling state and step 4 run
+ * as one kernel (a block per token), then steps 5-6 as engram_forward with
+ * a conv state.  The same results, bit for bit, as engram_hash_indices
+ * (T = 1, with ngram_state) followed by engram_forward (table non-NULL,
+ * conv_state non-NULL), with one kernel launch fewer per step ([p4]
+ * indices depend only on the tokens; [p5 三.4] per-token inference).
+ *   proj, ids        as engram_hash_indices: ids device int32 [B].
+ *   ngram_state      device int32 [B, 2], in/out: (c_{t-1}, c_{t-2}).
+ *   idx              device int32 [B, J] out (the step's slots), or NULL.
+ *   table, e, h, Wk, Wv, conv_w, conv_state, out, ws
+ *                    as engram_forward with T = 1 (conv_state required;
+ *                    nothing is saved for a backward).
+ */
+int engram_decode_step(const engram_cfg_t* cfg, const int32_t* proj, const int32_t* ids,
+                       int32_t* ngram_state, int32_t* idx, const void* table, void* e,
+                       const void* h, const void* Wk, const void* Wv, const float* conv_w,
+                       float* conv_state, void* out, int32_t B, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
  * Backward of engram_forward for L = sum(dout * out) ([p4]: end-to-end
  * training; lookups are deterministic, so a slot gets consistent gradients).
  * Inputs as in engram_forward (e as the forward left it; saved may be NULL:

@@ -339,3 +339,55 @@ def test_forward_in_place_equals_separate_output(B, T, d, dtype):
     assert torch.equal(L.h, sep)
     assert np.array_equal(_alpha(L, N, 1), alpha_sep)
     assert eg.engram_get_status() == 0
+
+
+@pytest.mark.parametrize("dtype,B,d,K,D_h,flags", [
+    ("bf16", 37, 256, 2, 32, 0),                  # narrow tensor-core tiles, ragged batch
+    ("bf16", 300, 512, 4, 16, eg.CONV_DILATED),   # two token tiles, dilated conv state
+    ("f32", 5, 64, 2, 16, 0),                     # fp32 layer
+    ("f32", 9, 64, 3, 16, 0),                     # J = 6 heads (two per hash thread)
+])
+def test_decode_step_equals_hash_then_forward(dtype, B, d, K, D_h, flags):
+    """engram_decode_step (hash and gather in one kernel, then the layer) gives
+    the same bits as engram_hash_indices followed by engram_forward, step after
+    step: slots, n-gram state, gathered rows, output and conv state."""
+    rng = np.random.default_rng(B * 7 + d)
+    J, E = 2 * K, 2 * K * D_h
+    rows = synth.primes_at_most(3001, J)
+    V = 1000
+    keys = synth.merge_keys(np.random.default_rng(5), V, synth.compressed_vocab(V))
+    proj, V_c = gpu_vocab_proj(keys)
+    mult = synth.hash_multipliers(77, J)
+    cfg = eg.make_cfg(K, D_h, d, 1, V, V_c, eg.BF16 if dtype == "bf16" else eg.F32, rows, mult,
+                      flags=flags)
+    tables = [rng.standard_normal((P, D_h)).astype(np.float32) for P in rows]
+    to = (lambda x: bf16_dev(x)) if dtype == "bf16" else (lambda x: dev(x))
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    table = packed_table(tables, dtype)
+    Wk = to((rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32))
+    Wv = to((rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32))
+    cw = dev((rng.standard_normal((d, 4)) * 0.5).astype(np.float32))
+    dil = 3 if flags & eg.CONV_DILATED else 1
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, B)
+    paths = []
+    for _ in range(2):
+        paths.append(dict(
+            state=torch.full((B, 2), V_c, dtype=torch.int32, device="cuda"),
+            conv=torch.zeros((B, 1, 3 * dil, d), dtype=torch.float32, device="cuda"),
+            idx=torch.empty((B, 1, J), dtype=torch.int32, device="cuda"),
+            e=torch.empty((B, E), dtype=tdt, device="cuda"),
+            out=torch.empty((B, 1, 1, d), dtype=tdt, device="cuda"),
+            ws=ws(fb)))
+    a, b = paths
+    for step in range(6):
+        ids = dev(rng.integers(0, V, size=B).astype(np.int32))
+        h = to(rng.standard_normal((B, 1, 1, d)).astype(np.float32))
+        eg.engram_hash_indices(cfg, proj, ids, B, 1, a["state"], a["idx"])
+        eg.engram_forward(cfg, a["idx"], table, a["e"], h, Wk, Wv, cw, a["conv"], a["out"], None,
+                          B, 1, a["ws"], fb)
+        eg.engram_decode_step(cfg, proj, ids, b["state"], b["idx"], table, b["e"], h, Wk, Wv, cw,
+                              b["conv"], b["out"], B, b["ws"], fb)
+        torch.cuda.synchronize()
+        assert eg.engram_get_status() == 0
+        for name in ("idx", "state", "e", "out", "conv"):
+            assert torch.equal(a[name], b[name]), (step, name)
