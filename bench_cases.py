@@ -18,8 +18,9 @@ without the rest of the layer's inputs on the device.
 `fused` runs engram_forward with table = NULL on random gathered rows, i.e.
 the two tensor-core passes; `gather` gathers from a table of --rows rows per
 head; `hash` runs the compress + n-gram + hash kernel; `decode` runs whole
-decode steps (hash with rolling n-gram state, then engram_forward with the
-table and the conv state) for --tokens sequences of one token each;
+decode steps (engram_decode_step: hash with the rolling n-gram state and
+gather in one kernel, then the passes with the conv state) for --tokens
+sequences of one token each;
 `tablegrad` runs the sparse table gradient (sort by row, segment sums) on
 fp32 rows of de for hash indices of Zipf(1.1) token ids; `hostgather` runs
 engram_forward_hosttable on a table in pinned host memory; `backward` runs
@@ -225,9 +226,9 @@ def main(argv=None):
         conv_state = torch.zeros((N, 1, 9 if a.dilated else 3, a.d), device=dev)
         idx = torch.empty((N, 1, a.heads), dtype=torch.int32, device=dev)
 
-        def run():
-            eg.engram_hash_indices(cfg, proj, ids, N, 1, state, idx)
-            eg.engram_forward(cfg, idx, table, e, h, Wk, Wv, cw, conv_state, out, None, N, 1, ws, nb)
+        def run():  # one decode step: hash and gather in one kernel, then the passes
+            eg.engram_decode_step(cfg, proj, ids, state, idx, table, e, h, Wk, Wv, cw, conv_state,
+                                  out, N, ws, nb)
     else:
         ids_np, keys_np = synth.host_ids_keys(synth.workload("layer27b"))
         keys = torch.from_numpy(keys_np).to(dev)
