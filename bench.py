@@ -493,10 +493,11 @@ def run_ours(args):
         import hashlib
         with open(tp) as f:
             rec = json.load(f)
-        src = os.path.join(ROOT, "hashed_gram_conditional_engram_b200", "csrc", "fusion_tc.cu")
-        with open(src, "rb") as f:
-            sha = hashlib.sha1(f.read()).hexdigest()
-        if rec.get("source_sha1_fusion_tc") == sha:
+        h_ = hashlib.sha1()
+        for rel in rec.get("source_files", []):
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h_.update(f.read())
+        if rec.get("source_files") and rec.get("source_sha1") == h_.hexdigest():
             traffic = rec.get("fused_tc_traffic_bytes_per_step")
 
     line = None
