@@ -143,11 +143,17 @@ def test_forward_bf16_multibranch_unsupported():
     assert ex.value.rc == -4
 
 
-def test_forward_bf16_decode_state():
+@pytest.mark.parametrize("B,d,K,D_h", [
+    (300, 256, 2, 32),     # more sequences than one token tile: plain narrow tiles
+    (200, 512, 2, 128),    # split units (each tile's K in two halves), ragged token tile
+    (1, 256, 4, 64),       # split units, a single sequence
+    (256, 256, 2, 256),    # split units, full token tiles, 8 K steps a half
+])
+def test_forward_bf16_decode_state(B, d, K, D_h):
     """One token per sequence, 6 steps, conv state carried across steps, against
     the oracle's decode step (and through it the sequence forward)."""
-    rng = np.random.default_rng(44)
-    B, d, K, D_h, steps = 300, 256, 2, 32, 6
+    rng = np.random.default_rng(44 + B + D_h)
+    steps = 6
     J, E = 2 * K, 2 * K * D_h
     rows = synth.primes_at_most(3001, J)
     tables = [rng.standard_normal((P, D_h)).astype(np.float32) for P in rows]
@@ -344,6 +350,8 @@ def test_forward_in_place_equals_separate_output(B, T, d, dtype):
 @pytest.mark.parametrize("dtype,B,d,K,D_h,flags", [
     ("bf16", 37, 256, 2, 32, 0),                  # narrow tensor-core tiles, ragged batch
     ("bf16", 300, 512, 4, 16, eg.CONV_DILATED),   # two token tiles, dilated conv state
+    ("bf16", 100, 512, 4, 64, 0),                 # split units (K in two halves per tile)
+    ("bf16", 256, 256, 2, 128, eg.CONV_DILATED),  # split units, dilated conv state
     ("f32", 5, 64, 2, 16, 0),                     # fp32 layer
     ("f32", 9, 64, 3, 16, 0),                     # J = 6 heads (two per hash thread)
 ])

@@ -245,15 +245,18 @@ def test_bf16_prenorm_forward_matches_oracle(B, T, d, flags):
         assert max_rel_err(kv[:, d:], ref["v"]) <= 1e-3
 
 
-@pytest.mark.parametrize("flags", [DIL, PRE, PRE | DIL | SC])
-def test_bf16_decode_matches_whole_sequences(flags):
+@pytest.mark.parametrize("flags,D_h", [
+    (DIL, 32), (PRE, 32), (PRE | DIL | SC, 32),
+    (DIL, 128), (SC, 128), (DIL | SC, 128),   # E = 512: split units (K in two halves per tile)
+])
+def test_bf16_decode_matches_whole_sequences(flags, D_h):
     """Decode steps of a bf16 layer (conv state [B, 1, 3 dil, d], the conv
     inputs of the previous steps: vt, or RMSNorm(vt) g_v with the pre-conv
     norm) against the oracle's whole-sequence forward, each step within the
     bf16 metric."""
     from tests.engram_cases import bf16_dev
-    rng = np.random.default_rng(70 + flags)
-    B, T, K, D_h, d = 24, 14, 2, 32, 256
+    rng = np.random.default_rng(70 + flags + D_h)
+    B, T, K, d = 24, 14, 2, 256
     E = 2 * K * D_h
     rows = synth.primes_at_most(1009, 2 * K)
     cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((2 * K, 3), np.uint64),
