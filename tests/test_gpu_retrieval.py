@@ -249,6 +249,43 @@ def test_gather_from_host_table_bit_exact():
     assert eg.engram_get_status() == 0
 
 
+@pytest.mark.parametrize("N,span", [
+    (2051, 5),      # every head's slots from a handful of rows: most items repeat
+    (1, 3),         # a single token
+    (777, 400),     # some repeats, ragged last warp
+])
+def test_host_table_repeats_and_invalid_slots(N, span):
+    """The host gather against the oracle when rows repeat across tokens and
+    heads, with -1 slots (zero rows, no status) mixed in; out-of-range slots
+    give zero rows and ENGRAM_STATUS_BAD_INDEX."""
+    rng = np.random.default_rng(N + span)
+    K, D_h = 4, 32
+    J = 2 * K
+    rows = synth.primes_at_most(1009, J)
+    tables = [rng.standard_normal((P, D_h)).astype(np.float32) for P in rows]
+    idx = np.stack([rng.integers(0, span, N) for _ in rows], -1).astype(np.int32)
+    idx[rng.random(idx.shape) < 0.05] = -1
+    tb = [synth.to_bf16_bits(t) for t in tables]
+    flat = np.concatenate([t.reshape(-1) for t in tb]).view(np.int16)
+    host = torch.from_numpy(flat).pin_memory()
+    cfg = eg.make_cfg(K, D_h, 256, 1, 1000, 770, eg.BF16, rows, np.ones((J, 3), np.uint64))
+    e = torch.full((N, J * D_h), 7.0, dtype=torch.bfloat16, device="cuda")
+    eg.engram_forward_hosttable(cfg, dev(idx), host.data_ptr(), N, e)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits(e), O.gather(idx, tb))
+    assert eg.engram_get_status() == 0
+    bad = idx.copy()
+    bad[0, 0] = rows[0]
+    bad[-1, J - 1] = rows[J - 1] + 5
+    eg.engram_forward_hosttable(cfg, dev(bad), host.data_ptr(), N, e)
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() & eg.STATUS_BAD_INDEX
+    ref = bad.copy()
+    ref[0, 0] = -1
+    ref[-1, J - 1] = -1
+    assert np.array_equal(bf16_bits(e), O.gather(ref, tb))
+
+
 def test_gather_from_host_table_rejects_unmapped_memory():
     cfg = eg.make_cfg(8, 160, 256, 1, 1000, 770, eg.BF16, synth.primes_at_most(3001, 16),
                       np.ones((16, 3), np.uint64))
