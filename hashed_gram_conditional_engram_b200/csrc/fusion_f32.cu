@@ -251,6 +251,7 @@ __global__ void rec_conv_dsilu_kernel(const double* __restrict__ v, const double
 //   dx = r dxh - r^3 x <dxh, x> / d, with dh^ = dz g_h g_k k^ / sqrt(d) and
 //   dk^ = dz g_h g_k h^ / sqrt(d).
 // dc (for g_v's gradient) and dz (for g_h's and g_k's) are kept when asked.
+template <int MAXC>
 __global__ void gate_bwd_kernel(const float* __restrict__ dout, const double* __restrict__ dy,
                                 const float* __restrict__ h, const double* __restrict__ k,
                                 const double* __restrict__ v, const double* __restrict__ alpha,
@@ -265,34 +266,57 @@ __global__ void gate_bwd_kernel(const float* __restrict__ dout, const double* __
   const int64_t n = wid / M;
   const int t = (int)(n % T);
   const double al = alpha[wid];
+  // MAXC > 0 (d <= 32 MAXC): this lane's features c = lane + 32 j are held in
+  // registers, their loads all issued up front; MAXC = 0: read where used
+  constexpr int R = MAXC > 0 ? MAXC : 1;
+  constexpr int JMAX = MAXC > 0 ? MAXC : 1 << 20;
+  double dout_r[R], v_r[R], g_r[R], h_r[R], k_r[R];
+  if constexpr (MAXC > 0) {
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+      const int c = lane + 32 * j;
+      dout_r[j] = c < d ? (double)dout[wid * d + c] : 0.0;
+      v_r[j] = c < d ? v[n * d + c] : 0.0;
+      h_r[j] = c < d ? (double)h[wid * d + c] : 0.0;
+      k_r[j] = c < d ? k[wid * d + c] : 0.0;
+    }
+  }
   // dc into dvt; with the pre-conv norm also <dc^, vt>
   double cv = 0.0;
-  for (int c = lane; c < d; c += 32) {
+#pragma unroll
+  for (int j = 0; j < JMAX; ++j) {
+    const int c = lane + 32 * j;
+    if (c >= d) break;
     const float* wp = var.taps(m, d, c);
     double g = 0.0;
     for (int L = 0; L <= 3; ++L) {
       const int lag = L * var.dil;
       if (t + lag < T) g = fma((double)wp[3 - L], dy[((n + lag) * M + m) * d + c], g);
     }
-    dvt[wid * d + c] = g;
+    if constexpr (MAXC > 0) g_r[j] = g; else dvt[wid * d + c] = g;
     if (dc_keep != nullptr) dc_keep[wid * d + c] = g;
     if (var.prenorm) {
       const double gvc = var.gv != nullptr ? (double)var.gv[m * d + c] : 1.0;
-      cv = fma(g * gvc, al * v[n * d + c], cv);
+      const double vc = MAXC > 0 ? v_r[MAXC > 0 ? j : 0] : v[n * d + c];
+      cv = fma(g * gvc, al * vc, cv);
     }
   }
   cv = warp_sum_d(cv);
   const double r = var.prenorm ? rc[wid] : 0.0;
   double da = 0.0;
-  for (int c = lane; c < d; c += 32) {
-    double g = dvt[wid * d + c];
+#pragma unroll
+  for (int j = 0; j < JMAX; ++j) {
+    const int c = lane + 32 * j;
+    if (c >= d) break;
+    double g = MAXC > 0 ? g_r[MAXC > 0 ? j : 0] : dvt[wid * d + c];
+    const double vc = MAXC > 0 ? v_r[MAXC > 0 ? j : 0] : v[n * d + c];
     if (var.prenorm) {
       const double gvc = var.gv != nullptr ? (double)var.gv[m * d + c] : 1.0;
-      g = r * (g * gvc) - r * r * r * (al * v[n * d + c]) * cv / d;
+      g = r * (g * gvc) - r * r * r * (al * vc) * cv / d;
     }
-    g += (double)dout[wid * d + c];
+    g += MAXC > 0 ? dout_r[MAXC > 0 ? j : 0] : (double)dout[wid * d + c];
     dvt[wid * d + c] = g;
-    da = fma(g, v[n * d + c], da);
+    da = fma(g, vc, da);
   }
   da = warp_sum_d(da);
   const double dz = da * al * (1.0 - al);
@@ -302,12 +326,17 @@ __global__ void gate_bwd_kernel(const float* __restrict__ dout, const double* __
   // <dh^, h> = dz/sqrt(d) * rk * <h g g, k>, <dk^, k> = dz/sqrt(d) * rh * <h g g, k>
   const double dot_hh = dz * isd * rk * hk;
   const double dot_kk = dz * isd * rh * hk;
-  for (int c = lane; c < d; c += 32) {
-    const double a = h[wid * d + c], b = k[wid * d + c];
+#pragma unroll
+  for (int j = 0; j < JMAX; ++j) {
+    const int c = lane + 32 * j;
+    if (c >= d) break;
+    const double a = MAXC > 0 ? h_r[MAXC > 0 ? j : 0] : (double)h[wid * d + c];
+    const double b = MAXC > 0 ? k_r[MAXC > 0 ? j : 0] : k[wid * d + c];
     const double gg = var.gg(m, d, c);
     const double dhh = dz * isd * rk * gg * b;
     const double dkh = dz * isd * rh * gg * a;
-    dh[wid * d + c] = (float)((double)dout[wid * d + c] + rh * dhh - rh * rh * rh * a * dot_hh / d);
+    const double dov = MAXC > 0 ? dout_r[MAXC > 0 ? j : 0] : (double)dout[wid * d + c];
+    dh[wid * d + c] = (float)(dov + rh * dhh - rh * rh * rh * a * dot_hh / d);
     dk[wid * d + c] = rk * dkh - rk * rk * rk * b * dot_kk / d;
   }
 }
@@ -325,29 +354,34 @@ __global__ void dv_kernel(const double* __restrict__ dvt, const double* __restri
 }
 
 // dconv_w[mc,c,i] = sum_n sum_m dy[n,m,c] c_{n-(3-i) dil}[m,c] over the
-// branches m that conv mc serves (all of them for a shared conv): tokens,
-// then branches, ascending
+// branches m that conv mc serves (all of them for a shared conv).  One warp
+// per weight: lane l takes the (token, branch) terms l, l + 32, ... (tokens
+// outer, branches inner, ascending), then a fixed butterfly, so the sum has
+// the same bits on every run.
 __global__ void dconv_kernel(const double* __restrict__ dy, const double* __restrict__ v,
                              const double* __restrict__ alpha, const double* __restrict__ rc,
                              const F32Var var, float* __restrict__ dw, int64_t N, int T, int M,
                              int d) {
   const int Mc = var.per_branch ? M : 1;
-  const int g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= Mc * d * 4) return;
-  const int i = g & 3, c = (g >> 2) % d, mc = (g >> 2) / d;
+  const int lane = threadIdx.x & 31;
+  const int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (g >= (int64_t)Mc * d * 4) return;
+  const int i = (int)(g & 3), c = (int)((g >> 2) % d), mc = (int)((g >> 2) / d);
   const int lag = (3 - i) * var.dil;
-  const int m0 = var.per_branch ? mc : 0, m1 = var.per_branch ? mc + 1 : M;
+  const int m0 = var.per_branch ? mc : 0, nm = var.per_branch ? 1 : M;
   double acc = 0.0;
-  for (int64_t n = 0; n < N; ++n) {
+  for (int64_t q = lane; q < N * nm; q += 32) {
+    const int64_t n = q / nm;
+    const int m = m0 + (int)(q - n * nm);
     if ((int)(n % T) < lag) continue;
-    for (int m = m0; m < m1; ++m)
-      acc = fma(dy[(n * M + m) * d + c], var.conv_in(alpha, v, rc, n - lag, m, M, d, c), acc);
+    acc = fma(dy[(n * M + m) * d + c], var.conv_in(alpha, v, rc, n - lag, m, M, d, c), acc);
   }
-  dw[g] = (float)acc;
+  acc = warp_sum_d(acc);
+  if (lane == 0) dw[g] = (float)acc;
 }
 
-// The learnable norm scales' gradients, one thread per (m, c), tokens in
-// ascending order:
+// The learnable norm scales' gradients, one warp per (m, c), lanes taking
+// the tokens l, l + 32, ... in ascending order, then a fixed butterfly:
 //   dg_h = sum_n dz h^ k^ g_k / sqrt(d),  dg_k = sum_n dz h^ k^ g_h / sqrt(d),
 //   dg_v = sum_n dc c^ (c^ = RMSNorm(vt), with the pre-conv norm).
 __global__ void dscale_kernel(const float* __restrict__ h, const double* __restrict__ k,
@@ -356,28 +390,37 @@ __global__ void dscale_kernel(const float* __restrict__ h, const double* __restr
                               const double* __restrict__ dz, const double* __restrict__ dc,
                               const F32Var var, float* __restrict__ dgh, float* __restrict__ dgk,
                               float* __restrict__ dgv, int64_t N, int M, int d) {
-  const int g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= M * d) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (gw >= (int64_t)M * d) return;
+  const int g = (int)gw;
   const int m = g / d, c = g % d;
   const double isd = 1.0 / sqrt((double)d);
   double ah = 0.0, ak = 0.0, avv = 0.0;
-  for (int64_t n = 0; n < N; ++n) {
+  for (int64_t n = lane; n < N; n += 32) {
     const int64_t w = n * M + m;
     const double hk = (double)h[w * d + c] * sums[3 * w] * k[w * d + c] * sums[3 * w + 1];
     ah = fma(dz[w] * hk, (double)var.gk[g] * isd, ah);
     ak = fma(dz[w] * hk, (double)var.gh[g] * isd, ak);
     if (var.prenorm) avv = fma(dc[w * d + c], alpha[w] * v[n * d + c] * rc[w], avv);
   }
+  ah = warp_sum_d(ah);
+  ak = warp_sum_d(ak);
+  avv = warp_sum_d(avv);
+  if (lane != 0) return;
   dgh[g] = (float)ah;
   dgk[g] = (float)ak;
   if (var.prenorm) dgv[g] = (float)avv;
 }
 
-// dWk[m,c,i] = sum_n dk[n,m,c] e[n,i]; dWv[c,i] = sum_n dv[n,c] e[n,i]
+// dWk[m,c,i] = sum_n dk[n,m,c] e[n,i]; dWv[c,i] = sum_n dv[n,c] e[n,i]: one
+// warp per weight, lanes taking the tokens l, l + 32, ..., then a fixed
+// butterfly
 __global__ void dweight_kernel(const double* __restrict__ dk, const double* __restrict__ dv,
                                const float* __restrict__ e, float* __restrict__ dWk,
                                float* __restrict__ dWv, int64_t N, int M, int d, int E) {
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t total = (int64_t)(M + 1) * d * E;
   if (g >= total) return;
   const int i = (int)(g % E);
@@ -385,28 +428,40 @@ __global__ void dweight_kernel(const double* __restrict__ dk, const double* __re
   const int m = (int)(g / ((int64_t)E * d));
   double acc = 0.0;
   if (m < M) {
-    for (int64_t n = 0; n < N; ++n) acc = fma(dk[(n * M + m) * d + c], (double)e[n * E + i], acc);
-    dWk[g] = (float)acc;
+    for (int64_t n = lane; n < N; n += 32)
+      acc = fma(dk[(n * M + m) * d + c], (double)e[n * E + i], acc);
   } else {
-    for (int64_t n = 0; n < N; ++n) acc = fma(dv[n * d + c], (double)e[n * E + i], acc);
-    dWv[(int64_t)c * E + i] = (float)acc;
+    for (int64_t n = lane; n < N; n += 32) acc = fma(dv[n * d + c], (double)e[n * E + i], acc);
   }
+  acc = warp_sum_d(acc);
+  if (lane != 0) return;
+  if (m < M)
+    dWk[g] = (float)acc;
+  else
+    dWv[(int64_t)c * E + i] = (float)acc;
 }
 
-// de[n,i] = sum_m sum_c Wk[m,c,i] dk[n,m,c] + sum_c Wv[c,i] dv[n,c]
+// de[n,i] = sum_m sum_c Wk[m,c,i] dk[n,m,c] + sum_c Wv[c,i] dv[n,c]: one warp
+// per element, lanes taking the terms l, l + 32, ... of the (m, c) then c
+// sequence, then a fixed butterfly
 __global__ void de_kernel(const double* __restrict__ dk, const double* __restrict__ dv,
                           const float* __restrict__ Wk, const float* __restrict__ Wv,
                           float* __restrict__ de, int64_t N, int M, int d, int E) {
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (g >= N * E) return;
   const int i = (int)(g % E);
   const int64_t n = g / E;
+  const int Md = M * d;
   double acc = 0.0;
-  for (int m = 0; m < M; ++m)
-    for (int c = 0; c < d; ++c)
-      acc = fma((double)Wk[((int64_t)m * d + c) * E + i], dk[(n * M + m) * d + c], acc);
-  for (int c = 0; c < d; ++c) acc = fma((double)Wv[(int64_t)c * E + i], dv[n * d + c], acc);
-  de[g] = (float)acc;
+  for (int q = lane; q < Md + d; q += 32) {
+    if (q < Md)  // q = m d + c
+      acc = fma((double)Wk[(int64_t)q * E + i], dk[n * Md + q], acc);
+    else
+      acc = fma((double)Wv[(int64_t)(q - Md) * E + i], dv[n * d + (q - Md)], acc);
+  }
+  acc = warp_sum_d(acc);
+  if (lane == 0) de[g] = (float)acc;
 }
 
 inline unsigned blocks_for(int64_t threads_total, int per_block) {
@@ -545,17 +600,23 @@ int launch_backward_f32(const float* e, const float* h, const float* Wk, const f
                                                               w.rc, N * M, M, d);
     rec_conv_dsilu_kernel<<<blocks_for(N * M * d, tb), tb, 0, s>>>(w.v, w.alpha, w.rc, var, dout,
                                                                    w.dy, N, T, M, d);
-    gate_bwd_kernel<<<blocks_for(N * M * 32, tb), tb, 0, s>>>(
-        dout, w.dy, h, w.k, w.v, w.alpha, w.sums, w.rc, var, w.dvt, scales ? w.dc : nullptr,
-        scales ? w.dz : nullptr, dh, w.dk, N, T, M, d);
+    // small d: each lane's features in registers, their loads issued together
+    if (d <= 128)
+      gate_bwd_kernel<4><<<blocks_for(N * M * 32, tb), tb, 0, s>>>(
+          dout, w.dy, h, w.k, w.v, w.alpha, w.sums, w.rc, var, w.dvt, scales ? w.dc : nullptr,
+          scales ? w.dz : nullptr, dh, w.dk, N, T, M, d);
+    else
+      gate_bwd_kernel<0><<<blocks_for(N * M * 32, tb), tb, 0, s>>>(
+          dout, w.dy, h, w.k, w.v, w.alpha, w.sums, w.rc, var, w.dvt, scales ? w.dc : nullptr,
+          scales ? w.dz : nullptr, dh, w.dk, N, T, M, d);
     dv_kernel<<<blocks_for(N * d, tb), tb, 0, s>>>(w.dvt, w.alpha, w.dv, N, M, d);
   }
   const int Mc = var.per_branch ? M : 1;
-  dconv_kernel<<<blocks_for((int64_t)Mc * d * 4, tb), tb, 0, s>>>(w.dy, w.v, w.alpha, w.rc, var,
-                                                                  dparams, N, T, M, d);
+  dconv_kernel<<<blocks_for((int64_t)Mc * d * 4 * 32, tb), tb, 0, s>>>(
+      w.dy, w.v, w.alpha, w.rc, var, dparams, N, T, M, d);
   if (scales) {
     if (N > 0) {
-      dscale_kernel<<<blocks_for((int64_t)M * d, tb), tb, 0, s>>>(
+      dscale_kernel<<<blocks_for((int64_t)M * d * 32, tb), tb, 0, s>>>(
           h, w.k, w.v, w.alpha, w.sums, w.rc, w.dz, w.dc, var, const_cast<float*>(dvar.gh),
           const_cast<float*>(dvar.gk), const_cast<float*>(dvar.gv), N, M, d);
     } else {  // no tokens: zero gradients
@@ -564,10 +625,10 @@ int launch_backward_f32(const float* e, const float* h, const float* Wk, const f
       if (rc) return rc;
     }
   }
-  dweight_kernel<<<blocks_for((int64_t)(M + 1) * d * E, tb), tb, 0, s>>>(w.dk, w.dv, e, dWk, dWv,
-                                                                         N, M, d, E);
+  dweight_kernel<<<blocks_for((int64_t)(M + 1) * d * E * 32, tb), tb, 0, s>>>(
+      w.dk, w.dv, e, dWk, dWv, N, M, d, E);
   if (N > 0)
-    de_kernel<<<blocks_for(N * E, tb), tb, 0, s>>>(w.dk, w.dv, Wk, Wv, de, N, M, d, E);
+    de_kernel<<<blocks_for(N * E * 32, tb), tb, 0, s>>>(w.dk, w.dv, Wk, Wv, de, N, M, d, E);
   return ck(cudaGetLastError());
 }
 

@@ -532,7 +532,8 @@ __global__ void __launch_bounds__(TG_LONG_THREADS) tg_long_reduce_kernel(
 
 // The whole table gradient in one block for up to TG_SMALL_MAX items (a
 // short sequence, a training step on a small batch): the items' (row id,
-// item) keys are sorted in shared memory by a bitonic network (the item index
+// item) keys are sorted in shared memory (by rank counting up to TG_RANK_MAX
+// items, else by a bitonic network; the item index
 // in the low bits keeps equal rows in ascending token order, as the stable
 // radix sort does), segment heads are counted by a block scan, and each
 // (row, 4 dimensions) sums its segment in that order from +0.  The same sums
@@ -540,6 +541,7 @@ __global__ void __launch_bounds__(TG_LONG_THREADS) tg_long_reduce_kernel(
 constexpr int TG_SMALL_MAX = 2048;   // 24 KB of static shared memory
 constexpr int TG_SMALL_THREADS = 1024;
 constexpr int TG_ITEM_BITS = 12;  // item index < 2^12
+constexpr int TG_RANK_MAX = 512;  // up to here, ranks by counting instead of the sorting network
 
 __global__ void __launch_bounds__(TG_SMALL_THREADS) tg_small_kernel(
     const __grid_constant__ HeadParams hp, const int32_t* __restrict__ idx, int n,
@@ -563,20 +565,35 @@ __global__ void __launch_bounds__(TG_SMALL_THREADS) tg_small_kernel(
     sk[i] = key;
   }
   __syncthreads();
-  for (int k = 2; k <= np2; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = tid; i < np2; i += TG_SMALL_THREADS) {
-        const int ixj = i ^ jj;
-        if (ixj > i) {
-          const uint64_t a = sk[i], b = sk[ixj];
-          const bool up = (i & k) == 0;
-          if ((a > b) == up) {
-            sk[i] = b;
-            sk[ixj] = a;
+  if (n <= TG_RANK_MAX) {
+    // few items: each key's sorted position is the number of smaller keys
+    // (keys are distinct: the item index is in their low bits); one pass
+    // instead of the network's log2(n) (log2(n) + 1) / 2 barrier stages
+    uint64_t key = 0;
+    int rank = 0;
+    if (tid < n) {
+      key = sk[tid];
+      for (int j = 0; j < n; ++j) rank += sk[j] < key ? 1 : 0;
+    }
+    __syncthreads();
+    if (tid < n) sk[rank] = key;
+    __syncthreads();
+  } else {
+    for (int k = 2; k <= np2; k <<= 1) {
+      for (int jj = k >> 1; jj > 0; jj >>= 1) {
+        for (int i = tid; i < np2; i += TG_SMALL_THREADS) {
+          const int ixj = i ^ jj;
+          if (ixj > i) {
+            const uint64_t a = sk[i], b = sk[ixj];
+            const bool up = (i & k) == 0;
+            if ((a > b) == up) {
+              sk[i] = b;
+              sk[ixj] = a;
+            }
           }
         }
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
   // segment heads over sorted positions, 4 consecutive positions per thread
@@ -636,8 +653,18 @@ __global__ void __launch_bounds__(TG_SMALL_THREADS) tg_small_kernel(
   for (int g = tid; g < all * D4; g += TG_SMALL_THREADS) {
     const int u = g / D4, c = g - u * D4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p = seg[u]; p < seg[u + 1]; ++p)
-      add4(acc, __ldg(de + (int64_t)(sk[p] & ITEM_MASK) * D4 + c));
+    const int pe = seg[u + 1];
+    // up to 8 of the segment's rows are loaded before any is added, then
+    // added in ascending order (the same sums, without a round trip each)
+    for (int p = seg[u]; p < pe; p += 8) {
+      float4 a[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (p + q < pe) a[q] = __ldg(de + (int64_t)(sk[p + q] & ITEM_MASK) * D4 + c);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (p + q < pe) add4(acc, a[q]);
+    }
     rows_out[g] = acc;
   }
 }
