@@ -14,6 +14,7 @@ without the rest of the layer's inputs on the device.
     python bench_cases.py backward [...]
     python bench_cases.py hostcache \
         --tokens 8192 --seq 2048 --dh 160 --rows 1000003 [--cache-rows 1048576]
+    python bench_cases.py tiny [--reps 3]
 
 `fused` runs engram_forward with table = NULL on random gathered rows, i.e.
 the two tensor-core passes; `gather` gathers from a table of --rows rows per
@@ -21,7 +22,8 @@ head; `hash` runs the compress + n-gram + hash kernel; `decode` runs whole
 decode steps (engram_decode_step: hash with the rolling n-gram state and
 gather in one kernel, then the passes with the conv state) for --tokens
 sequences of one token each;
-`tablegrad` runs the sparse table gradient (sort by row, segment sums) on
+`tiny` runs the tiny fp32 layer's step (hash, forward, backward; its own
+fixed shape); `tablegrad` runs the sparse table gradient (sort by row, segment sums) on
 fp32 rows of de for hash indices of Zipf(1.1) token ids; `hostgather` runs
 engram_forward_hosttable on a table in pinned host memory; `backward` runs
 the bf16 engram_backward (column walk, row kernel, GEMMs, sparse table
@@ -45,7 +47,7 @@ from hashed_gram_conditional_engram_b200 import synth
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("kernel", choices=["fused", "gather", "hash", "decode", "tablegrad",
-                                       "hostgather", "backward", "hostcache"])
+                                       "hostgather", "backward", "hostcache", "tiny"])
     ap.add_argument("--tokens", type=int, default=32768)
     ap.add_argument("--seq", type=int, default=4096)
     ap.add_argument("--d", type=int, default=2560)
@@ -81,7 +83,9 @@ def main(argv=None):
     g.manual_seed(7)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    if a.kernel == "fused":
+    if a.kernel == "tiny":
+        run = _tiny_step(dev)
+    elif a.kernel == "fused":
         e = (torch.randn((N, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
         h = torch.randn((N, a.d), generator=g, device=dev).to(torch.bfloat16)
         Wk = (torch.randn((a.d, E), generator=g, device=dev) * 0.02).to(torch.bfloat16)
@@ -254,6 +258,45 @@ def main(argv=None):
     st = eg.engram_get_status()
     if st != 0:
         raise SystemExit(f"device status word {st}")
+
+
+def _tiny_step(dev):
+    """The tiny fp32 layer (1 x 64 tokens, d 64, 4 heads x 16 dims): hash,
+    forward with the gather, backward with the sparse table gradient."""
+    w = synth.workload("tiny")
+    inp = synth.host_inputs(w)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+    keys = t(inp["keys"])
+    proj = torch.empty(w.V, dtype=torch.int32, device=dev)
+    vb = eg.engram_workspace_size(None, eg.WS_VOCAB, w.V)
+    V_c = eg.engram_build_vocab_proj(keys, w.V, proj,
+                                     torch.empty(vb, dtype=torch.uint8, device=dev), vb)
+    cfg = eg.make_cfg(w.K, w.D_h, w.d, w.M, w.V, V_c, eg.F32, w.rows, inp["mult"])
+    N, E = w.N, w.E
+    ids, table = t(inp["ids"]), t(np.concatenate([x.reshape(-1) for x in inp["tables"]]))
+    h, Wk, Wv, dout = t(inp["h"]), t(inp["Wk"]), t(inp["Wv"]), t(inp["dout"])
+    cw = t(np.asarray(inp["conv_w"], np.float32).reshape(-1))
+    idx = torch.empty((w.B, w.T, w.J), dtype=torch.int32, device=dev)
+    e = torch.empty((N, E), device=dev)
+    out = torch.empty((N, w.M, w.d), device=dev)
+    saved = torch.empty(eg.engram_saved_size(cfg, N), dtype=torch.uint8, device=dev)
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, N)
+    fws = torch.empty(fb, dtype=torch.uint8, device=dev)
+    bb = eg.engram_workspace_size(cfg, eg.WS_BACKWARD, N)
+    bws = torch.empty(bb, dtype=torch.uint8, device=dev)
+    dh = torch.empty((N, w.M, w.d), device=dev)
+    dWk, dWv = torch.empty((w.M, w.d, E), device=dev), torch.empty((w.d, E), device=dev)
+    dcw = torch.empty(eg.engram_param_floats(cfg), device=dev)
+    keys_out = torch.empty(N * w.J, dtype=torch.int64, device=dev)
+    rows_out = torch.empty((N * w.J, w.D_h), device=dev)
+    nu = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def run():
+        eg.engram_hash_indices(cfg, proj, ids, w.B, w.T, None, idx)
+        eg.engram_forward(cfg, idx, table, e, h, Wk, Wv, cw, None, out, saved, w.B, w.T, fws, fb)
+        eg.engram_backward(cfg, idx, e, h, Wk, Wv, cw, saved, dout, dh, dWk, dWv, dcw, None,
+                           keys_out, rows_out, nu, w.B, w.T, bws, bb)
+    return run
 
 
 if __name__ == "__main__":
