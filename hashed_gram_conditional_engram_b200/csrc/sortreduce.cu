@@ -800,9 +800,8 @@ int launch_hot_rows(const HeadParams& hp, const int32_t* idx, int64_t n_tok, int
 // ------------------------------------------------- table gradient without allocation
 //
 // For callers that cannot allocate device memory themselves (a host that
-// hands this library a fixed pool, code running inside a CUDA graph capture
-// where allocation calls are not allowed, or a plugin whose host framework
-// owns every allocation), the sparse table gradient can run on a scratch
+// hands this library a fixed pool, or a plugin whose host framework owns
+// every allocation), the sparse table gradient can run on a scratch
 // array that is part of the library image: the GPU reserves it when the
 // library's device code is loaded and keeps it until the process exits.  It
 // holds the sort buffers for up to ENGRAM_NOALLOC_MAX_ITEMS (token, head)

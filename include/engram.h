@@ -305,8 +305,7 @@ int engram_table_grad(const engram_cfg_t* cfg, const int32_t* idx, const float* 
 /*
  * engram_table_grad without a workspace argument, for callers that cannot
  * allocate device memory: a host framework that owns every allocation and
- * hands out none for scratch, code recording a CUDA graph where allocation
- * calls are not allowed, or a runtime with a fixed memory pool.  (The pages
+ * hands out none for scratch, or a runtime with a fixed memory pool.  (The pages
  * have no counterpart: this is an interface variant, not part of the method.)
  *   Same arguments, outputs and results as engram_table_grad, minus ws.
  *   The sort buffers live in a device array built into the library, sized
@@ -314,8 +313,7 @@ int engram_table_grad(const engram_cfg_t* cfg, const int32_t* idx, const float* 
  *   4.8 MB, held on every GPU that loads the library until the process
  *   exits).  Larger inputs return ENGRAM_ERR_TOO_LARGE and launch nothing.
  *   The call allocates nothing.  Its first call on a device looks up the
- *   array's device address (cudaGetSymbolAddress); make that first call
- *   before capturing a stream into a graph.
+ *   array's device address (cudaGetSymbolAddress).
  *   All calls share the array: calls that overlap on the GPU (other streams,
  *   other host threads) race and must be serialised by the caller.
  *   The looked-up address is kept for the life of the process: after a

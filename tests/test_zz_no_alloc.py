@@ -1,6 +1,6 @@
 """engram_table_grad_noalloc: the sparse table gradient for callers that cannot
-allocate device memory (a host framework that owns every allocation, code
-recording a CUDA graph where allocation calls are not allowed).  It sorts in a
+allocate device memory (a host framework that owns every allocation, or a
+runtime with a fixed memory pool).  It sorts in a
 scratch array built into the library instead of a caller workspace, so its
 results must equal those of engram_table_grad on the same inputs, bit for bit
 (the reduction is deterministic).  Two calls in a row check that the second
