@@ -500,33 +500,72 @@ __global__ void tg_long_list_kernel(const int32_t* __restrict__ seg_start,
   if (seg_start[u + 1] - seg_start[u] > TG_LONG) list[atomicAdd(count, 1)] = u;
 }
 
-// One block per long row at a time: the block loads TG_LONG items' rows of de
-// into shared memory together (all their loads in flight at once), then one
-// thread per 4 dimensions adds them in order; the next chunk follows.  The
-// same fp32 sums as tg_reduce_kernel, bit for bit.
+// One block per long row at a time, its segment in chunks of TG_LONG items:
+// the block copies a chunk's rows of de into shared memory (cp.async, 16
+// bytes a thread at a time), BUFS chunks in flight, then one thread per 4
+// dimensions adds the chunk's rows in order while the next chunks land.  A
+// chunk's item ids are read one chunk further ahead, so no copy waits on an
+// id load.  The same fp32 sums as tg_reduce_kernel, bit for bit.
 constexpr int TG_LONG_THREADS = 256;
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(smem)),
+               "l"(gmem)
+               : "memory");
+}
+template <int BUFS>
 __global__ void __launch_bounds__(TG_LONG_THREADS) tg_long_reduce_kernel(
     const int32_t* __restrict__ seg_start, const uint32_t* __restrict__ vals,
     const float4* __restrict__ de, const int32_t* __restrict__ list,
     const int32_t* __restrict__ count, int D4, float4* __restrict__ rows) {
-  extern __shared__ float4 chunk[];  // [TG_LONG][D4]
+  extern __shared__ float4 chunk[];               // [BUFS][TG_LONG * D4]
+  __shared__ uint32_t ids[BUFS + 1][TG_LONG];     // item ids of the chunks ahead
   const int n = *count;
+  const int tid = threadIdx.x;
+  const int CH = TG_LONG * D4;
   for (int li = blockIdx.x; li < n; li += gridDim.x) {
     const int32_t u = list[li];
     const int32_t b = seg_start[u], e = seg_start[u + 1];
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int32_t p0 = b; p0 < e; p0 += TG_LONG) {
-      const int m = e - p0 < TG_LONG ? e - p0 : TG_LONG;
-      for (int i = threadIdx.x; i < m * D4; i += TG_LONG_THREADS) {
-        const int it = i / D4, c = i - it * D4;
-        chunk[i] = __ldg(de + (int64_t)__ldg(vals + p0 + it) * D4 + c);
+    const int nch = (int)((e - b + TG_LONG - 1) / TG_LONG);
+    auto load_ids = [&](int q) {  // chunk q's item ids -> ids[q % (BUFS + 1)]
+      const int32_t p = b + q * TG_LONG + tid;
+      if (q < nch && tid < TG_LONG && p < e) ids[q % (BUFS + 1)][tid] = __ldg(vals + p);
+    };
+    auto issue = [&](int q) {  // chunk q's rows -> buffer q % BUFS; one group per chunk
+      if (q < nch) {
+        const int32_t p0 = b + q * TG_LONG;
+        const int m = e - p0 < TG_LONG ? (int)(e - p0) : TG_LONG;
+        float4* buf = chunk + (q % BUFS) * CH;
+        const uint32_t* id = ids[q % (BUFS + 1)];
+        for (int i = tid; i < m * D4; i += TG_LONG_THREADS) {
+          const int it = i / D4, c = i - it * D4;
+          cp_async16(buf + i, de + (int64_t)id[it] * D4 + c);
+        }
       }
-      __syncthreads();
-      if (threadIdx.x < D4)
-        for (int it = 0; it < m; ++it) add4(acc, chunk[it * D4 + threadIdx.x]);
-      __syncthreads();
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    for (int q = 0; q < BUFS; ++q) load_ids(q);
+    __syncthreads();
+    for (int q = 0; q < BUFS - 1; ++q) issue(q);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < nch; ++q) {
+      // buffer (q - 1) % BUFS was released at the end of the previous chunk;
+      // ids of chunk q + BUFS - 1 were made visible by that barrier too
+      issue(q + BUFS - 1);
+      load_ids(q + BUFS);  // the slot of chunk q - 1's ids, issued already
+      asm volatile("cp.async.wait_group %0;" ::"n"(BUFS - 1) : "memory");
+      __syncthreads();  // chunk q has landed for every thread
+      if (tid < D4) {
+        const int32_t p0 = b + q * TG_LONG;
+        const int m = e - p0 < TG_LONG ? (int)(e - p0) : TG_LONG;
+        const float4* buf = chunk + (q % BUFS) * CH + tid;
+        for (int it = 0; it < m; ++it) add4(acc, buf[it * D4]);
+      }
+      __syncthreads();  // buffer q % BUFS is free
     }
-    if (threadIdx.x < D4) rows[(int64_t)u * D4 + threadIdx.x] = acc;
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    if (tid < D4) rows[(int64_t)u * D4 + tid] = acc;
   }
 }
 
@@ -709,16 +748,25 @@ int launch_table_grad(const HeadParams& hp, const int32_t* idx, const float* de,
   int32_t* long_count = w.scal + 2;
   if ((rc = ck(cudaMemsetAsync(long_count, 0, sizeof(int32_t), s)))) return rc;
   tg_long_list_kernel<<<nb(n), 256, 0, s>>>(w.c, n_unique, w.a, long_count);
-  const size_t long_smem = (size_t)TG_LONG * D4 * sizeof(float4);
-  if (D4 > TG_LONG_THREADS || long_smem > 227 * 1024) return ENGRAM_ERR_UNSUPPORTED;
-  if (long_smem > 48 * 1024 &&
-      (rc = ck(cudaFuncSetAttribute(tg_long_reduce_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)long_smem))))
-    return rc;
-  tg_long_reduce_kernel<<<(unsigned)sms, TG_LONG_THREADS, long_smem, s>>>(
-      w.c, v, reinterpret_cast<const float4*>(de), w.a, long_count, D4,
-      reinterpret_cast<float4*>(rows_out));
-  return ck(cudaGetLastError());
+  // as many chunk buffers (4, 2 or 1) as 220 KB of shared memory holds
+  const size_t chunk_bytes = (size_t)TG_LONG * D4 * sizeof(float4);
+  if (D4 > TG_LONG_THREADS || chunk_bytes > 220 * 1024) return ENGRAM_ERR_UNSUPPORTED;
+  const int bufs = 4 * chunk_bytes <= 220 * 1024 ? 4 : 2 * chunk_bytes <= 220 * 1024 ? 2 : 1;
+  const size_t long_smem = bufs * chunk_bytes;
+  const float4* de4 = reinterpret_cast<const float4*>(de);
+  float4* rows4 = reinterpret_cast<float4*>(rows_out);
+  auto run_long = [&](auto kern) -> int {
+    if (long_smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)long_smem) != cudaSuccess)
+      return (int)ENGRAM_ERR_CUDA;
+    kern<<<(unsigned)sms, TG_LONG_THREADS, long_smem, s>>>(w.c, v, de4, w.a, long_count, D4,
+                                                           rows4);
+    return ck(cudaGetLastError());
+  };
+  return bufs == 4   ? run_long(tg_long_reduce_kernel<4>)
+         : bufs == 2 ? run_long(tg_long_reduce_kernel<2>)
+                     : run_long(tg_long_reduce_kernel<1>);
 }
 
 size_t vocab_ws_bytes(int64_t V) { return sort_ws_bytes(V); }
