@@ -52,20 +52,40 @@ __global__ void __launch_bounds__(SORT_THREADS) radix_hist_kernel(const uint64_t
     hist[(int64_t)i * gridDim.x + blockIdx.x] = cnt[i];
 }
 
+__device__ __forceinline__ int32_t block_scan(int32_t t, int32_t* excl);
+
 // Stable scatter: item order inside the tile is (warp, chunk, lane); each
-// item's destination = start of its digit for this block + items of the same
-// digit before it in that order.
+// item's destination = start of its digit (the exclusive scan of the digit
+// totals dtot, formed here) + the digit's items in earlier blocks (offsets,
+// per digit) + items of the same digit before it in that order.
 __global__ void __launch_bounds__(SORT_THREADS) radix_scatter_kernel(
     const uint64_t* __restrict__ keys_in, const uint32_t* __restrict__ vals_in, int64_t n,
-    int shift, int radix, const int32_t* __restrict__ offsets, uint64_t* __restrict__ keys_out,
-    uint32_t* __restrict__ vals_out) {
+    int shift, int radix, const int32_t* __restrict__ offsets, const int32_t* __restrict__ dtot,
+    uint64_t* __restrict__ keys_out, uint32_t* __restrict__ vals_out) {
   __shared__ int32_t wcnt[SORT_WARPS][RADIX_MAX];
   __shared__ int32_t boff[RADIX_MAX];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int w = 0; w < SORT_WARPS; ++w)
     for (int i = threadIdx.x; i < radix; i += SORT_THREADS) wcnt[w][i] = 0;
-  for (int i = threadIdx.x; i < radix; i += SORT_THREADS)
-    boff[i] = offsets[(int64_t)i * gridDim.x + blockIdx.x];
+  {
+    // digits 4 t .. 4 t + 3 of this thread (radix <= 4 * SORT_THREADS)
+    constexpr int PD = RADIX_MAX / SORT_THREADS;
+    int32_t tv[PD], sum = 0;
+#pragma unroll
+    for (int q = 0; q < PD; ++q) {
+      const int dq = threadIdx.x * PD + q;
+      tv[q] = dq < radix ? dtot[dq] : 0;
+      sum += tv[q];
+    }
+    int32_t run;
+    block_scan(sum, &run);
+#pragma unroll
+    for (int q = 0; q < PD; ++q) {
+      const int dq = threadIdx.x * PD + q;
+      if (dq < radix) boff[dq] = run + offsets[(int64_t)dq * gridDim.x + blockIdx.x];
+      run += tv[q];
+    }
+  }
   __syncthreads();
 
   const int64_t wbase = (int64_t)blockIdx.x * TILE + (int64_t)warp * 32 * CHUNKS_PER_WARP;
@@ -168,6 +188,26 @@ __device__ __forceinline__ int32_t block_scan(int32_t t, int32_t* excl) {
   return all;
 }
 
+// The per-block counts of one digit (hist[d * nblocks + b], b ascending)
+// replaced by their exclusive prefix, one block per digit; the digit's total
+// into dtot[d].  Each thread takes a run of consecutive blocks.
+__global__ void __launch_bounds__(SCAN_THREADS) radix_digit_scan_kernel(int32_t* hist, int nblocks,
+                                                                        int32_t* dtot) {
+  int32_t* h = hist + (int64_t)blockIdx.x * nblocks;
+  const int per = (nblocks + SCAN_THREADS - 1) / SCAN_THREADS;
+  const int lo = threadIdx.x * per, hi = lo + per < nblocks ? lo + per : nblocks;
+  int32_t s = 0;
+  for (int b = lo; b < hi; ++b) s += h[b];
+  int32_t run;
+  const int32_t all = block_scan(s, &run);
+  for (int b = lo; b < hi; ++b) {
+    const int32_t t = h[b];
+    h[b] = run;
+    run += t;
+  }
+  if (threadIdx.x == 0) dtot[blockIdx.x] = all;
+}
+
 __global__ void __launch_bounds__(SCAN_THREADS) scan_reduce_kernel(const int32_t* x, int64_t n,
                                                                    int64_t chunk,
                                                                    int32_t* bsum) {
@@ -252,6 +292,8 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_apply_kernel(const int32_t*
 }
 
 constexpr size_t scan_ws_bytes() { return up256((SCAN_MAX_BLOCKS + 1) * 4); }
+static_assert(SCAN_THREADS == SORT_THREADS, "the scatter kernel uses block_scan");
+static_assert(RADIX_MAX <= SCAN_MAX_BLOCKS, "digit totals fit the scan scratch");
 
 // x and y 16-byte aligned; bsum: scan_ws_bytes() of workspace.
 int launch_scan(const int32_t* x, int32_t* y, int64_t n, int32_t* total, int32_t* bsum,
@@ -272,12 +314,12 @@ int radix_sort_pairs(uint64_t*& keys, uint32_t*& vals, uint64_t* keys_alt, uint3
   const int passes = (key_bits + RADIX_MAX_BITS - 1) / RADIX_MAX_BITS;
   const int bits = (key_bits + passes - 1) / passes;
   const int radix = 1 << bits;
+  // bsum holds the digit totals (radix <= SCAN_MAX_BLOCKS ints)
   for (int shift = 0; shift < key_bits; shift += bits) {
     radix_hist_kernel<<<(unsigned)nblocks, SORT_THREADS, 0, s>>>(keys, n, shift, radix, hist);
-    const int rc = launch_scan(hist, hist, (int64_t)radix * nblocks, nullptr, bsum, s);
-    if (rc) return rc;
-    radix_scatter_kernel<<<(unsigned)nblocks, SORT_THREADS, 0, s>>>(keys, vals, n, shift, radix,
-                                                                    hist, keys_alt, vals_alt);
+    radix_digit_scan_kernel<<<(unsigned)radix, SCAN_THREADS, 0, s>>>(hist, (int)nblocks, bsum);
+    radix_scatter_kernel<<<(unsigned)nblocks, SORT_THREADS, 0, s>>>(
+        keys, vals, n, shift, radix, hist, bsum, keys_alt, vals_alt);
     uint64_t* tk = keys;
     keys = keys_alt;
     keys_alt = tk;
