@@ -27,7 +27,8 @@
  *   - All device pointers are raw CUDA device addresses, 16-byte aligned.
  *     Host pointers are named so.  The caller owns every buffer; the library
  *     allocates no device memory and keeps no state besides one device status
- *     word per device.
+ *     word per device (and the built-in scratch array that
+ *     engram_table_grad_noalloc sorts in).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls are asynchronous and never synchronise, except
  *     engram_build_vocab_proj (returns V_c on the host) and engram_get_status.
@@ -117,14 +118,15 @@ enum {
  *            them: 8 * n_tok * d_model more bytes of `saved` for one GEMM
  *            less in the backward.
  *            ENGRAM_CONV_DILATED, ENGRAM_CONV_PRENORM, ENGRAM_CONV_PER_BRANCH,
- *            ENGRAM_NORM_SCALES: formulation variants (fp32 layers: any
- *            combination on fp32 and on bf16 layers).
+ *            ENGRAM_NORM_SCALES: formulation variants, in any combination,
+ *            on fp32 and on bf16 layers.
  *            z = <RMSNorm(h) g_h, RMSNorm(k) g_k> / sqrt(d),
  *            vt = alpha v, c = RMSNorm(vt) g_v (PRENORM) or vt,
  *            y_t = sum_i w[:, i] c_{t-(3-i) dil} (dil 3 with DILATED, else 1),
  *            out = h + vt + SiLU(y); each branch m has its own w (PER_BRANCH)
  *            and its own g_h, g_k, g_v (NORM_SCALES).  Their parameters form
  *            the conv_w block (engram_param_floats floats).
+ *            ENGRAM_TEST_STALL: see above (tests only).
  *            Any other bit is ENGRAM_ERR_INVALID_ARG.
  *   rows[j]  P_j, row count (a prime) of head j's table.  Head j's rows sit
  *            in one packed table after those of heads 0..j-1.
@@ -140,7 +142,7 @@ typedef struct engram_cfg {
   int32_t V_raw;
   int32_t V_c;
   int32_t dtype;
-  int32_t flags; /* 0, or ENGRAM_SAVE_KV */
+  int32_t flags; /* ENGRAM_SAVE_KV, the variant flags, ENGRAM_TEST_STALL */
   int64_t rows[ENGRAM_MAX_HEADS];
   uint64_t mult[ENGRAM_MAX_HEADS][3];
 } engram_cfg_t;
