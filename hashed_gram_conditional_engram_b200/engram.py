@@ -23,7 +23,7 @@ F32, BF16 = 0, 1
 WS_VOCAB, WS_FORWARD, WS_BACKWARD, WS_TABLE_GRAD = 0, 1, 2, 3
 WS_HOSTCACHE_RANK, WS_HOSTCACHE_GATHER = 4, 5
 SAVE_KV = 1  # EngramCfg.flags
-# formulation variants (fp32 layers)
+# formulation variants (fp32 and bf16 layers)
 CONV_DILATED, CONV_PRENORM, CONV_PER_BRANCH, NORM_SCALES = 2, 4, 8, 16
 STATUS_BAD_ID, STATUS_BAD_INDEX, STATUS_TIMEOUT = 1, 2, 4
 # test only: the call's bounded device-side waits run out (see engram.h)
