@@ -423,6 +423,27 @@ def run_ours(args):
     ms_per_step = elapsed_ms / args.steps
     value = aggregate_rate(N, ws_, args.steps, elapsed_ms)
 
+    # ---- the gather alone: back to back (the slots and whatever rows the
+    # previous call left in L2 stay warm) and with a 256 MB memset between
+    # calls (L2 flushed)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    gev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    t_warm, t_cold = [], []
+    for k in range(21):
+        flushed = k % 2 == 1
+        if flushed:
+            flush.zero_()
+        gev[0].record(stream)
+        eg.engram_gather(cfg, idx, table, N, e, stream)
+        gev[1].record(stream)
+        torch.cuda.synchronize()
+        (t_cold if flushed else t_warm).append(gev[0].elapsed_time(gev[1]))
+    del flush
+    gather_l2 = {"warm_us": float(np.median(t_warm[1:])) * 1e3,
+                 "l2_flushed_us": float(np.median(t_cold)) * 1e3,
+                 "what": "engram_gather alone, median of 10 calls each: back to back, and "
+                         "after a 256 MB memset (L2 flushed)"}
+
     # ---- end to end through the public API with host buffers.  Each step
     # uploads its ids and h from pinned host memory, runs hash + forward and
     # reads its output back.  Steps are double-buffered over three streams
@@ -530,6 +551,7 @@ def run_ours(args):
             },
             "breakdown_ms": {"hash": t_hash, "gather": t_gather, "fused_tc_passes": t_fuse},
             "gather_gbs": (N * w.J * 4 + N * w.J * w.D_h * 2 + N * w.E * 2) / (t_gather / 1e3) / 1e9,
+            "gather_alone": gather_l2,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "kernel": "engram_forward(table=NULL): tc_fused_kernel pass K, gate kernel, tc_fused_kernel pass V",
