@@ -251,17 +251,34 @@ __global__ void rec_conv_dsilu_kernel(const double* __restrict__ v, const double
 //   dx = r dxh - r^3 x <dxh, x> / d, with dh^ = dz g_h g_k k^ / sqrt(d) and
 //   dk^ = dz g_h g_k h^ / sqrt(d).
 // dc (for g_v's gradient) and dz (for g_h's and g_k's) are kept when asked.
+struct GateBwdArgs {
+  const float* dout;
+  const double *dy, *k, *v, *alpha, *sums, *rc;
+  const float* h;
+  double *dvt, *dc_keep, *dz_keep, *dk;
+  float* dh;
+  int64_t N;
+  int T, M, d;
+};
+
+// the gate backward of row wid = n M + m, by one warp
 template <int MAXC>
-__global__ void gate_bwd_kernel(const float* __restrict__ dout, const double* __restrict__ dy,
-                                const float* __restrict__ h, const double* __restrict__ k,
-                                const double* __restrict__ v, const double* __restrict__ alpha,
-                                const double* __restrict__ sums, const double* __restrict__ rc,
-                                const F32Var var, double* __restrict__ dvt, double* __restrict__ dc_keep,
-                                double* __restrict__ dz_keep, float* __restrict__ dh,
-                                double* __restrict__ dk, int64_t N, int T, int M, int d) {
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (wid >= N * M) return;
+__device__ __forceinline__ void gate_bwd_row(const GateBwdArgs& ga, const F32Var& var,
+                                             int64_t wid, int lane) {
+  const float* __restrict__ dout = ga.dout;
+  const double* __restrict__ dy = ga.dy;
+  const float* __restrict__ h = ga.h;
+  const double* __restrict__ k = ga.k;
+  const double* __restrict__ v = ga.v;
+  const double* __restrict__ alpha = ga.alpha;
+  const double* __restrict__ sums = ga.sums;
+  const double* __restrict__ rc = ga.rc;
+  double* __restrict__ dvt = ga.dvt;
+  double* __restrict__ dc_keep = ga.dc_keep;
+  double* __restrict__ dz_keep = ga.dz_keep;
+  float* __restrict__ dh = ga.dh;
+  double* __restrict__ dk = ga.dk;
+  const int T = ga.T, M = ga.M, d = ga.d;
   const int m = (int)(wid % M);
   const int64_t n = wid / M;
   const int t = (int)(n % T);
@@ -341,16 +358,24 @@ __global__ void gate_bwd_kernel(const float* __restrict__ dout, const double* __
   }
 }
 
-// dv[n,c] = sum_m alpha[n,m] dvt[n,m,c], branches in ascending order
-__global__ void dv_kernel(const double* __restrict__ dvt, const double* __restrict__ alpha,
-                          double* __restrict__ dv, int64_t N, int M, int d) {
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= N * d) return;
-  const int c = (int)(g % d);
-  const int64_t n = g / d;
-  double acc = 0.0;
-  for (int m = 0; m < M; ++m) acc = fma(alpha[n * M + m], dvt[(n * M + m) * d + c], acc);
-  dv[g] = acc;
+// A block per token: its warps take the token's M rows of the gate
+// backward, then the block forms dv[n,c] = sum_m alpha[n,m] dvt[n,m,c]
+// (branches in ascending order) from the rows just written.
+constexpr int GB_THREADS = 256;
+template <int MAXC>
+__global__ void __launch_bounds__(GB_THREADS) gate_bwd_dv_kernel(const GateBwdArgs ga,
+                                                                 const F32Var var,
+                                                                 double* __restrict__ dv) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t n = blockIdx.x;
+  const int M = ga.M, d = ga.d;
+  for (int m = warp; m < M; m += GB_THREADS / 32) gate_bwd_row<MAXC>(ga, var, n * M + m, lane);
+  __syncthreads();  // the rows' dvt are written (global memory, this block)
+  for (int c = threadIdx.x; c < d; c += GB_THREADS) {
+    double acc = 0.0;
+    for (int m = 0; m < M; ++m) acc = fma(ga.alpha[n * M + m], ga.dvt[(n * M + m) * d + c], acc);
+    dv[n * d + c] = acc;
+  }
 }
 
 // dconv_w[mc,c,i] = sum_n sum_m dy[n,m,c] c_{n-(3-i) dil}[m,c] over the
@@ -358,14 +383,12 @@ __global__ void dv_kernel(const double* __restrict__ dvt, const double* __restri
 // per weight: lane l takes the (token, branch) terms l, l + 32, ... (tokens
 // outer, branches inner, ascending), then a fixed butterfly, so the sum has
 // the same bits on every run.
-__global__ void dconv_kernel(const double* __restrict__ dy, const double* __restrict__ v,
-                             const double* __restrict__ alpha, const double* __restrict__ rc,
-                             const F32Var var, float* __restrict__ dw, int64_t N, int T, int M,
-                             int d) {
-  const int Mc = var.per_branch ? M : 1;
-  const int lane = threadIdx.x & 31;
-  const int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (g >= (int64_t)Mc * d * 4) return;
+__device__ __forceinline__ void dconv_out(const double* __restrict__ dy,
+                                          const double* __restrict__ v,
+                                          const double* __restrict__ alpha,
+                                          const double* __restrict__ rc, const F32Var& var,
+                                          float* __restrict__ dw, int64_t N, int T, int M, int d,
+                                          int64_t g, int lane) {
   const int i = (int)(g & 3), c = (int)((g >> 2) % d), mc = (int)((g >> 2) / d);
   const int lag = (3 - i) * var.dil;
   const int m0 = var.per_branch ? mc : 0, nm = var.per_branch ? 1 : M;
@@ -384,15 +407,17 @@ __global__ void dconv_kernel(const double* __restrict__ dy, const double* __rest
 // the tokens l, l + 32, ... in ascending order, then a fixed butterfly:
 //   dg_h = sum_n dz h^ k^ g_k / sqrt(d),  dg_k = sum_n dz h^ k^ g_h / sqrt(d),
 //   dg_v = sum_n dc c^ (c^ = RMSNorm(vt), with the pre-conv norm).
-__global__ void dscale_kernel(const float* __restrict__ h, const double* __restrict__ k,
-                              const double* __restrict__ v, const double* __restrict__ alpha,
-                              const double* __restrict__ sums, const double* __restrict__ rc,
-                              const double* __restrict__ dz, const double* __restrict__ dc,
-                              const F32Var var, float* __restrict__ dgh, float* __restrict__ dgk,
-                              float* __restrict__ dgv, int64_t N, int M, int d) {
-  const int lane = threadIdx.x & 31;
-  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (gw >= (int64_t)M * d) return;
+__device__ __forceinline__ void dscale_out(const float* __restrict__ h,
+                                           const double* __restrict__ k,
+                                           const double* __restrict__ v,
+                                           const double* __restrict__ alpha,
+                                           const double* __restrict__ sums,
+                                           const double* __restrict__ rc,
+                                           const double* __restrict__ dz,
+                                           const double* __restrict__ dc, const F32Var& var,
+                                           float* __restrict__ dgh, float* __restrict__ dgk,
+                                           float* __restrict__ dgv, int64_t N, int M, int d,
+                                           int64_t gw, int lane) {
   const int g = (int)gw;
   const int m = g / d, c = g % d;
   const double isd = 1.0 / sqrt((double)d);
@@ -416,13 +441,11 @@ __global__ void dscale_kernel(const float* __restrict__ h, const double* __restr
 // dWk[m,c,i] = sum_n dk[n,m,c] e[n,i]; dWv[c,i] = sum_n dv[n,c] e[n,i]: one
 // warp per weight, lanes taking the tokens l, l + 32, ..., then a fixed
 // butterfly
-__global__ void dweight_kernel(const double* __restrict__ dk, const double* __restrict__ dv,
-                               const float* __restrict__ e, float* __restrict__ dWk,
-                               float* __restrict__ dWv, int64_t N, int M, int d, int E) {
-  const int lane = threadIdx.x & 31;
-  const int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t total = (int64_t)(M + 1) * d * E;
-  if (g >= total) return;
+__device__ __forceinline__ void dweight_out(const double* __restrict__ dk,
+                                            const double* __restrict__ dv,
+                                            const float* __restrict__ e, float* __restrict__ dWk,
+                                            float* __restrict__ dWv, int64_t N, int M, int d, int E,
+                                            int64_t g, int lane) {
   const int i = (int)(g % E);
   const int c = (int)((g / E) % d);
   const int m = (int)(g / ((int64_t)E * d));
@@ -444,12 +467,10 @@ __global__ void dweight_kernel(const double* __restrict__ dk, const double* __re
 // de[n,i] = sum_m sum_c Wk[m,c,i] dk[n,m,c] + sum_c Wv[c,i] dv[n,c]: one warp
 // per element, lanes taking the terms l, l + 32, ... of the (m, c) then c
 // sequence, then a fixed butterfly
-__global__ void de_kernel(const double* __restrict__ dk, const double* __restrict__ dv,
-                          const float* __restrict__ Wk, const float* __restrict__ Wv,
-                          float* __restrict__ de, int64_t N, int M, int d, int E) {
-  const int lane = threadIdx.x & 31;
-  const int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (g >= N * E) return;
+__device__ __forceinline__ void de_out(const double* __restrict__ dk,
+                                       const double* __restrict__ dv, const float* __restrict__ Wk,
+                                       const float* __restrict__ Wv, float* __restrict__ de,
+                                       int64_t N, int M, int d, int E, int64_t g, int lane) {
   const int i = (int)(g % E);
   const int64_t n = g / E;
   const int Md = M * d;
@@ -462,6 +483,38 @@ __global__ void de_kernel(const double* __restrict__ dk, const double* __restric
   }
   acc = warp_sum_d(acc);
   if (lane == 0) de[g] = (float)acc;
+}
+
+// The backward's sums over tokens or features in one launch, one warp per
+// output: warps [0, n_conv) the conv weights, then n_scale norm scales,
+// n_w weights of W_k and W_v, n_de elements of de.
+struct SumsArgs {
+  const double *dy, *v, *alpha, *rc, *k, *sums, *dz, *dc, *dk, *dv;
+  const float *h, *e, *Wk, *Wv;
+  float *dw, *dgh, *dgk, *dgv, *dWk, *dWv, *de;
+  int64_t N, n_conv, n_scale, n_w, n_de;
+  int T, M, d, E;
+};
+__global__ void bwd_sums_kernel(const SumsArgs a, const F32Var var) {
+  const int lane = threadIdx.x & 31;
+  int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (g < a.n_conv) {
+    dconv_out(a.dy, a.v, a.alpha, a.rc, var, a.dw, a.N, a.T, a.M, a.d, g, lane);
+    return;
+  }
+  g -= a.n_conv;
+  if (g < a.n_scale) {
+    dscale_out(a.h, a.k, a.v, a.alpha, a.sums, a.rc, a.dz, a.dc, var, a.dgh, a.dgk, a.dgv, a.N,
+               a.M, a.d, g, lane);
+    return;
+  }
+  g -= a.n_scale;
+  if (g < a.n_w) {
+    dweight_out(a.dk, a.dv, a.e, a.dWk, a.dWv, a.N, a.M, a.d, a.E, g, lane);
+    return;
+  }
+  g -= a.n_w;
+  if (g < a.n_de) de_out(a.dk, a.dv, a.Wk, a.Wv, a.de, a.N, a.M, a.d, a.E, g, lane);
 }
 
 inline unsigned blocks_for(int64_t threads_total, int per_block) {
@@ -535,6 +588,9 @@ int launch_forward_f32(const float* e, const float* h, const float* Wk, const fl
   F32Saved sv = f32_saved_layout(saved != nullptr ? static_cast<void*>(saved) : p, N, M, d);
   const F32Var var = make_var(flags, params, M, d);
   const int tb = 256;
+  // (a block per token computing its projections and then its gate measured
+  // alike for one branch and 7% slower for four: the warp-per-output
+  // projections keep more loads in flight)
   proj_f32_kernel<<<blocks_for(N * (M + 1) * d * 32, tb), tb, 0, s>>>(e, Wk, Wv, k64, v64, sv.k,
                                                                       sv.v, N, M, d, E);
   gate_f32_kernel<<<blocks_for(N * M * 32, tb), tb, 0, s>>>(h, k64, v64, var, a64, sv.alpha,
@@ -600,35 +656,38 @@ int launch_backward_f32(const float* e, const float* h, const float* Wk, const f
                                                               w.rc, N * M, M, d);
     rec_conv_dsilu_kernel<<<blocks_for(N * M * d, tb), tb, 0, s>>>(w.v, w.alpha, w.rc, var, dout,
                                                                    w.dy, N, T, M, d);
-    // small d: each lane's features in registers, their loads issued together
+    // a block per token: its rows of the gate backward, then dv; small d:
+    // each lane's features in registers, their loads issued together
+    const GateBwdArgs ga = {dout, w.dy, w.k, w.v, w.alpha, w.sums, w.rc, h, w.dvt,
+                            scales ? w.dc : nullptr, scales ? w.dz : nullptr, w.dk, dh, N, T, M, d};
     if (d <= 128)
-      gate_bwd_kernel<4><<<blocks_for(N * M * 32, tb), tb, 0, s>>>(
-          dout, w.dy, h, w.k, w.v, w.alpha, w.sums, w.rc, var, w.dvt, scales ? w.dc : nullptr,
-          scales ? w.dz : nullptr, dh, w.dk, N, T, M, d);
+      gate_bwd_dv_kernel<4><<<(unsigned)N, GB_THREADS, 0, s>>>(ga, var, w.dv);
     else
-      gate_bwd_kernel<0><<<blocks_for(N * M * 32, tb), tb, 0, s>>>(
-          dout, w.dy, h, w.k, w.v, w.alpha, w.sums, w.rc, var, w.dvt, scales ? w.dc : nullptr,
-          scales ? w.dz : nullptr, dh, w.dk, N, T, M, d);
-    dv_kernel<<<blocks_for(N * d, tb), tb, 0, s>>>(w.dvt, w.alpha, w.dv, N, M, d);
+      gate_bwd_dv_kernel<0><<<(unsigned)N, GB_THREADS, 0, s>>>(ga, var, w.dv);
   }
   const int Mc = var.per_branch ? M : 1;
-  dconv_kernel<<<blocks_for((int64_t)Mc * d * 4 * 32, tb), tb, 0, s>>>(
-      w.dy, w.v, w.alpha, w.rc, var, dparams, N, T, M, d);
-  if (scales) {
-    if (N > 0) {
-      dscale_kernel<<<blocks_for((int64_t)M * d * 32, tb), tb, 0, s>>>(
-          h, w.k, w.v, w.alpha, w.sums, w.rc, w.dz, w.dc, var, const_cast<float*>(dvar.gh),
-          const_cast<float*>(dvar.gk), const_cast<float*>(dvar.gv), N, M, d);
-    } else {  // no tokens: zero gradients
-      const size_t nb = (size_t)(f32_param_floats(flags, M, d) - (int64_t)Mc * d * 4) * 4;
-      const int rc = ck(cudaMemsetAsync(const_cast<float*>(dvar.gh), 0, nb, s));
-      if (rc) return rc;
-    }
+  if (scales && N == 0) {  // no tokens: zero scale gradients
+    const size_t nb = (size_t)(f32_param_floats(flags, M, d) - (int64_t)Mc * d * 4) * 4;
+    const int rc = ck(cudaMemsetAsync(const_cast<float*>(dvar.gh), 0, nb, s));
+    if (rc) return rc;
   }
-  dweight_kernel<<<blocks_for((int64_t)(M + 1) * d * E * 32, tb), tb, 0, s>>>(
-      w.dk, w.dv, e, dWk, dWv, N, M, d, E);
-  if (N > 0)
-    de_kernel<<<blocks_for(N * E * 32, tb), tb, 0, s>>>(w.dk, w.dv, Wk, Wv, de, N, M, d, E);
+  // conv weights, norm scales, W_k and W_v, de: one warp per output, one launch
+  SumsArgs sa;
+  sa.dy = w.dy; sa.v = w.v; sa.alpha = w.alpha; sa.rc = w.rc; sa.k = w.k; sa.sums = w.sums;
+  sa.dz = w.dz; sa.dc = w.dc; sa.dk = w.dk; sa.dv = w.dv;
+  sa.h = h; sa.e = e; sa.Wk = Wk; sa.Wv = Wv;
+  sa.dw = dparams;
+  sa.dgh = const_cast<float*>(dvar.gh);
+  sa.dgk = const_cast<float*>(dvar.gk);
+  sa.dgv = const_cast<float*>(dvar.gv);
+  sa.dWk = dWk; sa.dWv = dWv; sa.de = de;
+  sa.N = N; sa.T = T; sa.M = M; sa.d = d; sa.E = E;
+  sa.n_conv = (int64_t)Mc * d * 4;
+  sa.n_scale = (scales && N > 0) ? (int64_t)M * d : 0;
+  sa.n_w = (int64_t)(M + 1) * d * E;
+  sa.n_de = N * E;
+  const int64_t warps = sa.n_conv + sa.n_scale + sa.n_w + sa.n_de;
+  bwd_sums_kernel<<<blocks_for(warps * 32, tb), tb, 0, s>>>(sa, var);
   return ck(cudaGetLastError());
 }
 
