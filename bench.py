@@ -667,7 +667,7 @@ def bench_fwd_bwd_27b(dev, steps=10):
     GEMMs, sparse table gradient); the same with k and v recomputed in the
     backward instead of saved; with the dilated conv (taps 3, 6 and 9
     tokens back); and with the pre-conv RMSNorm."""
-    keys = ("ms_per_step", "ms_per_step_graph", "fwd_bwd_tokens_per_s", "breakdown_ms", "roofline")
+    keys = ("ms_per_step", "fwd_bwd_tokens_per_s", "breakdown_ms", "roofline")
     kept = _fwd_bwd_27b_run(dev, steps, save_kv=True, cpu=True)
     recomputed = _fwd_bwd_27b_run(dev, steps, save_kv=False)
     kept["recompute_kv"] = {k: recomputed[k] for k in keys}
@@ -766,14 +766,10 @@ def _fwd_bwd_27b_run(dev, steps, save_kv, variant=0, cpu=False):
         if mark:
             ev[2].record(s)
 
-    nodes = []
     with torch.cuda.stream(s):
         ms = _time_loop(step, steps, 3, s)
         step(mark=True)
         torch.cuda.synchronize()
-        # the same step captured into a CUDA graph (the launches' host cost
-        # and the gaps between dependent launches out of the way)
-        ms_graph = _graph_time(step, steps, 3, s, nodes)
     if eg.engram_get_status(s) != 0:
         raise RuntimeError("device status word set in the 27B-shaped training step")
     # dense contractions of one step: forward k and v; backward [dW_k; dW_v]
@@ -793,7 +789,6 @@ def _fwd_bwd_27b_run(dev, steps, save_kv, variant=0, cpu=False):
                     "5.7B bf16 params; forward (hash, gather, fused passes"
                     + (", k and v saved" if save_kv else "") + ") + bf16 backward",
         "fwd_bwd_tokens_per_s": N / (ms / 1e3), "ms_per_step": ms,
-        "ms_per_step_graph": ms_graph, "kernels_per_step": nodes[0] if nodes else None,
         "breakdown_ms": {"forward": ev[0].elapsed_time(ev[1]), "backward": t_bwd},
         # the step's dense flops over the whole step's time (the elementwise
         # kernels between the GEMMs included): a floor on the GEMMs' own rate,
