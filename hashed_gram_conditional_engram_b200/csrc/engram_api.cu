@@ -62,7 +62,7 @@ inline size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
 // bf16 forward workspace: the passes' buffers, then g_h g_k (norm scales),
 // then with the pre-conv norm v [N, d] fp32 and rc [N]
 struct Bf16FwdWs {
-  size_t gg, vbuf, rc, total;
+  size_t gg, vbuf, rc, ctr, total;
 };
 inline Bf16FwdWs bf16_fwd_ws(const engram_cfg_t* c, int64_t n) {
   const int d = c->d_model, E = 2 * c->K * c->D_h;
@@ -71,7 +71,8 @@ inline Bf16FwdWs bf16_fwd_ws(const engram_cfg_t* c, int64_t n) {
   w.vbuf = w.gg + (bf16_scaled(c) ? up256((size_t)d * 4) : 0);
   const bool pn = bf16_prenorm(c);
   w.rc = w.vbuf + (pn ? up256((size_t)n * d * 4) : 0);
-  w.total = w.rc + (pn ? up256((size_t)n * 4) : 0);
+  w.ctr = w.rc + (pn ? up256((size_t)n * 4) : 0);  // two counters of the decode kernel
+  w.total = w.ctr + 256;
   return w;
 }
 
@@ -115,7 +116,7 @@ HeadParams make_head_params(const engram_cfg_t* cfg) {
 int forward_from_e(const engram_cfg_t* cfg, const HeadParams& hp, void* e, const void* h,
                    const void* Wk, const void* Wv, const float* conv_w, float* conv_state,
                    void* out, float* saved, int64_t N, int32_t T, void* ws, size_t ws_bytes,
-                   bool chained, cudaStream_t s) {
+                   bool chained, cudaStream_t s, bool counters_zeroed = false) {
   const int M = cfg->n_branch, d = cfg->d_model, E = hp.E;
   int rc;
   if (cfg->dtype == ENGRAM_F32)
@@ -133,6 +134,21 @@ int forward_from_e(const engram_cfg_t* cfg, const HeadParams& hp, void* e, const
   if (bf16_scaled(cfg)) {
     gg = reinterpret_cast<float*>(wsb + wl.gg);
     if ((rc = launch_scale_product(conv_w + 4 * d, conv_w + 5 * d, d, gg, s))) return rc;
+  }
+  // a decode step: both passes, the gate, the conv and the residual in one
+  // persistent launch
+  const int dil = (cfg->flags & ENGRAM_CONV_DILATED) ? 3 : 1;
+  const bool stall = (cfg->flags & ENGRAM_TEST_STALL) != 0;
+  if (conv_state != nullptr && !bf16_prenorm(cfg) && decode_fused_ok(N, d, E)) {
+    float4* part = reinterpret_cast<float4*>(wsb);
+    float* alpha = reinterpret_cast<float*>(wsb + (size_t)N * (d / 32) * sizeof(float4));
+    return launch_decode_fused(static_cast<const __nv_bfloat16*>(e),
+                               static_cast<const __nv_bfloat16*>(h),
+                               static_cast<const __nv_bfloat16*>(Wk),
+                               static_cast<const __nv_bfloat16*>(Wv), conv_w, conv_state,
+                               static_cast<__nv_bfloat16*>(out), saved, gg, dil, N, d, E, part,
+                               alpha, reinterpret_cast<int*>(wsb + wl.ctr), counters_zeroed,
+                               chained, stall, s);
   }
   // the pre-conv norm: v into the kept [k | v] rows when there are any
   PrenormFwd pn{bf16_scaled(cfg) ? conv_w + 6 * d : nullptr,
@@ -251,12 +267,17 @@ int engram_forward(const engram_cfg_t* cfg, const int32_t* idx, const void* tabl
   if (cfg->dtype == ENGRAM_BF16 &&
       (!tc_supported(cfg->d_model, hp.E, cfg->n_branch) || !bf16_variant_ok(cfg)))
     return ENGRAM_ERR_UNSUPPORTED;
+  // a bf16 decode step: the gather zeroes the decode kernel's counters, so
+  // that the two stay one launch chain
+  const bool zero_first = table != nullptr && conv_state != nullptr && cfg->dtype == ENGRAM_BF16;
   if (table != nullptr) {
-    rc = launch_gather(hp, idx, table, N, elem_bytes(cfg), e, s);
+    int* ctr = zero_first ? reinterpret_cast<int*>(static_cast<char*>(ws) + bf16_fwd_ws(cfg, N).ctr)
+                          : nullptr;
+    rc = launch_gather(hp, idx, table, N, elem_bytes(cfg), e, s, ctr);
     if (rc) return rc;
   }
   return forward_from_e(cfg, hp, e, h, Wk, Wv, conv_w, conv_state, out, saved, N, T, ws, ws_bytes,
-                        table != nullptr, s);
+                        table != nullptr, s, zero_first);
 }
 
 int engram_decode_step(const engram_cfg_t* cfg, const int32_t* proj, const int32_t* ids,
@@ -284,11 +305,15 @@ int engram_decode_step(const engram_cfg_t* cfg, const int32_t* proj, const int32
   if (cfg->dtype == ENGRAM_BF16 &&
       (!tc_supported(cfg->d_model, hp.E, cfg->n_branch) || !bf16_variant_ok(cfg)))
     return ENGRAM_ERR_UNSUPPORTED;
+  // bf16 decode: the gather also zeroes the counters of the decode kernel
+  int* ctr = cfg->dtype == ENGRAM_BF16
+                 ? reinterpret_cast<int*>(static_cast<char*>(ws) + bf16_fwd_ws(cfg, B).ctr)
+                 : nullptr;
   if ((rc = launch_hash_gather_decode(hp, proj, ids, B, ngram_state, idx, table, elem_bytes(cfg),
-                                      e, s)))
+                                      e, ctr, s)))
     return rc;
   return forward_from_e(cfg, hp, e, h, Wk, Wv, conv_w, conv_state, out, nullptr, B, 1, ws,
-                        ws_bytes, true, s);
+                        ws_bytes, true, s, ctr != nullptr);
 }
 
 int engram_backward(const engram_cfg_t* cfg, const int32_t* idx, const void* e, const void* h,

@@ -79,13 +79,17 @@ int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaS
 // ---------------------------------------------------------------- launches
 int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, int B, int T,
                 int32_t* ngram_state, int32_t* idx, cudaStream_t s);
+// zero_counters (may be NULL): two ints set to zero before the gather ends
+// (the counters of the decode kernel launched after it)
 int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,
-                  int elem_bytes, void* e, cudaStream_t s);
+                  int elem_bytes, void* e, cudaStream_t s, int* zero_counters = nullptr);
 // one decode step's hash (rolling n-gram state, idx optional) and gather in
 // one launch, B sequences of one token
+// zero_counters (may be NULL): two ints set to zero by the kernel (the
+// counters of the decode kernel launched after it)
 int launch_hash_gather_decode(const HeadParams& hp, const int32_t* proj, const int32_t* ids,
                               int64_t B, int32_t* ngram_state, int32_t* idx, const void* table,
-                              int elem_bytes, void* e, cudaStream_t s);
+                              int elem_bytes, void* e, int* zero_counters, cudaStream_t s);
 // the same gather from pinned host memory: a small fixed grid, deep per-thread
 // load queues (PCIe latency), the GPU's other SMs left free
 int launch_gather_host(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,
@@ -193,6 +197,14 @@ int launch_backward_bf16(const HeadParams& hp, const int32_t* idx, const __nv_bf
 
 // bf16 tensor-core path (sm_100a tcgen05)
 size_t tc_forward_ws_bytes(int64_t N, int d, int E);
+// one decode step's passes, gate, conv and residual in one persistent launch
+// (bf16; part and alpha: the layout of tc_forward_ws_bytes for N <= 4096)
+bool decode_fused_ok(int64_t N, int d, int E);
+int launch_decode_fused(const __nv_bfloat16* e, const __nv_bfloat16* h, const __nv_bfloat16* Wk,
+                        const __nv_bfloat16* Wv, const float* conv_w, float* conv_state,
+                        __nv_bfloat16* out, float* alpha_saved, const float* gg, int dil,
+                        int64_t N, int d, int E, float4* part, float* alpha, int* counters,
+                        bool counters_zeroed, bool chained, bool stall, cudaStream_t s);
 int tc_supported(int d, int E, int M);
 // gg[f] = gh[f] * gk[f] (the learnable norm scales' product the gate uses)
 int launch_scale_product(const float* gh, const float* gk, int d, float* gg, cudaStream_t s);

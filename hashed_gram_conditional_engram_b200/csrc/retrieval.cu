@@ -124,8 +124,9 @@ __global__ void __launch_bounds__(256) hash_gather_decode_kernel(
     const __grid_constant__ HeadParams hp, const int32_t* __restrict__ proj,
     const int32_t* __restrict__ ids, int32_t* __restrict__ ngram_state,
     int32_t* __restrict__ idx, const uint4* __restrict__ table, int CR,
-    uint4* __restrict__ e, unsigned int* status) {
+    uint4* __restrict__ e, int* __restrict__ zero_counters, unsigned int* status) {
   allow_dependents();
+  if (zero_counters != nullptr && blockIdx.x == 0 && threadIdx.x < 2) zero_counters[threadIdx.x] = 0;
   __shared__ int32_t cid[3];
   __shared__ int32_t slot[ENGRAM_MAX_HEADS];
   const int64_t n = blockIdx.x;
@@ -176,8 +177,10 @@ __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ Hea
                                                      const uint4* __restrict__ table,
                                                      int64_t n_tok, int CR,
                                                      uint4* __restrict__ e,
+                                                     int* __restrict__ zero_counters,
                                                      unsigned int* status) {
   allow_dependents();
+  if (zero_counters != nullptr && blockIdx.x == 0 && threadIdx.x < 2) zero_counters[threadIdx.x] = 0;
   const int per_tok = hp.J * CR;
   const int64_t total = n_tok * per_tok;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -291,7 +294,7 @@ int launch_hash(const HeadParams& hp, const int32_t* proj, const int32_t* ids, i
 }
 
 int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, int64_t n_tok,
-                  int elem_bytes, void* e, cudaStream_t s) {
+                  int elem_bytes, void* e, cudaStream_t s, int* zero_counters) {
   if (n_tok == 0) return ENGRAM_OK;
   const int CR = hp.D_h * elem_bytes / 16;
   int dev = 0, sms = 148;
@@ -317,8 +320,12 @@ int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, i
     const int64_t blocks =
         (total + (int64_t)threads * UNROLL_SMALL - 1) / ((int64_t)threads * UNROLL_SMALL);
     gather_kernel<UNROLL_SMALL><<<(unsigned)blocks, threads, 0, s>>>(hp, idx, tb, n_tok, CR, eo,
-                                                                     st);
+                                                                     zero_counters, st);
     return ck(cudaGetLastError());
+  }
+  if (zero_counters != nullptr) {
+    const int rc = ck(cudaMemsetAsync(zero_counters, 0, 2 * sizeof(int), s));
+    if (rc) return rc;
   }
   const int key = hp.J * 100 + CR;
   switch (key) {
@@ -333,13 +340,14 @@ int launch_gather(const HeadParams& hp, const int32_t* idx, const void* table, i
   const int64_t cap = (int64_t)sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  gather_kernel<UNROLL><<<(unsigned)blocks, threads, 0, s>>>(hp, idx, tb, n_tok, CR, eo, st);
+  gather_kernel<UNROLL><<<(unsigned)blocks, threads, 0, s>>>(hp, idx, tb, n_tok, CR, eo, nullptr,
+                                                             st);
   return ck(cudaGetLastError());
 }
 
 int launch_hash_gather_decode(const HeadParams& hp, const int32_t* proj, const int32_t* ids,
                               int64_t B, int32_t* ngram_state, int32_t* idx, const void* table,
-                              int elem_bytes, void* e, cudaStream_t s) {
+                              int elem_bytes, void* e, int* zero_counters, cudaStream_t s) {
   if (B == 0) return ENGRAM_OK;
   const int CR = hp.D_h * elem_bytes / 16;
   const int per_tok = hp.J * CR;
@@ -348,7 +356,7 @@ int launch_hash_gather_decode(const HeadParams& hp, const int32_t* proj, const i
   if (threads > 256) threads = 256;
   hash_gather_decode_kernel<<<(unsigned)B, (unsigned)threads, 0, s>>>(
       hp, proj, ids, ngram_state, idx, static_cast<const uint4*>(table), CR,
-      static_cast<uint4*>(e), status_ptr());
+      static_cast<uint4*>(e), zero_counters, status_ptr());
   return ck(cudaGetLastError());
 }
 
@@ -504,7 +512,7 @@ int launch_gather_host(const HeadParams& hp, const int32_t* idx, const void* tab
     int64_t blocks = (total + 128 * UNROLL - 1) / (128 * UNROLL);
     if (blocks > ENGRAM_HOST_GATHER_CTAS) blocks = ENGRAM_HOST_GATHER_CTAS;
     gather_kernel<UNROLL><<<(unsigned)blocks, 128, 0, s>>>(
-        hp, idx, static_cast<const uint4*>(table), n_tok, CR, static_cast<uint4*>(e),
+        hp, idx, static_cast<const uint4*>(table), n_tok, CR, static_cast<uint4*>(e), nullptr,
         status_ptr());
     return ck(cudaGetLastError());
   }

@@ -41,8 +41,9 @@ def test_workspace_sizes_host_only():
     assert eg.engram_saved_size(c, 64) >= 64 * (1 + 3 * 64) * 4
     b = _cfg(K=8, D_h=80, d_model=2560, dtype=eg.BF16, rows=[4449997] * 16,
              mult=np.ones((16, 3), np.uint64))
-    # bf16: gate partials (2 per 256-column tile per token) and the gate itself
-    assert eg.engram_workspace_size(b, eg.WS_FORWARD, 32768) == 32768 * 20 * 16 + 32768 * 4
+    # bf16: gate partials (2 per 256-column tile per token), the gate itself and
+    # the two counters of the one-launch decode step
+    assert eg.engram_workspace_size(b, eg.WS_FORWARD, 32768) == 32768 * 20 * 16 + 32768 * 4 + 256
     assert eg.engram_saved_size(b, 32768) == 32768 * 4
     # keeping k and v: alpha up to the next 256 bytes, then fp32 [N, 2d]; the
     # backward then needs no room of its own for them
