@@ -623,18 +623,38 @@ int launch_decode_fused(const __nv_bfloat16* e, const __nv_bfloat16* h, const __
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ENGRAM_ERR_CUDA;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // one CTA per SM at most: every CTA of the grid is resident at once
   const int units = a.tiles_k > a.tiles_v ? a.tiles_k : a.tiles_v;
-  const int pairs = units < sms / 2 ? units : sms / 2;
   auto run = [&](auto kern) -> int {
     static bool configured[64][4] = {};
+    static int max_pairs[64][4] = {};
     const int key = (dil == 3 ? 2 : 0) + (gg != nullptr ? 1 : 0);
     if (!configured[dev][key]) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)D_SMEM) !=
           cudaSuccess)
         return (int)ENGRAM_ERR_CUDA;
+      // the CTA pairs that fit on the GPU at once (one CTA per SM; a pair
+      // needs two SMs of one cluster-capable group): the waits at the gate
+      // need every CTA of the grid resident
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3((unsigned)(sms & ~1));
+      q.blockDim = dim3(D_THREADS);
+      q.dynamicSmemBytes = D_SMEM;
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = 2;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &q) != cudaSuccess || clusters <= 0) {
+        cudaGetLastError();
+        clusters = sms / 2;
+      }
+      max_pairs[dev][key] = clusters < sms / 2 ? clusters : sms / 2;
       configured[dev][key] = true;
     }
+    const int pairs = units < max_pairs[dev][key] ? units : max_pairs[dev][key];
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(D_THREADS);

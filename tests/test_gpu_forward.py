@@ -148,6 +148,7 @@ def test_forward_bf16_multibranch_unsupported():
     (200, 512, 2, 128),    # split units (each tile's K in two halves), ragged token tile
     (1, 256, 4, 64),       # split units, a single sequence
     (256, 256, 2, 256),    # split units, full token tiles, 8 K steps a half
+    (1024, 4096, 2, 64),   # more tiles than CTA pairs fit at once: several per pair
 ])
 def test_forward_bf16_decode_state(B, d, K, D_h):
     """One token per sequence, 6 steps, conv state carried across steps, against
@@ -352,6 +353,7 @@ def test_forward_in_place_equals_separate_output(B, T, d, dtype):
     ("bf16", 300, 512, 4, 16, eg.CONV_DILATED),   # two token tiles, dilated conv state
     ("bf16", 100, 512, 4, 64, 0),                 # split units (K in two halves per tile)
     ("bf16", 256, 256, 2, 128, eg.CONV_DILATED),  # split units, dilated conv state
+    ("bf16", 700, 2048, 2, 64, eg.CONV_DILATED),  # several tiles per CTA pair, dilated
     ("f32", 5, 64, 2, 16, 0),                     # fp32 layer
     ("f32", 9, 64, 3, 16, 0),                     # J = 6 heads (two per hash thread)
 ])
