@@ -996,8 +996,8 @@ def bench_decode(dev):
     steps of Zipf(1.1) ids, each step with its own pregenerated hidden state
     N(0, 1); d 4,096, K 8 x ~6.35M rows x 128 (13B bf16 parameters, 26 GB on
     the device), rolling n-gram and conv state.  One step = hash with the
-    n-gram state and gather (one kernel), fused passes in decode mode
-    (engram_decode_step).  All 2,000 steps are
+    n-gram state and gather (one kernel), then pass K, the gate and pass V
+    in one persistent launch (engram_decode_step).  All 2,000 steps are
     captured into one CUDA graph (each step reading its own ids and h rows),
     replayed once untimed and once timed from the same initial state."""
     import torch
@@ -1032,7 +1032,7 @@ def bench_decode(dev):
     fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, w.B)
     fws = torch.empty(fb, dtype=torch.uint8, device=dev)
 
-    def step(k):  # hash + gather in one kernel, then the fused passes
+    def step(k):  # hash + gather in one kernel, then the one-launch decode kernel
         eg.engram_decode_step(cfg, proj, ids[k], state, None, table, e, hs[k], Wk, Wv, cw,
                               conv_state, out, w.B, fws, fb, s)
 

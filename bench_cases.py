@@ -20,7 +20,8 @@ without the rest of the layer's inputs on the device.
 the two tensor-core passes; `gather` gathers from a table of --rows rows per
 head; `hash` runs the compress + n-gram + hash kernel; `decode` runs whole
 decode steps (engram_decode_step: hash with the rolling n-gram state and
-gather in one kernel, then the passes with the conv state) for --tokens
+gather in one kernel, then one persistent launch for pass K, the gate and
+pass V with the conv state) for --tokens
 sequences of one token each;
 `tiny` runs the tiny fp32 layer's step (hash, forward, backward; its own
 fixed shape); `tablegrad` runs the sparse table gradient (sort by row, segment sums) on
