@@ -3,8 +3,9 @@ allocate device memory (a host framework that owns every allocation, or a
 runtime with a fixed memory pool).  It sorts in a
 scratch array built into the library instead of a caller workspace, so its
 results must equal those of engram_table_grad on the same inputs, bit for bit
-(the reduction is deterministic).  Two calls in a row check that the second
-does not depend on what the first left in the shared array.
+(the reduction is deterministic), and equal the oracle's reduction.  Two
+calls in a row check that the second does not depend on what the first left
+in the shared array.
 
 This file is collected last on purpose, so that a run stopping at its first
 failure has run every other test before it."""
@@ -14,6 +15,7 @@ import torch
 
 from hashed_gram_conditional_engram_b200 import engram as eg
 from hashed_gram_conditional_engram_b200 import synth
+from oracle import engram_oracle as O
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +59,24 @@ def test_noalloc_equals_workspace_entry_point_on_two_calls_in_a_row():
         assert U > 0 and int(u_na.item()) == U
         assert torch.equal(k_na[:U], k_ws[:U])
         assert torch.equal(r_na[:U].view(torch.int32), r_ws[:U].view(torch.int32))
+    assert eg.engram_get_status() == 0
+
+
+@pytest.mark.parametrize("n_tok", [1, 777, eg.NOALLOC_MAX_ITEMS // (2 * K)])
+def test_noalloc_equals_oracle(n_tok):
+    """Distinct rows ascending and each row's fp32 sum of its tokens' de
+    segments in ascending token order, bit for bit against the oracle's
+    deterministic reduction (one token; a ragged count; the array full)."""
+    cfg = _cfg()
+    idx, de = _inputs(100 + n_tok, n_tok)
+    k, r, u = _outputs(n_tok * 2 * K)
+    eg.engram_table_grad_noalloc(cfg, idx, de, n_tok, k, r, u)
+    torch.cuda.synchronize()
+    k_ref, r_ref = O.table_grad_segments_fast(idx.cpu().numpy(), de.cpu().numpy(), ROWS, D_H)
+    U = int(u.item())
+    assert U == len(k_ref)
+    assert np.array_equal(k[:U].cpu().numpy(), k_ref)
+    assert np.array_equal(r[:U].cpu().numpy().view(np.int32), r_ref.view(np.int32))
     assert eg.engram_get_status() == 0
 
 
