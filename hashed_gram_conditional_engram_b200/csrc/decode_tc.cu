@@ -660,11 +660,16 @@ int launch_decode_fused(const __nv_bfloat16* e, const __nv_bfloat16* h, const __
     cfg.blockDim = dim3(D_THREADS);
     cfg.dynamicSmemBytes = D_SMEM;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    // cooperative: the CTAs start together or not at all, so work on other
+    // streams cannot hold back part of the grid while the rest waits at the
+    // gate
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = chained ? 1 : 0;
+    cfg.numAttrs = chained ? 2 : 1;
     return ck(cudaLaunchKernelEx(&cfg, kern, tak, tbk, tav, tbv, th, to, a));
   };
   if (dil == 3)

@@ -220,6 +220,11 @@ int engram_gather(const engram_cfg_t* cfg, const int32_t* idx, const void* table
  *           device fp32 [B, M, 3 dil, d], the conv inputs (vt, or the
  *           normalised vt with ENGRAM_CONV_PRENORM) of the 3 dil previous
  *           steps, oldest first, zeros at the start; updated in place.
+ *           A bf16 decode call (B <= 4,096, d a multiple of 256, E of 128,
+ *           no ENGRAM_CONV_PRENORM) runs both projections, the gate and the
+ *           conv as one cooperative launch of at most one CTA per SM, whose
+ *           CTAs wait for one another at the gate (each wait bounded by 2 s,
+ *           then ENGRAM_STATUS_TIMEOUT in the status word).
  *   out     device [B, T, M, d] (cfg->dtype); may be h itself (the residual
  *           applied in place): every read of h precedes the write of the same
  *           element.  engram_backward needs the original h, so a forward that

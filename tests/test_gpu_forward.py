@@ -401,3 +401,62 @@ def test_decode_step_equals_hash_then_forward(dtype, B, d, K, D_h, flags):
         assert eg.engram_get_status() == 0
         for name in ("idx", "state", "e", "out", "conv"):
             assert torch.equal(a[name], b[name]), (step, name)
+
+
+def test_decode_steps_on_two_streams_at_once():
+    """Two independent decode streams (own n-gram state, conv state, buffers
+    and workspace) issued on two CUDA streams with no synchronisation between
+    them give the same bits as each run alone.  Each step's layer kernel
+    needs all of its CTAs resident at once (its CTAs wait for one another at
+    the gate); two such grids do not fit the GPU together, so this checks
+    that one cannot hold part of the SMs while the other waits."""
+    rng = np.random.default_rng(808)
+    B, d, K, D_h = 256, 4096, 2, 64
+    J, E = 2 * K, 2 * K * D_h
+    rows = synth.primes_at_most(3001, J)
+    V = 1000
+    keys = synth.merge_keys(np.random.default_rng(6), V, synth.compressed_vocab(V))
+    proj, V_c = gpu_vocab_proj(keys)
+    cfg = eg.make_cfg(K, D_h, d, 1, V, V_c, eg.BF16, rows, synth.hash_multipliers(78, J))
+    table = packed_table([rng.standard_normal((P, D_h)).astype(np.float32) for P in rows], "bf16")
+    Wk = bf16_dev((rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32))
+    Wv = bf16_dev((rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32))
+    cw = dev((rng.standard_normal((d, 4)) * 0.5).astype(np.float32))
+    fb = eg.engram_workspace_size(cfg, eg.WS_FORWARD, B)
+    steps = 6
+    inputs = [[(dev(rng.integers(0, V, size=B).astype(np.int32)),
+                bf16_dev(rng.standard_normal((B, 1, 1, d)).astype(np.float32)))
+               for _ in range(steps)] for _ in range(2)]
+
+    def fresh():
+        return dict(state=torch.full((B, 2), V_c, dtype=torch.int32, device="cuda"),
+                    conv=torch.zeros((B, 1, 3, d), dtype=torch.float32, device="cuda"),
+                    e=torch.empty((B, E), dtype=torch.bfloat16, device="cuda"),
+                    out=torch.empty((B, steps, d), dtype=torch.bfloat16, device="cuda"),
+                    ws=ws(fb))
+
+    def step(p, k, ids, h, stream):
+        with torch.cuda.stream(stream):  # o belongs to the stream that uses it
+            o = torch.empty((B, 1, 1, d), dtype=torch.bfloat16, device="cuda")
+            eg.engram_decode_step(cfg, proj, ids, p["state"], None, table, p["e"], h, Wk, Wv, cw,
+                                  p["conv"], o, B, p["ws"], fb, stream)
+            p["out"][:, k] = o[:, 0, 0]
+
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    alone = [fresh(), fresh()]
+    torch.cuda.synchronize()
+    for i in range(2):
+        for k in range(steps):
+            step(alone[i], k, *inputs[i][k], s1)
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    both = [fresh(), fresh()]
+    torch.cuda.synchronize()
+    for k in range(steps):
+        step(both[0], k, *inputs[0][k], s1)
+        step(both[1], k, *inputs[1][k], s2)
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    for i in range(2):
+        for name in ("state", "conv", "out"):
+            assert torch.equal(both[i][name], alone[i][name]), (i, name)
