@@ -482,8 +482,24 @@ int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& t
   const int64_t units = (int64_t)tiles * a.splits;
   const int pairs = (int)(units < P ? units : P);
   if (pairs <= 0) return ENGRAM_OK;
-  kern<<<dim3(2 * pairs), dim3(G_THREADS), G_SMEM, s>>>(ta, tb0, tb1, tc0, tc1, a);
-  return ck(cudaGetLastError());
+  if (a.splits == 1) {
+    kern<<<dim3(2 * pairs), dim3(G_THREADS), G_SMEM, s>>>(ta, tb0, tb1, tc0, tc1, a);
+    return ck(cudaGetLastError());
+  }
+  // split tiles: a part waits for the part before it, run by another pair,
+  // so every pair must be resident together: a cooperative launch starts
+  // them together or not at all
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(G_THREADS);
+  cfg.dynamicSmemBytes = G_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return ck(cudaLaunchKernelEx(&cfg, kern, ta, tb0, tb1, tc0, tc1, a));
 }
 
 GemmArgs gemm_args(int64_t M, int64_t Nc, int64_t K, bool stall) {

@@ -450,3 +450,48 @@ def test_forward_saved_kv(B, T, d, E_heads):
         want = e64 @ W.T
         bound = np.abs(e64) @ np.abs(W).T
         assert float(np.max(np.abs(got - want) - E * 2.0 ** -24 * bound)) <= 0.0
+
+
+def test_backward_bf16_on_two_streams_at_once():
+    """Two layers' bf16 backwards issued on two CUDA streams with no
+    synchronisation between them give the same bits as each run alone.  The
+    weight-gradient GEMM cuts each output tile's 8,192-token range into
+    parts that wait for one another, so its CTAs must all be resident
+    together; two such grids do not fit the GPU at once."""
+    from tests.engram_cases import bf16_dev
+    B, T, d, K, D_h = 2, 4096, 1024, 2, 128
+    J, E, N = 2 * K, 2 * K * D_h, B * T
+    rows = synth.primes_at_most(2003, J)
+    layers, idxs, douts = [], [], []
+    for seed in (31, 32):
+        rng = np.random.default_rng(seed)
+        cfg = eg.make_cfg(K, D_h, d, 1, 1000, 770, eg.BF16, rows, np.ones((J, 3), np.uint64))
+        tables = [rng.standard_normal((P, D_h)).astype(np.float32) for P in rows]
+        L = Layer(cfg, B, T, packed_table(tables, "bf16"),
+                  bf16_dev(rng.standard_normal((B, T, 1, d)).astype(np.float32)),
+                  bf16_dev((rng.standard_normal((1, d, E)) / np.sqrt(E)).astype(np.float32)),
+                  bf16_dev((rng.standard_normal((d, E)) / np.sqrt(E)).astype(np.float32)),
+                  dev((rng.standard_normal((d, 4)) * 0.5).astype(np.float32)), torch.bfloat16)
+        idx = dev(np.stack([rng.integers(0, P, N) for P in rows], -1).astype(np.int32)
+                  .reshape(B, T, J))
+        L.forward(idx)
+        layers.append(L)
+        idxs.append(idx)
+        douts.append(dev(rng.standard_normal((N, 1, d)).astype(np.float32)))
+    torch.cuda.synchronize()
+    alone = [layers[i].backward(idxs[i], douts[i]) for i in range(2)]
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    streams = (torch.cuda.Stream(), torch.cuda.Stream())
+    both = []
+    for i in range(2):
+        with torch.cuda.stream(streams[i]):  # buffers and calls on stream i
+            both.append(layers[i].backward(idxs[i], douts[i]))
+    torch.cuda.synchronize()
+    assert eg.engram_get_status() == 0
+    for i in range(2):
+        for name in ("dh", "dWk", "dWv", "dconv_w", "de", "n_unique"):
+            assert torch.equal(both[i][name], alone[i][name]), (i, name)
+        U = int(alone[i]["n_unique"].item())
+        assert torch.equal(both[i]["keys"][:U], alone[i]["keys"][:U])
+        assert torch.equal(both[i]["rows"][:U], alone[i]["rows"][:U])
